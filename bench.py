@@ -1,0 +1,474 @@
+#!/usr/bin/env python
+"""Benchmark of the single-GPU MoE FFN forward pass (router -> slots -> dispatch
+-> grouped expert FFN -> combine -> aux loss) through the C ABI.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one moe_layer_fwd call over one batch of T synthetic tokens already
+resident in HBM.  L2 is flushed (a 320 MiB write, outside the timed events)
+before every step.  Each rank of a multi-GPU launch (torchrun) runs an
+independent replica on its own batch: the layer has no exchange step on one
+device, so there is no data-path collective; the host-side barrier and the
+max-over-ranks timing reduction are plumbing.
+
+Prints one JSON line (rank 0).  `value` = tokens/s over all ranks, device-timed
+with CUDA events; `e2e` = the same metric with the step's inputs copied from
+pinned host memory and the result read back inside the timed region.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer tokens/s on 1 B200; dispatch/combine HBM GB/s; expert GEMM TC util %"
+DEFAULT_WORKLOAD = "switch_top1_T8192_H768_E64"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
+LAUNCHES_PER_STEP = 11      # router 1, slots 4, dispatch 1, expert FFN 2, combine 1, aux 2
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ plumbing
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["_source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["_source"] = "fallback"
+    return d
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 100 ms in the background."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        import torch
+        self.samples = []
+        self.marks = []
+        try:
+            pr = torch.cuda.get_device_properties(device_index)
+            sel = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+        except Exception:
+            sel = str(device_index)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", sel, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def wait_first(self, timeout=5.0):
+        t0 = time.time()
+        while self.proc is not None and not self.samples and time.time() - t0 < timeout:
+            time.sleep(0.02)
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        rows = [s for (t, s) in self.samples if t0 <= t <= t1] or [s for (_, s) in self.samples]
+        in_region = any(t0 <= t <= t1 for (t, _) in self.samples)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            f = [x.strip() for x in r.split(",")]
+            if len(f) < 7:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx = float(f[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm), "in_timed_region": in_region}
+
+
+def traffic_from_profiles(workload: str, kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.md")
+    if not os.path.exists(p):
+        return None
+    src = os.path.join(ROOT, "expert_dispatch_router_b200", "csrc", kernel_source(kernel))
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:12]
+    for line in open(p):
+        cells = [c.strip() for c in line.strip().strip("|").split("|")]
+        if len(cells) >= 4 and cells[0] == workload and cells[1] == kernel and cells[2] == sha:
+            try:
+                return float(cells[3])
+            except ValueError:
+                return None
+    return None
+
+
+def kernel_source(stage: str) -> str:
+    return {"router": "router.cu", "dispatch": "permute.cu", "combine": "permute.cu",
+            "ffn_gemm1": "grouped_gemm.cu", "ffn_gemm2": "grouped_gemm.cu"}.get(stage, "moe_abi.cu")
+
+
+# ------------------------------------------------------------------ algorithmic work
+def stage_work(shape, kept: int, experts_used: int):
+    """Algorithmic bytes and flops of one launch of each kernel (padding rows and
+    unused capacity count as waste, not work)."""
+    b = 2 if shape.dtype == 1 else 4
+    T, H, F, E, k = shape.T, shape.H, shape.F, shape.E, shape.k
+    sh = shape.n_shared
+    rows = kept + sh * T
+    nm1 = 2 if shape.act == 2 else 1
+    wexp = experts_used + sh
+    add = T * E * 4 if shape.zipf_skew else 0
+    return {
+        "router": {"flops": 2.0 * T * H * E, "bytes": T * H * b + E * H * 4 + T * k * 8 + add},
+        "dispatch": {"flops": 0.0, "bytes": T * H * b + kept * H * b + T * k * 8},
+        "ffn_gemm1": {"flops": 2.0 * rows * H * F * nm1,
+                      "bytes": wexp * nm1 * F * H * b + rows * H * b + rows * F * b},
+        "ffn_gemm2": {"flops": 2.0 * rows * F * H, "bytes": wexp * H * F * b + rows * F * b + rows * H * b},
+        "combine": {"flops": 0.0, "bytes": kept * H * b + sh * T * H * b + T * H * b + T * k * 12},
+    }
+
+
+def roofline(stage: str, work: dict, ms: float, peaks: dict, workload: str):
+    """Bound = whichever of HBM bytes / tensor or ALU flops takes longer at peak."""
+    hbm = peaks["hbm_gbs"]
+    tc = peaks["bf16_tflops"]
+    alu = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12   # fp32 FFMA TFLOP/s at max clock
+    w = work[stage]
+    s = ms / 1e3
+    t_hbm = w["bytes"] / (hbm * 1e9)
+    if stage == "router":
+        cpeak, cbound = alu, "alu"
+    else:
+        cpeak, cbound = tc, "tensor"
+    t_cmp = w["flops"] / (cpeak * 1e12) if w["flops"] else 0.0
+    if t_cmp > t_hbm:
+        ach = w["flops"] / s / 1e12
+        out = {"bound": cbound, "achieved": ach, "peak": cpeak, "unit": "TFLOP/s", "frac": ach / cpeak}
+        out["peak_source"] = (f"{peaks['_source']} bf16 burst" if cbound == "tensor"
+                              else "148 SM x 128 FP32 lanes x 2 x max SM clock (derived)")
+    else:
+        ach = w["bytes"] / s / 1e9
+        out = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+               "peak_source": f"{peaks['_source']} HBM copy"}
+    out.update(kernel=stage, algorithmic_bytes=w["bytes"], algorithmic_flops=w["flops"], ms_per_launch=ms,
+               traffic=traffic_from_profiles(workload, stage))
+    return out
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+def oracle_sample_time(shape, inp_cpu: dict, tokens: int):
+    """Run the CPU oracle on the first `tokens` tokens as a layer of its own."""
+    import numpy as np
+    import oracle.moe_oracle as O
+    sub = shape.replace(T=tokens)
+    layer = O.OracleLayer.from_mapping(sub.as_dict())
+    d = lambda t: None if t is None else t
+    x = inp_cpu["x"][:tokens]
+    add = None if inp_cpu["logit_add"] is None else inp_cpu["logit_add"][:tokens]
+    t0 = time.perf_counter()
+    O.layer_forward(layer, x, inp_cpu["wg"], inp_cpu["w1"], inp_cpu["w2"], d(inp_cpu["w3"]), d(inp_cpu["sw1"]),
+                    d(inp_cpu["sw2"]), d(inp_cpu["sw3"]), logit_add=add)
+    return time.perf_counter() - t0
+
+
+def host_inputs(inp: dict):
+    """float64 numpy copies for the oracle; expert weights copied lazily."""
+    import torch
+
+    class Lazy:
+        def __init__(self, w):
+            self.w = w
+
+        def __getitem__(self, e):
+            return self.w[e].to("cpu", torch.float64).numpy()
+
+    d = lambda t: None if t is None else t.to("cpu", torch.float64).numpy()
+    return {"x": d(inp["x"]), "wg": d(inp["wg"]), "w1": Lazy(inp["w1"]), "w2": Lazy(inp["w2"]),
+            "w3": None if inp["w3"] is None else Lazy(inp["w3"]), "sw1": d(inp["sw1"]), "sw2": d(inp["sw2"]),
+            "sw3": d(inp["sw3"]), "logit_add": None if inp["logit_add"] is None else inp["logit_add"].cpu().numpy()}
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(shape, inp, budget_s=15.0):
+    host = host_inputs(inp)
+    n = min(shape.T, 256)
+    t = oracle_sample_time(shape, host, n)
+    while t < budget_s / 3 and n < shape.T:
+        n = min(shape.T, max(n * 2, int(n * budget_s / max(t, 1e-3) * 0.8)))
+        t = oracle_sample_time(shape, host, n)
+    return {"value": n / t, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"the oracle's whole layer on the first {n} of {shape.T} tokens as a batch of its own "
+                      f"({t:.1f} s, capacity recomputed for that batch)"}
+
+
+# ------------------------------------------------------------------ arms
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    import torch
+    from expert_dispatch_router_b200 import synth
+    shape = synth.WORKLOADS[args.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = synth.make_inputs(shape, seed=args.seed, device=dev)
+    host = host_inputs(inp)
+    budget = max(0.05, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    n = 16
+    t = oracle_sample_time(shape, host, n)
+    while t < budget * 0.5 and n < shape.T:
+        n = min(shape.T, n * 2)
+        t = oracle_sample_time(shape, host, n)
+    for _ in range(args.warmup):
+        oracle_sample_time(shape, host, n)
+    times = [oracle_sample_time(shape, host, n) for _ in range(args.steps)]
+    ms = 1e3 * sum(times) / len(times)
+    value = n / (ms / 1e3)
+    sample = f"the oracle's whole layer on the first {n} of {shape.T} tokens per step"
+    print(json.dumps({"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 1,
+                      "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                      "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                      "config": {"workload": shape.name, "tokens_per_step": n},
+                      "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                                       "sample": sample},
+                      "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+          flush=True)
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    from expert_dispatch_router_b200 import binding as B
+    from expert_dispatch_router_b200 import synth
+
+    B.load()                                     # raises if the CUDA library is missing
+    shape = synth.WORKLOADS[args.workload]
+    peaks = load_peaks()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp = synth.make_inputs(shape, seed=args.seed + rank, device="cuda")
+    cfg = B.make_cfg(shape)
+    ws = B.alloc_workspace(cfg)
+    T, H = shape.T, shape.H
+    edt = inp["x"].dtype
+    y = torch.empty((T, H), dtype=edt, device=dev)
+    aux = torch.empty(1, dtype=torch.float32, device=dev)
+    wts = B.make_weights(inp)
+    flush = torch.empty(320 * 2**20 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(events=None):
+        flush.zero_()
+        B.moe_layer_fwd(cfg, inp["x"], inp["wg"], inp["logit_add"], wts, y, aux, None, ws, stage_events=events,
+                        stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    st = B.moe_sync_status(ws, stream)
+    if st != B.MOE_OK:
+        raise RuntimeError(f"device status after warm-up: {B.strerror(st)}")
+    wt = B.workspace_tensors(cfg, ws)
+    kept = int(wt["kept_count"].sum().item())
+    experts_used = int((wt["kept_count"] > 0).sum().item())
+    rows_used = int(wt["expert_offset"][-1].item())
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(B.MOE_N_STAGE_EVENTS)] for _ in range(args.steps)]
+    for row in evs:                 # torch creates the CUDA event at its first record
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev.index) if rank == 0 else None
+    if sampler:
+        sampler.wait_first()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    for i in range(args.steps):
+        step(evs[i])
+    torch.cuda.synchronize()
+    t1 = time.time()
+    barrier(world)
+    clocks = None
+    if sampler:
+        sampler.stop()
+        clocks = sampler.summary(t0, t1)
+    st = B.moe_sync_status(ws, stream)
+    if st != B.MOE_OK:
+        raise RuntimeError(f"device status after the timed region: {B.strerror(st)}")
+
+    per_step = [e[0].elapsed_time(e[-1]) for e in evs]
+    stage_ms = {}
+    for j, name in enumerate(B.STAGES):
+        stage_ms[name] = sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps
+    ms_local = sum(per_step) / args.steps
+    ms = max_over_ranks(ms_local, world)
+    value = world * T / (ms / 1e3)
+
+    work = stage_work(shape, kept, experts_used)
+    single = ["router", "dispatch", "ffn_gemm1", "ffn_gemm2", "combine"]
+    dom = max(single, key=lambda s: stage_ms[s])
+    roof = roofline(dom, work, stage_ms[dom], peaks, shape.name)
+    per_stage = {s: roofline(s, work, stage_ms[s], peaks, shape.name) for s in single}
+    gemm_flops = work["ffn_gemm1"]["flops"] + work["ffn_gemm2"]["flops"]
+    gemm_ms = stage_ms["ffn_gemm1"] + stage_ms["ffn_gemm2"]
+    tc_util = 100.0 * gemm_flops / (gemm_ms / 1e3) / (peaks["bf16_tflops"] * 1e12)
+
+    # end to end: pinned host inputs in, result read back, every step
+    x_host = inp["x"].cpu().pin_memory()
+    add_host = None if inp["logit_add"] is None else inp["logit_add"].cpu().pin_memory()
+    x_dev = torch.empty_like(inp["x"])
+    add_dev = None if add_host is None else torch.empty_like(inp["logit_add"])
+    y_host = torch.empty((T, H), dtype=edt).pin_memory()
+    aux_host = torch.empty(1, dtype=torch.float32).pin_memory()
+    h2d = x_host.numel() * x_host.element_size() + (0 if add_host is None else add_host.numel() * 4)
+    d2h = y_host.numel() * y_host.element_size() + 4
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        if add_host is not None:
+            add_dev.copy_(add_host, non_blocking=True)
+        B.moe_layer_fwd(cfg, x_dev, inp["wg"], add_dev, wts, y, aux, None, ws, stream=stream)
+        y_host.copy_(y, non_blocking=True)
+        aux_host.copy_(aux, non_blocking=True)
+
+    for _ in range(max(args.warmup, 3)):
+        e2e_step()
+    e2e_steps = args.steps
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    ea.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    eb.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(ea.elapsed_time(eb) / e2e_steps, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(shape, inp)
+
+    if rank == 0:
+        C = B.moe_capacity(cfg)
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if shape.dtype == 1 else "f32", "data": "synthetic",
+            "config": {"workload": shape.name, "T": T, "H": H, "F": shape.F, "E": shape.E, "k": shape.k,
+                       "n_shared": shape.n_shared, "act": ["relu", "gelu", "swiglu"][shape.act],
+                       "capacity": C, "kept_assignments": kept, "rows_used": rows_used,
+                       "l2": "flushed before every step (320 MiB write outside the timed events)",
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "stages_ms": stage_ms,
+            "dispatch_gbs": per_stage["dispatch"]["achieved"] if per_stage["dispatch"]["unit"] == "GB/s" else None,
+            "combine_gbs": per_stage["combine"]["achieved"] if per_stage["combine"]["unit"] == "GB/s" else None,
+            "expert_gemm_tc_util_pct": tc_util,
+            "roofline": {k: roof[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")},
+            "roofline_detail": {s: {k: v[k] for k in ("bound", "achieved", "unit", "frac", "ms_per_launch")}
+                                for s, v in per_stage.items()},
+            "dominant_kernel": dom,
+            "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

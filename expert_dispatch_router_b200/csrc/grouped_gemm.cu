@@ -1,0 +1,439 @@
+// Grouped expert GEMM on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// Method: the per-expert FFN of an MoE layer ("Expert-parallel MoE training"
+// explainer: experts as grouped MLPs, SwiGLU experts with gate / up / down
+// matrices in worked example 2; MegaBlocks' dropless layout with every expert
+// batch padded to a multiple of 128 rows).  The expert FFN is the only dense
+// contraction of the layer; "The MoE spends too much time on the gate network"
+// measures it at 87-99% of the layer once dispatch is fixed.
+//
+// One launch computes, for every 128-row block of every expert g,
+//     D[rows, n-tile] = epi( A[rows, :] * B_g[n-tile, :]^T )
+// with bf16 operands, fp32 accumulation in tensor memory, and a bf16 store.
+//   GEMM1: A = dispatched rows (the shared expert's block reads x directly),
+//          B = W_in^T (or W_gate^T | W_up^T stacked for SwiGLU), epi = act.
+//   GEMM2: A = activations h, B = W_out^T, epi = none.
+//
+// Kernel structure (one persistent CTA per SM, 320 threads):
+//   warp 0      TMA producer: A tile 128x64 and B tile 256x64 per stage,
+//               128-byte swizzle, 4-stage ring guarded by full/empty mbarriers.
+//   warp 1      allocates 512 TMEM columns and issues tcgen05.mma
+//               (M=128, N=256, K=16, kind::f16) from one lane; commits free the
+//               smem stage and, per tile, signal the accumulator as full.
+//   warps 2-9   epilogue: tcgen05.ld of the fp32 accumulator (each warp owns
+//               one 32-lane TMEM sub-partition and half the columns), the
+//               activation, bf16 packing and 16-byte global stores.
+// Two accumulators of 256 columns let the epilogue of one tile overlap the
+// main loop of the next.  Tiles are walked m-block-major, n fastest, so CTAs
+// running at the same time share the A block and the expert's weights in L2.
+// The expert of an m-block comes from a binary search over the device-side
+// expert offsets, so no host synchronisation is needed between routing and
+// the GEMM.  Every mbarrier wait is bounded; on expiry the CTA records
+// MOE_ETIMEOUT, stops issuing work, drains what it issued and frees TMEM.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace gg {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = 64 + EPI_WARPS * 32;
+constexpr int TMEM_COLS = 512;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+
+struct KParams {
+  CUtensorMap tmA, tmAs, tmB0, tmB1, tmSB0, tmSB1;
+  void* d;
+  const int32_t* off;
+  DevStatus* status;
+  int64_t ld_d, rows_max;
+  int K, N_out, n_tiles_n, E, n_shared, epi;
+  int as_sep;   // 1: the shared block's A rows come from tmAs (row - off[E]); 0: from tmA in place
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile("{\n\t.reg .pred p;\n\t"
+               "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+               "selp.u32 %0, 1, 0, p;\n\t}"
+               : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0;
+}
+// Bounded wait: false when the CTA was told to abort or the wait ran out.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitCycles) return false;
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+               :: "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar) {
+  asm volatile("cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+               :: "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar) : "memory");
+}
+__device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
+// 128 bytes, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);        // start address
+  d |= (uint64_t)1u << 16;                          // leading byte offset (unused for this layout)
+  d |= (uint64_t)(1024u >> 4) << 32;                // stride byte offset
+  d |= (uint64_t)1u << 46;                          // descriptor version (sm_100)
+  d |= (uint64_t)2u << 61;                          // layout: 128-byte swizzle
+  return d;
+}
+// Instruction descriptor: bf16 x bf16 -> fp32, both operands K-major, M=128, N=256.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+
+__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accum) {
+  asm volatile("{\n\t.reg .pred p;\n\t"
+               "setp.ne.b32 p, %4, 0;\n\t"
+               "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+               :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accum) : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" :: "r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+               "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+               "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                 "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+                 "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+                 "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+               : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ int find_group(const int32_t* off, int ngroups, int64_t row) {
+  int lo = 0, hi = ngroups - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (off[mid] <= row) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_constant__ KParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stage_base = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES);
+  const uint32_t tfull0 = smem_u32(bars + 2 * STAGES), tempty0 = smem_u32(bars + 2 * STAGES + 2);
+  const uint32_t drain = smem_u32(bars + 2 * STAGES + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool swiglu = p.epi == MOE_ACT_SWIGLU;
+  const int ngroups = p.E + (p.n_shared ? 1 : 0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(full0 + 8 * s, 1); mbar_init(empty0 + 8 * s, 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(tfull0 + 8 * b, 1); mbar_init(tempty0 + 8 * b, EPI_WARPS * 32); }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    prefetch_map(&p.tmA); prefetch_map(&p.tmB0);
+    if (p.n_shared) { prefetch_map(&p.tmAs); prefetch_map(&p.tmSB0); }
+    if (swiglu) { prefetch_map(&p.tmB1); if (p.n_shared) prefetch_map(&p.tmSB1); }
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(smem_u32(tmem_slot)), "r"(TMEM_COLS) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int64_t rows_used = min((int64_t)p.off[ngroups], p.rows_max);
+  const int64_t n_mtiles = rows_used / BM;
+  const int64_t n_tiles = n_mtiles * p.n_tiles_n;
+  const int nk = (p.K + BK - 1) / BK;
+  const int n_step = swiglu ? BN / 2 : BN;       // output columns per tile
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t fills[STAGES] = {0, 0, 0, 0};
+      bool ok = true;
+      for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+        const int64_t mt = tile / p.n_tiles_n;
+        const int nt = (int)(tile % p.n_tiles_n);
+        const int64_t row0 = mt * BM;
+        const int g = find_group(p.off, ngroups, row0);
+        const bool sh = g == p.E;
+        const bool sep = sh && p.as_sep;
+        const CUtensorMap* ma = sep ? &p.tmAs : &p.tmA;
+        const CUtensorMap* mb0 = sh ? &p.tmSB0 : &p.tmB0;
+        const CUtensorMap* mb1 = sh ? &p.tmSB1 : &p.tmB1;
+        const int arow = (int)(sep ? row0 - p.off[p.E] : row0);
+        const int z = sh ? 0 : g;
+        const int n0 = nt * n_step;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag)) { ok = false; break; }
+          const uint32_t sa = smem_u32(stage_base + stage * STAGE_BYTES);
+          const uint32_t sb = sa + A_BYTES;
+          const uint32_t fb = full0 + 8 * stage;
+          mbar_expect_tx(fb, STAGE_BYTES);
+          tma_load_2d(sa, ma, kb * BK, arow, fb);
+          if (swiglu) {
+            tma_load_3d(sb, mb0, kb * BK, n0, z, fb);
+            tma_load_3d(sb + B_BYTES / 2, mb1, kb * BK, n0, z, fb);
+          } else {
+            tma_load_3d(sb, mb0, kb * BK, n0, z, fb);
+          }
+          fills[stage]++;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        set_status(p.status, MOE_ETIMEOUT, 10);
+      }
+      // never leave with a bulk copy still writing this CTA's shared memory
+      for (int s = 0; s < STAGES; ++s)
+        if (fills[s]) {
+          const long long t0 = clock64();
+          while (!mbar_try_wait(full0 + 8 * s, (fills[s] - 1) & 1u) && clock64() - t0 < kWaitCycles) {}
+        }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+        if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(stage_base + stage * STAGE_BYTES);
+          const uint32_t sb = sa + A_BYTES;
+          const uint64_t ad = sw128_desc(sa), bd = sw128_desc(sb);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)   // advance 16 elements = 32 bytes along K
+            umma(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), (kb | kk) != 0 ? 1u : 0u);
+          umma_commit(empty0 + 8 * stage);      // stage free once these MMAs finish
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(tfull0 + 8 * acc);          // accumulator ready for the epilogue
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        set_status(p.status, MOE_ETIMEOUT, 11);
+      }
+      // wait for every MMA issued by this CTA before TMEM is released
+      umma_commit(drain);
+      const long long t0 = clock64();
+      while (!mbar_try_wait(drain, 0) && clock64() - t0 < kWaitCycles) {}
+    }
+  } else {
+    // ---------------- epilogue
+    const int ew = warp - 2;
+    const int sub = warp & 3;                  // TMEM sub-partition this warp may access
+    const int half = ew >> 2;                  // which half of the output columns
+    const int row_in_tile = sub * 32 + lane;
+    const int cols_per_warp = n_step / 2;      // 128 (plain) or 64 (SwiGLU)
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+      if (!mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag)) {
+        *abort_flag = 1;
+        set_status(p.status, MOE_ETIMEOUT, 12);
+        break;
+      }
+      tc_fence_after();
+      const int64_t mt = tile / p.n_tiles_n;
+      const int nt = (int)(tile % p.n_tiles_n);
+      const int64_t grow = mt * BM + row_in_tile;
+      const int ncol0 = nt * n_step + half * cols_per_warp;    // first output column of this warp
+      const uint32_t tbase = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * BN);
+      uint8_t* drow = static_cast<uint8_t*>(p.d) + grow * p.ld_d * 2;
+      for (int c = 0; c < cols_per_warp; c += 32) {
+        float v[32];
+        const int acol = half * cols_per_warp + c;             // accumulator column
+        tmem_ld32(tbase + (uint32_t)acol, v);
+        if (swiglu) {
+          float u[32];
+          tmem_ld32(tbase + (uint32_t)(BN / 2 + acol), u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = act_silu(v[i]) * u[i];
+        } else {
+          tmem_wait_ld();
+          if (p.epi == MOE_ACT_RELU) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = act_relu(v[i]);
+          } else if (p.epi == MOE_ACT_GELU) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = act_gelu(v[i]);
+          }
+        }
+        const int col = ncol0 + c;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (col + 8 * q + 8 <= p.N_out) {
+            int4 o;
+            o.x = (int)pack_bf16(v[8 * q + 0], v[8 * q + 1]);
+            o.y = (int)pack_bf16(v[8 * q + 2], v[8 * q + 3]);
+            o.z = (int)pack_bf16(v[8 * q + 4], v[8 * q + 5]);
+            o.w = (int)pack_bf16(v[8 * q + 6], v[8 * q + 7]);
+            st_v4(drow + (int64_t)(col + 8 * q) * 2, o);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(tempty0 + 8 * acc);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem_base), "r"(TMEM_COLS) : "memory");
+  }
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 2-D map over a row-major bf16 matrix [rows, K], box 64 x 128.
+static bool make_map_a(CUtensorMap* m, const void* base, int64_t rows, int K) {
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  cuuint32_t box[2] = {BK, BM};
+  cuuint32_t es[2] = {1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D map over stacked weights [G, N, K], box 64 x box_n x 1 (rows past N read as zero).
+static bool make_map_b(CUtensorMap* m, const void* base, int G, int N, int K, int box_n) {
+  cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)N, (cuuint64_t)G};
+  cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)N * K * 2};
+  cuuint32_t box[3] = {BK, (cuuint32_t)box_n, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace gg
+
+cudaError_t launch_grouped_gemm(const GemmParams& p, cudaStream_t stream) {
+  using namespace gg;
+  if (p.rows_max == 0) return cudaSuccess;
+  if (encode_fn() == nullptr) return cudaErrorNotSupported;
+  const bool swiglu = p.epi == MOE_ACT_SWIGLU;
+  const int box_n = swiglu ? BN / 2 : BN;
+  KParams k{};
+  bool ok = make_map_a(&k.tmA, p.a_routed, p.rows_max, p.K);
+  ok = ok && make_map_a(&k.tmAs, p.a_shared ? p.a_shared : p.a_routed, p.a_shared ? p.T : p.rows_max, p.K);
+  ok = ok && make_map_b(&k.tmB0, p.b0, p.E, p.Nw, p.K, box_n);
+  ok = ok && make_map_b(&k.tmB1, p.b1 ? p.b1 : p.b0, p.E, p.Nw, p.K, box_n);
+  ok = ok && make_map_b(&k.tmSB0, p.sb0 ? p.sb0 : p.b0, 1, p.Nw, p.K, box_n);
+  ok = ok && make_map_b(&k.tmSB1, p.sb1 ? p.sb1 : (p.sb0 ? p.sb0 : p.b0), 1, p.Nw, p.K, box_n);
+  if (!ok) return cudaErrorInvalidValue;
+  k.d = p.d;
+  k.off = p.expert_offset;
+  k.status = p.status;
+  k.ld_d = p.Nw;
+  k.rows_max = p.rows_max;
+  k.as_sep = p.a_shared != nullptr;
+  k.K = p.K;
+  k.N_out = p.Nw;
+  k.n_tiles_n = (p.Nw + (swiglu ? BN / 2 : BN) - 1) / (swiglu ? BN / 2 : BN);
+  k.E = p.E;
+  k.n_shared = p.n_shared;
+  k.epi = p.epi;
+  static int smem_set = 0;
+  if (!smem_set) {
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    smem_set = 1;
+  }
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // grid: one CTA per SM, never more than the largest possible tile count
+  const int64_t max_tiles = (p.rows_max / BM) * k.n_tiles_n;
+  const int grid = (int)(max_tiles < sms ? (max_tiles > 0 ? max_tiles : 1) : sms);
+  grouped_gemm_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(k);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,90 @@
+// Internal launch interface between the C ABI (moe_abi.cu) and the kernels.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+struct RouterParams {
+  const void* x;            // [T,H] bf16 or fp32 (unused when logits_in is set)
+  const float* wg;          // [E,H]
+  const float* logit_add;   // [T,E] or null
+  const float* logits_in;   // [T,E] or null: skip the GEMM, route these logits
+  int32_t* ids;             // [T,k]
+  float* gates;             // [T,k]
+  float* logits_out;        // [T,E] or null
+  float* psum_part;         // [nblk,E]
+  int32_t* cnt_part;        // [nblk,E]
+  int64_t T;
+  int H, E, k, score, renorm;
+};
+int router_tile_tokens(int E);
+cudaError_t launch_router(const RouterParams& p, bool bf16, cudaStream_t stream);
+cudaError_t launch_aux(const float* psum_part, const int32_t* cnt_part, int nblk, int E, int64_t T, int k,
+                       float alpha, double* term, float* aux, cudaStream_t stream);
+
+struct SlotParams {
+  const int32_t* ids;       // [T,k]
+  int32_t* slot;            // [T,k]
+  int32_t* expert_count;    // [E]
+  int32_t* kept_count;      // [E]
+  int32_t* expert_offset;   // [E+2]
+  int32_t* row_token;       // [rows_max]
+  int32_t* chunk_cnt;       // [E, nchunk] scratch
+  int64_t T;
+  int E, k, n_shared;
+  int64_t capacity;         // < 0: dropless
+  int64_t rows_max;
+  DevStatus* status;
+};
+constexpr int kSlotChunk = 2048;   // assignments per CTA of the slot kernels
+cudaError_t launch_slots(const SlotParams& p, cudaStream_t stream);
+
+struct PermuteParams {
+  const void* src;          // dispatch: x [T,H]; combine: ybuf [rows,H]
+  void* dst;                // dispatch: xbuf [rows,H]; combine: y [T,H]
+  const int32_t* ids;
+  const int32_t* slot;
+  const float* gates;
+  const int32_t* expert_offset;
+  int64_t T, rows_max;
+  int H, E, k, n_shared;
+  int elem_bytes;           // 2 (bf16) or 4 (fp32)
+};
+cudaError_t launch_dispatch(const PermuteParams& p, cudaStream_t stream);
+cudaError_t launch_combine(const PermuteParams& p, cudaStream_t stream);
+
+// fp32 SIMT grouped FFN (one GEMM per call).
+struct FfnF32Params {
+  const float* a_routed;    // [rows_max, K]
+  const float* a_shared;    // [T, K], or null: the shared block's rows sit in a_routed in place
+  const float* b0;          // routed [E, N, K]
+  const float* b1;          // SwiGLU up [E, N, K] or null
+  const float* sb0;         // shared [1, N, K] or null
+  const float* sb1;
+  float* d;                 // [rows_max, N]
+  const int32_t* expert_offset;
+  int64_t T, rows_max;
+  int K, N, E, n_shared, epi;  // epi: -1 none, else MOE_ACT_*
+};
+cudaError_t launch_ffn_f32(const FfnF32Params& p, cudaStream_t stream);
+
+// tcgen05 grouped GEMM (bf16 in, fp32 accumulate in TMEM, bf16 out).
+struct GemmParams {
+  const void* a_routed;     // [rows_max, K] bf16
+  const void* a_shared;     // [T, K] bf16, or null: the shared block's rows sit in a_routed in place
+  const void* b0;           // routed [E, Nw, K] (W_in^T, W_gate^T or W_out^T)
+  const void* b1;           // routed SwiGLU up [E, Nw, K] or null
+  const void* sb0;          // shared [1, Nw, K] or null
+  const void* sb1;
+  void* d;                  // [rows_max, N_out] bf16
+  const int32_t* expert_offset;   // [E+2]
+  int64_t T, rows_max;
+  int K, Nw, E, n_shared, epi;    // epi: -1 none, else MOE_ACT_*
+  DevStatus* status;
+};
+cudaError_t launch_grouped_gemm(const GemmParams& p, cudaStream_t stream);
+
+}  // namespace moe

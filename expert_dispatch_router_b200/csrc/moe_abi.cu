@@ -1,0 +1,471 @@
+// Host side of the C ABI declared in include/moe_b200.h: validation, the exact
+// capacity, the row bound, the workspace layout, and the stage launches.
+// Nothing here allocates device memory or synchronises (moe_sync_status
+// excepted, which exists to do exactly that).
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace moe;
+
+namespace {
+
+constexpr int64_t kMaxCf = int64_t(1) << 20;
+
+struct Layout {
+  size_t status, psum, cnt, term, chunk, ids, gates, slot, ecount, kept, off, rowtok, logits, xbuf, hbuf, ybuf;
+  size_t total;
+  int nblk_router, nchunk;
+  int64_t rows_max;
+};
+
+bool valid_cfg(const moe_cfg* c) {
+  if (c == nullptr) return false;
+  if (c->T < 0 || c->E < 1 || c->k < 1 || c->H < 1 || c->F < 1) return false;
+  if (c->k > c->E) return false;
+  if (c->n_shared != 0 && c->n_shared != 1) return false;
+  if (c->act < MOE_ACT_RELU || c->act > MOE_ACT_SWIGLU) return false;
+  if (c->score != MOE_SCORE_SOFTMAX_TOPK && c->score != MOE_SCORE_TOPK_SOFTMAX) return false;
+  if (c->renorm != 0 && c->renorm != 1) return false;
+  if (c->cap_mode != MOE_CAP_CAPACITY && c->cap_mode != MOE_CAP_DROPLESS) return false;
+  if (c->dtype != MOE_DTYPE_F32 && c->dtype != MOE_DTYPE_BF16) return false;
+  if (c->cap_mode == MOE_CAP_CAPACITY && (c->cf_num <= 0 || c->cf_den <= 0)) return false;
+  if (c->min_capacity < 0) return false;
+  return true;
+}
+
+// MOE_OK, MOE_EINVAL or MOE_EUNSUPPORTED.
+int check_cfg(const moe_cfg* c) {
+  if (!valid_cfg(c)) return MOE_EINVAL;
+  if (c->E > kMaxE || c->k > kMaxK) return MOE_EUNSUPPORTED;
+  if (c->H % 8 != 0 || c->F % 8 != 0) return MOE_EUNSUPPORTED;
+  if (c->cap_mode == MOE_CAP_CAPACITY && (c->cf_num > kMaxCf || c->cf_den > kMaxCf)) return MOE_EUNSUPPORTED;
+  if (c->T * (int64_t)c->k >= (int64_t(1) << 31)) return MOE_EUNSUPPORTED;
+  return MOE_OK;
+}
+
+int64_t capacity_of(const moe_cfg* c) {
+  if (c->cap_mode == MOE_CAP_DROPLESS) return -1;
+  const int64_t num = c->T * c->k * c->cf_num;
+  const int64_t den = (int64_t)c->E * c->cf_den;
+  int64_t cap = (num + den - 1) / den;              // exact ceiling of the rational T*k*cf/E
+  return cap > c->min_capacity ? cap : c->min_capacity;
+}
+
+int64_t rows_max_of(const moe_cfg* c) {
+  const int64_t A = c->T * c->k;
+  const int64_t nonempty = A < c->E ? A : c->E;     // experts that can own a block
+  int64_t routed = A + (kRowPad - 1) * nonempty;
+  if (c->cap_mode == MOE_CAP_CAPACITY) {
+    const int64_t C = capacity_of(c);
+    const int64_t kept = A < (int64_t)c->E * C ? A : (int64_t)c->E * C;
+    const int64_t b1 = kept + (kRowPad - 1) * nonempty;
+    const int64_t b2 = (int64_t)c->E * round_up(C, kRowPad);
+    routed = b1 < b2 ? b1 : b2;
+  }
+  routed = round_up(routed, kRowPad);
+  return routed + (c->n_shared ? round_up(c->T, kRowPad) : 0);
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+Layout layout_of(const moe_cfg* c) {
+  Layout L{};
+  const size_t T = (size_t)c->T, E = (size_t)c->E, k = (size_t)c->k;
+  const size_t esz = c->dtype == MOE_DTYPE_BF16 ? 2 : 4;
+  L.rows_max = rows_max_of(c);
+  const int bt = router_tile_tokens(c->E);
+  L.nblk_router = (int)((c->T + bt - 1) / bt);
+  L.nchunk = (int)((c->T * c->k + kSlotChunk - 1) / kSlotChunk);
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align256(o + (bytes ? bytes : 1)); return at; };
+  L.status = take(sizeof(DevStatus));
+  L.psum = take(sizeof(float) * L.nblk_router * E);
+  L.cnt = take(sizeof(int32_t) * L.nblk_router * E);
+  L.term = take(sizeof(double) * E);
+  L.chunk = take(sizeof(int32_t) * E * (size_t)L.nchunk);
+  L.ids = take(sizeof(int32_t) * T * k);
+  L.gates = take(sizeof(float) * T * k);
+  L.slot = take(sizeof(int32_t) * T * k);
+  L.ecount = take(sizeof(int32_t) * E);
+  L.kept = take(sizeof(int32_t) * E);
+  L.off = take(sizeof(int32_t) * (E + 2));
+  L.rowtok = take(sizeof(int32_t) * (size_t)L.rows_max);
+  L.logits = take((c->flags & MOE_FLAG_KEEP_LOGITS) ? sizeof(float) * T * E : 0);
+  L.xbuf = take(esz * (size_t)L.rows_max * c->H);
+  L.hbuf = take(esz * (size_t)L.rows_max * c->F);
+  L.ybuf = take(esz * (size_t)L.rows_max * c->H);
+  L.total = o;
+  return L;
+}
+
+template <typename P>
+P* at(void* ws, size_t off) { return reinterpret_cast<P*>(static_cast<char*>(ws) + off); }
+
+cudaStream_t S(moe_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ECUDA; }
+
+RouterParams router_params(const moe_cfg* c, const Layout& L, void* ws) {
+  RouterParams p{};
+  p.psum_part = at<float>(ws, L.psum);
+  p.cnt_part = at<int32_t>(ws, L.cnt);
+  p.T = c->T;
+  p.H = c->H;
+  p.E = c->E;
+  p.k = c->k;
+  p.score = c->score;
+  p.renorm = c->renorm;
+  return p;
+}
+
+int run_route(const moe_cfg* c, const Layout& L, const void* x, const float* wg, const float* logit_add,
+              const float* logits_in, int32_t* ids, float* gates, float* logits_out, void* ws, cudaStream_t s) {
+  RouterParams p = router_params(c, L, ws);
+  p.x = x;
+  p.wg = wg;
+  p.logit_add = logit_add;
+  p.logits_in = logits_in;
+  p.ids = ids;
+  p.gates = gates;
+  p.logits_out = logits_out;
+  return cuda_status(launch_router(p, c->dtype == MOE_DTYPE_BF16, s));
+}
+
+int run_slots(const moe_cfg* c, const Layout& L, const int32_t* ids, int32_t* slot, int32_t* ecount, int32_t* kept,
+              int32_t* off, int32_t* rowtok, void* ws, cudaStream_t s) {
+  SlotParams p{};
+  p.ids = ids;
+  p.slot = slot;
+  p.expert_count = ecount;
+  p.kept_count = kept;
+  p.expert_offset = off;
+  p.row_token = rowtok;
+  p.chunk_cnt = at<int32_t>(ws, L.chunk);
+  p.T = c->T;
+  p.E = c->E;
+  p.k = c->k;
+  p.n_shared = c->n_shared;
+  p.capacity = capacity_of(c);
+  p.rows_max = L.rows_max;
+  p.status = at<DevStatus>(ws, L.status);
+  return cuda_status(launch_slots(p, s));
+}
+
+PermuteParams permute_params(const moe_cfg* c, const Layout& L) {
+  PermuteParams p{};
+  p.T = c->T;
+  p.rows_max = L.rows_max;
+  p.H = c->H;
+  p.E = c->E;
+  p.k = c->k;
+  p.n_shared = c->n_shared;
+  p.elem_bytes = c->dtype == MOE_DTYPE_BF16 ? 2 : 4;
+  return p;
+}
+
+int record(const moe_event_t* ev, int i, cudaStream_t s) {
+  if (ev == nullptr) return MOE_OK;
+  return cuda_status(cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev[i]), s));
+}
+
+// Both contractions of the expert FFN; `ev_mid`, if non-NULL, is recorded between them.
+int run_ffn(const moe_cfg* c, const Layout& L, const void* xbuf, const void* x, const int32_t* off,
+            const moe_weights* w, void* ybuf, void* ws, cudaStream_t s, const moe_event_t* ev_mid = nullptr) {
+  void* hbuf = at<void>(ws, L.hbuf);
+  const bool sh = c->n_shared != 0;
+  if (c->dtype == MOE_DTYPE_BF16) {
+    GemmParams g1{};
+    g1.a_routed = xbuf;
+    g1.a_shared = sh ? x : nullptr;
+    g1.b0 = w->w1;
+    g1.b1 = c->act == MOE_ACT_SWIGLU ? w->w3 : nullptr;
+    g1.sb0 = sh ? w->sw1 : nullptr;
+    g1.sb1 = sh && c->act == MOE_ACT_SWIGLU ? w->sw3 : nullptr;
+    g1.d = hbuf;
+    g1.expert_offset = off;
+    g1.T = c->T;
+    g1.rows_max = L.rows_max;
+    g1.K = c->H;
+    g1.Nw = c->F;
+    g1.E = c->E;
+    g1.n_shared = c->n_shared;
+    g1.epi = c->act;
+    g1.status = at<DevStatus>(ws, L.status);
+    cudaError_t e = launch_grouped_gemm(g1, s);
+    if (e != cudaSuccess) return MOE_ECUDA;
+    if (record(ev_mid, 0, s) != MOE_OK) return MOE_ECUDA;
+    GemmParams g2 = g1;
+    g2.a_routed = hbuf;
+    g2.a_shared = nullptr;
+    g2.b0 = w->w2;
+    g2.b1 = nullptr;
+    g2.sb0 = sh ? w->sw2 : nullptr;
+    g2.sb1 = nullptr;
+    g2.d = ybuf;
+    g2.K = c->F;
+    g2.Nw = c->H;
+    g2.epi = -1;
+    return cuda_status(launch_grouped_gemm(g2, s));
+  }
+  FfnF32Params f1{};
+  f1.a_routed = static_cast<const float*>(xbuf);
+  f1.a_shared = sh ? static_cast<const float*>(x) : nullptr;
+  f1.b0 = static_cast<const float*>(w->w1);
+  f1.b1 = c->act == MOE_ACT_SWIGLU ? static_cast<const float*>(w->w3) : nullptr;
+  f1.sb0 = sh ? static_cast<const float*>(w->sw1) : nullptr;
+  f1.sb1 = sh && c->act == MOE_ACT_SWIGLU ? static_cast<const float*>(w->sw3) : nullptr;
+  f1.d = static_cast<float*>(hbuf);
+  f1.expert_offset = off;
+  f1.T = c->T;
+  f1.rows_max = L.rows_max;
+  f1.K = c->H;
+  f1.N = c->F;
+  f1.E = c->E;
+  f1.n_shared = c->n_shared;
+  f1.epi = c->act;
+  cudaError_t e = launch_ffn_f32(f1, s);
+  if (e != cudaSuccess) return MOE_ECUDA;
+  if (record(ev_mid, 0, s) != MOE_OK) return MOE_ECUDA;
+  FfnF32Params f2 = f1;
+  f2.a_routed = static_cast<const float*>(hbuf);
+  f2.a_shared = nullptr;
+  f2.b0 = static_cast<const float*>(w->w2);
+  f2.b1 = nullptr;
+  f2.sb0 = sh ? static_cast<const float*>(w->sw2) : nullptr;
+  f2.sb1 = nullptr;
+  f2.d = static_cast<float*>(ybuf);
+  f2.K = c->F;
+  f2.N = c->H;
+  f2.epi = -1;
+  return cuda_status(launch_ffn_f32(f2, s));
+}
+
+int check_weights(const moe_cfg* c, const moe_weights* w) {
+  if (w == nullptr || w->w1 == nullptr || w->w2 == nullptr) return MOE_EINVAL;
+  if (c->act == MOE_ACT_SWIGLU && w->w3 == nullptr) return MOE_EINVAL;
+  if (c->n_shared) {
+    if (w->sw1 == nullptr || w->sw2 == nullptr) return MOE_EINVAL;
+    if (c->act == MOE_ACT_SWIGLU && w->sw3 == nullptr) return MOE_EINVAL;
+  }
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_capacity(const moe_cfg* cfg, int64_t* capacity) {
+  if (capacity == nullptr) return MOE_EINVAL;
+  const int st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  *capacity = capacity_of(cfg);
+  return MOE_OK;
+}
+
+int moe_rows_max(const moe_cfg* cfg, int64_t* rows_max) {
+  if (rows_max == nullptr) return MOE_EINVAL;
+  const int st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  const int64_t r = rows_max_of(cfg);
+  if (r >= (int64_t(1) << 31)) return MOE_EUNSUPPORTED;
+  *rows_max = r;
+  return MOE_OK;
+}
+
+int moe_workspace_size(const moe_cfg* cfg, size_t* bytes) {
+  if (bytes == nullptr) return MOE_EINVAL;
+  const int st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (rows_max_of(cfg) >= (int64_t(1) << 31)) return MOE_EUNSUPPORTED;
+  *bytes = layout_of(cfg).total;
+  return MOE_OK;
+}
+
+int moe_workspace_views(const moe_cfg* cfg, void* ws, moe_ws_views* v) {
+  if (ws == nullptr || v == nullptr) return MOE_EINVAL;
+  const int st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  const Layout L = layout_of(cfg);
+  v->ids = at<int32_t>(ws, L.ids);
+  v->gates = at<float>(ws, L.gates);
+  v->slot = at<int32_t>(ws, L.slot);
+  v->expert_count = at<int32_t>(ws, L.ecount);
+  v->kept_count = at<int32_t>(ws, L.kept);
+  v->expert_offset = at<int32_t>(ws, L.off);
+  v->row_token = at<int32_t>(ws, L.rowtok);
+  v->logits = (cfg->flags & MOE_FLAG_KEEP_LOGITS) ? at<float>(ws, L.logits) : nullptr;
+  v->xbuf = at<void>(ws, L.xbuf);
+  v->hbuf = at<void>(ws, L.hbuf);
+  v->ybuf = at<void>(ws, L.ybuf);
+  v->rows_max = L.rows_max;
+  return MOE_OK;
+}
+
+int moe_route(const moe_cfg* cfg, const void* x, const float* wg, const float* logit_add, int32_t* ids,
+              float* gates, float* logits_out, void* ws, moe_stream_t stream) {
+  const int st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T > 0 && (x == nullptr || wg == nullptr || ids == nullptr || gates == nullptr)) return MOE_EINVAL;
+  if (ws == nullptr) return MOE_EINVAL;
+  return run_route(cfg, layout_of(cfg), x, wg, logit_add, nullptr, ids, gates, logits_out, ws, S(stream));
+}
+
+int moe_route_from_logits(const moe_cfg* cfg, const float* logits, int32_t* ids, float* gates, void* ws,
+                          moe_stream_t stream) {
+  const int st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T > 0 && (logits == nullptr || ids == nullptr || gates == nullptr)) return MOE_EINVAL;
+  if (ws == nullptr) return MOE_EINVAL;
+  return run_route(cfg, layout_of(cfg), nullptr, nullptr, nullptr, logits, ids, gates, nullptr, ws, S(stream));
+}
+
+int moe_assign_slots(const moe_cfg* cfg, const int32_t* ids, int32_t* slot, int32_t* expert_count,
+                     int32_t* kept_count, int32_t* expert_offset, int32_t* row_token, void* ws,
+                     moe_stream_t stream) {
+  const int st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (ws == nullptr || expert_count == nullptr || kept_count == nullptr || expert_offset == nullptr) return MOE_EINVAL;
+  if (cfg->T > 0 && (ids == nullptr || slot == nullptr || row_token == nullptr)) return MOE_EINVAL;
+  return run_slots(cfg, layout_of(cfg), ids, slot, expert_count, kept_count, expert_offset, row_token, ws, S(stream));
+}
+
+int moe_dispatch(const moe_cfg* cfg, const void* x, const int32_t* ids, const int32_t* slot,
+                 const int32_t* expert_offset, void* xbuf, moe_stream_t stream) {
+  const int st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T > 0 && (x == nullptr || ids == nullptr || slot == nullptr || expert_offset == nullptr || xbuf == nullptr))
+    return MOE_EINVAL;
+  PermuteParams p = permute_params(cfg, layout_of(cfg));
+  p.src = x;
+  p.dst = xbuf;
+  p.ids = ids;
+  p.slot = slot;
+  p.expert_offset = expert_offset;
+  return cuda_status(launch_dispatch(p, S(stream)));
+}
+
+int moe_expert_ffn(const moe_cfg* cfg, const void* xbuf, const void* x, const int32_t* expert_offset,
+                   const moe_weights* w, void* ybuf, void* ws, moe_stream_t stream) {
+  int st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  st = check_weights(cfg, w);
+  if (st != MOE_OK) return st;
+  if (xbuf == nullptr || expert_offset == nullptr || ybuf == nullptr || ws == nullptr) return MOE_EINVAL;
+  if (cfg->n_shared && x == nullptr) return MOE_EINVAL;
+  return run_ffn(cfg, layout_of(cfg), xbuf, x, expert_offset, w, ybuf, ws, S(stream));
+}
+
+int moe_combine(const moe_cfg* cfg, const void* ybuf, const int32_t* ids, const int32_t* slot, const float* gates,
+                const int32_t* expert_offset, void* y, moe_stream_t stream) {
+  const int st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T > 0 && (ybuf == nullptr || ids == nullptr || slot == nullptr || gates == nullptr ||
+                     expert_offset == nullptr || y == nullptr))
+    return MOE_EINVAL;
+  PermuteParams p = permute_params(cfg, layout_of(cfg));
+  p.src = ybuf;
+  p.dst = y;
+  p.ids = ids;
+  p.slot = slot;
+  p.gates = gates;
+  p.expert_offset = expert_offset;
+  return cuda_status(launch_combine(p, S(stream)));
+}
+
+int moe_aux_loss(const moe_cfg* cfg, const void* ws, float* aux, moe_stream_t stream) {
+  const int st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (ws == nullptr || aux == nullptr) return MOE_EINVAL;
+  const Layout L = layout_of(cfg);
+  void* w = const_cast<void*>(ws);
+  return cuda_status(launch_aux(at<float>(w, L.psum), at<int32_t>(w, L.cnt), L.nblk_router, cfg->E, cfg->T, cfg->k,
+                                cfg->aux_alpha, at<double>(w, L.term), aux, S(stream)));
+}
+
+int moe_layer_fwd(const moe_cfg* cfg, const void* x, const float* wg, const float* logit_add, const moe_weights* w,
+                  void* y, float* aux, int32_t* expert_count, void* ws, size_t ws_bytes,
+                  const moe_event_t* stage_events, moe_stream_t stream) {
+  int st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  st = check_weights(cfg, w);
+  if (st != MOE_OK) return st;
+  if (ws == nullptr || aux == nullptr) return MOE_EINVAL;
+  if (cfg->T > 0 && (x == nullptr || wg == nullptr || y == nullptr)) return MOE_EINVAL;
+  if (rows_max_of(cfg) >= (int64_t(1) << 31)) return MOE_EUNSUPPORTED;
+  const Layout L = layout_of(cfg);
+  if (ws_bytes < L.total) return MOE_EWORKSPACE;
+  cudaStream_t s = S(stream);
+  int32_t* ids = at<int32_t>(ws, L.ids);
+  float* gates = at<float>(ws, L.gates);
+  int32_t* slot = at<int32_t>(ws, L.slot);
+  int32_t* off = at<int32_t>(ws, L.off);
+  void* xbuf = at<void>(ws, L.xbuf);
+  void* ybuf = at<void>(ws, L.ybuf);
+  float* logits = (cfg->flags & MOE_FLAG_KEEP_LOGITS) ? at<float>(ws, L.logits) : nullptr;
+
+  if ((st = record(stage_events, 0, s)) != MOE_OK) return st;
+  if ((st = run_route(cfg, L, x, wg, logit_add, nullptr, ids, gates, logits, ws, s)) != MOE_OK) return st;
+  if ((st = record(stage_events, 1, s)) != MOE_OK) return st;
+  if ((st = run_slots(cfg, L, ids, slot, at<int32_t>(ws, L.ecount), at<int32_t>(ws, L.kept), off,
+                      at<int32_t>(ws, L.rowtok), ws, s)) != MOE_OK)
+    return st;
+  if ((st = record(stage_events, 2, s)) != MOE_OK) return st;
+  PermuteParams pp = permute_params(cfg, L);
+  pp.ids = ids;
+  pp.slot = slot;
+  pp.gates = gates;
+  pp.expert_offset = off;
+  pp.src = x;
+  pp.dst = xbuf;
+  if (launch_dispatch(pp, s) != cudaSuccess) return MOE_ECUDA;
+  if ((st = record(stage_events, 3, s)) != MOE_OK) return st;
+  if ((st = run_ffn(cfg, L, xbuf, x, off, w, ybuf, ws, s, stage_events ? stage_events + 4 : nullptr)) != MOE_OK)
+    return st;
+  if ((st = record(stage_events, 5, s)) != MOE_OK) return st;
+  pp.src = ybuf;
+  pp.dst = y;
+  if (launch_combine(pp, s) != cudaSuccess) return MOE_ECUDA;
+  if ((st = record(stage_events, 6, s)) != MOE_OK) return st;
+  if (launch_aux(at<float>(ws, L.psum), at<int32_t>(ws, L.cnt), L.nblk_router, cfg->E, cfg->T, cfg->k,
+                 cfg->aux_alpha, at<double>(ws, L.term), aux, s) != cudaSuccess)
+    return MOE_ECUDA;
+  if (expert_count != nullptr && cfg->E > 0)
+    if (cudaMemcpyAsync(expert_count, at<int32_t>(ws, L.ecount), sizeof(int32_t) * cfg->E, cudaMemcpyDeviceToDevice,
+                        s) != cudaSuccess)
+      return MOE_ECUDA;
+  return record(stage_events, 7, s);
+}
+
+int moe_sync_status(void* ws, moe_stream_t stream) {
+  if (ws == nullptr) return MOE_EINVAL;
+  cudaStream_t s = S(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ECUDA;
+  DevStatus h{0, 0};
+  if (cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ECUDA;
+  if (cudaMemset(ws, 0, sizeof(DevStatus)) != cudaSuccess) return MOE_ECUDA;
+  return h.code;
+}
+
+int moe_clear_status(void* ws, moe_stream_t stream) {
+  if (ws == nullptr) return MOE_EINVAL;
+  return cuda_status(cudaMemsetAsync(ws, 0, sizeof(DevStatus), S(stream)));
+}
+
+const char* moe_strerror(int status) {
+  switch (status) {
+    case MOE_OK: return "ok";
+    case MOE_EINVAL: return "invalid argument or configuration";
+    case MOE_EUNSUPPORTED: return "configuration outside the supported limits";
+    case MOE_ECUDA: return "CUDA launch or runtime error";
+    case MOE_ETIMEOUT: return "a bounded wait inside a kernel ran out";
+    case MOE_EDEVICE: return "device-side index check failed";
+    case MOE_EWORKSPACE: return "workspace smaller than moe_workspace_size()";
+    default: return "unknown status";
+  }
+}
+
+const char* moe_version(void) { return "moe_b200 0.1 sm_100a"; }
+
+}  // extern "C"

@@ -1,0 +1,128 @@
+// Dispatch permutation and gate-weighted combine: the single-GPU replacements of
+// the dispatch and combine all-to-alls ("Expert-parallel MoE training"
+// explainer: token dispatch to experts and the unpermute / multiply-by-gate /
+// sum step; "Switch Routing" 2.1: y = p_i(x) E_i(x); dropped tokens contribute
+// nothing and reach the output through the caller's residual).
+//
+// Both kernels are token-centric and HBM-bound: one warp per token, 16-byte
+// vectors, every source row read exactly once.  Dispatch writes the token's
+// row to each of its kept destination rows; combine reads the token's kept
+// expert rows (plus its shared-expert row), accumulates in fp32 in choice-rank
+// order and rounds once.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+constexpr int kPermWarps = 8;
+constexpr int kUnroll = 4;
+
+// Destination / source row of each choice of token t (-1 when dropped).
+__device__ __forceinline__ void token_rows(const PermuteParams& p, int64_t t, int64_t (&row)[kMaxK],
+                                           float (&g)[kMaxK]) {
+#pragma unroll
+  for (int r = 0; r < kMaxK; ++r) {
+    row[r] = -1;
+    g[r] = 0.0f;
+    if (r < p.k) {
+      const int s = p.slot[t * p.k + r];
+      const int e = p.ids[t * p.k + r];
+      if (s >= 0 && e >= 0 && e < p.E && (int64_t)p.expert_offset[e] + s < p.rows_max) {
+        row[r] = (int64_t)p.expert_offset[e] + s;
+        if (p.gates != nullptr) g[r] = p.gates[t * p.k + r];
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kPermWarps * 32) dispatch_kernel(PermuteParams p) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * kPermWarps + (threadIdx.x >> 5);
+  if (t >= p.T) return;
+  int64_t row[kMaxK];
+  float g[kMaxK];
+  token_rows(p, t, row, g);
+  const int64_t rowbytes = (int64_t)p.H * p.elem_bytes;
+  const int nvec = (int)(rowbytes / 16);
+  const char* src = static_cast<const char*>(p.src) + t * rowbytes;
+  char* dst = static_cast<char*>(p.dst);
+  for (int v0 = lane; v0 < nvec; v0 += 32 * kUnroll) {
+    int4 val[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int v = v0 + u * 32;
+      if (v < nvec) val[u] = ld_nc_v4(src + (int64_t)v * 16);
+    }
+#pragma unroll
+    for (int r = 0; r < kMaxK; ++r) {
+      if (r < p.k && row[r] >= 0) {
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          const int v = v0 + u * 32;
+          if (v < nvec) st_v4(dst + row[r] * rowbytes + (int64_t)v * 16, val[u]);
+        }
+      }
+    }
+  }
+}
+
+template <typename ET>
+__global__ void __launch_bounds__(kPermWarps * 32) combine_kernel(PermuteParams p) {
+  constexpr int NE = 16 / sizeof(ET);
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * kPermWarps + (threadIdx.x >> 5);
+  if (t >= p.T) return;
+  int64_t row[kMaxK];
+  float g[kMaxK];
+  token_rows(p, t, row, g);
+  const int64_t shared_row = p.n_shared ? (int64_t)p.expert_offset[p.E] + t : -1;
+  const int64_t rowbytes = (int64_t)p.H * sizeof(ET);
+  const int nvec = (int)(rowbytes / 16);
+  const char* ybuf = static_cast<const char*>(p.src);
+  char* y = static_cast<char*>(p.dst) + t * rowbytes;
+  for (int v = lane; v < nvec; v += 32) {
+    float acc[NE];
+#pragma unroll
+    for (int c = 0; c < NE; ++c) acc[c] = 0.0f;
+    int4 val[kMaxK];
+#pragma unroll
+    for (int r = 0; r < kMaxK; ++r)
+      if (r < p.k && row[r] >= 0) val[r] = ld_nc_v4(ybuf + row[r] * rowbytes + (int64_t)v * 16);
+#pragma unroll
+    for (int r = 0; r < kMaxK; ++r) {
+      if (r < p.k && row[r] >= 0) {
+        const ET* e = reinterpret_cast<const ET*>(&val[r]);
+#pragma unroll
+        for (int c = 0; c < NE; ++c) acc[c] = fmaf(g[r], Elem<ET>::to_f(e[c]), acc[c]);
+      }
+    }
+    if (shared_row >= 0) {
+      int4 s = ld_nc_v4(ybuf + shared_row * rowbytes + (int64_t)v * 16);
+      const ET* e = reinterpret_cast<const ET*>(&s);
+#pragma unroll
+      for (int c = 0; c < NE; ++c) acc[c] += Elem<ET>::to_f(e[c]);
+    }
+    int4 out;
+    ET* o = reinterpret_cast<ET*>(&out);
+#pragma unroll
+    for (int c = 0; c < NE; ++c) o[c] = Elem<ET>::from_f(acc[c]);
+    st_v4(y + (int64_t)v * 16, out);
+  }
+}
+
+cudaError_t launch_dispatch(const PermuteParams& p, cudaStream_t stream) {
+  if (p.T == 0) return cudaSuccess;
+  const unsigned grid = (unsigned)((p.T + kPermWarps - 1) / kPermWarps);
+  dispatch_kernel<<<grid, kPermWarps * 32, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const PermuteParams& p, cudaStream_t stream) {
+  if (p.T == 0) return cudaSuccess;
+  const unsigned grid = (unsigned)((p.T + kPermWarps - 1) / kPermWarps);
+  if (p.elem_bytes == 2) combine_kernel<__nv_bfloat16><<<grid, kPermWarps * 32, 0, stream>>>(p);
+  else combine_kernel<float><<<grid, kPermWarps * 32, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

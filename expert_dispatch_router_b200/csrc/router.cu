@@ -1,0 +1,354 @@
+// Router (fp32 logits GEMM + fused softmax / top-k / gates) and the Switch
+// load-balancing loss reduction.
+//
+// Method: "Expert-parallel MoE training" explainer, router section (a linear
+// gate with E outputs, softmax then top-k, Megatron pre_softmax=False) and
+// aux-loss section (alpha * E * sum f_i P_i with top-k in f's denominator);
+// "Switch Routing", 2.1 (p_i(x) softmax, gate = p_i(x)) and 2.2 (the router
+// runs in float32).
+//
+// Design: one CTA of four warps owns BT tokens and all E experts.  The H
+// reduction walks 16-wide chunks: x (bf16 or fp32) is widened to fp32 into
+// shared memory, the Wg chunk is stored transposed so that a lane reads its
+// experts with one conflict-free vector load, and every lane accumulates a
+// TW x EJ register tile with FFMA.  The epilogue keeps each token's E logits
+// spread over the 32 lanes of a warp and does max, sum-of-exp and k rounds of
+// arg-max with warp shuffles, so no logit row ever goes back to memory.  Per-CTA
+// sums of p and selection counts are reduced over the warps in a fixed order
+// (deterministic) and left in the workspace for the aux-loss kernel.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+constexpr int kRouterWarps = 4;
+constexpr int kRouterThreads = kRouterWarps * 32;
+constexpr int kKC = 16;   // H chunk
+
+// Expert held by (lane, j): EJ==1 -> lane; EJ==2 -> 2*lane+j; EJ>=4 -> groups of
+// four consecutive experts per lane, 128 experts per group row.
+template <int EJ>
+__device__ __forceinline__ int lane_expert(int lane, int j) {
+  if constexpr (EJ == 1) return lane;
+  else if constexpr (EJ == 2) return 2 * lane + j;
+  else return 4 * lane + 128 * (j >> 2) + (j & 3);
+}
+
+// Strict order used for top-k: larger logit first, equal logits -> smaller index.
+__device__ __forceinline__ bool better(float la, int ea, float lb, int eb) {
+  return la > lb || (la == lb && ea < eb);
+}
+
+template <int EJ, int TW>
+constexpr int router_smem_floats() {
+  constexpr int EP = 32 * EJ;
+  constexpr int main_ = kRouterWarps * TW * kKC + kKC * (EP + 4);
+  constexpr int red = 2 * kRouterWarps * EP;
+  return main_ > red ? main_ : red;
+}
+
+template <int EJ, int TW, typename XT>
+__global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterParams p) {
+  constexpr int EP = 32 * EJ;
+  constexpr int BT = kRouterWarps * TW;
+  constexpr int WS = EP + 4;
+  extern __shared__ __align__(16) float smem[];
+  float* xs = smem;                       // [BT][kKC]
+  float* wgs = smem + BT * kKC;           // [kKC][WS]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t t0 = (int64_t)blockIdx.x * BT;
+  const int E = p.E, H = p.H;
+
+  float acc[TW][EJ];
+#pragma unroll
+  for (int i = 0; i < TW; ++i)
+#pragma unroll
+    for (int j = 0; j < EJ; ++j) acc[i][j] = 0.0f;
+
+  if (p.logits_in == nullptr) {
+    constexpr int XV = 16 / sizeof(XT);              // elements per 16-byte vector
+    constexpr int XVEC = BT * kKC / XV;              // x vectors per chunk
+    for (int k0 = 0; k0 < H; k0 += kKC) {
+      // global -> registers
+      float xr[(XVEC + kRouterThreads - 1) / kRouterThreads][XV];
+#pragma unroll
+      for (int m = 0; m < (XVEC + kRouterThreads - 1) / kRouterThreads; ++m) {
+        const int q = tid + m * kRouterThreads;
+        const int tok = q / (kKC / XV), kv = q % (kKC / XV);
+        const int64_t t = t0 + tok;
+        const int kk = k0 + kv * XV;
+#pragma unroll
+        for (int c = 0; c < XV; ++c) xr[m][c] = 0.0f;
+        if (q < XVEC && t < p.T && kk < H) {
+          int4 v = ld_nc_v4(static_cast<const XT*>(p.x) + t * H + kk);
+          const XT* e = reinterpret_cast<const XT*>(&v);
+#pragma unroll
+          for (int c = 0; c < XV; ++c) xr[m][c] = Elem<XT>::to_f(e[c]);
+        }
+      }
+      float4 wr[EJ];
+#pragma unroll
+      for (int m = 0; m < EJ; ++m) {
+        const int q = tid + m * kRouterThreads;      // float4 index in [0, EP*4)
+        const int e = q >> 2, kq = q & 3;
+        wr[m] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (e < E && k0 + 4 * kq < H)
+          wr[m] = __ldg(reinterpret_cast<const float4*>(p.wg + (int64_t)e * H + k0 + 4 * kq));
+      }
+      __syncthreads();  // previous chunk consumed
+#pragma unroll
+      for (int m = 0; m < (XVEC + kRouterThreads - 1) / kRouterThreads; ++m) {
+        const int q = tid + m * kRouterThreads;
+        if (q < XVEC) {
+          const int tok = q / (kKC / XV), kv = q % (kKC / XV);
+#pragma unroll
+          for (int c = 0; c < XV; ++c) xs[tok * kKC + kv * XV + c] = xr[m][c];
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < EJ; ++m) {
+        const int q = tid + m * kRouterThreads;
+        const int e = q >> 2, kq = q & 3;
+        wgs[(4 * kq + 0) * WS + e] = wr[m].x;
+        wgs[(4 * kq + 1) * WS + e] = wr[m].y;
+        wgs[(4 * kq + 2) * WS + e] = wr[m].z;
+        wgs[(4 * kq + 3) * WS + e] = wr[m].w;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int kk = 0; kk < kKC; kk += 4) {
+        float4 xv[TW];
+#pragma unroll
+        for (int i = 0; i < TW; ++i)
+          xv[i] = *reinterpret_cast<const float4*>(&xs[(warp * TW + i) * kKC + kk]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float* wrow = wgs + (kk + c) * WS;
+          float wv[EJ];
+          if constexpr (EJ == 1) {
+            wv[0] = wrow[lane];
+          } else if constexpr (EJ == 2) {
+            float2 v = *reinterpret_cast<const float2*>(wrow + 2 * lane);
+            wv[0] = v.x; wv[1] = v.y;
+          } else {
+#pragma unroll
+            for (int g = 0; g < EJ / 4; ++g) {
+              float4 v = *reinterpret_cast<const float4*>(wrow + 4 * lane + 128 * g);
+              wv[4 * g + 0] = v.x; wv[4 * g + 1] = v.y; wv[4 * g + 2] = v.z; wv[4 * g + 3] = v.w;
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < TW; ++i) {
+            const float xc = c == 0 ? xv[i].x : c == 1 ? xv[i].y : c == 2 ? xv[i].z : xv[i].w;
+#pragma unroll
+            for (int j = 0; j < EJ; ++j) acc[i][j] = fmaf(xc, wv[j], acc[i][j]);
+          }
+        }
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < TW; ++i) {
+      const int64_t t = t0 + warp * TW + i;
+#pragma unroll
+      for (int j = 0; j < EJ; ++j) {
+        const int e = lane_expert<EJ>(lane, j);
+        if (t < p.T && e < E) acc[i][j] = p.logits_in[t * E + e];
+      }
+    }
+  }
+
+  // ---------------- epilogue: softmax, top-k, gates, partial sums
+  float psum[EJ];
+  int cnt[EJ];
+#pragma unroll
+  for (int j = 0; j < EJ; ++j) { psum[j] = 0.0f; cnt[j] = 0; }
+
+#pragma unroll
+  for (int i = 0; i < TW; ++i) {
+    const int64_t t = t0 + warp * TW + i;
+    if (t >= p.T) continue;                    // uniform across the warp
+    float l[EJ];
+    float m = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < EJ; ++j) {
+      const int e = lane_expert<EJ>(lane, j);
+      float v = acc[i][j];
+      if (e < E) {
+        if (p.logits_in == nullptr && p.logit_add != nullptr) v += p.logit_add[t * E + e];
+        if (p.logits_out != nullptr) p.logits_out[t * E + e] = v;
+        l[j] = v;
+        m = fmaxf(m, v);
+      } else {
+        l[j] = -INFINITY;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float s = 0.0f, ex[EJ];
+#pragma unroll
+    for (int j = 0; j < EJ; ++j) {
+      ex[j] = lane_expert<EJ>(lane, j) < E ? expf(l[j] - m) : 0.0f;
+      s += ex[j];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const float inv_s = 1.0f / s;
+#pragma unroll
+    for (int j = 0; j < EJ; ++j) psum[j] += ex[j] * inv_s;
+
+    unsigned selected = 0u;
+    float my_l = -INFINITY;
+    int my_e = -1;
+#pragma unroll 1
+    for (int r = 0; r < p.k; ++r) {
+      float bl = -INFINITY;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int j = 0; j < EJ; ++j) {
+        const int e = lane_expert<EJ>(lane, j);
+        if (e < E && !((selected >> j) & 1u) && better(l[j], e, bl, be)) { bl = l[j]; be = e; }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ol = __shfl_xor_sync(0xffffffffu, bl, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        if (better(ol, oe, bl, be)) { bl = ol; be = oe; }
+      }
+#pragma unroll
+      for (int j = 0; j < EJ; ++j)
+        if (lane_expert<EJ>(lane, j) == be) { selected |= 1u << j; cnt[j] += 1; }
+      if (lane == r) { my_l = bl; my_e = be; }
+    }
+    // gates: lane r holds the rank-r selection
+    float g = 0.0f;
+    if (lane < p.k) g = expf(my_l - m);        // top-1 logit equals m
+    if (p.score == MOE_SCORE_SOFTMAX_TOPK) {
+      g *= inv_s;
+      if (p.renorm) {
+        float gs = g;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) gs += __shfl_xor_sync(0xffffffffu, gs, o);
+        g = g / gs;
+      }
+    } else {
+      float gs = g;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) gs += __shfl_xor_sync(0xffffffffu, gs, o);
+      g = g / gs;
+    }
+    if (lane < p.k) {
+      p.ids[t * p.k + lane] = my_e;
+      p.gates[t * p.k + lane] = g;
+    }
+  }
+
+  // ---------------- fixed-order reduction of the per-warp partials
+  __syncthreads();
+  float* rp = smem;                                     // [warps][EP]
+  int* rc = reinterpret_cast<int*>(smem + kRouterWarps * EP);
+#pragma unroll
+  for (int j = 0; j < EJ; ++j) {
+    const int e = lane_expert<EJ>(lane, j);
+    rp[warp * EP + e] = psum[j];
+    rc[warp * EP + e] = cnt[j];
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += kRouterThreads) {
+    float ps = 0.0f;
+    int cs = 0;
+#pragma unroll
+    for (int w = 0; w < kRouterWarps; ++w) { ps += rp[w * EP + e]; cs += rc[w * EP + e]; }
+    p.psum_part[(int64_t)blockIdx.x * E + e] = ps;
+    p.cnt_part[(int64_t)blockIdx.x * E + e] = cs;
+  }
+}
+
+// Tokens per CTA of the router for E experts (the host needs it to size the
+// partial-sum arrays).
+int router_tile_tokens(int E) {
+  const int ej = E <= 32 ? 1 : E <= 64 ? 2 : E <= 128 ? 4 : E <= 256 ? 8 : E <= 512 ? 16 : 32;
+  const int tw = ej <= 8 ? 8 : ej == 16 ? 4 : 2;
+  return kRouterWarps * tw;
+}
+
+template <int EJ, int TW>
+static cudaError_t launch_router_ej(const RouterParams& p, bool bf16, cudaStream_t stream) {
+  constexpr int BT = kRouterWarps * TW;
+  const size_t smem = sizeof(float) * router_smem_floats<EJ, TW>();
+  const unsigned grid = (unsigned)((p.T + BT - 1) / BT);
+  if (bf16) {
+    auto k = router_kernel<EJ, TW, __nv_bfloat16>;
+    if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<grid, kRouterThreads, smem, stream>>>(p);
+  } else {
+    auto k = router_kernel<EJ, TW, float>;
+    if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<grid, kRouterThreads, smem, stream>>>(p);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_router(const RouterParams& p, bool bf16, cudaStream_t stream) {
+  if (p.T == 0) return cudaSuccess;
+  const int E = p.E;
+  if (E <= 32) return launch_router_ej<1, 8>(p, bf16, stream);
+  if (E <= 64) return launch_router_ej<2, 8>(p, bf16, stream);
+  if (E <= 128) return launch_router_ej<4, 8>(p, bf16, stream);
+  if (E <= 256) return launch_router_ej<8, 8>(p, bf16, stream);
+  if (E <= 512) return launch_router_ej<16, 4>(p, bf16, stream);
+  return launch_router_ej<32, 2>(p, bf16, stream);
+}
+
+// ---------------------------------------------------------------- aux loss
+// Warp per expert: P_e and f_e from the router partials (fp64, fixed lane
+// assignment and butterfly order), term[e] = f_e * P_e.
+__global__ void aux_terms_kernel(const float* psum_part, const int32_t* cnt_part, int nblk, int E,
+                                 int64_t T, int k, double* term) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= E) return;
+  double ps = 0.0;
+  long long cs = 0;
+  for (int b = lane; b < nblk; b += 32) {
+    ps += (double)psum_part[(int64_t)b * E + warp];
+    cs += cnt_part[(int64_t)b * E + warp];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    ps += __shfl_xor_sync(0xffffffffu, ps, o);
+    cs += __shfl_xor_sync(0xffffffffu, cs, o);
+  }
+  if (lane == 0) term[warp] = ((double)cs / ((double)T * k)) * (ps / (double)T);
+}
+
+__global__ void aux_final_kernel(const double* term, int E, float alpha, float* aux) {
+  __shared__ double sh[1024];
+  const int tid = threadIdx.x;
+  sh[tid] = tid < E ? term[tid] : 0.0;
+  __syncthreads();
+  for (int s = 512; s > 0; s >>= 1) {
+    if (tid < s) sh[tid] += sh[tid + s];
+    __syncthreads();
+  }
+  if (tid == 0) *aux = (float)((double)alpha * (double)E * sh[0]);
+}
+
+__global__ void aux_zero_kernel(float* aux) { *aux = 0.0f; }
+
+cudaError_t launch_aux(const float* psum_part, const int32_t* cnt_part, int nblk, int E, int64_t T, int k,
+                       float alpha, double* term, float* aux, cudaStream_t stream) {
+  if (T == 0) {
+    aux_zero_kernel<<<1, 1, 0, stream>>>(aux);
+    return cudaGetLastError();
+  }
+  const int threads = 256;
+  const int blocks = (E * 32 + threads - 1) / threads;
+  aux_terms_kernel<<<blocks, threads, 0, stream>>>(psum_part, cnt_part, nblk, E, T, k, term);
+  aux_final_kernel<<<1, 1024, 0, stream>>>(term, E, alpha, aux);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

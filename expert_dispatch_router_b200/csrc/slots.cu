@@ -1,0 +1,216 @@
+// Capacity-slot assignment without a dense [T,E,C] mask.
+//
+// Method: "Expert-parallel MoE training" explainer, drop/pad section ("position"
+// policy: overflow beyond the expert's capacity is dropped in arrival order) and
+// capacity section; "The MoE spends too much time on the gate network"
+// (DeepSpeed discussion 7508) for why the one-hot [T,E,C] mask must not exist.
+//
+// The assignment sequence is a = r*T + t (every first choice in token order,
+// then every second choice, ...).  slot(a) = number of earlier assignments of
+// the same expert.  Four small kernels, all deterministic:
+//   1. count   : CTA c counts its 2048-assignment chunk per expert (shared-memory
+//                histogram) -> chunk_cnt[e][c].
+//   2. scan    : CTA e scans chunk_cnt[e][*] -> chunk base offsets, the expert's
+//                pre-drop count and kept count.
+//   3. offsets : one CTA: exclusive scan of the 128-padded kept counts -> the
+//                per-expert row blocks, then the padding / shared rows of row_token.
+//   4. rank    : CTA c re-reads its chunk; warps rank equal experts inside each
+//                32-assignment step with match_any, carry per-warp running counts,
+//                prefix them over the warps in order, and add the chunk base.
+// Total metadata traffic is O(T*k + E*chunks); nothing scales with C.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+constexpr int kSlotThreads = 256;
+constexpr int kSlotWarps = kSlotThreads / 32;
+constexpr int kStepsPerWarp = kSlotChunk / (kSlotWarps * 32);   // 8
+
+__device__ __forceinline__ int load_assignment(const SlotParams& p, int64_t a, int64_t A) {
+  if (a >= A) return -1;
+  const int64_t r = a / p.T, t = a - r * p.T;
+  return p.ids[t * p.k + r];
+}
+
+__global__ void __launch_bounds__(kSlotThreads) slot_count_kernel(SlotParams p, int nchunk) {
+  extern __shared__ int hist[];
+  const int64_t A = p.T * p.k;
+  for (int e = threadIdx.x; e < p.E; e += kSlotThreads) hist[e] = 0;
+  __syncthreads();
+  const int64_t a0 = (int64_t)blockIdx.x * kSlotChunk;
+  for (int i = threadIdx.x; i < kSlotChunk; i += kSlotThreads) {
+    const int e = load_assignment(p, a0 + i, A);
+    if (a0 + i >= A) break;
+    if (e < 0 || e >= p.E) { set_status(p.status, MOE_EDEVICE, 1); continue; }
+    atomicAdd(&hist[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < p.E; e += kSlotThreads)
+    p.chunk_cnt[(int64_t)e * nchunk + blockIdx.x] = hist[e];
+}
+
+// Exclusive block scan of 256 ints; returns the block total.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* sh, int& excl) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sh[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < kSlotWarps ? sh[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < kSlotWarps; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < kSlotWarps) sh[lane] = w;     // inclusive warp totals
+  }
+  __syncthreads();
+  const int before = warp == 0 ? 0 : sh[warp - 1];
+  const int total = sh[kSlotWarps - 1];
+  excl = before + x - v;
+  __syncthreads();
+  return total;
+}
+
+__global__ void __launch_bounds__(kSlotThreads) slot_scan_kernel(SlotParams p, int nchunk) {
+  __shared__ int sh[kSlotWarps];
+  const int e = blockIdx.x;
+  int* row = p.chunk_cnt + (int64_t)e * nchunk;
+  int running = 0;
+  for (int base = 0; base < nchunk; base += kSlotThreads) {
+    const int c = base + threadIdx.x;
+    const int v = c < nchunk ? row[c] : 0;
+    int excl;
+    const int tot = block_exclusive_scan(v, sh, excl);
+    if (c < nchunk) row[c] = running + excl;        // chunk base, in place
+    running += tot;
+  }
+  if (threadIdx.x == 0) {
+    p.expert_count[e] = running;
+    const int kept = p.capacity < 0 ? running : (int)min((int64_t)running, p.capacity);
+    p.kept_count[e] = kept;
+  }
+}
+
+__global__ void __launch_bounds__(1024) slot_offsets_kernel(SlotParams p) {
+  __shared__ int sh[32];
+  __shared__ int sh_off[kMaxE + 2];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int kept = tid < p.E ? p.kept_count[tid] : 0;
+  const int v = (int)round_up(kept, kRowPad);
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sh[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = sh[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    sh[lane] = w;
+  }
+  __syncthreads();
+  const int excl = (warp == 0 ? 0 : sh[warp - 1]) + x - v;
+  if (tid < p.E) sh_off[tid] = excl;
+  if (tid == 0) {
+    const int routed = sh[31];
+    sh_off[p.E] = routed;
+    const int64_t end = routed + (p.n_shared ? round_up(p.T, kRowPad) : 0);
+    sh_off[p.E + 1] = (int)end;
+    if (end > p.rows_max) set_status(p.status, MOE_EDEVICE, 2);
+  }
+  __syncthreads();
+  for (int i = tid; i < p.E + 2; i += 1024) p.expert_offset[i] = sh_off[i];
+  // padding rows of each routed block -> -1
+  for (int e = warp; e < p.E; e += 32) {
+    const int start = sh_off[e] + p.kept_count[e], stop = sh_off[e + 1];
+    for (int r = start + lane; r < stop; r += 32) p.row_token[r] = -1;
+  }
+  if (p.n_shared) {
+    const int64_t s0 = sh_off[p.E], n = round_up(p.T, kRowPad);
+    for (int64_t i = tid; i < n; i += 1024) p.row_token[s0 + i] = i < p.T ? (int)i : -1;
+  }
+}
+
+__global__ void __launch_bounds__(kSlotThreads) slot_rank_kernel(SlotParams p, int nchunk) {
+  extern __shared__ int wcnt[];                 // [warps][E]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t A = p.T * p.k;
+  for (int i = tid; i < kSlotWarps * p.E; i += kSlotThreads) wcnt[i] = 0;
+  __syncthreads();
+  const int64_t a_warp = (int64_t)blockIdx.x * kSlotChunk + (int64_t)warp * (kStepsPerWarp * 32);
+  const unsigned lt_mask = (1u << lane) - 1u;
+  int local[kStepsPerWarp];
+  int expert[kStepsPerWarp];
+#pragma unroll
+  for (int s = 0; s < kStepsPerWarp; ++s) {
+    const int64_t a = a_warp + s * 32 + lane;
+    int e = load_assignment(p, a, A);          // -1 past the end
+    if (a < A && (e < 0 || e >= p.E)) e = -2;  // bad id: reported by the count kernel
+    expert[s] = e;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    int prior = 0;
+    if (e >= 0) prior = wcnt[warp * p.E + e];
+    local[s] = prior + __popc(peers & lt_mask);
+    __syncwarp();
+    if (e >= 0 && lane == __ffs(peers) - 1) wcnt[warp * p.E + e] = prior + __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  for (int e = tid; e < p.E; e += kSlotThreads) {
+    int run = 0;
+#pragma unroll
+    for (int w = 0; w < kSlotWarps; ++w) {
+      const int v = wcnt[w * p.E + e];
+      wcnt[w * p.E + e] = run;
+      run += v;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int s = 0; s < kStepsPerWarp; ++s) {
+    const int e = expert[s];
+    if (e == -1) continue;
+    const int64_t a = a_warp + s * 32 + lane;
+    const int64_t r = a / p.T, t = a - r * p.T;
+    if (e < 0) { p.slot[t * p.k + r] = -1; continue; }
+    const int pos = p.chunk_cnt[(int64_t)e * nchunk + blockIdx.x] + wcnt[warp * p.E + e] + local[s];
+    const bool kept = p.capacity < 0 || pos < p.capacity;
+    p.slot[t * p.k + r] = kept ? pos : -1;
+    const int64_t row = (int64_t)p.expert_offset[e] + pos;
+    if (kept && row < p.rows_max) p.row_token[row] = (int)t;
+  }
+}
+
+cudaError_t launch_slots(const SlotParams& p, cudaStream_t stream) {
+  const int64_t A = p.T * p.k;
+  const int nchunk = (int)((A + kSlotChunk - 1) / kSlotChunk);
+  if (A > 0) {
+    slot_count_kernel<<<nchunk, kSlotThreads, p.E * sizeof(int), stream>>>(p, nchunk);
+    slot_scan_kernel<<<p.E, kSlotThreads, 0, stream>>>(p, nchunk);
+  } else {
+    cudaMemsetAsync(p.expert_count, 0, p.E * sizeof(int32_t), stream);
+    cudaMemsetAsync(p.kept_count, 0, p.E * sizeof(int32_t), stream);
+  }
+  slot_offsets_kernel<<<1, 1024, 0, stream>>>(p);
+  if (A > 0) {
+    const size_t sm = (size_t)kSlotWarps * p.E * sizeof(int);
+    if (sm > 48 * 1024) cudaFuncSetAttribute(slot_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    slot_rank_kernel<<<nchunk, kSlotThreads, sm, stream>>>(p, nchunk);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,248 @@
+/*
+ * moe_b200.h — C ABI of the B200 (sm_100a) forward pass of one
+ * Mixture-of-Experts FFN layer on a single GPU.
+ *
+ * The pass: router (fp32 logits, softmax, top-k, optional renormalisation),
+ * capacity-slot assignment ("position" policy, or dropless with each expert's
+ * rows padded to a multiple of 128), dispatch permutation into per-expert row
+ * blocks, grouped expert FFN, gate-weighted combine, and the Switch
+ * load-balancing loss.  The two all-to-alls of the multi-device method are
+ * replaced by a local permutation; the dense one-hot [T,E,C] dispatch mask is
+ * never built.
+ *
+ * Sources, cited by page title and section:
+ *   [EP]     "Expert-parallel MoE training" explainer (blog.vllbc.top):
+ *            router, capacity, drop/pad, aux-loss and shared-expert sections,
+ *            worked examples "capacity overflow" and "parameter and dispatch bytes".
+ *   [DS7508] "The MoE spends too much time on the gate network" (DeepSpeed
+ *            discussion 7508): k>2 capacity, dense [T,E,C] mask, cost that must
+ *            follow real tokens rather than capacity.
+ *   [SWITCH] "Switch Routing — MoE Routing, Communication, and Stability":
+ *            2.1 routing math, load balance & capacity; 2.2 selective precision.
+ *   [WIDEEP] InferenceX v2 "WideEP" note: 256 routed + 1 shared expert, top-8.
+ *
+ * Conventions for every entry point below:
+ *   - Pointers named x, wg, ids, ... are DEVICE pointers owned by the caller;
+ *     `cfg` and `w` point to HOST structs read during the call only.
+ *   - The library never allocates device memory.  Scratch lives in a caller
+ *     workspace of moe_workspace_size() bytes, 256-byte aligned.
+ *   - Every compute call is asynchronous on `stream` and never synchronises.
+ *     The return value reports host-side validation and launch errors only;
+ *     errors found on the device (a bad expert id, an exhausted wait) are
+ *     written to a status word in the workspace and read by moe_sync_status().
+ *   - Inputs are read-only; no output may alias an input.
+ *   - Row-major layouts throughout.  Matrices of expert weights are stored the
+ *     way a linear layer stores them, [out_features, in_features].
+ *   - ids, slot, expert_count, kept_count, expert_offset and row_token are
+ *     deterministic: identical inputs give bitwise identical outputs.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t;   /* a cudaStream_t; NULL = legacy default stream */
+typedef struct CUevent_st* moe_event_t;     /* a cudaEvent_t */
+
+/* Status codes. */
+enum {
+  MOE_OK = 0,
+  MOE_EINVAL = 1,        /* null pointer or inconsistent configuration (before any launch) */
+  MOE_EUNSUPPORTED = 2,  /* valid but outside this build's limits (see moe_cfg) */
+  MOE_ECUDA = 3,         /* a CUDA launch or runtime call failed */
+  MOE_ETIMEOUT = 4,      /* device: a bounded wait inside a kernel ran out */
+  MOE_EDEVICE = 5,       /* device: an index check failed (e.g. expert id outside [0,E)) */
+  MOE_EWORKSPACE = 6     /* workspace smaller than moe_workspace_size() */
+};
+
+enum { MOE_ACT_RELU = 0, MOE_ACT_GELU = 1, MOE_ACT_SWIGLU = 2 };
+/* SOFTMAX_TOPK: gates are full-softmax probabilities of the selected experts
+ * ([SWITCH] 2.1), optionally renormalised over the k selected.
+ * TOPK_SOFTMAX: softmax over the k selected logits only ([EP] router section,
+ * Megatron pre_softmax=False). */
+enum { MOE_SCORE_SOFTMAX_TOPK = 0, MOE_SCORE_TOPK_SOFTMAX = 1 };
+/* CAPACITY: C = ceil(T*k*cf/E) slots per expert, overflow dropped ([EP]
+ * capacity and drop/pad sections; [DS7508]).  DROPLESS: every assignment kept
+ * (MegaBlocks as summarised in [EP]). */
+enum { MOE_CAP_CAPACITY = 0, MOE_CAP_DROPLESS = 1 };
+/* Element type of x, expert weights, dispatch buffers and y.  The router
+ * weight, logits, gates and the aux loss are always fp32 ([SWITCH] 2.2). */
+enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
+/* moe_cfg.flags */
+enum { MOE_FLAG_KEEP_LOGITS = 1 };   /* moe_layer_fwd also stores fp32 logits in the workspace */
+
+/* Layer configuration.  Limits of this build: 1 <= E <= 1024, 1 <= k <= min(E,16),
+ * H and F multiples of 8, n_shared in {0,1}, T >= 0 with T*k < 2^31 and every
+ * row count below 2^31.  bf16 uses the tcgen05 tensor-core expert FFN; fp32 uses
+ * an fp32 SIMT expert FFN. */
+typedef struct moe_cfg {
+  int64_t T;             /* tokens */
+  int32_t H;             /* hidden size */
+  int32_t F;             /* expert FFN inner size */
+  int32_t E;             /* routed experts */
+  int32_t k;             /* experts per token */
+  int32_t n_shared;      /* 0 or 1 always-on shared expert ([EP] shared-expert paragraph; [WIDEEP]) */
+  int32_t act;           /* MOE_ACT_* */
+  int32_t score;         /* MOE_SCORE_* */
+  int32_t renorm;        /* 1: divide SOFTMAX_TOPK gates by their sum over the k selected */
+  int32_t cap_mode;      /* MOE_CAP_* */
+  int32_t dtype;         /* MOE_DTYPE_* */
+  int64_t cf_num;        /* capacity factor cf = cf_num / cf_den (exact) */
+  int64_t cf_den;
+  int64_t min_capacity;  /* lower clamp of C (DeepSpeed min_capacity), 0 = none */
+  float aux_alpha;       /* alpha of the load-balancing loss ([SWITCH] 2.1: 1e-2) */
+  int32_t flags;         /* MOE_FLAG_* */
+} moe_cfg;
+
+/* Expert weights (device pointers, element type cfg->dtype).
+ *   w1  [E, F, H]  W_in transposed (ReLU/GELU) or W_gate transposed (SwiGLU)
+ *   w3  [E, F, H]  W_up transposed (SwiGLU only, else NULL)
+ *   w2  [E, H, F]  W_out / W_down transposed
+ *   sw1, sw3, sw2  the shared expert's matrices with the same shapes and E=1
+ *                  (NULL when n_shared == 0). */
+typedef struct moe_weights {
+  const void* w1;
+  const void* w3;
+  const void* w2;
+  const void* sw1;
+  const void* sw3;
+  const void* sw2;
+} moe_weights;
+
+/* Device pointers into a workspace after moe_layer_fwd (see moe_workspace_views). */
+typedef struct moe_ws_views {
+  int32_t* ids;            /* [T,k] selected experts, rank order (largest logit first) */
+  float* gates;            /* [T,k] gate of each selection */
+  int32_t* slot;           /* [T,k] position in the expert's slots, -1 = dropped */
+  int32_t* expert_count;   /* [E] selections per expert before dropping */
+  int32_t* kept_count;     /* [E] kept assignments per expert */
+  int32_t* expert_offset;  /* [E+2] first row of each expert's block; [E] shared block; [E+1] end */
+  int32_t* row_token;      /* [rows_max] source token of each row, -1 for padding rows */
+  float* logits;           /* [T,E] fp32 logits (written only with MOE_FLAG_KEEP_LOGITS) */
+  void* xbuf;              /* [rows_max, H] dispatched rows */
+  void* hbuf;              /* [rows_max, F] expert activations (bf16; fp32 for MOE_DTYPE_F32) */
+  void* ybuf;              /* [rows_max, H] un-gated expert outputs */
+  int64_t rows_max;
+} moe_ws_views;
+
+/* ---- sizing (host only, no CUDA calls) ------------------------------------ */
+
+/* Capacity C of cfg ([EP] capacity section: ceil((T*k/E)*cf), evaluated exactly
+ * in integers; [DS7508]'s ceil((T/E)*cf*k) is the same number), clamped below by
+ * min_capacity.  Writes -1 for MOE_CAP_DROPLESS.  Returns MOE_EINVAL on a bad cfg. */
+MOE_API int moe_capacity(const moe_cfg* cfg, int64_t* capacity);
+
+/* Upper bound on the number of rows of the per-expert buffers (xbuf, hbuf, ybuf):
+ * every expert block padded to 128 rows plus the shared block.  */
+MOE_API int moe_rows_max(const moe_cfg* cfg, int64_t* rows_max);
+
+/* Bytes of workspace needed by moe_layer_fwd; the same workspace serves every
+ * per-stage entry point.  O(T*k + rows_max*(2H+F) + E*blocks) bytes: never the
+ * T*E*C of a dense dispatch mask. */
+MOE_API int moe_workspace_size(const moe_cfg* cfg, size_t* bytes);
+
+/* Device pointers of the workspace regions (host arithmetic on `ws` only). */
+MOE_API int moe_workspace_views(const moe_cfg* cfg, void* ws, moe_ws_views* views);
+
+/* ---- stages ---------------------------------------------------------------- */
+
+/* Router ([EP] router section; [SWITCH] 2.1, 2.2).
+ *   x [T,H] (cfg->dtype), wg [E,H] fp32 (one row per expert), logit_add [T,E] fp32
+ *   or NULL (an additive offset on the logits, e.g. for synthetic load skew).
+ *   logits[t,e] = sum_h x[t,h]*wg[e,h] (+ logit_add) accumulated in fp32;
+ *   p = softmax(logits[t,:]); top-k on the logits (ties to the lower index);
+ *   gates per cfg->score / cfg->renorm.
+ * Writes ids [T,k] int32, gates [T,k] fp32, logits_out [T,E] fp32 if non-NULL,
+ * and per-block sums of p and selection counts into `ws` for moe_aux_loss. */
+MOE_API int moe_route(const moe_cfg* cfg, const void* x, const float* wg, const float* logit_add,
+              int32_t* ids, float* gates, float* logits_out, void* ws, moe_stream_t stream);
+
+/* Same as moe_route after the logits: takes fp32 logits [T,E] (so routing can be
+ * reproduced bit-exactly from given logits). */
+MOE_API int moe_route_from_logits(const moe_cfg* cfg, const float* logits, int32_t* ids, float* gates,
+                          void* ws, moe_stream_t stream);
+
+/* Slot assignment ([EP] drop/pad section, "position" policy; [DS7508] without
+ * the [T,E,C] mask).  Assignments are ordered by (choice rank, token); an
+ * assignment's slot is the number of earlier assignments of its expert; it is
+ * kept iff slot < C (always, when dropless).  Outputs: slot [T,k] (-1 dropped),
+ * expert_count [E] (pre-drop), kept_count [E], expert_offset [E+2] (expert e owns
+ * rows [off[e], off[e]+kept[e]) of a 128-row-padded block; the shared block
+ * [off[E], off[E]+T) follows; off[E+1] = rows used), row_token [rows_max]
+ * (-1 on padding rows).  ids entries outside [0,E) set MOE_EDEVICE. */
+MOE_API int moe_assign_slots(const moe_cfg* cfg, const int32_t* ids, int32_t* slot, int32_t* expert_count,
+                     int32_t* kept_count, int32_t* expert_offset, int32_t* row_token, void* ws,
+                     moe_stream_t stream);
+
+/* Dispatch permutation (the local replacement of the dispatch all-to-all, [EP]):
+ * xbuf[off[e]+slot[t,r], :] = x[t, :] for every kept (t,r).  Padding rows are not
+ * written.  xbuf has rows_max rows. */
+MOE_API int moe_dispatch(const moe_cfg* cfg, const void* x, const int32_t* ids, const int32_t* slot,
+                 const int32_t* expert_offset, void* xbuf, moe_stream_t stream);
+
+/* Grouped expert FFN over the variable per-expert row blocks ([EP] experts and
+ * worked example 2; SwiGLU = silu(x W_gate) * (x W_up) then W_down).  For every
+ * 128-row block of every expert: ybuf = act(xbuf W_in) W_out with fp32
+ * accumulation and the activation rounded once to cfg->dtype.  The shared
+ * expert's block reads its rows straight from x (NULL when n_shared == 0).
+ * Padding rows of ybuf hold unspecified values. */
+MOE_API int moe_expert_ffn(const moe_cfg* cfg, const void* xbuf, const void* x, const int32_t* expert_offset,
+                   const moe_weights* w, void* ybuf, void* ws, moe_stream_t stream);
+
+/* Gate-weighted combine (the local replacement of the combine all-to-all, [EP];
+ * [SWITCH] 2.1 y = p_i(x) E_i(x)): y[t] = sum_{r kept} gates[t,r]*ybuf[row(t,r)]
+ * (+ ybuf[off[E]+t] with weight 1 for the shared expert), fp32 accumulation,
+ * one rounding.  A fully dropped token gets y[t] = 0: the residual is the
+ * caller's ([EP] drop/pad section; [SWITCH] overflow bypass). */
+MOE_API int moe_combine(const moe_cfg* cfg, const void* ybuf, const int32_t* ids, const int32_t* slot,
+                const float* gates, const int32_t* expert_offset, void* y, moe_stream_t stream);
+
+/* Switch load-balancing loss ([SWITCH] 2.1; [EP] aux-loss section):
+ * aux = alpha * E * sum_i f_i * P_i, f_i = pre-drop selections of i / (T*k),
+ * P_i = mean_t p_i(t).  Reads the partials left in `ws` by the last moe_route /
+ * moe_route_from_logits with the same cfg; writes one fp32 to `aux` (device). */
+MOE_API int moe_aux_loss(const moe_cfg* cfg, const void* ws, float* aux, moe_stream_t stream);
+
+/* The whole layer: route -> assign slots -> dispatch -> expert FFN -> combine,
+ * plus the aux loss, on `stream`.  y [T,H] (cfg->dtype) and aux (one fp32) are
+ * device outputs; expert_count [E] is optional (NULL to skip).  The
+ * intermediates stay in `ws` (see moe_workspace_views).  `stage_events`, if
+ * non-NULL, is an array of MOE_N_STAGE_EVENTS events recorded on `stream` before
+ * the router and after each of: router, slots, dispatch, expert FFN first
+ * contraction (with the activation), expert FFN second contraction, combine,
+ * aux loss. */
+enum { MOE_N_STAGE_EVENTS = 8 };
+MOE_API int moe_layer_fwd(const moe_cfg* cfg, const void* x, const float* wg, const float* logit_add,
+                  const moe_weights* w, void* y, float* aux, int32_t* expert_count, void* ws,
+                  size_t ws_bytes, const moe_event_t* stage_events, moe_stream_t stream);
+
+/* ---- status ---------------------------------------------------------------- */
+
+/* Synchronises `stream`, returns the device status word of `ws` (MOE_OK,
+ * MOE_ETIMEOUT or MOE_EDEVICE) and clears it.  MOE_ECUDA if the sync fails. */
+MOE_API int moe_sync_status(void* ws, moe_stream_t stream);
+
+/* Clears the device status word of `ws` (asynchronously on `stream`). */
+MOE_API int moe_clear_status(void* ws, moe_stream_t stream);
+
+/* Static description of a status code. */
+MOE_API const char* moe_strerror(int status);
+
+/* Version string of the library build. */
+MOE_API const char* moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

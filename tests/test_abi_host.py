@@ -1,0 +1,118 @@
+"""The C-ABI library builds, loads without a GPU, exports every symbol that
+include/moe_b200.h declares, and its host-only entry points (sizing,
+validation) behave.  No kernel is launched here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle.moe_oracle as O
+from expert_dispatch_router_b200 import binding as B
+from expert_dispatch_router_b200 import build as build_mod
+from expert_dispatch_router_b200 import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return B.load()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "moe_b200.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(lib, n), n
+    assert lib.moe_version().startswith(b"moe_b200")
+    # nothing but the C ABI is exported
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    assert {n for n in exported if n.startswith("moe_")} == set(names)
+
+
+@pytest.mark.parametrize("shape", list(synth.WORKLOADS.values()), ids=list(synth.WORKLOADS))
+def test_capacity_matches_oracle(lib, shape):
+    cfg = B.make_cfg(shape)
+    want = -1 if shape.cap_mode == synth.CAP_DROPLESS else O.capacity(shape.T, shape.E, shape.k, shape.cf_num,
+                                                                       shape.cf_den, shape.min_capacity)
+    assert B.moe_capacity(cfg) == want
+
+
+def test_capacity_variants(lib):
+    for cf, want in [((1, 1), 10923), ((1, 2), 5462), ((1, 4), 2731), ((2, 1), 21846)]:
+        cfg = B.make_cfg(synth.DS_HIGHK, cf_num=cf[0], cf_den=cf[1])
+        assert B.moe_capacity(cfg) == want
+    cfg = B.make_cfg(synth.SWITCH_TOP1, T=10, E=8, k=1, cf_num=1, cf_den=1, min_capacity=4)
+    assert B.moe_capacity(cfg) == 4
+
+
+def _rows_brute(shape, counts):
+    C = None if shape.cap_mode == synth.CAP_DROPLESS else O.capacity(shape.T, shape.E, shape.k, shape.cf_num,
+                                                                      shape.cf_den, shape.min_capacity)
+    kept = [c if C is None else min(c, C) for c in counts]
+    return int(O.row_layout(kept, shape.T, shape.n_shared)[-1])
+
+
+def test_rows_max_bounds_every_routing(lib):
+    import numpy as np
+    rng = np.random.default_rng(0)
+    for shape in synth.WORKLOADS.values():
+        bound = B.moe_rows_max(B.make_cfg(shape))
+        assert bound % 128 == 0
+        A = shape.T * shape.k
+        # adversarial count vectors: balanced, one hot expert, random
+        cands = [[A // shape.E + (1 if e < A % shape.E else 0) for e in range(shape.E)],
+                 [A] + [0] * (shape.E - 1)]
+        for _ in range(20):
+            cands.append(list(rng.multinomial(A, rng.dirichlet(np.ones(shape.E) * 0.3))))
+        for counts in cands:
+            assert _rows_brute(shape, counts) <= bound
+
+
+def test_workspace_is_not_dense_mask_sized(lib):
+    shape = synth.DS_HIGHK
+    ws = B.moe_workspace_size(B.make_cfg(shape))
+    C = B.moe_capacity(B.make_cfg(shape))
+    dense = O.dense_mask_bytes(shape.T, shape.E, C)
+    assert dense == 34360786944
+    # the workspace holds the three row buffers plus O(T*k) metadata, far below the mask
+    assert ws < dense / 40
+
+
+def test_validation_errors(lib):
+    bad = [dict(k=0), dict(k=13), dict(E=0), dict(E=2000), dict(H=100), dict(F=12), dict(n_shared=2), dict(act=7),
+           dict(score=3), dict(renorm=2), dict(cap_mode=5), dict(dtype=9), dict(cf_num=0), dict(cf_den=-1),
+           dict(T=-1), dict(min_capacity=-3)]
+    for kw in bad:
+        cfg = B.make_cfg(synth.DS_HIGHK, **kw)
+        with pytest.raises(B.MoeError) as ei:
+            B.moe_workspace_size(cfg)
+        assert ei.value.code in (B.MOE_EINVAL, B.MOE_EUNSUPPORTED), kw
+    with pytest.raises(B.MoeError):
+        B.moe_capacity(B.make_cfg(synth.DS_HIGHK, T=1 << 30))      # T*k beyond 2^31
+    # null configuration and null outputs are rejected before any CUDA call
+    assert lib.moe_capacity(None, None) == B.MOE_EINVAL
+    assert lib.moe_route(None, None, None, None, None, None, None, None, None) == B.MOE_EINVAL
+    cfg = B.make_cfg(synth.SWITCH_TINY_F32)
+    assert lib.moe_layer_fwd(ctypes.byref(cfg), None, None, None, None, None, None, None, None, 0, None, None) \
+        == B.MOE_EINVAL
+    w = B.moe_weights()
+    assert lib.moe_expert_ffn(ctypes.byref(cfg), None, None, None, ctypes.byref(w), None, None, None) == B.MOE_EINVAL
+    for code in range(7):
+        assert B.strerror(code)
+
+
+def test_empty_batch_sizes(lib):
+    cfg = B.make_cfg(synth.SWITCH_TOP1, T=0)
+    assert B.moe_rows_max(cfg) == 0
+    assert B.moe_workspace_size(cfg) > 0
