@@ -35,7 +35,7 @@ if ROOT not in sys.path:
 METRIC = "MoE layer tokens/s on 1 B200; dispatch/combine HBM GB/s; expert GEMM TC util %"
 DEFAULT_WORKLOAD = "switch_top1_T8192_H768_E64"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
-LAUNCHES_PER_STEP = 11      # router 1, slots 4, dispatch 1, expert FFN 2, combine 1, aux 2
+LAUNCHES_PER_STEP = 10      # router 1, slots 4, dispatch 1, expert FFN 2, combine 1, aux 1
 
 
 def parse_args():
@@ -74,13 +74,26 @@ def barrier(world):
 
 
 def max_over_ranks(v: float, world: int) -> float:
+    """Largest per-rank value (timing is reported as the slowest rank's)."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cpu" if dist.get_backend() == "gloo" else "cuda"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_seed(base: int, rank: int) -> int:
+    """Each replica draws its own batch (and its own weights) from seed base + rank."""
+    return base + rank
+
+
+def job_tokens_per_s(T: int, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank processes T tokens per step; the step
+    time is the slowest rank's."""
+    return world * T / (ms_per_step / 1e3)
 
 
 def load_peaks():
@@ -325,7 +338,7 @@ def run_ours(args, world, rank, local):
     shape = synth.WORKLOADS[args.workload]
     peaks = load_peaks()
     dev = torch.device("cuda", torch.cuda.current_device())
-    inp = synth.make_inputs(shape, seed=args.seed + rank, device="cuda")
+    inp = synth.make_inputs(shape, seed=replica_seed(args.seed, rank), device="cuda")
     cfg = B.make_cfg(shape)
     ws = B.alloc_workspace(cfg)
     T, H = shape.T, shape.H
@@ -381,7 +394,7 @@ def run_ours(args, world, rank, local):
         stage_ms[name] = sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps
     ms_local = sum(per_step) / args.steps
     ms = max_over_ranks(ms_local, world)
-    value = world * T / (ms / 1e3)
+    value = job_tokens_per_s(T, world, ms)
 
     work = stage_work(shape, kept, experts_used)
     single = ["router", "dispatch", "ffn_gemm1", "ffn_gemm2", "combine"]
@@ -447,7 +460,7 @@ def run_ours(args, world, rank, local):
             "roofline_detail": {s: {k: v[k] for k in ("bound", "achieved", "unit", "frac", "ms_per_launch")}
                                 for s, v in per_stage.items()},
             "dominant_kernel": dom,
-            "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "e2e": {"value": job_tokens_per_s(T, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,
             "clocks": clocks,

@@ -66,6 +66,7 @@ _SIGS = {
     "moe_combine": [CFGP, P, P, P, P, P, P, P],
     "moe_aux_loss": [CFGP, P, P, P],
     "moe_layer_fwd": [CFGP, P, P, P, ctypes.POINTER(moe_weights), P, P, P, P, ctypes.c_size_t, P, P],
+    "moe_activation_eval": [ctypes.c_int, P, P, P, ctypes.c_int64, P],
     "moe_sync_status": [P, P],
     "moe_clear_status": [P, P],
 }
@@ -195,6 +196,11 @@ def moe_layer_fwd(cfg, x, wg, logit_add, weights: moe_weights, y, aux, expert_co
     _check(load().moe_layer_fwd(ctypes.byref(cfg), _ptr(x), _ptr(wg), _ptr(logit_add), ctypes.byref(weights),
                                 _ptr(y), _ptr(aux), _ptr(expert_count), _ptr(ws), ws.numel() * ws.element_size(),
                                 ev, _stream(stream)), "moe_layer_fwd")
+
+
+def moe_activation_eval(act, z, u, out, stream=None):
+    _check(load().moe_activation_eval(int(act), _ptr(z), _ptr(u), _ptr(out), z.numel(), _stream(stream)),
+           "moe_activation_eval")
 
 
 def moe_sync_status(ws, stream=None) -> int:

@@ -47,14 +47,61 @@ __device__ __forceinline__ void st_v4(void* p, int4 v) {
   asm volatile("st.global.v4.s32 [%0], {%1,%2,%3,%4};" :: "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
 
-// Activation functions on fp32 values.
+// Activation functions on fp32 values, written for the GEMM epilogue's
+// instruction budget.
 __device__ __forceinline__ float act_relu(float z) { return fmaxf(z, 0.0f); }
-__device__ __forceinline__ float act_gelu(float z) { return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f)); }
-__device__ __forceinline__ float act_silu(float z) { return z / (1.0f + expf(-z)); }
+
+// erf from Abramowitz & Stegun, Handbook of Mathematical Functions (1964),
+// formula 7.1.26: erf(x) = 1 - (a1 t + ... + a5 t^5) exp(-x^2), t = 1/(1 + p x),
+// x >= 0, absolute error <= 1.5e-7; odd symmetry for x < 0.  The exponential
+// and the reciprocal use the special-function unit.
+__device__ __forceinline__ float erf_as7126(float x) {
+  const float ax = fabsf(x);
+  const float t = __frcp_rn(fmaf(0.3275911f, ax, 1.0f));
+  float poly = fmaf(1.061405429f, t, -1.453152027f);
+  poly = fmaf(poly, t, 1.421413741f);
+  poly = fmaf(poly, t, -0.284496736f);
+  poly = fmaf(poly, t, 0.254829592f);
+  poly *= t;
+  const float r = 1.0f - poly * __expf(-ax * ax);
+  return copysignf(r, x);
+}
+// Exact-form GELU: 0.5 z (1 + erf(z / sqrt 2)).
+__device__ __forceinline__ float act_gelu(float z) { return 0.5f * z * (1.0f + erf_as7126(z * 0.70710678118654752f)); }
+// SiLU: z * sigmoid(z) = z / (1 + exp(-z)).
+__device__ __forceinline__ float act_silu(float z) { return z * __frcp_rn(1.0f + __expf(-z)); }
 
 // Upper bound on the cycles any bounded wait spins before it gives up (~1 s
 // at the B200's boost clock).  Normal waits in these kernels last microseconds.
 constexpr long long kWaitCycles = 2000000000LL;
+
+// Host: raise a kernel's dynamic shared memory limit once per device.
+template <typename Kernel>
+inline cudaError_t ensure_smem(Kernel k, size_t bytes) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  static unsigned long long done = 0;          // one bit per device ordinal (< 64)
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (__atomic_load_n(&done, __ATOMIC_ACQUIRE) & bit) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) __atomic_fetch_or(&done, bit, __ATOMIC_RELEASE);
+  return e;
+}
+
+// Host: multiprocessor count of the current device (cached per device).
+inline int sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int& c = cache[dev & 63];
+  if (c == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    c = n > 0 ? n : 148;
+  }
+  return c;
+}
 
 }  // namespace moe
 

@@ -89,6 +89,21 @@ __global__ void __launch_bounds__(kFThreads) ffn_f32_kernel(FfnF32Params p) {
   }
 }
 
+__global__ void activation_eval_kernel(int act, const float* z, const float* u, float* out, int64_t n) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const float v = z[i];
+    out[i] = act == MOE_ACT_RELU ? act_relu(v) : act == MOE_ACT_GELU ? act_gelu(v) : act_silu(v) * u[i];
+  }
+}
+
+cudaError_t launch_activation_eval(int act, const float* z, const float* u, float* out, int64_t n,
+                                   cudaStream_t stream) {
+  if (n == 0) return cudaSuccess;
+  const int64_t blocks = (n + 255) / 256;
+  activation_eval_kernel<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0, stream>>>(act, z, u, out, n);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_ffn_f32(const FfnF32Params& p, cudaStream_t stream) {
   if (p.rows_max == 0) return cudaSuccess;
   dim3 grid((unsigned)((p.rows_max + kFBM - 1) / kFBM), (unsigned)((p.N + kFBN - 1) / kFBN));

@@ -32,6 +32,9 @@
 // MOE_ETIMEOUT, stops issuing work, drains what it issued and frees TMEM.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <string.h>
+
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -39,14 +42,16 @@
 namespace moe {
 namespace gg {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;
-constexpr int B_BYTES = BN * BK * 2;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int BM = 128, BN = 256, BK = 64;
+constexpr int A_BYTES = BM * BK * 2;              // 16 KB
+constexpr int BBOX = 128;                          // B rows per TMA box
+constexpr int BBOX_BYTES = BBOX * BK * 2;          // 16 KB
+constexpr int RING_BYTES = 4 * (A_BYTES + 2 * BBOX_BYTES);   // 192 KB: 4 wide or 6 narrow stages
+constexpr int MAX_STAGES = 6;
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 64 + EPI_WARPS * 32;
 constexpr int TMEM_COLS = 512;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int SMEM_BYTES = RING_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 
 struct KParams {
   CUtensorMap tmA, tmAs, tmB0, tmB1, tmSB0, tmSB1;
@@ -54,7 +59,7 @@ struct KParams {
   const int32_t* off;
   DevStatus* status;
   int64_t ld_d, rows_max;
-  int K, N_out, n_tiles_n, E, n_shared, epi;
+  int K, N_out, E, n_shared, epi;
   int as_sep;   // 1: the shared block's A rows come from tmAs (row - off[E]); 0: from tmA in place
 };
 
@@ -113,14 +118,16 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
   d |= (uint64_t)2u << 61;                          // layout: 128-byte swizzle
   return d;
 }
-// Instruction descriptor: bf16 x bf16 -> fp32, both operands K-major, M=128, N=256.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+// Instruction descriptor: bf16 x bf16 -> fp32, both operands K-major, M=128, N=n.
+__device__ __forceinline__ uint32_t make_idesc(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
 
-__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accum) {
+__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accum) {
   asm volatile("{\n\t.reg .pred p;\n\t"
                "setp.ne.b32 p, %4, 0;\n\t"
                "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-               :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accum) : "memory");
+               :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum) : "memory");
 }
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" :: "r"(bar) : "memory");
@@ -161,12 +168,12 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-  // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
-  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES);
-  const uint32_t tfull0 = smem_u32(bars + 2 * STAGES), tempty0 = smem_u32(bars + 2 * STAGES + 2);
-  const uint32_t drain = smem_u32(bars + 2 * STAGES + 4);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + RING_BYTES);
+  // bars: full[MAX_STAGES], empty[MAX_STAGES], tfull[2], tempty[2], drain
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + MAX_STAGES);
+  const uint32_t tfull0 = smem_u32(bars + 2 * MAX_STAGES), tempty0 = smem_u32(bars + 2 * MAX_STAGES + 2);
+  const uint32_t drain = smem_u32(bars + 2 * MAX_STAGES + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * MAX_STAGES + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -174,7 +181,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
   const int ngroups = p.E + (p.n_shared ? 1 : 0);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) { mbar_init(full0 + 8 * s, 1); mbar_init(empty0 + 8 * s, 1); }
+    for (int s = 0; s < MAX_STAGES; ++s) { mbar_init(full0 + 8 * s, 1); mbar_init(empty0 + 8 * s, 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(tfull0 + 8 * b, 1); mbar_init(tempty0 + 8 * b, EPI_WARPS * 32); }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -195,20 +202,33 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
 
   const int64_t rows_used = min((int64_t)p.off[ngroups], p.rows_max);
   const int64_t n_mtiles = rows_used / BM;
-  const int64_t n_tiles = n_mtiles * p.n_tiles_n;
   const int nk = (p.K + BK - 1) / BK;
-  const int n_step = swiglu ? BN / 2 : BN;       // output columns per tile
+  // Tile width: SwiGLU tiles hold 128 gate + 128 up columns (128 outputs).
+  // Otherwise 256 columns, or 128 when the wider tile leaves the last wave of
+  // CTAs mostly idle (a narrow tile costs ~0.55 of a wide one).
+  bool narrow = false;
+  if (!swiglu) {
+    const int64_t t256 = n_mtiles * ((p.N_out + 255) / 256), t128 = n_mtiles * ((p.N_out + 127) / 128);
+    const int64_t w256 = (t256 + gridDim.x - 1) / gridDim.x, w128 = (t128 + gridDim.x - 1) / gridDim.x;
+    narrow = 0.55 * (double)w128 < (double)w256;
+  }
+  const int bn = narrow ? 128 : 256;                 // MMA N
+  const int n_step = swiglu ? 128 : bn;              // output columns per tile
+  const int n_tiles_n = (p.N_out + n_step - 1) / n_step;
+  const int64_t n_tiles = n_mtiles * n_tiles_n;
+  const int stage_bytes = A_BYTES + (bn / BBOX) * BBOX_BYTES;
+  const int n_stages = narrow ? 6 : 4;
 
   if (warp == 0) {
     // ---------------- TMA producer
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t fills[STAGES] = {0, 0, 0, 0};
+      uint32_t fills[MAX_STAGES] = {0, 0, 0, 0, 0, 0};
       bool ok = true;
       for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
-        const int64_t mt = tile / p.n_tiles_n;
-        const int nt = (int)(tile % p.n_tiles_n);
+        const int64_t mt = tile / n_tiles_n;
+        const int nt = (int)(tile % n_tiles_n);
         const int64_t row0 = mt * BM;
         const int g = find_group(p.off, ngroups, row0);
         const bool sh = g == p.E;
@@ -221,19 +241,16 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
         const int n0 = nt * n_step;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag)) { ok = false; break; }
-          const uint32_t sa = smem_u32(stage_base + stage * STAGE_BYTES);
+          const uint32_t sa = smem_u32(stage_base + stage * stage_bytes);
           const uint32_t sb = sa + A_BYTES;
           const uint32_t fb = full0 + 8 * stage;
-          mbar_expect_tx(fb, STAGE_BYTES);
+          mbar_expect_tx(fb, stage_bytes);
           tma_load_2d(sa, ma, kb * BK, arow, fb);
-          if (swiglu) {
-            tma_load_3d(sb, mb0, kb * BK, n0, z, fb);
-            tma_load_3d(sb + B_BYTES / 2, mb1, kb * BK, n0, z, fb);
-          } else {
-            tma_load_3d(sb, mb0, kb * BK, n0, z, fb);
-          }
+          tma_load_3d(sb, mb0, kb * BK, n0, z, fb);               // gate / first 128 columns
+          if (swiglu) tma_load_3d(sb + BBOX_BYTES, mb1, kb * BK, n0, z, fb);           // up
+          else if (!narrow) tma_load_3d(sb + BBOX_BYTES, mb0, kb * BK, n0 + BBOX, z, fb);  // next 128
           fills[stage]++;
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          if (++stage == n_stages) { stage = 0; phase ^= 1u; }
         }
       }
       if (!ok) {
@@ -241,7 +258,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
         set_status(p.status, MOE_ETIMEOUT, 10);
       }
       // never leave with a bulk copy still writing this CTA's shared memory
-      for (int s = 0; s < STAGES; ++s)
+      for (int s = 0; s < n_stages; ++s)
         if (fills[s]) {
           const long long t0 = clock64();
           while (!mbar_try_wait(full0 + 8 * s, (fills[s] - 1) & 1u) && clock64() - t0 < kWaitCycles) {}
@@ -255,6 +272,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
+      const uint32_t idesc = make_idesc(bn);
       for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
         if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
@@ -262,14 +280,14 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(full0 + 8 * stage, phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sa = smem_u32(stage_base + stage * STAGE_BYTES);
+          const uint32_t sa = smem_u32(stage_base + stage * stage_bytes);
           const uint32_t sb = sa + A_BYTES;
           const uint64_t ad = sw128_desc(sa), bd = sw128_desc(sb);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)   // advance 16 elements = 32 bytes along K
-            umma(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), (kb | kk) != 0 ? 1u : 0u);
+            umma(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
           umma_commit(empty0 + 8 * stage);      // stage free once these MMAs finish
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          if (++stage == n_stages) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
         umma_commit(tfull0 + 8 * acc);          // accumulator ready for the epilogue
@@ -290,7 +308,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
     const int sub = warp & 3;                  // TMEM sub-partition this warp may access
     const int half = ew >> 2;                  // which half of the output columns
     const int row_in_tile = sub * 32 + lane;
-    const int cols_per_warp = n_step / 2;      // 128 (plain) or 64 (SwiGLU)
+    const int cols_per_warp = n_step / 2;      // 128 or 64 (narrow tile or SwiGLU)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
@@ -300,8 +318,8 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
         break;
       }
       tc_fence_after();
-      const int64_t mt = tile / p.n_tiles_n;
-      const int nt = (int)(tile % p.n_tiles_n);
+      const int64_t mt = tile / n_tiles_n;
+      const int nt = (int)(tile % n_tiles_n);
       const int64_t grow = mt * BM + row_in_tile;
       const int ncol0 = nt * n_step + half * cols_per_warp;    // first output column of this warp
       const uint32_t tbase = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * BN);
@@ -370,26 +388,68 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Encoded maps are cached (keyed by every encode argument), so steady-state
+// launches on the same buffers make no driver call.
+struct MapKey {
+  const void* base;
+  uint32_t rank;
+  cuuint64_t dims[3];
+  cuuint64_t strides[2];
+  cuuint32_t box[3];
+  bool operator==(const MapKey& o) const { return memcmp(this, &o, sizeof(MapKey)) == 0; }
+};
+
+static bool encode_cached(CUtensorMap* out, const MapKey& key) {
+  constexpr int kSlots = 64;
+  static MapKey keys[kSlots];
+  static CUtensorMap maps[kSlots];
+  static int used = 0, next = 0;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (keys[i] == key) { *out = maps[i]; return true; }
+  cuuint32_t es[3] = {1, 1, 1};
+  CUtensorMap m;
+  if (encode_fn()(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, key.rank, const_cast<void*>(key.base), key.dims, key.strides,
+                  key.box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  const int slot = used < kSlots ? used++ : (next++ % kSlots);
+  keys[slot] = key;
+  maps[slot] = m;
+  *out = m;
+  return true;
+}
+
 // 2-D map over a row-major bf16 matrix [rows, K], box 64 x 128.
 static bool make_map_a(CUtensorMap* m, const void* base, int64_t rows, int K) {
-  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-  cuuint32_t box[2] = {BK, BM};
-  cuuint32_t es[2] = {1, 1};
-  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  MapKey key;
+  memset(&key, 0, sizeof(key));
+  key.base = base;
+  key.rank = 2;
+  key.dims[0] = (cuuint64_t)K;
+  key.dims[1] = (cuuint64_t)rows;
+  key.strides[0] = (cuuint64_t)K * 2;
+  key.box[0] = BK;
+  key.box[1] = BM;
+  return encode_cached(m, key);
 }
 
 // 3-D map over stacked weights [G, N, K], box 64 x box_n x 1 (rows past N read as zero).
 static bool make_map_b(CUtensorMap* m, const void* base, int G, int N, int K, int box_n) {
-  cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)N, (cuuint64_t)G};
-  cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)N * K * 2};
-  cuuint32_t box[3] = {BK, (cuuint32_t)box_n, 1};
-  cuuint32_t es[3] = {1, 1, 1};
-  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  MapKey key;
+  memset(&key, 0, sizeof(key));
+  key.base = base;
+  key.rank = 3;
+  key.dims[0] = (cuuint64_t)K;
+  key.dims[1] = (cuuint64_t)N;
+  key.dims[2] = (cuuint64_t)G;
+  key.strides[0] = (cuuint64_t)K * 2;
+  key.strides[1] = (cuuint64_t)N * K * 2;
+  key.box[0] = BK;
+  key.box[1] = (cuuint32_t)box_n;
+  key.box[2] = 1;
+  return encode_cached(m, key);
 }
 
 }  // namespace gg
@@ -398,8 +458,7 @@ cudaError_t launch_grouped_gemm(const GemmParams& p, cudaStream_t stream) {
   using namespace gg;
   if (p.rows_max == 0) return cudaSuccess;
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
-  const bool swiglu = p.epi == MOE_ACT_SWIGLU;
-  const int box_n = swiglu ? BN / 2 : BN;
+  const int box_n = BBOX;
   KParams k{};
   bool ok = make_map_a(&k.tmA, p.a_routed, p.rows_max, p.K);
   ok = ok && make_map_a(&k.tmAs, p.a_shared ? p.a_shared : p.a_routed, p.a_shared ? p.T : p.rows_max, p.K);
@@ -416,21 +475,14 @@ cudaError_t launch_grouped_gemm(const GemmParams& p, cudaStream_t stream) {
   k.as_sep = p.a_shared != nullptr;
   k.K = p.K;
   k.N_out = p.Nw;
-  k.n_tiles_n = (p.Nw + (swiglu ? BN / 2 : BN) - 1) / (swiglu ? BN / 2 : BN);
   k.E = p.E;
   k.n_shared = p.n_shared;
   k.epi = p.epi;
-  static int smem_set = 0;
-  if (!smem_set) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    smem_set = 1;
-  }
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaError_t e = ensure_smem(grouped_gemm_kernel, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const int sms = sm_count();
   // grid: one CTA per SM, never more than the largest possible tile count
-  const int64_t max_tiles = (p.rows_max / BM) * k.n_tiles_n;
+  const int64_t max_tiles = (p.rows_max / BM) * ((p.Nw + BBOX - 1) / BBOX);
   const int grid = (int)(max_tiles < sms ? (max_tiles > 0 ? max_tiles : 1) : sms);
   grouped_gemm_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(k);
   return cudaGetLastError();

@@ -17,13 +17,18 @@ struct RouterParams {
   float* logits_out;        // [T,E] or null
   float* psum_part;         // [nblk,E]
   int32_t* cnt_part;        // [nblk,E]
+  unsigned* aux_counter;    // ticket counter of the aux-loss kernel (re-armed here)
   int64_t T;
   int H, E, k, score, renorm;
 };
 int router_tile_tokens(int E);
 cudaError_t launch_router(const RouterParams& p, bool bf16, cudaStream_t stream);
+// term: E doubles of scratch followed by one unsigned ticket counter.
 cudaError_t launch_aux(const float* psum_part, const int32_t* cnt_part, int nblk, int E, int64_t T, int k,
                        float alpha, double* term, float* aux, cudaStream_t stream);
+// Evaluates the GEMM epilogue's activation: out = act(z) (ReLU, GELU) or silu(z) * u (SwiGLU).
+cudaError_t launch_activation_eval(int act, const float* z, const float* u, float* out, int64_t n,
+                                   cudaStream_t stream);
 
 struct SlotParams {
   const int32_t* ids;       // [T,k]
@@ -39,7 +44,7 @@ struct SlotParams {
   int64_t rows_max;
   DevStatus* status;
 };
-constexpr int kSlotChunk = 2048;   // assignments per CTA of the slot kernels
+constexpr int kSlotChunk = 256;    // assignments per CTA of the slot kernels (one per thread)
 cudaError_t launch_slots(const SlotParams& p, cudaStream_t stream);
 
 struct PermuteParams {

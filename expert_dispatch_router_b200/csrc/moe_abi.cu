@@ -83,7 +83,7 @@ Layout layout_of(const moe_cfg* c) {
   L.status = take(sizeof(DevStatus));
   L.psum = take(sizeof(float) * L.nblk_router * E);
   L.cnt = take(sizeof(int32_t) * L.nblk_router * E);
-  L.term = take(sizeof(double) * E);
+  L.term = take(sizeof(double) * (E + 1));      // E terms + the aux ticket counter
   L.chunk = take(sizeof(int32_t) * E * (size_t)L.nchunk);
   L.ids = take(sizeof(int32_t) * T * k);
   L.gates = take(sizeof(float) * T * k);
@@ -111,6 +111,7 @@ RouterParams router_params(const moe_cfg* c, const Layout& L, void* ws) {
   RouterParams p{};
   p.psum_part = at<float>(ws, L.psum);
   p.cnt_part = at<int32_t>(ws, L.cnt);
+  p.aux_counter = reinterpret_cast<unsigned*>(at<double>(ws, L.term) + c->E);
   p.T = c->T;
   p.H = c->H;
   p.E = c->E;
@@ -464,6 +465,12 @@ const char* moe_strerror(int status) {
     case MOE_EWORKSPACE: return "workspace smaller than moe_workspace_size()";
     default: return "unknown status";
   }
+}
+
+int moe_activation_eval(int act, const float* z, const float* u, float* out, int64_t n, moe_stream_t stream) {
+  if (act < MOE_ACT_RELU || act > MOE_ACT_SWIGLU || n < 0) return MOE_EINVAL;
+  if (n > 0 && (z == nullptr || out == nullptr || (act == MOE_ACT_SWIGLU && u == nullptr))) return MOE_EINVAL;
+  return cuda_status(launch_activation_eval(act, z, u, out, n, S(stream)));
 }
 
 const char* moe_version(void) { return "moe_b200 0.1 sm_100a"; }

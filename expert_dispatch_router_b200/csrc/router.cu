@@ -61,6 +61,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterParams p) 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t t0 = (int64_t)blockIdx.x * BT;
   const int E = p.E, H = p.H;
+  if (blockIdx.x == 0 && tid == 0 && p.aux_counter != nullptr) *p.aux_counter = 0u;
 
   float acc[TW][EJ];
 #pragma unroll
@@ -71,25 +72,20 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterParams p) 
   if (p.logits_in == nullptr) {
     constexpr int XV = 16 / sizeof(XT);              // elements per 16-byte vector
     constexpr int XVEC = BT * kKC / XV;              // x vectors per chunk
-    for (int k0 = 0; k0 < H; k0 += kKC) {
-      // global -> registers
-      float xr[(XVEC + kRouterThreads - 1) / kRouterThreads][XV];
+    constexpr int XM = (XVEC + kRouterThreads - 1) / kRouterThreads;
+    int4 xraw[XM];
+    float4 wr[EJ];
+    // global -> registers for the chunk at k0 (issued one chunk ahead of its use)
+    auto fetch = [&](int k0) {
 #pragma unroll
-      for (int m = 0; m < (XVEC + kRouterThreads - 1) / kRouterThreads; ++m) {
+      for (int m = 0; m < XM; ++m) {
         const int q = tid + m * kRouterThreads;
         const int tok = q / (kKC / XV), kv = q % (kKC / XV);
         const int64_t t = t0 + tok;
         const int kk = k0 + kv * XV;
-#pragma unroll
-        for (int c = 0; c < XV; ++c) xr[m][c] = 0.0f;
-        if (q < XVEC && t < p.T && kk < H) {
-          int4 v = ld_nc_v4(static_cast<const XT*>(p.x) + t * H + kk);
-          const XT* e = reinterpret_cast<const XT*>(&v);
-#pragma unroll
-          for (int c = 0; c < XV; ++c) xr[m][c] = Elem<XT>::to_f(e[c]);
-        }
+        xraw[m] = make_int4(0, 0, 0, 0);
+        if (q < XVEC && t < p.T && kk < H) xraw[m] = ld_nc_v4(static_cast<const XT*>(p.x) + t * H + kk);
       }
-      float4 wr[EJ];
 #pragma unroll
       for (int m = 0; m < EJ; ++m) {
         const int q = tid + m * kRouterThreads;      // float4 index in [0, EP*4)
@@ -98,9 +94,19 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterParams p) 
         if (e < E && k0 + 4 * kq < H)
           wr[m] = __ldg(reinterpret_cast<const float4*>(p.wg + (int64_t)e * H + k0 + 4 * kq));
       }
+    };
+    fetch(0);
+    for (int k0 = 0; k0 < H; k0 += kKC) {
+      float xr[XM][XV];
+#pragma unroll
+      for (int m = 0; m < XM; ++m) {
+        const XT* e = reinterpret_cast<const XT*>(&xraw[m]);
+#pragma unroll
+        for (int c = 0; c < XV; ++c) xr[m][c] = Elem<XT>::to_f(e[c]);
+      }
       __syncthreads();  // previous chunk consumed
 #pragma unroll
-      for (int m = 0; m < (XVEC + kRouterThreads - 1) / kRouterThreads; ++m) {
+      for (int m = 0; m < XM; ++m) {
         const int q = tid + m * kRouterThreads;
         if (q < XVEC) {
           const int tok = q / (kKC / XV), kv = q % (kKC / XV);
@@ -118,6 +124,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterParams p) 
         wgs[(4 * kq + 3) * WS + e] = wr[m].w;
       }
       __syncthreads();
+      if (k0 + kKC < H) fetch(k0 + kKC);             // next chunk's loads overlap this chunk's FFMAs
 #pragma unroll
       for (int kk = 0; kk < kKC; kk += 4) {
         float4 xv[TW];
@@ -282,11 +289,13 @@ static cudaError_t launch_router_ej(const RouterParams& p, bool bf16, cudaStream
   const unsigned grid = (unsigned)((p.T + BT - 1) / BT);
   if (bf16) {
     auto k = router_kernel<EJ, TW, __nv_bfloat16>;
-    if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_smem(k, smem);
+    if (e != cudaSuccess) return e;
     k<<<grid, kRouterThreads, smem, stream>>>(p);
   } else {
     auto k = router_kernel<EJ, TW, float>;
-    if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_smem(k, smem);
+    if (e != cudaSuccess) return e;
     k<<<grid, kRouterThreads, smem, stream>>>(p);
   }
   return cudaGetLastError();
@@ -304,50 +313,62 @@ cudaError_t launch_router(const RouterParams& p, bool bf16, cudaStream_t stream)
 }
 
 // ---------------------------------------------------------------- aux loss
-// Warp per expert: P_e and f_e from the router partials (fp64, fixed lane
-// assignment and butterfly order), term[e] = f_e * P_e.
-__global__ void aux_terms_kernel(const float* psum_part, const int32_t* cnt_part, int nblk, int E,
-                                 int64_t T, int k, double* term) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (warp >= E) return;
-  double ps = 0.0;
-  long long cs = 0;
-  for (int b = lane; b < nblk; b += 32) {
-    ps += (double)psum_part[(int64_t)b * E + warp];
-    cs += cnt_part[(int64_t)b * E + warp];
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    ps += __shfl_xor_sync(0xffffffffu, ps, o);
-    cs += __shfl_xor_sync(0xffffffffu, cs, o);
-  }
-  if (lane == 0) term[warp] = ((double)cs / ((double)T * k)) * (ps / (double)T);
-}
+// Warp per expert: its lanes stride over the router blocks' partials in fp64
+// and reduce with a fixed butterfly into term[e] = f_e * P_e.  The last CTA to
+// finish (a ticket counter) sums the terms in a fixed order, so the result is
+// deterministic, and re-arms the counter.  The router also re-arms it.
+constexpr int kAuxWarps = 8;
 
-__global__ void aux_final_kernel(const double* term, int E, float alpha, float* aux) {
-  __shared__ double sh[1024];
-  const int tid = threadIdx.x;
-  sh[tid] = tid < E ? term[tid] : 0.0;
+__global__ void __launch_bounds__(kAuxWarps * 32) aux_kernel(const float* psum_part, const int32_t* cnt_part,
+                                                             int nblk, int E, int64_t T, int k, float alpha,
+                                                             double* term, unsigned* counter, float* aux) {
+  __shared__ double sh[kAuxWarps * 32];
+  __shared__ bool last;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+  if (T == 0) {
+    if (tid == 0) *aux = 0.0f;
+    return;
+  }
+  const int e = blockIdx.x * kAuxWarps + warp;
+  if (e < E) {
+    double ps = 0.0;
+    long long cs = 0;
+    for (int b = lane; b < nblk; b += 32) {
+      ps += (double)psum_part[(int64_t)b * E + e];
+      cs += cnt_part[(int64_t)b * E + e];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      ps += __shfl_xor_sync(0xffffffffu, ps, o);
+      cs += __shfl_xor_sync(0xffffffffu, cs, o);
+    }
+    if (lane == 0) term[e] = ((double)cs / ((double)T * k)) * (ps / (double)T);
+  }
+  __threadfence();
   __syncthreads();
-  for (int s = 512; s > 0; s >>= 1) {
-    if (tid < s) sh[tid] += sh[tid + s];
+  if (tid == 0) last = atomicAdd(counter, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  double v = 0.0;
+  for (int i = tid; i < E; i += kAuxWarps * 32) v += __ldcg(term + i);
+  sh[tid] = v;
+  __syncthreads();
+  for (int s2 = kAuxWarps * 16; s2 > 0; s2 >>= 1) {
+    if (tid < s2) sh[tid] += sh[tid + s2];
     __syncthreads();
   }
-  if (tid == 0) *aux = (float)((double)alpha * (double)E * sh[0]);
+  if (tid == 0) {
+    *aux = (float)((double)alpha * (double)E * sh[0]);
+    *counter = 0u;
+  }
 }
-
-__global__ void aux_zero_kernel(float* aux) { *aux = 0.0f; }
 
 cudaError_t launch_aux(const float* psum_part, const int32_t* cnt_part, int nblk, int E, int64_t T, int k,
                        float alpha, double* term, float* aux, cudaStream_t stream) {
-  if (T == 0) {
-    aux_zero_kernel<<<1, 1, 0, stream>>>(aux);
-    return cudaGetLastError();
-  }
-  const int threads = 256;
-  const int blocks = (E * 32 + threads - 1) / threads;
-  aux_terms_kernel<<<blocks, threads, 0, stream>>>(psum_part, cnt_part, nblk, E, T, k, term);
-  aux_final_kernel<<<1, 1024, 0, stream>>>(term, E, alpha, aux);
+  unsigned* counter = reinterpret_cast<unsigned*>(term + E);
+  const int grid = T == 0 ? 1 : (E + kAuxWarps - 1) / kAuxWarps;
+  aux_kernel<<<grid, kAuxWarps * 32, 0, stream>>>(psum_part, cnt_part, nblk, E, T, k, alpha, term, counter, aux);
   return cudaGetLastError();
 }
 

@@ -207,7 +207,8 @@ cudaError_t launch_slots(const SlotParams& p, cudaStream_t stream) {
   slot_offsets_kernel<<<1, 1024, 0, stream>>>(p);
   if (A > 0) {
     const size_t sm = (size_t)kSlotWarps * p.E * sizeof(int);
-    if (sm > 48 * 1024) cudaFuncSetAttribute(slot_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    cudaError_t e = ensure_smem(slot_rank_kernel, sm);
+    if (e != cudaSuccess) return e;
     slot_rank_kernel<<<nchunk, kSlotThreads, sm, stream>>>(p, nchunk);
   }
   return cudaGetLastError();

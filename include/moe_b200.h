@@ -227,6 +227,13 @@ MOE_API int moe_layer_fwd(const moe_cfg* cfg, const void* x, const float* wg, co
                   const moe_weights* w, void* y, float* aux, int32_t* expert_count, void* ws,
                   size_t ws_bytes, const moe_event_t* stage_events, moe_stream_t stream);
 
+/* The activation exactly as the expert-FFN epilogues evaluate it, on n fp32
+ * values (device pointers): out = relu(z) or gelu(z) = 0.5 z (1 + erf(z/sqrt 2))
+ * with erf from Abramowitz & Stegun formula 7.1.26 (|error| <= 1.5e-7), or for
+ * MOE_ACT_SWIGLU out = silu(z) * u.  Exposed so the approximation can be
+ * checked against its error bound. */
+MOE_API int moe_activation_eval(int act, const float* z, const float* u, float* out, int64_t n, moe_stream_t stream);
+
 /* ---- status ---------------------------------------------------------------- */
 
 /* Synchronises `stream`, returns the device status word of `ws` (MOE_OK,
