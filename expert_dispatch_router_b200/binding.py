@@ -61,6 +61,7 @@ _SIGS = {
     "moe_route": [CFGP, P, P, P, P, P, P, P, P],
     "moe_route_from_logits": [CFGP, P, P, P, P, P],
     "moe_assign_slots": [CFGP, P, P, P, P, P, P, P, P],
+    "moe_assign_slots_static": [CFGP, P, P, P, P, P, P, P],
     "moe_dispatch": [CFGP, P, P, P, P, P, P],
     "moe_expert_ffn": [CFGP, P, P, P, ctypes.POINTER(moe_weights), P, P, P],
     "moe_combine": [CFGP, P, P, P, P, P, P, P],
@@ -166,6 +167,12 @@ def moe_assign_slots(cfg, ids, slot, expert_count, kept_count, expert_offset, ro
     _check(load().moe_assign_slots(ctypes.byref(cfg), _ptr(ids), _ptr(slot), _ptr(expert_count), _ptr(kept_count),
                                    _ptr(expert_offset), _ptr(row_token), _ptr(ws), _stream(stream)),
            "moe_assign_slots")
+
+
+def moe_assign_slots_static(cfg, ids, slot, expert_count, kept_count, expert_offset, row_token, stream=None):
+    _check(load().moe_assign_slots_static(ctypes.byref(cfg), _ptr(ids), _ptr(slot), _ptr(expert_count),
+                                          _ptr(kept_count), _ptr(expert_offset), _ptr(row_token), _stream(stream)),
+           "moe_assign_slots_static")
 
 
 def moe_dispatch(cfg, x, ids, slot, expert_offset, xbuf, stream=None):

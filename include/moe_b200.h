@@ -185,6 +185,29 @@ MOE_API int moe_assign_slots(const moe_cfg* cfg, const int32_t* ids, int32_t* sl
                      int32_t* kept_count, int32_t* expert_offset, int32_t* row_token, void* ws,
                      moe_stream_t stream);
 
+/* moe_assign_slots for callers that cannot allocate device memory.  No source
+ * page has a counterpart: this is a deployment variant.  Some callers get
+ * only their input and output buffers and may not allocate anything else, for
+ * example a plugin inside a framework whose memory pool owns the whole device,
+ * or a latency-critical path where an allocation (and the synchronisation it
+ * can imply) is not allowed.  This entry point takes no workspace and calls no
+ * allocator; it computes exactly what moe_assign_slots computes (same
+ * arguments, same outputs, same kernels).
+ * Scratch: a fixed 1 MiB device array inside the library, held by every GPU that
+ * loads the library until the process exits.  It fits E * ceil(T*k/256) <=
+ * 262080 (e.g. E=256 with T*k up to 262,080 assignments); larger configurations
+ * return MOE_EUNSUPPORTED before any launch.
+ * All calls on a device share that array and it keeps the last call's contents;
+ * the call clears the part that must start at zero.  Calls whose work
+ * overlaps on the GPU (concurrent streams) race on the array: order them.
+ * The first call on each device looks up the array's device address (with that
+ * device current); make that first call before any stream capture.  An expert
+ * id outside [0,E) gives slot -1 for that assignment; this variant has no
+ * status word for the caller to read. */
+MOE_API int moe_assign_slots_static(const moe_cfg* cfg, const int32_t* ids, int32_t* slot, int32_t* expert_count,
+                                    int32_t* kept_count, int32_t* expert_offset, int32_t* row_token,
+                                    moe_stream_t stream);
+
 /* Dispatch permutation (the local replacement of the dispatch all-to-all, [EP]):
  * xbuf[off[e]+slot[t,r], :] = x[t, :] for every kept (t,r).  Padding rows are not
  * written.  xbuf has rows_max rows. */
