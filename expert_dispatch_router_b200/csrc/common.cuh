@@ -51,13 +51,21 @@ __device__ __forceinline__ void st_v4(void* p, int4 v) {
 // instruction budget.
 __device__ __forceinline__ float act_relu(float z) { return fmaxf(z, 0.0f); }
 
+// Reciprocal on the special-function unit (PTX rcp.approx: about 1 ulp;
+// rcp(+inf) = 0).
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
 // erf from Abramowitz & Stegun, Handbook of Mathematical Functions (1964),
 // formula 7.1.26: erf(x) = 1 - (a1 t + ... + a5 t^5) exp(-x^2), t = 1/(1 + p x),
 // x >= 0, absolute error <= 1.5e-7; odd symmetry for x < 0.  The exponential
 // and the reciprocal use the special-function unit.
 __device__ __forceinline__ float erf_as7126(float x) {
   const float ax = fabsf(x);
-  const float t = __frcp_rn(fmaf(0.3275911f, ax, 1.0f));
+  const float t = rcp_approx(fmaf(0.3275911f, ax, 1.0f));
   float poly = fmaf(1.061405429f, t, -1.453152027f);
   poly = fmaf(poly, t, 1.421413741f);
   poly = fmaf(poly, t, -0.284496736f);
@@ -69,7 +77,7 @@ __device__ __forceinline__ float erf_as7126(float x) {
 // Exact-form GELU: 0.5 z (1 + erf(z / sqrt 2)).
 __device__ __forceinline__ float act_gelu(float z) { return 0.5f * z * (1.0f + erf_as7126(z * 0.70710678118654752f)); }
 // SiLU: z * sigmoid(z) = z / (1 + exp(-z)).
-__device__ __forceinline__ float act_silu(float z) { return z * __frcp_rn(1.0f + __expf(-z)); }
+__device__ __forceinline__ float act_silu(float z) { return z * rcp_approx(1.0f + __expf(-z)); }
 
 // Upper bound on the cycles any bounded wait spins before it gives up (~1 s
 // at the B200's boost clock).  Normal waits in these kernels last microseconds.

@@ -1,35 +1,39 @@
-// Grouped expert GEMM on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+// Grouped GEMM on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
 //
 // Method: the per-expert FFN of an MoE layer ("Expert-parallel MoE training"
 // explainer: experts as grouped MLPs, SwiGLU experts with gate / up / down
 // matrices in worked example 2; MegaBlocks' dropless layout with every expert
 // batch padded to a multiple of 128 rows).  The expert FFN is the only dense
 // contraction of the layer; "The MoE spends too much time on the gate network"
-// measures it at 87-99% of the layer once dispatch is fixed.
+// measures it at 87-99% of the layer once dispatch is fixed.  The same kernel
+// also computes the router logits (one group, fp32 store; see
+// launch_router_gemm).
 //
-// One launch computes, for every 128-row block of every expert g,
+// One launch computes, for every 128-row block of every group g,
 //     D[rows, n-tile] = epi( A[rows, :] * B_g[n-tile, :]^T )
-// with bf16 operands, fp32 accumulation in tensor memory, and a bf16 store.
+// with bf16 operands and fp32 accumulation in tensor memory.
 //   GEMM1: A = dispatched rows (the shared expert's block reads x directly),
-//          B = W_in^T (or W_gate^T | W_up^T stacked for SwiGLU), epi = act.
-//   GEMM2: A = activations h, B = W_out^T, epi = none.
+//          B = W_in^T (or W_gate^T | W_up^T stacked for SwiGLU), epi = act, bf16 out.
+//   GEMM2: A = activations h, B = W_out^T, epi = none, bf16 out.
+//   router: A = x (its k coordinate wraps every H' columns), B = the three bf16
+//          planes of Wg laid side by side along K, fp32 out.
 //
 // Kernel structure (one persistent CTA per SM, 320 threads):
-//   warp 0      TMA producer: A tile 128x64 and B tile 256x64 per stage,
-//               128-byte swizzle, 4-stage ring guarded by full/empty mbarriers.
+//   warp 0      TMA producer: A box 64x128 and B boxes 64 x (<=128) per stage,
+//               128-byte swizzle, a 4-8 stage ring guarded by full/empty mbarriers.
 //   warp 1      allocates 512 TMEM columns and issues tcgen05.mma
-//               (M=128, N=256, K=16, kind::f16) from one lane; commits free the
+//               (M=128, N<=256, K=16, kind::f16) from one lane; commits free the
 //               smem stage and, per tile, signal the accumulator as full.
 //   warps 2-9   epilogue: tcgen05.ld of the fp32 accumulator (each warp owns
 //               one 32-lane TMEM sub-partition and half the columns), the
-//               activation, bf16 packing and 16-byte global stores.
+//               activation, packing and 16-byte global stores.
 // Two accumulators of 256 columns let the epilogue of one tile overlap the
 // main loop of the next.  Tiles are walked m-block-major, n fastest, so CTAs
-// running at the same time share the A block and the expert's weights in L2.
-// The expert of an m-block comes from a binary search over the device-side
-// expert offsets, so no host synchronisation is needed between routing and
-// the GEMM.  Every mbarrier wait is bounded; on expiry the CTA records
-// MOE_ETIMEOUT, stops issuing work, drains what it issued and frees TMEM.
+// running at the same time share the A block and the group's weights in L2.
+// The group of an m-block comes from a binary search over the device-side
+// offsets, so no host synchronisation is needed between routing and the GEMM.
+// Every mbarrier wait is bounded; on expiry the CTA records MOE_ETIMEOUT, stops
+// issuing work, drains what it issued and frees TMEM.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <string.h>
@@ -44,10 +48,8 @@ namespace gg {
 
 constexpr int BM = 128, BN = 256, BK = 64;
 constexpr int A_BYTES = BM * BK * 2;              // 16 KB
-constexpr int BBOX = 128;                          // B rows per TMA box
-constexpr int BBOX_BYTES = BBOX * BK * 2;          // 16 KB
-constexpr int RING_BYTES = 4 * (A_BYTES + 2 * BBOX_BYTES);   // 192 KB: 4 wide or 6 narrow stages
-constexpr int MAX_STAGES = 6;
+constexpr int RING_BYTES = 4 * (A_BYTES + BN * BK * 2);   // 192 KB: 4 stages at N=256, more when narrower
+constexpr int MAX_STAGES = 8;
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 64 + EPI_WARPS * 32;
 constexpr int TMEM_COLS = 512;
@@ -59,8 +61,15 @@ struct KParams {
   const int32_t* off;
   DevStatus* status;
   int64_t ld_d, rows_max;
+  int64_t rows_static;   // >= 0: one group of this many rows (off unused)
+  int64_t rows_store;    // rows >= rows_store are not stored
   int K, N_out, E, n_shared, epi;
-  int as_sep;   // 1: the shared block's A rows come from tmAs (row - off[E]); 0: from tmA in place
+  int as_sep;            // 1: the shared block's A rows come from tmAs (row - off[E]); 0: from tmA in place
+  int bn_fixed;          // 0: N tile chosen on the device (256 or 128); else this MMA N (multiple of 16)
+  int bbox;              // rows of one B TMA box (128, or bn_fixed when smaller)
+  int a_kwrap;           // > 0 (router): B holds 3 planes of a_kwrap k blocks; A's k block = kb / 3
+  int plane_split;       // router: 1 = one tile per (m-block, n-tile, plane), fp32 partials per plane
+  int out_f32;           // 1: store the raw fp32 accumulator
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -135,16 +144,35 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+// tcgen05.ld 32x32b of n (32, 16 or 8, warp-uniform) consecutive columns into v[0..n).
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[32], int n) {
   uint32_t r[32];
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-               "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-               "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-                 "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-                 "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-                 "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-               : "r"(taddr));
+  if (n == 32) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+                 "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+                 "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+                   "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+                   "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+                   "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+                 : "r"(taddr));
+  } else if (n == 16) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+                 "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+                   "=r"(r[15])
+                 : "r"(taddr));
+#pragma unroll
+    for (int i = 16; i < 32; ++i) r[i] = 0u;
+  } else {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+#pragma unroll
+    for (int i = 8; i < 32; ++i) r[i] = 0u;
+  }
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
@@ -178,6 +206,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool swiglu = p.epi == MOE_ACT_SWIGLU;
+  const bool grouped = p.rows_static < 0;
   const int ngroups = p.E + (p.n_shared ? 1 : 0);
 
   if (threadIdx.x == 0) {
@@ -200,38 +229,43 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int64_t rows_used = min((int64_t)p.off[ngroups], p.rows_max);
-  const int64_t n_mtiles = rows_used / BM;
+  const int64_t rows_used = grouped ? min((int64_t)p.off[ngroups], p.rows_max) : p.rows_static;
+  const int64_t n_mtiles = (rows_used + BM - 1) / BM;
   const int nk = (p.K + BK - 1) / BK;
   // Tile width: SwiGLU tiles hold 128 gate + 128 up columns (128 outputs).
   // Otherwise 256 columns, or 128 when the wider tile leaves the last wave of
-  // CTAs mostly idle (a narrow tile costs ~0.55 of a wide one).
+  // CTAs mostly idle (a narrow tile costs ~0.55 of a wide one), or a fixed N.
   bool narrow = false;
-  if (!swiglu) {
+  if (!swiglu && p.bn_fixed == 0) {
     const int64_t t256 = n_mtiles * ((p.N_out + 255) / 256), t128 = n_mtiles * ((p.N_out + 127) / 128);
     const int64_t w256 = (t256 + gridDim.x - 1) / gridDim.x, w128 = (t128 + gridDim.x - 1) / gridDim.x;
     narrow = 0.55 * (double)w128 < (double)w256;
   }
-  const int bn = narrow ? 128 : 256;                 // MMA N
-  const int n_step = swiglu ? 128 : bn;              // output columns per tile
+  const int bn = p.bn_fixed ? p.bn_fixed : (narrow ? 128 : 256);   // MMA N
+  const int n_step = swiglu ? BN / 2 : bn;                          // output columns per tile
   const int n_tiles_n = (p.N_out + n_step - 1) / n_step;
-  const int64_t n_tiles = n_mtiles * n_tiles_n;
-  const int stage_bytes = A_BYTES + (bn / BBOX) * BBOX_BYTES;
-  const int n_stages = narrow ? 6 : 4;
+  const int n_planes = p.plane_split ? 3 : 1;
+  const int64_t n_tiles = n_mtiles * n_tiles_n * n_planes;
+  const int nk_tile = p.plane_split ? p.a_kwrap : nk;    // k blocks per tile
+  const int box_bytes = p.bbox * BK * 2;
+  const int n_boxes = swiglu ? 2 : bn / p.bbox;
+  const int stage_bytes = A_BYTES + n_boxes * box_bytes;
+  const int n_stages = min(MAX_STAGES, RING_BYTES / stage_bytes);
 
   if (warp == 0) {
     // ---------------- TMA producer
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t fills[MAX_STAGES] = {0, 0, 0, 0, 0, 0};
+      uint32_t fills[MAX_STAGES] = {0, 0, 0, 0, 0, 0, 0, 0};
       bool ok = true;
       for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
-        const int64_t mt = tile / n_tiles_n;
-        const int nt = (int)(tile % n_tiles_n);
+        const int plane = (int)(tile % n_planes);
+        const int64_t mt = tile / n_planes / n_tiles_n;
+        const int nt = (int)(tile / n_planes % n_tiles_n);
         const int64_t row0 = mt * BM;
-        const int g = find_group(p.off, ngroups, row0);
-        const bool sh = g == p.E;
+        const int g = grouped ? find_group(p.off, ngroups, row0) : 0;
+        const bool sh = grouped && g == p.E;
         const bool sep = sh && p.as_sep;
         const CUtensorMap* ma = sep ? &p.tmAs : &p.tmA;
         const CUtensorMap* mb0 = sh ? &p.tmSB0 : &p.tmB0;
@@ -239,16 +273,24 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
         const int arow = (int)(sep ? row0 - p.off[p.E] : row0);
         const int z = sh ? 0 : g;
         const int n0 = nt * n_step;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = 0; kb < nk_tile; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag)) { ok = false; break; }
           const uint32_t sa = smem_u32(stage_base + stage * stage_bytes);
           const uint32_t sb = sa + A_BYTES;
           const uint32_t fb = full0 + 8 * stage;
+          // Router mode (a_kwrap = H'/64 > 0): the three weight planes of one A chunk
+          // are consecutive k blocks, so the A chunk is re-read from L2 right away.
+          const int ka = (p.a_kwrap > 0 && !p.plane_split ? kb / 3 : kb) * BK;
+          const int kbb = (p.plane_split ? plane * p.a_kwrap + kb
+                           : p.a_kwrap > 0 ? (kb % 3) * p.a_kwrap + kb / 3 : kb) * BK;
           mbar_expect_tx(fb, stage_bytes);
-          tma_load_2d(sa, ma, kb * BK, arow, fb);
-          tma_load_3d(sb, mb0, kb * BK, n0, z, fb);               // gate / first 128 columns
-          if (swiglu) tma_load_3d(sb + BBOX_BYTES, mb1, kb * BK, n0, z, fb);           // up
-          else if (!narrow) tma_load_3d(sb + BBOX_BYTES, mb0, kb * BK, n0 + BBOX, z, fb);  // next 128
+          tma_load_2d(sa, ma, ka, arow, fb);
+          if (swiglu) {
+            tma_load_3d(sb, mb0, kbb, n0, z, fb);                 // gate rows
+            tma_load_3d(sb + box_bytes, mb1, kbb, n0, z, fb);     // up rows
+          } else {
+            for (int b = 0; b < n_boxes; ++b) tma_load_3d(sb + b * box_bytes, mb0, kbb, n0 + b * p.bbox, z, fb);
+          }
           fills[stage]++;
           if (++stage == n_stages) { stage = 0; phase ^= 1u; }
         }
@@ -277,7 +319,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
         if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = 0; kb < nk_tile; ++kb) {
           if (!mbar_wait(full0 + 8 * stage, phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(stage_base + stage * stage_bytes);
@@ -308,7 +350,8 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
     const int sub = warp & 3;                  // TMEM sub-partition this warp may access
     const int half = ew >> 2;                  // which half of the output columns
     const int row_in_tile = sub * 32 + lane;
-    const int cols_per_warp = n_step / 2;      // 128 or 64 (narrow tile or SwiGLU)
+    const int cols_per_warp = n_step / 2;      // 128, 64, or bn/2 for a fixed N
+    const int chunk = cols_per_warp >= 32 ? 32 : cols_per_warp >= 16 ? 16 : 8;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
@@ -318,19 +361,20 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
         break;
       }
       tc_fence_after();
-      const int64_t mt = tile / n_tiles_n;
-      const int nt = (int)(tile % n_tiles_n);
+      const int plane = (int)(tile % n_planes);
+      const int64_t mt = tile / n_planes / n_tiles_n;
+      const int nt = (int)(tile / n_planes % n_tiles_n);
       const int64_t grow = mt * BM + row_in_tile;
+      const bool row_ok = grow < p.rows_store;
       const int ncol0 = nt * n_step + half * cols_per_warp;    // first output column of this warp
       const uint32_t tbase = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * BN);
-      uint8_t* drow = static_cast<uint8_t*>(p.d) + grow * p.ld_d * 2;
-      for (int c = 0; c < cols_per_warp; c += 32) {
+      for (int c = 0; c < cols_per_warp; c += chunk) {
         float v[32];
         const int acol = half * cols_per_warp + c;             // accumulator column
-        tmem_ld32(tbase + (uint32_t)acol, v);
+        tmem_ld(tbase + (uint32_t)acol, v, chunk);
         if (swiglu) {
           float u[32];
-          tmem_ld32(tbase + (uint32_t)(BN / 2 + acol), u);
+          tmem_ld(tbase + (uint32_t)(BN / 2 + acol), u, chunk);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = act_silu(v[i]) * u[i];
@@ -345,15 +389,34 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
           }
         }
         const int col = ncol0 + c;
+        if (!row_ok) continue;
+        if (p.out_f32) {
+          float* drow = static_cast<float*>(p.d) + (int64_t)plane * p.rows_store * p.ld_d + grow * p.ld_d;
+          const bool vec = (p.ld_d & 3) == 0;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          if (col + 8 * q + 8 <= p.N_out) {
-            int4 o;
-            o.x = (int)pack_bf16(v[8 * q + 0], v[8 * q + 1]);
-            o.y = (int)pack_bf16(v[8 * q + 2], v[8 * q + 3]);
-            o.z = (int)pack_bf16(v[8 * q + 4], v[8 * q + 5]);
-            o.w = (int)pack_bf16(v[8 * q + 6], v[8 * q + 7]);
-            st_v4(drow + (int64_t)(col + 8 * q) * 2, o);
+          for (int q = 0; q < 8; ++q) {
+            if (4 * q >= chunk) continue;
+            const int cc = col + 4 * q;
+            if (vec && cc + 4 <= p.N_out) {
+              *reinterpret_cast<float4*>(drow + cc) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                if (cc + i < p.N_out) drow[cc + i] = v[4 * q + i];
+            }
+          }
+        } else {
+          uint8_t* drow = static_cast<uint8_t*>(p.d) + grow * p.ld_d * 2;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (8 * q < chunk && col + 8 * q + 8 <= p.N_out) {
+              int4 o;
+              o.x = (int)pack_bf16(v[8 * q + 0], v[8 * q + 1]);
+              o.y = (int)pack_bf16(v[8 * q + 2], v[8 * q + 3]);
+              o.z = (int)pack_bf16(v[8 * q + 4], v[8 * q + 5]);
+              o.w = (int)pack_bf16(v[8 * q + 6], v[8 * q + 7]);
+              st_v4(drow + (int64_t)(col + 8 * q) * 2, o);
+            }
           }
         }
       }
@@ -452,13 +515,23 @@ static bool make_map_b(CUtensorMap* m, const void* base, int G, int N, int K, in
   return encode_cached(m, key);
 }
 
+static cudaError_t launch_kernel(KParams& k, int64_t max_tiles, cudaStream_t stream) {
+  cudaError_t e = ensure_smem(grouped_gemm_kernel, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const int sms = sm_count();
+  // grid: one CTA per SM, never more than the largest possible tile count
+  const int grid = (int)(max_tiles < sms ? (max_tiles > 0 ? max_tiles : 1) : sms);
+  grouped_gemm_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(k);
+  return cudaGetLastError();
+}
+
 }  // namespace gg
 
 cudaError_t launch_grouped_gemm(const GemmParams& p, cudaStream_t stream) {
   using namespace gg;
   if (p.rows_max == 0) return cudaSuccess;
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
-  const int box_n = BBOX;
+  const int box_n = 128;
   KParams k{};
   bool ok = make_map_a(&k.tmA, p.a_routed, p.rows_max, p.K);
   ok = ok && make_map_a(&k.tmAs, p.a_shared ? p.a_shared : p.a_routed, p.a_shared ? p.T : p.rows_max, p.K);
@@ -472,20 +545,91 @@ cudaError_t launch_grouped_gemm(const GemmParams& p, cudaStream_t stream) {
   k.status = p.status;
   k.ld_d = p.Nw;
   k.rows_max = p.rows_max;
+  k.rows_static = -1;
+  k.rows_store = p.rows_max;
   k.as_sep = p.a_shared != nullptr;
   k.K = p.K;
   k.N_out = p.Nw;
   k.E = p.E;
   k.n_shared = p.n_shared;
   k.epi = p.epi;
-  cudaError_t e = ensure_smem(grouped_gemm_kernel, SMEM_BYTES);
-  if (e != cudaSuccess) return e;
-  const int sms = sm_count();
-  // grid: one CTA per SM, never more than the largest possible tile count
-  const int64_t max_tiles = (p.rows_max / BM) * ((p.Nw + BBOX - 1) / BBOX);
-  const int grid = (int)(max_tiles < sms ? (max_tiles > 0 ? max_tiles : 1) : sms);
-  grouped_gemm_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(k);
-  return cudaGetLastError();
+  k.bn_fixed = 0;
+  k.bbox = box_n;
+  k.a_kwrap = 0;
+  k.plane_split = 0;
+  k.out_f32 = 0;
+  return launch_kernel(k, (p.rows_max / BM) * ((p.Nw + box_n - 1) / box_n), stream);
+}
+
+// ---------------------------------------------------------------- router logits on tensor cores
+// Wg (fp32) is split into three bf16 planes hi + mid + lo (each the bf16
+// rounding of what the previous planes leave), laid side by side along K with
+// each plane padded to Hp = H rounded up to 64.  x is bf16, so every product
+// x_h * plane_j(w) is exact in fp32 and the tensor core's fp32 accumulation
+// gives fp32 logits of the same quality as an fp32 dot product.
+__global__ void split_router_weight_kernel(const float* wg, __nv_bfloat16* planes, int E, int H, int Hp) {
+  const int64_t n = (int64_t)E * Hp;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int e = (int)(i / Hp), h = (int)(i % Hp);
+    const float w = h < H ? wg[(int64_t)e * H + h] : 0.0f;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+    const float r1 = w - __bfloat162float(hi);
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(mid);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
+    __nv_bfloat16* row = planes + (int64_t)e * 3 * Hp;
+    row[h] = hi;
+    row[Hp + h] = mid;
+    row[2 * Hp + h] = lo;
+  }
+}
+
+int router_plane_width(int H) { return (H + gg::BK - 1) / gg::BK * gg::BK; }
+
+cudaError_t launch_router_gemm(const void* x, const float* wg, void* planes, float* logits, int64_t T, int H, int E,
+                               DevStatus* status, int* parts, cudaStream_t stream) {
+  using namespace gg;
+  if (T == 0) return cudaSuccess;
+  if (encode_fn() == nullptr) return cudaErrorNotSupported;
+  const int Hp = router_plane_width(H);
+  {
+    const int64_t n = (int64_t)E * Hp;
+    const int64_t blocks = (n + 255) / 256;
+    split_router_weight_kernel<<<(unsigned)(blocks < 2048 ? blocks : 2048), 256, 0, stream>>>(
+        wg, static_cast<__nv_bfloat16*>(planes), E, H, Hp);
+  }
+  const int bn = E >= 256 ? 256 : (E + 15) / 16 * 16;
+  const int bbox = bn < 128 ? bn : 128;
+  KParams k{};
+  bool ok = make_map_a(&k.tmA, x, T, H);
+  ok = ok && make_map_b(&k.tmB0, planes, 1, E, 3 * Hp, bbox);
+  if (!ok) return cudaErrorInvalidValue;
+  k.tmAs = k.tmA;
+  k.tmB1 = k.tmSB0 = k.tmSB1 = k.tmB0;
+  k.d = logits;
+  k.off = nullptr;
+  k.status = status;
+  k.ld_d = E;
+  k.rows_max = T;
+  k.rows_static = T;
+  k.rows_store = T;
+  k.K = 3 * Hp;
+  k.N_out = E;
+  k.E = 1;
+  k.n_shared = 0;
+  k.epi = -1;
+  k.as_sep = 0;
+  k.bn_fixed = bn;
+  k.bbox = bbox;
+  k.a_kwrap = Hp / BK;
+  k.out_f32 = 1;
+  // One tile per (m-block, n-tile).  (Giving each weight plane its own tile to
+  // fill more SMs at small T measured slower: three partial arrays to write and
+  // add, and three times the tile start-up cost.)
+  const int64_t tiles = ((T + BM - 1) / BM) * ((E + bn - 1) / bn);
+  k.plane_split = 0;
+  *parts = 1;
+  return launch_kernel(k, tiles * (*parts), stream);
 }
 
 }  // namespace moe

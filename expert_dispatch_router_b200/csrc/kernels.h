@@ -12,6 +12,7 @@ struct RouterParams {
   const float* wg;          // [E,H]
   const float* logit_add;   // [T,E] or null
   const float* logits_in;   // [T,E] or null: skip the GEMM, route these logits
+  int logits_parts;         // logits_in holds this many [T,E] partials to add in order (1 or 3)
   int32_t* ids;             // [T,k]
   float* gates;             // [T,k]
   float* logits_out;        // [T,E] or null
@@ -22,6 +23,13 @@ struct RouterParams {
   int H, E, k, score, renorm;
 };
 int router_tile_tokens(int E);
+// bf16 x: fp32 router logits [T,E] on the tensor cores (Wg split into three bf16
+// planes in `planes`, E * 3 * router_plane_width(H) bf16 of scratch).
+int router_plane_width(int H);
+// `logits` holds 3*T*E floats; *parts (1 or 3) is how many fp32 partial [T,E]
+// arrays were written (their sum, in order, is the logits).
+cudaError_t launch_router_gemm(const void* x, const float* wg, void* planes, float* logits, int64_t T, int H, int E,
+                               DevStatus* status, int* parts, cudaStream_t stream);
 cudaError_t launch_router(const RouterParams& p, bool bf16, cudaStream_t stream);
 // term: E doubles of scratch followed by one unsigned ticket counter.
 cudaError_t launch_aux(const float* psum_part, const int32_t* cnt_part, int nblk, int E, int64_t T, int k,
@@ -43,6 +51,13 @@ struct SlotParams {
   int64_t capacity;         // < 0: dropless
   int64_t rows_max;
   DevStatus* status;
+  // optional aux loss (fused layer path): router partial sums of p, one fp64 term
+  // per expert, and the output scalar
+  const float* psum_part;   // [nblk_router, E] or null
+  int nblk_router;
+  double* aux_term;         // [E]
+  float* aux;
+  float aux_alpha;
 };
 constexpr int kSlotChunk = 256;    // assignments per CTA of the slot kernels (one per thread)
 cudaError_t launch_slots(const SlotParams& p, cudaStream_t stream);

@@ -14,7 +14,8 @@ namespace {
 constexpr int64_t kMaxCf = int64_t(1) << 20;
 
 struct Layout {
-  size_t status, psum, cnt, term, chunk, ids, gates, slot, ecount, kept, off, rowtok, logits, xbuf, hbuf, ybuf;
+  size_t status, psum, cnt, term, chunk, ids, gates, slot, ecount, kept, off, rowtok, logits, lparts, planes, xbuf,
+      hbuf, ybuf;
   size_t total;
   int nblk_router, nchunk;
   int64_t rows_max;
@@ -92,7 +93,10 @@ Layout layout_of(const moe_cfg* c) {
   L.kept = take(sizeof(int32_t) * E);
   L.off = take(sizeof(int32_t) * (E + 2));
   L.rowtok = take(sizeof(int32_t) * (size_t)L.rows_max);
-  L.logits = take((c->flags & MOE_FLAG_KEEP_LOGITS) ? sizeof(float) * T * E : 0);
+  const bool tc_router = c->dtype == MOE_DTYPE_BF16;   // bf16 x: router logits on the tensor cores
+  L.logits = take(((c->flags & MOE_FLAG_KEEP_LOGITS) || tc_router) ? sizeof(float) * T * E : 0);
+  L.lparts = take(tc_router ? sizeof(float) * 3 * T * E : 0);   // router GEMM partials
+  L.planes = take(tc_router ? sizeof(uint16_t) * E * 3 * (size_t)router_plane_width(c->H) : 0);
   L.xbuf = take(esz * (size_t)L.rows_max * c->H);
   L.hbuf = take(esz * (size_t)L.rows_max * c->F);
   L.ybuf = take(esz * (size_t)L.rows_max * c->H);
@@ -124,6 +128,17 @@ RouterParams router_params(const moe_cfg* c, const Layout& L, void* ws) {
 int run_route(const moe_cfg* c, const Layout& L, const void* x, const float* wg, const float* logit_add,
               const float* logits_in, int32_t* ids, float* gates, float* logits_out, void* ws, cudaStream_t s) {
   RouterParams p = router_params(c, L, ws);
+  p.logits_parts = 1;
+  if (logits_in == nullptr && c->dtype == MOE_DTYPE_BF16 && c->T > 0) {
+    // logits on the tensor cores, then the softmax / top-k / gate kernel on them
+    float* buf = at<float>(ws, L.lparts);
+    int parts = 1;
+    if (launch_router_gemm(x, wg, at<void>(ws, L.planes), buf, c->T, c->H, c->E, at<DevStatus>(ws, L.status), &parts,
+                           s) != cudaSuccess)
+      return MOE_ECUDA;
+    logits_in = buf;
+    p.logits_parts = parts;
+  }
   p.x = x;
   p.wg = wg;
   p.logit_add = logit_add;
@@ -135,7 +150,7 @@ int run_route(const moe_cfg* c, const Layout& L, const void* x, const float* wg,
 }
 
 int run_slots(const moe_cfg* c, const Layout& L, const int32_t* ids, int32_t* slot, int32_t* ecount, int32_t* kept,
-              int32_t* off, int32_t* rowtok, void* ws, cudaStream_t s) {
+              int32_t* off, int32_t* rowtok, void* ws, cudaStream_t s, float* aux = nullptr) {
   SlotParams p{};
   p.ids = ids;
   p.slot = slot;
@@ -151,6 +166,13 @@ int run_slots(const moe_cfg* c, const Layout& L, const int32_t* ids, int32_t* sl
   p.capacity = capacity_of(c);
   p.rows_max = L.rows_max;
   p.status = at<DevStatus>(ws, L.status);
+  if (aux != nullptr) {            // fuse the aux loss into the slot kernels
+    p.psum_part = at<float>(ws, L.psum);
+    p.nblk_router = L.nblk_router;
+    p.aux_term = at<double>(ws, L.term);
+    p.aux = aux;
+    p.aux_alpha = c->aux_alpha;
+  }
   return cuda_status(launch_slots(p, s));
 }
 
@@ -410,7 +432,7 @@ int moe_layer_fwd(const moe_cfg* cfg, const void* x, const float* wg, const floa
   if ((st = run_route(cfg, L, x, wg, logit_add, nullptr, ids, gates, logits, ws, s)) != MOE_OK) return st;
   if ((st = record(stage_events, 1, s)) != MOE_OK) return st;
   if ((st = run_slots(cfg, L, ids, slot, at<int32_t>(ws, L.ecount), at<int32_t>(ws, L.kept), off,
-                      at<int32_t>(ws, L.rowtok), ws, s)) != MOE_OK)
+                      at<int32_t>(ws, L.rowtok), ws, s, aux)) != MOE_OK)
     return st;
   if ((st = record(stage_events, 2, s)) != MOE_OK) return st;
   PermuteParams pp = permute_params(cfg, L);
@@ -429,9 +451,6 @@ int moe_layer_fwd(const moe_cfg* cfg, const void* x, const float* wg, const floa
   pp.dst = y;
   if (launch_combine(pp, s) != cudaSuccess) return MOE_ECUDA;
   if ((st = record(stage_events, 6, s)) != MOE_OK) return st;
-  if (launch_aux(at<float>(ws, L.psum), at<int32_t>(ws, L.cnt), L.nblk_router, cfg->E, cfg->T, cfg->k,
-                 cfg->aux_alpha, at<double>(ws, L.term), aux, s) != cudaSuccess)
-    return MOE_ECUDA;
   if (expert_count != nullptr && cfg->E > 0)
     if (cudaMemcpyAsync(expert_count, at<int32_t>(ws, L.ecount), sizeof(int32_t) * cfg->E, cudaMemcpyDeviceToDevice,
                         s) != cudaSuccess)

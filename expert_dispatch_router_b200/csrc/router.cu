@@ -36,9 +36,133 @@ __device__ __forceinline__ int lane_expert(int lane, int j) {
   else return 4 * lane + 128 * (j >> 2) + (j & 3);
 }
 
-// Strict order used for top-k: larger logit first, equal logits -> smaller index.
-__device__ __forceinline__ bool better(float la, int ea, float lb, int eb) {
-  return la > lb || (la == lb && ea < eb);
+// Order-preserving map from fp32 to uint32 (a > b as floats <=> key(a) > key(b)
+// as integers); -0 is mapped like +0 so equal logits get equal keys.  Top-k
+// order: larger logit first, equal logits -> smaller expert index.
+__device__ __forceinline__ uint32_t to_ordered(float v) {
+  const uint32_t b = __float_as_uint(v == 0.0f ? 0.0f : v);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float from_ordered(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Softmax, top-k and gates of token t from its E values spread over the warp's
+// lanes (val[j] belongs to expert lane_expert(lane, j)), adding the logit offset
+// and storing the logits if asked; accumulates this lane's sums of p and
+// selection counts.
+template <int EJ>
+__device__ __forceinline__ void route_token(const RouterParams& p, int64_t t, int lane, const float (&val)[EJ],
+                                            float (&psum)[EJ], int (&cnt)[EJ]) {
+  const int E = p.E;
+    float l[EJ];
+    float m = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < EJ; ++j) {
+      const int e = lane_expert<EJ>(lane, j);
+      float v = val[j];
+      if (e < E) {
+        if (p.logit_add != nullptr) v += p.logit_add[t * E + e];
+        if (p.logits_out != nullptr) p.logits_out[t * E + e] = v;
+        l[j] = v;
+        m = fmaxf(m, v);
+      } else {
+        l[j] = -INFINITY;
+      }
+    }
+    m = from_ordered(__reduce_max_sync(0xffffffffu, to_ordered(m)));
+    float s = 0.0f, ex[EJ];
+#pragma unroll
+    for (int j = 0; j < EJ; ++j) {
+      ex[j] = lane_expert<EJ>(lane, j) < E ? expf(l[j] - m) : 0.0f;
+      s += ex[j];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const float inv_s = 1.0f / s;
+#pragma unroll
+    for (int j = 0; j < EJ; ++j) psum[j] += ex[j] * inv_s;
+
+    // top-k: each round, the warp's best remaining (logit, lower index) key is found
+    // with two 32-bit max reductions: first the order-preserving logit bits, then,
+    // among lanes holding that logit, the complemented expert index.
+    unsigned selected = 0u;
+    float my_l = -INFINITY;
+    int my_e = -1;
+    uint32_t bh = 0u, bl = 0u;      // this lane's best unselected candidate
+    int bj = -1;
+    auto lane_best = [&]() {
+      bh = 0u; bl = 0u; bj = -1;
+#pragma unroll
+      for (int j = 0; j < EJ; ++j) {
+        const int e = lane_expert<EJ>(lane, j);
+        if (e < E && !((selected >> j) & 1u)) {
+          const uint32_t h = to_ordered(l[j]), lo = 0xffffffffu - (uint32_t)e;
+          if (h > bh || (h == bh && lo > bl)) { bh = h; bl = lo; bj = j; }
+        }
+      }
+    };
+    lane_best();
+#pragma unroll 1
+    for (int r = 0; r < p.k; ++r) {
+      const uint32_t wh = __reduce_max_sync(0xffffffffu, bh);
+      const uint32_t wl = __reduce_max_sync(0xffffffffu, bh == wh ? bl : 0u);
+      if (lane == r) { my_l = from_ordered(wh); my_e = (int)(0xffffffffu - wl); }
+      if (bj >= 0 && bh == wh && bl == wl) {      // this lane owned the winner
+        selected |= 1u << bj;
+#pragma unroll
+        for (int j = 0; j < EJ; ++j)
+          if (j == bj) cnt[j] += 1;
+        lane_best();
+      }
+    }
+    // gates: lane r holds the rank-r selection
+    float g = 0.0f;
+    if (lane < p.k) g = expf(my_l - m);        // top-1 logit equals m
+    if (p.score == MOE_SCORE_SOFTMAX_TOPK) {
+      g *= inv_s;
+      if (p.renorm) {
+        float gs = g;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) gs += __shfl_xor_sync(0xffffffffu, gs, o);
+        g = g / gs;
+      }
+    } else {
+      float gs = g;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) gs += __shfl_xor_sync(0xffffffffu, gs, o);
+      g = g / gs;
+    }
+    if (lane < p.k) {
+      p.ids[t * p.k + lane] = my_e;
+      p.gates[t * p.k + lane] = g;
+    }
+}
+
+// Sums the warps' per-expert partials in a fixed order and stores this CTA's row
+// of psum_part / cnt_part.  `smem` must hold 2 * WARPS * 32 * EJ words.
+template <int EJ, int WARPS>
+__device__ __forceinline__ void write_partials(const RouterParams& p, float* smem, const float (&psum)[EJ],
+                                               const int (&cnt)[EJ]) {
+  constexpr int EP = 32 * EJ;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  float* rp = smem;                                     // [WARPS][EP]
+  int* rc = reinterpret_cast<int*>(smem + WARPS * EP);
+#pragma unroll
+  for (int j = 0; j < EJ; ++j) {
+    const int e = lane_expert<EJ>(lane, j);
+    rp[warp * EP + e] = psum[j];
+    rc[warp * EP + e] = cnt[j];
+  }
+  __syncthreads();
+  for (int e = tid; e < p.E; e += WARPS * 32) {
+    float ps = 0.0f;
+    int cs = 0;
+#pragma unroll
+    for (int w = 0; w < WARPS; ++w) { ps += rp[w * EP + e]; cs += rc[w * EP + e]; }
+    p.psum_part[(int64_t)blockIdx.x * p.E + e] = ps;
+    p.cnt_part[(int64_t)blockIdx.x * p.E + e] = cs;
+  }
 }
 
 template <int EJ, int TW>
@@ -69,7 +193,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterParams p) 
 #pragma unroll
     for (int j = 0; j < EJ; ++j) acc[i][j] = 0.0f;
 
-  if (p.logits_in == nullptr) {
+  {
     constexpr int XV = 16 / sizeof(XT);              // elements per 16-byte vector
     constexpr int XVEC = BT * kKC / XV;              // x vectors per chunk
     constexpr int XM = (XVEC + kRouterThreads - 1) / kRouterThreads;
@@ -156,16 +280,6 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterParams p) 
         }
       }
     }
-  } else {
-#pragma unroll
-    for (int i = 0; i < TW; ++i) {
-      const int64_t t = t0 + warp * TW + i;
-#pragma unroll
-      for (int j = 0; j < EJ; ++j) {
-        const int e = lane_expert<EJ>(lane, j);
-        if (t < p.T && e < E) acc[i][j] = p.logits_in[t * E + e];
-      }
-    }
   }
 
   // ---------------- epilogue: softmax, top-k, gates, partial sums
@@ -173,105 +287,51 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterParams p) 
   int cnt[EJ];
 #pragma unroll
   for (int j = 0; j < EJ; ++j) { psum[j] = 0.0f; cnt[j] = 0; }
-
 #pragma unroll
   for (int i = 0; i < TW; ++i) {
     const int64_t t = t0 + warp * TW + i;
-    if (t >= p.T) continue;                    // uniform across the warp
-    float l[EJ];
-    float m = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < EJ; ++j) {
-      const int e = lane_expert<EJ>(lane, j);
-      float v = acc[i][j];
-      if (e < E) {
-        if (p.logits_in == nullptr && p.logit_add != nullptr) v += p.logit_add[t * E + e];
-        if (p.logits_out != nullptr) p.logits_out[t * E + e] = v;
-        l[j] = v;
-        m = fmaxf(m, v);
-      } else {
-        l[j] = -INFINITY;
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float s = 0.0f, ex[EJ];
-#pragma unroll
-    for (int j = 0; j < EJ; ++j) {
-      ex[j] = lane_expert<EJ>(lane, j) < E ? expf(l[j] - m) : 0.0f;
-      s += ex[j];
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    const float inv_s = 1.0f / s;
-#pragma unroll
-    for (int j = 0; j < EJ; ++j) psum[j] += ex[j] * inv_s;
-
-    unsigned selected = 0u;
-    float my_l = -INFINITY;
-    int my_e = -1;
-#pragma unroll 1
-    for (int r = 0; r < p.k; ++r) {
-      float bl = -INFINITY;
-      int be = 0x7fffffff;
-#pragma unroll
-      for (int j = 0; j < EJ; ++j) {
-        const int e = lane_expert<EJ>(lane, j);
-        if (e < E && !((selected >> j) & 1u) && better(l[j], e, bl, be)) { bl = l[j]; be = e; }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ol = __shfl_xor_sync(0xffffffffu, bl, o);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-        if (better(ol, oe, bl, be)) { bl = ol; be = oe; }
-      }
-#pragma unroll
-      for (int j = 0; j < EJ; ++j)
-        if (lane_expert<EJ>(lane, j) == be) { selected |= 1u << j; cnt[j] += 1; }
-      if (lane == r) { my_l = bl; my_e = be; }
-    }
-    // gates: lane r holds the rank-r selection
-    float g = 0.0f;
-    if (lane < p.k) g = expf(my_l - m);        // top-1 logit equals m
-    if (p.score == MOE_SCORE_SOFTMAX_TOPK) {
-      g *= inv_s;
-      if (p.renorm) {
-        float gs = g;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) gs += __shfl_xor_sync(0xffffffffu, gs, o);
-        g = g / gs;
-      }
-    } else {
-      float gs = g;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) gs += __shfl_xor_sync(0xffffffffu, gs, o);
-      g = g / gs;
-    }
-    if (lane < p.k) {
-      p.ids[t * p.k + lane] = my_e;
-      p.gates[t * p.k + lane] = g;
-    }
+    if (t < p.T) route_token<EJ>(p, t, lane, acc[i], psum, cnt);
   }
 
   // ---------------- fixed-order reduction of the per-warp partials
   __syncthreads();
-  float* rp = smem;                                     // [warps][EP]
-  int* rc = reinterpret_cast<int*>(smem + kRouterWarps * EP);
+  write_partials<EJ, kRouterWarps>(p, smem, psum, cnt);
+}
+
+// Routing from given fp32 logits (the tensor-core router's output, or the
+// caller's for moe_route_from_logits): 8 warps, the same BT tokens per CTA as
+// the FFMA router so the partial-sum rows line up; a warp routes one token at a
+// time with nothing but that token's logits in registers.
+constexpr int kLogitWarps = 8;
+
+template <int EJ>
+__global__ void __launch_bounds__(kLogitWarps * 32) route_logits_kernel(RouterParams p, int bt) {
+  extern __shared__ __align__(16) float smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t t0 = (int64_t)blockIdx.x * bt;
+  if (blockIdx.x == 0 && tid == 0 && p.aux_counter != nullptr) *p.aux_counter = 0u;
+  float psum[EJ];
+  int cnt[EJ];
 #pragma unroll
-  for (int j = 0; j < EJ; ++j) {
-    const int e = lane_expert<EJ>(lane, j);
-    rp[warp * EP + e] = psum[j];
-    rc[warp * EP + e] = cnt[j];
+  for (int j = 0; j < EJ; ++j) { psum[j] = 0.0f; cnt[j] = 0; }
+  for (int i = warp; i < bt; i += kLogitWarps) {
+    const int64_t t = t0 + i;
+    if (t >= p.T) break;
+    float val[EJ];
+#pragma unroll
+    for (int j = 0; j < EJ; ++j) {
+      const int e = lane_expert<EJ>(lane, j);
+      float v = 0.0f;
+      if (e < p.E) {
+        v = p.logits_in[t * p.E + e];
+        for (int q = 1; q < p.logits_parts; ++q) v += p.logits_in[(int64_t)q * p.T * p.E + t * p.E + e];
+      }
+      val[j] = v;
+    }
+    route_token<EJ>(p, t, lane, val, psum, cnt);
   }
   __syncthreads();
-  for (int e = tid; e < E; e += kRouterThreads) {
-    float ps = 0.0f;
-    int cs = 0;
-#pragma unroll
-    for (int w = 0; w < kRouterWarps; ++w) { ps += rp[w * EP + e]; cs += rc[w * EP + e]; }
-    p.psum_part[(int64_t)blockIdx.x * E + e] = ps;
-    p.cnt_part[(int64_t)blockIdx.x * E + e] = cs;
-  }
+  write_partials<EJ, kLogitWarps>(p, smem, psum, cnt);
 }
 
 // Tokens per CTA of the router for E experts (the host needs it to size the
@@ -301,9 +361,29 @@ static cudaError_t launch_router_ej(const RouterParams& p, bool bf16, cudaStream
   return cudaGetLastError();
 }
 
+template <int EJ>
+static cudaError_t launch_route_logits_ej(const RouterParams& p, cudaStream_t stream) {
+  const int bt = router_tile_tokens(p.E);
+  const size_t smem = sizeof(float) * 2 * kLogitWarps * 32 * EJ;
+  const unsigned grid = (unsigned)((p.T + bt - 1) / bt);
+  auto k = route_logits_kernel<EJ>;
+  cudaError_t e = ensure_smem(k, smem);
+  if (e != cudaSuccess) return e;
+  k<<<grid, kLogitWarps * 32, smem, stream>>>(p, bt);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_router(const RouterParams& p, bool bf16, cudaStream_t stream) {
   if (p.T == 0) return cudaSuccess;
   const int E = p.E;
+  if (p.logits_in != nullptr) {
+    if (E <= 32) return launch_route_logits_ej<1>(p, stream);
+    if (E <= 64) return launch_route_logits_ej<2>(p, stream);
+    if (E <= 128) return launch_route_logits_ej<4>(p, stream);
+    if (E <= 256) return launch_route_logits_ej<8>(p, stream);
+    if (E <= 512) return launch_route_logits_ej<16>(p, stream);
+    return launch_route_logits_ej<32>(p, stream);
+  }
   if (E <= 32) return launch_router_ej<1, 8>(p, bf16, stream);
   if (E <= 64) return launch_router_ej<2, 8>(p, bf16, stream);
   if (E <= 128) return launch_router_ej<4, 8>(p, bf16, stream);

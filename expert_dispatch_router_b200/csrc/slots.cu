@@ -96,6 +96,21 @@ __global__ void __launch_bounds__(kSlotThreads) slot_scan_kernel(SlotParams p, i
     const int kept = p.capacity < 0 ? running : (int)min((int64_t)running, p.capacity);
     p.kept_count[e] = kept;
   }
+  if (p.psum_part != nullptr) {
+    // this expert's aux-loss term f_e * P_e: f from the pre-drop count, P from the
+    // router's per-CTA sums of p (fp64, fixed block-then-tree order)
+    __shared__ double red[kSlotThreads];
+    double ps = 0.0;
+    for (int b = threadIdx.x; b < p.nblk_router; b += kSlotThreads) ps += (double)p.psum_part[(int64_t)b * p.E + e];
+    red[threadIdx.x] = ps;
+    __syncthreads();
+    for (int s = kSlotThreads / 2; s > 0; s >>= 1) {
+      if ((int)threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
+      __syncthreads();
+    }
+    if (threadIdx.x == 0)
+      p.aux_term[e] = ((double)running / ((double)p.T * p.k)) * (red[0] / (double)p.T);
+  }
 }
 
 __global__ void __launch_bounds__(1024) slot_offsets_kernel(SlotParams p) {
@@ -133,6 +148,17 @@ __global__ void __launch_bounds__(1024) slot_offsets_kernel(SlotParams p) {
   }
   __syncthreads();
   for (int i = tid; i < p.E + 2; i += 1024) p.expert_offset[i] = sh_off[i];
+  if (p.aux != nullptr) {
+    // aux loss = alpha * E * sum_e term[e], summed by a fixed tree
+    __shared__ double red[1024];
+    red[tid] = (p.T > 0 && tid < p.E) ? p.aux_term[tid] : 0.0;
+    __syncthreads();
+    for (int s = 512; s > 0; s >>= 1) {
+      if (tid < s) red[tid] += red[tid + s];
+      __syncthreads();
+    }
+    if (tid == 0) *p.aux = (float)((double)p.aux_alpha * (double)p.E * red[0]);
+  }
   // padding rows of each routed block -> -1
   for (int e = warp; e < p.E; e += 32) {
     const int start = sh_off[e] + p.kept_count[e], stop = sh_off[e + 1];

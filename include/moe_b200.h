@@ -242,9 +242,10 @@ MOE_API int moe_aux_loss(const moe_cfg* cfg, const void* ws, float* aux, moe_str
  * device outputs; expert_count [E] is optional (NULL to skip).  The
  * intermediates stay in `ws` (see moe_workspace_views).  `stage_events`, if
  * non-NULL, is an array of MOE_N_STAGE_EVENTS events recorded on `stream` before
- * the router and after each of: router, slots, dispatch, expert FFN first
- * contraction (with the activation), expert FFN second contraction, combine,
- * aux loss. */
+ * the router and after each of: router, slots (which here also reduce the aux
+ * loss), dispatch, expert FFN first contraction (with the activation), expert
+ * FFN second contraction, combine, and the end of the call (the copy of
+ * expert_count, if requested). */
 enum { MOE_N_STAGE_EVENTS = 8 };
 MOE_API int moe_layer_fwd(const moe_cfg* cfg, const void* x, const float* wg, const float* logit_add,
                   const moe_weights* w, void* y, float* aux, int32_t* expert_count, void* ws,
