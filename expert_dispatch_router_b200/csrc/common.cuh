@@ -58,6 +58,12 @@ __device__ __forceinline__ float rcp_approx(float x) {
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
   return r;
 }
+// 2^x on the special-function unit (PTX ex2.approx, about 2 ulp).
+__device__ __forceinline__ float exp2f_approx(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
 
 // erf from Abramowitz & Stegun, Handbook of Mathematical Functions (1964),
 // formula 7.1.26: erf(x) = 1 - (a1 t + ... + a5 t^5) exp(-x^2), t = 1/(1 + p x),
@@ -74,8 +80,22 @@ __device__ __forceinline__ float erf_as7126(float x) {
   const float r = 1.0f - poly * __expf(-ax * ax);
   return copysignf(r, x);
 }
-// Exact-form GELU: 0.5 z (1 + erf(z / sqrt 2)).
-__device__ __forceinline__ float act_gelu(float z) { return 0.5f * z * (1.0f + erf_as7126(z * 0.70710678118654752f)); }
+// Exact-form GELU, 0.5 z (1 + erf(z / sqrt 2)), evaluated through erfc: formula
+// 7.1.26 is erfc(x) = P(t) exp(-x^2) for x >= 0, so with x = |z| / sqrt 2,
+//   z <  0:  0.5 z (1 + erf(z/sqrt 2)) = 0.5 z erfc(x)
+//   z >= 0:  0.5 z (1 + erf(z/sqrt 2)) = z - 0.5 z erfc(x).
+// Constants are pre-scaled: p/sqrt 2 in t, 0.5 a_i in the polynomial, and
+// exp(-z^2/2) = 2^(-z^2 log2(e) / 2).  Same error bound as erf_as7126.
+__device__ __forceinline__ float act_gelu(float z) {
+  const float t = rcp_approx(fmaf(0.23164189f, fabsf(z), 1.0f));           // 0.3275911 / sqrt 2
+  float q = fmaf(0.5307027145f, t, -0.7265760135f);                        // 0.5 * a5, 0.5 * a4
+  q = fmaf(q, t, 0.7107068705f);                                            // 0.5 * a3
+  q = fmaf(q, t, -0.142248368f);                                            // 0.5 * a2
+  q = fmaf(q, t, 0.127414796f);                                             // 0.5 * a1
+  const float e = exp2f_approx(z * z * -0.72134752044448170f);             // exp(-z^2 / 2)
+  const float h = z * (q * t) * e;                                          // 0.5 z erfc(|z| / sqrt 2)
+  return z >= 0.0f ? z - h : h;
+}
 // SiLU: z * sigmoid(z) = z / (1 + exp(-z)).
 __device__ __forceinline__ float act_silu(float z) { return z * rcp_approx(1.0f + __expf(-z)); }
 

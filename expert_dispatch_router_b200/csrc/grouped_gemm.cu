@@ -18,14 +18,14 @@
 //   router: A = x (its k coordinate wraps every H' columns), B = the three bf16
 //          planes of Wg laid side by side along K, fp32 out.
 //
-// Kernel structure (one persistent CTA per SM, 320 threads):
+// Kernel structure (one persistent CTA per SM, 576 threads):
 //   warp 0      TMA producer: A box 64x128 and B boxes 64 x (<=128) per stage,
 //               128-byte swizzle, a 4-8 stage ring guarded by full/empty mbarriers.
 //   warp 1      allocates 512 TMEM columns and issues tcgen05.mma
 //               (M=128, N<=256, K=16, kind::f16) from one lane; commits free the
 //               smem stage and, per tile, signal the accumulator as full.
-//   warps 2-9   epilogue: tcgen05.ld of the fp32 accumulator (each warp owns
-//               one 32-lane TMEM sub-partition and half the columns), the
+//   warps 2-17  epilogue: tcgen05.ld of the fp32 accumulator (four warps per
+//               32-lane TMEM sub-partition, interleaving column chunks), the
 //               activation, packing and 16-byte global stores.
 // Two accumulators of 256 columns let the epilogue of one tile overlap the
 // main loop of the next.  Tiles are walked m-block-major, n fastest, so CTAs
@@ -50,13 +50,16 @@ constexpr int BM = 128, BN = 256, BK = 64;
 constexpr int A_BYTES = BM * BK * 2;              // 16 KB
 constexpr int RING_BYTES = 4 * (A_BYTES + BN * BK * 2);   // 192 KB: 4 stages at N=256, more when narrower
 constexpr int MAX_STAGES = 8;
-constexpr int EPI_WARPS = 8;
+constexpr int EPI_WARPS = 16;                      // 4 per TMEM sub-partition
 constexpr int THREADS = 64 + EPI_WARPS * 32;
 constexpr int TMEM_COLS = 512;
-constexpr int SMEM_BYTES = RING_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int STAGE_OUT_BYTES = 32 * 32 * 2;       // one warp's 32 x 32 bf16 output sub-tile
+constexpr int STAGING_BYTES = EPI_WARPS * STAGE_OUT_BYTES;   // 32 KB
+constexpr int SMEM_BYTES = RING_BYTES + STAGING_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 
 struct KParams {
   CUtensorMap tmA, tmAs, tmB0, tmB1, tmSB0, tmSB1;
+  CUtensorMap tmD;       // bf16 output [rows, N_out], box 32 x 32, 64-byte swizzle (TMA store)
   void* d;
   const int32_t* off;
   DevStatus* status;
@@ -112,6 +115,18 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
   asm volatile("cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
                :: "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar) : "memory");
 }
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];"
+               :: "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(src) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" :: "r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
 __device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -196,7 +211,8 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + RING_BYTES);
+  uint8_t* staging = smem + RING_BYTES;                 // per epilogue warp: 32 x 32 bf16, swizzled
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + RING_BYTES + STAGING_BYTES);
   // bars: full[MAX_STAGES], empty[MAX_STAGES], tfull[2], tempty[2], drain
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + MAX_STAGES);
   const uint32_t tfull0 = smem_u32(bars + 2 * MAX_STAGES), tempty0 = smem_u32(bars + 2 * MAX_STAGES + 2);
@@ -348,10 +364,10 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
     // ---------------- epilogue
     const int ew = warp - 2;
     const int sub = warp & 3;                  // TMEM sub-partition this warp may access
-    const int half = ew >> 2;                  // which half of the output columns
+    const int quarter = ew >> 2;               // the four warps of a sub-partition split the chunks
     const int row_in_tile = sub * 32 + lane;
-    const int cols_per_warp = n_step / 2;      // 128, 64, or bn/2 for a fixed N
-    const int chunk = cols_per_warp >= 32 ? 32 : cols_per_warp >= 16 ? 16 : 8;
+    const int chunk = n_step >= 128 ? 32 : n_step >= 64 ? 16 : 8;   // columns per tcgen05.ld
+    const uint32_t stage_out = smem_u32(staging + ew * STAGE_OUT_BYTES);
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
@@ -366,11 +382,11 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       const int nt = (int)(tile / n_planes % n_tiles_n);
       const int64_t grow = mt * BM + row_in_tile;
       const bool row_ok = grow < p.rows_store;
-      const int ncol0 = nt * n_step + half * cols_per_warp;    // first output column of this warp
+      const int ncol0 = nt * n_step;                           // first output column of the tile
       const uint32_t tbase = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * BN);
-      for (int c = 0; c < cols_per_warp; c += chunk) {
+      for (int c = quarter * chunk; c < n_step; c += 4 * chunk) {
         float v[32];
-        const int acol = half * cols_per_warp + c;             // accumulator column
+        const int acol = c;                                     // accumulator column
         tmem_ld(tbase + (uint32_t)acol, v, chunk);
         if (swiglu) {
           float u[32];
@@ -389,8 +405,8 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
           }
         }
         const int col = ncol0 + c;
-        if (!row_ok) continue;
         if (p.out_f32) {
+          if (!row_ok) continue;
           float* drow = static_cast<float*>(p.d) + (int64_t)plane * p.rows_store * p.ld_d + grow * p.ld_d;
           const bool vec = (p.ld_d & 3) == 0;
 #pragma unroll
@@ -406,17 +422,21 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
             }
           }
         } else {
-          uint8_t* drow = static_cast<uint8_t*>(p.d) + grow * p.ld_d * 2;
+          // bf16: this warp's 32 rows x 32 columns go through its staging buffer
+          // (16-byte chunk j of row r at chunk j ^ ((r >> 1) & 3): the TMA 64-byte
+          // swizzle, bank-conflict free) and out with one TMA store of full lines.
+          if (lane == 0) bulk_wait_read0();          // the previous store has read the buffer
+          __syncwarp();
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            if (8 * q < chunk && col + 8 * q + 8 <= p.N_out) {
-              int4 o;
-              o.x = (int)pack_bf16(v[8 * q + 0], v[8 * q + 1]);
-              o.y = (int)pack_bf16(v[8 * q + 2], v[8 * q + 3]);
-              o.z = (int)pack_bf16(v[8 * q + 4], v[8 * q + 5]);
-              o.w = (int)pack_bf16(v[8 * q + 6], v[8 * q + 7]);
-              st_v4(drow + (int64_t)(col + 8 * q) * 2, o);
-            }
+          for (int q = 0; q < 4; ++q)
+            st_shared_v4(stage_out + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4),
+                         pack_bf16(v[8 * q + 0], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
+                         pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7]));
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&p.tmD, stage_out, col, (int)(mt * BM + sub * 32));
+            bulk_commit();
           }
         }
       }
@@ -424,6 +444,8 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       mbar_arrive(tempty0 + 8 * acc);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
+    if (lane == 0) bulk_wait0();                 // this warp's output stores are complete
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -456,6 +478,7 @@ static EncodeTiledFn encode_fn() {
 struct MapKey {
   const void* base;
   uint32_t rank;
+  uint32_t swizzle;      // CUtensorMapSwizzle
   cuuint64_t dims[3];
   cuuint64_t strides[2];
   cuuint32_t box[3];
@@ -474,7 +497,7 @@ static bool encode_cached(CUtensorMap* out, const MapKey& key) {
   cuuint32_t es[3] = {1, 1, 1};
   CUtensorMap m;
   if (encode_fn()(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, key.rank, const_cast<void*>(key.base), key.dims, key.strides,
-                  key.box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  key.box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, (CUtensorMapSwizzle)key.swizzle,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return false;
   const int slot = used < kSlots ? used++ : (next++ % kSlots);
@@ -490,6 +513,7 @@ static bool make_map_a(CUtensorMap* m, const void* base, int64_t rows, int K) {
   memset(&key, 0, sizeof(key));
   key.base = base;
   key.rank = 2;
+  key.swizzle = CU_TENSOR_MAP_SWIZZLE_128B;
   key.dims[0] = (cuuint64_t)K;
   key.dims[1] = (cuuint64_t)rows;
   key.strides[0] = (cuuint64_t)K * 2;
@@ -504,6 +528,7 @@ static bool make_map_b(CUtensorMap* m, const void* base, int G, int N, int K, in
   memset(&key, 0, sizeof(key));
   key.base = base;
   key.rank = 3;
+  key.swizzle = CU_TENSOR_MAP_SWIZZLE_128B;
   key.dims[0] = (cuuint64_t)K;
   key.dims[1] = (cuuint64_t)N;
   key.dims[2] = (cuuint64_t)G;
@@ -512,6 +537,21 @@ static bool make_map_b(CUtensorMap* m, const void* base, int G, int N, int K, in
   key.box[0] = BK;
   key.box[1] = (cuuint32_t)box_n;
   key.box[2] = 1;
+  return encode_cached(m, key);
+}
+
+// 2-D map over the bf16 output [rows, N], box 32 x 32, 64-byte swizzle (TMA store).
+static bool make_map_d(CUtensorMap* m, const void* base, int64_t rows, int N) {
+  MapKey key;
+  memset(&key, 0, sizeof(key));
+  key.base = base;
+  key.rank = 2;
+  key.swizzle = CU_TENSOR_MAP_SWIZZLE_64B;
+  key.dims[0] = (cuuint64_t)N;
+  key.dims[1] = (cuuint64_t)rows;
+  key.strides[0] = (cuuint64_t)N * 2;
+  key.box[0] = 32;
+  key.box[1] = 32;
   return encode_cached(m, key);
 }
 
@@ -539,6 +579,7 @@ cudaError_t launch_grouped_gemm(const GemmParams& p, cudaStream_t stream) {
   ok = ok && make_map_b(&k.tmB1, p.b1 ? p.b1 : p.b0, p.E, p.Nw, p.K, box_n);
   ok = ok && make_map_b(&k.tmSB0, p.sb0 ? p.sb0 : p.b0, 1, p.Nw, p.K, box_n);
   ok = ok && make_map_b(&k.tmSB1, p.sb1 ? p.sb1 : (p.sb0 ? p.sb0 : p.b0), 1, p.Nw, p.K, box_n);
+  ok = ok && make_map_d(&k.tmD, p.d, p.rows_max, p.Nw);
   if (!ok) return cudaErrorInvalidValue;
   k.d = p.d;
   k.off = p.expert_offset;
@@ -606,6 +647,7 @@ cudaError_t launch_router_gemm(const void* x, const float* wg, void* planes, flo
   if (!ok) return cudaErrorInvalidValue;
   k.tmAs = k.tmA;
   k.tmB1 = k.tmSB0 = k.tmSB1 = k.tmB0;
+  k.tmD = k.tmA;                                   // unused: fp32 output is stored directly
   k.d = logits;
   k.off = nullptr;
   k.status = status;
