@@ -40,6 +40,18 @@ notes):
   * gates are fixed before capacity; a dropped choice contributes zero and the
     kept gates are not renormalised again.
   * f_i counts pre-drop selections over T*k; P_i is the mean full softmax.
+  * sigmoid scores ([EP] router section names sigmoid as the alternative to
+    softmax and says nothing more): top-k on the logits as for softmax (the
+    sigmoid is monotone), gate = sigmoid(logit), optionally renormalised over
+    the k selected; for the aux loss P_i averages the sigmoids divided by their
+    sum over the E experts, so that equal logits still give aux = alpha.
+  * z-loss ([EP] aux-loss section, z_loss_func): coef * mean_t lse(logits_t)^2
+    on the float32 logits, reported beside the aux loss rather than added to it.
+  * GShard random second expert ([EP] router section: sent at random according
+    to its weight): the rank-1 choice is dispatched iff u_t < 2 g_t1, GShard's
+    own rule (with top-2 renormalised gates 2 g_t1 <= 1), u_t ~ U[0, 1) an
+    input.  A choice that is not dispatched keeps its place in f_i (selected),
+    takes no slot and adds nothing to y; g_t0 is not changed.
   * the layer returns the MoE branch only (y = 0 for a fully dropped token); the
     caller adds the residual.
   * GELU is the exact erf form; SwiGLU is silu(x W_gate) * (x W_up) then W_down.
@@ -57,7 +69,7 @@ from typing import Optional
 import numpy as np
 
 ACT_RELU, ACT_GELU, ACT_SWIGLU = 0, 1, 2
-SCORE_SOFTMAX_TOPK, SCORE_TOPK_SOFTMAX = 0, 1
+SCORE_SOFTMAX_TOPK, SCORE_TOPK_SOFTMAX, SCORE_SIGMOID_TOPK = 0, 1, 2
 CAP_CAPACITY, CAP_DROPLESS = 0, 1
 ROW_PAD = 128
 
@@ -79,6 +91,8 @@ class OracleLayer:
     min_capacity: int = 0
     n_shared: int = 0
     aux_alpha: float = 1e-2
+    z_coef: float = 0.0          # router z-loss coefficient, 0 = off
+    random_second: int = 0       # GShard: dispatch the second choice at random
 
     @classmethod
     def from_mapping(cls, m) -> "OracleLayer":
@@ -142,19 +156,65 @@ def topk_ids(logits: np.ndarray, k: int) -> np.ndarray:
     return order[:, :k].astype(np.int32)
 
 
+def sigmoid(logits: np.ndarray) -> np.ndarray:
+    """sigma(l) = 1 / (1 + exp(-l)), float64 ([EP] router section: softmax or sigmoid)."""
+    return 1.0 / (1.0 + np.exp(-np.asarray(logits, dtype=np.float64)))
+
+
+def router_probs(logits: np.ndarray, score: int) -> np.ndarray:
+    """The per-expert probabilities P_i averages ([EP] aux-loss section).  Softmax
+    for the softmax scores; for sigmoid scores the sigmoids normalised over the
+    experts (so that they sum to one per token and uniform routing still gives
+    aux = alpha)."""
+    if score == SCORE_SIGMOID_TOPK:
+        s = sigmoid(logits)
+        return s / s.sum(axis=-1, keepdims=True)
+    return softmax(logits)
+
+
 def gate_values(logits: np.ndarray, probs: np.ndarray, ids: np.ndarray, score: int, renorm: int) -> np.ndarray:
     """Gate of each selected expert.
     SOFTMAX_TOPK: g = p[e] (Switch: y = p_i(x) E_i(x)), optionally divided by the
     sum over the k selected.  TOPK_SOFTMAX ([EP] router section, Megatron
-    pre_softmax=False): softmax taken over the k selected logits only."""
+    pre_softmax=False): softmax taken over the k selected logits only.
+    SIGMOID_TOPK ([EP] router section, sigmoid scores): g = sigmoid(l[e]),
+    optionally divided by the sum over the k selected."""
     t = np.arange(ids.shape[0])[:, None]
+    sel = np.asarray(logits, dtype=np.float64)[t, ids]
     if score == SCORE_SOFTMAX_TOPK:
         g = probs[t, ids]
-        if renorm:
-            g = g / g.sum(axis=1, keepdims=True)
-        return g
-    sel = np.asarray(logits, dtype=np.float64)[t, ids]
-    return softmax(sel)
+    elif score == SCORE_SIGMOID_TOPK:
+        g = sigmoid(sel)
+    else:
+        return softmax(sel)
+    if renorm:
+        g = g / g.sum(axis=1, keepdims=True)
+    return g
+
+
+def random_second_dispatch(ids: np.ndarray, gates: np.ndarray, uniform: np.ndarray):
+    """GShard top-2 ([EP] router section: the second expert receives the token at
+    random, in proportion to its weight): the rank-1 choice of token t is
+    dispatched iff u_t < 2 g_t1 (g renormalised over the two, so 2 g_t1 <= 1);
+    otherwise its id becomes -1 (not dispatched) and its gate 0.  The uniforms
+    u_t in [0,1) are an input."""
+    ids = ids.copy()
+    gates = gates.copy()
+    u = np.asarray(uniform, dtype=np.float64)
+    for t in range(ids.shape[0]):
+        if not (u[t] < 2.0 * gates[t, 1]):
+            ids[t, 1] = -1
+            gates[t, 1] = 0.0
+    return ids, gates
+
+
+def z_loss(logits: np.ndarray, coef: float) -> float:
+    """Router z-loss ([EP] aux-loss section, z_loss_func): coef * mean over tokens
+    of logsumexp(logits_t)^2."""
+    l = np.asarray(logits, dtype=np.float64)
+    m = l.max(axis=-1)
+    lse = m + np.log(np.exp(l - m[:, None]).sum(axis=-1))
+    return float(coef * np.mean(lse ** 2)) if l.shape[0] else 0.0
 
 
 # ---------------------------------------------------------------- slots
@@ -162,14 +222,18 @@ def assign_slots(ids: np.ndarray, E: int, C: Optional[int]):
     """Literal walk of the 'position' drop policy ([EP] drop/pad section):
     assignments are visited choice rank first, then token order; each takes the
     next free position of its expert and is kept iff that position < C
-    (C=None: dropless, always kept).  Returns (slot[T,k] with -1 = dropped,
-    count[E] pre-drop selections, kept[E])."""
+    (C=None: dropless, always kept).  An id of -1 is a choice that is not
+    dispatched (GShard random second expert): it takes no position.  Returns
+    (slot[T,k] with -1 = dropped or not dispatched, count[E] assignments per
+    expert before the capacity drop, kept[E])."""
     T, k = ids.shape
     fill = [0] * E
     slot = np.full((T, k), -1, dtype=np.int32)
     for r in range(k):
         for t in range(T):
             e = int(ids[t, r])
+            if e < 0:
+                continue
             pos = fill[e]
             fill[e] += 1
             if C is None or pos < C:
@@ -244,7 +308,8 @@ def expert_ffn(X: np.ndarray, w1: np.ndarray, w2: np.ndarray, act: int,
 def aux_loss(probs: np.ndarray, ids: np.ndarray, E: int, alpha: float) -> float:
     """Switch load-balancing loss alpha * N * sum_i f_i P_i ([SWITCH] 2.1, [EP]
     aux-loss section): f_i = selections of expert i / (T*k) (top-k in the
-    denominator, pre-drop), P_i = mean over tokens of the full softmax p_i."""
+    denominator, pre-drop), P_i = mean over tokens of the router probabilities
+    p_i (softmax, or the normalised sigmoids of router_probs)."""
     T, k = ids.shape
     f = np.bincount(ids.reshape(-1), minlength=E).astype(np.float64) / (T * k)
     P = np.asarray(probs, dtype=np.float64).mean(axis=0)
@@ -253,11 +318,22 @@ def aux_loss(probs: np.ndarray, ids: np.ndarray, E: int, alpha: float) -> float:
 
 # ---------------------------------------------------------------- layer
 def route(layer: OracleLayer, logits: np.ndarray):
-    """Router steps after the logits: softmax, top-k, gates."""
-    probs = softmax(logits)
+    """Router steps after the logits: scores, top-k, gates."""
+    probs = router_probs(logits, layer.score)
     ids = topk_ids(logits, layer.k)
     gates = gate_values(logits, probs, ids, layer.score, layer.renorm)
     return probs, ids, gates
+
+
+def route_and_dispatch(layer: OracleLayer, logits: np.ndarray, uniform=None):
+    """route(), then GShard's random second-expert dispatch when enabled.
+    Returns (probs, selected ids, dispatched ids, gates): the aux loss counts
+    the selected ids, slots take the dispatched ones."""
+    probs, ids, gates = route(layer, logits)
+    disp = ids
+    if layer.random_second and layer.k >= 2:
+        disp, gates = random_second_dispatch(ids, gates, uniform)
+    return probs, ids, disp, gates
 
 
 def layer_capacity(layer: OracleLayer) -> Optional[int]:
@@ -267,7 +343,7 @@ def layer_capacity(layer: OracleLayer) -> Optional[int]:
 
 
 def layer_forward(layer: OracleLayer, x, wg, w1, w2, w3=None, sw1=None, sw2=None, sw3=None,
-                  logit_add=None, logits=None, tokens=None, want_rows=False) -> dict:
+                  logit_add=None, logits=None, tokens=None, want_rows=False, uniform=None) -> dict:
     """The whole forward pass, stage by stage.
 
     `logits` (optional) replaces the router GEMM with given float32 logits, so
@@ -277,18 +353,21 @@ def layer_forward(layer: OracleLayer, x, wg, w1, w2, w3=None, sw1=None, sw2=None
     and the aux loss always cover every token.  Returns a dict with logits,
     probs, ids, gates, capacity, slot, count, kept, offsets, row_token, aux,
     y (for `tokens`, or all) and, with want_rows, the un-gated expert output of
-    every kept (token, choice) of those tokens.
+    every kept (token, choice) of those tokens.  `uniform` [T] drives GShard's
+    random second-expert dispatch when the layer enables it; `ids` are then the
+    dispatched ids (-1 = not dispatched) and `selected` the top-k ids.
     """
     T, E, k = layer.T, layer.E, layer.k
     if logits is None:
         logits = router_logits(x, wg, logit_add)
     logits = np.asarray(logits, dtype=np.float32)
-    probs, ids, gates = route(layer, logits)
+    probs, selected, ids, gates = route_and_dispatch(layer, logits, uniform)
     C = layer_capacity(layer)
     slot, count, kept = assign_slots(ids, E, C)
     off = row_layout(kept, T, layer.n_shared)
     rt = row_tokens(ids, slot, off, layer.n_shared)
-    aux = aux_loss(probs, ids, E, layer.aux_alpha)
+    aux = aux_loss(probs, selected, E, layer.aux_alpha)
+    zl = z_loss(logits, layer.z_coef)
 
     tok = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
     X = np.asarray(x, dtype=np.float64)
@@ -315,7 +394,7 @@ def layer_forward(layer: OracleLayer, x, wg, w1, w2, w3=None, sw1=None, sw2=None
         if want_rows:
             for i, t in enumerate(tok):
                 rows[(int(t), -1)] = Ys[i]
-    out = dict(logits=logits, probs=probs, ids=ids, gates=gates, capacity=C, slot=slot,
+    out = dict(logits=logits, probs=probs, ids=ids, selected=selected, gates=gates, capacity=C, slot=slot, zloss=zl,
                count=count, kept=kept, offsets=off, row_token=rt, aux=aux, y=y, tokens=tok)
     if want_rows:
         out["rows"] = rows

@@ -380,3 +380,132 @@ def test_planted_mistakes_are_caught(monkeypatch, golden):
     pr = O.softmax(lg)
     idk = O.topk_ids(lg, 2)
     assert not np.allclose(pr[np.arange(5)[:, None], idk].sum(1), 1.0)
+
+
+# ------------------------------------------------------------ router variants
+def test_sigmoid_scores_against_expit():
+    from scipy.special import expit
+    rng = np.random.default_rng(31)
+    l = (rng.standard_normal((40, 11)) * 5).astype(np.float32)
+    np.testing.assert_allclose(O.sigmoid(l), expit(l.astype(np.float64)), rtol=1e-14, atol=0)
+    assert O.sigmoid(np.float32(0.0)) == 0.5
+    assert O.sigmoid(np.float32(-200.0)) < 1e-80 and O.sigmoid(np.float32(200.0)) == 1.0
+    # P for sigmoid scores: normalised over the experts
+    P = O.router_probs(l, O.SCORE_SIGMOID_TOPK)
+    np.testing.assert_allclose(P.sum(1), 1.0, atol=1e-14)
+    a, b = 0.3, -1.2
+    P2 = O.router_probs(np.array([[a, b]], np.float32), O.SCORE_SIGMOID_TOPK)[0]
+    sa, sb = expit(float(np.float32(a))), expit(float(np.float32(b)))
+    assert abs(P2[0] - sa / (sa + sb)) < 1e-15
+    # equal logits: P = 1/E, so the aux loss is alpha whatever f is
+    z = np.full((16, 8), 0.7, np.float32)
+    Pz = O.router_probs(z, O.SCORE_SIGMOID_TOPK)
+    np.testing.assert_allclose(Pz, 1 / 8, atol=1e-15)
+    ids = np.array([[t % 3, 3 + t % 5] for t in range(16)], np.int32)
+    assert abs(O.aux_loss(Pz, ids, 8, 1e-2) - 1e-2) < 1e-15
+    # softmax scores are unchanged by the new branch
+    np.testing.assert_array_equal(O.router_probs(l, O.SCORE_SOFTMAX_TOPK), O.softmax(l))
+
+
+def test_sigmoid_gates():
+    from scipy.special import expit
+    rng = np.random.default_rng(32)
+    l = rng.standard_normal((50, 9)).astype(np.float32)
+    layer = O.OracleLayer(T=50, H=1, F=1, E=9, k=3, score=O.SCORE_SIGMOID_TOPK)
+    probs, ids, g = O.route(layer, l)
+    # selection is the same as under softmax (sigmoid is monotone)
+    np.testing.assert_array_equal(ids, O.topk_ids(l, 3))
+    sel = l.astype(np.float64)[np.arange(50)[:, None], ids]
+    np.testing.assert_allclose(g, expit(sel), rtol=1e-14)
+    assert (np.diff(g, axis=1) <= 0).all()
+    g_r = O.gate_values(l, probs, ids, O.SCORE_SIGMOID_TOPK, 1)
+    np.testing.assert_allclose(g_r.sum(1), 1.0, atol=1e-14)
+    np.testing.assert_allclose(g_r, expit(sel) / expit(sel).sum(1, keepdims=True), rtol=1e-14)
+
+
+def test_z_loss_closed_forms():
+    from scipy.special import logsumexp
+    rng = np.random.default_rng(33)
+    l = (rng.standard_normal((70, 13)) * 4).astype(np.float32)
+    want = 1e-3 * np.mean(logsumexp(l.astype(np.float64), axis=1) ** 2)
+    assert abs(O.z_loss(l, 1e-3) - want) <= 1e-15 * want
+    # equal logits c over E experts: lse = c + ln E
+    for c, E in [(0.0, 8), (2.5, 64), (-7.0, 3)]:
+        z = np.full((5, E), c, np.float32)
+        assert abs(O.z_loss(z, 0.1) - 0.1 * (c + math.log(E)) ** 2) < 1e-13
+    # one dominant logit: lse -> that logit, stable at large magnitudes
+    big = np.full((2, 4), -1e4, np.float32)
+    big[:, 1] = 1000.0
+    assert abs(O.z_loss(big, 1.0) - 1e6) < 1e-6
+    assert O.z_loss(np.zeros((0, 4), np.float32), 1.0) == 0.0
+    assert O.z_loss(l, 0.0) == 0.0
+    # planted slips: the mean of lse (not squared) and the max instead of lse
+    assert abs(1e-3 * np.mean(logsumexp(l.astype(np.float64), axis=1)) - want) > 1e-6
+    assert abs(1e-3 * np.mean(l.max(axis=1).astype(np.float64) ** 2) - want) > 1e-6
+
+
+def test_random_second_dispatch_rule():
+    T = 1000
+    ids = np.tile(np.array([[3, 5]], np.int32), (T, 1))
+    # second gate g: kept iff u < 2 g; on the grid u = i / T exactly ceil(2 g T) are kept
+    for g1 in (0.0, 0.05, 0.25, 0.3125, 0.5):
+        gates = np.tile(np.array([[1 - g1, g1]]), (T, 1))
+        u = np.arange(T) / T
+        d_ids, d_g = O.random_second_dispatch(ids, gates, u)
+        kept = d_ids[:, 1] >= 0
+        assert int(kept.sum()) == math.ceil(2 * g1 * T)
+        assert (d_ids[:, 0] == 3).all() and (d_g[:, 0] == 1 - g1).all()
+        assert (d_g[~kept, 1] == 0).all() and (d_g[kept, 1] == g1).all()
+        assert (d_ids[kept, 1] == 5).all() and (d_ids[~kept, 1] == -1).all()
+    # u = 0 keeps any positive gate; the inputs are not modified
+    gates = np.tile(np.array([[0.9, 1e-30]]), (T, 1))
+    d_ids, _ = O.random_second_dispatch(ids, gates, np.zeros(T))
+    assert (d_ids[:, 1] == 5).all() and (ids[:, 1] == 5).all()
+    # k=3: only the rank-1 choice is subject to the draw
+    ids3 = np.tile(np.array([[0, 1, 2]], np.int32), (4, 1))
+    g3 = np.tile(np.array([[0.5, 0.3, 0.2]]), (4, 1))
+    d3, _ = O.random_second_dispatch(ids3, g3, np.array([0.1, 0.59, 0.6, 0.99]))
+    np.testing.assert_array_equal(d3, [[0, 1, 2], [0, 1, 2], [0, -1, 2], [0, -1, 2]])
+
+
+def test_slots_skip_minus_one_equals_extra_expert():
+    """An undispatched choice (-1) takes no slot: the slots equal those of the
+    same assignments with -1 sent to an extra expert E that nobody reads."""
+    E, k, T = 3, 2, 4
+    pats = list(itertools.permutations(range(E), k))
+    rng = np.random.default_rng(34)
+    for combo in itertools.product(pats, repeat=T):
+        ids = np.array(combo, dtype=np.int32)
+        ids[rng.random(T) < 0.5, 1] = -1
+        alt = np.where(ids < 0, E, ids).astype(np.int32)
+        for C in (1, 2, None):
+            slot, count, kept = O.assign_slots(ids, E, C)
+            s2, c2, k2 = O.assign_slots(alt, E + 1, C)
+            np.testing.assert_array_equal(slot[ids >= 0], s2[ids >= 0])
+            assert (slot[ids < 0] == -1).all()
+            np.testing.assert_array_equal(count, c2[:E])
+            np.testing.assert_array_equal(kept, k2[:E])
+
+
+def test_layer_random_second_counts_selections_and_drops_rows():
+    E, k, T, H, F = 4, 2, 40, 8, 16
+    rng = np.random.default_rng(35)
+    x = rng.standard_normal((T, H))
+    wg = rng.standard_normal((E, H)) * 0.5
+    w1 = rng.standard_normal((E, F, H)) * 0.3
+    w2 = rng.standard_normal((E, H, F)) * 0.3
+    base = O.OracleLayer(T=T, H=H, F=F, E=E, k=k, score=O.SCORE_TOPK_SOFTMAX, cap_mode=O.CAP_DROPLESS)
+    rnd = O.OracleLayer(T=T, H=H, F=F, E=E, k=k, score=O.SCORE_TOPK_SOFTMAX, cap_mode=O.CAP_DROPLESS,
+                        random_second=1, z_coef=1e-2)
+    keep_all = O.layer_forward(rnd, x, wg, w1, w2, uniform=np.zeros(T))
+    ref = O.layer_forward(base, x, wg, w1, w2)
+    np.testing.assert_allclose(keep_all["y"], ref["y"], rtol=1e-13, atol=1e-13)
+    drop_all = O.layer_forward(rnd, x, wg, w1, w2, uniform=np.full(T, 0.999999))
+    assert drop_all["aux"] == ref["aux"]               # f counts the selections
+    assert int(drop_all["kept"].sum()) == T
+    # with every second choice gone, y is the first choice's output times g_t0
+    for t in range(T):
+        e = int(ref["ids"][t, 0])
+        h = np.maximum(w1[e] @ x[t], 0)
+        np.testing.assert_allclose(drop_all["y"][t], ref["gates"][t, 0] * (w2[e] @ h), rtol=1e-12, atol=1e-13)
+    assert drop_all["zloss"] == O.z_loss(drop_all["logits"], 1e-2)
