@@ -364,7 +364,7 @@ def run_ours(args, world, rank, local):
 
     def step(events=None):
         flush_l2()
-        B.moe_layer_fwd(cfg, inp["x"], inp["wg"], inp["logit_add"], wts, y, aux, None, ws, stage_events=events,
+        B.moe_layer_fwd(cfg, inp["x"], inp["wg"], inp["logit_add"], None, wts, y, aux, None, ws, stage_events=events,
                         stream=stream)
 
     for _ in range(max(args.warmup, 3)):
@@ -435,7 +435,7 @@ def run_ours(args, world, rank, local):
         x_dev.copy_(x_host, non_blocking=True)
         if add_host is not None:
             add_dev.copy_(add_host, non_blocking=True)
-        B.moe_layer_fwd(cfg, x_dev, inp["wg"], add_dev, wts, y, aux, None, ws, stream=stream)
+        B.moe_layer_fwd(cfg, x_dev, inp["wg"], add_dev, None, wts, y, aux, None, ws, stream=stream)
         y_host.copy_(y, non_blocking=True)
         aux_host.copy_(aux, non_blocking=True)
 

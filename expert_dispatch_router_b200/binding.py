@@ -19,7 +19,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libmoe_b200.so")
 
 MOE_OK, MOE_EINVAL, MOE_EUNSUPPORTED, MOE_ECUDA, MOE_ETIMEOUT, MOE_EDEVICE, MOE_EWORKSPACE = range(7)
-MOE_FLAG_KEEP_LOGITS = 1
+MOE_FLAG_KEEP_LOGITS, MOE_FLAG_RANDOM_SECOND = 1, 2
 MOE_N_STAGE_EVENTS = 8
 STAGES = ("router", "slots", "dispatch", "ffn_gemm1", "ffn_gemm2", "combine", "aux")
 
@@ -35,7 +35,8 @@ class moe_cfg(ctypes.Structure):
                 ("k", ctypes.c_int32), ("n_shared", ctypes.c_int32), ("act", ctypes.c_int32),
                 ("score", ctypes.c_int32), ("renorm", ctypes.c_int32), ("cap_mode", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("cf_num", ctypes.c_int64), ("cf_den", ctypes.c_int64),
-                ("min_capacity", ctypes.c_int64), ("aux_alpha", ctypes.c_float), ("flags", ctypes.c_int32)]
+                ("min_capacity", ctypes.c_int64), ("aux_alpha", ctypes.c_float), ("flags", ctypes.c_int32),
+                ("z_coef", ctypes.c_float)]
 
 
 class moe_weights(ctypes.Structure):
@@ -58,15 +59,15 @@ _SIGS = {
     "moe_rows_max": [CFGP, I64P],
     "moe_workspace_size": [CFGP, SZP],
     "moe_workspace_views": [CFGP, P, ctypes.POINTER(moe_ws_views)],
-    "moe_route": [CFGP, P, P, P, P, P, P, P, P],
-    "moe_route_from_logits": [CFGP, P, P, P, P, P],
+    "moe_route": [CFGP, P, P, P, P, P, P, P, P, P],
+    "moe_route_from_logits": [CFGP, P, P, P, P, P, P],
     "moe_assign_slots": [CFGP, P, P, P, P, P, P, P, P],
     "moe_assign_slots_static": [CFGP, P, P, P, P, P, P, P],
     "moe_dispatch": [CFGP, P, P, P, P, P, P],
     "moe_expert_ffn": [CFGP, P, P, P, ctypes.POINTER(moe_weights), P, P, P],
     "moe_combine": [CFGP, P, P, P, P, P, P, P],
     "moe_aux_loss": [CFGP, P, P, P],
-    "moe_layer_fwd": [CFGP, P, P, P, ctypes.POINTER(moe_weights), P, P, P, P, ctypes.c_size_t, P, P],
+    "moe_layer_fwd": [CFGP, P, P, P, P, ctypes.POINTER(moe_weights), P, P, P, P, ctypes.c_size_t, P, P],
     "moe_activation_eval": [ctypes.c_int, P, P, P, ctypes.c_int64, P],
     "moe_sync_status": [P, P],
     "moe_clear_status": [P, P],
@@ -120,7 +121,8 @@ def make_cfg(shape: synth.LayerShape, flags: int = 0, **override) -> moe_cfg:
     s = shape.replace(**override) if override else shape
     return moe_cfg(T=s.T, H=s.H, F=s.F, E=s.E, k=s.k, n_shared=s.n_shared, act=s.act, score=s.score,
                    renorm=s.renorm, cap_mode=s.cap_mode, dtype=s.dtype, cf_num=s.cf_num, cf_den=s.cf_den,
-                   min_capacity=s.min_capacity, aux_alpha=s.aux_alpha, flags=flags)
+                   min_capacity=s.min_capacity, aux_alpha=s.aux_alpha,
+                   flags=flags | (MOE_FLAG_RANDOM_SECOND if s.random_second else 0), z_coef=s.z_coef)
 
 
 def make_weights(inp: dict) -> moe_weights:
@@ -153,14 +155,14 @@ def moe_workspace_views(cfg: moe_cfg, ws: torch.Tensor) -> moe_ws_views:
 
 
 # ------------------------------------------------------------------ stages
-def moe_route(cfg, x, wg, logit_add, ids, gates, logits_out, ws, stream=None):
-    _check(load().moe_route(ctypes.byref(cfg), _ptr(x), _ptr(wg), _ptr(logit_add), _ptr(ids), _ptr(gates),
-                            _ptr(logits_out), _ptr(ws), _stream(stream)), "moe_route")
+def moe_route(cfg, x, wg, logit_add, uniform, ids, gates, logits_out, ws, stream=None):
+    _check(load().moe_route(ctypes.byref(cfg), _ptr(x), _ptr(wg), _ptr(logit_add), _ptr(uniform), _ptr(ids),
+                            _ptr(gates), _ptr(logits_out), _ptr(ws), _stream(stream)), "moe_route")
 
 
-def moe_route_from_logits(cfg, logits, ids, gates, ws, stream=None):
-    _check(load().moe_route_from_logits(ctypes.byref(cfg), _ptr(logits), _ptr(ids), _ptr(gates), _ptr(ws),
-                                        _stream(stream)), "moe_route_from_logits")
+def moe_route_from_logits(cfg, logits, uniform, ids, gates, ws, stream=None):
+    _check(load().moe_route_from_logits(ctypes.byref(cfg), _ptr(logits), _ptr(uniform), _ptr(ids), _ptr(gates),
+                                        _ptr(ws), _stream(stream)), "moe_route_from_logits")
 
 
 def moe_assign_slots(cfg, ids, slot, expert_count, kept_count, expert_offset, row_token, ws, stream=None):
@@ -194,13 +196,14 @@ def moe_aux_loss(cfg, ws, aux, stream=None):
     _check(load().moe_aux_loss(ctypes.byref(cfg), _ptr(ws), _ptr(aux), _stream(stream)), "moe_aux_loss")
 
 
-def moe_layer_fwd(cfg, x, wg, logit_add, weights: moe_weights, y, aux, expert_count, ws, stage_events=None,
-                  stream=None):
+def moe_layer_fwd(cfg, x, wg, logit_add, uniform, weights: moe_weights, y, aux, expert_count, ws,
+                  stage_events=None, stream=None):
     ev = None
     if stage_events is not None:
         arr = (ctypes.c_void_p * MOE_N_STAGE_EVENTS)(*[e.cuda_event for e in stage_events])
         ev = ctypes.cast(arr, ctypes.c_void_p)
-    _check(load().moe_layer_fwd(ctypes.byref(cfg), _ptr(x), _ptr(wg), _ptr(logit_add), ctypes.byref(weights),
+    _check(load().moe_layer_fwd(ctypes.byref(cfg), _ptr(x), _ptr(wg), _ptr(logit_add), _ptr(uniform),
+                                ctypes.byref(weights),
                                 _ptr(y), _ptr(aux), _ptr(expert_count), _ptr(ws), ws.numel() * ws.element_size(),
                                 ev, _stream(stream)), "moe_layer_fwd")
 

@@ -19,6 +19,8 @@ struct RouterParams {
   float* psum_part;         // [nblk,E]
   int32_t* cnt_part;        // [nblk,E]
   unsigned* aux_counter;    // ticket counter of the aux-loss kernel (re-armed here)
+  float* zsum_part;         // [nblk] per-CTA sums of lse^2 (z-loss), or null
+  const float* uniform;     // [T] GShard random second dispatch, or null
   int64_t T;
   int H, E, k, score, renorm;
 };
@@ -32,8 +34,9 @@ cudaError_t launch_router_gemm(const void* x, const float* wg, void* planes, flo
                                DevStatus* status, int* parts, cudaStream_t stream);
 cudaError_t launch_router(const RouterParams& p, bool bf16, cudaStream_t stream);
 // term: E doubles of scratch followed by one unsigned ticket counter.
-cudaError_t launch_aux(const float* psum_part, const int32_t* cnt_part, int nblk, int E, int64_t T, int k,
-                       float alpha, double* term, float* aux, cudaStream_t stream);
+// zsum_part (or null): per-CTA sums of lse^2; aux[1] = z_coef * their mean.
+cudaError_t launch_aux(const float* psum_part, const int32_t* cnt_part, const float* zsum_part, int nblk, int E,
+                       int64_t T, int k, float alpha, float z_coef, double* term, float* aux, cudaStream_t stream);
 // Evaluates the GEMM epilogue's activation: out = act(z) (ReLU, GELU) or silu(z) * u (SwiGLU).
 cudaError_t launch_activation_eval(int act, const float* z, const float* u, float* out, int64_t n,
                                    cudaStream_t stream);
@@ -54,10 +57,13 @@ struct SlotParams {
   // optional aux loss (fused layer path): router partial sums of p, one fp64 term
   // per expert, and the output scalar
   const float* psum_part;   // [nblk_router, E] or null
+  const int32_t* cnt_part;  // [nblk_router, E] selection counts, or null: count the dispatched ids
   int nblk_router;
   double* aux_term;         // [E]
-  float* aux;
+  float* aux;               // [1], or [2] with the z-loss in aux[1]
   float aux_alpha;
+  const float* zsum_part;   // [nblk_router] router sums of lse^2, or null: no z-loss
+  float z_coef;
 };
 constexpr int kSlotChunk = 256;    // assignments per CTA of the slot kernels (one per thread)
 cudaError_t launch_slots(const SlotParams& p, cudaStream_t stream);

@@ -2,6 +2,7 @@
 // capacity, the row bound, the workspace layout, and the stage launches.
 // Nothing here allocates device memory or synchronises (moe_sync_status
 // excepted, which exists to do exactly that).
+#include <math.h>
 #include <string.h>
 
 #include "common.cuh"
@@ -14,7 +15,7 @@ namespace {
 constexpr int64_t kMaxCf = int64_t(1) << 20;
 
 struct Layout {
-  size_t status, psum, cnt, term, chunk, ids, gates, slot, ecount, kept, off, rowtok, logits, lparts, planes, xbuf,
+  size_t status, psum, cnt, zsum, term, chunk, ids, gates, slot, ecount, kept, off, rowtok, logits, lparts, planes, xbuf,
       hbuf, ybuf;
   size_t total;
   int nblk_router, nchunk;
@@ -27,12 +28,14 @@ bool valid_cfg(const moe_cfg* c) {
   if (c->k > c->E) return false;
   if (c->n_shared != 0 && c->n_shared != 1) return false;
   if (c->act < MOE_ACT_RELU || c->act > MOE_ACT_SWIGLU) return false;
-  if (c->score != MOE_SCORE_SOFTMAX_TOPK && c->score != MOE_SCORE_TOPK_SOFTMAX) return false;
+  if (c->score < MOE_SCORE_SOFTMAX_TOPK || c->score > MOE_SCORE_SIGMOID_TOPK) return false;
   if (c->renorm != 0 && c->renorm != 1) return false;
   if (c->cap_mode != MOE_CAP_CAPACITY && c->cap_mode != MOE_CAP_DROPLESS) return false;
   if (c->dtype != MOE_DTYPE_F32 && c->dtype != MOE_DTYPE_BF16) return false;
   if (c->cap_mode == MOE_CAP_CAPACITY && (c->cf_num <= 0 || c->cf_den <= 0)) return false;
   if (c->min_capacity < 0) return false;
+  if (!(c->z_coef >= 0.0f) || isinf(c->z_coef)) return false;
+  if (c->flags & ~(MOE_FLAG_KEEP_LOGITS | MOE_FLAG_RANDOM_SECOND)) return false;
   return true;
 }
 
@@ -84,6 +87,7 @@ Layout layout_of(const moe_cfg* c) {
   L.status = take(sizeof(DevStatus));
   L.psum = take(sizeof(float) * L.nblk_router * E);
   L.cnt = take(sizeof(int32_t) * L.nblk_router * E);
+  L.zsum = take(sizeof(float) * L.nblk_router);
   L.term = take(sizeof(double) * (E + 1));      // E terms + the aux ticket counter
   L.chunk = take(sizeof(int32_t) * E * (size_t)L.nchunk);
   L.ids = take(sizeof(int32_t) * T * k);
@@ -111,11 +115,15 @@ cudaStream_t S(moe_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ECUDA; }
 
+bool random_second(const moe_cfg* c) { return (c->flags & MOE_FLAG_RANDOM_SECOND) && c->k >= 2; }
+bool has_zloss(const moe_cfg* c) { return c->z_coef != 0.0f; }
+
 RouterParams router_params(const moe_cfg* c, const Layout& L, void* ws) {
   RouterParams p{};
   p.psum_part = at<float>(ws, L.psum);
   p.cnt_part = at<int32_t>(ws, L.cnt);
   p.aux_counter = reinterpret_cast<unsigned*>(at<double>(ws, L.term) + c->E);
+  p.zsum_part = has_zloss(c) ? at<float>(ws, L.zsum) : nullptr;
   p.T = c->T;
   p.H = c->H;
   p.E = c->E;
@@ -126,8 +134,11 @@ RouterParams router_params(const moe_cfg* c, const Layout& L, void* ws) {
 }
 
 int run_route(const moe_cfg* c, const Layout& L, const void* x, const float* wg, const float* logit_add,
-              const float* logits_in, int32_t* ids, float* gates, float* logits_out, void* ws, cudaStream_t s) {
+              const float* logits_in, const float* uniform, int32_t* ids, float* gates, float* logits_out, void* ws,
+              cudaStream_t s) {
+  if (random_second(c) && c->T > 0 && uniform == nullptr) return MOE_EINVAL;
   RouterParams p = router_params(c, L, ws);
+  p.uniform = random_second(c) ? uniform : nullptr;
   p.logits_parts = 1;
   if (logits_in == nullptr && c->dtype == MOE_DTYPE_BF16 && c->T > 0) {
     // logits on the tensor cores, then the softmax / top-k / gate kernel on them
@@ -172,6 +183,9 @@ int run_slots(const moe_cfg* c, const Layout& L, const int32_t* ids, int32_t* sl
     p.aux_term = at<double>(ws, L.term);
     p.aux = aux;
     p.aux_alpha = c->aux_alpha;
+    p.cnt_part = random_second(c) ? at<int32_t>(ws, L.cnt) : nullptr;   // f counts selections, not dispatches
+    p.zsum_part = has_zloss(c) ? at<float>(ws, L.zsum) : nullptr;
+    p.z_coef = c->z_coef;
   }
   return cuda_status(launch_slots(p, s));
 }
@@ -326,22 +340,23 @@ int moe_workspace_views(const moe_cfg* cfg, void* ws, moe_ws_views* v) {
   return MOE_OK;
 }
 
-int moe_route(const moe_cfg* cfg, const void* x, const float* wg, const float* logit_add, int32_t* ids,
-              float* gates, float* logits_out, void* ws, moe_stream_t stream) {
+int moe_route(const moe_cfg* cfg, const void* x, const float* wg, const float* logit_add, const float* uniform,
+              int32_t* ids, float* gates, float* logits_out, void* ws, moe_stream_t stream) {
   const int st = check_cfg(cfg);
   if (st != MOE_OK) return st;
   if (cfg->T > 0 && (x == nullptr || wg == nullptr || ids == nullptr || gates == nullptr)) return MOE_EINVAL;
   if (ws == nullptr) return MOE_EINVAL;
-  return run_route(cfg, layout_of(cfg), x, wg, logit_add, nullptr, ids, gates, logits_out, ws, S(stream));
+  return run_route(cfg, layout_of(cfg), x, wg, logit_add, nullptr, uniform, ids, gates, logits_out, ws, S(stream));
 }
 
-int moe_route_from_logits(const moe_cfg* cfg, const float* logits, int32_t* ids, float* gates, void* ws,
-                          moe_stream_t stream) {
+int moe_route_from_logits(const moe_cfg* cfg, const float* logits, const float* uniform, int32_t* ids, float* gates,
+                          void* ws, moe_stream_t stream) {
   const int st = check_cfg(cfg);
   if (st != MOE_OK) return st;
   if (cfg->T > 0 && (logits == nullptr || ids == nullptr || gates == nullptr)) return MOE_EINVAL;
   if (ws == nullptr) return MOE_EINVAL;
-  return run_route(cfg, layout_of(cfg), nullptr, nullptr, nullptr, logits, ids, gates, nullptr, ws, S(stream));
+  return run_route(cfg, layout_of(cfg), nullptr, nullptr, nullptr, logits, uniform, ids, gates, nullptr, ws,
+                   S(stream));
 }
 
 int moe_assign_slots(const moe_cfg* cfg, const int32_t* ids, int32_t* slot, int32_t* expert_count,
@@ -403,12 +418,13 @@ int moe_aux_loss(const moe_cfg* cfg, const void* ws, float* aux, moe_stream_t st
   if (ws == nullptr || aux == nullptr) return MOE_EINVAL;
   const Layout L = layout_of(cfg);
   void* w = const_cast<void*>(ws);
-  return cuda_status(launch_aux(at<float>(w, L.psum), at<int32_t>(w, L.cnt), L.nblk_router, cfg->E, cfg->T, cfg->k,
-                                cfg->aux_alpha, at<double>(w, L.term), aux, S(stream)));
+  return cuda_status(launch_aux(at<float>(w, L.psum), at<int32_t>(w, L.cnt),
+                                has_zloss(cfg) ? at<float>(w, L.zsum) : nullptr, L.nblk_router, cfg->E, cfg->T,
+                                cfg->k, cfg->aux_alpha, cfg->z_coef, at<double>(w, L.term), aux, S(stream)));
 }
 
-int moe_layer_fwd(const moe_cfg* cfg, const void* x, const float* wg, const float* logit_add, const moe_weights* w,
-                  void* y, float* aux, int32_t* expert_count, void* ws, size_t ws_bytes,
+int moe_layer_fwd(const moe_cfg* cfg, const void* x, const float* wg, const float* logit_add, const float* uniform,
+                  const moe_weights* w, void* y, float* aux, int32_t* expert_count, void* ws, size_t ws_bytes,
                   const moe_event_t* stage_events, moe_stream_t stream) {
   int st = check_cfg(cfg);
   if (st != MOE_OK) return st;
@@ -429,7 +445,7 @@ int moe_layer_fwd(const moe_cfg* cfg, const void* x, const float* wg, const floa
   float* logits = (cfg->flags & MOE_FLAG_KEEP_LOGITS) ? at<float>(ws, L.logits) : nullptr;
 
   if ((st = record(stage_events, 0, s)) != MOE_OK) return st;
-  if ((st = run_route(cfg, L, x, wg, logit_add, nullptr, ids, gates, logits, ws, s)) != MOE_OK) return st;
+  if ((st = run_route(cfg, L, x, wg, logit_add, nullptr, uniform, ids, gates, logits, ws, s)) != MOE_OK) return st;
   if ((st = record(stage_events, 1, s)) != MOE_OK) return st;
   if ((st = run_slots(cfg, L, ids, slot, at<int32_t>(ws, L.ecount), at<int32_t>(ws, L.kept), off,
                       at<int32_t>(ws, L.rowtok), ws, s, aux)) != MOE_OK)

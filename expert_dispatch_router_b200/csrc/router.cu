@@ -47,113 +47,136 @@ __device__ __forceinline__ float from_ordered(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
-// Softmax, top-k and gates of token t from its E values spread over the warp's
+// Scores, top-k and gates of token t from its E values spread over the warp's
 // lanes (val[j] belongs to expert lane_expert(lane, j)), adding the logit offset
-// and storing the logits if asked; accumulates this lane's sums of p and
-// selection counts.
+// and storing the logits if asked.  Accumulates this lane's sums of the
+// probabilities the aux loss averages (softmax, or sigmoids normalised over the
+// experts), its selection counts, and (zacc, same value in every lane) the
+// squared log-sum-exp of the z-loss.
 template <int EJ>
 __device__ __forceinline__ void route_token(const RouterParams& p, int64_t t, int lane, const float (&val)[EJ],
-                                            float (&psum)[EJ], int (&cnt)[EJ]) {
+                                            float (&psum)[EJ], int (&cnt)[EJ], float& zacc) {
   const int E = p.E;
-    float l[EJ];
-    float m = -INFINITY;
+  float l[EJ];
+  float m = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < EJ; ++j) {
+    const int e = lane_expert<EJ>(lane, j);
+    float v = val[j];
+    if (e < E) {
+      if (p.logit_add != nullptr) v += p.logit_add[t * E + e];
+      if (p.logits_out != nullptr) p.logits_out[t * E + e] = v;
+      l[j] = v;
+      m = fmaxf(m, v);
+    } else {
+      l[j] = -INFINITY;
+    }
+  }
+  m = from_ordered(__reduce_max_sync(0xffffffffu, to_ordered(m)));
+  float s = 0.0f, ex[EJ];
+#pragma unroll
+  for (int j = 0; j < EJ; ++j) {
+    ex[j] = lane_expert<EJ>(lane, j) < E ? expf(l[j] - m) : 0.0f;
+    s += ex[j];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  const bool sigmoid = p.score == MOE_SCORE_SIGMOID_TOPK;
+  if (sigmoid) {
+    float ss = 0.0f, sg[EJ];
 #pragma unroll
     for (int j = 0; j < EJ; ++j) {
-      const int e = lane_expert<EJ>(lane, j);
-      float v = val[j];
-      if (e < E) {
-        if (p.logit_add != nullptr) v += p.logit_add[t * E + e];
-        if (p.logits_out != nullptr) p.logits_out[t * E + e] = v;
-        l[j] = v;
-        m = fmaxf(m, v);
-      } else {
-        l[j] = -INFINITY;
-      }
-    }
-    m = from_ordered(__reduce_max_sync(0xffffffffu, to_ordered(m)));
-    float s = 0.0f, ex[EJ];
-#pragma unroll
-    for (int j = 0; j < EJ; ++j) {
-      ex[j] = lane_expert<EJ>(lane, j) < E ? expf(l[j] - m) : 0.0f;
-      s += ex[j];
+      sg[j] = lane_expert<EJ>(lane, j) < E ? 1.0f / (1.0f + expf(-l[j])) : 0.0f;
+      ss += sg[j];
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float inv_ss = 1.0f / ss;
+#pragma unroll
+    for (int j = 0; j < EJ; ++j) psum[j] += sg[j] * inv_ss;
+  } else {
     const float inv_s = 1.0f / s;
 #pragma unroll
     for (int j = 0; j < EJ; ++j) psum[j] += ex[j] * inv_s;
+  }
+  if (p.zsum_part != nullptr) {
+    const float lse = m + logf(s);
+    zacc += lse * lse;
+  }
 
-    // top-k: each round, the warp's best remaining (logit, lower index) key is found
-    // with two 32-bit max reductions: first the order-preserving logit bits, then,
-    // among lanes holding that logit, the complemented expert index.
-    unsigned selected = 0u;
-    float my_l = -INFINITY;
-    int my_e = -1;
-    uint32_t bh = 0u, bl = 0u;      // this lane's best unselected candidate
-    int bj = -1;
-    auto lane_best = [&]() {
-      bh = 0u; bl = 0u; bj = -1;
+  // top-k: each round, the warp's best remaining (logit, lower index) key is found
+  // with two 32-bit max reductions: first the order-preserving logit bits, then,
+  // among lanes holding that logit, the complemented expert index.
+  unsigned selected = 0u;
+  float my_l = -INFINITY;
+  int my_e = -1;
+  uint32_t bh = 0u, bl = 0u;      // this lane's best unselected candidate
+  int bj = -1;
+  auto lane_best = [&]() {
+    bh = 0u; bl = 0u; bj = -1;
 #pragma unroll
-      for (int j = 0; j < EJ; ++j) {
-        const int e = lane_expert<EJ>(lane, j);
-        if (e < E && !((selected >> j) & 1u)) {
-          const uint32_t h = to_ordered(l[j]), lo = 0xffffffffu - (uint32_t)e;
-          if (h > bh || (h == bh && lo > bl)) { bh = h; bl = lo; bj = j; }
-        }
+    for (int j = 0; j < EJ; ++j) {
+      const int e = lane_expert<EJ>(lane, j);
+      if (e < E && !((selected >> j) & 1u)) {
+        const uint32_t h = to_ordered(l[j]), lo = 0xffffffffu - (uint32_t)e;
+        if (h > bh || (h == bh && lo > bl)) { bh = h; bl = lo; bj = j; }
       }
-    };
-    lane_best();
+    }
+  };
+  lane_best();
 #pragma unroll 1
-    for (int r = 0; r < p.k; ++r) {
-      const uint32_t wh = __reduce_max_sync(0xffffffffu, bh);
-      const uint32_t wl = __reduce_max_sync(0xffffffffu, bh == wh ? bl : 0u);
-      if (lane == r) { my_l = from_ordered(wh); my_e = (int)(0xffffffffu - wl); }
-      if (bj >= 0 && bh == wh && bl == wl) {      // this lane owned the winner
-        selected |= 1u << bj;
+  for (int r = 0; r < p.k; ++r) {
+    const uint32_t wh = __reduce_max_sync(0xffffffffu, bh);
+    const uint32_t wl = __reduce_max_sync(0xffffffffu, bh == wh ? bl : 0u);
+    if (lane == r) { my_l = from_ordered(wh); my_e = (int)(0xffffffffu - wl); }
+    if (bj >= 0 && bh == wh && bl == wl) {      // this lane owned the winner
+      selected |= 1u << bj;
 #pragma unroll
-        for (int j = 0; j < EJ; ++j)
-          if (j == bj) cnt[j] += 1;
-        lane_best();
-      }
+      for (int j = 0; j < EJ; ++j)
+        if (j == bj) cnt[j] += 1;
+      lane_best();
     }
-    // gates: lane r holds the rank-r selection
-    float g = 0.0f;
-    if (lane < p.k) g = expf(my_l - m);        // top-1 logit equals m
-    if (p.score == MOE_SCORE_SOFTMAX_TOPK) {
-      g *= inv_s;
-      if (p.renorm) {
-        float gs = g;
+  }
+  // gates: lane r holds the rank-r selection
+  float g = 0.0f;
+  if (lane < p.k) g = sigmoid ? 1.0f / (1.0f + expf(-my_l)) : expf(my_l - m);   // top-1 logit equals m
+  if (p.score == MOE_SCORE_TOPK_SOFTMAX || p.renorm) {
+    float gs = g;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) gs += __shfl_xor_sync(0xffffffffu, gs, o);
-        g = g / gs;
-      }
-    } else {
-      float gs = g;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) gs += __shfl_xor_sync(0xffffffffu, gs, o);
-      g = g / gs;
-    }
-    if (lane < p.k) {
-      p.ids[t * p.k + lane] = my_e;
-      p.gates[t * p.k + lane] = g;
-    }
+    for (int o = 16; o > 0; o >>= 1) gs += __shfl_xor_sync(0xffffffffu, gs, o);
+    g = g / gs;
+  } else if (p.score == MOE_SCORE_SOFTMAX_TOPK) {
+    g = g / s;
+  }
+  // GShard top-2: the second choice is dispatched iff u_t < 2 g_t1
+  if (p.uniform != nullptr && lane == 1 && !(p.uniform[t] < 2.0f * g)) {
+    my_e = -1;
+    g = 0.0f;
+  }
+  if (lane < p.k) {
+    p.ids[t * p.k + lane] = my_e;
+    p.gates[t * p.k + lane] = g;
+  }
 }
 
-// Sums the warps' per-expert partials in a fixed order and stores this CTA's row
-// of psum_part / cnt_part.  `smem` must hold 2 * WARPS * 32 * EJ words.
+// Sums the warps' per-expert partials (and z-loss sums) in a fixed order and
+// stores this CTA's row of psum_part / cnt_part (and zsum_part).  `smem` must
+// hold 2 * WARPS * 32 * EJ + WARPS words.
 template <int EJ, int WARPS>
 __device__ __forceinline__ void write_partials(const RouterParams& p, float* smem, const float (&psum)[EJ],
-                                               const int (&cnt)[EJ]) {
+                                               const int (&cnt)[EJ], float zacc) {
   constexpr int EP = 32 * EJ;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   float* rp = smem;                                     // [WARPS][EP]
   int* rc = reinterpret_cast<int*>(smem + WARPS * EP);
+  float* rz = smem + 2 * WARPS * EP;                    // [WARPS]
 #pragma unroll
   for (int j = 0; j < EJ; ++j) {
     const int e = lane_expert<EJ>(lane, j);
     rp[warp * EP + e] = psum[j];
     rc[warp * EP + e] = cnt[j];
   }
+  if (lane == 0) rz[warp] = zacc;
   __syncthreads();
   for (int e = tid; e < p.E; e += WARPS * 32) {
     float ps = 0.0f;
@@ -163,13 +186,19 @@ __device__ __forceinline__ void write_partials(const RouterParams& p, float* sme
     p.psum_part[(int64_t)blockIdx.x * p.E + e] = ps;
     p.cnt_part[(int64_t)blockIdx.x * p.E + e] = cs;
   }
+  if (tid == 0 && p.zsum_part != nullptr) {
+    float z = 0.0f;
+#pragma unroll
+    for (int w = 0; w < WARPS; ++w) z += rz[w];
+    p.zsum_part[blockIdx.x] = z;
+  }
 }
 
 template <int EJ, int TW>
 constexpr int router_smem_floats() {
   constexpr int EP = 32 * EJ;
   constexpr int main_ = kRouterWarps * TW * kKC + kKC * (EP + 4);
-  constexpr int red = 2 * kRouterWarps * EP;
+  constexpr int red = 2 * kRouterWarps * EP + kRouterWarps;
   return main_ > red ? main_ : red;
 }
 
@@ -283,19 +312,19 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterParams p) 
   }
 
   // ---------------- epilogue: softmax, top-k, gates, partial sums
-  float psum[EJ];
+  float psum[EJ], zacc = 0.0f;
   int cnt[EJ];
 #pragma unroll
   for (int j = 0; j < EJ; ++j) { psum[j] = 0.0f; cnt[j] = 0; }
 #pragma unroll
   for (int i = 0; i < TW; ++i) {
     const int64_t t = t0 + warp * TW + i;
-    if (t < p.T) route_token<EJ>(p, t, lane, acc[i], psum, cnt);
+    if (t < p.T) route_token<EJ>(p, t, lane, acc[i], psum, cnt, zacc);
   }
 
   // ---------------- fixed-order reduction of the per-warp partials
   __syncthreads();
-  write_partials<EJ, kRouterWarps>(p, smem, psum, cnt);
+  write_partials<EJ, kRouterWarps>(p, smem, psum, cnt, zacc);
 }
 
 // Routing from given fp32 logits (the tensor-core router's output, or the
@@ -305,12 +334,12 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterParams p) 
 constexpr int kLogitWarps = 8;
 
 template <int EJ>
-__global__ void __launch_bounds__(kLogitWarps * 32) route_logits_kernel(RouterParams p, int bt) {
+__global__ void __launch_bounds__(kLogitWarps * 32, EJ <= 4 ? 3 : 1) route_logits_kernel(RouterParams p, int bt) {
   extern __shared__ __align__(16) float smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t t0 = (int64_t)blockIdx.x * bt;
   if (blockIdx.x == 0 && tid == 0 && p.aux_counter != nullptr) *p.aux_counter = 0u;
-  float psum[EJ];
+  float psum[EJ], zacc = 0.0f;
   int cnt[EJ];
 #pragma unroll
   for (int j = 0; j < EJ; ++j) { psum[j] = 0.0f; cnt[j] = 0; }
@@ -328,10 +357,10 @@ __global__ void __launch_bounds__(kLogitWarps * 32) route_logits_kernel(RouterPa
       }
       val[j] = v;
     }
-    route_token<EJ>(p, t, lane, val, psum, cnt);
+    route_token<EJ>(p, t, lane, val, psum, cnt, zacc);
   }
   __syncthreads();
-  write_partials<EJ, kLogitWarps>(p, smem, psum, cnt);
+  write_partials<EJ, kLogitWarps>(p, smem, psum, cnt, zacc);
 }
 
 // Tokens per CTA of the router for E experts (the host needs it to size the
@@ -364,7 +393,7 @@ static cudaError_t launch_router_ej(const RouterParams& p, bool bf16, cudaStream
 template <int EJ>
 static cudaError_t launch_route_logits_ej(const RouterParams& p, cudaStream_t stream) {
   const int bt = router_tile_tokens(p.E);
-  const size_t smem = sizeof(float) * 2 * kLogitWarps * 32 * EJ;
+  const size_t smem = sizeof(float) * (2 * kLogitWarps * 32 * EJ + kLogitWarps);
   const unsigned grid = (unsigned)((p.T + bt - 1) / bt);
   auto k = route_logits_kernel<EJ>;
   cudaError_t e = ensure_smem(k, smem);
@@ -400,13 +429,17 @@ cudaError_t launch_router(const RouterParams& p, bool bf16, cudaStream_t stream)
 constexpr int kAuxWarps = 8;
 
 __global__ void __launch_bounds__(kAuxWarps * 32) aux_kernel(const float* psum_part, const int32_t* cnt_part,
-                                                             int nblk, int E, int64_t T, int k, float alpha,
-                                                             double* term, unsigned* counter, float* aux) {
+                                                             const float* zsum_part, int nblk, int E, int64_t T,
+                                                             int k, float alpha, float z_coef, double* term,
+                                                             unsigned* counter, float* aux) {
   __shared__ double sh[kAuxWarps * 32];
   __shared__ bool last;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
   if (T == 0) {
-    if (tid == 0) *aux = 0.0f;
+    if (tid == 0) {
+      aux[0] = 0.0f;
+      if (zsum_part != nullptr) aux[1] = 0.0f;
+    }
     return;
   }
   const int e = blockIdx.x * kAuxWarps + warp;
@@ -438,17 +471,29 @@ __global__ void __launch_bounds__(kAuxWarps * 32) aux_kernel(const float* psum_p
     if (tid < s2) sh[tid] += sh[tid + s2];
     __syncthreads();
   }
-  if (tid == 0) {
-    *aux = (float)((double)alpha * (double)E * sh[0]);
-    *counter = 0u;
+  if (tid == 0) aux[0] = (float)((double)alpha * (double)E * sh[0]);
+  if (zsum_part != nullptr) {
+    // z-loss = coef * mean_t lse_t^2 over the router CTAs' sums, fixed tree
+    __syncthreads();
+    double z = 0.0;
+    for (int b = tid; b < nblk; b += kAuxWarps * 32) z += (double)zsum_part[b];
+    sh[tid] = z;
+    __syncthreads();
+    for (int s2 = kAuxWarps * 16; s2 > 0; s2 >>= 1) {
+      if (tid < s2) sh[tid] += sh[tid + s2];
+      __syncthreads();
+    }
+    if (tid == 0) aux[1] = (float)((double)z_coef * sh[0] / (double)T);
   }
+  if (tid == 0) *counter = 0u;
 }
 
-cudaError_t launch_aux(const float* psum_part, const int32_t* cnt_part, int nblk, int E, int64_t T, int k,
-                       float alpha, double* term, float* aux, cudaStream_t stream) {
+cudaError_t launch_aux(const float* psum_part, const int32_t* cnt_part, const float* zsum_part, int nblk, int E,
+                       int64_t T, int k, float alpha, float z_coef, double* term, float* aux, cudaStream_t stream) {
   unsigned* counter = reinterpret_cast<unsigned*>(term + E);
   const int grid = T == 0 ? 1 : (E + kAuxWarps - 1) / kAuxWarps;
-  aux_kernel<<<grid, kAuxWarps * 32, 0, stream>>>(psum_part, cnt_part, nblk, E, T, k, alpha, term, counter, aux);
+  aux_kernel<<<grid, kAuxWarps * 32, 0, stream>>>(psum_part, cnt_part, zsum_part, nblk, E, T, k, alpha, z_coef,
+                                                  term, counter, aux);
   return cudaGetLastError();
 }
 

@@ -42,6 +42,7 @@ __global__ void __launch_bounds__(kSlotThreads) slot_count_kernel(SlotParams p, 
   for (int i = threadIdx.x; i < kSlotChunk; i += kSlotThreads) {
     const int e = load_assignment(p, a0 + i, A);
     if (a0 + i >= A) break;
+    if (e == -1) continue;                      // a choice that is not dispatched
     if (e < 0 || e >= p.E) { set_status(p.status, MOE_EDEVICE, 1); continue; }
     atomicAdd(&hist[e], 1);
   }
@@ -97,19 +98,31 @@ __global__ void __launch_bounds__(kSlotThreads) slot_scan_kernel(SlotParams p, i
     p.kept_count[e] = kept;
   }
   if (p.psum_part != nullptr) {
-    // this expert's aux-loss term f_e * P_e: f from the pre-drop count, P from the
-    // router's per-CTA sums of p (fp64, fixed block-then-tree order)
+    // this expert's aux-loss term f_e * P_e: f from the pre-drop count (or, when
+    // some choices were not dispatched, from the router's selection counts), P
+    // from the router's per-CTA sums of p (fp64, fixed block-then-tree order)
     __shared__ double red[kSlotThreads];
+    __shared__ long long redc[kSlotThreads];
     double ps = 0.0;
-    for (int b = threadIdx.x; b < p.nblk_router; b += kSlotThreads) ps += (double)p.psum_part[(int64_t)b * p.E + e];
+    long long cs = 0;
+    for (int b = threadIdx.x; b < p.nblk_router; b += kSlotThreads) {
+      ps += (double)p.psum_part[(int64_t)b * p.E + e];
+      if (p.cnt_part != nullptr) cs += p.cnt_part[(int64_t)b * p.E + e];
+    }
     red[threadIdx.x] = ps;
+    redc[threadIdx.x] = cs;
     __syncthreads();
     for (int s = kSlotThreads / 2; s > 0; s >>= 1) {
-      if ((int)threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
+      if ((int)threadIdx.x < s) {
+        red[threadIdx.x] += red[threadIdx.x + s];
+        redc[threadIdx.x] += redc[threadIdx.x + s];
+      }
       __syncthreads();
     }
-    if (threadIdx.x == 0)
-      p.aux_term[e] = ((double)running / ((double)p.T * p.k)) * (red[0] / (double)p.T);
+    if (threadIdx.x == 0) {
+      const double f = (double)(p.cnt_part != nullptr ? redc[0] : running) / ((double)p.T * p.k);
+      p.aux_term[e] = f * (red[0] / (double)p.T);
+    }
   }
 }
 
@@ -158,6 +171,19 @@ __global__ void __launch_bounds__(1024) slot_offsets_kernel(SlotParams p) {
       __syncthreads();
     }
     if (tid == 0) *p.aux = (float)((double)p.aux_alpha * (double)p.E * red[0]);
+    if (p.zsum_part != nullptr) {
+      // z-loss = coef * mean_t lse_t^2 from the router's per-CTA sums, fixed tree
+      __syncthreads();
+      double z = 0.0;
+      for (int b = tid; b < p.nblk_router; b += 1024) z += (double)p.zsum_part[b];
+      red[tid] = z;
+      __syncthreads();
+      for (int s = 512; s > 0; s >>= 1) {
+        if (tid < s) red[tid] += red[tid + s];
+        __syncthreads();
+      }
+      if (tid == 0) p.aux[1] = p.T > 0 ? (float)((double)p.z_coef * red[0] / (double)p.T) : 0.0f;
+    }
   }
   // padding rows of each routed block -> -1
   for (int e = warp; e < p.E; e += 32) {

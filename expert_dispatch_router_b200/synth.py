@@ -26,6 +26,9 @@ Recipe (documented once here, used by tests and the benchmark):
     draws experts with Zipf(1.1)-skewed loads.
   * "unit" scale variant: x ~ N(0, 1), weights ~ N(0, 1/fan_in), used where the
     configuration's tiny output scale would make an absolute tolerance vacuous.
+  * layers with GShard's random second-expert dispatch get uniform [T] fp32
+    draws in [0, 1), drawn after everything else (the other tensors are the
+    same as without the option).
 """
 from __future__ import annotations
 
@@ -37,7 +40,7 @@ import torch
 
 # Activation / scoring / capacity / dtype enumerations shared by the harness.
 ACT_RELU, ACT_GELU, ACT_SWIGLU = 0, 1, 2
-SCORE_SOFTMAX_TOPK, SCORE_TOPK_SOFTMAX = 0, 1
+SCORE_SOFTMAX_TOPK, SCORE_TOPK_SOFTMAX, SCORE_SIGMOID_TOPK = 0, 1, 2
 CAP_CAPACITY, CAP_DROPLESS = 0, 1
 DTYPE_F32, DTYPE_BF16 = 0, 1
 
@@ -63,6 +66,8 @@ class LayerShape:
     dtype: int = DTYPE_BF16
     bias_row0: float = 0.0        # added to router row 0 (overflowing expert)
     zipf_skew: float = 0.0        # >0: Gumbel/Zipf logit offset exponent
+    z_coef: float = 0.0           # router z-loss coefficient (0 = off)
+    random_second: int = 0        # GShard random dispatch of the second choice
 
     def replace(self, **kw) -> "LayerShape":
         return dataclasses.replace(self, **kw)
@@ -99,7 +104,8 @@ def make_inputs(shape: LayerShape, seed: int = 0, device: str = "cpu",
     Returns a dict of torch tensors on `device`:
       x [T,H] (bf16, or fp32 for the fp32 layer), wg [E,H] fp32,
       w1 [E,F,H], w2 [E,H,F], w3 [E,F,H] or None, and for a shared expert
-      sw1 [1,F,H], sw2 [1,H,F], sw3 [1,F,H] or None; logit_add [T,E] fp32 or None.
+      sw1 [1,F,H], sw2 [1,H,F], sw3 [1,F,H] or None; logit_add [T,E] fp32 or None;
+      uniform [T] fp32 in [0,1) or None (random second-expert dispatch).
     `experts` (optional) draws only that many routed experts' weights, for
     host-side tests that never route to the others.
     """
@@ -122,7 +128,7 @@ def make_inputs(shape: LayerShape, seed: int = 0, device: str = "cpu",
     w3 = _normal(gen, (nE, F, H), math.sqrt(s / H), device).to(wdt) if shape.act == ACT_SWIGLU else None
     w2 = _normal(gen, (nE, H, F), math.sqrt(s / F), device).to(wdt)
     out = dict(x=x.to(wdt), wg=wg.contiguous(), w1=w1, w2=w2, w3=w3,
-               sw1=None, sw2=None, sw3=None, logit_add=None)
+               sw1=None, sw2=None, sw3=None, logit_add=None, uniform=None)
     if shape.n_shared:
         out["sw1"] = _normal(gen, (1, F, H), math.sqrt(s / H), device).to(wdt)
         out["sw3"] = (_normal(gen, (1, F, H), math.sqrt(s / H), device).to(wdt)
@@ -138,6 +144,8 @@ def make_inputs(shape: LayerShape, seed: int = 0, device: str = "cpu",
         u = u.clamp_(min=1e-300)
         gumbel = -torch.log(-torch.log(u))
         out["logit_add"] = (logp[None, :] + gumbel).to(torch.float32).contiguous()
+    if shape.random_second:
+        out["uniform"] = torch.rand((T,), generator=gen, device=device, dtype=torch.float32)
     return out
 
 

@@ -70,8 +70,12 @@ enum { MOE_ACT_RELU = 0, MOE_ACT_GELU = 1, MOE_ACT_SWIGLU = 2 };
 /* SOFTMAX_TOPK: gates are full-softmax probabilities of the selected experts
  * ([SWITCH] 2.1), optionally renormalised over the k selected.
  * TOPK_SOFTMAX: softmax over the k selected logits only ([EP] router section,
- * Megatron pre_softmax=False). */
-enum { MOE_SCORE_SOFTMAX_TOPK = 0, MOE_SCORE_TOPK_SOFTMAX = 1 };
+ * Megatron pre_softmax=False).
+ * SIGMOID_TOPK: gates are sigmoid(logit) of the selected experts ([EP] router
+ * section: sigmoid instead of softmax), optionally renormalised over the k
+ * selected; the aux loss's P_i then averages the sigmoids divided by their sum
+ * over the E experts.  Every score selects the k largest logits. */
+enum { MOE_SCORE_SOFTMAX_TOPK = 0, MOE_SCORE_TOPK_SOFTMAX = 1, MOE_SCORE_SIGMOID_TOPK = 2 };
 /* CAPACITY: C = ceil(T*k*cf/E) slots per expert, overflow dropped ([EP]
  * capacity and drop/pad sections; [DS7508]).  DROPLESS: every assignment kept
  * (MegaBlocks as summarised in [EP]). */
@@ -79,8 +83,15 @@ enum { MOE_CAP_CAPACITY = 0, MOE_CAP_DROPLESS = 1 };
 /* Element type of x, expert weights, dispatch buffers and y.  The router
  * weight, logits, gates and the aux loss are always fp32 ([SWITCH] 2.2). */
 enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
-/* moe_cfg.flags */
-enum { MOE_FLAG_KEEP_LOGITS = 1 };   /* moe_layer_fwd also stores fp32 logits in the workspace */
+/* moe_cfg.flags
+ * KEEP_LOGITS: moe_layer_fwd also stores fp32 logits in the workspace.
+ * RANDOM_SECOND: GShard top-2 ([EP] router section: the second expert receives
+ *   the token at random, according to its weight).  For k >= 2 the rank-1
+ *   choice of token t is dispatched iff uniform[t] < 2 * gate[t,1], with
+ *   uniform [T] fp32 in [0,1) supplied by the caller; otherwise its id becomes
+ *   -1 and its gate 0 (it takes no slot and adds nothing to y).  The aux loss
+ *   still counts it as selected.  No effect when k == 1. */
+enum { MOE_FLAG_KEEP_LOGITS = 1, MOE_FLAG_RANDOM_SECOND = 2 };
 
 /* Layer configuration.  Limits of this build: 1 <= E <= 1024, 1 <= k <= min(E,16),
  * H and F multiples of 8, n_shared in {0,1}, T >= 0 with T*k < 2^31 and every
@@ -103,6 +114,7 @@ typedef struct moe_cfg {
   int64_t min_capacity;  /* lower clamp of C (DeepSpeed min_capacity), 0 = none */
   float aux_alpha;       /* alpha of the load-balancing loss ([SWITCH] 2.1: 1e-2) */
   int32_t flags;         /* MOE_FLAG_* */
+  float z_coef;          /* router z-loss coefficient ([EP] aux-loss section), >= 0; 0 = no z-loss */
 } moe_cfg;
 
 /* Expert weights (device pointers, element type cfg->dtype).
@@ -125,7 +137,7 @@ typedef struct moe_ws_views {
   int32_t* ids;            /* [T,k] selected experts, rank order (largest logit first) */
   float* gates;            /* [T,k] gate of each selection */
   int32_t* slot;           /* [T,k] position in the expert's slots, -1 = dropped */
-  int32_t* expert_count;   /* [E] selections per expert before dropping */
+  int32_t* expert_count;   /* [E] dispatched choices per expert before the capacity drop */
   int32_t* kept_count;     /* [E] kept assignments per expert */
   int32_t* expert_offset;  /* [E+2] first row of each expert's block; [E] shared block; [E+1] end */
   int32_t* row_token;      /* [rows_max] source token of each row, -1 for padding rows */
@@ -159,19 +171,24 @@ MOE_API int moe_workspace_views(const moe_cfg* cfg, void* ws, moe_ws_views* view
 
 /* Router ([EP] router section; [SWITCH] 2.1, 2.2).
  *   x [T,H] (cfg->dtype), wg [E,H] fp32 (one row per expert), logit_add [T,E] fp32
- *   or NULL (an additive offset on the logits, e.g. for synthetic load skew).
+ *   or NULL (an additive offset on the logits, e.g. for synthetic load skew),
+ *   uniform [T] fp32 in [0,1): the random draws of MOE_FLAG_RANDOM_SECOND
+ *   (required with that flag and k >= 2, else ignored and may be NULL).
  *   logits[t,e] = sum_h x[t,h]*wg[e,h] (+ logit_add) accumulated in fp32;
- *   p = softmax(logits[t,:]); top-k on the logits (ties to the lower index);
- *   gates per cfg->score / cfg->renorm.
- * Writes ids [T,k] int32, gates [T,k] fp32, logits_out [T,E] fp32 if non-NULL,
- * and per-block sums of p and selection counts into `ws` for moe_aux_loss. */
+ *   p = softmax(logits[t,:]) (normalised sigmoids for SIGMOID_TOPK); top-k on
+ *   the logits (ties to the lower index); gates per cfg->score / cfg->renorm.
+ * Writes ids [T,k] int32 (-1: a second choice not dispatched), gates [T,k]
+ * fp32, logits_out [T,E] fp32 if non-NULL, and per-block sums of p, selection
+ * counts and, when cfg->z_coef != 0, squared log-sum-exps into `ws` for
+ * moe_aux_loss. */
 MOE_API int moe_route(const moe_cfg* cfg, const void* x, const float* wg, const float* logit_add,
-              int32_t* ids, float* gates, float* logits_out, void* ws, moe_stream_t stream);
+                      const float* uniform, int32_t* ids, float* gates, float* logits_out, void* ws,
+                      moe_stream_t stream);
 
 /* Same as moe_route after the logits: takes fp32 logits [T,E] (so routing can be
  * reproduced bit-exactly from given logits). */
-MOE_API int moe_route_from_logits(const moe_cfg* cfg, const float* logits, int32_t* ids, float* gates,
-                          void* ws, moe_stream_t stream);
+MOE_API int moe_route_from_logits(const moe_cfg* cfg, const float* logits, const float* uniform, int32_t* ids,
+                                  float* gates, void* ws, moe_stream_t stream);
 
 /* Slot assignment ([EP] drop/pad section, "position" policy; [DS7508] without
  * the [T,E,C] mask).  Assignments are ordered by (choice rank, token); an
@@ -180,7 +197,8 @@ MOE_API int moe_route_from_logits(const moe_cfg* cfg, const float* logits, int32
  * expert_count [E] (pre-drop), kept_count [E], expert_offset [E+2] (expert e owns
  * rows [off[e], off[e]+kept[e]) of a 128-row-padded block; the shared block
  * [off[E], off[E]+T) follows; off[E+1] = rows used), row_token [rows_max]
- * (-1 on padding rows).  ids entries outside [0,E) set MOE_EDEVICE. */
+ * (-1 on padding rows).  An id of -1 is a choice that is not dispatched: it
+ * takes no slot and gets slot -1.  Other ids outside [0,E) set MOE_EDEVICE. */
 MOE_API int moe_assign_slots(const moe_cfg* cfg, const int32_t* ids, int32_t* slot, int32_t* expert_count,
                      int32_t* kept_count, int32_t* expert_offset, int32_t* row_token, void* ws,
                      moe_stream_t stream);
@@ -233,13 +251,16 @@ MOE_API int moe_combine(const moe_cfg* cfg, const void* ybuf, const int32_t* ids
 
 /* Switch load-balancing loss ([SWITCH] 2.1; [EP] aux-loss section):
  * aux = alpha * E * sum_i f_i * P_i, f_i = pre-drop selections of i / (T*k),
- * P_i = mean_t p_i(t).  Reads the partials left in `ws` by the last moe_route /
- * moe_route_from_logits with the same cfg; writes one fp32 to `aux` (device). */
+ * P_i = mean_t p_i(t).  With cfg->z_coef != 0 also the router z-loss ([EP]
+ * aux-loss section): aux[1] = z_coef * mean_t logsumexp(logits[t,:])^2.
+ * Reads the partials left in `ws` by the last moe_route / moe_route_from_logits
+ * with the same cfg; writes aux[0] (and aux[1]) fp32 on the device. */
 MOE_API int moe_aux_loss(const moe_cfg* cfg, const void* ws, float* aux, moe_stream_t stream);
 
 /* The whole layer: route -> assign slots -> dispatch -> expert FFN -> combine,
- * plus the aux loss, on `stream`.  y [T,H] (cfg->dtype) and aux (one fp32) are
- * device outputs; expert_count [E] is optional (NULL to skip).  The
+ * plus the aux loss, on `stream`.  y [T,H] (cfg->dtype) and aux (one fp32, two
+ * with the z-loss: see moe_aux_loss) are device outputs; uniform is moe_route's;
+ * expert_count [E] (optional, NULL to skip) counts dispatched choices.  The
  * intermediates stay in `ws` (see moe_workspace_views).  `stage_events`, if
  * non-NULL, is an array of MOE_N_STAGE_EVENTS events recorded on `stream` before
  * the router and after each of: router, slots (which here also reduce the aux
@@ -248,8 +269,8 @@ MOE_API int moe_aux_loss(const moe_cfg* cfg, const void* ws, float* aux, moe_str
  * expert_count, if requested). */
 enum { MOE_N_STAGE_EVENTS = 8 };
 MOE_API int moe_layer_fwd(const moe_cfg* cfg, const void* x, const float* wg, const float* logit_add,
-                  const moe_weights* w, void* y, float* aux, int32_t* expert_count, void* ws,
-                  size_t ws_bytes, const moe_event_t* stage_events, moe_stream_t stream);
+                          const float* uniform, const moe_weights* w, void* y, float* aux, int32_t* expert_count,
+                          void* ws, size_t ws_bytes, const moe_event_t* stage_events, moe_stream_t stream);
 
 /* The activation exactly as the expert-FFN epilogues evaluate it, on n fp32
  * values (device pointers): out = relu(z) or gelu(z) = 0.5 z (1 + erf(z/sqrt 2))

@@ -102,9 +102,9 @@ def test_validation_errors(lib):
         B.moe_capacity(B.make_cfg(synth.DS_HIGHK, T=1 << 30))      # T*k beyond 2^31
     # null configuration and null outputs are rejected before any CUDA call
     assert lib.moe_capacity(None, None) == B.MOE_EINVAL
-    assert lib.moe_route(None, None, None, None, None, None, None, None, None) == B.MOE_EINVAL
+    assert lib.moe_route(None, None, None, None, None, None, None, None, None, None) == B.MOE_EINVAL
     cfg = B.make_cfg(synth.SWITCH_TINY_F32)
-    assert lib.moe_layer_fwd(ctypes.byref(cfg), None, None, None, None, None, None, None, None, 0, None, None) \
+    assert lib.moe_layer_fwd(ctypes.byref(cfg), None, None, None, None, None, None, None, None, None, 0, None, None) \
         == B.MOE_EINVAL
     w = B.moe_weights()
     assert lib.moe_expert_ffn(ctypes.byref(cfg), None, None, None, ctypes.byref(w), None, None, None) == B.MOE_EINVAL
@@ -116,3 +116,27 @@ def test_empty_batch_sizes(lib):
     cfg = B.make_cfg(synth.SWITCH_TOP1, T=0)
     assert B.moe_rows_max(cfg) == 0
     assert B.moe_workspace_size(cfg) > 0
+
+
+def test_router_variant_validation(lib):
+    """Sigmoid scores, the z-loss coefficient and the random-second flag are
+    validated on the host before any launch."""
+    g = synth.GSHARD_TOP2
+    assert B.moe_workspace_size(B.make_cfg(g.replace(score=synth.SCORE_SIGMOID_TOPK, z_coef=1e-3))) > 0
+    for kw in (dict(score=3), dict(z_coef=-1e-3), dict(z_coef=float("nan")), dict(z_coef=float("inf"))):
+        with pytest.raises(B.MoeError) as ei:
+            B.moe_workspace_size(B.make_cfg(g, **kw))
+        assert ei.value.code == B.MOE_EINVAL, kw
+    with pytest.raises(B.MoeError) as ei:
+        B.moe_workspace_size(B.make_cfg(g, flags=8))
+    assert ei.value.code == B.MOE_EINVAL
+    # the flag needs the draws (k >= 2, T > 0); dummy device pointers are never touched
+    cfg = B.make_cfg(g.replace(random_second=1))
+    assert cfg.flags & B.MOE_FLAG_RANDOM_SECOND
+    d = ctypes.c_void_p(256)
+    assert lib.moe_route(ctypes.byref(cfg), d, d, None, None, d, d, None, d, None) == B.MOE_EINVAL
+    assert lib.moe_route_from_logits(ctypes.byref(cfg), d, None, d, d, d, None) == B.MOE_EINVAL
+    # the z-loss partials add T/BT floats to the workspace, nothing that scales with E
+    a = B.moe_workspace_size(B.make_cfg(g))
+    b = B.moe_workspace_size(B.make_cfg(g, z_coef=1e-3))
+    assert a == b

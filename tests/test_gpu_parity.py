@@ -10,7 +10,7 @@ import oracle.moe_oracle as O
 from expert_dispatch_router_b200 import binding as B
 from expert_dispatch_router_b200 import build as build_mod
 from expert_dispatch_router_b200 import synth
-from tests.parity_utils import check_layer, run_layer, to64
+from tests.parity_utils import check_layer, condition_uniform, run_layer, to64
 
 pytestmark = pytest.mark.gpu
 
@@ -108,7 +108,7 @@ def test_route_from_logits_bitexact_with_ties():
             lg = torch.from_numpy(base).cuda()
             ids = torch.empty((T, k), dtype=torch.int32, device="cuda")
             gates = torch.empty((T, k), dtype=torch.float32, device="cuda")
-            B.moe_route_from_logits(cfg, lg, ids, gates, ws)
+            B.moe_route_from_logits(cfg, lg, None, ids, gates, ws)
             aux = torch.empty(1, device="cuda")
             B.moe_aux_loss(cfg, ws, aux)
             assert B.moe_sync_status(ws) == 0
@@ -190,7 +190,7 @@ def test_empty_batch_layer():
     ws = B.alloc_workspace(cfg)
     y = torch.empty((0, shape.H), dtype=torch.bfloat16, device="cuda")
     aux = torch.full((1,), float("nan"), device="cuda")
-    B.moe_layer_fwd(cfg, inp["x"], inp["wg"], inp["logit_add"], B.make_weights(inp), y, aux, None, ws)
+    B.moe_layer_fwd(cfg, inp["x"], inp["wg"], inp["logit_add"], None, B.make_weights(inp), y, aux, None, ws)
     assert B.moe_sync_status(ws) == 0
     assert aux.item() == 0.0
 
@@ -221,12 +221,18 @@ def test_deterministic_bitwise():
     b = run_layer(shape, inp)
     for n, v in snap.items():
         w = b[n] if n != "row_token" else b["row_token"][: int(b["expert_offset"][-1])]
-        assert torch.equal(v, w), n
+        assert torch.equal(v.contiguous().view(torch.uint8), w.contiguous().view(torch.uint8)), n   # bits, NaN too
 
 
-def test_stage_entry_points_match_layer():
+@pytest.mark.parametrize("variant", ["plain", "zloss_random_second", "sigmoid_zloss"])
+def test_stage_entry_points_match_layer(variant):
     shape = SMALL["gshard_top2"].replace(n_shared=1)
+    if variant == "zloss_random_second":
+        shape = shape.replace(z_coef=1e-3, random_second=1)
+    elif variant == "sigmoid_zloss":
+        shape = shape.replace(z_coef=1e-3, score=synth.SCORE_SIGMOID_TOPK)
     inp = synth.make_inputs(shape, seed=7, device="cuda")
+    condition_uniform(shape, inp)
     full = run_layer(shape, inp)
     cfg = B.make_cfg(shape)
     ws = B.alloc_workspace(cfg)
@@ -244,8 +250,8 @@ def test_stage_entry_points_match_layer():
     xbuf = torch.empty((R, H), dtype=torch.bfloat16, device=dev)
     ybuf = torch.empty((R, H), dtype=torch.bfloat16, device=dev)
     y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
-    aux = torch.empty(1, device=dev)
-    B.moe_route(cfg, inp["x"], inp["wg"], None, ids, gates, logits, ws)
+    aux = torch.full((2,), float("nan"), device=dev)
+    B.moe_route(cfg, inp["x"], inp["wg"], None, inp["uniform"], ids, gates, logits, ws)
     B.moe_assign_slots(cfg, ids, slot, cnt, kept, off, rt, ws)
     B.moe_dispatch(cfg, inp["x"], ids, slot, off, xbuf)
     B.moe_expert_ffn(cfg, xbuf, inp["x"], off, B.make_weights(inp), ybuf, ws)
@@ -253,8 +259,14 @@ def test_stage_entry_points_match_layer():
     B.moe_aux_loss(cfg, ws, aux)
     assert B.moe_sync_status(ws) == 0
     assert torch.equal(logits, full["logits"])
-    for n, v in dict(ids=ids, gates=gates, slot=slot, expert_offset=off, y=y, aux=aux).items():
+    for n, v in dict(ids=ids, gates=gates, slot=slot, expert_offset=off, y=y).items():
         assert torch.equal(v, full[n]), n
+    # the standalone aux kernel and the slot-fused reduction sum in different orders
+    torch.testing.assert_close(aux[0], full["aux"][0], rtol=1e-6, atol=0)
+    if shape.z_coef:
+        torch.testing.assert_close(aux[1], full["aux"][1], rtol=1e-6, atol=0)
+    else:
+        assert torch.isnan(aux[1]) and torch.isnan(full["aux"][1])
     used = int(off[-1])
     assert torch.equal(rt[:used], full["row_token"][:used])
     assert torch.equal(ybuf[:used][rt[:used] >= 0], full["ybuf"][:used][full["row_token"][:used] >= 0])
