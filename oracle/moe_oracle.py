@@ -39,6 +39,11 @@ notes):
   * top-k ties: larger logit first, equal logits go to the lower expert index.
   * gates are fixed before capacity; a dropped choice contributes zero and the
     kept gates are not renormalised again.
+  * "probs" drop policy ([EP] drop/pad section names it: drop the lowest
+    probability): the probability is the assignment's gate, compared in float32
+    (the precision gates are stored in); equal gates keep the earlier
+    assignment in (rank, token) order; kept assignments take slots in that
+    order, so equal gates reduce it to the "position" policy.
   * f_i counts pre-drop selections over T*k; P_i is the mean full softmax.
   * sigmoid scores ([EP] router section names sigmoid as the alternative to
     softmax and says nothing more): top-k on the logits as for softmax (the
@@ -71,6 +76,7 @@ import numpy as np
 ACT_RELU, ACT_GELU, ACT_SWIGLU = 0, 1, 2
 SCORE_SOFTMAX_TOPK, SCORE_TOPK_SOFTMAX, SCORE_SIGMOID_TOPK = 0, 1, 2
 CAP_CAPACITY, CAP_DROPLESS = 0, 1
+DROP_POSITION, DROP_PROBS = 0, 1
 ROW_PAD = 128
 
 
@@ -93,6 +99,7 @@ class OracleLayer:
     aux_alpha: float = 1e-2
     z_coef: float = 0.0          # router z-loss coefficient, 0 = off
     random_second: int = 0       # GShard: dispatch the second choice at random
+    drop_policy: int = DROP_POSITION
 
     @classmethod
     def from_mapping(cls, m) -> "OracleLayer":
@@ -243,6 +250,39 @@ def assign_slots(ids: np.ndarray, E: int, C: Optional[int]):
     return slot, count.astype(np.int32), kept.astype(np.int32)
 
 
+def assign_slots_probs(ids: np.ndarray, gates: np.ndarray, E: int, C: Optional[int]):
+    """The 'probs' drop policy ([EP] drop/pad section: Megatron-Core's
+    moe_token_drop_policy="probs" drops the lowest-probability assignments).
+    Each expert keeps the C of its assignments with the largest gate; among
+    equal gates the one earlier in (choice rank, token) order is kept.  Kept
+    assignments take slots 0.. in (choice rank, token) order.  Ids of -1 take no
+    slot.  Same returns as assign_slots."""
+    T, k = ids.shape
+    per = [[] for _ in range(E)]               # (t, r) of each assignment, arrival order
+    for r in range(k):
+        for t in range(T):
+            e = int(ids[t, r])
+            if e >= 0:
+                per[e].append((t, r))
+    slot = np.full((T, k), -1, dtype=np.int32)
+    g = np.asarray(gates, dtype=np.float64)
+    for e in range(E):
+        lst = per[e]
+        if C is None or len(lst) <= C:
+            keep = set(range(len(lst)))
+        else:
+            order = sorted(range(len(lst)), key=lambda i: (-g[lst[i]], i))
+            keep = set(order[:C])
+        j = 0
+        for i, (t, r) in enumerate(lst):
+            if i in keep:
+                slot[t, r] = j
+                j += 1
+    count = np.array([len(p) for p in per], dtype=np.int64)
+    kept = count.copy() if C is None else np.minimum(count, C)
+    return slot, count.astype(np.int32), kept.astype(np.int32)
+
+
 def round_up(n: int, m: int = ROW_PAD) -> int:
     return -(-int(n) // m) * m
 
@@ -363,7 +403,11 @@ def layer_forward(layer: OracleLayer, x, wg, w1, w2, w3=None, sw1=None, sw2=None
     logits = np.asarray(logits, dtype=np.float32)
     probs, selected, ids, gates = route_and_dispatch(layer, logits, uniform)
     C = layer_capacity(layer)
-    slot, count, kept = assign_slots(ids, E, C)
+    if layer.drop_policy == DROP_PROBS:
+        # the decision compares gates in float32, the precision they are stored in
+        slot, count, kept = assign_slots_probs(ids, gates.astype(np.float32), E, C)
+    else:
+        slot, count, kept = assign_slots(ids, E, C)
     off = row_layout(kept, T, layer.n_shared)
     rt = row_tokens(ids, slot, off, layer.n_shared)
     aux = aux_loss(probs, selected, E, layer.aux_alpha)

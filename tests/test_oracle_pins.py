@@ -509,3 +509,56 @@ def test_layer_random_second_counts_selections_and_drops_rows():
         h = np.maximum(w1[e] @ x[t], 0)
         np.testing.assert_allclose(drop_all["y"][t], ref["gates"][t, 0] * (w2[e] @ h), rtol=1e-12, atol=1e-13)
     assert drop_all["zloss"] == O.z_loss(drop_all["logits"], 1e-2)
+
+
+# ------------------------------------------------------------ "probs" drop policy
+def test_probs_policy_equal_gates_is_position_policy():
+    E, k, T = 3, 2, 4
+    pats = list(itertools.permutations(range(E), k))
+    for combo in itertools.product(pats, repeat=T):
+        ids = np.array(combo, dtype=np.int32)
+        g = np.full((T, k), 0.25)
+        for C in (1, 2, 3, None):
+            a = O.assign_slots_probs(ids, g, E, C)
+            b = O.assign_slots(ids, E, C)
+            for u, v in zip(a, b):
+                np.testing.assert_array_equal(u, v)
+
+
+def test_probs_policy_keeps_the_best_subset_bruteforce():
+    """With distinct gates the kept set of each expert is the unique size-C
+    subset of largest gate sum; slots follow (rank, token) order."""
+    rng = np.random.default_rng(41)
+    E, k, T = 3, 2, 5
+    for _ in range(300):
+        ids = np.argsort(rng.random((T, E)), axis=1)[:, :k].astype(np.int32)
+        if rng.random() < 0.3:
+            ids[rng.random(T) < 0.5, 1] = -1
+        g = rng.permutation(T * k).reshape(T, k) / (T * k) + 0.01
+        for C in (1, 2, 3):
+            slot, count, kept = O.assign_slots_probs(ids, g, E, C)
+            for e in range(E):
+                arr = [(t, r) for r in range(k) for t in range(T) if ids[t, r] == e]
+                assert count[e] == len(arr) and kept[e] == min(len(arr), C)
+                best = max(itertools.combinations(range(len(arr)), min(C, len(arr))),
+                           key=lambda s: sum(g[arr[i]] for i in s))
+                got = [i for i, (t, r) in enumerate(arr) if slot[t, r] >= 0]
+                assert sorted(got) == sorted(best)
+                assert [slot[arr[i]] for i in got] == list(range(len(got)))
+            assert (slot[ids < 0] == -1).all()
+    # planted slip: dropping the highest gates instead fails the subset check
+    ids = np.array([[0, 1], [0, 1], [0, 1]], np.int32)
+    g = np.array([[0.9, 0.1], [0.5, 0.5], [0.2, 0.8]])
+    slot, _, _ = O.assign_slots_probs(ids, g, 2, 1)
+    assert list(slot[:, 0]) == [0, -1, -1] and list(slot[:, 1]) == [-1, -1, 0]
+
+
+def test_probs_policy_ties_keep_earlier_arrivals():
+    ids = np.array([[0, 1], [0, 1], [0, 1], [1, 0]], np.int32)
+    g = np.array([[0.5, 0.3], [0.5, 0.3], [0.7, 0.3], [0.3, 0.5]])
+    slot, count, kept = O.assign_slots_probs(ids, g, 2, 2)
+    # expert 0: arrivals (t0,r0)=.5 (t1,r0)=.5 (t2,r0)=.7 (t3,r1)=.5 -> keep t2 and t0
+    assert [slot[0, 0], slot[1, 0], slot[2, 0], slot[3, 1]] == [0, -1, 1, -1]
+    # expert 1: arrivals (t3,r0)=.3 (t0,r1)=.3 (t1,r1)=.3 (t2,r1)=.3 -> first two arrivals
+    assert [slot[3, 0], slot[0, 1], slot[1, 1], slot[2, 1]] == [0, 1, -1, -1]
+    assert list(count) == [4, 4] and list(kept) == [2, 2]
