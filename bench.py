@@ -111,7 +111,8 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 100 ms in the background."""
+    """SM clocks and throttle reasons sampled in the background: through NVML
+    every 2 ms (read-only queries), else nvidia-smi every 100 ms."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
@@ -120,12 +121,41 @@ class ClockSampler:
     def __init__(self, device_index: int):
         import torch
         self.samples = []
-        self.marks = []
+        self.proc = None
+        self._stop = threading.Event()
         try:
             pr = torch.cuda.get_device_properties(device_index)
             sel = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
         except Exception:
             sel = str(device_index)
+        try:
+            import pynvml as N
+            N.nvmlInit()
+            h = N.nvmlDeviceGetHandleByPciBusId(sel) if ":" in sel else N.nvmlDeviceGetHandleByIndex(device_index)
+            mx = N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM)
+            bits = (N.nvmlClocksEventReasonHwSlowdown, N.nvmlClocksEventReasonHwThermalSlowdown,
+                    N.nvmlClocksEventReasonSwThermalSlowdown, N.nvmlClocksEventReasonSwPowerCap)
+
+            def poll():
+                while not self._stop.is_set():
+                    try:
+                        sm = N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM)
+                        r = N.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    except Exception:
+                        break
+                    flags = ",".join("Active" if r & b else "Not Active" for b in bits)
+                    self.samples.append((time.time(), f"{sm}, {mx}, 0, {flags}"))
+                    time.sleep(0.002)
+                try:
+                    N.nvmlShutdown()
+                except Exception:
+                    pass
+
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            pass
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", sel, f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "100"],
@@ -142,16 +172,19 @@ class ClockSampler:
 
     def wait_first(self, timeout=5.0):
         t0 = time.time()
-        while self.proc is not None and not self.samples and time.time() - t0 < timeout:
+        while not self.samples and time.time() - t0 < timeout:
             time.sleep(0.02)
 
     def stop(self):
+        self._stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
+        elif getattr(self, "thread", None) is not None:
+            self.thread.join(timeout=2)
 
     def summary(self, t0, t1):
         rows = [s for (t, s) in self.samples if t0 <= t <= t1] or [s for (_, s) in self.samples]

@@ -36,7 +36,7 @@ class moe_cfg(ctypes.Structure):
                 ("score", ctypes.c_int32), ("renorm", ctypes.c_int32), ("cap_mode", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("cf_num", ctypes.c_int64), ("cf_den", ctypes.c_int64),
                 ("min_capacity", ctypes.c_int64), ("aux_alpha", ctypes.c_float), ("flags", ctypes.c_int32),
-                ("z_coef", ctypes.c_float)]
+                ("z_coef", ctypes.c_float), ("drop_policy", ctypes.c_int32)]
 
 
 class moe_weights(ctypes.Structure):
@@ -61,7 +61,7 @@ _SIGS = {
     "moe_workspace_views": [CFGP, P, ctypes.POINTER(moe_ws_views)],
     "moe_route": [CFGP, P, P, P, P, P, P, P, P, P],
     "moe_route_from_logits": [CFGP, P, P, P, P, P, P],
-    "moe_assign_slots": [CFGP, P, P, P, P, P, P, P, P],
+    "moe_assign_slots": [CFGP, P, P, P, P, P, P, P, P, P],
     "moe_assign_slots_static": [CFGP, P, P, P, P, P, P, P],
     "moe_dispatch": [CFGP, P, P, P, P, P, P],
     "moe_expert_ffn": [CFGP, P, P, P, ctypes.POINTER(moe_weights), P, P, P],
@@ -122,7 +122,8 @@ def make_cfg(shape: synth.LayerShape, flags: int = 0, **override) -> moe_cfg:
     return moe_cfg(T=s.T, H=s.H, F=s.F, E=s.E, k=s.k, n_shared=s.n_shared, act=s.act, score=s.score,
                    renorm=s.renorm, cap_mode=s.cap_mode, dtype=s.dtype, cf_num=s.cf_num, cf_den=s.cf_den,
                    min_capacity=s.min_capacity, aux_alpha=s.aux_alpha,
-                   flags=flags | (MOE_FLAG_RANDOM_SECOND if s.random_second else 0), z_coef=s.z_coef)
+                   flags=flags | (MOE_FLAG_RANDOM_SECOND if s.random_second else 0), z_coef=s.z_coef,
+                   drop_policy=s.drop_policy)
 
 
 def make_weights(inp: dict) -> moe_weights:
@@ -165,10 +166,10 @@ def moe_route_from_logits(cfg, logits, uniform, ids, gates, ws, stream=None):
                                         _ptr(ws), _stream(stream)), "moe_route_from_logits")
 
 
-def moe_assign_slots(cfg, ids, slot, expert_count, kept_count, expert_offset, row_token, ws, stream=None):
-    _check(load().moe_assign_slots(ctypes.byref(cfg), _ptr(ids), _ptr(slot), _ptr(expert_count), _ptr(kept_count),
-                                   _ptr(expert_offset), _ptr(row_token), _ptr(ws), _stream(stream)),
-           "moe_assign_slots")
+def moe_assign_slots(cfg, ids, gates, slot, expert_count, kept_count, expert_offset, row_token, ws, stream=None):
+    _check(load().moe_assign_slots(ctypes.byref(cfg), _ptr(ids), _ptr(gates), _ptr(slot), _ptr(expert_count),
+                                   _ptr(kept_count), _ptr(expert_offset), _ptr(row_token), _ptr(ws),
+                                   _stream(stream)), "moe_assign_slots")
 
 
 def moe_assign_slots_static(cfg, ids, slot, expert_count, kept_count, expert_offset, row_token, stream=None):

@@ -36,6 +36,16 @@ template <> struct Elem<__nv_bfloat16> {
   static __device__ __forceinline__ __nv_bfloat16 from_f(float v) { return __float2bfloat16_rn(v); }
 };
 
+// Order-preserving map from fp32 to uint32 (a > b as floats <=> key(a) > key(b)
+// as integers); -0 is mapped like +0 so equal values get equal keys.
+__device__ __forceinline__ uint32_t to_ordered(float v) {
+  const uint32_t b = __float_as_uint(v == 0.0f ? 0.0f : v);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float from_ordered(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
 // 16-byte vector helpers.
 __device__ __forceinline__ int4 ld_nc_v4(const void* p) {
   int4 v;

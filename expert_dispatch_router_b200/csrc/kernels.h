@@ -64,6 +64,13 @@ struct SlotParams {
   float aux_alpha;
   const float* zsum_part;   // [nblk_router] router sums of lse^2, or null: no z-loss
   float z_coef;
+  // "probs" drop policy (capacity mode only): experts with more assignments than
+  // C keep the C largest gates.  Their assignments are listed in arrival order at
+  // list_*[cum[e] .. cum[e] + count[e]) and resolved by a per-expert select.
+  const float* gates;       // [T,k] or null: "position" policy
+  int32_t* cum;             // [E] exclusive prefix of expert_count
+  uint32_t* list_key;       // [T*k] order-preserving gate keys
+  uint32_t* list_idx;       // [T*k] assignment index r*T + t
 };
 constexpr int kSlotChunk = 256;    // assignments per CTA of the slot kernels (one per thread)
 cudaError_t launch_slots(const SlotParams& p, cudaStream_t stream);

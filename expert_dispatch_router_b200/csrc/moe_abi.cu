@@ -15,7 +15,7 @@ namespace {
 constexpr int64_t kMaxCf = int64_t(1) << 20;
 
 struct Layout {
-  size_t status, psum, cnt, zsum, term, chunk, ids, gates, slot, ecount, kept, off, rowtok, logits, lparts, planes, xbuf,
+  size_t status, psum, cnt, zsum, term, chunk, cum, lkey, lidx, ids, gates, slot, ecount, kept, off, rowtok, logits, lparts, planes, xbuf,
       hbuf, ybuf;
   size_t total;
   int nblk_router, nchunk;
@@ -36,6 +36,7 @@ bool valid_cfg(const moe_cfg* c) {
   if (c->min_capacity < 0) return false;
   if (!(c->z_coef >= 0.0f) || isinf(c->z_coef)) return false;
   if (c->flags & ~(MOE_FLAG_KEEP_LOGITS | MOE_FLAG_RANDOM_SECOND)) return false;
+  if (c->drop_policy != MOE_DROP_POSITION && c->drop_policy != MOE_DROP_PROBS) return false;
   return true;
 }
 
@@ -74,6 +75,8 @@ int64_t rows_max_of(const moe_cfg* c) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+bool drop_probs(const moe_cfg* c) { return c->cap_mode == MOE_CAP_CAPACITY && c->drop_policy == MOE_DROP_PROBS; }
+
 Layout layout_of(const moe_cfg* c) {
   Layout L{};
   const size_t T = (size_t)c->T, E = (size_t)c->E, k = (size_t)c->k;
@@ -90,6 +93,10 @@ Layout layout_of(const moe_cfg* c) {
   L.zsum = take(sizeof(float) * L.nblk_router);
   L.term = take(sizeof(double) * (E + 1));      // E terms + the aux ticket counter
   L.chunk = take(sizeof(int32_t) * E * (size_t)L.nchunk);
+  const bool probs = drop_probs(c);
+  L.cum = take(probs ? sizeof(int32_t) * E : 0);
+  L.lkey = take(probs ? sizeof(uint32_t) * T * k : 0);
+  L.lidx = take(probs ? sizeof(uint32_t) * T * k : 0);
   L.ids = take(sizeof(int32_t) * T * k);
   L.gates = take(sizeof(float) * T * k);
   L.slot = take(sizeof(int32_t) * T * k);
@@ -160,9 +167,17 @@ int run_route(const moe_cfg* c, const Layout& L, const void* x, const float* wg,
   return cuda_status(launch_router(p, c->dtype == MOE_DTYPE_BF16, s));
 }
 
-int run_slots(const moe_cfg* c, const Layout& L, const int32_t* ids, int32_t* slot, int32_t* ecount, int32_t* kept,
-              int32_t* off, int32_t* rowtok, void* ws, cudaStream_t s, float* aux = nullptr) {
+int run_slots(const moe_cfg* c, const Layout& L, const int32_t* ids, const float* gates, int32_t* slot,
+              int32_t* ecount, int32_t* kept, int32_t* off, int32_t* rowtok, void* ws, cudaStream_t s,
+              float* aux = nullptr) {
   SlotParams p{};
+  if (drop_probs(c)) {
+    if (c->T > 0 && gates == nullptr) return MOE_EINVAL;
+    p.gates = gates;
+    p.cum = at<int32_t>(ws, L.cum);
+    p.list_key = at<uint32_t>(ws, L.lkey);
+    p.list_idx = at<uint32_t>(ws, L.lidx);
+  }
   p.ids = ids;
   p.slot = slot;
   p.expert_count = ecount;
@@ -359,14 +374,15 @@ int moe_route_from_logits(const moe_cfg* cfg, const float* logits, const float* 
                    S(stream));
 }
 
-int moe_assign_slots(const moe_cfg* cfg, const int32_t* ids, int32_t* slot, int32_t* expert_count,
-                     int32_t* kept_count, int32_t* expert_offset, int32_t* row_token, void* ws,
+int moe_assign_slots(const moe_cfg* cfg, const int32_t* ids, const float* gates, int32_t* slot,
+                     int32_t* expert_count, int32_t* kept_count, int32_t* expert_offset, int32_t* row_token, void* ws,
                      moe_stream_t stream) {
   const int st = check_cfg(cfg);
   if (st != MOE_OK) return st;
   if (ws == nullptr || expert_count == nullptr || kept_count == nullptr || expert_offset == nullptr) return MOE_EINVAL;
   if (cfg->T > 0 && (ids == nullptr || slot == nullptr || row_token == nullptr)) return MOE_EINVAL;
-  return run_slots(cfg, layout_of(cfg), ids, slot, expert_count, kept_count, expert_offset, row_token, ws, S(stream));
+  return run_slots(cfg, layout_of(cfg), ids, gates, slot, expert_count, kept_count, expert_offset, row_token, ws,
+                   S(stream));
 }
 
 int moe_dispatch(const moe_cfg* cfg, const void* x, const int32_t* ids, const int32_t* slot,
@@ -447,7 +463,7 @@ int moe_layer_fwd(const moe_cfg* cfg, const void* x, const float* wg, const floa
   if ((st = record(stage_events, 0, s)) != MOE_OK) return st;
   if ((st = run_route(cfg, L, x, wg, logit_add, nullptr, uniform, ids, gates, logits, ws, s)) != MOE_OK) return st;
   if ((st = record(stage_events, 1, s)) != MOE_OK) return st;
-  if ((st = run_slots(cfg, L, ids, slot, at<int32_t>(ws, L.ecount), at<int32_t>(ws, L.kept), off,
+  if ((st = run_slots(cfg, L, ids, gates, slot, at<int32_t>(ws, L.ecount), at<int32_t>(ws, L.kept), off,
                       at<int32_t>(ws, L.rowtok), ws, s, aux)) != MOE_OK)
     return st;
   if ((st = record(stage_events, 2, s)) != MOE_OK) return st;

@@ -36,16 +36,8 @@ __device__ __forceinline__ int lane_expert(int lane, int j) {
   else return 4 * lane + 128 * (j >> 2) + (j & 3);
 }
 
-// Order-preserving map from fp32 to uint32 (a > b as floats <=> key(a) > key(b)
-// as integers); -0 is mapped like +0 so equal logits get equal keys.  Top-k
-// order: larger logit first, equal logits -> smaller expert index.
-__device__ __forceinline__ uint32_t to_ordered(float v) {
-  const uint32_t b = __float_as_uint(v == 0.0f ? 0.0f : v);
-  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
-__device__ __forceinline__ float from_ordered(uint32_t k) {
-  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
-}
+// Top-k order: larger logit first (order-preserving keys, to_ordered), equal
+// logits -> smaller expert index.
 
 // Scores, top-k and gates of token t from its E values spread over the warp's
 // lanes (val[j] belongs to expert lane_expert(lane, j)), adding the logit offset

@@ -18,6 +18,13 @@
 //                32-assignment step with match_any, carry per-warp running counts,
 //                prefix them over the warps in order, and add the chunk base.
 // Total metadata traffic is O(T*k + E*chunks); nothing scales with C.
+//
+// "probs" policy (same section: drop the lowest-probability assignments): the
+// rank kernel lists every assignment of an over-full expert, in arrival order,
+// as (order-preserving gate key, assignment index); one CTA per such expert
+// then finds the C-th largest key with a 4 x 8-bit radix select and makes one
+// ordered pass that keeps the keys above it plus the earliest arrivals equal to
+// it, numbering the kept ones in arrival order.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -51,9 +58,12 @@ __global__ void __launch_bounds__(kSlotThreads) slot_count_kernel(SlotParams p, 
     p.chunk_cnt[(int64_t)e * nchunk + blockIdx.x] = hist[e];
 }
 
-// Exclusive block scan of 256 ints; returns the block total.
-__device__ __forceinline__ int block_exclusive_scan(int v, int* sh, int& excl) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+// Exclusive scan of one int per thread over a block of NW warps: returns the
+// thread's exclusive prefix and sets `total`.  `sh` holds NW ints; the trailing
+// barrier lets the caller reuse it at once.
+template <int NW>
+__device__ __forceinline__ int block_scan_excl(int v, int* sh, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -63,20 +73,19 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* sh, int& excl) {
   if (lane == 31) sh[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    int w = lane < kSlotWarps ? sh[lane] : 0;
+    int w = lane < NW ? sh[lane] : 0;
 #pragma unroll
-    for (int o = 1; o < kSlotWarps; o <<= 1) {
+    for (int o = 1; o < NW; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, w, o);
       if (lane >= o) w += y;
     }
-    if (lane < kSlotWarps) sh[lane] = w;     // inclusive warp totals
+    if (lane < NW) sh[lane] = w;             // inclusive warp totals
   }
   __syncthreads();
-  const int before = warp == 0 ? 0 : sh[warp - 1];
-  const int total = sh[kSlotWarps - 1];
-  excl = before + x - v;
+  const int excl = (warp == 0 ? 0 : sh[warp - 1]) + x - v;
+  total = sh[NW - 1];
   __syncthreads();
-  return total;
+  return excl;
 }
 
 __global__ void __launch_bounds__(kSlotThreads) slot_scan_kernel(SlotParams p, int nchunk) {
@@ -87,8 +96,8 @@ __global__ void __launch_bounds__(kSlotThreads) slot_scan_kernel(SlotParams p, i
   for (int base = 0; base < nchunk; base += kSlotThreads) {
     const int c = base + threadIdx.x;
     const int v = c < nchunk ? row[c] : 0;
-    int excl;
-    const int tot = block_exclusive_scan(v, sh, excl);
+    int tot;
+    const int excl = block_scan_excl<kSlotWarps>(v, sh, tot);
     if (c < nchunk) row[c] = running + excl;        // chunk base, in place
     running += tot;
   }
@@ -131,29 +140,16 @@ __global__ void __launch_bounds__(1024) slot_offsets_kernel(SlotParams p) {
   __shared__ int sh_off[kMaxE + 2];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int kept = tid < p.E ? p.kept_count[tid] : 0;
-  const int v = (int)round_up(kept, kRowPad);
-  int x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) sh[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    int w = sh[lane];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += y;
-    }
-    sh[lane] = w;
-  }
-  __syncthreads();
-  const int excl = (warp == 0 ? 0 : sh[warp - 1]) + x - v;
+  int routed;
+  const int excl = block_scan_excl<32>((int)round_up(kept, kRowPad), sh, routed);
   if (tid < p.E) sh_off[tid] = excl;
+  if (p.gates != nullptr) {
+    // "probs" policy: where each expert's arrival-ordered list starts
+    int total;
+    const int c = block_scan_excl<32>(tid < p.E ? p.expert_count[tid] : 0, sh, total);
+    if (tid < p.E) p.cum[tid] = c;
+  }
   if (tid == 0) {
-    const int routed = sh[31];
     sh_off[p.E] = routed;
     const int64_t end = routed + (p.n_shared ? round_up(p.T, kRowPad) : 0);
     sh_off[p.E + 1] = (int)end;
@@ -239,10 +235,102 @@ __global__ void __launch_bounds__(kSlotThreads) slot_rank_kernel(SlotParams p, i
     const int64_t r = a / p.T, t = a - r * p.T;
     if (e < 0) { p.slot[t * p.k + r] = -1; continue; }
     const int pos = p.chunk_cnt[(int64_t)e * nchunk + blockIdx.x] + wcnt[warp * p.E + e] + local[s];
+    if (p.gates != nullptr && p.expert_count[e] > p.capacity) {
+      // over-full expert under the "probs" policy: list it for the select kernel
+      const int64_t li = (int64_t)p.cum[e] + pos;
+      p.list_key[li] = to_ordered(p.gates[t * p.k + r]);
+      p.list_idx[li] = (uint32_t)a;
+      continue;
+    }
     const bool kept = p.capacity < 0 || pos < p.capacity;
     p.slot[t * p.k + r] = kept ? pos : -1;
     const int64_t row = (int64_t)p.expert_offset[e] + pos;
     if (kept && row < p.rows_max) p.row_token[row] = (int)t;
+  }
+}
+
+// One CTA per expert; only experts with more than C assignments do work.
+constexpr int kSelThreads = 1024;
+constexpr int kSelWarps = kSelThreads / 32;
+
+__global__ void __launch_bounds__(kSelThreads) slot_select_kernel(SlotParams p) {
+  __shared__ int hist[256];
+  __shared__ int sh[kSelWarps];
+  __shared__ uint32_t s_prefix;
+  __shared__ int s_need;
+  const int e = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int n = p.expert_count[e];
+  if ((int64_t)n <= p.capacity) return;
+  const int64_t base = p.cum[e];
+  const uint32_t* key = p.list_key + base;
+  const uint32_t* idx = p.list_idx + base;
+
+  // radix select: after the four 8-bit passes, `prefix` is the C-th largest key
+  // and `need` is how many of the keys equal to it are kept (the earliest ones)
+  uint32_t prefix = 0u, mask = 0u;
+  int need = (int)p.capacity;
+  if (need <= 0) prefix = 0xffffffffu;         // nothing is kept (C = 0 cannot arise with T*k > 0)
+  for (int shift = 24; shift >= 0 && need > 0; shift -= 8) {
+    for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < n; i += kSelThreads) {
+      const uint32_t kv = key[i];
+      if ((kv & mask) == prefix) atomicAdd(&hist[(kv >> shift) & 255u], 1);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // lane l holds bins 255-8l .. 248-8l (descending); find where the count from
+      // the top reaches `need`
+      int loc[8], s = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) { loc[j] = hist[255 - (8 * lane + j)]; s += loc[j]; }
+      int incl = s;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const int excl = incl - s;
+      if (excl < need && need <= incl) {
+        int run = excl;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (run < need && need <= run + loc[j]) {
+            s_prefix = prefix | ((uint32_t)(255 - (8 * lane + j)) << shift);
+            s_need = need - run;
+          }
+          run += loc[j];
+        }
+      }
+    }
+    __syncthreads();
+    prefix = s_prefix;
+    need = s_need;
+    mask |= 255u << shift;
+    __syncthreads();
+  }
+
+  // ordered pass: keep keys above the threshold and the first `need` equal ones
+  const int64_t off = p.expert_offset[e];
+  int run_eq = 0, run_keep = 0;
+  for (int b0 = 0; b0 < n; b0 += kSelThreads) {
+    const int i = b0 + tid;
+    const bool valid = i < n;
+    const uint32_t kv = valid ? key[i] : 0u;
+    const int eq = valid && kv == prefix;
+    int tot_eq;
+    const int eq_rank = run_eq + block_scan_excl<kSelWarps>(eq, sh, tot_eq);
+    const int keep = valid && (kv > prefix || (eq && eq_rank < need));
+    int tot_keep;
+    const int rank = run_keep + block_scan_excl<kSelWarps>(keep, sh, tot_keep);
+    if (valid) {
+      const uint32_t a = idx[i];
+      const int64_t r = (int64_t)a / p.T, t = (int64_t)a - r * p.T;
+      p.slot[t * p.k + r] = keep ? rank : -1;
+      if (keep && off + rank < p.rows_max) p.row_token[off + rank] = (int)t;
+    }
+    run_eq += tot_eq;
+    run_keep += tot_keep;
   }
 }
 
@@ -262,6 +350,7 @@ cudaError_t launch_slots(const SlotParams& p, cudaStream_t stream) {
     cudaError_t e = ensure_smem(slot_rank_kernel, sm);
     if (e != cudaSuccess) return e;
     slot_rank_kernel<<<nchunk, kSlotThreads, sm, stream>>>(p, nchunk);
+    if (p.gates != nullptr) slot_select_kernel<<<p.E, kSelThreads, 0, stream>>>(p);
   }
   return cudaGetLastError();
 }

@@ -62,6 +62,7 @@ extern "C" int moe_assign_slots_static(const moe_cfg* cfg, const int32_t* ids, i
   if (st != MOE_OK) return st;
   if (expert_count == nullptr || kept_count == nullptr || expert_offset == nullptr) return MOE_EINVAL;
   if (cfg->T > 0 && (ids == nullptr || slot == nullptr || row_token == nullptr)) return MOE_EINVAL;
+  if (cfg->cap_mode == MOE_CAP_CAPACITY && cfg->drop_policy == MOE_DROP_PROBS) return MOE_EUNSUPPORTED;
   const int64_t nchunk = (cfg->T * cfg->k + kSlotChunk - 1) / kSlotChunk;
   if ((int64_t)cfg->E * nchunk > kStaticChunkInts) return MOE_EUNSUPPORTED;   // beyond the fixed scratch
   int err = MOE_OK;

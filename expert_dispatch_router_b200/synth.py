@@ -42,6 +42,7 @@ import torch
 ACT_RELU, ACT_GELU, ACT_SWIGLU = 0, 1, 2
 SCORE_SOFTMAX_TOPK, SCORE_TOPK_SOFTMAX, SCORE_SIGMOID_TOPK = 0, 1, 2
 CAP_CAPACITY, CAP_DROPLESS = 0, 1
+DROP_POSITION, DROP_PROBS = 0, 1
 DTYPE_F32, DTYPE_BF16 = 0, 1
 
 
@@ -68,6 +69,7 @@ class LayerShape:
     zipf_skew: float = 0.0        # >0: Gumbel/Zipf logit offset exponent
     z_coef: float = 0.0           # router z-loss coefficient (0 = off)
     random_second: int = 0        # GShard random dispatch of the second choice
+    drop_policy: int = DROP_POSITION
 
     def replace(self, **kw) -> "LayerShape":
         return dataclasses.replace(self, **kw)

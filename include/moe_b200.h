@@ -80,6 +80,12 @@ enum { MOE_SCORE_SOFTMAX_TOPK = 0, MOE_SCORE_TOPK_SOFTMAX = 1, MOE_SCORE_SIGMOID
  * capacity and drop/pad sections; [DS7508]).  DROPLESS: every assignment kept
  * (MegaBlocks as summarised in [EP]). */
 enum { MOE_CAP_CAPACITY = 0, MOE_CAP_DROPLESS = 1 };
+/* Which assignments an over-full expert drops in MOE_CAP_CAPACITY mode ([EP]
+ * drop/pad section, Megatron-Core moe_token_drop_policy).  POSITION: the
+ * latest in (choice rank, token) order.  PROBS: the lowest gates; each expert
+ * keeps its C largest gates (fp32 comparison), equal gates keep the earlier
+ * assignment, and kept assignments take slots in (choice rank, token) order. */
+enum { MOE_DROP_POSITION = 0, MOE_DROP_PROBS = 1 };
 /* Element type of x, expert weights, dispatch buffers and y.  The router
  * weight, logits, gates and the aux loss are always fp32 ([SWITCH] 2.2). */
 enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
@@ -115,6 +121,7 @@ typedef struct moe_cfg {
   float aux_alpha;       /* alpha of the load-balancing loss ([SWITCH] 2.1: 1e-2) */
   int32_t flags;         /* MOE_FLAG_* */
   float z_coef;          /* router z-loss coefficient ([EP] aux-loss section), >= 0; 0 = no z-loss */
+  int32_t drop_policy;   /* MOE_DROP_* (ignored when dropless) */
 } moe_cfg;
 
 /* Expert weights (device pointers, element type cfg->dtype).
@@ -190,20 +197,24 @@ MOE_API int moe_route(const moe_cfg* cfg, const void* x, const float* wg, const 
 MOE_API int moe_route_from_logits(const moe_cfg* cfg, const float* logits, const float* uniform, int32_t* ids,
                                   float* gates, void* ws, moe_stream_t stream);
 
-/* Slot assignment ([EP] drop/pad section, "position" policy; [DS7508] without
- * the [T,E,C] mask).  Assignments are ordered by (choice rank, token); an
- * assignment's slot is the number of earlier assignments of its expert; it is
- * kept iff slot < C (always, when dropless).  Outputs: slot [T,k] (-1 dropped),
+/* Slot assignment ([EP] drop/pad section; [DS7508] without the [T,E,C] mask).
+ * Assignments are ordered by (choice rank, token).  "position" policy: an
+ * assignment's slot is the number of earlier assignments of its expert and it
+ * is kept iff slot < C (always, when dropless).  "probs" policy
+ * (cfg->drop_policy, capacity mode): gates [T,k] fp32 decide which C
+ * assignments an over-full expert keeps (see MOE_DROP_PROBS); gates may be NULL
+ * otherwise.  Outputs: slot [T,k] (-1 dropped),
  * expert_count [E] (pre-drop), kept_count [E], expert_offset [E+2] (expert e owns
  * rows [off[e], off[e]+kept[e]) of a 128-row-padded block; the shared block
  * [off[E], off[E]+T) follows; off[E+1] = rows used), row_token [rows_max]
  * (-1 on padding rows).  An id of -1 is a choice that is not dispatched: it
  * takes no slot and gets slot -1.  Other ids outside [0,E) set MOE_EDEVICE. */
-MOE_API int moe_assign_slots(const moe_cfg* cfg, const int32_t* ids, int32_t* slot, int32_t* expert_count,
-                     int32_t* kept_count, int32_t* expert_offset, int32_t* row_token, void* ws,
-                     moe_stream_t stream);
+MOE_API int moe_assign_slots(const moe_cfg* cfg, const int32_t* ids, const float* gates, int32_t* slot,
+                             int32_t* expert_count, int32_t* kept_count, int32_t* expert_offset, int32_t* row_token,
+                             void* ws, moe_stream_t stream);
 
-/* moe_assign_slots for callers that cannot allocate device memory.  No source
+/* moe_assign_slots ("position" policy only: MOE_DROP_PROBS in capacity mode
+ * returns MOE_EUNSUPPORTED) for callers that cannot allocate device memory.  No source
  * page has a counterpart: this is a deployment variant.  Some callers get
  * only their input and output buffers and may not allocate anything else, for
  * example a plugin inside a framework whose memory pool owns the whole device,

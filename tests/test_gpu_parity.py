@@ -133,7 +133,7 @@ def _slots_gpu(ids_np, E, cap_mode, cf=(1, 1), n_shared=0):
     kept = torch.empty(E, dtype=torch.int32, device="cuda")
     off = torch.empty(E + 2, dtype=torch.int32, device="cuda")
     rt = torch.empty(max(R, 1), dtype=torch.int32, device="cuda")
-    B.moe_assign_slots(cfg, ids, slot, cnt, kept, off, rt, ws)
+    B.moe_assign_slots(cfg, ids, None, slot, cnt, kept, off, rt, ws)
     st = B.moe_sync_status(ws)
     return st, slot.cpu().numpy(), cnt.cpu().numpy(), kept.cpu().numpy(), off.cpu().numpy(), rt.cpu().numpy()
 
@@ -252,7 +252,7 @@ def test_stage_entry_points_match_layer(variant):
     y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
     aux = torch.full((2,), float("nan"), device=dev)
     B.moe_route(cfg, inp["x"], inp["wg"], None, inp["uniform"], ids, gates, logits, ws)
-    B.moe_assign_slots(cfg, ids, slot, cnt, kept, off, rt, ws)
+    B.moe_assign_slots(cfg, ids, gates, slot, cnt, kept, off, rt, ws)
     B.moe_dispatch(cfg, inp["x"], ids, slot, off, xbuf)
     B.moe_expert_ffn(cfg, xbuf, inp["x"], off, B.make_weights(inp), ybuf, ws)
     B.moe_combine(cfg, ybuf, ids, slot, gates, off, y)

@@ -143,7 +143,7 @@ def test_slots_skip_undispatched_choices():
         kc = torch.zeros(E, dtype=torch.int32, device="cuda")
         off = torch.zeros(E + 2, dtype=torch.int32, device="cuda")
         rt = torch.full((rows,), -9, dtype=torch.int32, device="cuda")
-        B.moe_assign_slots(cfg, d_ids, slot, ec, kc, off, rt, ws)
+        B.moe_assign_slots(cfg, d_ids, None, slot, ec, kc, off, rt, ws)
         assert B.moe_sync_status(ws) == B.MOE_OK
         C = O.layer_capacity(oracle_layer(shape))
         r_slot, r_count, r_kept = O.assign_slots(ids, E, C)
@@ -154,3 +154,79 @@ def test_slots_skip_undispatched_choices():
         np.testing.assert_array_equal(off.cpu().numpy(), r_off)
         used = int(r_off[-1])
         np.testing.assert_array_equal(rt[:used].cpu().numpy(), O.row_tokens(ids, r_slot, r_off, 0))
+
+
+# ------------------------------------------------------------ "probs" drop policy
+def _slots_probs_gpu(shape, ids, gates):
+    cfg = B.make_cfg(shape)
+    ws = B.alloc_workspace(cfg)
+    T, k, E = shape.T, shape.k, shape.E
+    rows = B.moe_rows_max(cfg)
+    slot = torch.full((T, k), -9, dtype=torch.int32, device="cuda")
+    ec = torch.zeros(E, dtype=torch.int32, device="cuda")
+    kc = torch.zeros(E, dtype=torch.int32, device="cuda")
+    off = torch.zeros(E + 2, dtype=torch.int32, device="cuda")
+    rt = torch.full((max(rows, 1),), -9, dtype=torch.int32, device="cuda")
+    B.moe_assign_slots(cfg, torch.from_numpy(ids).cuda(), torch.from_numpy(gates).cuda(), slot, ec, kc, off, rt, ws)
+    assert B.moe_sync_status(ws) == B.MOE_OK
+    return slot.cpu().numpy(), ec.cpu().numpy(), kc.cpu().numpy(), off.cpu().numpy(), rt.cpu().numpy()
+
+
+@pytest.mark.parametrize("E,k,T,cf,quant,minus1", [
+    (3, 2, 4, (1, 2), 0, False), (8, 2, 3001, (1, 2), 0, True), (12, 4, 32768, (1, 2), 64, False),
+    (12, 4, 32768, (1, 4), 0, False), (64, 1, 8192, (5, 4), 16, False), (256, 8, 4099, (1, 1), 8, True),
+    (5, 3, 20000, (1, 8), 1, False)])
+def test_slots_probs_policy_exact(E, k, T, cf, quant, minus1):
+    """Exact parity of the per-expert top-C selection, including many equal gates
+    (quantised gates; quant=1 makes every gate equal) and undispatched ids."""
+    rng = np.random.default_rng(E * 7 + k)
+    skew = np.linspace(0, 2.0, E)
+    ids = np.argsort(-(rng.gumbel(size=(T, E)) + skew), axis=1)[:, :k].astype(np.int32)
+    if minus1:
+        ids[rng.random(T) < 0.3, 1] = -1
+    g = rng.random((T, k)).astype(np.float32)
+    if quant:
+        g = (np.floor(g * quant) / quant).astype(np.float32)
+    shape = synth.LayerShape("slots_probs", T=T, H=8, F=8, E=E, k=k, cf_num=cf[0], cf_den=cf[1],
+                             drop_policy=synth.DROP_PROBS)
+    slot, ec, kc, off, rt = _slots_probs_gpu(shape, ids, g)
+    C = O.capacity(T, E, k, *cf)
+    r_slot, r_count, r_kept = O.assign_slots_probs(ids, g.astype(np.float64), E, C)
+    assert (r_count > C).any()                   # some expert overflows
+    np.testing.assert_array_equal(slot, r_slot)
+    np.testing.assert_array_equal(ec, r_count)
+    np.testing.assert_array_equal(kc, r_kept)
+    r_off = O.row_layout(r_kept, T, 0)
+    np.testing.assert_array_equal(off, r_off)
+    used = int(r_off[-1])
+    np.testing.assert_array_equal(rt[:used], O.row_tokens(ids, r_slot, r_off, 0))
+    if quant == 1:                               # all gates equal: the position policy
+        p_slot, _, _ = O.assign_slots(ids, E, C)
+        np.testing.assert_array_equal(slot, p_slot)
+
+
+PROBS_CASES = {
+    "switch_probs": SWITCH_SMALL.replace(drop_policy=synth.DROP_PROBS),
+    "ds_k4_probs": DS_SMALL.replace(drop_policy=synth.DROP_PROBS),
+    "gshard_probs_random_second": GSHARD_SMALL.replace(drop_policy=synth.DROP_PROBS, random_second=1, cf_num=1,
+                                                       cf_den=2),
+}
+
+
+@pytest.mark.parametrize("name", list(PROBS_CASES))
+def test_layer_probs_policy(name):
+    shape = PROBS_CASES[name]
+    inp = synth.make_inputs(shape, seed=4, device="cuda")
+    condition_uniform(shape, inp)
+    out = run_layer(shape, inp)
+    ref = check_layer(shape, inp, out)
+    assert (ref["count"] > ref["capacity"]).any()
+
+
+def test_probs_policy_static_variant_unsupported():
+    shape = DS_SMALL.replace(drop_policy=synth.DROP_PROBS)
+    cfg = B.make_cfg(shape)
+    z = torch.zeros(1, dtype=torch.int32, device="cuda")
+    with pytest.raises(B.MoeError) as ei:
+        B.moe_assign_slots_static(cfg, z, z, z, z, z, z)
+    assert ei.value.code == B.MOE_EUNSUPPORTED

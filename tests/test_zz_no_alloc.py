@@ -54,7 +54,7 @@ def test_static_scratch_matches_workspace_version(shape):
     for call, seed in enumerate((11, 12)):                 # two calls in a row, different routings
         ids = _ids(shape.T, shape.E, shape.k, seed)
         ref, got = _outputs(cfg, R), _outputs(cfg, R)
-        B.moe_assign_slots(cfg, ids, ref["slot"], ref["count"], ref["kept"], ref["off"], ref["rt"], ws)
+        B.moe_assign_slots(cfg, ids, None, ref["slot"], ref["count"], ref["kept"], ref["off"], ref["rt"], ws)
         B.moe_assign_slots_static(cfg, ids, got["slot"], got["count"], got["kept"], got["off"], got["rt"])
         torch.cuda.synchronize()
         assert B.moe_sync_status(ws) == B.MOE_OK
