@@ -3,6 +3,11 @@
 -> grouped expert FFN -> combine -> aux loss) through the C ABI.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                  [--set FIELD=VALUE ...]
+
+--set overrides one routing option of the workload (score, renorm, z_coef,
+random_second, drop_policy, cf_num, cf_den); the workload name then carries the
+overrides, e.g. deepspeed_k4_T32768_H512_E12+drop_policy=1.
 
 One step = one moe_layer_fwd call over one batch of T synthetic tokens already
 resident in HBM.  L2 is flushed before every step, outside the timed events:
@@ -36,8 +41,18 @@ if ROOT not in sys.path:
 METRIC = "MoE layer tokens/s on 1 B200; dispatch/combine HBM GB/s; expert GEMM TC util %"
 DEFAULT_WORKLOAD = "switch_top1_T8192_H768_E64"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
-LAUNCHES_PER_STEP = 11      # router 3 (weight split, logits GEMM, softmax/top-k), slots 4 (aux loss
-                            # folded in), dispatch 1, expert FFN 2, combine 1
+SETTABLE = {"score": int, "renorm": int, "z_coef": float, "random_second": int, "drop_policy": int,
+            "cf_num": int, "cf_den": int}
+
+
+def launches_per_step(shape) -> int:
+    """Kernels one moe_layer_fwd call launches: router 3 for bf16 x (weight split,
+    logits GEMM, softmax/top-k) or 1 for fp32 x; slots 4 (aux loss folded in),
+    plus the per-expert select of the "probs" policy; dispatch 1; expert FFN 2;
+    combine 1."""
+    router = 3 if shape.dtype == 1 else 1
+    slots = 4 + (1 if shape.drop_policy == 1 and shape.cap_mode == 0 else 0)
+    return router + slots + 1 + 2 + 1
 
 
 def parse_args():
@@ -49,7 +64,24 @@ def parse_args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE")
     return ap.parse_args()
+
+
+def workload_shape(args):
+    """The named workload with the --set overrides applied."""
+    from expert_dispatch_router_b200 import synth
+    shape = synth.WORKLOADS[args.workload]
+    over = {}
+    for item in args.set:
+        key, _, val = item.partition("=")
+        if key not in SETTABLE:
+            raise SystemExit(f"--set: unknown field {key!r} (one of {sorted(SETTABLE)})")
+        over[key] = SETTABLE[key](val)
+    if over:
+        tag = "+".join(f"{k}={v}" for k, v in over.items())
+        shape = shape.replace(name=f"{shape.name}+{tag}", **over)
+    return shape
 
 
 # ------------------------------------------------------------------ plumbing
@@ -290,9 +322,10 @@ def oracle_sample_time(shape, inp_cpu: dict, tokens: int):
     d = lambda t: None if t is None else t
     x = inp_cpu["x"][:tokens]
     add = None if inp_cpu["logit_add"] is None else inp_cpu["logit_add"][:tokens]
+    uni = None if inp_cpu.get("uniform") is None else inp_cpu["uniform"][:tokens]
     t0 = time.perf_counter()
     O.layer_forward(layer, x, inp_cpu["wg"], inp_cpu["w1"], inp_cpu["w2"], d(inp_cpu["w3"]), d(inp_cpu["sw1"]),
-                    d(inp_cpu["sw2"]), d(inp_cpu["sw3"]), logit_add=add)
+                    d(inp_cpu["sw2"]), d(inp_cpu["sw3"]), logit_add=add, uniform=uni)
     return time.perf_counter() - t0
 
 
@@ -310,7 +343,8 @@ def host_inputs(inp: dict):
     d = lambda t: None if t is None else t.to("cpu", torch.float64).numpy()
     return {"x": d(inp["x"]), "wg": d(inp["wg"]), "w1": Lazy(inp["w1"]), "w2": Lazy(inp["w2"]),
             "w3": None if inp["w3"] is None else Lazy(inp["w3"]), "sw1": d(inp["sw1"]), "sw2": d(inp["sw2"]),
-            "sw3": d(inp["sw3"]), "logit_add": None if inp["logit_add"] is None else inp["logit_add"].cpu().numpy()}
+            "sw3": d(inp["sw3"]), "logit_add": None if inp["logit_add"] is None else inp["logit_add"].cpu().numpy(),
+            "uniform": None if inp.get("uniform") is None else inp["uniform"].cpu().numpy()}
 
 
 def blas_threads():
@@ -340,7 +374,7 @@ def run_reference(args, world, rank):
         return
     import torch
     from expert_dispatch_router_b200 import synth
-    shape = synth.WORKLOADS[args.workload]
+    shape = workload_shape(args)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     inp = synth.make_inputs(shape, seed=args.seed, device=dev)
     host = host_inputs(inp)
@@ -372,7 +406,7 @@ def run_ours(args, world, rank, local):
     from expert_dispatch_router_b200 import synth
 
     B.load()                                     # raises if the CUDA library is missing
-    shape = synth.WORKLOADS[args.workload]
+    shape = workload_shape(args)
     peaks = load_peaks()
     dev = torch.device("cuda", torch.cuda.current_device())
     inp = synth.make_inputs(shape, seed=replica_seed(args.seed, rank), device="cuda")
@@ -381,7 +415,7 @@ def run_ours(args, world, rank, local):
     T, H = shape.T, shape.H
     edt = inp["x"].dtype
     y = torch.empty((T, H), dtype=edt, device=dev)
-    aux = torch.empty(1, dtype=torch.float32, device=dev)
+    aux = torch.empty(2, dtype=torch.float32, device=dev)
     wts = B.make_weights(inp)
     # L2 flush between steps (outside the timed events): write one 320 MiB buffer,
     # then read another, so the timed step starts with an L2 that holds no data
@@ -397,7 +431,8 @@ def run_ours(args, world, rank, local):
 
     def step(events=None):
         flush_l2()
-        B.moe_layer_fwd(cfg, inp["x"], inp["wg"], inp["logit_add"], None, wts, y, aux, None, ws, stage_events=events,
+        B.moe_layer_fwd(cfg, inp["x"], inp["wg"], inp["logit_add"], inp["uniform"], wts, y, aux, None, ws,
+                        stage_events=events,
                         stream=stream)
 
     for _ in range(max(args.warmup, 3)):
@@ -454,34 +489,62 @@ def run_ours(args, world, rank, local):
     tc_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) if long_step else peaks["bf16_tflops"]
     tc_util = 100.0 * gemm_flops / (gemm_ms / 1e3) / (tc_peak * 1e12)
 
-    # end to end: pinned host inputs in, result read back, every step
+    # end to end: every step copies its inputs from pinned host memory and reads
+    # its result back.  Steps are pipelined over two buffer sets and three
+    # streams (host->device copies, the layer, device->host copies), as a caller
+    # streaming batches would run them: step i+1's inputs and step i-1's result
+    # cross PCIe while step i computes.
+    aux_n = 2 if shape.z_coef else 1
     x_host = inp["x"].cpu().pin_memory()
     add_host = None if inp["logit_add"] is None else inp["logit_add"].cpu().pin_memory()
-    x_dev = torch.empty_like(inp["x"])
-    add_dev = None if add_host is None else torch.empty_like(inp["logit_add"])
-    y_host = torch.empty((T, H), dtype=edt).pin_memory()
-    aux_host = torch.empty(1, dtype=torch.float32).pin_memory()
-    h2d = x_host.numel() * x_host.element_size() + (0 if add_host is None else add_host.numel() * 4)
-    d2h = y_host.numel() * y_host.element_size() + 4
+    uni_host = None if inp["uniform"] is None else inp["uniform"].cpu().pin_memory()
+    h2d = x_host.numel() * x_host.element_size() + (0 if add_host is None else add_host.numel() * 4) \
+        + (0 if uni_host is None else uni_host.numel() * 4)
+    d2h = T * H * x_host.element_size() + 4 * aux_n
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    bufs = []
+    for _ in range(2):
+        b = {"x": torch.empty_like(inp["x"]),
+             "add": None if add_host is None else torch.empty_like(inp["logit_add"]),
+             "uni": None if uni_host is None else torch.empty_like(inp["uniform"]),
+             "y": torch.empty((T, H), dtype=edt, device=dev), "aux": torch.empty(2, dtype=torch.float32, device=dev),
+             "y_host": torch.empty((T, H), dtype=edt).pin_memory(),
+             "aux_host": torch.empty(aux_n, dtype=torch.float32).pin_memory()}
+        for name in ("loaded", "computed", "drained"):
+            b[name] = torch.cuda.Event()
+            b[name].record(stream)          # created (and complete) before first use
+        bufs.append(b)
 
-    def e2e_step():
-        x_dev.copy_(x_host, non_blocking=True)
-        if add_host is not None:
-            add_dev.copy_(add_host, non_blocking=True)
-        B.moe_layer_fwd(cfg, x_dev, inp["wg"], add_dev, None, wts, y, aux, None, ws, stream=stream)
-        y_host.copy_(y, non_blocking=True)
-        aux_host.copy_(aux, non_blocking=True)
+    def e2e_step(i):
+        b = bufs[i % 2]
+        s_in.wait_event(b["computed"])      # the layer that read these inputs is done
+        with torch.cuda.stream(s_in):
+            b["x"].copy_(x_host, non_blocking=True)
+            if add_host is not None:
+                b["add"].copy_(add_host, non_blocking=True)
+            if uni_host is not None:
+                b["uni"].copy_(uni_host, non_blocking=True)
+        b["loaded"].record(s_in)
+        stream.wait_event(b["loaded"])
+        stream.wait_event(b["drained"])     # this y buffer has been read back
+        B.moe_layer_fwd(cfg, b["x"], inp["wg"], b["add"], b["uni"], wts, b["y"], b["aux"], None, ws, stream=stream)
+        b["computed"].record(stream)
+        s_out.wait_event(b["computed"])
+        with torch.cuda.stream(s_out):
+            b["y_host"].copy_(b["y"], non_blocking=True)
+            b["aux_host"].copy_(b["aux"][:aux_n], non_blocking=True)
+        b["drained"].record(s_out)
 
-    for _ in range(max(args.warmup, 3)):
-        e2e_step()
+    for i in range(max(args.warmup, 3)):
+        e2e_step(i)
     e2e_steps = args.steps
     ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
-    ea.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    eb.record(stream)
+    ea.record(s_in)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    eb.record(s_out)                        # after the last read-back
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(ea.elapsed_time(eb) / e2e_steps, world)
@@ -510,8 +573,8 @@ def run_ours(args, world, rank, local):
                                 for s, v in per_stage.items()},
             "dominant_kernel": dom,
             "e2e": {"value": job_tokens_per_s(T, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
-            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+                    "d2h_bytes_per_step": d2h, "pipelining": "2 buffer sets; copy-in, layer, copy-out streams"},
+            "gpu_launches": launches_per_step(shape) * args.steps,
             "clocks": clocks,
             "cpu_baseline": cpu,
         }

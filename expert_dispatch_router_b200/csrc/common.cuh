@@ -4,6 +4,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/moe_b200.h"
 
 namespace moe {
@@ -113,18 +115,29 @@ __device__ __forceinline__ float act_silu(float z) { return z * rcp_approx(1.0f 
 // at the B200's boost clock).  Normal waits in these kernels last microseconds.
 constexpr long long kWaitCycles = 2000000000LL;
 
-// Host: raise a kernel's dynamic shared memory limit once per device.
-template <typename Kernel>
-inline cudaError_t ensure_smem(Kernel k, size_t bytes) {
+// Host: raise a kernel's dynamic shared memory limit to at least `bytes` on the
+// current device.  Remembers, per (kernel, device), the largest limit set.
+inline cudaError_t ensure_smem_ptr(const void* k, size_t bytes) {
   if (bytes <= 48 * 1024) return cudaSuccess;
-  static unsigned long long done = 0;          // one bit per device ordinal (< 64)
   int dev = 0;
   cudaGetDevice(&dev);
-  const unsigned long long bit = 1ull << (dev & 63);
-  if (__atomic_load_n(&done, __ATOMIC_ACQUIRE) & bit) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-  if (e == cudaSuccess) __atomic_fetch_or(&done, bit, __ATOMIC_RELEASE);
-  return e;
+  struct Entry { const void* k; int dev; size_t bytes; };
+  static std::mutex mu;
+  static Entry tab[256];
+  static int n = 0;
+  std::lock_guard<std::mutex> lock(mu);
+  int i = 0;
+  while (i < n && !(tab[i].k == k && tab[i].dev == dev)) ++i;
+  if (i < n && tab[i].bytes >= bytes) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return e;
+  if (i < n) tab[i].bytes = bytes;
+  else if (n < 256) tab[n++] = Entry{k, dev, bytes};
+  return cudaSuccess;
+}
+template <typename Kernel>
+inline cudaError_t ensure_smem(Kernel k, size_t bytes) {
+  return ensure_smem_ptr(reinterpret_cast<const void*>(k), bytes);
 }
 
 // Host: multiprocessor count of the current device (cached per device).

@@ -70,7 +70,7 @@ struct SlotParams {
   const float* gates;       // [T,k] or null: "position" policy
   int32_t* cum;             // [E] exclusive prefix of expert_count
   uint32_t* list_key;       // [T*k] order-preserving gate keys
-  uint32_t* list_idx;       // [T*k] assignment index r*T + t
+  uint32_t* list_idx;       // [T*k] the assignment's flat index t*k + r
 };
 constexpr int kSlotChunk = 256;    // assignments per CTA of the slot kernels (one per thread)
 cudaError_t launch_slots(const SlotParams& p, cudaStream_t stream);

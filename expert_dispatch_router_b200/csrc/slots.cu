@@ -239,7 +239,7 @@ __global__ void __launch_bounds__(kSlotThreads) slot_rank_kernel(SlotParams p, i
       // over-full expert under the "probs" policy: list it for the select kernel
       const int64_t li = (int64_t)p.cum[e] + pos;
       p.list_key[li] = to_ordered(p.gates[t * p.k + r]);
-      p.list_idx[li] = (uint32_t)a;
+      p.list_idx[li] = (uint32_t)(t * p.k + r);
       continue;
     }
     const bool kept = p.capacity < 0 || pos < p.capacity;
@@ -249,11 +249,15 @@ __global__ void __launch_bounds__(kSlotThreads) slot_rank_kernel(SlotParams p, i
   }
 }
 
-// One CTA per expert; only experts with more than C assignments do work.
+// One CTA per expert; only experts with more than C assignments do work.  An
+// expert's list (keys and slot indices) is staged in shared memory when it fits
+// (kSelSmemElems); otherwise it is read from global memory.
 constexpr int kSelThreads = 1024;
 constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kSelSmemElems = 24576;         // 192 KB of (key, index) pairs
 
 __global__ void __launch_bounds__(kSelThreads) slot_select_kernel(SlotParams p) {
+  extern __shared__ uint32_t sbuf[];           // [kSelSmemElems] keys, then [kSelSmemElems] indices
   __shared__ int hist[256];
   __shared__ int sh[kSelWarps];
   __shared__ uint32_t s_prefix;
@@ -262,8 +266,16 @@ __global__ void __launch_bounds__(kSelThreads) slot_select_kernel(SlotParams p) 
   const int n = p.expert_count[e];
   if ((int64_t)n <= p.capacity) return;
   const int64_t base = p.cum[e];
-  const uint32_t* key = p.list_key + base;
-  const uint32_t* idx = p.list_idx + base;
+  const bool staged = n <= kSelSmemElems;
+  if (staged) {
+    for (int i = tid; i < n; i += kSelThreads) {
+      sbuf[i] = p.list_key[base + i];
+      sbuf[kSelSmemElems + i] = p.list_idx[base + i];
+    }
+    __syncthreads();
+  }
+  const uint32_t* key = staged ? sbuf : p.list_key + base;
+  const uint32_t* idx = staged ? sbuf + kSelSmemElems : p.list_idx + base;
 
   // radix select: after the four 8-bit passes, `prefix` is the C-th largest key
   // and `need` is how many of the keys equal to it are kept (the earliest ones)
@@ -273,9 +285,12 @@ __global__ void __launch_bounds__(kSelThreads) slot_select_kernel(SlotParams p) 
   for (int shift = 24; shift >= 0 && need > 0; shift -= 8) {
     for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
     __syncthreads();
-    for (int i = tid; i < n; i += kSelThreads) {
-      const uint32_t kv = key[i];
-      if ((kv & mask) == prefix) atomicAdd(&hist[(kv >> shift) & 255u], 1);
+    for (int i0 = 0; i0 < n; i0 += kSelThreads) {   // warp-uniform trip count for match_any
+      const int i = i0 + tid;
+      const uint32_t kv = i < n ? key[i] : 0u;
+      const int bin = (i < n && (kv & mask) == prefix) ? (int)((kv >> shift) & 255u) : -1;
+      const unsigned peers = __match_any_sync(0xffffffffu, bin);
+      if (bin >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
     }
     __syncthreads();
     if (warp == 0) {
@@ -310,27 +325,44 @@ __global__ void __launch_bounds__(kSelThreads) slot_select_kernel(SlotParams p) 
     __syncthreads();
   }
 
-  // ordered pass: keep keys above the threshold and the first `need` equal ones
+  // ordered pass.  Kept = every key above the threshold and the first `need`
+  // keys equal to it, so the kept elements before position i number
+  // gt_before(i) + min(eq_before(i), need).  Warp w owns a contiguous segment of
+  // the arrival order: one block scan of the warps' (eq, gt) totals, then each
+  // warp walks its segment with ballots, free of block barriers.
+  const int seg = ((n + kSelWarps - 1) / kSelWarps + 31) & ~31;
+  const int s0 = min(n, warp * seg), s1 = min(n, s0 + seg);
+  int my_eq = 0, my_gt = 0;
+  for (int i = s0 + lane; i < s1; i += 32) {
+    const uint32_t kv = key[i];
+    my_eq += kv == prefix;
+    my_gt += kv > prefix;
+  }
+  my_eq = __reduce_add_sync(0xffffffffu, my_eq);
+  my_gt = __reduce_add_sync(0xffffffffu, my_gt);
+  int tot;
+  // only lane 0 carries its warp's totals, so the exclusive prefix at lane 0 is
+  // the warp's base
+  int eq_before = __shfl_sync(0xffffffffu, block_scan_excl<kSelWarps>(lane == 0 ? my_eq : 0, sh, tot), 0);
+  int gt_before = __shfl_sync(0xffffffffu, block_scan_excl<kSelWarps>(lane == 0 ? my_gt : 0, sh, tot), 0);
   const int64_t off = p.expert_offset[e];
-  int run_eq = 0, run_keep = 0;
-  for (int b0 = 0; b0 < n; b0 += kSelThreads) {
-    const int i = b0 + tid;
-    const bool valid = i < n;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int i0 = s0; i0 < s1; i0 += 32) {
+    const int i = i0 + lane;
+    const bool valid = i < s1;
     const uint32_t kv = valid ? key[i] : 0u;
-    const int eq = valid && kv == prefix;
-    int tot_eq;
-    const int eq_rank = run_eq + block_scan_excl<kSelWarps>(eq, sh, tot_eq);
-    const int keep = valid && (kv > prefix || (eq && eq_rank < need));
-    int tot_keep;
-    const int rank = run_keep + block_scan_excl<kSelWarps>(keep, sh, tot_keep);
+    const unsigned beq = __ballot_sync(0xffffffffu, valid && kv == prefix);
+    const unsigned bgt = __ballot_sync(0xffffffffu, valid && kv > prefix);
     if (valid) {
-      const uint32_t a = idx[i];
-      const int64_t r = (int64_t)a / p.T, t = (int64_t)a - r * p.T;
-      p.slot[t * p.k + r] = keep ? rank : -1;
-      if (keep && off + rank < p.rows_max) p.row_token[off + rank] = (int)t;
+      const int eqb = eq_before + __popc(beq & lt), gtb = gt_before + __popc(bgt & lt);
+      const bool keep = kv > prefix || (kv == prefix && eqb < need);
+      const int rank = gtb + min(eqb, need);
+      const uint32_t flat = idx[i];                // t * k + r
+      p.slot[flat] = keep ? rank : -1;
+      if (keep && off + rank < p.rows_max) p.row_token[off + rank] = (int)(flat / (uint32_t)p.k);
     }
-    run_eq += tot_eq;
-    run_keep += tot_keep;
+    eq_before += __popc(beq);
+    gt_before += __popc(bgt);
   }
 }
 
@@ -350,7 +382,12 @@ cudaError_t launch_slots(const SlotParams& p, cudaStream_t stream) {
     cudaError_t e = ensure_smem(slot_rank_kernel, sm);
     if (e != cudaSuccess) return e;
     slot_rank_kernel<<<nchunk, kSlotThreads, sm, stream>>>(p, nchunk);
-    if (p.gates != nullptr) slot_select_kernel<<<p.E, kSelThreads, 0, stream>>>(p);
+    if (p.gates != nullptr) {
+      const size_t ssm = 2 * sizeof(uint32_t) * kSelSmemElems;
+      e = ensure_smem(slot_select_kernel, ssm);
+      if (e != cudaSuccess) return e;
+      slot_select_kernel<<<p.E, kSelThreads, ssm, stream>>>(p);
+    }
   }
   return cudaGetLastError();
 }

@@ -175,10 +175,11 @@ def _slots_probs_gpu(shape, ids, gates):
 @pytest.mark.parametrize("E,k,T,cf,quant,minus1", [
     (3, 2, 4, (1, 2), 0, False), (8, 2, 3001, (1, 2), 0, True), (12, 4, 32768, (1, 2), 64, False),
     (12, 4, 32768, (1, 4), 0, False), (64, 1, 8192, (5, 4), 16, False), (256, 8, 4099, (1, 1), 8, True),
-    (5, 3, 20000, (1, 8), 1, False)])
+    (5, 3, 20000, (1, 8), 1, False), (4, 2, 40000, (1, 4), 0, False)])
 def test_slots_probs_policy_exact(E, k, T, cf, quant, minus1):
     """Exact parity of the per-expert top-C selection, including many equal gates
-    (quantised gates; quant=1 makes every gate equal) and undispatched ids."""
+    (quantised gates; quant=1 makes every gate equal), undispatched ids, and an
+    expert with more assignments than the select kernel stages on chip."""
     rng = np.random.default_rng(E * 7 + k)
     skew = np.linspace(0, 2.0, E)
     ids = np.argsort(-(rng.gumbel(size=(T, E)) + skew), axis=1)[:, :k].astype(np.int32)
@@ -193,6 +194,8 @@ def test_slots_probs_policy_exact(E, k, T, cf, quant, minus1):
     C = O.capacity(T, E, k, *cf)
     r_slot, r_count, r_kept = O.assign_slots_probs(ids, g.astype(np.float64), E, C)
     assert (r_count > C).any()                   # some expert overflows
+    if T == 40000:
+        assert r_count.max() > 24576
     np.testing.assert_array_equal(slot, r_slot)
     np.testing.assert_array_equal(ec, r_count)
     np.testing.assert_array_equal(kc, r_kept)
