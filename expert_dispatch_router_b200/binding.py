@@ -19,7 +19,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libmoe_b200.so")
 
 MOE_OK, MOE_EINVAL, MOE_EUNSUPPORTED, MOE_ECUDA, MOE_ETIMEOUT, MOE_EDEVICE, MOE_EWORKSPACE = range(7)
-MOE_FLAG_KEEP_LOGITS, MOE_FLAG_RANDOM_SECOND = 1, 2
+MOE_FLAG_KEEP_LOGITS, MOE_FLAG_RANDOM_SECOND, MOE_FLAG_UNFUSED = 1, 2, 4
 MOE_N_STAGE_EVENTS = 8
 STAGES = ("router", "slots", "dispatch", "ffn_gemm1", "ffn_gemm2", "combine", "aux")
 

@@ -52,6 +52,8 @@ constexpr int RING_BYTES = 4 * (A_BYTES + BN * BK * 2);   // 192 KB: 4 stages at
 constexpr int MAX_STAGES = 8;
 constexpr int EPI_WARPS = 16;                      // 4 per TMEM sub-partition
 constexpr int THREADS = 64 + EPI_WARPS * 32;
+constexpr int GATHER_WARPS = 2;                    // fused dispatch: cp.async row gathers, 64 rows each
+constexpr int THREADS_GATHER = THREADS + GATHER_WARPS * 32;
 constexpr int TMEM_COLS = 512;
 constexpr int STAGE_OUT_BYTES = 32 * 32 * 2;       // one warp's 32 x 32 bf16 output sub-tile
 constexpr int STAGING_BYTES = EPI_WARPS * STAGE_OUT_BYTES;   // 32 KB
@@ -73,6 +75,13 @@ struct KParams {
   int a_kwrap;           // > 0 (router): B holds 3 planes of a_kwrap k blocks; A's k block = kb / 3
   int plane_split;       // router: 1 = one tile per (m-block, n-tile, plane), fp32 partials per plane
   int out_f32;           // 1: store the raw fp32 accumulator
+  // fused dispatch: routed A rows gathered from gsrc [rows of K elements] by gidx
+  // (warp 0 issues cp.async with the 128-byte swizzle applied by hand)
+  const __nv_bfloat16* gsrc;
+  const int32_t* gidx;
+  // fused top-1 combine: routed rows stored to sdst[gidx[row]] * sgate[gidx[row]]
+  __nv_bfloat16* sdst;
+  const float* sgate;
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -126,6 +135,17 @@ __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.a
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" :: "r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
+
+// 16-byte cp.async from global to shared; src_bytes = 0 writes zeros.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+// The mbarrier receives one arrival once all of this thread's earlier cp.async
+// operations have completed (the arrival is part of its expected count).
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" :: "r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -207,7 +227,12 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-__global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_constant__ KParams p) {
+// GATHER: routed A rows are gathered from p.gsrc by warps 18-19 (fused
+// dispatch).  SCATTER: routed output rows go to p.sdst[token] * gate (fused
+// top-1 combine).  Both false: every operand moves by TMA.
+template <bool GATHER, bool SCATTER>
+__global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
+    grouped_gemm_kernel(const __grid_constant__ KParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
@@ -224,9 +249,12 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
   const bool swiglu = p.epi == MOE_ACT_SWIGLU;
   const bool grouped = p.rows_static < 0;
   const int ngroups = p.E + (p.n_shared ? 1 : 0);
+  // full barrier arrivals per stage: the TMA lane's arrive.expect_tx, plus one
+  // per gather lane
+  const uint32_t full_count = GATHER ? 1u + GATHER_WARPS * 32u : 1u;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < MAX_STAGES; ++s) { mbar_init(full0 + 8 * s, 1); mbar_init(empty0 + 8 * s, 1); }
+    for (int s = 0; s < MAX_STAGES; ++s) { mbar_init(full0 + 8 * s, full_count); mbar_init(empty0 + 8 * s, 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(tfull0 + 8 * b, 1); mbar_init(tempty0 + 8 * b, EPI_WARPS * 32); }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -283,6 +311,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
         const int g = grouped ? find_group(p.off, ngroups, row0) : 0;
         const bool sh = grouped && g == p.E;
         const bool sep = sh && p.as_sep;
+        const bool gat = GATHER && !sh;          // the gather warps fill this tile's A
         const CUtensorMap* ma = sep ? &p.tmAs : &p.tmA;
         const CUtensorMap* mb0 = sh ? &p.tmSB0 : &p.tmB0;
         const CUtensorMap* mb1 = sh ? &p.tmSB1 : &p.tmB1;
@@ -299,8 +328,8 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
           const int ka = (p.a_kwrap > 0 && !p.plane_split ? kb / 3 : kb) * BK;
           const int kbb = (p.plane_split ? plane * p.a_kwrap + kb
                            : p.a_kwrap > 0 ? (kb % 3) * p.a_kwrap + kb / 3 : kb) * BK;
-          mbar_expect_tx(fb, stage_bytes);
-          tma_load_2d(sa, ma, ka, arow, fb);
+          mbar_expect_tx(fb, gat ? stage_bytes - A_BYTES : stage_bytes);
+          if (!gat) tma_load_2d(sa, ma, ka, arow, fb);
           if (swiglu) {
             tma_load_3d(sb, mb0, kbb, n0, z, fb);                 // gate rows
             tma_load_3d(sb + box_bytes, mb1, kbb, n0, z, fb);     // up rows
@@ -322,6 +351,57 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
           while (!mbar_try_wait(full0 + 8 * s, (fills[s] - 1) & 1u) && clock64() - t0 < kWaitCycles) {}
         }
     }
+  } else if (GATHER && warp >= 2 + EPI_WARPS) {
+    // ---------------- gather producers (fused dispatch): warp gw fills A rows
+    // [64 gw, 64 gw + 64) of every routed tile with 16-byte cp.async copies of x
+    // rows, applying the 128-byte swizzle (chunk c of row r at c ^ (r & 7)).
+    // Lane l copies chunk (l & 7) of rows 64 gw + 4 i + (l >> 3), i < 16.
+    const int gw = warp - 2 - EPI_WARPS;
+    const int c = lane & 7, lr = lane >> 3;
+    const uint32_t sw_even = (uint32_t)((c ^ (lr & 7)) << 4), sw_odd = (uint32_t)((c ^ ((4 + lr) & 7)) << 4);
+    const uint32_t row_off = (uint32_t)((64 * gw + lr) * 128);
+    const int64_t rowbytes = (int64_t)p.K * 2;
+    const char* xsrc = reinterpret_cast<const char*>(p.gsrc);
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+      const int64_t mt = tile / n_tiles_n;
+      const int64_t row0 = mt * BM;
+      const int g = find_group(p.off, ngroups, row0);
+      const bool gat = g != p.E;
+      int tok[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) tok[i] = gat ? __ldg(p.gidx + row0 + 64 * gw + 4 * i + lr) : -1;
+      for (int kb = 0; kb < nk_tile; ++kb) {
+        int good = 1;
+        if (lane == 0) good = mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag);
+        good = __shfl_sync(0xffffffffu, good, 0);
+        if (!good) { ok = false; break; }
+        const uint32_t sa = smem_u32(stage_base + stage * stage_bytes);
+        const uint32_t fb = full0 + 8 * stage;
+        if (gat) {
+          const int kk = kb * BK + c * 8;
+          const bool kin = kk < p.K;
+          const char* kbase = xsrc + (int64_t)kk * 2;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const uint32_t dst = sa + row_off + (uint32_t)(i * 512) + ((i & 1) ? sw_odd : sw_even);
+            const bool live = kin && tok[i] >= 0;
+            cp_async16(dst, live ? kbase + (int64_t)tok[i] * rowbytes : xsrc, live ? 16u : 0u);
+          }
+          cp_async_arrive(fb);
+        } else {
+          mbar_arrive(fb);                       // this tile's A comes by TMA
+        }
+        if (++stage == n_stages) { stage = 0; phase ^= 1u; }
+      }
+    }
+    cp_async_wait_all();                         // no copy still writing shared memory
+    if (!ok && lane == 0) {
+      *abort_flag = 1;
+      set_status(p.status, MOE_ETIMEOUT, 13);
+    }
   } else if (warp == 1) {
     // ---------------- MMA issuer
     if (lane == 0) {
@@ -338,6 +418,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
         for (int kb = 0; kb < nk_tile; ++kb) {
           if (!mbar_wait(full0 + 8 * stage, phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
+          if (GATHER) fence_async_smem();       // cp.async data (generic proxy) -> tensor-core reads
           const uint32_t sa = smem_u32(stage_base + stage * stage_bytes);
           const uint32_t sb = sa + A_BYTES;
           const uint64_t ad = sw128_desc(sa), bd = sw128_desc(sb);
@@ -360,7 +441,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       const long long t0 = clock64();
       while (!mbar_try_wait(drain, 0) && clock64() - t0 < kWaitCycles) {}
     }
-  } else {
+  } else if (warp < 2 + EPI_WARPS) {
     // ---------------- epilogue
     const int ew = warp - 2;
     const int sub = warp & 3;                  // TMEM sub-partition this warp may access
@@ -382,6 +463,13 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       const int nt = (int)(tile / n_planes % n_tiles_n);
       const int64_t grow = mt * BM + row_in_tile;
       const bool row_ok = grow < p.rows_store;
+      // fused top-1 combine: this lane's row is token st of the batch, weighted by sg
+      int st = -1;
+      float sg = 0.0f;
+      if (SCATTER && row_ok) {
+        st = __ldg(p.gidx + grow);
+        if (st >= 0) sg = __ldg(p.sgate + st);
+      }
       const int ncol0 = nt * n_step;                           // first output column of the tile
       const uint32_t tbase = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * BN);
       for (int c = quarter * chunk; c < n_step; c += 4 * chunk) {
@@ -421,6 +509,16 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
                 if (cc + i < p.N_out) drow[cc + i] = v[4 * q + i];
             }
           }
+        } else if (SCATTER) {
+          if (st < 0) continue;
+          __nv_bfloat16* dst = p.sdst + (int64_t)st * p.N_out + col;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (8 * q < chunk && col + 8 * q < p.N_out)
+              st_v4(dst + 8 * q, make_int4((int)pack_bf16(sg * v[8 * q + 0], sg * v[8 * q + 1]),
+                                           (int)pack_bf16(sg * v[8 * q + 2], sg * v[8 * q + 3]),
+                                           (int)pack_bf16(sg * v[8 * q + 4], sg * v[8 * q + 5]),
+                                           (int)pack_bf16(sg * v[8 * q + 6], sg * v[8 * q + 7])));
         } else {
           // bf16: this warp's 32 rows x 32 columns go through its staging buffer
           // (16-byte chunk j of row r at chunk j ^ ((r >> 1) & 3): the TMA 64-byte
@@ -555,14 +653,22 @@ static bool make_map_d(CUtensorMap* m, const void* base, int64_t rows, int N) {
   return encode_cached(m, key);
 }
 
-static cudaError_t launch_kernel(KParams& k, int64_t max_tiles, cudaStream_t stream) {
-  cudaError_t e = ensure_smem(grouped_gemm_kernel, SMEM_BYTES);
+template <bool GATHER, bool SCATTER>
+static cudaError_t launch_variant(KParams& k, int grid, cudaStream_t stream) {
+  auto kern = grouped_gemm_kernel<GATHER, SCATTER>;
+  cudaError_t e = ensure_smem(kern, SMEM_BYTES);
   if (e != cudaSuccess) return e;
+  kern<<<grid, GATHER ? THREADS_GATHER : THREADS, SMEM_BYTES, stream>>>(k);
+  return cudaGetLastError();
+}
+
+static cudaError_t launch_kernel(KParams& k, int64_t max_tiles, cudaStream_t stream) {
   const int sms = sm_count();
   // grid: one CTA per SM, never more than the largest possible tile count
   const int grid = (int)(max_tiles < sms ? (max_tiles > 0 ? max_tiles : 1) : sms);
-  grouped_gemm_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(k);
-  return cudaGetLastError();
+  const bool gather = k.gsrc != nullptr, scatter = k.sdst != nullptr;
+  if (gather) return scatter ? launch_variant<true, true>(k, grid, stream) : launch_variant<true, false>(k, grid, stream);
+  return scatter ? launch_variant<false, true>(k, grid, stream) : launch_variant<false, false>(k, grid, stream);
 }
 
 }  // namespace gg
@@ -573,7 +679,7 @@ cudaError_t launch_grouped_gemm(const GemmParams& p, cudaStream_t stream) {
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
   const int box_n = 128;
   KParams k{};
-  bool ok = make_map_a(&k.tmA, p.a_routed, p.rows_max, p.K);
+  bool ok = make_map_a(&k.tmA, p.a_routed ? p.a_routed : p.gather_src, p.a_routed ? p.rows_max : p.T, p.K);
   ok = ok && make_map_a(&k.tmAs, p.a_shared ? p.a_shared : p.a_routed, p.a_shared ? p.T : p.rows_max, p.K);
   ok = ok && make_map_b(&k.tmB0, p.b0, p.E, p.Nw, p.K, box_n);
   ok = ok && make_map_b(&k.tmB1, p.b1 ? p.b1 : p.b0, p.E, p.Nw, p.K, box_n);
@@ -599,6 +705,10 @@ cudaError_t launch_grouped_gemm(const GemmParams& p, cudaStream_t stream) {
   k.a_kwrap = 0;
   k.plane_split = 0;
   k.out_f32 = 0;
+  k.gsrc = static_cast<const __nv_bfloat16*>(p.gather_src);
+  k.gidx = p.gather_idx;
+  k.sdst = static_cast<__nv_bfloat16*>(p.scatter_dst);
+  k.sgate = p.scatter_gate;
   return launch_kernel(k, (p.rows_max / BM) * ((p.Nw + box_n - 1) / box_n), stream);
 }
 

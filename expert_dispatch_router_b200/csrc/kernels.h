@@ -88,6 +88,8 @@ struct PermuteParams {
 };
 cudaError_t launch_dispatch(const PermuteParams& p, cudaStream_t stream);
 cudaError_t launch_combine(const PermuteParams& p, cudaStream_t stream);
+// y[t] = 0 for every token with no kept choice (dst = y).
+cudaError_t launch_zero_dropped(const PermuteParams& p, cudaStream_t stream);
 
 // fp32 SIMT grouped FFN (one GEMM per call).
 struct FfnF32Params {
@@ -117,6 +119,14 @@ struct GemmParams {
   int64_t T, rows_max;
   int K, Nw, E, n_shared, epi;    // epi: -1 none, else MOE_ACT_*
   DevStatus* status;
+  // Fused dispatch: routed A rows are gathered from gather_src [T, K] by
+  // gather_idx (row_token; -1 = padding row, read as zeros); a_routed unused.
+  const void* gather_src;
+  const int32_t* gather_idx;
+  // Fused top-1 combine: routed output rows go to scatter_dst[token] scaled by
+  // scatter_gate[token] instead of d (no shared expert, k = 1).
+  void* scatter_dst;
+  const float* scatter_gate;
 };
 cudaError_t launch_grouped_gemm(const GemmParams& p, cudaStream_t stream);
 

@@ -35,7 +35,7 @@ bool valid_cfg(const moe_cfg* c) {
   if (c->cap_mode == MOE_CAP_CAPACITY && (c->cf_num <= 0 || c->cf_den <= 0)) return false;
   if (c->min_capacity < 0) return false;
   if (!(c->z_coef >= 0.0f) || isinf(c->z_coef)) return false;
-  if (c->flags & ~(MOE_FLAG_KEEP_LOGITS | MOE_FLAG_RANDOM_SECOND)) return false;
+  if (c->flags & ~(MOE_FLAG_KEEP_LOGITS | MOE_FLAG_RANDOM_SECOND | MOE_FLAG_UNFUSED)) return false;
   if (c->drop_policy != MOE_DROP_POSITION && c->drop_policy != MOE_DROP_PROBS) return false;
   return true;
 }
@@ -223,8 +223,12 @@ int record(const moe_event_t* ev, int i, cudaStream_t s) {
 }
 
 // Both contractions of the expert FFN; `ev_mid`, if non-NULL, is recorded between them.
+// bf16 only: with `rowtok`, GEMM1 gathers its routed A rows from x (fused
+// dispatch; xbuf unused); with `y_top1` as well, GEMM2 writes gate * row to
+// y[token] (fused top-1 combine; ybuf's routed rows are not written).
 int run_ffn(const moe_cfg* c, const Layout& L, const void* xbuf, const void* x, const int32_t* off,
-            const moe_weights* w, void* ybuf, void* ws, cudaStream_t s, const moe_event_t* ev_mid = nullptr) {
+            const moe_weights* w, void* ybuf, void* ws, cudaStream_t s, const moe_event_t* ev_mid = nullptr,
+            const int32_t* rowtok = nullptr, void* y_top1 = nullptr, const float* gates_top1 = nullptr) {
   void* hbuf = at<void>(ws, L.hbuf);
   const bool sh = c->n_shared != 0;
   if (c->dtype == MOE_DTYPE_BF16) {
@@ -245,6 +249,11 @@ int run_ffn(const moe_cfg* c, const Layout& L, const void* xbuf, const void* x, 
     g1.n_shared = c->n_shared;
     g1.epi = c->act;
     g1.status = at<DevStatus>(ws, L.status);
+    if (rowtok != nullptr) {
+      g1.a_routed = nullptr;
+      g1.gather_src = x;
+      g1.gather_idx = rowtok;
+    }
     cudaError_t e = launch_grouped_gemm(g1, s);
     if (e != cudaSuccess) return MOE_ECUDA;
     if (record(ev_mid, 0, s) != MOE_OK) return MOE_ECUDA;
@@ -259,6 +268,13 @@ int run_ffn(const moe_cfg* c, const Layout& L, const void* xbuf, const void* x, 
     g2.K = c->F;
     g2.Nw = c->H;
     g2.epi = -1;
+    g2.gather_src = nullptr;
+    g2.gather_idx = nullptr;
+    if (y_top1 != nullptr) {
+      g2.gather_idx = rowtok;
+      g2.scatter_dst = y_top1;
+      g2.scatter_gate = gates_top1;
+    }
     return cuda_status(launch_grouped_gemm(g2, s));
   }
   FfnF32Params f1{};
@@ -467,6 +483,11 @@ int moe_layer_fwd(const moe_cfg* cfg, const void* x, const float* wg, const floa
                       at<int32_t>(ws, L.rowtok), ws, s, aux)) != MOE_OK)
     return st;
   if ((st = record(stage_events, 2, s)) != MOE_OK) return st;
+  // bf16: dispatch fused into the first contraction's A loads and, for top-1
+  // without a shared expert, the combine fused into the second's epilogue
+  const bool fuse = cfg->dtype == MOE_DTYPE_BF16 && !(cfg->flags & MOE_FLAG_UNFUSED);
+  const bool fuse_combine = fuse && cfg->k == 1 && cfg->n_shared == 0;
+  int32_t* rowtok = at<int32_t>(ws, L.rowtok);
   PermuteParams pp = permute_params(cfg, L);
   pp.ids = ids;
   pp.slot = slot;
@@ -474,14 +495,15 @@ int moe_layer_fwd(const moe_cfg* cfg, const void* x, const float* wg, const floa
   pp.expert_offset = off;
   pp.src = x;
   pp.dst = xbuf;
-  if (launch_dispatch(pp, s) != cudaSuccess) return MOE_ECUDA;
+  if (!fuse && launch_dispatch(pp, s) != cudaSuccess) return MOE_ECUDA;
   if ((st = record(stage_events, 3, s)) != MOE_OK) return st;
-  if ((st = run_ffn(cfg, L, xbuf, x, off, w, ybuf, ws, s, stage_events ? stage_events + 4 : nullptr)) != MOE_OK)
+  if ((st = run_ffn(cfg, L, xbuf, x, off, w, ybuf, ws, s, stage_events ? stage_events + 4 : nullptr,
+                    fuse ? rowtok : nullptr, fuse_combine ? y : nullptr, fuse_combine ? gates : nullptr)) != MOE_OK)
     return st;
   if ((st = record(stage_events, 5, s)) != MOE_OK) return st;
   pp.src = ybuf;
   pp.dst = y;
-  if (launch_combine(pp, s) != cudaSuccess) return MOE_ECUDA;
+  if ((fuse_combine ? launch_zero_dropped(pp, s) : launch_combine(pp, s)) != cudaSuccess) return MOE_ECUDA;
   if ((st = record(stage_events, 6, s)) != MOE_OK) return st;
   if (expert_count != nullptr && cfg->E > 0)
     if (cudaMemcpyAsync(expert_count, at<int32_t>(ws, L.ecount), sizeof(int32_t) * cfg->E, cudaMemcpyDeviceToDevice,

@@ -166,4 +166,26 @@ cudaError_t launch_combine(const PermuteParams& p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+// With the combine fused into the second GEMM (top-1, no shared expert), the
+// GEMM writes the rows of kept tokens; this writes y[t] = 0 for every token
+// whose choices were all dropped.  One warp per token.
+__global__ void __launch_bounds__(kPermWarps * 32) zero_dropped_kernel(PermuteParams p) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * kPermWarps + (threadIdx.x >> 5);
+  if (t >= p.T) return;
+  bool any = false;
+  for (int r = 0; r < p.k; ++r) any |= p.slot[t * p.k + r] >= 0 && p.ids[t * p.k + r] >= 0;
+  if (any) return;
+  const int64_t rowbytes = (int64_t)p.H * p.elem_bytes;
+  char* y = static_cast<char*>(p.dst) + t * rowbytes;
+  for (int64_t v = lane; v < rowbytes / 16; v += 32) st_v4(y + v * 16, make_int4(0, 0, 0, 0));
+}
+
+cudaError_t launch_zero_dropped(const PermuteParams& p, cudaStream_t stream) {
+  if (p.T == 0) return cudaSuccess;
+  const unsigned grid = (unsigned)((p.T + kPermWarps - 1) / kPermWarps);
+  zero_dropped_kernel<<<grid, kPermWarps * 32, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
 }  // namespace moe

@@ -91,13 +91,18 @@ enum { MOE_DROP_POSITION = 0, MOE_DROP_PROBS = 1 };
 enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
 /* moe_cfg.flags
  * KEEP_LOGITS: moe_layer_fwd also stores fp32 logits in the workspace.
+ * UNFUSED: moe_layer_fwd runs dispatch and combine as separate kernels (the
+ *   pages' literal sequence, filling xbuf and ybuf).  By default, for bf16,
+ *   the first expert contraction gathers its rows straight from x (xbuf is not
+ *   written) and, for k == 1 without a shared expert, the second contraction
+ *   writes gate * row to y[token] (ybuf's routed rows are not written).
  * RANDOM_SECOND: GShard top-2 ([EP] router section: the second expert receives
  *   the token at random, according to its weight).  For k >= 2 the rank-1
  *   choice of token t is dispatched iff uniform[t] < 2 * gate[t,1], with
  *   uniform [T] fp32 in [0,1) supplied by the caller; otherwise its id becomes
  *   -1 and its gate 0 (it takes no slot and adds nothing to y).  The aux loss
  *   still counts it as selected.  No effect when k == 1. */
-enum { MOE_FLAG_KEEP_LOGITS = 1, MOE_FLAG_RANDOM_SECOND = 2 };
+enum { MOE_FLAG_KEEP_LOGITS = 1, MOE_FLAG_RANDOM_SECOND = 2, MOE_FLAG_UNFUSED = 4 };
 
 /* Layer configuration.  Limits of this build: 1 <= E <= 1024, 1 <= k <= min(E,16),
  * H and F multiples of 8, n_shared in {0,1}, T >= 0 with T*k < 2^31 and every
@@ -149,9 +154,9 @@ typedef struct moe_ws_views {
   int32_t* expert_offset;  /* [E+2] first row of each expert's block; [E] shared block; [E+1] end */
   int32_t* row_token;      /* [rows_max] source token of each row, -1 for padding rows */
   float* logits;           /* [T,E] fp32 logits (written only with MOE_FLAG_KEEP_LOGITS) */
-  void* xbuf;              /* [rows_max, H] dispatched rows */
+  void* xbuf;              /* [rows_max, H] dispatched rows (moe_layer_fwd: MOE_FLAG_UNFUSED or fp32 only) */
   void* hbuf;              /* [rows_max, F] expert activations (bf16; fp32 for MOE_DTYPE_F32) */
-  void* ybuf;              /* [rows_max, H] un-gated expert outputs */
+  void* ybuf;              /* [rows_max, H] un-gated expert outputs (routed rows not written by a fused top-1 combine) */
   int64_t rows_max;
 } moe_ws_views;
 
@@ -269,15 +274,17 @@ MOE_API int moe_combine(const moe_cfg* cfg, const void* ybuf, const int32_t* ids
 MOE_API int moe_aux_loss(const moe_cfg* cfg, const void* ws, float* aux, moe_stream_t stream);
 
 /* The whole layer: route -> assign slots -> dispatch -> expert FFN -> combine,
- * plus the aux loss, on `stream`.  y [T,H] (cfg->dtype) and aux (one fp32, two
+ * plus the aux loss, on `stream` (dispatch and the top-1 combine fused into the
+ * expert contractions unless MOE_FLAG_UNFUSED; see the flags).  y [T,H] (cfg->dtype) and aux (one fp32, two
  * with the z-loss: see moe_aux_loss) are device outputs; uniform is moe_route's;
  * expert_count [E] (optional, NULL to skip) counts dispatched choices.  The
  * intermediates stay in `ws` (see moe_workspace_views).  `stage_events`, if
  * non-NULL, is an array of MOE_N_STAGE_EVENTS events recorded on `stream` before
  * the router and after each of: router, slots (which here also reduce the aux
- * loss), dispatch, expert FFN first contraction (with the activation), expert
- * FFN second contraction, combine, and the end of the call (the copy of
- * expert_count, if requested). */
+ * loss), dispatch (an empty interval when fused), expert FFN first contraction
+ * (with the activation), expert FFN second contraction, combine (when fused:
+ * the zeroing of fully dropped tokens' rows), and the end of the call (the copy
+ * of expert_count, if requested). */
 enum { MOE_N_STAGE_EVENTS = 8 };
 MOE_API int moe_layer_fwd(const moe_cfg* cfg, const void* x, const float* wg, const float* logit_add,
                           const float* uniform, const moe_weights* w, void* y, float* aux, int32_t* expert_count,

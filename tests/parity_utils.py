@@ -114,8 +114,12 @@ def condition_uniform(shape: synth.LayerShape, inp: dict, margin: float = 1e-4) 
     inp["uniform"].copy_(torch.from_numpy(np.clip(u, 0.0, np.nextafter(1.0, 0.0)).astype(np.float32)))
 
 
-def run_layer(shape: synth.LayerShape, inp: dict, keep_logits=True, ws=None):
-    cfg = B.make_cfg(shape, flags=B.MOE_FLAG_KEEP_LOGITS if keep_logits else 0)
+def run_layer(shape: synth.LayerShape, inp: dict, keep_logits=True, ws=None, unfused=False):
+    """One moe_layer_fwd call.  By default dispatch (and, for top-1 without a
+    shared expert, the combine) run fused into the expert contractions;
+    unfused=True runs them as separate kernels and fills xbuf / ybuf."""
+    flags = (B.MOE_FLAG_KEEP_LOGITS if keep_logits else 0) | (B.MOE_FLAG_UNFUSED if unfused else 0)
+    cfg = B.make_cfg(shape, flags=flags)
     if ws is None:
         ws = B.alloc_workspace(cfg)
     T, H = shape.T, shape.H
@@ -126,7 +130,9 @@ def run_layer(shape: synth.LayerShape, inp: dict, keep_logits=True, ws=None):
     st = B.moe_sync_status(ws)
     assert st == B.MOE_OK, f"device status {st}: {B.strerror(st)}"
     out = B.workspace_tensors(cfg, ws)
-    out.update(y=y, aux=aux, expert_count_out=ecount, cfg=cfg, ws=ws)
+    fused = shape.dtype == synth.DTYPE_BF16 and not unfused
+    out.update(y=y, aux=aux, expert_count_out=ecount, cfg=cfg, ws=ws, fused_dispatch=fused,
+               fused_combine=fused and shape.k == 1 and shape.n_shared == 0)
     return out
 
 
@@ -166,10 +172,11 @@ def check_layer(shape: synth.LayerShape, inp: dict, out: dict, tokens=None, logi
         assert abs(zl - ref["zloss"]) <= 1e-5 * abs(ref["zloss"]) + 1e-12, (zl, ref["zloss"])
     else:
         assert np.isnan(out["aux"][1].item()), "aux[1] written without a z-loss"
-    # 3. dispatch: every kept row is a bitwise copy of its token's x row
+    # 3. dispatch: every kept row is a bitwise copy of its token's x row (when
+    # dispatch is fused there is no dispatched buffer: the GEMM reads x itself)
     rt = ref["row_token"]
     kept_rows = np.nonzero(rt[:int(ref["offsets"][E])] >= 0)[0]
-    if len(kept_rows):
+    if len(kept_rows) and not out.get("fused_dispatch"):
         sel = torch.from_numpy(kept_rows).cuda()
         src = torch.from_numpy(rt[kept_rows].astype(np.int64)).cuda()
         assert torch.equal(out["xbuf"][sel], inp["x"][src]), "dispatched rows differ from x"
@@ -180,6 +187,10 @@ def check_layer(shape: synth.LayerShape, inp: dict, out: dict, tokens=None, logi
     else:
         close = assert_f32_close
     yb = out["ybuf"]
+    if out.get("fused_combine"):
+        # the second contraction wrote gate * row straight to y: only the shared
+        # rows (none here) would remain in ybuf
+        ref["rows"] = {key: v for key, v in ref["rows"].items() if key[1] < 0}
     if ref["rows"]:
         keys = list(ref["rows"].keys())
         ridx = []

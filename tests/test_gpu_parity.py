@@ -43,11 +43,35 @@ SMALL = {
 
 @pytest.mark.parametrize("name", list(SMALL))
 @pytest.mark.parametrize("seed", [1, 2])
-def test_layer_small(name, seed):
+@pytest.mark.parametrize("mode", ["fused", "unfused"])
+def test_layer_small(name, seed, mode):
     shape = SMALL[name]
     inp = synth.make_inputs(shape, seed=seed, device="cuda")
-    out = run_layer(shape, inp)
+    out = run_layer(shape, inp, unfused=mode == "unfused")
     check_layer(shape, inp, out)
+
+
+@pytest.mark.parametrize("name", ["switch_top1", "gshard_top2", "wideep", "ds_k4_cf05"])
+def test_fused_matches_unfused(name):
+    """Fusing dispatch into the first contraction changes nothing but where A
+    comes from: routing, slots, h and the expert outputs are bitwise equal.  The
+    fused top-1 combine rounds gate * accumulator once instead of twice."""
+    shape = SMALL[name]
+    inp = synth.make_inputs(shape, seed=9, device="cuda")
+    a = run_layer(shape, inp)
+    snap = {n: a[n].clone() for n in ("ids", "slot", "expert_offset", "y", "hbuf", "ybuf")}
+    b = run_layer(shape, inp, unfused=True)
+    used = int(b["expert_offset"][-1])
+    live = b["row_token"][:used] >= 0
+    for n in ("ids", "slot", "expert_offset"):
+        assert torch.equal(snap[n], b[n]), n
+    assert torch.equal(snap["hbuf"][:used][live], b["hbuf"][:used][live])
+    if a["fused_combine"]:
+        ya, yb = snap["y"].float(), b["y"].float()
+        assert ((ya - yb).abs() <= 2.0 ** -7 * yb.abs()).all()   # one bf16 rounding apart
+    else:
+        assert torch.equal(snap["ybuf"][:used][live], b["ybuf"][:used][live])
+        assert torch.equal(snap["y"], b["y"])
 
 
 @pytest.mark.parametrize("name", ["switch_top1", "gshard_top2", "wideep", "ds_k4_cf05"])
