@@ -116,9 +116,11 @@ __device__ __forceinline__ float act_silu(float z) { return z * rcp_approx(1.0f 
 constexpr long long kWaitCycles = 2000000000LL;
 
 // Host: raise a kernel's dynamic shared memory limit to at least `bytes` on the
-// current device.  Remembers, per (kernel, device), the largest limit set.
+// current device (the default limit counts the kernel's static shared memory
+// too, so any non-zero request is set explicitly).  Remembers, per (kernel,
+// device), the largest limit set.
 inline cudaError_t ensure_smem_ptr(const void* k, size_t bytes) {
-  if (bytes <= 48 * 1024) return cudaSuccess;
+  if (bytes == 0) return cudaSuccess;
   int dev = 0;
   cudaGetDevice(&dev);
   struct Entry { const void* k; int dev; size_t bytes; };
