@@ -48,13 +48,16 @@ SETTABLE = {"score": int, "renorm": int, "z_coef": float, "random_second": int, 
 def launches_per_step(shape) -> int:
     """Kernels one moe_layer_fwd call launches: router 3 for bf16 x (weight split,
     logits GEMM, softmax/top-k) or 1 for fp32 x; slots 4 (aux loss folded in),
-    plus the per-expert select of the "probs" policy; dispatch 1 for fp32 x (for
-    bf16 it is fused into the first expert contraction); expert FFN 2; combine 1
-    (for bf16 top-1 without a shared expert: the zeroing of dropped rows)."""
+    plus the per-expert select of the "probs" policy; dispatch 1 (0 when fused
+    into the first expert contraction: bf16 with T*k <= 256*E); expert FFN 2;
+    combine 1 (0 when fused into the second: the fused case with top-1 and no
+    shared expert)."""
     router = 3 if shape.dtype == 1 else 1
     slots = 4 + (1 if shape.drop_policy == 1 and shape.cap_mode == 0 else 0)
-    dispatch = 0 if shape.dtype == 1 else 1
-    return router + slots + dispatch + 2 + 1
+    fused = shape.dtype == 1 and shape.T * shape.k <= 256 * shape.E
+    dispatch = 0 if fused else 1
+    combine = 0 if fused and shape.k == 1 and shape.n_shared == 0 else 1
+    return router + slots + dispatch + 2 + combine
 
 
 def parse_args():

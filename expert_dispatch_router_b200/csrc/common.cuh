@@ -111,6 +111,32 @@ __device__ __forceinline__ float act_gelu(float z) {
 // SiLU: z * sigmoid(z) = z / (1 + exp(-z)).
 __device__ __forceinline__ float act_silu(float z) { return z * rcp_approx(1.0f + __expf(-z)); }
 
+// Programmatic dependent launch.  The layer's kernels are launched so that the
+// next kernel on the stream may be scheduled while this one drains: every such
+// kernel calls pdl_wait() before it touches global memory that an earlier
+// launch writes or reads (griddepcontrol.wait returns once the preceding grid
+// has completed and its writes are visible), and pdl_trigger() to let the next
+// grid launch early; its CTAs then block in their own pdl_wait().
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Host: launch `kern` with programmatic stream serialization allowed.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // Upper bound on the cycles any bounded wait spins before it gives up (~1 s
 // at the B200's boost clock).  Normal waits in these kernels last microseconds.
 constexpr long long kWaitCycles = 2000000000LL;

@@ -21,6 +21,8 @@ __device__ __forceinline__ int find_group(const int32_t* off, int ngroups, int64
 }
 
 __global__ void __launch_bounds__(kFThreads) ffn_f32_kernel(FfnF32Params p) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float As[kFBK][kFBM + 4];
   __shared__ float Bs[2][kFBK][kFBN + 4];
   const int64_t row0 = (int64_t)blockIdx.x * kFBM;
@@ -107,7 +109,7 @@ cudaError_t launch_activation_eval(int act, const float* z, const float* u, floa
 cudaError_t launch_ffn_f32(const FfnF32Params& p, cudaStream_t stream) {
   if (p.rows_max == 0) return cudaSuccess;
   dim3 grid((unsigned)((p.rows_max + kFBM - 1) / kFBM), (unsigned)((p.N + kFBN - 1) / kFBN));
-  ffn_f32_kernel<<<grid, kFThreads, 0, stream>>>(p);
+  launch_pdl(ffn_f32_kernel, grid, kFThreads, 0, stream, p);
   return cudaGetLastError();
 }
 

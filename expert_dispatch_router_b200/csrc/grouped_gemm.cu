@@ -79,9 +79,12 @@ struct KParams {
   // (warp 0 issues cp.async with the 128-byte swizzle applied by hand)
   const __nv_bfloat16* gsrc;
   const int32_t* gidx;
-  // fused top-1 combine: routed rows stored to sdst[gidx[row]] * sgate[gidx[row]]
+  // fused top-1 combine: routed rows stored to sdst[gidx[row]] * sgate[gidx[row]];
+  // warp 0's idle lanes also zero sdst[t] for every token t with sslot[t] < 0
   __nv_bfloat16* sdst;
   const float* sgate;
+  const int32_t* sslot;
+  int64_t sT;
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -272,6 +275,7 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();                                    // inputs of earlier launches are complete from here on
 
   const int64_t rows_used = grouped ? min((int64_t)p.off[ngroups], p.rows_max) : p.rows_static;
   const int64_t n_mtiles = (rows_used + BM - 1) / BM;
@@ -297,6 +301,14 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
   const int n_stages = min(MAX_STAGES, RING_BYTES / stage_bytes);
 
   if (warp == 0) {
+    if (SCATTER && lane > 0) {
+      // fused top-1 combine: rows of fully dropped tokens are zero
+      const int64_t nthr = (int64_t)gridDim.x * 31;
+      const int nvec = p.N_out / 8;
+      for (int64_t t = (int64_t)blockIdx.x * 31 + (lane - 1); t < p.sT; t += nthr)
+        if (__ldg(p.sslot + t) < 0)
+          for (int v = 0; v < nvec; ++v) st_v4(p.sdst + t * p.N_out + 8 * v, make_int4(0, 0, 0, 0));
+    }
     // ---------------- TMA producer
     if (lane == 0) {
       int stage = 0;
@@ -510,15 +522,29 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
             }
           }
         } else if (SCATTER) {
-          if (st < 0) continue;
-          __nv_bfloat16* dst = p.sdst + (int64_t)st * p.N_out + col;
+          // the warp's 32 rows x 32 columns go through its staging buffer (same
+          // swizzle as below), then out row by row: lanes 4j..4j+3 write the 64
+          // bytes of one row, eight rows per store instruction
+          __syncwarp();                              // the previous chunk's reads are done
 #pragma unroll
           for (int q = 0; q < 4; ++q)
-            if (8 * q < chunk && col + 8 * q < p.N_out)
-              st_v4(dst + 8 * q, make_int4((int)pack_bf16(sg * v[8 * q + 0], sg * v[8 * q + 1]),
-                                           (int)pack_bf16(sg * v[8 * q + 2], sg * v[8 * q + 3]),
-                                           (int)pack_bf16(sg * v[8 * q + 4], sg * v[8 * q + 5]),
-                                           (int)pack_bf16(sg * v[8 * q + 6], sg * v[8 * q + 7])));
+            st_shared_v4(stage_out + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4),
+                         pack_bf16(sg * v[8 * q + 0], sg * v[8 * q + 1]), pack_bf16(sg * v[8 * q + 2], sg * v[8 * q + 3]),
+                         pack_bf16(sg * v[8 * q + 4], sg * v[8 * q + 5]), pack_bf16(sg * v[8 * q + 6], sg * v[8 * q + 7]));
+          __syncwarp();
+          const int j = lane & 3;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int r = 8 * q + (lane >> 2);
+            const int tr = __shfl_sync(0xffffffffu, st, r);
+            if (tr >= 0 && 8 * j < chunk && col + 8 * j < p.N_out) {
+              int4 val;
+              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
+                           : "r"(stage_out + r * 64 + ((j ^ ((r >> 1) & 3)) << 4)));
+              st_v4(p.sdst + (int64_t)tr * p.N_out + col + 8 * j, val);
+            }
+          }
         } else {
           // bf16: this warp's 32 rows x 32 columns go through its staging buffer
           // (16-byte chunk j of row r at chunk j ^ ((r >> 1) & 3): the TMA 64-byte
@@ -549,6 +575,9 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // The next launch may start only now: its CTAs could otherwise sit on this
+  // SM beside the GEMM while they wait for it.
+  pdl_trigger();
   if (warp == 1) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem_base), "r"(TMEM_COLS) : "memory");
   }
@@ -658,7 +687,7 @@ static cudaError_t launch_variant(KParams& k, int grid, cudaStream_t stream) {
   auto kern = grouped_gemm_kernel<GATHER, SCATTER>;
   cudaError_t e = ensure_smem(kern, SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  kern<<<grid, GATHER ? THREADS_GATHER : THREADS, SMEM_BYTES, stream>>>(k);
+  launch_pdl(kern, grid, GATHER ? THREADS_GATHER : THREADS, SMEM_BYTES, stream, k);
   return cudaGetLastError();
 }
 
@@ -709,6 +738,8 @@ cudaError_t launch_grouped_gemm(const GemmParams& p, cudaStream_t stream) {
   k.gidx = p.gather_idx;
   k.sdst = static_cast<__nv_bfloat16*>(p.scatter_dst);
   k.sgate = p.scatter_gate;
+  k.sslot = p.scatter_slot;
+  k.sT = p.T;
   return launch_kernel(k, (p.rows_max / BM) * ((p.Nw + box_n - 1) / box_n), stream);
 }
 
@@ -719,6 +750,8 @@ cudaError_t launch_grouped_gemm(const GemmParams& p, cudaStream_t stream) {
 // x_h * plane_j(w) is exact in fp32 and the tensor core's fp32 accumulation
 // gives fp32 logits of the same quality as an fp32 dot product.
 __global__ void split_router_weight_kernel(const float* wg, __nv_bfloat16* planes, int E, int H, int Hp) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t n = (int64_t)E * Hp;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     const int e = (int)(i / Hp), h = (int)(i % Hp);
@@ -746,7 +779,7 @@ cudaError_t launch_router_gemm(const void* x, const float* wg, void* planes, flo
   {
     const int64_t n = (int64_t)E * Hp;
     const int64_t blocks = (n + 255) / 256;
-    split_router_weight_kernel<<<(unsigned)(blocks < 2048 ? blocks : 2048), 256, 0, stream>>>(
+    launch_pdl(split_router_weight_kernel, (unsigned)(blocks < 2048 ? blocks : 2048), 256, 0, stream, 
         wg, static_cast<__nv_bfloat16*>(planes), E, H, Hp);
   }
   const int bn = E >= 256 ? 256 : (E + 15) / 16 * 16;

@@ -88,8 +88,6 @@ struct PermuteParams {
 };
 cudaError_t launch_dispatch(const PermuteParams& p, cudaStream_t stream);
 cudaError_t launch_combine(const PermuteParams& p, cudaStream_t stream);
-// y[t] = 0 for every token with no kept choice (dst = y).
-cudaError_t launch_zero_dropped(const PermuteParams& p, cudaStream_t stream);
 
 // fp32 SIMT grouped FFN (one GEMM per call).
 struct FfnF32Params {
@@ -124,9 +122,11 @@ struct GemmParams {
   const void* gather_src;
   const int32_t* gather_idx;
   // Fused top-1 combine: routed output rows go to scatter_dst[token] scaled by
-  // scatter_gate[token] instead of d (no shared expert, k = 1).
+  // scatter_gate[token] instead of d (no shared expert, k = 1); rows of tokens
+  // with scatter_slot[token] < 0 (dropped) are zeroed by the same launch.
   void* scatter_dst;
   const float* scatter_gate;
+  const int32_t* scatter_slot;
 };
 cudaError_t launch_grouped_gemm(const GemmParams& p, cudaStream_t stream);
 

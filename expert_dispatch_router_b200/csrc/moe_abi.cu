@@ -228,7 +228,8 @@ int record(const moe_event_t* ev, int i, cudaStream_t s) {
 // y[token] (fused top-1 combine; ybuf's routed rows are not written).
 int run_ffn(const moe_cfg* c, const Layout& L, const void* xbuf, const void* x, const int32_t* off,
             const moe_weights* w, void* ybuf, void* ws, cudaStream_t s, const moe_event_t* ev_mid = nullptr,
-            const int32_t* rowtok = nullptr, void* y_top1 = nullptr, const float* gates_top1 = nullptr) {
+            const int32_t* rowtok = nullptr, void* y_top1 = nullptr, const float* gates_top1 = nullptr,
+            const int32_t* slot_top1 = nullptr) {
   void* hbuf = at<void>(ws, L.hbuf);
   const bool sh = c->n_shared != 0;
   if (c->dtype == MOE_DTYPE_BF16) {
@@ -274,6 +275,7 @@ int run_ffn(const moe_cfg* c, const Layout& L, const void* xbuf, const void* x, 
       g2.gather_idx = rowtok;
       g2.scatter_dst = y_top1;
       g2.scatter_gate = gates_top1;
+      g2.scatter_slot = slot_top1;
     }
     return cuda_status(launch_grouped_gemm(g2, s));
   }
@@ -483,9 +485,14 @@ int moe_layer_fwd(const moe_cfg* cfg, const void* x, const float* wg, const floa
                       at<int32_t>(ws, L.rowtok), ws, s, aux)) != MOE_OK)
     return st;
   if ((st = record(stage_events, 2, s)) != MOE_OK) return st;
-  // bf16: dispatch fused into the first contraction's A loads and, for top-1
-  // without a shared expert, the combine fused into the second's epilogue
-  const bool fuse = cfg->dtype == MOE_DTYPE_BF16 && !(cfg->flags & MOE_FLAG_UNFUSED);
+  // bf16 with at most two 128-row blocks per expert on average: the expert
+  // contractions stream weights from HBM, so dispatch is fused into the first
+  // one's A loads and, for top-1 without a shared expert, the combine into the
+  // second one's epilogue.  With more rows per expert the contractions are fed
+  // from L2, where the TMA loads of a dispatched buffer feed faster than
+  // per-row cp.async gathers.
+  const bool fuse = cfg->dtype == MOE_DTYPE_BF16 && !(cfg->flags & MOE_FLAG_UNFUSED) &&
+                    cfg->T * cfg->k <= 2 * kRowPad * (int64_t)cfg->E;
   const bool fuse_combine = fuse && cfg->k == 1 && cfg->n_shared == 0;
   int32_t* rowtok = at<int32_t>(ws, L.rowtok);
   PermuteParams pp = permute_params(cfg, L);
@@ -498,12 +505,13 @@ int moe_layer_fwd(const moe_cfg* cfg, const void* x, const float* wg, const floa
   if (!fuse && launch_dispatch(pp, s) != cudaSuccess) return MOE_ECUDA;
   if ((st = record(stage_events, 3, s)) != MOE_OK) return st;
   if ((st = run_ffn(cfg, L, xbuf, x, off, w, ybuf, ws, s, stage_events ? stage_events + 4 : nullptr,
-                    fuse ? rowtok : nullptr, fuse_combine ? y : nullptr, fuse_combine ? gates : nullptr)) != MOE_OK)
+                    fuse ? rowtok : nullptr, fuse_combine ? y : nullptr, fuse_combine ? gates : nullptr,
+                    fuse_combine ? slot : nullptr)) != MOE_OK)
     return st;
   if ((st = record(stage_events, 5, s)) != MOE_OK) return st;
   pp.src = ybuf;
   pp.dst = y;
-  if ((fuse_combine ? launch_zero_dropped(pp, s) : launch_combine(pp, s)) != cudaSuccess) return MOE_ECUDA;
+  if (!fuse_combine && launch_combine(pp, s) != cudaSuccess) return MOE_ECUDA;
   if ((st = record(stage_events, 6, s)) != MOE_OK) return st;
   if (expert_count != nullptr && cfg->E > 0)
     if (cudaMemcpyAsync(expert_count, at<int32_t>(ws, L.ecount), sizeof(int32_t) * cfg->E, cudaMemcpyDeviceToDevice,

@@ -38,6 +38,8 @@ __device__ __forceinline__ void token_rows(const PermuteParams& p, int64_t t, in
 
 template <int KM, int U>
 __global__ void __launch_bounds__(kPermWarps * 32) dispatch_kernel(PermuteParams p) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t t = (int64_t)blockIdx.x * kPermWarps + (threadIdx.x >> 5);
   if (t >= p.T) return;
@@ -71,6 +73,8 @@ __global__ void __launch_bounds__(kPermWarps * 32) dispatch_kernel(PermuteParams
 
 template <typename ET, int KM, int U>
 __global__ void __launch_bounds__(kPermWarps * 32) combine_kernel(PermuteParams p) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int NE = 16 / sizeof(ET);
   const int lane = threadIdx.x & 31;
   const int64_t t = (int64_t)blockIdx.x * kPermWarps + (threadIdx.x >> 5);
@@ -129,13 +133,13 @@ __global__ void __launch_bounds__(kPermWarps * 32) combine_kernel(PermuteParams 
 template <int KM>
 static void launch_dispatch_km(const PermuteParams& p, unsigned grid, cudaStream_t s) {
   constexpr int U = KM >= 8 ? 2 : 4;
-  dispatch_kernel<KM, U><<<grid, kPermWarps * 32, 0, s>>>(p);
+  launch_pdl(dispatch_kernel<KM, U>, grid, kPermWarps * 32, 0, s, p);
 }
 
 template <typename ET, int KM>
 static void launch_combine_km(const PermuteParams& p, unsigned grid, cudaStream_t s) {
   constexpr int U = KM >= 16 ? 1 : KM >= 8 ? 2 : 4;
-  combine_kernel<ET, KM, U><<<grid, kPermWarps * 32, 0, s>>>(p);
+  launch_pdl(combine_kernel<ET, KM, U>, grid, kPermWarps * 32, 0, s, p);
 }
 
 cudaError_t launch_dispatch(const PermuteParams& p, cudaStream_t stream) {
@@ -163,28 +167,6 @@ cudaError_t launch_combine(const PermuteParams& p, cudaStream_t stream) {
   const unsigned grid = (unsigned)((p.T + kPermWarps - 1) / kPermWarps);
   if (p.elem_bytes == 2) launch_combine_t<__nv_bfloat16>(p, grid, stream);
   else launch_combine_t<float>(p, grid, stream);
-  return cudaGetLastError();
-}
-
-// With the combine fused into the second GEMM (top-1, no shared expert), the
-// GEMM writes the rows of kept tokens; this writes y[t] = 0 for every token
-// whose choices were all dropped.  One warp per token.
-__global__ void __launch_bounds__(kPermWarps * 32) zero_dropped_kernel(PermuteParams p) {
-  const int lane = threadIdx.x & 31;
-  const int64_t t = (int64_t)blockIdx.x * kPermWarps + (threadIdx.x >> 5);
-  if (t >= p.T) return;
-  bool any = false;
-  for (int r = 0; r < p.k; ++r) any |= p.slot[t * p.k + r] >= 0 && p.ids[t * p.k + r] >= 0;
-  if (any) return;
-  const int64_t rowbytes = (int64_t)p.H * p.elem_bytes;
-  char* y = static_cast<char*>(p.dst) + t * rowbytes;
-  for (int64_t v = lane; v < rowbytes / 16; v += 32) st_v4(y + v * 16, make_int4(0, 0, 0, 0));
-}
-
-cudaError_t launch_zero_dropped(const PermuteParams& p, cudaStream_t stream) {
-  if (p.T == 0) return cudaSuccess;
-  const unsigned grid = (unsigned)((p.T + kPermWarps - 1) / kPermWarps);
-  zero_dropped_kernel<<<grid, kPermWarps * 32, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

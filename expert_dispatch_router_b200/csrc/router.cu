@@ -196,6 +196,8 @@ constexpr int router_smem_floats() {
 
 template <int EJ, int TW, typename XT>
 __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterParams p) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int EP = 32 * EJ;
   constexpr int BT = kRouterWarps * TW;
   constexpr int WS = EP + 4;
@@ -327,6 +329,8 @@ constexpr int kLogitWarps = 8;
 
 template <int EJ>
 __global__ void __launch_bounds__(kLogitWarps * 32, EJ <= 4 ? 3 : 1) route_logits_kernel(RouterParams p, int bt) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(16) float smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t t0 = (int64_t)blockIdx.x * bt;
@@ -372,12 +376,12 @@ static cudaError_t launch_router_ej(const RouterParams& p, bool bf16, cudaStream
     auto k = router_kernel<EJ, TW, __nv_bfloat16>;
     cudaError_t e = ensure_smem(k, smem);
     if (e != cudaSuccess) return e;
-    k<<<grid, kRouterThreads, smem, stream>>>(p);
+    launch_pdl(k, grid, kRouterThreads, smem, stream, p);
   } else {
     auto k = router_kernel<EJ, TW, float>;
     cudaError_t e = ensure_smem(k, smem);
     if (e != cudaSuccess) return e;
-    k<<<grid, kRouterThreads, smem, stream>>>(p);
+    launch_pdl(k, grid, kRouterThreads, smem, stream, p);
   }
   return cudaGetLastError();
 }
@@ -390,7 +394,7 @@ static cudaError_t launch_route_logits_ej(const RouterParams& p, cudaStream_t st
   auto k = route_logits_kernel<EJ>;
   cudaError_t e = ensure_smem(k, smem);
   if (e != cudaSuccess) return e;
-  k<<<grid, kLogitWarps * 32, smem, stream>>>(p, bt);
+  launch_pdl(k, grid, kLogitWarps * 32, smem, stream, p, bt);
   return cudaGetLastError();
 }
 
@@ -424,6 +428,8 @@ __global__ void __launch_bounds__(kAuxWarps * 32) aux_kernel(const float* psum_p
                                                              const float* zsum_part, int nblk, int E, int64_t T,
                                                              int k, float alpha, float z_coef, double* term,
                                                              unsigned* counter, float* aux) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ double sh[kAuxWarps * 32];
   __shared__ bool last;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
@@ -484,7 +490,7 @@ cudaError_t launch_aux(const float* psum_part, const int32_t* cnt_part, const fl
                        int64_t T, int k, float alpha, float z_coef, double* term, float* aux, cudaStream_t stream) {
   unsigned* counter = reinterpret_cast<unsigned*>(term + E);
   const int grid = T == 0 ? 1 : (E + kAuxWarps - 1) / kAuxWarps;
-  aux_kernel<<<grid, kAuxWarps * 32, 0, stream>>>(psum_part, cnt_part, zsum_part, nblk, E, T, k, alpha, z_coef,
+  launch_pdl(aux_kernel, grid, kAuxWarps * 32, 0, stream, psum_part, cnt_part, zsum_part, nblk, E, T, k, alpha, z_coef,
                                                   term, counter, aux);
   return cudaGetLastError();
 }

@@ -41,6 +41,8 @@ __device__ __forceinline__ int load_assignment(const SlotParams& p, int64_t a, i
 }
 
 __global__ void __launch_bounds__(kSlotThreads) slot_count_kernel(SlotParams p, int nchunk) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int hist[];
   const int64_t A = p.T * p.k;
   for (int e = threadIdx.x; e < p.E; e += kSlotThreads) hist[e] = 0;
@@ -89,6 +91,8 @@ __device__ __forceinline__ int block_scan_excl(int v, int* sh, int& total) {
 }
 
 __global__ void __launch_bounds__(kSlotThreads) slot_scan_kernel(SlotParams p, int nchunk) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int sh[kSlotWarps];
   const int e = blockIdx.x;
   int* row = p.chunk_cnt + (int64_t)e * nchunk;
@@ -136,6 +140,8 @@ __global__ void __launch_bounds__(kSlotThreads) slot_scan_kernel(SlotParams p, i
 }
 
 __global__ void __launch_bounds__(1024) slot_offsets_kernel(SlotParams p) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int sh[32];
   __shared__ int sh_off[kMaxE + 2];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -193,6 +199,8 @@ __global__ void __launch_bounds__(1024) slot_offsets_kernel(SlotParams p) {
 }
 
 __global__ void __launch_bounds__(kSlotThreads) slot_rank_kernel(SlotParams p, int nchunk) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int wcnt[];                 // [warps][E]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t A = p.T * p.k;
@@ -257,6 +265,8 @@ constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kSelSmemElems = 24576;         // 192 KB of (key, index) pairs
 
 __global__ void __launch_bounds__(kSelThreads) slot_select_kernel(SlotParams p) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ uint32_t sbuf[];           // [kSelSmemElems] keys, then [kSelSmemElems] indices
   __shared__ int hist[256];
   __shared__ int sh[kSelWarps];
@@ -370,23 +380,23 @@ cudaError_t launch_slots(const SlotParams& p, cudaStream_t stream) {
   const int64_t A = p.T * p.k;
   const int nchunk = (int)((A + kSlotChunk - 1) / kSlotChunk);
   if (A > 0) {
-    slot_count_kernel<<<nchunk, kSlotThreads, p.E * sizeof(int), stream>>>(p, nchunk);
-    slot_scan_kernel<<<p.E, kSlotThreads, 0, stream>>>(p, nchunk);
+    launch_pdl(slot_count_kernel, nchunk, kSlotThreads, p.E * sizeof(int), stream, p, nchunk);
+    launch_pdl(slot_scan_kernel, p.E, kSlotThreads, 0, stream, p, nchunk);
   } else {
     cudaMemsetAsync(p.expert_count, 0, p.E * sizeof(int32_t), stream);
     cudaMemsetAsync(p.kept_count, 0, p.E * sizeof(int32_t), stream);
   }
-  slot_offsets_kernel<<<1, 1024, 0, stream>>>(p);
+  launch_pdl(slot_offsets_kernel, 1, 1024, 0, stream, p);
   if (A > 0) {
     const size_t sm = (size_t)kSlotWarps * p.E * sizeof(int);
     cudaError_t e = ensure_smem(slot_rank_kernel, sm);
     if (e != cudaSuccess) return e;
-    slot_rank_kernel<<<nchunk, kSlotThreads, sm, stream>>>(p, nchunk);
+    launch_pdl(slot_rank_kernel, nchunk, kSlotThreads, sm, stream, p, nchunk);
     if (p.gates != nullptr) {
       const size_t ssm = 2 * sizeof(uint32_t) * kSelSmemElems;
       e = ensure_smem(slot_select_kernel, ssm);
       if (e != cudaSuccess) return e;
-      slot_select_kernel<<<p.E, kSelThreads, ssm, stream>>>(p);
+      launch_pdl(slot_select_kernel, p.E, kSelThreads, ssm, stream, p);
     }
   }
   return cudaGetLastError();

@@ -92,10 +92,13 @@ enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
 /* moe_cfg.flags
  * KEEP_LOGITS: moe_layer_fwd also stores fp32 logits in the workspace.
  * UNFUSED: moe_layer_fwd runs dispatch and combine as separate kernels (the
- *   pages' literal sequence, filling xbuf and ybuf).  By default, for bf16,
- *   the first expert contraction gathers its rows straight from x (xbuf is not
- *   written) and, for k == 1 without a shared expert, the second contraction
- *   writes gate * row to y[token] (ybuf's routed rows are not written).
+ *   pages' literal sequence, filling xbuf and ybuf).  Without it, a bf16 layer
+ *   with T*k <= 256*E (at most two 128-row blocks per expert on average, where
+ *   the expert contractions stream weights from HBM) runs fused: the first
+ *   expert contraction gathers its rows straight from x (xbuf is not written)
+ *   and, for k == 1 without a shared expert, the second contraction writes
+ *   gate * row to y[token] and zeroes the rows of fully dropped tokens (ybuf's
+ *   routed rows are not written).  Larger layers run the separate kernels.
  * RANDOM_SECOND: GShard top-2 ([EP] router section: the second expert receives
  *   the token at random, according to its weight).  For k >= 2 the rank-1
  *   choice of token t is dispatched iff uniform[t] < 2 * gate[t,1], with
@@ -282,9 +285,9 @@ MOE_API int moe_aux_loss(const moe_cfg* cfg, const void* ws, float* aux, moe_str
  * non-NULL, is an array of MOE_N_STAGE_EVENTS events recorded on `stream` before
  * the router and after each of: router, slots (which here also reduce the aux
  * loss), dispatch (an empty interval when fused), expert FFN first contraction
- * (with the activation), expert FFN second contraction, combine (when fused:
- * the zeroing of fully dropped tokens' rows), and the end of the call (the copy
- * of expert_count, if requested). */
+ * (with the activation), expert FFN second contraction, combine (an empty
+ * interval when fused), and the end of the call (the copy of expert_count, if
+ * requested). */
 enum { MOE_N_STAGE_EVENTS = 8 };
 MOE_API int moe_layer_fwd(const moe_cfg* cfg, const void* x, const float* wg, const float* logit_add,
                           const float* uniform, const moe_weights* w, void* y, float* aux, int32_t* expert_count,

@@ -130,7 +130,7 @@ def run_layer(shape: synth.LayerShape, inp: dict, keep_logits=True, ws=None, unf
     st = B.moe_sync_status(ws)
     assert st == B.MOE_OK, f"device status {st}: {B.strerror(st)}"
     out = B.workspace_tensors(cfg, ws)
-    fused = shape.dtype == synth.DTYPE_BF16 and not unfused
+    fused = shape.dtype == synth.DTYPE_BF16 and not unfused and shape.T * shape.k <= 256 * shape.E
     out.update(y=y, aux=aux, expert_count_out=ecount, cfg=cfg, ws=ws, fused_dispatch=fused,
                fused_combine=fused and shape.k == 1 and shape.n_shared == 0)
     return out
