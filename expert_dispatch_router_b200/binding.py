@@ -19,7 +19,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libmoe_b200.so")
 
 MOE_OK, MOE_EINVAL, MOE_EUNSUPPORTED, MOE_ECUDA, MOE_ETIMEOUT, MOE_EDEVICE, MOE_EWORKSPACE = range(7)
-MOE_FLAG_KEEP_LOGITS, MOE_FLAG_RANDOM_SECOND, MOE_FLAG_UNFUSED = 1, 2, 4
+MOE_FLAG_KEEP_LOGITS, MOE_FLAG_RANDOM_SECOND, MOE_FLAG_UNFUSED, MOE_FLAG_PACKED_WEIGHTS = 1, 2, 4, 8
 MOE_N_STAGE_EVENTS = 8
 STAGES = ("router", "slots", "dispatch", "ffn_gemm1", "ffn_gemm2", "combine", "aux")
 
@@ -70,6 +70,8 @@ _SIGS = {
     "moe_layer_fwd": [CFGP, P, P, P, P, ctypes.POINTER(moe_weights), P, P, P, P, ctypes.c_size_t, P, P],
     "moe_activation_eval": [ctypes.c_int, P, P, P, ctypes.c_int64, P],
     "moe_sync_status": [P, P],
+    "moe_packed_weight_bytes": [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, SZP],
+    "moe_pack_weight": [P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, P, P],
     "moe_clear_status": [P, P],
 }
 
@@ -212,6 +214,33 @@ def moe_layer_fwd(cfg, x, wg, logit_add, uniform, weights: moe_weights, y, aux, 
 def moe_activation_eval(act, z, u, out, stream=None):
     _check(load().moe_activation_eval(int(act), _ptr(z), _ptr(u), _ptr(out), z.numel(), _stream(stream)),
            "moe_activation_eval")
+
+
+def moe_packed_weight_bytes(G: int, N: int, K: int) -> int:
+    v = ctypes.c_size_t()
+    _check(load().moe_packed_weight_bytes(G, N, K, ctypes.byref(v)), "moe_packed_weight_bytes")
+    return v.value
+
+
+def moe_pack_weight(w, packed, stream=None):
+    G, N, K = w.shape
+    _check(load().moe_pack_weight(_ptr(w), G, N, K, _ptr(packed), _stream(stream)), "moe_pack_weight")
+
+
+def pack_weights(inp: dict, stream=None) -> dict:
+    """Packed copies (moe_pack_weight) of every expert matrix in `inp`; the
+    result replaces w1/w3/w2/sw1/sw3/sw2 for a layer run with
+    MOE_FLAG_PACKED_WEIGHTS."""
+    out = dict(inp)
+    for n in ("w1", "w3", "w2", "sw1", "sw3", "sw2"):
+        w = inp.get(n)
+        if w is None:
+            continue
+        G, N, K = w.shape
+        buf = torch.empty(moe_packed_weight_bytes(G, N, K) // 2, dtype=torch.bfloat16, device=w.device)
+        moe_pack_weight(w, buf, stream)
+        out[n] = buf
+    return out
 
 
 def moe_sync_status(ws, stream=None) -> int:

@@ -75,6 +75,7 @@ struct KParams {
   int a_kwrap;           // > 0 (router): B holds 3 planes of a_kwrap k blocks; A's k block = kb / 3
   int plane_split;       // router: 1 = one tile per (m-block, n-tile, plane), fp32 partials per plane
   int out_f32;           // 1: store the raw fp32 accumulator
+  int b_packed;          // 1: B maps are 5-D over packed weights (16 KB blocks of 128 rows x 64 k)
   // fused dispatch: routed A rows gathered from gsrc [rows of K elements] by gidx
   // (warp 0 issues cp.async with the 128-byte swizzle applied by hand)
   const __nv_bfloat16* gsrc;
@@ -126,6 +127,13 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar) {
   asm volatile("cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
                :: "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar) : "memory");
+}
+// 5-D load from a packed weight map: coordinates (0, 0, k block, n block, group).
+__device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map, int c2, int c3, int c4, uint32_t bar) {
+  asm volatile("cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes"
+               " [%0], [%1, {%2, %2, %3, %4, %5}], [%6];"
+               :: "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(c2), "r"(c3), "r"(c4), "r"(bar)
+               : "memory");
 }
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];"
@@ -342,7 +350,15 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
                            : p.a_kwrap > 0 ? (kb % 3) * p.a_kwrap + kb / 3 : kb) * BK;
           mbar_expect_tx(fb, gat ? stage_bytes - A_BYTES : stage_bytes);
           if (!gat) tma_load_2d(sa, ma, ka, arow, fb);
-          if (swiglu) {
+          if (p.b_packed) {
+            // packed weights: every box is one contiguous 16 KB block
+            if (swiglu) {
+              tma_load_5d(sb, mb0, kbb / BK, n0 / 128, z, fb);
+              tma_load_5d(sb + box_bytes, mb1, kbb / BK, n0 / 128, z, fb);
+            } else {
+              for (int b = 0; b < n_boxes; ++b) tma_load_5d(sb + b * box_bytes, mb0, kbb / BK, n0 / 128 + b, z, fb);
+            }
+          } else if (swiglu) {
             tma_load_3d(sb, mb0, kbb, n0, z, fb);                 // gate rows
             tma_load_3d(sb + box_bytes, mb1, kbb, n0, z, fb);     // up rows
           } else {
@@ -606,9 +622,9 @@ struct MapKey {
   const void* base;
   uint32_t rank;
   uint32_t swizzle;      // CUtensorMapSwizzle
-  cuuint64_t dims[3];
-  cuuint64_t strides[2];
-  cuuint32_t box[3];
+  cuuint64_t dims[5];
+  cuuint64_t strides[4];
+  cuuint32_t box[5];
   bool operator==(const MapKey& o) const { return memcmp(this, &o, sizeof(MapKey)) == 0; }
 };
 
@@ -621,7 +637,7 @@ static bool encode_cached(CUtensorMap* out, const MapKey& key) {
   std::lock_guard<std::mutex> lock(mu);
   for (int i = 0; i < used; ++i)
     if (keys[i] == key) { *out = maps[i]; return true; }
-  cuuint32_t es[3] = {1, 1, 1};
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
   CUtensorMap m;
   if (encode_fn()(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, key.rank, const_cast<void*>(key.base), key.dims, key.strides,
                   key.box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, (CUtensorMapSwizzle)key.swizzle,
@@ -664,6 +680,30 @@ static bool make_map_b(CUtensorMap* m, const void* base, int G, int N, int K, in
   key.box[0] = BK;
   key.box[1] = (cuuint32_t)box_n;
   key.box[2] = 1;
+  return encode_cached(m, key);
+}
+
+// 5-D map over packed weights [G][N/128][K/64][128][64] (see launch_pack_weight):
+// dims (64, 128, K/64, N/128, G), box 64 x 128 x 1 x 1 x 1 = one 16 KB block.
+static bool make_map_b_packed(CUtensorMap* m, const void* base, int G, int N, int K) {
+  const cuuint64_t kb = (cuuint64_t)((K + BK - 1) / BK), nb = (cuuint64_t)((N + 127) / 128);
+  MapKey key;
+  memset(&key, 0, sizeof(key));
+  key.base = base;
+  key.rank = 5;
+  key.swizzle = CU_TENSOR_MAP_SWIZZLE_128B;
+  key.dims[0] = BK;
+  key.dims[1] = 128;
+  key.dims[2] = kb;
+  key.dims[3] = nb;
+  key.dims[4] = (cuuint64_t)G;
+  key.strides[0] = BK * 2;
+  key.strides[1] = (cuuint64_t)BK * 128 * 2;
+  key.strides[2] = key.strides[1] * kb;
+  key.strides[3] = key.strides[2] * nb;
+  key.box[0] = BK;
+  key.box[1] = 128;
+  key.box[2] = key.box[3] = key.box[4] = 1;
   return encode_cached(m, key);
 }
 
@@ -710,10 +750,17 @@ cudaError_t launch_grouped_gemm(const GemmParams& p, cudaStream_t stream) {
   KParams k{};
   bool ok = make_map_a(&k.tmA, p.a_routed ? p.a_routed : p.gather_src, p.a_routed ? p.rows_max : p.T, p.K);
   ok = ok && make_map_a(&k.tmAs, p.a_shared ? p.a_shared : p.a_routed, p.a_shared ? p.T : p.rows_max, p.K);
-  ok = ok && make_map_b(&k.tmB0, p.b0, p.E, p.Nw, p.K, box_n);
-  ok = ok && make_map_b(&k.tmB1, p.b1 ? p.b1 : p.b0, p.E, p.Nw, p.K, box_n);
-  ok = ok && make_map_b(&k.tmSB0, p.sb0 ? p.sb0 : p.b0, 1, p.Nw, p.K, box_n);
-  ok = ok && make_map_b(&k.tmSB1, p.sb1 ? p.sb1 : (p.sb0 ? p.sb0 : p.b0), 1, p.Nw, p.K, box_n);
+  if (p.b_packed) {
+    ok = ok && make_map_b_packed(&k.tmB0, p.b0, p.E, p.Nw, p.K);
+    ok = ok && make_map_b_packed(&k.tmB1, p.b1 ? p.b1 : p.b0, p.E, p.Nw, p.K);
+    ok = ok && make_map_b_packed(&k.tmSB0, p.sb0 ? p.sb0 : p.b0, 1, p.Nw, p.K);
+    ok = ok && make_map_b_packed(&k.tmSB1, p.sb1 ? p.sb1 : (p.sb0 ? p.sb0 : p.b0), 1, p.Nw, p.K);
+  } else {
+    ok = ok && make_map_b(&k.tmB0, p.b0, p.E, p.Nw, p.K, box_n);
+    ok = ok && make_map_b(&k.tmB1, p.b1 ? p.b1 : p.b0, p.E, p.Nw, p.K, box_n);
+    ok = ok && make_map_b(&k.tmSB0, p.sb0 ? p.sb0 : p.b0, 1, p.Nw, p.K, box_n);
+    ok = ok && make_map_b(&k.tmSB1, p.sb1 ? p.sb1 : (p.sb0 ? p.sb0 : p.b0), 1, p.Nw, p.K, box_n);
+  }
   ok = ok && make_map_d(&k.tmD, p.d, p.rows_max, p.Nw);
   if (!ok) return cudaErrorInvalidValue;
   k.d = p.d;
@@ -734,6 +781,7 @@ cudaError_t launch_grouped_gemm(const GemmParams& p, cudaStream_t stream) {
   k.a_kwrap = 0;
   k.plane_split = 0;
   k.out_f32 = 0;
+  k.b_packed = p.b_packed;
   k.gsrc = static_cast<const __nv_bfloat16*>(p.gather_src);
   k.gidx = p.gather_idx;
   k.sdst = static_cast<__nv_bfloat16*>(p.scatter_dst);

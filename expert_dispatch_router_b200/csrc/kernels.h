@@ -127,7 +127,14 @@ struct GemmParams {
   void* scatter_dst;
   const float* scatter_gate;
   const int32_t* scatter_slot;
+  int b_packed;             // 1: b0/b1/sb0/sb1 are packed (launch_pack_weight)
 };
 cudaError_t launch_grouped_gemm(const GemmParams& p, cudaStream_t stream);
+
+// Packed weight layout for the grouped GEMM: w [G, N, K] bf16 (K contiguous) ->
+// [G][ceil(N/128)][ceil(K/64)][128][64], zero-padded, so every TMA box of 128
+// rows x 64 k is one contiguous 16 KB block.
+size_t packed_weight_bytes(int G, int N, int K);
+cudaError_t launch_pack_weight(const void* w, int G, int N, int K, void* packed, cudaStream_t stream);
 
 }  // namespace moe

@@ -35,7 +35,9 @@ bool valid_cfg(const moe_cfg* c) {
   if (c->cap_mode == MOE_CAP_CAPACITY && (c->cf_num <= 0 || c->cf_den <= 0)) return false;
   if (c->min_capacity < 0) return false;
   if (!(c->z_coef >= 0.0f) || isinf(c->z_coef)) return false;
-  if (c->flags & ~(MOE_FLAG_KEEP_LOGITS | MOE_FLAG_RANDOM_SECOND | MOE_FLAG_UNFUSED)) return false;
+  if (c->flags & ~(MOE_FLAG_KEEP_LOGITS | MOE_FLAG_RANDOM_SECOND | MOE_FLAG_UNFUSED | MOE_FLAG_PACKED_WEIGHTS))
+    return false;
+  if ((c->flags & MOE_FLAG_PACKED_WEIGHTS) && c->dtype != MOE_DTYPE_BF16) return false;
   if (c->drop_policy != MOE_DROP_POSITION && c->drop_policy != MOE_DROP_PROBS) return false;
   return true;
 }
@@ -250,6 +252,7 @@ int run_ffn(const moe_cfg* c, const Layout& L, const void* xbuf, const void* x, 
     g1.n_shared = c->n_shared;
     g1.epi = c->act;
     g1.status = at<DevStatus>(ws, L.status);
+    g1.b_packed = (c->flags & MOE_FLAG_PACKED_WEIGHTS) ? 1 : 0;
     if (rowtok != nullptr) {
       g1.a_routed = nullptr;
       g1.gather_src = x;
@@ -552,6 +555,22 @@ int moe_activation_eval(int act, const float* z, const float* u, float* out, int
   if (act < MOE_ACT_RELU || act > MOE_ACT_SWIGLU || n < 0) return MOE_EINVAL;
   if (n > 0 && (z == nullptr || out == nullptr || (act == MOE_ACT_SWIGLU && u == nullptr))) return MOE_EINVAL;
   return cuda_status(launch_activation_eval(act, z, u, out, n, S(stream)));
+}
+
+int moe_packed_weight_bytes(int32_t G, int32_t N, int32_t K, size_t* bytes) {
+  if (bytes == nullptr || G < 1 || N < 1 || K < 1) return MOE_EINVAL;
+  if (K % 8 != 0) return MOE_EUNSUPPORTED;
+  *bytes = packed_weight_bytes(G, N, K);
+  return MOE_OK;
+}
+
+int moe_pack_weight(const void* w, int32_t G, int32_t N, int32_t K, void* packed, moe_stream_t stream) {
+  size_t bytes = 0;
+  const int st = moe_packed_weight_bytes(G, N, K, &bytes);
+  if (st != MOE_OK) return st;
+  if (w == nullptr || packed == nullptr) return MOE_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(w) | reinterpret_cast<uintptr_t>(packed)) & 15) return MOE_EINVAL;
+  return cuda_status(launch_pack_weight(w, G, N, K, packed, S(stream)));
 }
 
 const char* moe_version(void) { return "moe_b200 0.1 sm_100a"; }

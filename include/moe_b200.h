@@ -91,6 +91,8 @@ enum { MOE_DROP_POSITION = 0, MOE_DROP_PROBS = 1 };
 enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
 /* moe_cfg.flags
  * KEEP_LOGITS: moe_layer_fwd also stores fp32 logits in the workspace.
+ * PACKED_WEIGHTS (bf16 only): every pointer of moe_weights is a packed buffer
+ *   written by moe_pack_weight (see there); results are bitwise the same. 
  * UNFUSED: moe_layer_fwd runs dispatch and combine as separate kernels (the
  *   pages' literal sequence, filling xbuf and ybuf).  Without it, a bf16 layer
  *   with T*k <= 256*E (at most two 128-row blocks per expert on average, where
@@ -105,7 +107,7 @@ enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
  *   uniform [T] fp32 in [0,1) supplied by the caller; otherwise its id becomes
  *   -1 and its gate 0 (it takes no slot and adds nothing to y).  The aux loss
  *   still counts it as selected.  No effect when k == 1. */
-enum { MOE_FLAG_KEEP_LOGITS = 1, MOE_FLAG_RANDOM_SECOND = 2, MOE_FLAG_UNFUSED = 4 };
+enum { MOE_FLAG_KEEP_LOGITS = 1, MOE_FLAG_RANDOM_SECOND = 2, MOE_FLAG_UNFUSED = 4, MOE_FLAG_PACKED_WEIGHTS = 8 };
 
 /* Layer configuration.  Limits of this build: 1 <= E <= 1024, 1 <= k <= min(E,16),
  * H and F multiples of 8, n_shared in {0,1}, T >= 0 with T*k < 2^31 and every
@@ -299,6 +301,20 @@ MOE_API int moe_layer_fwd(const moe_cfg* cfg, const void* x, const float* wg, co
  * MOE_ACT_SWIGLU out = silu(z) * u.  Exposed so the approximation can be
  * checked against its error bound. */
 MOE_API int moe_activation_eval(int act, const float* z, const float* u, float* out, int64_t n, moe_stream_t stream);
+
+/* Expert weights in the grouped GEMM's block layout.  No source page has a
+ * counterpart: this is weight preprocessing, done once per weight.  The
+ * contractions read weights in boxes of 128 rows x 64 k; in the linear-layer
+ * layout a box is 128 pieces of 128 bytes K*2 bytes apart, which HBM serves at
+ * a fraction of its streaming rate.  Packed, each box is one contiguous 16 KB
+ * block: P[g][n/128][k/64][n%128][k%64], zero-padded to whole blocks.
+ *   moe_packed_weight_bytes: bytes of the packed form of a [G, N, K] bf16 matrix.
+ *   moe_pack_weight: w [G, N, K] bf16 (device, K % 8 == 0) -> packed (device,
+ *   moe_packed_weight_bytes bytes, 16-byte aligned), asynchronous on `stream`.
+ * Pack w1 and w3 as [E, F, H], w2 as [E, H, F], the shared matrices with G = 1,
+ * then set MOE_FLAG_PACKED_WEIGHTS. */
+MOE_API int moe_packed_weight_bytes(int32_t G, int32_t N, int32_t K, size_t* bytes);
+MOE_API int moe_pack_weight(const void* w, int32_t G, int32_t N, int32_t K, void* packed, moe_stream_t stream);
 
 /* ---- status ---------------------------------------------------------------- */
 

@@ -128,7 +128,7 @@ def test_router_variant_validation(lib):
             B.moe_workspace_size(B.make_cfg(g, **kw))
         assert ei.value.code == B.MOE_EINVAL, kw
     with pytest.raises(B.MoeError) as ei:
-        B.moe_workspace_size(B.make_cfg(g, flags=8))
+        B.moe_workspace_size(B.make_cfg(g, flags=16))
     assert ei.value.code == B.MOE_EINVAL
     # the flag needs the draws (k >= 2, T > 0); dummy device pointers are never touched
     cfg = B.make_cfg(g.replace(random_second=1))
@@ -140,3 +140,15 @@ def test_router_variant_validation(lib):
     a = B.moe_workspace_size(B.make_cfg(g))
     b = B.moe_workspace_size(B.make_cfg(g, z_coef=1e-3))
     assert a == b
+
+
+def test_packed_weight_sizes(lib):
+    assert B.moe_packed_weight_bytes(64, 3072, 768) == 64 * 24 * 12 * 16384
+    assert B.moe_packed_weight_bytes(1, 1, 8) == 16384
+    for args, code in [((0, 8, 8), B.MOE_EINVAL), ((1, 8, 12), B.MOE_EUNSUPPORTED), ((1, -1, 8), B.MOE_EINVAL)]:
+        with pytest.raises(B.MoeError) as ei:
+            B.moe_packed_weight_bytes(*args)
+        assert ei.value.code == code
+    # packed weights are a bf16 feature
+    with pytest.raises(B.MoeError):
+        B.moe_workspace_size(B.make_cfg(synth.SWITCH_TINY_F32, flags=B.MOE_FLAG_PACKED_WEIGHTS))

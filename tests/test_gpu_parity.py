@@ -294,3 +294,35 @@ def test_stage_entry_points_match_layer(variant):
     used = int(off[-1])
     assert torch.equal(rt[:used], full["row_token"][:used])
     assert torch.equal(ybuf[:used][rt[:used] >= 0], full["ybuf"][:used][full["row_token"][:used] >= 0])
+
+
+@pytest.mark.parametrize("G,N,K", [(3, 200, 136), (1, 128, 64), (2, 300, 520)])
+def test_pack_weight_layout(G, N, K):
+    """moe_pack_weight is pure data movement into [G][N/128][K/64][128][64]."""
+    w = (torch.arange(G * N * K, device="cuda", dtype=torch.float32) % 251).to(torch.bfloat16).reshape(G, N, K)
+    nb, kb = (N + 127) // 128, (K + 63) // 64
+    assert B.moe_packed_weight_bytes(G, N, K) == G * nb * kb * 128 * 64 * 2
+    got = torch.full((G * nb * kb * 128 * 64,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    B.moe_pack_weight(w, got)
+    torch.cuda.synchronize()
+    pad = torch.zeros((G, nb * 128, kb * 64), dtype=torch.bfloat16, device="cuda")
+    pad[:, :N, :K] = w
+    want = pad.reshape(G, nb, 128, kb, 64).permute(0, 1, 3, 2, 4).reshape(-1)
+    assert torch.equal(got.view(torch.int16), want.view(torch.int16))
+
+
+@pytest.mark.parametrize("name", ["switch_top1", "gshard_top2", "wideep", "ds_k4_cf05", "switch_relu_dropless_shared"])
+def test_packed_weights_bitwise(name):
+    """Packed weights change only where the contractions read B from."""
+    shape = SMALL[name]
+    inp = synth.make_inputs(shape, seed=11, device="cuda")
+    a = run_layer(shape, inp)
+    snap = {n: a[n].clone() for n in ("y", "hbuf", "ybuf", "expert_offset", "row_token")}
+    b = run_layer(shape, inp, packed=True)
+    used = int(b["expert_offset"][-1])
+    live = b["row_token"][:used] >= 0
+    assert torch.equal(snap["y"], b["y"])
+    assert torch.equal(snap["hbuf"][:used][live], b["hbuf"][:used][live])
+    if not a["fused_combine"]:
+        assert torch.equal(snap["ybuf"][:used][live], b["ybuf"][:used][live])
+    check_layer(shape, inp, b)
