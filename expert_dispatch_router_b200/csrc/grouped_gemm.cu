@@ -72,8 +72,9 @@ struct KParams {
   int as_sep;            // 1: the shared block's A rows come from tmAs (row - off[E]); 0: from tmA in place
   int bn_fixed;          // 0: N tile chosen on the device (256 or 128); else this MMA N (multiple of 16)
   int bbox;              // rows of one B TMA box (128, or bn_fixed when smaller)
-  int a_kwrap;           // > 0 (router): B holds 3 planes of a_kwrap k blocks; A's k block = kb / 3
-  int plane_split;       // router: 1 = one tile per (m-block, n-tile, plane), fp32 partials per plane
+  int b_planes;          // router: 3 weight planes laid side by side along B's K; one stage holds the A
+                         // chunk and the matching chunk of every plane, multiplied into one accumulator
+  int plane_k;           // elements between planes along B's K
   int out_f32;           // 1: store the raw fp32 accumulator
   int b_packed;          // 1: B maps are 5-D over packed weights (16 KB blocks of 128 rows x 64 k)
   // fused dispatch: routed A rows gathered from gsrc [rows of K elements] by gidx
@@ -300,12 +301,12 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
   const int bn = p.bn_fixed ? p.bn_fixed : (narrow ? 128 : 256);   // MMA N
   const int n_step = swiglu ? BN / 2 : bn;                          // output columns per tile
   const int n_tiles_n = (p.N_out + n_step - 1) / n_step;
-  const int n_planes = p.plane_split ? 3 : 1;
-  const int64_t n_tiles = n_mtiles * n_tiles_n * n_planes;
-  const int nk_tile = p.plane_split ? p.a_kwrap : nk;    // k blocks per tile
+  const int64_t n_tiles = n_mtiles * n_tiles_n;
+  const int nk_tile = nk;                                // k blocks per tile
   const int box_bytes = p.bbox * BK * 2;
   const int n_boxes = swiglu ? 2 : bn / p.bbox;
-  const int stage_bytes = A_BYTES + n_boxes * box_bytes;
+  const int plane_bytes = n_boxes * box_bytes;          // one plane's B chunk
+  const int stage_bytes = A_BYTES + p.b_planes * plane_bytes;
   const int n_stages = min(MAX_STAGES, RING_BYTES / stage_bytes);
 
   if (warp == 0) {
@@ -324,9 +325,8 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
       uint32_t fills[MAX_STAGES] = {0, 0, 0, 0, 0, 0, 0, 0};
       bool ok = true;
       for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
-        const int plane = (int)(tile % n_planes);
-        const int64_t mt = tile / n_planes / n_tiles_n;
-        const int nt = (int)(tile / n_planes % n_tiles_n);
+        const int64_t mt = tile / n_tiles_n;
+        const int nt = (int)(tile % n_tiles_n);
         const int64_t row0 = mt * BM;
         const int g = grouped ? find_group(p.off, ngroups, row0) : 0;
         const bool sh = grouped && g == p.E;
@@ -343,11 +343,7 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
           const uint32_t sa = smem_u32(stage_base + stage * stage_bytes);
           const uint32_t sb = sa + A_BYTES;
           const uint32_t fb = full0 + 8 * stage;
-          // Router mode (a_kwrap = H'/64 > 0): the three weight planes of one A chunk
-          // are consecutive k blocks, so the A chunk is re-read from L2 right away.
-          const int ka = (p.a_kwrap > 0 && !p.plane_split ? kb / 3 : kb) * BK;
-          const int kbb = (p.plane_split ? plane * p.a_kwrap + kb
-                           : p.a_kwrap > 0 ? (kb % 3) * p.a_kwrap + kb / 3 : kb) * BK;
+          const int ka = kb * BK, kbb = kb * BK;
           mbar_expect_tx(fb, gat ? stage_bytes - A_BYTES : stage_bytes);
           if (!gat) tma_load_2d(sa, ma, ka, arow, fb);
           if (p.b_packed) {
@@ -362,7 +358,9 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
             tma_load_3d(sb, mb0, kbb, n0, z, fb);                 // gate rows
             tma_load_3d(sb + box_bytes, mb1, kbb, n0, z, fb);     // up rows
           } else {
-            for (int b = 0; b < n_boxes; ++b) tma_load_3d(sb + b * box_bytes, mb0, kbb, n0 + b * p.bbox, z, fb);
+            for (int j = 0; j < p.b_planes; ++j)
+              for (int b = 0; b < n_boxes; ++b)
+                tma_load_3d(sb + j * plane_bytes + b * box_bytes, mb0, j * p.plane_k + kbb, n0 + b * p.bbox, z, fb);
           }
           fills[stage]++;
           if (++stage == n_stages) { stage = 0; phase ^= 1u; }
@@ -449,10 +447,13 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
           if (GATHER) fence_async_smem();       // cp.async data (generic proxy) -> tensor-core reads
           const uint32_t sa = smem_u32(stage_base + stage * stage_bytes);
           const uint32_t sb = sa + A_BYTES;
-          const uint64_t ad = sw128_desc(sa), bd = sw128_desc(sb);
+          const uint64_t ad = sw128_desc(sa);
+          for (int j = 0; j < p.b_planes; ++j) {
+            const uint64_t bd = sw128_desc(sb + j * plane_bytes);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)   // advance 16 elements = 32 bytes along K
-            umma(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < BK / 16; ++kk)   // advance 16 elements = 32 bytes along K
+              umma(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (kb | kk | j) != 0 ? 1u : 0u);
+          }
           umma_commit(empty0 + 8 * stage);      // stage free once these MMAs finish
           if (++stage == n_stages) { stage = 0; phase ^= 1u; }
         }
@@ -486,9 +487,8 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
         break;
       }
       tc_fence_after();
-      const int plane = (int)(tile % n_planes);
-      const int64_t mt = tile / n_planes / n_tiles_n;
-      const int nt = (int)(tile / n_planes % n_tiles_n);
+      const int64_t mt = tile / n_tiles_n;
+      const int nt = (int)(tile % n_tiles_n);
       const int64_t grow = mt * BM + row_in_tile;
       const bool row_ok = grow < p.rows_store;
       // fused top-1 combine: this lane's row is token st of the batch, weighted by sg
@@ -523,7 +523,7 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
         const int col = ncol0 + c;
         if (p.out_f32) {
           if (!row_ok) continue;
-          float* drow = static_cast<float*>(p.d) + (int64_t)plane * p.rows_store * p.ld_d + grow * p.ld_d;
+          float* drow = static_cast<float*>(p.d) + grow * p.ld_d;
           const bool vec = (p.ld_d & 3) == 0;
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
@@ -778,8 +778,8 @@ cudaError_t launch_grouped_gemm(const GemmParams& p, cudaStream_t stream) {
   k.epi = p.epi;
   k.bn_fixed = 0;
   k.bbox = box_n;
-  k.a_kwrap = 0;
-  k.plane_split = 0;
+  k.b_planes = 1;
+  k.plane_k = 0;
   k.out_f32 = 0;
   k.b_packed = p.b_packed;
   k.gsrc = static_cast<const __nv_bfloat16*>(p.gather_src);
@@ -830,8 +830,10 @@ cudaError_t launch_router_gemm(const void* x, const float* wg, void* planes, flo
     launch_pdl(split_router_weight_kernel, (unsigned)(blocks < 2048 ? blocks : 2048), 256, 0, stream, 
         wg, static_cast<__nv_bfloat16*>(planes), E, H, Hp);
   }
-  const int bn = E >= 256 ? 256 : (E + 15) / 16 * 16;
-  const int bbox = bn < 128 ? bn : 128;
+  // one stage = an A chunk plus the matching 64-k chunk of all three planes, so
+  // the N tile stays <= 128 columns to keep at least three stages in the ring
+  const int bn = E >= 128 ? 128 : (E + 15) / 16 * 16;
+  const int bbox = bn;
   KParams k{};
   bool ok = make_map_a(&k.tmA, x, T, H);
   ok = ok && make_map_b(&k.tmB0, planes, 1, E, 3 * Hp, bbox);
@@ -846,7 +848,7 @@ cudaError_t launch_router_gemm(const void* x, const float* wg, void* planes, flo
   k.rows_max = T;
   k.rows_static = T;
   k.rows_store = T;
-  k.K = 3 * Hp;
+  k.K = Hp;
   k.N_out = E;
   k.E = 1;
   k.n_shared = 0;
@@ -854,13 +856,12 @@ cudaError_t launch_router_gemm(const void* x, const float* wg, void* planes, flo
   k.as_sep = 0;
   k.bn_fixed = bn;
   k.bbox = bbox;
-  k.a_kwrap = Hp / BK;
+  k.b_planes = 3;
+  k.plane_k = Hp;
   k.out_f32 = 1;
-  // One tile per (m-block, n-tile).  (Giving each weight plane its own tile to
-  // fill more SMs at small T measured slower: three partial arrays to write and
-  // add, and three times the tile start-up cost.)
+  // One tile per (m-block, n-tile); each k step multiplies the A chunk by the
+  // hi, mid and lo planes in that order, into one fp32 accumulator.
   const int64_t tiles = ((T + BM - 1) / BM) * ((E + bn - 1) / bn);
-  k.plane_split = 0;
   *parts = 1;
   return launch_kernel(k, tiles * (*parts), stream);
 }
