@@ -505,7 +505,10 @@ def run_ours(args, world, rank, local):
     value = job_tokens_per_s(T, world, ms)
 
     work = stage_work(shape, kept, experts_used)
-    single = ["router", "dispatch", "ffn_gemm1", "ffn_gemm2", "combine"]
+    fused = shape.dtype == 1 and shape.T * shape.k <= 256 * shape.E      # dispatch inside GEMM1
+    fused_combine = fused and shape.k == 1 and shape.n_shared == 0       # combine inside GEMM2
+    single = ["router", "ffn_gemm1", "ffn_gemm2"] + ([] if fused else ["dispatch"]) \
+        + ([] if fused_combine else ["combine"])
     dom = max(single, key=lambda s: stage_ms[s])
     bf16 = shape.dtype == 1
     long_step = ms_local > 5.0          # seconds-long power-capped regime: sustained tensor peak
@@ -595,8 +598,9 @@ def run_ours(args, world, rank, local):
             "stages_ms": stage_ms,
             "stages_note": f"second timed pass of {n_stage_steps} steps with per-stage events "
                            f"({stage_sum_ms:.4f} ms per step including the events' own cost)",
-            "dispatch_gbs": per_stage["dispatch"]["achieved"] if per_stage["dispatch"]["unit"] == "GB/s" else None,
-            "combine_gbs": per_stage["combine"]["achieved"] if per_stage["combine"]["unit"] == "GB/s" else None,
+            "dispatch_gbs": per_stage["dispatch"]["achieved"] if "dispatch" in per_stage else None,
+            "combine_gbs": per_stage["combine"]["achieved"] if "combine" in per_stage else None,
+            "fused": {"dispatch_into_gemm1": fused, "combine_into_gemm2": fused_combine},
             "expert_gemm_tc_util_pct": tc_util,
             "roofline": {k: roof[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic", "peak_source")},
             "roofline_detail": {s: {k: v[k] for k in ("bound", "achieved", "unit", "frac", "ms_per_launch")}
