@@ -75,6 +75,8 @@ struct KParams {
   int b_planes;          // router: 3 weight planes laid side by side along B's K; one stage holds the A
                          // chunk and the matching chunk of every plane, multiplied into one accumulator
   int plane_k;           // elements between planes along B's K
+  int k_split;           // fp32 output only: each tile's k blocks split over this many tiles, each
+                         // storing its partial sums to d + part * rows_store * ld_d
   int out_f32;           // 1: store the raw fp32 accumulator
   int b_packed;          // 1: B maps are 5-D over packed weights (16 KB blocks of 128 rows x 64 k)
   // fused dispatch: routed A rows gathered from gsrc [rows of K elements] by gidx
@@ -301,8 +303,11 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
   const int bn = p.bn_fixed ? p.bn_fixed : (narrow ? 128 : 256);   // MMA N
   const int n_step = swiglu ? BN / 2 : bn;                          // output columns per tile
   const int n_tiles_n = (p.N_out + n_step - 1) / n_step;
-  const int64_t n_tiles = n_mtiles * n_tiles_n;
-  const int nk_tile = nk;                                // k blocks per tile
+  // tile = (m-block, n-tile, k part), k part fastest; part q owns k blocks
+  // [q * nk_part, min(nk, (q + 1) * nk_part))
+  const int n_parts = p.k_split;
+  const int nk_part = (nk + n_parts - 1) / n_parts;
+  const int64_t n_tiles = n_mtiles * n_tiles_n * n_parts;
   const int box_bytes = p.bbox * BK * 2;
   const int n_boxes = swiglu ? 2 : bn / p.bbox;
   const int plane_bytes = n_boxes * box_bytes;          // one plane's B chunk
@@ -325,8 +330,10 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
       uint32_t fills[MAX_STAGES] = {0, 0, 0, 0, 0, 0, 0, 0};
       bool ok = true;
       for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
-        const int64_t mt = tile / n_tiles_n;
-        const int nt = (int)(tile % n_tiles_n);
+        const int part = (int)(tile % n_parts);
+        const int64_t mt = tile / n_parts / n_tiles_n;
+        const int nt = (int)(tile / n_parts % n_tiles_n);
+        const int kb0 = part * nk_part, kb1 = min(nk, kb0 + nk_part);
         const int64_t row0 = mt * BM;
         const int g = grouped ? find_group(p.off, ngroups, row0) : 0;
         const bool sh = grouped && g == p.E;
@@ -338,7 +345,7 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
         const int arow = (int)(sep ? row0 - p.off[p.E] : row0);
         const int z = sh ? 0 : g;
         const int n0 = nt * n_step;
-        for (int kb = 0; kb < nk_tile; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag)) { ok = false; break; }
           const uint32_t sa = smem_u32(stage_base + stage * stage_bytes);
           const uint32_t sb = sa + A_BYTES;
@@ -392,14 +399,15 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
     uint32_t phase = 0;
     bool ok = true;
     for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
-      const int64_t mt = tile / n_tiles_n;
+      const int64_t mt = tile / n_parts / n_tiles_n;
+      const int kb0 = (int)(tile % n_parts) * nk_part, kb1 = min(nk, kb0 + nk_part);
       const int64_t row0 = mt * BM;
       const int g = find_group(p.off, ngroups, row0);
       const bool gat = g != p.E;
       int tok[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) tok[i] = gat ? __ldg(p.gidx + row0 + 64 * gw + 4 * i + lr) : -1;
-      for (int kb = 0; kb < nk_tile; ++kb) {
+      for (int kb = kb0; kb < kb1; ++kb) {
         int good = 1;
         if (lane == 0) good = mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag);
         good = __shfl_sync(0xffffffffu, good, 0);
@@ -438,10 +446,11 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
       bool ok = true;
       const uint32_t idesc = make_idesc(bn);
       for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+        const int kb0 = (int)(tile % n_parts) * nk_part, kb1 = min(nk, kb0 + nk_part);
         if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-        for (int kb = 0; kb < nk_tile; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(full0 + 8 * stage, phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
           if (GATHER) fence_async_smem();       // cp.async data (generic proxy) -> tensor-core reads
@@ -452,7 +461,8 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
             const uint64_t bd = sw128_desc(sb + j * plane_bytes);
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk)   // advance 16 elements = 32 bytes along K
-              umma(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (kb | kk | j) != 0 ? 1u : 0u);
+              umma(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc,
+                   ((kb - kb0) | kk | j) != 0 ? 1u : 0u);
           }
           umma_commit(empty0 + 8 * stage);      // stage free once these MMAs finish
           if (++stage == n_stages) { stage = 0; phase ^= 1u; }
@@ -487,8 +497,9 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
         break;
       }
       tc_fence_after();
-      const int64_t mt = tile / n_tiles_n;
-      const int nt = (int)(tile % n_tiles_n);
+      const int part = (int)(tile % n_parts);
+      const int64_t mt = tile / n_parts / n_tiles_n;
+      const int nt = (int)(tile / n_parts % n_tiles_n);
       const int64_t grow = mt * BM + row_in_tile;
       const bool row_ok = grow < p.rows_store;
       // fused top-1 combine: this lane's row is token st of the batch, weighted by sg
@@ -523,7 +534,7 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
         const int col = ncol0 + c;
         if (p.out_f32) {
           if (!row_ok) continue;
-          float* drow = static_cast<float*>(p.d) + grow * p.ld_d;
+          float* drow = static_cast<float*>(p.d) + (int64_t)part * p.rows_store * p.ld_d + grow * p.ld_d;
           const bool vec = (p.ld_d & 3) == 0;
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
@@ -780,6 +791,7 @@ cudaError_t launch_grouped_gemm(const GemmParams& p, cudaStream_t stream) {
   k.bbox = box_n;
   k.b_planes = 1;
   k.plane_k = 0;
+  k.k_split = 1;
   k.out_f32 = 0;
   k.b_packed = p.b_packed;
   k.gsrc = static_cast<const __nv_bfloat16*>(p.gather_src);
@@ -860,10 +872,14 @@ cudaError_t launch_router_gemm(const void* x, const float* wg, void* planes, flo
   k.plane_k = Hp;
   k.out_f32 = 1;
   // One tile per (m-block, n-tile); each k step multiplies the A chunk by the
-  // hi, mid and lo planes in that order, into one fp32 accumulator.
+  // hi, mid and lo planes in that order, into one fp32 accumulator.  When the
+  // tiles cannot fill half the SMs, each tile's k blocks are split in two and
+  // the partial logits are added by the routing kernel.
   const int64_t tiles = ((T + BM - 1) / BM) * ((E + bn - 1) / bn);
-  *parts = 1;
-  return launch_kernel(k, tiles * (*parts), stream);
+  const int nk = Hp / BK;
+  k.k_split = (tiles * 2 <= sm_count() && nk >= 4) ? 2 : 1;
+  *parts = k.k_split;
+  return launch_kernel(k, tiles * k.k_split, stream);
 }
 
 }  // namespace moe

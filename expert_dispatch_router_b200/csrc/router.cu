@@ -322,13 +322,17 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterParams p) 
 }
 
 // Routing from given fp32 logits (the tensor-core router's output, or the
-// caller's for moe_route_from_logits): 8 warps, the same BT tokens per CTA as
-// the FFMA router so the partial-sum rows line up; a warp routes one token at a
-// time with nothing but that token's logits in registers.
-constexpr int kLogitWarps = 8;
+// caller's for moe_route_from_logits): the same BT tokens per CTA as the FFMA
+// router so the partial-sum rows line up; a warp routes one token at a time with
+// nothing but that token's logits in registers.  Warps per CTA: 32 (one token
+// each) for E <= 64, 16 for E <= 128 (the register budget of 1024 threads is
+// too small there), 8 for wider E, whose partial sums need more shared memory.
+template <int EJ>
+constexpr int logit_warps() { return EJ <= 2 ? 32 : EJ == 4 ? 16 : 8; }
 
 template <int EJ>
-__global__ void __launch_bounds__(kLogitWarps * 32, EJ <= 4 ? 3 : 1) route_logits_kernel(RouterParams p, int bt) {
+__global__ void __launch_bounds__(logit_warps<EJ>() * 32, 1) route_logits_kernel(RouterParams p, int bt) {
+  constexpr int kLogitWarps = logit_warps<EJ>();
   pdl_wait();
   pdl_trigger();
   extern __shared__ __align__(16) float smem[];
@@ -389,6 +393,7 @@ static cudaError_t launch_router_ej(const RouterParams& p, bool bf16, cudaStream
 template <int EJ>
 static cudaError_t launch_route_logits_ej(const RouterParams& p, cudaStream_t stream) {
   const int bt = router_tile_tokens(p.E);
+  constexpr int kLogitWarps = logit_warps<EJ>();
   const size_t smem = sizeof(float) * (2 * kLogitWarps * 32 * EJ + kLogitWarps);
   const unsigned grid = (unsigned)((p.T + bt - 1) / bt);
   auto k = route_logits_kernel<EJ>;
