@@ -72,6 +72,8 @@ def parse_args():
     ap.add_argument("--unpacked", action="store_true",
                     help="read expert weights in the linear-layer layout instead of packed blocks")
     ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE")
+    ap.add_argument("--pass", dest="pass_", default="forward", choices=["forward", "train"],
+                    help="train: one step is moe_layer_fwd (MOE_FLAG_TRAINING) followed by moe_layer_bwd")
     return ap.parse_args()
 
 
@@ -266,7 +268,15 @@ def traffic_from_profiles(workload: str, kernel: str):
 
 def kernel_source(stage: str) -> str:
     return {"router": "router.cu", "dispatch": "permute.cu", "combine": "permute.cu",
-            "ffn_gemm1": "grouped_gemm.cu", "ffn_gemm2": "grouped_gemm.cu"}.get(stage, "moe_abi.cu")
+            "ffn_gemm1": "grouped_gemm.cu", "ffn_gemm2": "grouped_gemm.cu",
+            "combine_bwd": "backward.cu", "dispatch_bwd": "backward.cu", "router_wgrad": "backward.cu",
+            "router_bwd": "router.cu", "dgrad_dh": "grouped_gemm_bwd.cu", "wgrad_w2": "grouped_gemm_bwd.cu",
+            "dact_dz": "grouped_gemm_bwd.cu", "wgrad_w1": "grouped_gemm_bwd.cu",
+            "dgrad_dx": "grouped_gemm_bwd.cu"}.get(stage, "moe_abi.cu")
+
+
+# kernels whose arithmetic runs on the fp32 FMA pipes, not the tensor cores
+SIMT_STAGES = ("dispatch_bwd", "router_wgrad")
 
 
 # ------------------------------------------------------------------ algorithmic work
@@ -300,7 +310,7 @@ def roofline(stage: str, work: dict, ms: float, peaks: dict, workload: str, bf16
     w = work[stage]
     s = ms / 1e3
     t_hbm = w["bytes"] / (hbm * 1e9)
-    if stage == "router" and not bf16:
+    if (stage == "router" and not bf16) or stage in SIMT_STAGES:
         cpeak, cbound = alu, "alu"
     else:
         cpeak, cbound = tc, "tensor"
@@ -317,6 +327,45 @@ def roofline(stage: str, work: dict, ms: float, peaks: dict, workload: str, bf16
     out.update(kernel=stage, algorithmic_bytes=w["bytes"], algorithmic_flops=w["flops"], ms_per_launch=ms,
                traffic=traffic_from_profiles(workload, stage))
     return out
+
+
+def train_launches_per_step(shape) -> int:
+    """Kernels of one training step: the forward with MOE_FLAG_TRAINING (always
+    unfused, plus the zeroing of xbuf's padding rows), then moe_layer_bwd:
+    combine backward and the zeroing of dyrow's padding rows, four expert
+    contractions of the backward plus the recomputed first one, the router
+    backward (the aux coefficients, then dlogits), the dispatch backward and
+    dWg (partial sums, then their reduction)."""
+    router = 3 if shape.dtype == 1 else 1
+    slots = 4 + (1 if shape.drop_policy == 1 and shape.cap_mode == 0 else 0)
+    fwd = router + slots + 1 + 1 + 2 + 1
+    bwd = 2 + 5 + 2 + 1 + 2
+    return fwd + bwd
+
+
+def bwd_stage_work(shape, kept: int, experts_used: int):
+    """Algorithmic bytes and flops of each kernel of moe_layer_bwd.  The dz
+    stage recomputes the first contraction (counted: it is the kernel's work);
+    weight gradients are written in fp32."""
+    b = 2
+    T, H, F, E, k = shape.T, shape.H, shape.F, shape.E, shape.k
+    sh = shape.n_shared
+    rows = kept + sh * T
+    nm1 = 2 if shape.act == 2 else 1
+    wexp = experts_used + sh
+    return {
+        "combine_bwd": {"flops": 0.0, "bytes": T * H * b + 2 * kept * H * b + sh * T * H * b + T * k * 16},
+        "dgrad_dh": {"flops": 2.0 * rows * H * F, "bytes": wexp * H * F * b + rows * H * b + rows * F * b},
+        "wgrad_w2": {"flops": 2.0 * rows * H * F, "bytes": rows * H * b + rows * F * b + wexp * H * F * 4},
+        "dact_dz": {"flops": 2.0 * rows * H * F * nm1,
+                    "bytes": wexp * nm1 * F * H * b + rows * H * b + rows * F * b + rows * F * nm1 * b},
+        "wgrad_w1": {"flops": 2.0 * rows * H * F * nm1, "bytes": rows * F * nm1 * b + rows * H * b + wexp * nm1 * F * H * 4},
+        "router_bwd": {"flops": 0.0, "bytes": 2 * T * E * 4 + T * k * 8},
+        "dgrad_dx": {"flops": 2.0 * rows * F * nm1 * H, "bytes": wexp * nm1 * F * H * b + rows * F * nm1 * b + rows * H * b},
+        "dispatch_bwd": {"flops": 2.0 * T * E * H,
+                         "bytes": kept * H * b + sh * T * H * b + T * H * b + T * E * 4 + E * H * 4 + T * k * 8},
+        "router_wgrad": {"flops": 2.0 * T * E * H, "bytes": T * E * 4 + T * H * b + E * H * 4},
+    }
 
 
 # ------------------------------------------------------------------ CPU oracle timing
@@ -354,6 +403,20 @@ def host_inputs(inp: dict):
             "uniform": None if inp.get("uniform") is None else inp["uniform"].cpu().numpy()}
 
 
+def oracle_train_sample_time(shape, inp_cpu: dict, dy, tokens: int):
+    """The oracle's forward and backward on the first `tokens` tokens as a layer of its own."""
+    import oracle.moe_oracle as O
+    import oracle.moe_oracle_bwd as OB
+    sub = shape.replace(T=tokens)
+    layer = O.OracleLayer.from_mapping(sub.as_dict())
+    add = None if inp_cpu["logit_add"] is None else inp_cpu["logit_add"][:tokens]
+    uni = None if inp_cpu.get("uniform") is None else inp_cpu["uniform"][:tokens]
+    t0 = time.perf_counter()
+    OB.layer_backward(layer, inp_cpu["x"][:tokens], inp_cpu["wg"], inp_cpu["w1"], inp_cpu["w2"], inp_cpu["w3"],
+                      inp_cpu["sw1"], inp_cpu["sw2"], inp_cpu["sw3"], dy=dy[:tokens], logit_add=add, uniform=uni)
+    return time.perf_counter() - t0
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -386,21 +449,31 @@ def run_reference(args, world, rank):
     inp = synth.make_inputs(shape, seed=args.seed, device=dev)
     host = host_inputs(inp)
     budget = max(0.05, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    run = lambda m: oracle_sample_time(shape, host, m)
+    what = "the oracle's whole layer"
+    if args.pass_ == "train":
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(args.seed + 1000)
+        dyh = torch.randn((shape.T, shape.H), generator=gen, device=dev).to(torch.bfloat16).to(
+            "cpu", torch.float64).numpy()
+        run = lambda m: oracle_train_sample_time(shape, host, dyh, m)
+        what = "the oracle's forward and backward"
     n = 16
-    t = oracle_sample_time(shape, host, n)
+    t = run(n)
     while t < budget * 0.5 and n < shape.T:
         n = min(shape.T, n * 2)
-        t = oracle_sample_time(shape, host, n)
+        t = run(n)
     for _ in range(args.warmup):
-        oracle_sample_time(shape, host, n)
-    times = [oracle_sample_time(shape, host, n) for _ in range(args.steps)]
+        run(n)
+    times = [run(n) for _ in range(args.steps)]
     ms = 1e3 * sum(times) / len(times)
     value = n / (ms / 1e3)
-    sample = f"the oracle's whole layer on the first {n} of {shape.T} tokens per step"
+    sample = f"{what} on the first {n} of {shape.T} tokens per step"
     print(json.dumps({"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 1,
                       "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
                       "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                      "config": {"workload": shape.name, "tokens_per_step": n},
+                      "config": {"workload": shape.name, "tokens_per_step": n,
+                                 "pass": "forward+backward" if args.pass_ == "train" else "forward"},
                       "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                                        "sample": sample},
                       "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
@@ -615,12 +688,190 @@ def run_ours(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def run_train(args, world, rank, local):
+    """One step = moe_layer_fwd with MOE_FLAG_TRAINING, then moe_layer_bwd with
+    a synthetic upstream gradient dy (and d_aux = d_z = 1)."""
+    import torch
+    from expert_dispatch_router_b200 import binding as B
+    from expert_dispatch_router_b200 import synth
+
+    B.load()                                     # raises if the CUDA library is missing
+    shape = workload_shape(args)
+    if shape.dtype != 1:
+        raise SystemExit("--pass train: the backward runs on bf16 layers only")
+    peaks = load_peaks()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp = synth.make_inputs(shape, seed=replica_seed(args.seed, rank), device="cuda")
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(replica_seed(args.seed, rank) + 1000)
+    T, H, F, E = shape.T, shape.H, shape.F, shape.E
+    dy = torch.randn((T, H), generator=gen, device=dev).to(torch.bfloat16)
+    cfg = B.make_cfg(shape, flags=B.MOE_FLAG_TRAINING)
+    ws = B.alloc_workspace(cfg)
+    wts = B.make_weights(inp)
+    sw = shape.act == synth.ACT_SWIGLU
+    g = dict(dw1=torch.empty((E, F, H), device=dev), dw2=torch.empty((E, H, F), device=dev),
+             dw3=torch.empty((E, F, H), device=dev) if sw else None)
+    if shape.n_shared:
+        g.update(dsw1=torch.empty((1, F, H), device=dev), dsw2=torch.empty((1, H, F), device=dev),
+                 dsw3=torch.empty((1, F, H), device=dev) if sw else None)
+    grads = B.make_weight_grads(g)
+    y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    aux = torch.empty(2, dtype=torch.float32, device=dev)
+    dx = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    dwg = torch.empty((E, H), dtype=torch.float32, device=dev)
+    flush_w = torch.empty(320 * 2**20 // 4, dtype=torch.float32, device=dev)
+    flush_r = torch.ones(320 * 2**20 // 4, dtype=torch.float32, device=dev)
+    flush_sink = torch.empty((), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def flush_l2():
+        flush_w.zero_()
+        torch.sum(flush_r, dim=0, out=flush_sink)
+
+    def layer(x, d, add, uni, fev=None, bev=None):
+        B.moe_layer_fwd(cfg, x, inp["wg"], add, uni, wts, y, aux, None, ws, stage_events=fev, stream=stream)
+        B.moe_layer_bwd(cfg, x, inp["wg"], wts, d, 1.0, 1.0, dx, dwg, grads, ws, stage_events=bev, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        flush_l2()
+        layer(inp["x"], dy, inp["logit_add"], inp["uniform"])
+    st = B.moe_sync_status(ws, stream)
+    if st != B.MOE_OK:
+        raise RuntimeError(f"device status after warm-up: {B.strerror(st)}")
+    wt = B.workspace_tensors(cfg, ws)
+    kept = int(wt["kept_count"].sum().item())
+    experts_used = int((wt["kept_count"] > 0).sum().item())
+
+    n_stage_steps = min(args.steps, 200)
+    ends = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    fevs = [[torch.cuda.Event(enable_timing=True) for _ in range(B.MOE_N_STAGE_EVENTS)] for _ in range(n_stage_steps)]
+    bevs = [[torch.cuda.Event(enable_timing=True) for _ in range(B.MOE_N_BWD_STAGE_EVENTS)]
+            for _ in range(n_stage_steps)]
+    for e in [x for pair in ends for x in pair] + [x for row in fevs + bevs for x in row]:
+        e.record(stream)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev.index) if rank == 0 else None
+    if sampler:
+        sampler.wait_first()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    for i in range(args.steps):
+        flush_l2()
+        ends[i][0].record(stream)
+        layer(inp["x"], dy, inp["logit_add"], inp["uniform"])
+        ends[i][1].record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    barrier(world)
+    for i in range(n_stage_steps):
+        flush_l2()
+        layer(inp["x"], dy, inp["logit_add"], inp["uniform"], fevs[i], bevs[i])
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = None
+    if sampler:
+        sampler.stop()
+        clocks = sampler.summary(t0, t1)
+    st = B.moe_sync_status(ws, stream)
+    if st != B.MOE_OK:
+        raise RuntimeError(f"device status after the timed region: {B.strerror(st)}")
+    ms_local = sum(a.elapsed_time(b) for a, b in ends) / args.steps
+    ms = max_over_ranks(ms_local, world)
+    value = job_tokens_per_s(T, world, ms)
+    fwd_ms = sum(e[0].elapsed_time(e[-1]) for e in fevs) / n_stage_steps
+    stage_ms = {name: sum(e[j].elapsed_time(e[j + 1]) for e in bevs) / n_stage_steps
+                for j, name in enumerate(B.BWD_STAGES)}
+    bwd_ms = sum(e[0].elapsed_time(e[-1]) for e in bevs) / n_stage_steps
+    work = bwd_stage_work(shape, kept, experts_used)
+    long_step = ms_local > 5.0
+    per_stage = {s_: roofline(s_, work, stage_ms[s_], peaks, shape.name, True, long_step) for s_ in B.BWD_STAGES}
+    dom = max(B.BWD_STAGES, key=lambda s_: stage_ms[s_])
+    roof = per_stage[dom]
+
+    # end to end: x and dy copied in from pinned host memory, the loss terms
+    # (aux, and the z-loss when on) read back, serially within each step
+    aux_n = 2 if shape.z_coef else 1
+    x_host = inp["x"].cpu().pin_memory()
+    dy_host = dy.cpu().pin_memory()
+    add_host = None if inp["logit_add"] is None else inp["logit_add"].cpu().pin_memory()
+    uni_host = None if inp["uniform"] is None else inp["uniform"].cpu().pin_memory()
+    xd, dyd = torch.empty_like(inp["x"]), torch.empty_like(dy)
+    addd = None if add_host is None else torch.empty_like(inp["logit_add"])
+    unid = None if uni_host is None else torch.empty_like(inp["uniform"])
+    aux_host = torch.empty(aux_n, dtype=torch.float32).pin_memory()
+    h2d = 2 * T * H * 2 + (0 if add_host is None else add_host.numel() * 4) + (0 if uni_host is None else T * 4)
+
+    def e2e_step():
+        xd.copy_(x_host, non_blocking=True)
+        dyd.copy_(dy_host, non_blocking=True)
+        if addd is not None:
+            addd.copy_(add_host, non_blocking=True)
+        if unid is not None:
+            unid.copy_(uni_host, non_blocking=True)
+        layer(xd, dyd, addd, unid)
+        aux_host.copy_(aux[:aux_n], non_blocking=True)
+
+    for _ in range(max(args.warmup, 3)):
+        e2e_step()
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    ea.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    eb.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(ea.elapsed_time(eb) / args.steps, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        host = host_inputs(inp)
+        dyh = dy.to("cpu", torch.float64).numpy()
+        n = min(T, 128)
+        t = oracle_train_sample_time(shape, host, dyh, n)
+        while t < 5.0 and n < T:
+            n = min(T, max(n * 2, int(n * 15.0 / max(t, 1e-3) * 0.8)))
+            t = oracle_train_sample_time(shape, host, dyh, n)
+        cpu = {"value": n / t, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"the oracle's forward and backward on the first {n} of {T} tokens as a batch of its own "
+                         f"({t:.1f} s, capacity recomputed for that batch)"}
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": shape.name, "pass": "forward+backward (moe_layer_fwd TRAINING + moe_layer_bwd)",
+                       "T": T, "H": H, "F": F, "E": E, "k": shape.k, "n_shared": shape.n_shared,
+                       "act": ["relu", "gelu", "swiglu"][shape.act], "kept_assignments": kept,
+                       "l2": "flushed before every step (320 MiB write + 320 MiB read, outside the timed events)",
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "weights": "linear-layer layout"},
+            "forward_ms": fwd_ms, "backward_ms": bwd_ms, "backward_stages_ms": stage_ms,
+            "stages_note": f"second timed pass of {n_stage_steps} steps with per-stage events",
+            "roofline": {k_: roof[k_] for k_ in ("bound", "achieved", "peak", "unit", "frac", "traffic", "peak_source")},
+            "roofline_detail": {s_: {k_: v[k_] for k_ in ("bound", "achieved", "unit", "frac", "ms_per_launch")}
+                                for s_, v in per_stage.items()},
+            "dominant_kernel": dom,
+            "e2e": {"value": job_tokens_per_s(T, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": 4 * aux_n, "pipelining": "none (copies serial with the step)"},
+            "gpu_launches": train_launches_per_step(shape) * args.steps,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     world, rank, local = dist_setup()
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.pass_ == "train":
+            run_train(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:

@@ -19,9 +19,13 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libmoe_b200.so")
 
 MOE_OK, MOE_EINVAL, MOE_EUNSUPPORTED, MOE_ECUDA, MOE_ETIMEOUT, MOE_EDEVICE, MOE_EWORKSPACE = range(7)
-MOE_FLAG_KEEP_LOGITS, MOE_FLAG_RANDOM_SECOND, MOE_FLAG_UNFUSED, MOE_FLAG_PACKED_WEIGHTS = 1, 2, 4, 8
+MOE_FLAG_KEEP_LOGITS, MOE_FLAG_RANDOM_SECOND, MOE_FLAG_UNFUSED, MOE_FLAG_PACKED_WEIGHTS, MOE_FLAG_TRAINING = \
+    1, 2, 4, 8, 16
 MOE_N_STAGE_EVENTS = 8
 STAGES = ("router", "slots", "dispatch", "ffn_gemm1", "ffn_gemm2", "combine", "aux")
+MOE_N_BWD_STAGE_EVENTS = 10
+BWD_STAGES = ("combine_bwd", "dgrad_dh", "wgrad_w2", "dact_dz", "wgrad_w1", "router_bwd", "dgrad_dx", "dispatch_bwd",
+              "router_wgrad")
 
 
 class MoeError(RuntimeError):
@@ -43,12 +47,18 @@ class moe_weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("w1", "w3", "w2", "sw1", "sw3", "sw2")]
 
 
+class moe_weight_grads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("dw1", "dw3", "dw2", "dsw1", "dsw3", "dsw2")]
+
+
 class moe_ws_views(ctypes.Structure):
     _fields_ = [("ids", ctypes.c_void_p), ("gates", ctypes.c_void_p), ("slot", ctypes.c_void_p),
                 ("expert_count", ctypes.c_void_p), ("kept_count", ctypes.c_void_p),
                 ("expert_offset", ctypes.c_void_p), ("row_token", ctypes.c_void_p), ("logits", ctypes.c_void_p),
                 ("xbuf", ctypes.c_void_p), ("hbuf", ctypes.c_void_p), ("ybuf", ctypes.c_void_p),
-                ("rows_max", ctypes.c_int64)]
+                ("rows_max", ctypes.c_int64), ("dgate", ctypes.c_void_p), ("dlogits", ctypes.c_void_p),
+                ("dyrow", ctypes.c_void_p), ("dh", ctypes.c_void_p), ("dz", ctypes.c_void_p),
+                ("dxrow", ctypes.c_void_p)]
 
 
 _lib = None
@@ -69,6 +79,8 @@ _SIGS = {
     "moe_aux_loss": [CFGP, P, P, P],
     "moe_layer_fwd": [CFGP, P, P, P, P, ctypes.POINTER(moe_weights), P, P, P, P, ctypes.c_size_t, P, P],
     "moe_activation_eval": [ctypes.c_int, P, P, P, ctypes.c_int64, P],
+    "moe_layer_bwd": [CFGP, P, P, ctypes.POINTER(moe_weights), P, ctypes.c_float, ctypes.c_float, P, P,
+                      ctypes.POINTER(moe_weight_grads), P, ctypes.c_size_t, P, P],
     "moe_sync_status": [P, P],
     "moe_packed_weight_bytes": [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, SZP],
     "moe_pack_weight": [P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, P, P],
@@ -211,6 +223,21 @@ def moe_layer_fwd(cfg, x, wg, logit_add, uniform, weights: moe_weights, y, aux, 
                                 ev, _stream(stream)), "moe_layer_fwd")
 
 
+def moe_layer_bwd(cfg, x, wg, weights: moe_weights, dy, d_aux, d_z, dx, dwg, grads: moe_weight_grads, ws,
+                  stage_events=None, stream=None):
+    ev = None
+    if stage_events is not None:
+        arr = (ctypes.c_void_p * MOE_N_BWD_STAGE_EVENTS)(*[e.cuda_event for e in stage_events])
+        ev = ctypes.cast(arr, ctypes.c_void_p)
+    _check(load().moe_layer_bwd(ctypes.byref(cfg), _ptr(x), _ptr(wg), ctypes.byref(weights), _ptr(dy), float(d_aux),
+                                float(d_z), _ptr(dx), _ptr(dwg), ctypes.byref(grads), _ptr(ws),
+                                ws.numel() * ws.element_size(), ev, _stream(stream)), "moe_layer_bwd")
+
+
+def make_weight_grads(g: dict) -> moe_weight_grads:
+    return moe_weight_grads(*(_ptr(g.get(n)) for n in ("dw1", "dw3", "dw2", "dsw1", "dsw3", "dsw2")))
+
+
 def moe_activation_eval(act, z, u, out, stream=None):
     _check(load().moe_activation_eval(int(act), _ptr(z), _ptr(u), _ptr(out), z.numel(), _stream(stream)),
            "moe_activation_eval")
@@ -288,4 +315,10 @@ def workspace_tensors(cfg: moe_cfg, ws: torch.Tensor) -> dict:
                ybuf=view_tensor(v.ybuf, (R, cfg.H), edt, ws), rows_max=R)
     if v.logits:
         out["logits"] = view_tensor(v.logits, (T, E), torch.float32, ws)
+    if v.dgate:
+        dzw = 2 * ((cfg.F + 63) // 64 * 64) if cfg.act == synth.ACT_SWIGLU else cfg.F
+        out.update(dgate=view_tensor(v.dgate, (T, k), torch.float32, ws),
+                   dlogits=view_tensor(v.dlogits, (T, E), torch.float32, ws),
+                   dyrow=view_tensor(v.dyrow, (R, cfg.H), edt, ws), dh=view_tensor(v.dh, (R, cfg.F), edt, ws),
+                   dz=view_tensor(v.dz, (R, dzw), edt, ws), dxrow=view_tensor(v.dxrow, (R, cfg.H), edt, ws))
     return out

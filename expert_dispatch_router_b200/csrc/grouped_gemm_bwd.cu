@@ -1,0 +1,544 @@
+// Grouped GEMMs of the expert FFN's backward pass on the sm_100a tensor cores.
+//
+// Method: the backward of "Expert-parallel MoE training"'s grouped expert MLPs
+// (the two permutations swap roles; every expert's rows are a 128-padded block
+// of the row layout).  For one expert with rows X, pre-activations z = X W1^T,
+// h = act(z), Y = h W2^T and output gradient dY (already gate-weighted):
+//   DGRAD  dh = dY W2,  dX = dz W1 (+ dz_up W3)   A = rows (K-major), B = weights
+//                                                  read along N (MN-major)
+//   DACT   dz = dh * act'(z) with z recomputed     A = X, B = W1 (| W3), like the
+//          on the tensor cores (SwiGLU: da, db)    forward's first contraction
+//   WGRAD  dW2 = dY^T h,  dW1 = dz^T X            A and B both rows read along
+//          (one output matrix per expert, K =      their feature dimension
+//          that expert's rows)                     (MN-major)
+// All three use the forward kernel's structure: one persistent CTA per SM, warp
+// 0 issues TMA loads into a ring of stages, warp 1 issues tcgen05.mma
+// (M=128, K=16, kind::f16, fp32 accumulators in TMEM, two 256-column buffers),
+// warps 2-17 drain the accumulators.  MN-major operands are loaded as boxes of
+// 64 features x 64 k (128-byte swizzle; 64-feature chunks 8 KB apart, 8-row k
+// groups 1 KB apart) and described to the MMA with the MN-major bit.
+// Every mbarrier wait is bounded.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_common.cuh"
+
+namespace moe {
+namespace gb {
+
+using namespace tcx;
+
+constexpr int BM = 128, BK = 64, BNMAX = 256;
+constexpr int A_BYTES = BM * BK * 2;                        // 16 KB
+constexpr int RING_BYTES = 4 * (A_BYTES + BNMAX * BK * 2);  // 192 KB
+constexpr int MAX_STAGES = 8;
+constexpr int EPI_WARPS = 16;
+constexpr int THREADS = 64 + EPI_WARPS * 32;
+constexpr int TMEM_COLS = 512;
+constexpr int STAGE_OUT_BYTES = 32 * 32 * 2;
+constexpr int STAGING_BYTES = EPI_WARPS * STAGE_OUT_BYTES;
+constexpr int SMEM_BYTES = RING_BYTES + STAGING_BYTES + 1024 + 256;
+constexpr int MN_CHUNK_BYTES = 64 * BK * 2;                 // one 64-feature x 64-k box: 8 KB
+
+enum Mode { DGRAD = 0, DACT = 1, WGRAD = 2 };
+
+struct BParams {
+  CUtensorMap tmA, tmAs;          // A (and the shared block's A when as_sep)
+  CUtensorMap tmB0, tmB1;         // routed B (DGRAD: map 1 after k_switch k blocks; DACT: SwiGLU up)
+  CUtensorMap tmSB0, tmSB1;       // shared expert's B (or, WGRAD with b_sep: the shared rows' B)
+  CUtensorMap tmD;                // bf16 output, box 32 x 32, 64-byte swizzle
+  const int32_t* off;             // [E+2]
+  DevStatus* status;
+  int mode, E, n_shared, act;
+  int64_t rows_max;
+  int K, N;                       // contraction length (DGRAD, DACT), output columns
+  int M;                          // WGRAD: output rows per expert
+  int k_switch;                   // DGRAD: k blocks read from tmB0 before tmB1 (0: never)
+  int as_sep, b_sep;              // shared block's A (DACT) / B (WGRAD) from a separate map, rows - off[E]
+  const __nv_bfloat16* dh;        // DACT: [rows_max, N] upstream gradient of h
+  int dz_ld;                      // DACT: row length of dz (N, or 2N for SwiGLU: da | db)
+  float *wout, *wout2;            // WGRAD: per-expert fp32 [M or m_split, N] (+ [M - m_split, N])
+  float *wsh, *wsh2;              // WGRAD: the shared expert's
+  int m_split;                    // WGRAD: output rows >= m_split go to wout2 / wsh2
+  int m_valid;                    // WGRAD: rows of each output part (rows beyond are padding, not stored)
+};
+
+// MN-major operand descriptor (128-byte swizzle): 64-feature chunks `lbo`
+// bytes apart, 8-row k groups 1 KB apart.
+__device__ __forceinline__ uint64_t mn_desc(uint32_t saddr, uint32_t lbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;
+  return d;
+}
+
+__device__ __forceinline__ float gelu_grad(float z) {
+  // d/dz [z Phi(z)] = Phi(z) + z phi(z); Phi from erf (Abramowitz & Stegun 7.1.26)
+  const float phi = 0.3989422804014327f * __expf(-0.5f * z * z);
+  return 0.5f * (1.0f + erf_as7126(z * 0.70710678118654752f)) + z * phi;
+}
+
+__global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __grid_constant__ BParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stage_base = smem;
+  uint8_t* staging = smem + RING_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + RING_BYTES + STAGING_BYTES);
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + MAX_STAGES);
+  const uint32_t tfull0 = smem_u32(bars + 2 * MAX_STAGES), tempty0 = smem_u32(bars + 2 * MAX_STAGES + 2);
+  const uint32_t drain = smem_u32(bars + 2 * MAX_STAGES + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * MAX_STAGES + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool swiglu = p.mode == DACT && p.act == MOE_ACT_SWIGLU;
+  const bool wgrad = p.mode == WGRAD;
+  const int a_mn = wgrad ? 1 : 0, b_mn = p.mode == DACT ? 0 : 1;
+  const int ngroups = p.E + (p.n_shared ? 1 : 0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < MAX_STAGES; ++s) { mbar_init(full0 + 8 * s, 1); mbar_init(empty0 + 8 * s, 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(tfull0 + 8 * b, 1); mbar_init(tempty0 + 8 * b, EPI_WARPS * 32); }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(smem_u32(tmem_slot)), "r"(TMEM_COLS) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();
+
+  // Tiles.  DGRAD / DACT: (128-row block of the row layout, N tile), the block's
+  // group by binary search.  WGRAD: (group, 128-row tile of M, N tile), the k
+  // blocks being the group's rows.
+  const int n_step = swiglu ? BNMAX / 2 : BNMAX;           // output columns per tile
+  const int bn = BNMAX;                                    // MMA N
+  const int n_tiles_n = (p.N + n_step - 1) / n_step;
+  const int64_t rows_used = min((int64_t)p.off[ngroups], p.rows_max);
+  const int m_tiles = wgrad ? (p.M + BM - 1) / BM : 0;
+  const int64_t n_tiles = wgrad ? (int64_t)ngroups * m_tiles * n_tiles_n : ((rows_used + BM - 1) / BM) * n_tiles_n;
+  const int nk = (p.K + BK - 1) / BK;
+  struct Tile {
+    int g, nt, kb0, kb1;
+    int64_t row0;                                          // DGRAD / DACT: first row; WGRAD: first output row m0
+  };
+  auto decode = [&](int64_t tile) -> Tile {
+    Tile d;
+    if (wgrad) {
+      d.nt = (int)(tile % n_tiles_n);
+      const int64_t rest = tile / n_tiles_n;
+      d.row0 = (rest % m_tiles) * BM;
+      d.g = (int)(rest / m_tiles);
+      d.kb0 = p.off[d.g] / BK;
+      d.kb1 = p.off[d.g + 1] / BK;
+    } else {
+      d.nt = (int)(tile % n_tiles_n);
+      d.row0 = (tile / n_tiles_n) * BM;
+      d.g = find_group(p.off, ngroups, d.row0);
+      d.kb0 = 0;
+      d.kb1 = nk;
+    }
+    return d;
+  };
+  const int b_bytes = bn * BK * 2;                         // 32 KB
+  const int stage_bytes = A_BYTES + b_bytes;
+  const int n_stages = min(MAX_STAGES, RING_BYTES / stage_bytes);
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t fills[MAX_STAGES] = {0, 0, 0, 0, 0, 0, 0, 0};
+      bool ok = true;
+      for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+        const Tile d = decode(tile);
+        const bool sh = d.g == p.E;
+        const int n0 = d.nt * n_step;
+        for (int kb = d.kb0; kb < d.kb1; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag)) { ok = false; break; }
+          const uint32_t sa = smem_u32(stage_base + stage * stage_bytes);
+          const uint32_t sb = sa + A_BYTES;
+          const uint32_t fb = full0 + 8 * stage;
+          mbar_expect_tx(fb, stage_bytes);
+          if (p.mode == WGRAD) {
+            // A: rows kb*64.. of the M-wide source, two 64-feature chunks
+            for (int i = 0; i < 2; ++i) tma_load_2d(sa + i * MN_CHUNK_BYTES, &p.tmA, (int)d.row0 + 64 * i, kb * BK, fb);
+            const bool bs = sh && p.b_sep;
+            const int krow = bs ? kb * BK - p.off[p.E] : kb * BK;
+            for (int j = 0; j < bn / 64; ++j)
+              tma_load_2d(sb + j * MN_CHUNK_BYTES, bs ? &p.tmSB0 : &p.tmB0, n0 + 64 * j, krow, fb);
+          } else {
+            const bool sep = sh && p.as_sep;
+            const int arow = (int)(sep ? d.row0 - p.off[p.E] : d.row0);
+            tma_load_2d(sa, sep ? &p.tmAs : &p.tmA, kb * BK, arow, fb);
+            const int z = sh ? 0 : d.g;
+            if (p.mode == DGRAD) {
+              const bool second = p.k_switch > 0 && kb >= p.k_switch;
+              const CUtensorMap* mb = sh ? (second ? &p.tmSB1 : &p.tmSB0) : (second ? &p.tmB1 : &p.tmB0);
+              const int kk = (second ? kb - p.k_switch : kb) * BK;
+              for (int j = 0; j < bn / 64; ++j) tma_load_3d(sb + j * MN_CHUNK_BYTES, mb, n0 + 64 * j, kk, z, fb);
+            } else if (swiglu) {
+              tma_load_3d(sb, sh ? &p.tmSB0 : &p.tmB0, kb * BK, n0, z, fb);                // gate rows
+              tma_load_3d(sb + b_bytes / 2, sh ? &p.tmSB1 : &p.tmB1, kb * BK, n0, z, fb);  // up rows
+            } else {
+              for (int b = 0; b < 2; ++b) tma_load_3d(sb + b * (b_bytes / 2), sh ? &p.tmSB0 : &p.tmB0, kb * BK, n0 + 128 * b, z, fb);
+            }
+          }
+          fills[stage]++;
+          if (++stage == n_stages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        set_status(p.status, MOE_ETIMEOUT, 20);
+      }
+      for (int s = 0; s < n_stages; ++s)
+        if (fills[s]) {
+          const long long t0 = clock64();
+          while (!mbar_try_wait(full0 + 8 * s, (fills[s] - 1) & 1u) && clock64() - t0 < kWaitCycles) {}
+        }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      const uint32_t idesc = make_idesc(bn, BM, a_mn, b_mn);
+      for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+        const Tile d = decode(tile);
+        if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BNMAX);
+        for (int kb = d.kb0; kb < d.kb1; ++kb) {
+          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(stage_base + stage * stage_bytes);
+          const uint32_t sb = sa + A_BYTES;
+          const uint64_t ad = a_mn ? mn_desc(sa, MN_CHUNK_BYTES) : sw128_desc(sa);
+          const uint64_t bd = b_mn ? mn_desc(sb, MN_CHUNK_BYTES) : sw128_desc(sb);
+          const uint64_t astep = a_mn ? 128 : 2, bstep = b_mn ? 128 : 2;   // 16 k: 2 KB (MN-major) or 32 B
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma(d_tmem, ad + astep * kk, bd + bstep * kk, idesc, ((kb - d.kb0) | kk) != 0 ? 1u : 0u);
+          umma_commit(empty0 + 8 * stage);
+          if (++stage == n_stages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(tfull0 + 8 * acc);         // also when the group had no rows: nothing to wait for
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        set_status(p.status, MOE_ETIMEOUT, 21);
+      }
+      umma_commit(drain);
+      const long long t0 = clock64();
+      while (!mbar_try_wait(drain, 0) && clock64() - t0 < kWaitCycles) {}
+    }
+  } else {
+    // ---------------- epilogue
+    const int ew = warp - 2;
+    const int sub = warp & 3;
+    const int quarter = ew >> 2;
+    const int row_in_tile = sub * 32 + lane;
+    const uint32_t stage_out = smem_u32(staging + ew * STAGE_OUT_BYTES);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    // bf16 store of this warp's 32 x 32 sub-tile through its staging buffer
+    auto store_bf16 = [&](const float (&v)[32], int col, int64_t row_base) {
+      if (lane == 0) bulk_wait_read0();
+      __syncwarp();
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        st_shared_v4(stage_out + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4), pack_bf16(v[8 * q], v[8 * q + 1]),
+                     pack_bf16(v[8 * q + 2], v[8 * q + 3]), pack_bf16(v[8 * q + 4], v[8 * q + 5]),
+                     pack_bf16(v[8 * q + 6], v[8 * q + 7]));
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(&p.tmD, stage_out, col, (int)row_base);
+        bulk_commit();
+      }
+    };
+    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+      if (!mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag)) {
+        *abort_flag = 1;
+        set_status(p.status, MOE_ETIMEOUT, 22);
+        break;
+      }
+      tc_fence_after();
+      const Tile d = decode(tile);
+      const bool empty = d.kb1 <= d.kb0;
+      const int ncol0 = d.nt * n_step;
+      const uint32_t tbase = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * BNMAX);
+      for (int c = quarter * 32; c < n_step; c += 4 * 32) {
+        const int col = ncol0 + c;
+        if (col >= p.N) break;
+        __syncwarp();                                // converged for the warp-wide tcgen05.ld
+        float v[32];
+        if (empty) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+        } else {
+          tmem_ld(tbase + (uint32_t)c, v, 32);
+        }
+        if (p.mode == WGRAD) {
+          tmem_wait_ld();
+          const int m = (int)d.row0 + row_in_tile;
+          if (m >= p.M) continue;
+          const bool hi = m >= p.m_split;
+          const int mr = hi ? m - p.m_split : m;
+          if (mr >= p.m_valid) continue;
+          float* base = d.g == p.E ? (hi ? p.wsh2 : p.wsh) : (hi ? p.wout2 : p.wout) + (int64_t)d.g * p.m_valid * p.N;
+          float* drow = base + (int64_t)mr * p.N + col;
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            if (col + 4 * q < p.N)
+              *reinterpret_cast<float4*>(drow + 4 * q) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          continue;
+        }
+        const int64_t row_base = d.row0 + sub * 32;
+        if (p.mode == DGRAD) {
+          tmem_wait_ld();
+          store_bf16(v, col, row_base);
+          continue;
+        }
+        // DACT: z (and the SwiGLU up projection) recomputed; dz = dh * act'(z)
+        float u[32];
+        if (swiglu) tmem_ld(tbase + (uint32_t)(BNMAX / 2 + c), u, 32);
+        tmem_wait_ld();
+        const int64_t grow = d.row0 + row_in_tile;
+        const __nv_bfloat16* src = p.dh + grow * (int64_t)p.N + col;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          // dh for 8 columns; columns past N read as zero, so dz is zero there
+          const int4 w = grow < p.rows_max && col + 8 * q < p.N ? ld_nc_v4(src + 8 * q) : make_int4(0, 0, 0, 0);
+          const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&w);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float gi = __bfloat162float(e[i]);
+            const float z = v[8 * q + i];
+            if (swiglu) {
+              const float s = 1.0f / (1.0f + __expf(-z));
+              v[8 * q + i] = gi * u[8 * q + i] * s * (1.0f + z * (1.0f - s));   // da
+              u[8 * q + i] = gi * z * s;                                        // db = dh * silu(a)
+            } else {
+              v[8 * q + i] = p.act == MOE_ACT_RELU ? (z > 0.0f ? gi : 0.0f) : gi * gelu_grad(z);
+            }
+          }
+        }
+        store_bf16(v, col, row_base);
+        if (swiglu) store_bf16(u, p.dz_ld / 2 + col, row_base);             // db at column Fp + col
+      }
+      tc_fence_before();
+      mbar_arrive(tempty0 + 8 * acc);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+    if (lane == 0) bulk_wait0();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  pdl_trigger();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem_base), "r"(TMEM_COLS) : "memory");
+  }
+}
+
+// ---------------------------------------------------------------- host side
+// [rows, W] bf16 read along W: box 64 x 64 (MN-major operand)
+static bool make_map_mn_rows(CUtensorMap* m, const void* base, int64_t rows, int W) {
+  MapKey key;
+  memset(&key, 0, sizeof(key));
+  key.base = base;
+  key.rank = 2;
+  key.swizzle = CU_TENSOR_MAP_SWIZZLE_128B;
+  key.dims[0] = (cuuint64_t)W;
+  key.dims[1] = (cuuint64_t)rows;
+  key.strides[0] = (cuuint64_t)W * 2;
+  key.box[0] = 64;
+  key.box[1] = 64;
+  return encode_cached(m, key);
+}
+// weights [G, K, N] bf16 read along N: box 64 x 64 x 1 (MN-major operand)
+static bool make_map_mn_weights(CUtensorMap* m, const void* base, int G, int K, int N) {
+  MapKey key;
+  memset(&key, 0, sizeof(key));
+  key.base = base;
+  key.rank = 3;
+  key.swizzle = CU_TENSOR_MAP_SWIZZLE_128B;
+  key.dims[0] = (cuuint64_t)N;
+  key.dims[1] = (cuuint64_t)K;
+  key.dims[2] = (cuuint64_t)G;
+  key.strides[0] = (cuuint64_t)N * 2;
+  key.strides[1] = (cuuint64_t)K * N * 2;
+  key.box[0] = 64;
+  key.box[1] = 64;
+  key.box[2] = 1;
+  return encode_cached(m, key);
+}
+// [rows, K] bf16 read along K: box 64 x 128 (K-major A)
+static bool make_map_k_rows(CUtensorMap* m, const void* base, int64_t rows, int K) {
+  MapKey key;
+  memset(&key, 0, sizeof(key));
+  key.base = base;
+  key.rank = 2;
+  key.swizzle = CU_TENSOR_MAP_SWIZZLE_128B;
+  key.dims[0] = (cuuint64_t)K;
+  key.dims[1] = (cuuint64_t)rows;
+  key.strides[0] = (cuuint64_t)K * 2;
+  key.box[0] = BK;
+  key.box[1] = BM;
+  return encode_cached(m, key);
+}
+// weights [G, N, K] bf16 read along K: box 64 x 128 x 1 (K-major B)
+static bool make_map_k_weights(CUtensorMap* m, const void* base, int G, int N, int K) {
+  MapKey key;
+  memset(&key, 0, sizeof(key));
+  key.base = base;
+  key.rank = 3;
+  key.swizzle = CU_TENSOR_MAP_SWIZZLE_128B;
+  key.dims[0] = (cuuint64_t)K;
+  key.dims[1] = (cuuint64_t)N;
+  key.dims[2] = (cuuint64_t)G;
+  key.strides[0] = (cuuint64_t)K * 2;
+  key.strides[1] = (cuuint64_t)N * K * 2;
+  key.box[0] = BK;
+  key.box[1] = 128;
+  key.box[2] = 1;
+  return encode_cached(m, key);
+}
+// bf16 output [rows, W], box 32 x 32, 64-byte swizzle (TMA store)
+static bool make_map_out(CUtensorMap* m, const void* base, int64_t rows, int W) {
+  MapKey key;
+  memset(&key, 0, sizeof(key));
+  key.base = base;
+  key.rank = 2;
+  key.swizzle = CU_TENSOR_MAP_SWIZZLE_64B;
+  key.dims[0] = (cuuint64_t)W;
+  key.dims[1] = (cuuint64_t)rows;
+  key.strides[0] = (cuuint64_t)W * 2;
+  key.box[0] = 32;
+  key.box[1] = 32;
+  return encode_cached(m, key);
+}
+
+static cudaError_t launch(BParams& k, int64_t max_tiles, cudaStream_t stream) {
+  cudaError_t e = ensure_smem(grouped_gemm_bwd_kernel, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const int sms = sm_count();
+  const int grid = (int)(max_tiles < sms ? (max_tiles > 0 ? max_tiles : 1) : sms);
+  launch_pdl(grouped_gemm_bwd_kernel, grid, THREADS, SMEM_BYTES, stream, k);
+  return cudaGetLastError();
+}
+
+}  // namespace gb
+
+cudaError_t launch_bwd_dgrad(const BwdGemm& q, cudaStream_t stream) {
+  using namespace gb;
+  if (q.rows_max == 0) return cudaSuccess;
+  if (encode_fn() == nullptr) return cudaErrorNotSupported;
+  BParams k{};
+  const int G = q.E;
+  bool ok = make_map_k_rows(&k.tmA, q.a, q.rows_max, q.K);
+  k.tmAs = k.tmA;
+  // map 0 covers the first q.K0 k of B (rows beyond read as zero); with
+  // k_switch, A's k blocks from k_switch on use map 1 (also q.K0 deep)
+  ok = ok && make_map_mn_weights(&k.tmB0, q.b0, G, q.K0, q.N);
+  ok = ok && make_map_mn_weights(&k.tmB1, q.b1 ? q.b1 : q.b0, G, q.K0, q.N);
+  ok = ok && make_map_mn_weights(&k.tmSB0, q.sb0 ? q.sb0 : q.b0, 1, q.K0, q.N);
+  ok = ok && make_map_mn_weights(&k.tmSB1, q.sb1 ? q.sb1 : (q.sb0 ? q.sb0 : q.b0), 1, q.K0, q.N);
+  ok = ok && make_map_out(&k.tmD, q.out, q.rows_max, q.N);
+  if (!ok) return cudaErrorInvalidValue;
+  k.off = q.off;
+  k.status = q.status;
+  k.mode = DGRAD;
+  k.E = q.E;
+  k.n_shared = q.n_shared;
+  k.rows_max = q.rows_max;
+  k.K = q.K;
+  k.N = q.N;
+  k.k_switch = q.k_switch;
+  return launch(k, (q.rows_max / BM) * ((q.N + BNMAX - 1) / BNMAX), stream);
+}
+
+cudaError_t launch_bwd_dact(const BwdGemm& q, cudaStream_t stream) {
+  using namespace gb;
+  if (q.rows_max == 0) return cudaSuccess;
+  if (encode_fn() == nullptr) return cudaErrorNotSupported;
+  BParams k{};
+  bool ok = make_map_k_rows(&k.tmA, q.a, q.rows_max, q.K);
+  ok = ok && make_map_k_rows(&k.tmAs, q.a_shared ? q.a_shared : q.a, q.a_shared ? q.T : q.rows_max, q.K);
+  ok = ok && make_map_k_weights(&k.tmB0, q.b0, q.E, q.N, q.K);
+  ok = ok && make_map_k_weights(&k.tmB1, q.b1 ? q.b1 : q.b0, q.E, q.N, q.K);
+  ok = ok && make_map_k_weights(&k.tmSB0, q.sb0 ? q.sb0 : q.b0, 1, q.N, q.K);
+  ok = ok && make_map_k_weights(&k.tmSB1, q.sb1 ? q.sb1 : (q.sb0 ? q.sb0 : q.b0), 1, q.N, q.K);
+  const int ld = q.act == MOE_ACT_SWIGLU ? 2 * ((q.N + BK - 1) / BK * BK) : q.N;   // da | db, db at column Fp
+  ok = ok && make_map_out(&k.tmD, q.out, q.rows_max, ld);
+  if (!ok) return cudaErrorInvalidValue;
+  k.off = q.off;
+  k.status = q.status;
+  k.mode = DACT;
+  k.E = q.E;
+  k.n_shared = q.n_shared;
+  k.act = q.act;
+  k.rows_max = q.rows_max;
+  k.K = q.K;
+  k.N = q.N;
+  k.as_sep = q.a_shared != nullptr;
+  k.dh = static_cast<const __nv_bfloat16*>(q.dh);
+  k.dz_ld = ld;
+  const int n_step = q.act == MOE_ACT_SWIGLU ? BNMAX / 2 : BNMAX;
+  return launch(k, (q.rows_max / BM) * ((q.N + n_step - 1) / n_step), stream);
+}
+
+cudaError_t launch_bwd_wgrad(const BwdGemm& q, cudaStream_t stream) {
+  using namespace gb;
+  if (encode_fn() == nullptr) return cudaErrorNotSupported;
+  BParams k{};
+  bool ok = make_map_mn_rows(&k.tmA, q.a, q.rows_max > 0 ? q.rows_max : 1, q.M);
+  ok = ok && make_map_mn_rows(&k.tmB0, q.b0, q.rows_max > 0 ? q.rows_max : 1, q.N);
+  ok = ok && make_map_mn_rows(&k.tmSB0, q.b_shared ? q.b_shared : q.b0, q.b_shared ? q.T : (q.rows_max > 0 ? q.rows_max : 1),
+                              q.N);
+  k.tmAs = k.tmA;
+  k.tmB1 = k.tmB0;
+  k.tmSB1 = k.tmSB0;
+  k.tmD = k.tmA;                                    // unused: fp32 stores
+  if (!ok) return cudaErrorInvalidValue;
+  k.off = q.off;
+  k.status = q.status;
+  k.mode = WGRAD;
+  k.E = q.E;
+  k.n_shared = q.n_shared;
+  k.rows_max = q.rows_max;
+  k.K = 0;
+  k.N = q.N;
+  k.M = q.M;
+  k.b_sep = q.b_shared != nullptr;
+  k.wout = q.w_out;
+  k.wout2 = q.w_out2;
+  k.wsh = q.w_sh;
+  k.wsh2 = q.w_sh2;
+  k.m_split = q.m_split > 0 ? q.m_split : q.M;
+  k.m_valid = q.m_valid > 0 ? q.m_valid : q.M;
+  const int64_t tiles = (int64_t)(q.E + (q.n_shared ? 1 : 0)) * ((q.M + BM - 1) / BM) * ((q.N + BNMAX - 1) / BNMAX);
+  return launch(k, tiles, stream);
+}
+
+}  // namespace moe

@@ -37,6 +37,54 @@ cudaError_t launch_router(const RouterParams& p, bool bf16, cudaStream_t stream)
 // zsum_part (or null): per-CTA sums of lse^2; aux[1] = z_coef * their mean.
 cudaError_t launch_aux(const float* psum_part, const int32_t* cnt_part, const float* zsum_part, int nblk, int E,
                        int64_t T, int k, float alpha, float z_coef, double* term, float* aux, cudaStream_t stream);
+// Router backward: dlogits [T,E] from dgate [T,k], the aux loss (through P_i,
+// fcoef[e] = d_aux * alpha * E * f_e / T, computed here from cnt_part) and the
+// z-loss (zc = d_z * z_coef).
+struct RouterBwdParams {
+  const float* logits;      // [T,E] the forward's
+  const float* dgate;       // [T,k]
+  const float* fcoef;       // [E]
+  float* dlogits;           // [T,E]
+  int64_t T;
+  int E, k, score, renorm;
+  float zc;
+};
+cudaError_t launch_router_bwd(const RouterBwdParams& p, const int32_t* cnt_part, int nblk, float d_aux_alpha,
+                              float* fcoef, cudaStream_t stream);
+
+// Backward permutations (backward.cu).
+struct CombineBwdParams {
+  const __nv_bfloat16* dy;  // [T,H]
+  const __nv_bfloat16* ybuf;// [rows,H] the forward's un-gated expert rows
+  const int32_t* ids;
+  const int32_t* slot;
+  const float* gates;
+  const int32_t* off;
+  __nv_bfloat16* dyrow;     // [rows,H]
+  float* dgate;             // [T,k]
+  int64_t T, rows_max;
+  int H, E, k, n_shared;
+};
+cudaError_t launch_combine_bwd(const CombineBwdParams& p, cudaStream_t stream);
+struct DispatchBwdParams {
+  const __nv_bfloat16* dxrow;   // [rows,H]
+  const float* dlogits;         // [T,E]
+  const float* wg;              // [E,H]
+  const int32_t* ids;
+  const int32_t* slot;
+  const int32_t* off;
+  __nv_bfloat16* dx;            // [T,H]
+  int64_t T, rows_max;
+  int H, E, k, n_shared;
+};
+cudaError_t launch_dispatch_bwd(const DispatchBwdParams& p, cudaStream_t stream);
+cudaError_t launch_zero_pad_rows(void* buf, int width, const int32_t* row_token, const int32_t* off, int ngroups,
+                                 int64_t rows_max, cudaStream_t stream);
+int dwg_chunks(int64_t T);
+// dwg [E,H] = dlogits^T x (part: dwg_chunks(T) * E * H floats of scratch)
+cudaError_t launch_router_wgrad(const float* dlogits, const void* x, int64_t T, int E, int H, float* part,
+                                float* dwg, cudaStream_t stream);
+
 // Evaluates the GEMM epilogue's activation: out = act(z) (ReLU, GELU) or silu(z) * u (SwiGLU).
 cudaError_t launch_activation_eval(int act, const float* z, const float* u, float* out, int64_t n,
                                    cudaStream_t stream);
@@ -130,6 +178,34 @@ struct GemmParams {
   int b_packed;             // 1: b0/b1/sb0/sb1 are packed (launch_pack_weight)
 };
 cudaError_t launch_grouped_gemm(const GemmParams& p, cudaStream_t stream);
+
+// Grouped GEMMs of the backward pass (grouped_gemm_bwd.cu).
+//   dgrad: out[rows, N] = a[rows, K] * B, B the weights [G, K0, N] read along N
+//          (k blocks >= k_switch from b1: SwiGLU's [W1; W3]); shared rows use sb0/sb1.
+//   dact:  out = dz[rows, ld] from z = a[rows, K] * b0^T (and the up projection
+//          b1 for SwiGLU, ld = 2 round_up(N, 64), db at column ld / 2) and dh[rows, N].
+//   wgrad: per expert g, w_out[g] = a[rows_g, M]^T * b0[rows_g, N] (fp32); output rows
+//          >= m_split go to w_out2 (m_valid rows each); the shared block to w_sh / w_sh2,
+//          its b rows from b_shared (row - off[E]) when given.
+struct BwdGemm {
+  const void* a;
+  const void* a_shared;     // dact: the shared block's A rows (x), or null
+  const void* b0;
+  const void* b1;
+  const void* sb0;
+  const void* sb1;
+  const void* b_shared;     // wgrad: the shared block's B rows (x), or null
+  void* out;                // dgrad / dact: bf16 output
+  const void* dh;           // dact
+  float *w_out, *w_out2, *w_sh, *w_sh2;
+  const int32_t* off;
+  DevStatus* status;
+  int64_t T, rows_max;
+  int K, K0, N, M, E, n_shared, act, k_switch, m_split, m_valid;
+};
+cudaError_t launch_bwd_dgrad(const BwdGemm& q, cudaStream_t stream);
+cudaError_t launch_bwd_dact(const BwdGemm& q, cudaStream_t stream);
+cudaError_t launch_bwd_wgrad(const BwdGemm& q, cudaStream_t stream);
 
 // Packed weight layout for the grouped GEMM: w [G, N, K] bf16 (K contiguous) ->
 // [G][ceil(N/128)][ceil(K/64)][128][64], zero-padded, so every TMA box of 128

@@ -16,7 +16,7 @@ constexpr int64_t kMaxCf = int64_t(1) << 20;
 
 struct Layout {
   size_t status, psum, cnt, zsum, term, chunk, cum, lkey, lidx, ids, gates, slot, ecount, kept, off, rowtok, logits, lparts, planes, xbuf,
-      hbuf, ybuf;
+      hbuf, ybuf, dyrow, dh, dz, dxrow, dgate, dlog, fcoef, dwgp;
   size_t total;
   int nblk_router, nchunk;
   int64_t rows_max;
@@ -35,7 +35,8 @@ bool valid_cfg(const moe_cfg* c) {
   if (c->cap_mode == MOE_CAP_CAPACITY && (c->cf_num <= 0 || c->cf_den <= 0)) return false;
   if (c->min_capacity < 0) return false;
   if (!(c->z_coef >= 0.0f) || isinf(c->z_coef)) return false;
-  if (c->flags & ~(MOE_FLAG_KEEP_LOGITS | MOE_FLAG_RANDOM_SECOND | MOE_FLAG_UNFUSED | MOE_FLAG_PACKED_WEIGHTS))
+  if (c->flags & ~(MOE_FLAG_KEEP_LOGITS | MOE_FLAG_RANDOM_SECOND | MOE_FLAG_UNFUSED | MOE_FLAG_PACKED_WEIGHTS |
+                   MOE_FLAG_TRAINING))
     return false;
   if ((c->flags & MOE_FLAG_PACKED_WEIGHTS) && c->dtype != MOE_DTYPE_BF16) return false;
   if (c->drop_policy != MOE_DROP_POSITION && c->drop_policy != MOE_DROP_PROBS) return false;
@@ -50,6 +51,11 @@ int check_cfg(const moe_cfg* c) {
   if (c->cap_mode == MOE_CAP_CAPACITY && (c->cf_num > kMaxCf || c->cf_den > kMaxCf)) return MOE_EUNSUPPORTED;
   if (c->T * (int64_t)c->k >= (int64_t(1) << 31)) return MOE_EUNSUPPORTED;
   return MOE_OK;
+}
+
+bool training(const moe_cfg* c) { return (c->flags & MOE_FLAG_TRAINING) != 0; }
+int dz_width(const moe_cfg* c) {                 // dz row length: F, or da | db with db at round_up(F, 64)
+  return c->act == MOE_ACT_SWIGLU ? 2 * ((c->F + 63) / 64 * 64) : c->F;
 }
 
 int64_t capacity_of(const moe_cfg* c) {
@@ -107,12 +113,21 @@ Layout layout_of(const moe_cfg* c) {
   L.off = take(sizeof(int32_t) * (E + 2));
   L.rowtok = take(sizeof(int32_t) * (size_t)L.rows_max);
   const bool tc_router = c->dtype == MOE_DTYPE_BF16;   // bf16 x: router logits on the tensor cores
-  L.logits = take(((c->flags & MOE_FLAG_KEEP_LOGITS) || tc_router) ? sizeof(float) * T * E : 0);
+  L.logits = take(((c->flags & (MOE_FLAG_KEEP_LOGITS | MOE_FLAG_TRAINING)) || tc_router) ? sizeof(float) * T * E : 0);
   L.lparts = take(tc_router ? sizeof(float) * 3 * T * E : 0);   // router GEMM partials
   L.planes = take(tc_router ? sizeof(uint16_t) * E * 3 * (size_t)router_plane_width(c->H) : 0);
   L.xbuf = take(esz * (size_t)L.rows_max * c->H);
   L.hbuf = take(esz * (size_t)L.rows_max * c->F);
   L.ybuf = take(esz * (size_t)L.rows_max * c->H);
+  const bool tr = training(c);
+  L.dyrow = take(tr ? esz * (size_t)L.rows_max * c->H : 0);
+  L.dh = take(tr ? esz * (size_t)L.rows_max * c->F : 0);
+  L.dz = take(tr ? esz * (size_t)L.rows_max * dz_width(c) : 0);
+  L.dxrow = take(tr ? esz * (size_t)L.rows_max * c->H : 0);
+  L.dgate = take(tr ? sizeof(float) * T * k : 0);
+  L.dlog = take(tr ? sizeof(float) * T * E : 0);
+  L.fcoef = take(tr ? sizeof(float) * E : 0);
+  L.dwgp = take(tr ? sizeof(float) * (size_t)dwg_chunks(c->T) * E * c->H : 0);
   L.total = o;
   return L;
 }
@@ -368,11 +383,18 @@ int moe_workspace_views(const moe_cfg* cfg, void* ws, moe_ws_views* v) {
   v->kept_count = at<int32_t>(ws, L.kept);
   v->expert_offset = at<int32_t>(ws, L.off);
   v->row_token = at<int32_t>(ws, L.rowtok);
-  v->logits = (cfg->flags & MOE_FLAG_KEEP_LOGITS) ? at<float>(ws, L.logits) : nullptr;
+  v->logits = (cfg->flags & (MOE_FLAG_KEEP_LOGITS | MOE_FLAG_TRAINING)) ? at<float>(ws, L.logits) : nullptr;
   v->xbuf = at<void>(ws, L.xbuf);
   v->hbuf = at<void>(ws, L.hbuf);
   v->ybuf = at<void>(ws, L.ybuf);
   v->rows_max = L.rows_max;
+  const bool tr = training(cfg);
+  v->dgate = tr ? at<float>(ws, L.dgate) : nullptr;
+  v->dlogits = tr ? at<float>(ws, L.dlog) : nullptr;
+  v->dyrow = tr ? at<void>(ws, L.dyrow) : nullptr;
+  v->dh = tr ? at<void>(ws, L.dh) : nullptr;
+  v->dz = tr ? at<void>(ws, L.dz) : nullptr;
+  v->dxrow = tr ? at<void>(ws, L.dxrow) : nullptr;
   return MOE_OK;
 }
 
@@ -479,7 +501,7 @@ int moe_layer_fwd(const moe_cfg* cfg, const void* x, const float* wg, const floa
   int32_t* off = at<int32_t>(ws, L.off);
   void* xbuf = at<void>(ws, L.xbuf);
   void* ybuf = at<void>(ws, L.ybuf);
-  float* logits = (cfg->flags & MOE_FLAG_KEEP_LOGITS) ? at<float>(ws, L.logits) : nullptr;
+  float* logits = (cfg->flags & (MOE_FLAG_KEEP_LOGITS | MOE_FLAG_TRAINING)) ? at<float>(ws, L.logits) : nullptr;
 
   if ((st = record(stage_events, 0, s)) != MOE_OK) return st;
   if ((st = run_route(cfg, L, x, wg, logit_add, nullptr, uniform, ids, gates, logits, ws, s)) != MOE_OK) return st;
@@ -494,7 +516,7 @@ int moe_layer_fwd(const moe_cfg* cfg, const void* x, const float* wg, const floa
   // second one's epilogue.  With more rows per expert the contractions are fed
   // from L2, where the TMA loads of a dispatched buffer feed faster than
   // per-row cp.async gathers.
-  const bool fuse = cfg->dtype == MOE_DTYPE_BF16 && !(cfg->flags & MOE_FLAG_UNFUSED) &&
+  const bool fuse = cfg->dtype == MOE_DTYPE_BF16 && !(cfg->flags & (MOE_FLAG_UNFUSED | MOE_FLAG_TRAINING)) &&
                     cfg->T * cfg->k <= 2 * kRowPad * (int64_t)cfg->E;
   const bool fuse_combine = fuse && cfg->k == 1 && cfg->n_shared == 0;
   int32_t* rowtok = at<int32_t>(ws, L.rowtok);
@@ -506,6 +528,10 @@ int moe_layer_fwd(const moe_cfg* cfg, const void* x, const float* wg, const floa
   pp.src = x;
   pp.dst = xbuf;
   if (!fuse && launch_dispatch(pp, s) != cudaSuccess) return MOE_ECUDA;
+  // training: padding rows of xbuf are zero (the weight gradients read them)
+  if (training(cfg) && launch_zero_pad_rows(xbuf, cfg->H, rowtok, off, cfg->E + (cfg->n_shared ? 1 : 0), L.rows_max,
+                                            s) != cudaSuccess)
+    return MOE_ECUDA;
   if ((st = record(stage_events, 3, s)) != MOE_OK) return st;
   if ((st = run_ffn(cfg, L, xbuf, x, off, w, ybuf, ws, s, stage_events ? stage_events + 4 : nullptr,
                     fuse ? rowtok : nullptr, fuse_combine ? y : nullptr, fuse_combine ? gates : nullptr,
@@ -521,6 +547,170 @@ int moe_layer_fwd(const moe_cfg* cfg, const void* x, const float* wg, const floa
                         s) != cudaSuccess)
       return MOE_ECUDA;
   return record(stage_events, 7, s);
+}
+
+int moe_layer_bwd(const moe_cfg* cfg, const void* x, const float* wg, const moe_weights* w, const void* dy,
+                  float d_aux, float d_z, void* dx, float* dwg, const moe_weight_grads* dw, void* ws, size_t ws_bytes,
+                  const moe_event_t* stage_events, moe_stream_t stream) {
+  int st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  st = check_weights(cfg, w);
+  if (st != MOE_OK) return st;
+  if (!training(cfg)) return MOE_EINVAL;
+  if (cfg->dtype != MOE_DTYPE_BF16 || (cfg->flags & MOE_FLAG_PACKED_WEIGHTS)) return MOE_EUNSUPPORTED;
+  if (ws == nullptr || dw == nullptr || dwg == nullptr || dw->dw1 == nullptr || dw->dw2 == nullptr) return MOE_EINVAL;
+  if (cfg->act == MOE_ACT_SWIGLU && dw->dw3 == nullptr) return MOE_EINVAL;
+  if (cfg->n_shared && (dw->dsw1 == nullptr || dw->dsw2 == nullptr ||
+                        (cfg->act == MOE_ACT_SWIGLU && dw->dsw3 == nullptr)))
+    return MOE_EINVAL;
+  if (cfg->T > 0 && (x == nullptr || wg == nullptr || dy == nullptr || dx == nullptr)) return MOE_EINVAL;
+  const Layout L = layout_of(cfg);
+  if (ws_bytes < L.total) return MOE_EWORKSPACE;
+  cudaStream_t s = S(stream);
+  const bool sw = cfg->act == MOE_ACT_SWIGLU, sh = cfg->n_shared != 0;
+  const int H = cfg->H, F = cfg->F, E = cfg->E;
+  const int ngroups = E + (sh ? 1 : 0);
+  const int Fp = (F + 63) / 64 * 64;
+  const int dzw = dz_width(cfg);
+  int32_t* ids = at<int32_t>(ws, L.ids);
+  int32_t* slot = at<int32_t>(ws, L.slot);
+  int32_t* off = at<int32_t>(ws, L.off);
+  int32_t* rowtok = at<int32_t>(ws, L.rowtok);
+  DevStatus* status = at<DevStatus>(ws, L.status);
+  auto bf = [&](size_t o) { return at<__nv_bfloat16>(ws, o); };
+
+  if ((st = record(stage_events, 0, s)) != MOE_OK) return st;
+  // 1. combine backward: gate-weighted rows of dy, gate gradients
+  CombineBwdParams cb{};
+  cb.dy = static_cast<const __nv_bfloat16*>(dy);
+  cb.ybuf = bf(L.ybuf);
+  cb.ids = ids;
+  cb.slot = slot;
+  cb.gates = at<float>(ws, L.gates);
+  cb.off = off;
+  cb.dyrow = bf(L.dyrow);
+  cb.dgate = at<float>(ws, L.dgate);
+  cb.T = cfg->T;
+  cb.rows_max = L.rows_max;
+  cb.H = H;
+  cb.E = E;
+  cb.k = cfg->k;
+  cb.n_shared = cfg->n_shared;
+  if (launch_combine_bwd(cb, s) != cudaSuccess) return MOE_ECUDA;
+  if (launch_zero_pad_rows(bf(L.dyrow), H, rowtok, off, ngroups, L.rows_max, s) != cudaSuccess) return MOE_ECUDA;
+  if ((st = record(stage_events, 1, s)) != MOE_OK) return st;
+
+  BwdGemm q{};
+  q.off = off;
+  q.status = status;
+  q.T = cfg->T;
+  q.rows_max = L.rows_max;
+  q.E = E;
+  q.n_shared = cfg->n_shared;
+  q.act = cfg->act;
+  // 2. dh = dyrow W2 (W2 read along F)
+  BwdGemm g = q;
+  g.a = bf(L.dyrow);
+  g.b0 = w->w2;
+  g.sb0 = sh ? w->sw2 : nullptr;
+  g.out = bf(L.dh);
+  g.K = H;
+  g.K0 = H;
+  g.N = F;
+  if (launch_bwd_dgrad(g, s) != cudaSuccess) return MOE_ECUDA;
+  if ((st = record(stage_events, 2, s)) != MOE_OK) return st;
+  // 3. dW2 = dyrow^T h per expert
+  g = q;
+  g.a = bf(L.dyrow);
+  g.b0 = bf(L.hbuf);
+  g.M = H;
+  g.N = F;
+  g.m_split = H;
+  g.m_valid = H;
+  g.w_out = dw->dw2;
+  g.w_sh = sh ? dw->dsw2 : nullptr;
+  if (launch_bwd_wgrad(g, s) != cudaSuccess) return MOE_ECUDA;
+  if ((st = record(stage_events, 3, s)) != MOE_OK) return st;
+  // 4. dz = dh * act'(z), z recomputed from the dispatched rows
+  g = q;
+  g.a = bf(L.xbuf);
+  g.a_shared = sh ? x : nullptr;
+  g.b0 = w->w1;
+  g.b1 = sw ? w->w3 : nullptr;
+  g.sb0 = sh ? w->sw1 : nullptr;
+  g.sb1 = sh && sw ? w->sw3 : nullptr;
+  g.dh = bf(L.dh);
+  g.out = bf(L.dz);
+  g.K = H;
+  g.N = F;
+  if (launch_bwd_dact(g, s) != cudaSuccess) return MOE_ECUDA;
+  if ((st = record(stage_events, 4, s)) != MOE_OK) return st;
+  // 5. dW1 (and dW3) = dz^T x_rows per expert; the shared block's rows are x
+  g = q;
+  g.a = bf(L.dz);
+  g.b0 = bf(L.xbuf);
+  g.b_shared = sh ? x : nullptr;
+  g.M = dzw;
+  g.N = H;
+  g.m_split = sw ? Fp : dzw;
+  g.m_valid = F;
+  g.w_out = dw->dw1;
+  g.w_out2 = sw ? dw->dw3 : nullptr;
+  g.w_sh = sh ? dw->dsw1 : nullptr;
+  g.w_sh2 = sh && sw ? dw->dsw3 : nullptr;
+  if (launch_bwd_wgrad(g, s) != cudaSuccess) return MOE_ECUDA;
+  if ((st = record(stage_events, 5, s)) != MOE_OK) return st;
+  // 6. router backward
+  RouterBwdParams rb{};
+  rb.logits = at<float>(ws, L.logits);
+  rb.dgate = at<float>(ws, L.dgate);
+  rb.fcoef = at<float>(ws, L.fcoef);
+  rb.dlogits = at<float>(ws, L.dlog);
+  rb.T = cfg->T;
+  rb.E = E;
+  rb.k = cfg->k;
+  rb.score = cfg->score;
+  rb.renorm = cfg->renorm;
+  rb.zc = d_z * cfg->z_coef;
+  if (launch_router_bwd(rb, at<int32_t>(ws, L.cnt), L.nblk_router, d_aux * cfg->aux_alpha, at<float>(ws, L.fcoef),
+                        s) != cudaSuccess)
+    return MOE_ECUDA;
+  if ((st = record(stage_events, 6, s)) != MOE_OK) return st;
+  // 7. dxrow = dz [W1; W3] (weights read along H)
+  g = q;
+  g.a = bf(L.dz);
+  g.b0 = w->w1;
+  g.b1 = sw ? w->w3 : nullptr;
+  g.sb0 = sh ? w->sw1 : nullptr;
+  g.sb1 = sh && sw ? w->sw3 : nullptr;
+  g.out = bf(L.dxrow);
+  g.K = dzw;
+  g.K0 = F;
+  g.k_switch = sw ? Fp / 64 : 0;
+  g.N = H;
+  if (launch_bwd_dgrad(g, s) != cudaSuccess) return MOE_ECUDA;
+  if ((st = record(stage_events, 7, s)) != MOE_OK) return st;
+  // 8. dx: tokens sum their rows' gradients, plus the router's dlogits Wg
+  DispatchBwdParams db{};
+  db.dxrow = bf(L.dxrow);
+  db.dlogits = at<float>(ws, L.dlog);
+  db.wg = wg;
+  db.ids = ids;
+  db.slot = slot;
+  db.off = off;
+  db.dx = static_cast<__nv_bfloat16*>(dx);
+  db.T = cfg->T;
+  db.rows_max = L.rows_max;
+  db.H = H;
+  db.E = E;
+  db.k = cfg->k;
+  db.n_shared = cfg->n_shared;
+  if (launch_dispatch_bwd(db, s) != cudaSuccess) return MOE_ECUDA;
+  if ((st = record(stage_events, 8, s)) != MOE_OK) return st;
+  // 9. dWg = dlogits^T x
+  if (launch_router_wgrad(at<float>(ws, L.dlog), x, cfg->T, E, H, at<float>(ws, L.dwgp), dwg, s) != cudaSuccess)
+    return MOE_ECUDA;
+  return record(stage_events, 9, s);
 }
 
 int moe_sync_status(void* ws, moe_stream_t stream) {

@@ -37,7 +37,45 @@ __device__ __forceinline__ int lane_expert(int lane, int j) {
 }
 
 // Top-k order: larger logit first (order-preserving keys, to_ordered), equal
-// logits -> smaller expert index.
+// logits -> smaller expert index.  Each round finds the warp's best remaining
+// (logit, lower index) key with two 32-bit max reductions: first the
+// order-preserving logit bits, then, among lanes holding that logit, the
+// complemented expert index.  Lane r < k receives the rank-r choice (its logit
+// and expert); the return value marks, per lane, which of its EJ experts were
+// chosen.
+template <int EJ>
+__device__ __forceinline__ unsigned select_topk(const float (&l)[EJ], int lane, int E, int k, float& my_l,
+                                                int& my_e) {
+  unsigned selected = 0u;
+  my_l = -INFINITY;
+  my_e = -1;
+  uint32_t bh = 0u, bl = 0u;      // this lane's best unselected candidate
+  int bj = -1;
+  auto lane_best = [&]() {
+    bh = 0u; bl = 0u; bj = -1;
+#pragma unroll
+    for (int j = 0; j < EJ; ++j) {
+      const int e = lane_expert<EJ>(lane, j);
+      if (e < E && !((selected >> j) & 1u)) {
+        const uint32_t h = to_ordered(l[j]), lo = 0xffffffffu - (uint32_t)e;
+        if (h > bh || (h == bh && lo > bl)) { bh = h; bl = lo; bj = j; }
+      }
+    }
+  };
+  lane_best();
+#pragma unroll 1
+  for (int r = 0; r < k; ++r) {
+    const uint32_t wh = __reduce_max_sync(0xffffffffu, bh);
+    const uint32_t wl = __reduce_max_sync(0xffffffffu, bh == wh ? bl : 0u);
+    if (lane == r) { my_l = from_ordered(wh); my_e = (int)(0xffffffffu - wl); }
+    if (bj >= 0 && bh == wh && bl == wl) {      // this lane owned the winner
+      selected |= 1u << bj;
+      lane_best();
+    }
+  }
+  return selected;
+}
+
 
 // Scores, top-k and gates of token t from its E values spread over the warp's
 // lanes (val[j] belongs to expert lane_expert(lane, j)), adding the logit offset
@@ -96,39 +134,11 @@ __device__ __forceinline__ void route_token(const RouterParams& p, int64_t t, in
     zacc += lse * lse;
   }
 
-  // top-k: each round, the warp's best remaining (logit, lower index) key is found
-  // with two 32-bit max reductions: first the order-preserving logit bits, then,
-  // among lanes holding that logit, the complemented expert index.
-  unsigned selected = 0u;
-  float my_l = -INFINITY;
-  int my_e = -1;
-  uint32_t bh = 0u, bl = 0u;      // this lane's best unselected candidate
-  int bj = -1;
-  auto lane_best = [&]() {
-    bh = 0u; bl = 0u; bj = -1;
+  float my_l;
+  int my_e;
+  const unsigned selected = select_topk<EJ>(l, lane, E, p.k, my_l, my_e);
 #pragma unroll
-    for (int j = 0; j < EJ; ++j) {
-      const int e = lane_expert<EJ>(lane, j);
-      if (e < E && !((selected >> j) & 1u)) {
-        const uint32_t h = to_ordered(l[j]), lo = 0xffffffffu - (uint32_t)e;
-        if (h > bh || (h == bh && lo > bl)) { bh = h; bl = lo; bj = j; }
-      }
-    }
-  };
-  lane_best();
-#pragma unroll 1
-  for (int r = 0; r < p.k; ++r) {
-    const uint32_t wh = __reduce_max_sync(0xffffffffu, bh);
-    const uint32_t wl = __reduce_max_sync(0xffffffffu, bh == wh ? bl : 0u);
-    if (lane == r) { my_l = from_ordered(wh); my_e = (int)(0xffffffffu - wl); }
-    if (bj >= 0 && bh == wh && bl == wl) {      // this lane owned the winner
-      selected |= 1u << bj;
-#pragma unroll
-      for (int j = 0; j < EJ; ++j)
-        if (j == bj) cnt[j] += 1;
-      lane_best();
-    }
-  }
+  for (int j = 0; j < EJ; ++j) cnt[j] += (selected >> j) & 1u;
   // gates: lane r holds the rank-r selection
   float g = 0.0f;
   if (lane < p.k) g = sigmoid ? 1.0f / (1.0f + expf(-my_l)) : expf(my_l - m);   // top-1 logit equals m
@@ -420,6 +430,197 @@ cudaError_t launch_router(const RouterParams& p, bool bf16, cudaStream_t stream)
   if (E <= 256) return launch_router_ej<8, 8>(p, bf16, stream);
   if (E <= 512) return launch_router_ej<16, 4>(p, bf16, stream);
   return launch_router_ej<32, 2>(p, bf16, stream);
+}
+
+// ---------------------------------------------------------------- backward
+// dL/dlogits of one token ("Expert-parallel MoE training" explainer, aux-loss
+// section: the aux loss reaches the router only through P_i, f_i being a
+// constant; the z-loss acts on the logits; "Switch Routing" 2.1: the gate is the
+// router's probability).  The selection is recomputed from the forward's logits
+// with the forward's own top-k; dgate is zero for choices that add nothing to y.
+template <int EJ>
+__device__ __forceinline__ void route_token_bwd(const RouterBwdParams& p, int64_t t, int lane) {
+  const int E = p.E;
+  float l[EJ];
+  float m = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < EJ; ++j) {
+    const int e = lane_expert<EJ>(lane, j);
+    l[j] = e < E ? p.logits[t * E + e] : -INFINITY;
+    m = fmaxf(m, l[j]);
+  }
+  m = from_ordered(__reduce_max_sync(0xffffffffu, to_ordered(m)));
+  float pr[EJ], s = 0.0f;
+#pragma unroll
+  for (int j = 0; j < EJ; ++j) {
+    pr[j] = lane_expert<EJ>(lane, j) < E ? expf(l[j] - m) : 0.0f;
+    s += pr[j];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  const float inv_s = 1.0f / s;
+#pragma unroll
+  for (int j = 0; j < EJ; ++j) pr[j] *= inv_s;                 // softmax
+  float my_l;
+  int my_e;
+  select_topk<EJ>(l, lane, E, p.k, my_l, my_e);
+  const int e_top = __shfl_sync(0xffffffffu, my_e, 0);         // argmax of the logits, p, the sigmoids
+  const bool sigmoid = p.score == MOE_SCORE_SIGMOID_TOPK;
+  const bool tks = p.score == MOE_SCORE_TOPK_SOFTMAX;
+  const bool norm = tks || p.renorm;
+  // Renormalised softmax gates are the softmax of the selected logits, the
+  // same function as TOPK_SOFTMAX: their gradient goes straight to the
+  // selected logits (through the full softmax it would cancel exactly for every
+  // other expert, in exact arithmetic only).
+  const bool direct = tks || (p.score == MOE_SCORE_SOFTMAX_TOPK && p.renorm);
+  // Every "v_j - sum_i w_i v_i" below (weights summing to one, the largest one
+  // w_m) is evaluated as (v_j - v_m) + sum_{i != m} w_i (v_m - v_i): equal in
+  // exact arithmetic, and free of the cancellation that the direct form suffers
+  // in fp32 when w_m is within rounding of 1 (a confidently routed token).
+  // gate of rank r (lane r) before renormalisation, and the normaliser S
+  float graw = 0.0f, dg = 0.0f;
+  if (lane < p.k) {
+    graw = sigmoid ? 1.0f / (1.0f + expf(-my_l)) : tks ? expf(my_l - m) : expf(my_l - m) * inv_s;
+    dg = p.dgate[t * p.k + lane];
+  }
+  float S = graw;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
+  const float g = norm ? graw / S : graw;
+  const float dg0 = __shfl_sync(0xffffffffu, dg, 0);
+  float rg = lane > 0 && lane < p.k ? g * (dg0 - dg) : 0.0f;     // sum_{r != 0} g_r (dg_0 - dg_r)
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) rg += __shfl_xor_sync(0xffffffffu, rg, o);
+  const float centred = (dg - dg0) + rg;                          // dg_r - sum_q g_q dg_q
+  // gradient with respect to the rank-r quantity before normalisation: the
+  // logit (TOPK_SOFTMAX, renormalised SOFTMAX_TOPK), p (SOFTMAX_TOPK) or the
+  // sigmoid (SIGMOID_TOPK)
+  const float val = direct ? g * centred : norm ? centred / S : dg;
+  float dpre[EJ], dl[EJ];
+#pragma unroll
+  for (int j = 0; j < EJ; ++j) { dpre[j] = 0.0f; dl[j] = 0.0f; }
+#pragma unroll 1
+  for (int r = 0; r < p.k; ++r) {
+    const int er = __shfl_sync(0xffffffffu, my_e, r);
+    const float vr = __shfl_sync(0xffffffffu, val, r);
+#pragma unroll
+    for (int j = 0; j < EJ; ++j)
+      if (lane_expert<EJ>(lane, j) == er) {
+        if (direct) dl[j] += vr;
+        else dpre[j] += vr;
+      }
+  }
+  // value v at the top expert, broadcast from the lane that holds it
+  auto at_top = [&](const float (&v)[EJ]) -> float {
+    float x = 0.0f;
+#pragma unroll
+    for (int j = 0; j < EJ; ++j)
+      if (lane_expert<EJ>(lane, j) == e_top) x = v[j];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);   // one lane holds it
+    return x;
+  };
+  if (sigmoid) {
+    // aux: P uses q = sigmoid / sum(sigmoid), dL/dq_i = fcoef_i;
+    // ds_j = dpre_j + (fcoef_j - sum_i q_i fcoef_i) / sum(sigmoid)
+    float sg[EJ], sgc[EJ], fc[EJ], Ss = 0.0f;
+#pragma unroll
+    for (int j = 0; j < EJ; ++j) {
+      const int e = lane_expert<EJ>(lane, j);
+      sg[j] = e < E ? 1.0f / (1.0f + expf(-l[j])) : 0.0f;
+      sgc[j] = e < E ? 1.0f / (1.0f + expf(l[j])) : 0.0f;        // 1 - sigmoid, without cancellation
+      fc[j] = e < E ? p.fcoef[e] : 0.0f;
+      Ss += sg[j];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) Ss += __shfl_xor_sync(0xffffffffu, Ss, o);
+    const float f_top = at_top(fc);
+    float rq = 0.0f;
+#pragma unroll
+    for (int j = 0; j < EJ; ++j)
+      if (lane_expert<EJ>(lane, j) < E && lane_expert<EJ>(lane, j) != e_top) rq += sg[j] * (f_top - fc[j]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) rq += __shfl_xor_sync(0xffffffffu, rq, o);
+    rq /= Ss;
+#pragma unroll
+    for (int j = 0; j < EJ; ++j) {
+      const int e = lane_expert<EJ>(lane, j);
+      if (e < E) {
+        const float ds = dpre[j] + ((fc[j] - f_top) + rq) / Ss;
+        dl[j] += ds * sg[j] * sgc[j];
+      }
+    }
+  } else {
+    // softmax backward of dp = (gate part) + aux part
+#pragma unroll
+    for (int j = 0; j < EJ; ++j) {
+      const int e = lane_expert<EJ>(lane, j);
+      if (e < E) dpre[j] += p.fcoef[e];
+    }
+    const float d_top = at_top(dpre);
+    float rp = 0.0f;                                              // sum_{i != top} p_i (dp_top - dp_i)
+#pragma unroll
+    for (int j = 0; j < EJ; ++j)
+      if (lane_expert<EJ>(lane, j) < E && lane_expert<EJ>(lane, j) != e_top) rp += pr[j] * (d_top - dpre[j]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) rp += __shfl_xor_sync(0xffffffffu, rp, o);
+#pragma unroll
+    for (int j = 0; j < EJ; ++j) dl[j] += pr[j] * ((dpre[j] - d_top) + rp);
+  }
+  if (p.zc != 0.0f) {
+    const float c = 2.0f * p.zc * (m + logf(s)) / (float)p.T;
+#pragma unroll
+    for (int j = 0; j < EJ; ++j) dl[j] += c * pr[j];
+  }
+#pragma unroll
+  for (int j = 0; j < EJ; ++j) {
+    const int e = lane_expert<EJ>(lane, j);
+    if (e < E) p.dlogits[t * E + e] = dl[j];
+  }
+}
+
+constexpr int kBwdRouterWarps = 8;
+
+template <int EJ>
+__global__ void __launch_bounds__(kBwdRouterWarps * 32) router_bwd_kernel(RouterBwdParams p) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t t = (int64_t)blockIdx.x * kBwdRouterWarps + (threadIdx.x >> 5);
+  if (t < p.T) route_token_bwd<EJ>(p, t, threadIdx.x & 31);
+}
+
+// fcoef[e] = d_aux * alpha * E * f_e / T, f_e = selections of e / (T k) from the
+// router's per-CTA counts (summed in block order).
+__global__ void aux_grad_prep_kernel(const int32_t* cnt_part, int nblk, int E, int64_t T, int k, float scale,
+                                     float* fcoef) {
+  pdl_wait();
+  pdl_trigger();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    long long c = 0;
+    for (int b = 0; b < nblk; ++b) c += cnt_part[(int64_t)b * E + e];
+    fcoef[e] = T > 0 ? (float)((double)scale * (double)E * ((double)c / ((double)T * k)) / (double)T) : 0.0f;
+  }
+}
+
+template <int EJ>
+static void launch_router_bwd_ej(const RouterBwdParams& p, cudaStream_t stream) {
+  launch_pdl(router_bwd_kernel<EJ>, (unsigned)((p.T + kBwdRouterWarps - 1) / kBwdRouterWarps), kBwdRouterWarps * 32,
+             0, stream, p);
+}
+
+cudaError_t launch_router_bwd(const RouterBwdParams& p, const int32_t* cnt_part, int nblk, float d_aux_alpha,
+                              float* fcoef, cudaStream_t stream) {
+  launch_pdl(aux_grad_prep_kernel, 1, 1024, 0, stream, cnt_part, nblk, p.E, p.T, p.k, d_aux_alpha, fcoef);
+  if (p.T > 0) {
+    const int E = p.E;
+    if (E <= 32) launch_router_bwd_ej<1>(p, stream);
+    else if (E <= 64) launch_router_bwd_ej<2>(p, stream);
+    else if (E <= 128) launch_router_bwd_ej<4>(p, stream);
+    else if (E <= 256) launch_router_bwd_ej<8>(p, stream);
+    else if (E <= 512) launch_router_bwd_ej<16>(p, stream);
+    else launch_router_bwd_ej<32>(p, stream);
+  }
+  return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------- aux loss

@@ -91,6 +91,10 @@ enum { MOE_DROP_POSITION = 0, MOE_DROP_PROBS = 1 };
 enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
 /* moe_cfg.flags
  * KEEP_LOGITS: moe_layer_fwd also stores fp32 logits in the workspace.
+ * TRAINING (bf16, weights not packed): moe_layer_fwd keeps everything
+ *   moe_layer_bwd needs in the workspace (logits, dispatched rows with zeroed
+ *   padding rows, activations, un-gated expert rows; it runs unfused), and
+ *   moe_workspace_size includes the backward pass's buffers.
  * PACKED_WEIGHTS (bf16 only): every pointer of moe_weights is a packed buffer
  *   written by moe_pack_weight (see there); results are bitwise the same. 
  * UNFUSED: moe_layer_fwd runs dispatch and combine as separate kernels (the
@@ -107,7 +111,13 @@ enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
  *   uniform [T] fp32 in [0,1) supplied by the caller; otherwise its id becomes
  *   -1 and its gate 0 (it takes no slot and adds nothing to y).  The aux loss
  *   still counts it as selected.  No effect when k == 1. */
-enum { MOE_FLAG_KEEP_LOGITS = 1, MOE_FLAG_RANDOM_SECOND = 2, MOE_FLAG_UNFUSED = 4, MOE_FLAG_PACKED_WEIGHTS = 8 };
+enum {
+  MOE_FLAG_KEEP_LOGITS = 1,
+  MOE_FLAG_RANDOM_SECOND = 2,
+  MOE_FLAG_UNFUSED = 4,
+  MOE_FLAG_PACKED_WEIGHTS = 8,
+  MOE_FLAG_TRAINING = 16
+};
 
 /* Layer configuration.  Limits of this build: 1 <= E <= 1024, 1 <= k <= min(E,16),
  * H and F multiples of 8, n_shared in {0,1}, T >= 0 with T*k < 2^31 and every
@@ -163,6 +173,13 @@ typedef struct moe_ws_views {
   void* hbuf;              /* [rows_max, F] expert activations (bf16; fp32 for MOE_DTYPE_F32) */
   void* ybuf;              /* [rows_max, H] un-gated expert outputs (routed rows not written by a fused top-1 combine) */
   int64_t rows_max;
+  /* MOE_FLAG_TRAINING only (else NULL), after moe_layer_bwd: */
+  float* dgate;            /* [T,k] gradient of each gate (0 for choices that add nothing to y) */
+  float* dlogits;          /* [T,E] gradient of the router logits */
+  void* dyrow;             /* [rows_max, H] gate-weighted output gradient of every row (bf16) */
+  void* dh;                /* [rows_max, F] gradient of the activations */
+  void* dz;                /* [rows_max, F] gradient of the pre-activations ([rows_max, 2*round_up(F,64)] for SwiGLU) */
+  void* dxrow;             /* [rows_max, H] input gradient of every row */
 } moe_ws_views;
 
 /* ---- sizing (host only, no CUDA calls) ------------------------------------ */
@@ -315,6 +332,41 @@ MOE_API int moe_activation_eval(int act, const float* z, const float* u, float* 
  * then set MOE_FLAG_PACKED_WEIGHTS. */
 MOE_API int moe_packed_weight_bytes(int32_t G, int32_t N, int32_t K, size_t* bytes);
 MOE_API int moe_pack_weight(const void* w, int32_t G, int32_t N, int32_t K, void* packed, moe_stream_t stream);
+
+/* Gradients of the expert weights (device pointers, fp32, the shapes of
+ * moe_weights: dw1/dw3 [E,F,H], dw2 [E,H,F], shared [1,...]; NULL where absent). */
+typedef struct moe_weight_grads {
+  float* dw1;
+  float* dw3;
+  float* dw2;
+  float* dsw1;
+  float* dsw3;
+  float* dsw2;
+} moe_weight_grads;
+
+/* Backward pass of the layer ([EP]: the backward runs the forward's
+ * permutations with their roles swapped; the aux loss is differentiable only
+ * through P_i; the z-loss acts on the logits; [SWITCH] 2.1 y = p_i E_i).
+ * Requires the workspace of a moe_layer_fwd call with MOE_FLAG_TRAINING on the
+ * same cfg, x, wg and w, untouched since.  Discrete decisions (top-k, random
+ * second dispatch, capacity) are constants.  Upstream gradients: dy [T,H]
+ * (bf16) of y, and scalars d_aux, d_z of the aux loss and the z-loss (1 when
+ * both are added to the loss).  Outputs (device, overwritten): dx [T,H] bf16,
+ * dwg [E,H] fp32, and the expert weight gradients in `dw` (fp32).
+ * Kernels: combine backward (gate-weighted rows of dy, gate gradients), the
+ * second contraction's data and weight gradients, the first contraction
+ * recomputed with the activation's derivative applied (no pre-activations are
+ * stored), its data and weight gradients, the router backward, the dispatch
+ * backward (tokens sum their rows, plus dlogits Wg), and dWg = dlogits^T x.
+ * `stage_events`, if non-NULL, is an array of MOE_N_BWD_STAGE_EVENTS events
+ * recorded on `stream` before the first kernel and after each of: combine
+ * backward (with the zeroing of padding rows), dh, dW2, dz, dW1/dW3, router
+ * backward, the rows' input gradients, dispatch backward, dWg.
+ * Errors: MOE_EUNSUPPORTED for fp32 layers or packed weights. */
+enum { MOE_N_BWD_STAGE_EVENTS = 10 };
+MOE_API int moe_layer_bwd(const moe_cfg* cfg, const void* x, const float* wg, const moe_weights* w, const void* dy,
+                          float d_aux, float d_z, void* dx, float* dwg, const moe_weight_grads* dw, void* ws,
+                          size_t ws_bytes, const moe_event_t* stage_events, moe_stream_t stream);
 
 /* ---- status ---------------------------------------------------------------- */
 

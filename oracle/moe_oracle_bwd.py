@@ -62,10 +62,11 @@ def act_backward(act: int, a: np.ndarray, b: Optional[np.ndarray], dh: np.ndarra
     raise ValueError(f"unknown activation {act}")
 
 
-def expert_backward(X: np.ndarray, w1, w2, act: int, w3, dyrow: np.ndarray):
+def expert_backward(X: np.ndarray, w1, w2, act: int, w3, dyrow: np.ndarray, inter: Optional[dict] = None):
     """One expert on rows X [n,H] with output gradient dyrow [n,H] (already
     gate-weighted).  Returns (yrow, dX, dW1, dW2, dW3); the forward is
-    yrow = act(X W1^T) W2^T, or (silu(X W1^T) * (X W3^T)) W2^T for SwiGLU."""
+    yrow = act(X W1^T) W2^T, or (silu(X W1^T) * (X W3^T)) W2^T for SwiGLU.
+    `inter` (optional dict) receives the intermediates a, b, h, dh, da, db."""
     X = np.asarray(X, dtype=np.float64)
     W1 = np.asarray(w1, dtype=np.float64)
     W2 = np.asarray(w2, dtype=np.float64)
@@ -84,6 +85,8 @@ def expert_backward(X: np.ndarray, w1, w2, act: int, w3, dyrow: np.ndarray):
     da, db = act_backward(act, a, b, dh)
     dW1 = da.T @ X
     dX = da @ W1
+    if inter is not None:
+        inter.update(a=a, b=b, h=h, dh=dh, da=da, db=db)
     dW3 = None
     if db is not None:
         dW3 = db.T @ X
@@ -157,12 +160,14 @@ def router_backward(layer: O.OracleLayer, logits: np.ndarray, selected: np.ndarr
 # ---------------------------------------------------------------- layer
 def layer_backward(layer: O.OracleLayer, x, wg, w1, w2, w3=None, sw1=None, sw2=None, sw3=None, dy=None,
                    logit_add=None, logits=None, uniform=None, d_aux: float = 1.0, d_z: float = 1.0,
-                   fwd: Optional[dict] = None) -> dict:
+                   fwd: Optional[dict] = None, want_rows: bool = False) -> dict:
     """Gradients of L = sum(dy * y) + d_aux * aux + d_z * zloss with respect to
     x, Wg and every expert matrix.  `fwd` (optional) is layer_forward's result
     for the same inputs; `logits` replaces the router GEMM as in layer_forward.
     Returns dx [T,H], dwg [E,H], dw1/dw3 [E,F,H], dw2 [E,H,F], dsw1/dsw3 [1,F,H],
-    dsw2 [1,H,F] (None where absent), and dgate [T,k], dlogits [T,E]."""
+    dsw2 [1,H,F] (None where absent), and dgate [T,k], dlogits [T,E].  With
+    want_rows, "experts" maps each expert (E for the shared one) to its tokens
+    and row intermediates (ts, rs, dyrow, a, b, h, dh, da, db)."""
     T, E, k, H, F = layer.T, layer.E, layer.k, layer.H, layer.F
     if fwd is None:
         fwd = O.layer_forward(layer, x, wg, w1, w2, w3, sw1, sw2, sw3, logit_add=logit_add, logits=logits,
@@ -175,6 +180,7 @@ def layer_backward(layer: O.OracleLayer, x, wg, w1, w2, w3=None, sw1=None, sw2=N
     dW1 = np.zeros((E, F, H))
     dW2 = np.zeros((E, H, F))
     dW3 = np.zeros((E, F, H)) if layer.act == O.ACT_SWIGLU else None
+    rows_out = {}
     # experts: the combine's gradient goes to each kept row (dispatch path), the
     # rows' input gradients return to their tokens (combine path)
     for e in range(E):
@@ -184,8 +190,11 @@ def layer_backward(layer: O.OracleLayer, x, wg, w1, w2, w3=None, sw1=None, sw2=N
         ts = np.array([t for t, _ in tr])
         rs = np.array([r for _, r in tr])
         dyrow = gates[ts, rs][:, None] * dY[ts]
+        inter = dict(ts=ts, rs=rs, dyrow=dyrow) if want_rows else None
         yrow, dXr, d1, d2, d3 = expert_backward(X[ts], w1[e], w2[e], layer.act,
-                                                None if w3 is None else w3[e], dyrow)
+                                                None if w3 is None else w3[e], dyrow, inter)
+        if want_rows:
+            rows_out[e] = inter
         dgate[ts, rs] = (dY[ts] * yrow).sum(axis=1)
         dW1[e], dW2[e] = d1, d2
         if d3 is not None:
@@ -193,7 +202,11 @@ def layer_backward(layer: O.OracleLayer, x, wg, w1, w2, w3=None, sw1=None, sw2=N
         np.add.at(dX, ts, dXr)
     out = dict(dsw1=None, dsw2=None, dsw3=None)
     if layer.n_shared:
-        _, dXs, d1, d2, d3 = expert_backward(X, sw1[0], sw2[0], layer.act, None if sw3 is None else sw3[0], dY)
+        inter = dict(ts=np.arange(T), rs=-np.ones(T, dtype=np.int64), dyrow=dY) if want_rows else None
+        _, dXs, d1, d2, d3 = expert_backward(X, sw1[0], sw2[0], layer.act, None if sw3 is None else sw3[0], dY,
+                                             inter)
+        if want_rows:
+            rows_out[E] = inter
         dX += dXs
         out.update(dsw1=d1[None], dsw2=d2[None], dsw3=None if d3 is None else d3[None])
     dl = router_backward(layer, fwd["logits"], selected, dgate, d_aux, d_z)
@@ -201,4 +214,6 @@ def layer_backward(layer: O.OracleLayer, x, wg, w1, w2, w3=None, sw1=None, sw2=N
     dWg = dl.T @ X
     dX += dl @ Wg
     out.update(dx=dX, dwg=dWg, dw1=dW1, dw2=dW2, dw3=dW3, dgate=dgate, dlogits=dl, fwd=fwd)
+    if want_rows:
+        out["experts"] = rows_out
     return out

@@ -128,7 +128,7 @@ def test_router_variant_validation(lib):
             B.moe_workspace_size(B.make_cfg(g, **kw))
         assert ei.value.code == B.MOE_EINVAL, kw
     with pytest.raises(B.MoeError) as ei:
-        B.moe_workspace_size(B.make_cfg(g, flags=16))
+        B.moe_workspace_size(B.make_cfg(g, flags=64))
     assert ei.value.code == B.MOE_EINVAL
     # the flag needs the draws (k >= 2, T > 0); dummy device pointers are never touched
     cfg = B.make_cfg(g.replace(random_second=1))
