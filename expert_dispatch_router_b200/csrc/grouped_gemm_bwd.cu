@@ -39,6 +39,13 @@ constexpr int TMEM_COLS = 512;
 constexpr int STAGE_OUT_BYTES = 32 * 32 * 2;
 constexpr int STAGING_BYTES = EPI_WARPS * STAGE_OUT_BYTES;
 constexpr int SMEM_BYTES = RING_BYTES + STAGING_BYTES + 1024 + 256;
+// WGRAD: the k loop of a tile is one expert's rows (a few blocks), and the fp32
+// output dominates, so the ring shrinks to two stages and each epilogue warp
+// gets two 4 KB buffers (32 rows x 32 fp32, 128-byte swizzle) for TMA stores.
+constexpr int WG_OUT_BYTES = 32 * 32 * 4;
+constexpr int WG_STAGING_BYTES = EPI_WARPS * 2 * WG_OUT_BYTES;   // 128 KB
+constexpr int WG_RING_BYTES = RING_BYTES + STAGING_BYTES - WG_STAGING_BYTES;
+static_assert(WG_RING_BYTES >= 2 * (A_BYTES + BNMAX * BK * 2), "WGRAD ring holds two stages");
 constexpr int MN_CHUNK_BYTES = 64 * BK * 2;                 // one 64-feature x 64-k box: 8 KB
 
 enum Mode { DGRAD = 0, DACT = 1, WGRAD = 2 };
@@ -58,9 +65,9 @@ struct BParams {
   int as_sep, b_sep;              // shared block's A (DACT) / B (WGRAD) from a separate map, rows - off[E]
   const __nv_bfloat16* dh;        // DACT: [rows_max, N] upstream gradient of h
   int dz_ld;                      // DACT: row length of dz (N, or 2N for SwiGLU: da | db)
-  float *wout, *wout2;            // WGRAD: per-expert fp32 [M or m_split, N] (+ [M - m_split, N])
-  float *wsh, *wsh2;              // WGRAD: the shared expert's
-  int m_split;                    // WGRAD: output rows >= m_split go to wout2 / wsh2
+  CUtensorMap tmW, tmW2;          // WGRAD: fp32 outputs [E, m_valid, N] (rows >= m_split: tmW2), box 32 x 32 x 1
+  CUtensorMap tmWs, tmWs2;        // WGRAD: the shared expert's, [1, m_valid, N]
+  int m_split;                    // WGRAD: output rows >= m_split go to tmW2 / tmWs2 (a multiple of 64)
   int m_valid;                    // WGRAD: rows of each output part (rows beyond are padding, not stored)
 };
 
@@ -85,8 +92,9 @@ __device__ __forceinline__ float gelu_grad(float z) {
 __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __grid_constant__ BParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const bool wgrad = p.mode == WGRAD;
   uint8_t* stage_base = smem;
-  uint8_t* staging = smem + RING_BYTES;
+  uint8_t* staging = smem + (wgrad ? WG_RING_BYTES : RING_BYTES);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + RING_BYTES + STAGING_BYTES);
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + MAX_STAGES);
   const uint32_t tfull0 = smem_u32(bars + 2 * MAX_STAGES), tempty0 = smem_u32(bars + 2 * MAX_STAGES + 2);
@@ -96,7 +104,6 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool swiglu = p.mode == DACT && p.act == MOE_ACT_SWIGLU;
-  const bool wgrad = p.mode == WGRAD;
   const int a_mn = wgrad ? 1 : 0, b_mn = p.mode == DACT ? 0 : 1;
   const int ngroups = p.E + (p.n_shared ? 1 : 0);
 
@@ -152,7 +159,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
   };
   const int b_bytes = bn * BK * 2;                         // 32 KB
   const int stage_bytes = A_BYTES + b_bytes;
-  const int n_stages = min(MAX_STAGES, RING_BYTES / stage_bytes);
+  const int n_stages = min(MAX_STAGES, (wgrad ? WG_RING_BYTES : RING_BYTES) / stage_bytes);
 
   if (warp == 0) {
     // ---------------- TMA producer
@@ -255,7 +262,8 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
     const int sub = warp & 3;
     const int quarter = ew >> 2;
     const int row_in_tile = sub * 32 + lane;
-    const uint32_t stage_out = smem_u32(staging + ew * STAGE_OUT_BYTES);
+    const uint32_t stage_out = smem_u32(staging + ew * (wgrad ? 2 * WG_OUT_BYTES : STAGE_OUT_BYTES));
+    int wbuf = 0;                                    // WGRAD: staging buffer of the next store
     int acc = 0;
     uint32_t acc_phase = 0;
     // bf16 store of this warp's 32 x 32 sub-tile through its staging buffer
@@ -298,17 +306,27 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
         }
         if (p.mode == WGRAD) {
           tmem_wait_ld();
-          const int m = (int)d.row0 + row_in_tile;
-          if (m >= p.M) continue;
-          const bool hi = m >= p.m_split;
-          const int mr = hi ? m - p.m_split : m;
-          if (mr >= p.m_valid) continue;
-          float* base = d.g == p.E ? (hi ? p.wsh2 : p.wsh) : (hi ? p.wout2 : p.wout) + (int64_t)d.g * p.m_valid * p.N;
-          float* drow = base + (int64_t)mr * p.N + col;
+          // this warp's 32 output rows lie on one side of m_split (a multiple
+          // of 64); rows past m_valid and columns past N are clipped by the map
+          const int m0 = (int)d.row0 + sub * 32;
+          if (m0 >= p.M) continue;
+          const bool hi = m0 >= p.m_split;
+          const uint32_t buf = stage_out + wbuf * WG_OUT_BYTES;
+          if (lane == 0) bulk_wait_read1();          // the store that last read `buf` is done with it
+          __syncwarp();
 #pragma unroll
           for (int q = 0; q < 8; ++q)
-            if (col + 4 * q < p.N)
-              *reinterpret_cast<float4*>(drow + 4 * q) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            st_shared_v4(buf + lane * 128 + ((q ^ (lane & 7)) << 4), __float_as_uint(v[4 * q]),
+                         __float_as_uint(v[4 * q + 1]), __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            const bool sh = d.g == p.E;
+            const CUtensorMap* mw = sh ? (hi ? &p.tmWs2 : &p.tmWs) : (hi ? &p.tmW2 : &p.tmW);
+            tma_store_3d(mw, buf, col, hi ? m0 - p.m_split : m0, sh ? 0 : d.g);
+            bulk_commit();
+          }
+          wbuf ^= 1;
           continue;
         }
         const int64_t row_base = d.row0 + sub * 32;
@@ -424,6 +442,24 @@ static bool make_map_k_weights(CUtensorMap* m, const void* base, int G, int N, i
   key.box[2] = 1;
   return encode_cached(m, key);
 }
+// fp32 weight gradients [G, rows, W], box 32 x 32 x 1, 128-byte swizzle (TMA store)
+static bool make_map_wout(CUtensorMap* m, const float* base, int G, int rows, int W) {
+  MapKey key;
+  memset(&key, 0, sizeof(key));
+  key.base = base;
+  key.rank = 3;
+  key.f32 = 1;
+  key.swizzle = CU_TENSOR_MAP_SWIZZLE_128B;
+  key.dims[0] = (cuuint64_t)W;
+  key.dims[1] = (cuuint64_t)rows;
+  key.dims[2] = (cuuint64_t)G;
+  key.strides[0] = (cuuint64_t)W * 4;
+  key.strides[1] = (cuuint64_t)rows * W * 4;
+  key.box[0] = 32;
+  key.box[1] = 32;
+  key.box[2] = 1;
+  return encode_cached(m, key);
+}
 // bf16 output [rows, W], box 32 x 32, 64-byte swizzle (TMA store)
 static bool make_map_out(CUtensorMap* m, const void* base, int64_t rows, int W) {
   MapKey key;
@@ -531,12 +567,14 @@ cudaError_t launch_bwd_wgrad(const BwdGemm& q, cudaStream_t stream) {
   k.N = q.N;
   k.M = q.M;
   k.b_sep = q.b_shared != nullptr;
-  k.wout = q.w_out;
-  k.wout2 = q.w_out2;
-  k.wsh = q.w_sh;
-  k.wsh2 = q.w_sh2;
   k.m_split = q.m_split > 0 ? q.m_split : q.M;
   k.m_valid = q.m_valid > 0 ? q.m_valid : q.M;
+  if (k.m_split < q.M && k.m_split % 64 != 0) return cudaErrorInvalidValue;
+  ok = make_map_wout(&k.tmW, q.w_out, q.E, k.m_valid, q.N);
+  ok = ok && make_map_wout(&k.tmW2, q.w_out2 ? q.w_out2 : q.w_out, q.E, k.m_valid, q.N);
+  ok = ok && make_map_wout(&k.tmWs, q.w_sh ? q.w_sh : q.w_out, 1, k.m_valid, q.N);
+  ok = ok && make_map_wout(&k.tmWs2, q.w_sh2 ? q.w_sh2 : (q.w_sh ? q.w_sh : q.w_out), 1, k.m_valid, q.N);
+  if (!ok) return cudaErrorInvalidValue;
   const int64_t tiles = (int64_t)(q.E + (q.n_shared ? 1 : 0)) * ((q.M + BM - 1) / BM) * ((q.N + BNMAX - 1) / BNMAX);
   return launch(k, tiles, stream);
 }

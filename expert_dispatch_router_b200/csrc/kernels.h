@@ -80,8 +80,8 @@ struct DispatchBwdParams {
 cudaError_t launch_dispatch_bwd(const DispatchBwdParams& p, cudaStream_t stream);
 cudaError_t launch_zero_pad_rows(void* buf, int width, const int32_t* row_token, const int32_t* off, int ngroups,
                                  int64_t rows_max, cudaStream_t stream);
-int dwg_chunks(int64_t T);
-// dwg [E,H] = dlogits^T x (part: dwg_chunks(T) * E * H floats of scratch)
+int dwg_chunks(int64_t T, int E, int H);
+// dwg [E,H] = dlogits^T x (part: dwg_chunks(T, E, H) * E * H floats of scratch)
 cudaError_t launch_router_wgrad(const float* dlogits, const void* x, int64_t T, int E, int H, float* part,
                                 float* dwg, cudaStream_t stream);
 

@@ -127,7 +127,7 @@ Layout layout_of(const moe_cfg* c) {
   L.dgate = take(tr ? sizeof(float) * T * k : 0);
   L.dlog = take(tr ? sizeof(float) * T * E : 0);
   L.fcoef = take(tr ? sizeof(float) * E : 0);
-  L.dwgp = take(tr ? sizeof(float) * (size_t)dwg_chunks(c->T) * E * c->H : 0);
+  L.dwgp = take(tr ? sizeof(float) * (size_t)dwg_chunks(c->T, E, c->H) * E * c->H : 0);
   L.total = o;
   return L;
 }

@@ -64,6 +64,11 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t sr
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];"
                :: "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(src) : "memory");
 }
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3}], [%4];"
+               :: "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(src) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
@@ -188,6 +193,7 @@ struct MapKey {
   const void* base;
   uint32_t rank;
   uint32_t swizzle;      // CUtensorMapSwizzle
+  uint32_t f32;          // element type: 0 bf16, 1 fp32
   cuuint64_t dims[5];
   cuuint64_t strides[4];
   cuuint32_t box[5];
@@ -205,7 +211,8 @@ inline bool encode_cached(CUtensorMap* out, const MapKey& key) {
     if (keys[i] == key) { *out = maps[i]; return true; }
   cuuint32_t es[5] = {1, 1, 1, 1, 1};
   CUtensorMap m;
-  if (encode_fn()(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, key.rank, const_cast<void*>(key.base), key.dims, key.strides,
+  const CUtensorMapDataType dt = key.f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (encode_fn()(&m, dt, key.rank, const_cast<void*>(key.base), key.dims, key.strides,
                   key.box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, (CUtensorMapSwizzle)key.swizzle,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return false;
