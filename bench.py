@@ -706,9 +706,12 @@ def run_train(args, world, rank, local):
     gen.manual_seed(replica_seed(args.seed, rank) + 1000)
     T, H, F, E = shape.T, shape.H, shape.F, shape.E
     dy = torch.randn((T, H), generator=gen, device=dev).to(torch.bfloat16)
-    cfg = B.make_cfg(shape, flags=B.MOE_FLAG_TRAINING)
+    packed = not args.unpacked
+    cfg = B.make_cfg(shape, flags=B.MOE_FLAG_TRAINING | (B.MOE_FLAG_PACKED_WEIGHTS if packed else 0))
     ws = B.alloc_workspace(cfg)
-    wts = B.make_weights(inp)
+    wsrc = B.pack_weights(inp) if packed else inp
+    torch.cuda.synchronize()
+    wts = B.make_weights(wsrc)
     sw = shape.act == synth.ACT_SWIGLU
     g = dict(dw1=torch.empty((E, F, H), device=dev), dw2=torch.empty((E, H, F), device=dev),
              dw3=torch.empty((E, F, H), device=dev) if sw else None)
@@ -848,7 +851,7 @@ def run_train(args, world, rank, local):
                        "act": ["relu", "gelu", "swiglu"][shape.act], "kept_assignments": kept,
                        "l2": "flushed before every step (320 MiB write + 320 MiB read, outside the timed events)",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "weights": "linear-layer layout"},
+                       "weights": "packed once before timing (moe_pack_weight)" if packed else "linear-layer layout"},
             "forward_ms": fwd_ms, "backward_ms": bwd_ms, "backward_stages_ms": stage_ms,
             "stages_note": f"second timed pass of {n_stage_steps} steps with per-stage events",
             "roofline": {k_: roof[k_] for k_ in ("bound", "achieved", "peak", "unit", "frac", "traffic", "peak_source")},

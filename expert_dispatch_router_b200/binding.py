@@ -141,7 +141,11 @@ def make_cfg(shape: synth.LayerShape, flags: int = 0, **override) -> moe_cfg:
 
 
 def make_weights(inp: dict) -> moe_weights:
-    return moe_weights(*(_ptr(inp.get(n)) for n in ("w1", "w3", "w2", "sw1", "sw3", "sw2")))
+    """Device pointers of the expert matrices; the struct keeps the tensors alive."""
+    names = ("w1", "w3", "w2", "sw1", "sw3", "sw2")
+    w = moe_weights(*(_ptr(inp.get(n)) for n in names))
+    w._keep = [inp.get(n) for n in names]
+    return w
 
 
 # ------------------------------------------------------------------ sizing
@@ -235,7 +239,11 @@ def moe_layer_bwd(cfg, x, wg, weights: moe_weights, dy, d_aux, d_z, dx, dwg, gra
 
 
 def make_weight_grads(g: dict) -> moe_weight_grads:
-    return moe_weight_grads(*(_ptr(g.get(n)) for n in ("dw1", "dw3", "dw2", "dsw1", "dsw3", "dsw2")))
+    """Device pointers of the weight-gradient outputs; the struct keeps the tensors alive."""
+    names = ("dw1", "dw3", "dw2", "dsw1", "dsw3", "dsw2")
+    w = moe_weight_grads(*(_ptr(g.get(n)) for n in names))
+    w._keep = [g.get(n) for n in names]
+    return w
 
 
 def moe_activation_eval(act, z, u, out, stream=None):

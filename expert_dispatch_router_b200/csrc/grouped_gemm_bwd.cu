@@ -69,6 +69,7 @@ struct BParams {
   CUtensorMap tmWs, tmWs2;        // WGRAD: the shared expert's, [1, m_valid, N]
   int m_split;                    // WGRAD: output rows >= m_split go to tmW2 / tmWs2 (a multiple of 64)
   int m_valid;                    // WGRAD: rows of each output part (rows beyond are padding, not stored)
+  int b_packed;                   // DGRAD / DACT: weight maps are 5-D over packed 128 x 64 blocks
 };
 
 // MN-major operand descriptor (128-byte swizzle): 64-feature chunks `lbo`
@@ -194,7 +195,22 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
               const bool second = p.k_switch > 0 && kb >= p.k_switch;
               const CUtensorMap* mb = sh ? (second ? &p.tmSB1 : &p.tmSB0) : (second ? &p.tmB1 : &p.tmB0);
               const int kk = (second ? kb - p.k_switch : kb) * BK;
-              for (int j = 0; j < bn / 64; ++j) tma_load_3d(sb + j * MN_CHUNK_BYTES, mb, n0 + 64 * j, kk, z, fb);
+              // packed: the weight's rows are this contraction's k, its columns
+              // the output features; a 64 x 64 box is 8 KB of one block
+              for (int j = 0; j < bn / 64; ++j) {
+                if (p.b_packed)
+                  tma_load_5d_at(sb + j * MN_CHUNK_BYTES, mb, kk & 127, (n0 >> 6) + j, kk >> 7, z, fb);
+                else
+                  tma_load_3d(sb + j * MN_CHUNK_BYTES, mb, n0 + 64 * j, kk, z, fb);
+              }
+            } else if (p.b_packed) {
+              const CUtensorMap* m0 = sh ? &p.tmSB0 : &p.tmB0;
+              if (swiglu) {
+                tma_load_5d(sb, m0, kb, n0 >> 7, z, fb);                                         // gate rows
+                tma_load_5d(sb + b_bytes / 2, sh ? &p.tmSB1 : &p.tmB1, kb, n0 >> 7, z, fb);     // up rows
+              } else {
+                for (int b = 0; b < 2; ++b) tma_load_5d(sb + b * (b_bytes / 2), m0, kb, (n0 >> 7) + b, z, fb);
+              }
             } else if (swiglu) {
               tma_load_3d(sb, sh ? &p.tmSB0 : &p.tmB0, kb * BK, n0, z, fb);                // gate rows
               tma_load_3d(sb + b_bytes / 2, sh ? &p.tmSB1 : &p.tmB1, kb * BK, n0, z, fb);  // up rows
@@ -411,6 +427,31 @@ static bool make_map_mn_weights(CUtensorMap* m, const void* base, int G, int K, 
   key.box[2] = 1;
   return encode_cached(m, key);
 }
+// packed weights (the layout of moe_pack_weight: [G][N/128][K/64][128][64] for a
+// [G, N, K] matrix) as 5-D (64 k, 128 n, K/64, N/128, G).  K-major B: box
+// 64 x 128 (one block); MN-major B (the block's k are the output features):
+// box 64 x 64 (half a block).
+static bool make_map_packed(CUtensorMap* m, const void* base, int G, int N, int K, bool mn) {
+  const cuuint64_t kb = (cuuint64_t)((K + BK - 1) / BK), nb = (cuuint64_t)((N + 127) / 128);
+  MapKey key;
+  memset(&key, 0, sizeof(key));
+  key.base = base;
+  key.rank = 5;
+  key.swizzle = CU_TENSOR_MAP_SWIZZLE_128B;
+  key.dims[0] = BK;
+  key.dims[1] = 128;
+  key.dims[2] = kb;
+  key.dims[3] = nb;
+  key.dims[4] = (cuuint64_t)G;
+  key.strides[0] = BK * 2;
+  key.strides[1] = (cuuint64_t)BK * 128 * 2;
+  key.strides[2] = key.strides[1] * kb;
+  key.strides[3] = key.strides[2] * nb;
+  key.box[0] = BK;
+  key.box[1] = mn ? 64 : 128;
+  key.box[2] = key.box[3] = key.box[4] = 1;
+  return encode_cached(m, key);
+}
 // [rows, K] bf16 read along K: box 64 x 128 (K-major A)
 static bool make_map_k_rows(CUtensorMap* m, const void* base, int64_t rows, int K) {
   MapKey key;
@@ -496,10 +537,21 @@ cudaError_t launch_bwd_dgrad(const BwdGemm& q, cudaStream_t stream) {
   k.tmAs = k.tmA;
   // map 0 covers the first q.K0 k of B (rows beyond read as zero); with
   // k_switch, A's k blocks from k_switch on use map 1 (also q.K0 deep)
-  ok = ok && make_map_mn_weights(&k.tmB0, q.b0, G, q.K0, q.N);
-  ok = ok && make_map_mn_weights(&k.tmB1, q.b1 ? q.b1 : q.b0, G, q.K0, q.N);
-  ok = ok && make_map_mn_weights(&k.tmSB0, q.sb0 ? q.sb0 : q.b0, 1, q.K0, q.N);
-  ok = ok && make_map_mn_weights(&k.tmSB1, q.sb1 ? q.sb1 : (q.sb0 ? q.sb0 : q.b0), 1, q.K0, q.N);
+  const void* b1 = q.b1 ? q.b1 : q.b0;
+  const void* s0 = q.sb0 ? q.sb0 : q.b0;
+  const void* s1 = q.sb1 ? q.sb1 : s0;
+  if (q.b_packed) {                                 // packed [G, K0, N]: rows K0, columns N
+    ok = ok && make_map_packed(&k.tmB0, q.b0, G, q.K0, q.N, true);
+    ok = ok && make_map_packed(&k.tmB1, b1, G, q.K0, q.N, true);
+    ok = ok && make_map_packed(&k.tmSB0, s0, 1, q.K0, q.N, true);
+    ok = ok && make_map_packed(&k.tmSB1, s1, 1, q.K0, q.N, true);
+  } else {
+    ok = ok && make_map_mn_weights(&k.tmB0, q.b0, G, q.K0, q.N);
+    ok = ok && make_map_mn_weights(&k.tmB1, b1, G, q.K0, q.N);
+    ok = ok && make_map_mn_weights(&k.tmSB0, s0, 1, q.K0, q.N);
+    ok = ok && make_map_mn_weights(&k.tmSB1, s1, 1, q.K0, q.N);
+  }
+  k.b_packed = q.b_packed;
   ok = ok && make_map_out(&k.tmD, q.out, q.rows_max, q.N);
   if (!ok) return cudaErrorInvalidValue;
   k.off = q.off;
@@ -521,10 +573,21 @@ cudaError_t launch_bwd_dact(const BwdGemm& q, cudaStream_t stream) {
   BParams k{};
   bool ok = make_map_k_rows(&k.tmA, q.a, q.rows_max, q.K);
   ok = ok && make_map_k_rows(&k.tmAs, q.a_shared ? q.a_shared : q.a, q.a_shared ? q.T : q.rows_max, q.K);
-  ok = ok && make_map_k_weights(&k.tmB0, q.b0, q.E, q.N, q.K);
-  ok = ok && make_map_k_weights(&k.tmB1, q.b1 ? q.b1 : q.b0, q.E, q.N, q.K);
-  ok = ok && make_map_k_weights(&k.tmSB0, q.sb0 ? q.sb0 : q.b0, 1, q.N, q.K);
-  ok = ok && make_map_k_weights(&k.tmSB1, q.sb1 ? q.sb1 : (q.sb0 ? q.sb0 : q.b0), 1, q.N, q.K);
+  const void* b1 = q.b1 ? q.b1 : q.b0;
+  const void* s0 = q.sb0 ? q.sb0 : q.b0;
+  const void* s1 = q.sb1 ? q.sb1 : s0;
+  if (q.b_packed) {
+    ok = ok && make_map_packed(&k.tmB0, q.b0, q.E, q.N, q.K, false);
+    ok = ok && make_map_packed(&k.tmB1, b1, q.E, q.N, q.K, false);
+    ok = ok && make_map_packed(&k.tmSB0, s0, 1, q.N, q.K, false);
+    ok = ok && make_map_packed(&k.tmSB1, s1, 1, q.N, q.K, false);
+  } else {
+    ok = ok && make_map_k_weights(&k.tmB0, q.b0, q.E, q.N, q.K);
+    ok = ok && make_map_k_weights(&k.tmB1, b1, q.E, q.N, q.K);
+    ok = ok && make_map_k_weights(&k.tmSB0, s0, 1, q.N, q.K);
+    ok = ok && make_map_k_weights(&k.tmSB1, s1, 1, q.N, q.K);
+  }
+  k.b_packed = q.b_packed;
   const int ld = q.act == MOE_ACT_SWIGLU ? 2 * ((q.N + BK - 1) / BK * BK) : q.N;   // da | db, db at column Fp
   ok = ok && make_map_out(&k.tmD, q.out, q.rows_max, ld);
   if (!ok) return cudaErrorInvalidValue;

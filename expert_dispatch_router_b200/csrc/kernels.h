@@ -202,6 +202,7 @@ struct BwdGemm {
   DevStatus* status;
   int64_t T, rows_max;
   int K, K0, N, M, E, n_shared, act, k_switch, m_split, m_valid;
+  int b_packed;             // dgrad / dact: weights in the packed block layout
 };
 cudaError_t launch_bwd_dgrad(const BwdGemm& q, cudaStream_t stream);
 cudaError_t launch_bwd_dact(const BwdGemm& q, cudaStream_t stream);

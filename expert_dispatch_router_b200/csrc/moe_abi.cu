@@ -557,7 +557,7 @@ int moe_layer_bwd(const moe_cfg* cfg, const void* x, const float* wg, const moe_
   st = check_weights(cfg, w);
   if (st != MOE_OK) return st;
   if (!training(cfg)) return MOE_EINVAL;
-  if (cfg->dtype != MOE_DTYPE_BF16 || (cfg->flags & MOE_FLAG_PACKED_WEIGHTS)) return MOE_EUNSUPPORTED;
+  if (cfg->dtype != MOE_DTYPE_BF16) return MOE_EUNSUPPORTED;
   if (ws == nullptr || dw == nullptr || dwg == nullptr || dw->dw1 == nullptr || dw->dw2 == nullptr) return MOE_EINVAL;
   if (cfg->act == MOE_ACT_SWIGLU && dw->dw3 == nullptr) return MOE_EINVAL;
   if (cfg->n_shared && (dw->dsw1 == nullptr || dw->dsw2 == nullptr ||
@@ -608,6 +608,7 @@ int moe_layer_bwd(const moe_cfg* cfg, const void* x, const float* wg, const moe_
   q.E = E;
   q.n_shared = cfg->n_shared;
   q.act = cfg->act;
+  const int packed = (cfg->flags & MOE_FLAG_PACKED_WEIGHTS) ? 1 : 0;
   // 2. dh = dyrow W2 (W2 read along F)
   BwdGemm g = q;
   g.a = bf(L.dyrow);
@@ -617,6 +618,7 @@ int moe_layer_bwd(const moe_cfg* cfg, const void* x, const float* wg, const moe_
   g.K = H;
   g.K0 = H;
   g.N = F;
+  g.b_packed = packed;
   if (launch_bwd_dgrad(g, s) != cudaSuccess) return MOE_ECUDA;
   if ((st = record(stage_events, 2, s)) != MOE_OK) return st;
   // 3. dW2 = dyrow^T h per expert
@@ -643,6 +645,7 @@ int moe_layer_bwd(const moe_cfg* cfg, const void* x, const float* wg, const moe_
   g.out = bf(L.dz);
   g.K = H;
   g.N = F;
+  g.b_packed = packed;
   if (launch_bwd_dact(g, s) != cudaSuccess) return MOE_ECUDA;
   if ((st = record(stage_events, 4, s)) != MOE_OK) return st;
   // 5. dW1 (and dW3) = dz^T x_rows per expert; the shared block's rows are x
@@ -688,6 +691,7 @@ int moe_layer_bwd(const moe_cfg* cfg, const void* x, const float* wg, const moe_
   g.K0 = F;
   g.k_switch = sw ? Fp / 64 : 0;
   g.N = H;
+  g.b_packed = packed;
   if (launch_bwd_dgrad(g, s) != cudaSuccess) return MOE_ECUDA;
   if ((st = record(stage_events, 7, s)) != MOE_OK) return st;
   // 8. dx: tokens sum their rows' gradients, plus the router's dlogits Wg

@@ -590,16 +590,22 @@ __global__ void __launch_bounds__(kBwdRouterWarps * 32) router_bwd_kernel(Router
 }
 
 // fcoef[e] = d_aux * alpha * E * f_e / T, f_e = selections of e / (T k) from the
-// router's per-CTA counts (summed in block order).
-__global__ void aux_grad_prep_kernel(const int32_t* cnt_part, int nblk, int E, int64_t T, int k, float scale,
-                                     float* fcoef) {
+// router's per-CTA counts: one warp per expert, lanes striding over the CTAs
+// (integer sums, exact in any order).
+constexpr int kPrepWarps = 8;
+
+__global__ void __launch_bounds__(kPrepWarps * 32) aux_grad_prep_kernel(const int32_t* cnt_part, int nblk, int E,
+                                                                         int64_t T, int k, float scale, float* fcoef) {
   pdl_wait();
   pdl_trigger();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    long long c = 0;
-    for (int b = 0; b < nblk; ++b) c += cnt_part[(int64_t)b * E + e];
+  const int e = blockIdx.x * kPrepWarps + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (e >= E) return;
+  long long c = 0;
+  for (int b = lane; b < nblk; b += 32) c += cnt_part[(int64_t)b * E + e];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  if (lane == 0)
     fcoef[e] = T > 0 ? (float)((double)scale * (double)E * ((double)c / ((double)T * k)) / (double)T) : 0.0f;
-  }
 }
 
 template <int EJ>
@@ -610,7 +616,8 @@ static void launch_router_bwd_ej(const RouterBwdParams& p, cudaStream_t stream) 
 
 cudaError_t launch_router_bwd(const RouterBwdParams& p, const int32_t* cnt_part, int nblk, float d_aux_alpha,
                               float* fcoef, cudaStream_t stream) {
-  launch_pdl(aux_grad_prep_kernel, 1, 1024, 0, stream, cnt_part, nblk, p.E, p.T, p.k, d_aux_alpha, fcoef);
+  launch_pdl(aux_grad_prep_kernel, (unsigned)((p.E + kPrepWarps - 1) / kPrepWarps), kPrepWarps * 32, 0, stream,
+             cnt_part, nblk, p.E, p.T, p.k, d_aux_alpha, fcoef);
   if (p.T > 0) {
     const int E = p.E;
     if (E <= 32) launch_router_bwd_ej<1>(p, stream);

@@ -91,7 +91,7 @@ enum { MOE_DROP_POSITION = 0, MOE_DROP_PROBS = 1 };
 enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
 /* moe_cfg.flags
  * KEEP_LOGITS: moe_layer_fwd also stores fp32 logits in the workspace.
- * TRAINING (bf16, weights not packed): moe_layer_fwd keeps everything
+ * TRAINING (bf16): moe_layer_fwd keeps everything
  *   moe_layer_bwd needs in the workspace (logits, dispatched rows with zeroed
  *   padding rows, activations, un-gated expert rows; it runs unfused), and
  *   moe_workspace_size includes the backward pass's buffers.
@@ -362,7 +362,10 @@ typedef struct moe_weight_grads {
  * recorded on `stream` before the first kernel and after each of: combine
  * backward (with the zeroing of padding rows), dh, dW2, dz, dW1/dW3, router
  * backward, the rows' input gradients, dispatch backward, dWg.
- * Errors: MOE_EUNSUPPORTED for fp32 layers or packed weights. */
+ * With MOE_FLAG_PACKED_WEIGHTS the data-gradient contractions read the packed
+ * blocks (the weight gradients are always written in the linear-layer layout);
+ * results are bitwise the same.
+ * Errors: MOE_EUNSUPPORTED for fp32 layers. */
 enum { MOE_N_BWD_STAGE_EVENTS = 10 };
 MOE_API int moe_layer_bwd(const moe_cfg* cfg, const void* x, const float* wg, const moe_weights* w, const void* dy,
                           float d_aux, float d_z, void* dx, float* dwg, const moe_weight_grads* dw, void* ws,

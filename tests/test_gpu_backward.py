@@ -57,14 +57,15 @@ def _lib():
     B.load()
 
 
-def run_fwd_bwd(shape, inp, dy, d_aux, d_z):
-    cfg = B.make_cfg(shape, flags=B.MOE_FLAG_TRAINING)
+def run_fwd_bwd(shape, inp, dy, d_aux, d_z, packed=False):
+    cfg = B.make_cfg(shape, flags=B.MOE_FLAG_TRAINING | (B.MOE_FLAG_PACKED_WEIGHTS if packed else 0))
     ws = B.alloc_workspace(cfg)
     T, H, F, E = shape.T, shape.H, shape.F, shape.E
     dev = "cuda"
     y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
     aux = torch.full((2,), float("nan"), device=dev)
-    wts = B.make_weights(inp)
+    wsrc = B.pack_weights(inp) if packed else inp       # the packed buffers must outlive both calls
+    wts = B.make_weights(wsrc)
     B.moe_layer_fwd(cfg, inp["x"], inp["wg"], inp["logit_add"], inp.get("uniform"), wts, y, aux, None, ws)
     sw = shape.act == synth.ACT_SWIGLU
     g = dict(dw1=torch.full((E, F, H), float("nan"), device=dev), dw2=torch.full((E, H, F), float("nan"), device=dev),
@@ -78,7 +79,7 @@ def run_fwd_bwd(shape, inp, dy, d_aux, d_z):
     st = B.moe_sync_status(ws)
     assert st == B.MOE_OK, B.strerror(st)
     out = B.workspace_tensors(cfg, ws)
-    out.update(y=y, aux=aux, dx=dx, dwg=dwg, grads=g)
+    out.update(y=y, aux=aux, dx=dx, dwg=dwg, grads=g, weights=wsrc)
     return out
 
 
@@ -237,6 +238,23 @@ def test_backward_full_switch_top1():
     dy = torch.randn((shape.T, shape.H), generator=gen, device="cuda").to(torch.bfloat16)
     out = run_fwd_bwd(shape, inp, dy, 1.0, 1.0)
     check_backward(shape, inp, out, dy, 1.0, 1.0)
+
+
+@pytest.mark.parametrize("name", ["switch_top1", "wideep", "relu_dropless_shared", "swiglu_softmax_renorm"])
+def test_backward_packed_matches_unpacked(name):
+    """Packed weights change only where the contractions read the weights from:
+    every output is bitwise the same (ragged F and the SwiGLU k switch included)."""
+    shape = BWD_SHAPES[name]
+    inp = synth.make_inputs(shape, seed=8, device="cuda", scale="unit")
+    condition_uniform(shape, inp)
+    dy = torch.randn((shape.T, shape.H), device="cuda").to(torch.bfloat16)
+    a = run_fwd_bwd(shape, inp, dy, 1.0, 1.0)
+    b = run_fwd_bwd(shape, inp, dy, 1.0, 1.0, packed=True)
+    for n in ("y", "dx", "dwg", "dgate", "dlogits"):
+        assert torch.equal(a[n].view(torch.uint8), b[n].view(torch.uint8)), n
+    for n, v in a["grads"].items():
+        if v is not None:
+            assert torch.equal(v.view(torch.uint8), b["grads"][n].view(torch.uint8)), n
 
 
 def test_backward_is_deterministic():
