@@ -90,10 +90,13 @@ __device__ __forceinline__ float gelu_grad(float z) {
   return 0.5f * (1.0f + erf_as7126(z * 0.70710678118654752f)) + z * phi;
 }
 
+// MODE and SWI (SwiGLU, DACT only) are template parameters so that each
+// variant's epilogue gets its own register allocation.
+template <int MODE, bool SWI>
 __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __grid_constant__ BParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const bool wgrad = p.mode == WGRAD;
+  constexpr bool wgrad = MODE == WGRAD;
   uint8_t* stage_base = smem;
   uint8_t* staging = smem + (wgrad ? WG_RING_BYTES : RING_BYTES);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + RING_BYTES + STAGING_BYTES);
@@ -104,8 +107,8 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool swiglu = p.mode == DACT && p.act == MOE_ACT_SWIGLU;
-  const int a_mn = wgrad ? 1 : 0, b_mn = p.mode == DACT ? 0 : 1;
+  constexpr bool swiglu = MODE == DACT && SWI;
+  constexpr int a_mn = wgrad ? 1 : 0, b_mn = MODE == DACT ? 0 : 1;
   const int ngroups = p.E + (p.n_shared ? 1 : 0);
 
   if (threadIdx.x == 0) {
@@ -129,7 +132,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
   // Tiles.  DGRAD / DACT: (128-row block of the row layout, N tile), the block's
   // group by binary search.  WGRAD: (group, 128-row tile of M, N tile), the k
   // blocks being the group's rows.
-  const int n_step = swiglu ? BNMAX / 2 : BNMAX;           // output columns per tile
+  constexpr int n_step = swiglu ? BNMAX / 2 : BNMAX;       // output columns per tile
   const int bn = BNMAX;                                    // MMA N
   const int n_tiles_n = (p.N + n_step - 1) / n_step;
   const int64_t rows_used = min((int64_t)p.off[ngroups], p.rows_max);
@@ -179,7 +182,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
           const uint32_t sb = sa + A_BYTES;
           const uint32_t fb = full0 + 8 * stage;
           mbar_expect_tx(fb, stage_bytes);
-          if (p.mode == WGRAD) {
+          if constexpr (MODE == WGRAD) {
             // A: rows kb*64.. of the M-wide source, two 64-feature chunks
             for (int i = 0; i < 2; ++i) tma_load_2d(sa + i * MN_CHUNK_BYTES, &p.tmA, (int)d.row0 + 64 * i, kb * BK, fb);
             const bool bs = sh && p.b_sep;
@@ -191,7 +194,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
             const int arow = (int)(sep ? d.row0 - p.off[p.E] : d.row0);
             tma_load_2d(sa, sep ? &p.tmAs : &p.tmA, kb * BK, arow, fb);
             const int z = sh ? 0 : d.g;
-            if (p.mode == DGRAD) {
+            if constexpr (MODE == DGRAD) {
               const bool second = p.k_switch > 0 && kb >= p.k_switch;
               const CUtensorMap* mb = sh ? (second ? &p.tmSB1 : &p.tmSB0) : (second ? &p.tmB1 : &p.tmB0);
               const int kk = (second ? kb - p.k_switch : kb) * BK;
@@ -299,15 +302,30 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
       }
     };
     for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+      const Tile d = decode(tile);
+      const int ncol0 = d.nt * n_step;
+      // DACT: this thread's dh (its row, 32 columns of each of its chunks) is
+      // loaded before the accumulator is ready, so the loads overlap the MMA
+      int4 dhv[2][4];
+      if constexpr (MODE == DACT) {
+        const int64_t grow = d.row0 + row_in_tile;
+#pragma unroll
+        for (int ci = 0; ci < 2; ++ci) {
+          const int col = ncol0 + quarter * 32 + ci * 128;
+          const __nv_bfloat16* src = p.dh + grow * (int64_t)p.N + col;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)     // columns past N read as zero, so dz is zero there
+            dhv[ci][q] = quarter * 32 + ci * 128 < n_step && grow < p.rows_max && col + 8 * q < p.N
+                             ? ld_nc_v4(src + 8 * q) : make_int4(0, 0, 0, 0);
+        }
+      }
       if (!mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag)) {
         *abort_flag = 1;
         set_status(p.status, MOE_ETIMEOUT, 22);
         break;
       }
       tc_fence_after();
-      const Tile d = decode(tile);
       const bool empty = d.kb1 <= d.kb0;
-      const int ncol0 = d.nt * n_step;
       const uint32_t tbase = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * BNMAX);
       for (int c = quarter * 32; c < n_step; c += 4 * 32) {
         const int col = ncol0 + c;
@@ -320,7 +338,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
         } else {
           tmem_ld(tbase + (uint32_t)c, v, 32);
         }
-        if (p.mode == WGRAD) {
+        if constexpr (MODE == WGRAD) {
           tmem_wait_ld();
           // this warp's 32 output rows lie on one side of m_split (a multiple
           // of 64); rows past m_valid and columns past N are clipped by the map
@@ -346,27 +364,25 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
           continue;
         }
         const int64_t row_base = d.row0 + sub * 32;
-        if (p.mode == DGRAD) {
+        if constexpr (MODE == DGRAD) {
           tmem_wait_ld();
           store_bf16(v, col, row_base);
           continue;
         }
         // DACT: z (and the SwiGLU up projection) recomputed; dz = dh * act'(z)
         float u[32];
-        if (swiglu) tmem_ld(tbase + (uint32_t)(BNMAX / 2 + c), u, 32);
+        if constexpr (swiglu) tmem_ld(tbase + (uint32_t)(BNMAX / 2 + c), u, 32);
         tmem_wait_ld();
-        const int64_t grow = d.row0 + row_in_tile;
-        const __nv_bfloat16* src = p.dh + grow * (int64_t)p.N + col;
+        const int ci = c >= 128 ? 1 : 0;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          // dh for 8 columns; columns past N read as zero, so dz is zero there
-          const int4 w = grow < p.rows_max && col + 8 * q < p.N ? ld_nc_v4(src + 8 * q) : make_int4(0, 0, 0, 0);
+          const int4 w = ci ? dhv[1][q] : dhv[0][q];
           const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&w);
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const float gi = __bfloat162float(e[i]);
             const float z = v[8 * q + i];
-            if (swiglu) {
+            if constexpr (swiglu) {
               const float s = 1.0f / (1.0f + __expf(-z));
               v[8 * q + i] = gi * u[8 * q + i] * s * (1.0f + z * (1.0f - s));   // da
               u[8 * q + i] = gi * z * s;                                        // db = dh * silu(a)
@@ -376,7 +392,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
           }
         }
         store_bf16(v, col, row_base);
-        if (swiglu) store_bf16(u, p.dz_ld / 2 + col, row_base);             // db at column Fp + col
+        if constexpr (swiglu) store_bf16(u, p.dz_ld / 2 + col, row_base);             // db at column Fp + col
       }
       tc_fence_before();
       mbar_arrive(tempty0 + 8 * acc);
@@ -516,13 +532,21 @@ static bool make_map_out(CUtensorMap* m, const void* base, int64_t rows, int W) 
   return encode_cached(m, key);
 }
 
-static cudaError_t launch(BParams& k, int64_t max_tiles, cudaStream_t stream) {
-  cudaError_t e = ensure_smem(grouped_gemm_bwd_kernel, SMEM_BYTES);
+template <int MODE, bool SWI>
+static cudaError_t launch_variant(BParams& k, int grid, cudaStream_t stream) {
+  cudaError_t e = ensure_smem(grouped_gemm_bwd_kernel<MODE, SWI>, SMEM_BYTES);
   if (e != cudaSuccess) return e;
+  launch_pdl(grouped_gemm_bwd_kernel<MODE, SWI>, grid, THREADS, SMEM_BYTES, stream, k);
+  return cudaGetLastError();
+}
+
+static cudaError_t launch(BParams& k, int64_t max_tiles, cudaStream_t stream) {
   const int sms = sm_count();
   const int grid = (int)(max_tiles < sms ? (max_tiles > 0 ? max_tiles : 1) : sms);
-  launch_pdl(grouped_gemm_bwd_kernel, grid, THREADS, SMEM_BYTES, stream, k);
-  return cudaGetLastError();
+  if (k.mode == DGRAD) return launch_variant<DGRAD, false>(k, grid, stream);
+  if (k.mode == WGRAD) return launch_variant<WGRAD, false>(k, grid, stream);
+  return k.act == MOE_ACT_SWIGLU ? launch_variant<DACT, true>(k, grid, stream)
+                                 : launch_variant<DACT, false>(k, grid, stream);
 }
 
 }  // namespace gb
