@@ -271,7 +271,7 @@ def kernel_source(stage: str) -> str:
             "ffn_gemm1": "grouped_gemm.cu", "ffn_gemm2": "grouped_gemm.cu",
             "combine_bwd": "backward.cu", "dispatch_bwd": "backward.cu", "router_wgrad": "backward.cu",
             "router_bwd": "router.cu", "dgrad_dh": "grouped_gemm_bwd.cu", "wgrad_w2": "grouped_gemm_bwd.cu",
-            "dact_dz": "grouped_gemm_bwd.cu", "wgrad_w1": "grouped_gemm_bwd.cu",
+            "dact_dz": "grouped_gemm_bwd.cu", "wgrad_w1": "grouped_gemm_bwd.cu", "dh_dz": "grouped_gemm_bwd.cu",
             "dgrad_dx": "grouped_gemm_bwd.cu"}.get(stage, "moe_abi.cu")
 
 
@@ -333,13 +333,13 @@ def train_launches_per_step(shape) -> int:
     """Kernels of one training step: the forward with MOE_FLAG_TRAINING (always
     unfused, plus the zeroing of xbuf's padding rows), then moe_layer_bwd:
     combine backward and the zeroing of dyrow's padding rows, four expert
-    contractions of the backward plus the recomputed first one, the router
+    contractions (dh and dz, with the first one recomputed, in one), the router
     backward (the aux coefficients, then dlogits), the dispatch backward and
     dWg (partial sums, then their reduction)."""
     router = 3 if shape.dtype == 1 else 1
     slots = 4 + (1 if shape.drop_policy == 1 and shape.cap_mode == 0 else 0)
     fwd = router + slots + 1 + 1 + 2 + 1
-    bwd = 2 + 5 + 2 + 1 + 2
+    bwd = 2 + 4 + 2 + 1 + 2            # dh and dz in one kernel
     return fwd + bwd
 
 
@@ -362,6 +362,9 @@ def bwd_stage_work(shape, kept: int, experts_used: int):
         "wgrad_w1": {"flops": 2.0 * rows * H * F * nm1, "bytes": rows * F * nm1 * b + rows * H * b + wexp * nm1 * F * H * 4},
         "router_bwd": {"flops": 0.0, "bytes": 2 * T * E * 4 + T * k * 8},
         "dgrad_dx": {"flops": 2.0 * rows * F * nm1 * H, "bytes": wexp * nm1 * F * H * b + rows * F * nm1 * b + rows * H * b},
+        # dh and dz in one kernel: both contractions, no dh round trip
+        "dh_dz": {"flops": 2.0 * rows * H * F * (1 + nm1),
+                  "bytes": wexp * H * F * b + wexp * nm1 * F * H * b + 2 * rows * H * b + rows * F * nm1 * b},
         "dispatch_bwd": {"flops": 2.0 * T * E * H,
                          "bytes": kept * H * b + sh * T * H * b + T * H * b + T * E * 4 + E * H * 4 + T * k * 8},
         "router_wgrad": {"flops": 2.0 * T * E * H, "bytes": T * E * 4 + T * H * b + E * H * 4},
@@ -786,11 +789,15 @@ def run_train(args, world, rank, local):
     fwd_ms = sum(e[0].elapsed_time(e[-1]) for e in fevs) / n_stage_steps
     stage_ms = {name: sum(e[j].elapsed_time(e[j + 1]) for e in bevs) / n_stage_steps
                 for j, name in enumerate(B.BWD_STAGES)}
+    # dh and dz come from one kernel: its interval is the dh one, dz's is empty
+    stage_ms["dh_dz"] = stage_ms.pop("dgrad_dh") + stage_ms.pop("dact_dz")
+    bwd_names = ["combine_bwd", "dh_dz", "wgrad_w2", "wgrad_w1", "router_bwd", "dgrad_dx", "dispatch_bwd",
+                 "router_wgrad"]
     bwd_ms = sum(e[0].elapsed_time(e[-1]) for e in bevs) / n_stage_steps
     work = bwd_stage_work(shape, kept, experts_used)
     long_step = ms_local > 5.0
-    per_stage = {s_: roofline(s_, work, stage_ms[s_], peaks, shape.name, True, long_step) for s_ in B.BWD_STAGES}
-    dom = max(B.BWD_STAGES, key=lambda s_: stage_ms[s_])
+    per_stage = {s_: roofline(s_, work, stage_ms[s_], peaks, shape.name, True, long_step) for s_ in bwd_names}
+    dom = max(bwd_names, key=lambda s_: stage_ms[s_])
     roof = per_stage[dom]
 
     # end to end: x and dy copied in from pinned host memory, the loss terms

@@ -82,13 +82,13 @@ __global__ void __launch_bounds__(kBwdWarps * 32) zero_pad_rows_kernel(__nv_bflo
 }
 
 // dx[t] = sum_r dxrow[row(t,r)] (+ dxrow[off[E] + t]) + sum_e dlogits[t,e] Wg[e,:],
-// fp32, one rounding.  CTA: 32 tokens x 256 columns; the router's part is a
+// fp32, one rounding.  CTA: 64 tokens x 256 columns; the router's part is a
 // small fp32 contraction over E, staged through shared memory in chunks of 32
-// experts: warp w owns tokens 4w..4w+3, lane l columns 4l..4l+3 and
-// 128+4l..128+4l+3, so each step reads one broadcast and two conflict-free
-// 16-byte words for 32 FMAs.  The rows are added in choice-rank order after
+// experts: warp w owns tokens 8w..8w+7, lane l columns 4l..4l+3 and
+// 128+4l..128+4l+3, so each step reads two broadcast and two conflict-free
+// 16-byte words for 64 FMAs.  The rows are added in choice-rank order after
 // the contraction.
-constexpr int kDxT = 32, kDxH = 256, kDxE = 32;
+constexpr int kDxT = 64, kDxH = 256, kDxE = 32;
 
 __global__ void __launch_bounds__(256) dispatch_bwd_kernel(DispatchBwdParams p) {
   __shared__ __align__(16) float sdl[kDxE][kDxT + 4];
@@ -98,9 +98,9 @@ __global__ void __launch_bounds__(256) dispatch_bwd_kernel(DispatchBwdParams p) 
   const int tid = threadIdx.x, ty = tid >> 5, tx = tid & 31;
   const int64_t t0 = (int64_t)blockIdx.x * kDxT;
   const int h0 = blockIdx.y * kDxH;
-  float acc[4][8];
+  float acc[8][8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
   for (int e0 = 0; e0 < p.E; e0 += kDxE) {
@@ -118,23 +118,24 @@ __global__ void __launch_bounds__(256) dispatch_bwd_kernel(DispatchBwdParams p) 
       *reinterpret_cast<float4*>(&swg[r][c]) = w;
     }
     __syncthreads();
-#pragma unroll 8
+#pragma unroll 4
     for (int e = 0; e < kDxE; ++e) {
-      const float4 d = *reinterpret_cast<const float4*>(&sdl[e][4 * ty]);
+      const float4 d0 = *reinterpret_cast<const float4*>(&sdl[e][8 * ty]);
+      const float4 d1 = *reinterpret_cast<const float4*>(&sdl[e][8 * ty + 4]);
       const float4 w0 = *reinterpret_cast<const float4*>(&swg[e][4 * tx]);
       const float4 w1 = *reinterpret_cast<const float4*>(&swg[e][128 + 4 * tx]);
-      const float dv[4] = {d.x, d.y, d.z, d.w};
+      const float dv[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
       const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 8; ++i)
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(dv[i], wv[j], acc[i][j]);
     }
     __syncthreads();
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int64_t t = t0 + 4 * ty + i;
+  for (int i = 0; i < 8; ++i) {
+    const int64_t t = t0 + 8 * ty + i;
     if (t >= p.T) break;
     int rows[kMaxK + 1];
     int nr = 0;
@@ -168,8 +169,8 @@ __global__ void __launch_bounds__(256) dispatch_bwd_kernel(DispatchBwdParams p) 
 // partial sum; the partials are added in chunk order.  Warp w owns experts
 // 8w..8w+7, lane l columns 4l..4l+3: per token, two broadcast and one
 // conflict-free 16-byte shared read feed 32 FMAs.  The chunk count is a pure
-// function of (T, E, H): enough CTAs for two per SM of a 148-SM part, at most
-// one chunk per 256 tokens.
+// function of (T, E, H): enough CTAs for four per SM of a 148-SM part, at most
+// one chunk per 128 tokens.
 constexpr int kDwgE = 64, kDwgH = 128, kDwgSub = 32;
 
 __global__ void __launch_bounds__(256) dwg_partial_kernel(const float* dlogits, const __nv_bfloat16* x, int64_t T,
@@ -244,8 +245,8 @@ __global__ void dwg_reduce_kernel(const float* part, int nchunk, int64_t n, floa
 
 int dwg_chunks(int64_t T, int E, int H) {
   const int64_t tiles = (int64_t)((E + kDwgE - 1) / kDwgE) * ((H + kDwgH - 1) / kDwgH);
-  const int64_t by_tokens = (T + 255) / 256;
-  const int64_t by_sms = (2 * 148 + tiles - 1) / tiles;
+  const int64_t by_tokens = (T + 127) / 128;
+  const int64_t by_sms = (4 * 148 + tiles - 1) / tiles;
   const int64_t c = by_tokens < by_sms ? by_tokens : by_sms;
   return (int)(c > 1 ? c : 1);
 }

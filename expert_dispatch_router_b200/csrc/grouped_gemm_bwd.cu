@@ -11,6 +11,10 @@
 //   WGRAD  dW2 = dY^T h,  dW1 = dz^T X            A and B both rows read along
 //          (one output matrix per expert, K =      their feature dimension
 //          that expert's rows)                     (MN-major)
+//   DHZ    DGRAD dh and DACT fused per tile: the   k runs twice over H: dY W2
+//          tile's dh and z accumulate side by      (MN-major B), then X W1^T
+//          side in TMEM, dz = bf16(dh) * act'(z)   (K-major B); dh never
+//                                                  reaches HBM
 // All three use the forward kernel's structure: one persistent CTA per SM, warp
 // 0 issues TMA loads into a ring of stages, warp 1 issues tcgen05.mma
 // (M=128, K=16, kind::f16, fp32 accumulators in TMEM, two 256-column buffers),
@@ -48,7 +52,7 @@ constexpr int WG_RING_BYTES = RING_BYTES + STAGING_BYTES - WG_STAGING_BYTES;
 static_assert(WG_RING_BYTES >= 2 * (A_BYTES + BNMAX * BK * 2), "WGRAD ring holds two stages");
 constexpr int MN_CHUNK_BYTES = 64 * BK * 2;                 // one 64-feature x 64-k box: 8 KB
 
-enum Mode { DGRAD = 0, DACT = 1, WGRAD = 2 };
+enum Mode { DGRAD = 0, DACT = 1, WGRAD = 2, DHZ = 3 };
 
 struct BParams {
   CUtensorMap tmA, tmAs;          // A (and the shared block's A when as_sep)
@@ -69,7 +73,9 @@ struct BParams {
   CUtensorMap tmWs, tmWs2;        // WGRAD: the shared expert's, [1, m_valid, N]
   int m_split;                    // WGRAD: output rows >= m_split go to tmW2 / tmWs2 (a multiple of 64)
   int m_valid;                    // WGRAD: rows of each output part (rows beyond are padding, not stored)
-  int b_packed;                   // DGRAD / DACT: weight maps are 5-D over packed 128 x 64 blocks
+  int b_packed;                   // DGRAD / DACT / DHZ: weight maps are 5-D over packed 128 x 64 blocks
+  CUtensorMap tmA2;               // DHZ: dyrow rows (K-major A of the dh pass)
+  CUtensorMap tmV, tmSV;          // DHZ: W2 (routed, shared) read along F (MN-major B of the dh pass)
 };
 
 // MN-major operand descriptor (128-byte swizzle): 64-feature chunks `lbo`
@@ -107,7 +113,8 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr bool swiglu = MODE == DACT && SWI;
+  constexpr bool dhz = MODE == DHZ;
+  constexpr bool swiglu = (MODE == DACT || dhz) && SWI;
   constexpr int a_mn = wgrad ? 1 : 0, b_mn = MODE == DACT ? 0 : 1;
   const int ngroups = p.E + (p.n_shared ? 1 : 0);
 
@@ -132,7 +139,9 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
   // Tiles.  DGRAD / DACT: (128-row block of the row layout, N tile), the block's
   // group by binary search.  WGRAD: (group, 128-row tile of M, N tile), the k
   // blocks being the group's rows.
-  constexpr int n_step = swiglu ? BNMAX / 2 : BNMAX;       // output columns per tile
+  // output columns per tile; DHZ holds dh (n_step columns) and z (n_step, or
+  // gate | up for SwiGLU) in one 256-column accumulator buffer
+  constexpr int n_step = dhz ? (swiglu ? 64 : 128) : (swiglu ? BNMAX / 2 : BNMAX);
   const int bn = BNMAX;                                    // MMA N
   const int n_tiles_n = (p.N + n_step - 1) / n_step;
   const int64_t rows_used = min((int64_t)p.off[ngroups], p.rows_max);
@@ -157,11 +166,11 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
       d.row0 = (tile / n_tiles_n) * BM;
       d.g = find_group(p.off, ngroups, d.row0);
       d.kb0 = 0;
-      d.kb1 = nk;
+      d.kb1 = dhz ? 2 * nk : nk;                           // DHZ: the dh pass, then the z pass
     }
     return d;
   };
-  const int b_bytes = bn * BK * 2;                         // 32 KB
+  const int b_bytes = dhz ? 128 * BK * 2 : bn * BK * 2;    // 16 KB (DHZ) or 32 KB
   const int stage_bytes = A_BYTES + b_bytes;
   const int n_stages = min(MAX_STAGES, (wgrad ? WG_RING_BYTES : RING_BYTES) / stage_bytes);
 
@@ -181,8 +190,37 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
           const uint32_t sa = smem_u32(stage_base + stage * stage_bytes);
           const uint32_t sb = sa + A_BYTES;
           const uint32_t fb = full0 + 8 * stage;
-          mbar_expect_tx(fb, stage_bytes);
-          if constexpr (MODE == WGRAD) {
+          if constexpr (!dhz) mbar_expect_tx(fb, stage_bytes);
+          if constexpr (dhz) {
+            const bool zp = kb >= nk;                      // z pass
+            const int kk = (zp ? kb - nk : kb) * BK;
+            const int z = sh ? 0 : d.g;
+            if (!zp) {
+              mbar_expect_tx(fb, A_BYTES + n_step * BK * 2);
+              tma_load_2d(sa, &p.tmA2, kk, (int)d.row0, fb);
+              const CUtensorMap* mv = sh ? &p.tmSV : &p.tmV;
+              for (int j = 0; j < n_step / 64; ++j) {
+                if (p.b_packed)
+                  tma_load_5d_at(sb + j * MN_CHUNK_BYTES, mv, kk & 127, (n0 >> 6) + j, kk >> 7, z, fb);
+                else
+                  tma_load_3d(sb + j * MN_CHUNK_BYTES, mv, n0 + 64 * j, kk, z, fb);
+              }
+            } else {
+              const bool sep = sh && p.as_sep;
+              mbar_expect_tx(fb, A_BYTES + (swiglu ? 2 : 1) * n_step * BK * 2);
+              tma_load_2d(sa, sep ? &p.tmAs : &p.tmA, kk, (int)(sep ? d.row0 - p.off[p.E] : d.row0), fb);
+              const CUtensorMap* m0 = sh ? &p.tmSB0 : &p.tmB0;
+              const CUtensorMap* m1 = sh ? &p.tmSB1 : &p.tmB1;
+              // W1 rows n0..n0+n_step (then W3's): one box each, n_step x 64 k
+              if (p.b_packed) {
+                tma_load_5d_at(sb, m0, n0 & 127, kb - nk, n0 >> 7, z, fb);
+                if (swiglu) tma_load_5d_at(sb + n_step * BK * 2, m1, n0 & 127, kb - nk, n0 >> 7, z, fb);
+              } else {
+                tma_load_3d(sb, m0, kk, n0, z, fb);
+                if (swiglu) tma_load_3d(sb + n_step * BK * 2, m1, kk, n0, z, fb);
+              }
+            }
+          } else if constexpr (MODE == WGRAD) {
             // A: rows kb*64.. of the M-wide source, two 64-feature chunks
             for (int i = 0; i < 2; ++i) tma_load_2d(sa + i * MN_CHUNK_BYTES, &p.tmA, (int)d.row0 + 64 * i, kb * BK, fb);
             const bool bs = sh && p.b_sep;
@@ -244,6 +282,10 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
       uint32_t acc_phase = 0;
       bool ok = true;
       const uint32_t idesc = make_idesc(bn, BM, a_mn, b_mn);
+      // DHZ: the dh pass (N = n_step, MN-major B) into columns [0, n_step), the
+      // z pass (N = n_step, or gate | up = 2 n_step, K-major B) after them
+      const uint32_t idesc_dh = make_idesc(n_step, BM, 0, 1);
+      const uint32_t idesc_z = make_idesc(swiglu ? 2 * n_step : n_step, BM, 0, 0);
       for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
         const Tile d = decode(tile);
         if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag)) { ok = false; break; }
@@ -254,12 +296,25 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
           tc_fence_after();
           const uint32_t sa = smem_u32(stage_base + stage * stage_bytes);
           const uint32_t sb = sa + A_BYTES;
-          const uint64_t ad = a_mn ? mn_desc(sa, MN_CHUNK_BYTES) : sw128_desc(sa);
-          const uint64_t bd = b_mn ? mn_desc(sb, MN_CHUNK_BYTES) : sw128_desc(sb);
-          const uint64_t astep = a_mn ? 128 : 2, bstep = b_mn ? 128 : 2;   // 16 k: 2 KB (MN-major) or 32 B
+          if constexpr (dhz) {
+            const bool zp = kb >= nk;
+            const uint64_t ad = sw128_desc(sa);
+            const uint64_t bd = zp ? sw128_desc(sb) : mn_desc(sb, MN_CHUNK_BYTES);
+            const uint64_t bstep = zp ? 2 : 128;
+            const uint32_t dt = d_tmem + (zp ? (uint32_t)n_step : 0u);
+            const uint32_t id = zp ? idesc_z : idesc_dh;
+            const int kfirst = zp ? nk : 0;
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            umma(d_tmem, ad + astep * kk, bd + bstep * kk, idesc, ((kb - d.kb0) | kk) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < BK / 16; ++kk)
+              umma(dt, ad + 2 * kk, bd + bstep * kk, id, ((kb - kfirst) | kk) != 0 ? 1u : 0u);
+          } else {
+            const uint64_t ad = a_mn ? mn_desc(sa, MN_CHUNK_BYTES) : sw128_desc(sa);
+            const uint64_t bd = b_mn ? mn_desc(sb, MN_CHUNK_BYTES) : sw128_desc(sb);
+            const uint64_t astep = a_mn ? 128 : 2, bstep = b_mn ? 128 : 2;   // 16 k: 2 KB (MN-major) or 32 B
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+              umma(d_tmem, ad + astep * kk, bd + bstep * kk, idesc, ((kb - d.kb0) | kk) != 0 ? 1u : 0u);
+          }
           umma_commit(empty0 + 8 * stage);
           if (++stage == n_stages) { stage = 0; phase ^= 1u; }
         }
@@ -369,6 +424,30 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
           store_bf16(v, col, row_base);
           continue;
         }
+        if constexpr (dhz) {
+          // v = dh; zv = z (SwiGLU: the gate pre-activation); u = the up projection.
+          // dh is rounded to bf16 first, as the unfused path stores it.
+          float zv[32];
+          tmem_ld(tbase + (uint32_t)(n_step + c), zv, 32);
+          float u[32];
+          if constexpr (swiglu) tmem_ld(tbase + (uint32_t)(2 * n_step + c), u, 32);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float gi = __bfloat162float(__float2bfloat16_rn(v[i]));
+            const float z = zv[i];
+            if constexpr (swiglu) {
+              const float s = 1.0f / (1.0f + __expf(-z));
+              v[i] = gi * u[i] * s * (1.0f + z * (1.0f - s));    // da
+              zv[i] = gi * z * s;                                 // db = dh * silu(a)
+            } else {
+              v[i] = p.act == MOE_ACT_RELU ? (z > 0.0f ? gi : 0.0f) : gi * gelu_grad(z);
+            }
+          }
+          store_bf16(v, col, row_base);
+          if constexpr (swiglu) store_bf16(zv, p.dz_ld / 2 + col, row_base);
+          continue;
+        }
         // DACT: z (and the SwiGLU up projection) recomputed; dz = dh * act'(z)
         float u[32];
         if constexpr (swiglu) tmem_ld(tbase + (uint32_t)(BNMAX / 2 + c), u, 32);
@@ -444,10 +523,10 @@ static bool make_map_mn_weights(CUtensorMap* m, const void* base, int G, int K, 
   return encode_cached(m, key);
 }
 // packed weights (the layout of moe_pack_weight: [G][N/128][K/64][128][64] for a
-// [G, N, K] matrix) as 5-D (64 k, 128 n, K/64, N/128, G).  K-major B: box
-// 64 x 128 (one block); MN-major B (the block's k are the output features):
-// box 64 x 64 (half a block).
-static bool make_map_packed(CUtensorMap* m, const void* base, int G, int N, int K, bool mn) {
+// [G, N, K] matrix) as 5-D (64 k, 128 n, K/64, N/128, G).  Box 64 x 128 (one
+// block) or, with `half`, 64 x 64 (half a block: an MN-major box, whose block k
+// are the output features, or a 64-row K-major box).
+static bool make_map_packed(CUtensorMap* m, const void* base, int G, int N, int K, bool half) {
   const cuuint64_t kb = (cuuint64_t)((K + BK - 1) / BK), nb = (cuuint64_t)((N + 127) / 128);
   MapKey key;
   memset(&key, 0, sizeof(key));
@@ -464,7 +543,7 @@ static bool make_map_packed(CUtensorMap* m, const void* base, int G, int N, int 
   key.strides[2] = key.strides[1] * kb;
   key.strides[3] = key.strides[2] * nb;
   key.box[0] = BK;
-  key.box[1] = mn ? 64 : 128;
+  key.box[1] = half ? 64 : 128;
   key.box[2] = key.box[3] = key.box[4] = 1;
   return encode_cached(m, key);
 }
@@ -482,8 +561,8 @@ static bool make_map_k_rows(CUtensorMap* m, const void* base, int64_t rows, int 
   key.box[1] = BM;
   return encode_cached(m, key);
 }
-// weights [G, N, K] bf16 read along K: box 64 x 128 x 1 (K-major B)
-static bool make_map_k_weights(CUtensorMap* m, const void* base, int G, int N, int K) {
+// weights [G, N, K] bf16 read along K: box 64 x box_n x 1 (K-major B)
+static bool make_map_k_weights(CUtensorMap* m, const void* base, int G, int N, int K, int box_n = 128) {
   MapKey key;
   memset(&key, 0, sizeof(key));
   key.base = base;
@@ -495,7 +574,7 @@ static bool make_map_k_weights(CUtensorMap* m, const void* base, int G, int N, i
   key.strides[0] = (cuuint64_t)K * 2;
   key.strides[1] = (cuuint64_t)N * K * 2;
   key.box[0] = BK;
-  key.box[1] = 128;
+  key.box[1] = box_n;
   key.box[2] = 1;
   return encode_cached(m, key);
 }
@@ -545,6 +624,9 @@ static cudaError_t launch(BParams& k, int64_t max_tiles, cudaStream_t stream) {
   const int grid = (int)(max_tiles < sms ? (max_tiles > 0 ? max_tiles : 1) : sms);
   if (k.mode == DGRAD) return launch_variant<DGRAD, false>(k, grid, stream);
   if (k.mode == WGRAD) return launch_variant<WGRAD, false>(k, grid, stream);
+  if (k.mode == DHZ)
+    return k.act == MOE_ACT_SWIGLU ? launch_variant<DHZ, true>(k, grid, stream)
+                                   : launch_variant<DHZ, false>(k, grid, stream);
   return k.act == MOE_ACT_SWIGLU ? launch_variant<DACT, true>(k, grid, stream)
                                  : launch_variant<DACT, false>(k, grid, stream);
 }
@@ -628,6 +710,57 @@ cudaError_t launch_bwd_dact(const BwdGemm& q, cudaStream_t stream) {
   k.dh = static_cast<const __nv_bfloat16*>(q.dh);
   k.dz_ld = ld;
   const int n_step = q.act == MOE_ACT_SWIGLU ? BNMAX / 2 : BNMAX;
+  return launch(k, (q.rows_max / BM) * ((q.N + n_step - 1) / n_step), stream);
+}
+
+cudaError_t launch_bwd_dhz(const BwdGemm& q, cudaStream_t stream) {
+  using namespace gb;
+  if (q.rows_max == 0) return cudaSuccess;
+  if (encode_fn() == nullptr) return cudaErrorNotSupported;
+  BParams k{};
+  const bool sw = q.act == MOE_ACT_SWIGLU;
+  const int n_step = sw ? 64 : 128;
+  const int G = q.E;
+  // z pass: A = dispatched rows (shared block: x), B = W1 (| W3) rows, n_step x 64 k boxes
+  bool ok = make_map_k_rows(&k.tmA, q.a, q.rows_max, q.K);
+  ok = ok && make_map_k_rows(&k.tmAs, q.a_shared ? q.a_shared : q.a, q.a_shared ? q.T : q.rows_max, q.K);
+  const void* b1 = q.b1 ? q.b1 : q.b0;
+  const void* s0 = q.sb0 ? q.sb0 : q.b0;
+  const void* s1 = q.sb1 ? q.sb1 : s0;
+  // dh pass: A = dyrow, B = W2 [G, K, N] read along N
+  ok = ok && make_map_k_rows(&k.tmA2, q.a2, q.rows_max, q.K);
+  const void* v0 = q.v;
+  const void* sv = q.sv ? q.sv : q.v;
+  if (q.b_packed) {
+    ok = ok && make_map_packed(&k.tmB0, q.b0, G, q.N, q.K, sw);
+    ok = ok && make_map_packed(&k.tmB1, b1, G, q.N, q.K, sw);
+    ok = ok && make_map_packed(&k.tmSB0, s0, 1, q.N, q.K, sw);
+    ok = ok && make_map_packed(&k.tmSB1, s1, 1, q.N, q.K, sw);
+    ok = ok && make_map_packed(&k.tmV, v0, G, q.K, q.N, true);
+    ok = ok && make_map_packed(&k.tmSV, sv, 1, q.K, q.N, true);
+  } else {
+    ok = ok && make_map_k_weights(&k.tmB0, q.b0, G, q.N, q.K, n_step);
+    ok = ok && make_map_k_weights(&k.tmB1, b1, G, q.N, q.K, n_step);
+    ok = ok && make_map_k_weights(&k.tmSB0, s0, 1, q.N, q.K, n_step);
+    ok = ok && make_map_k_weights(&k.tmSB1, s1, 1, q.N, q.K, n_step);
+    ok = ok && make_map_mn_weights(&k.tmV, v0, G, q.K, q.N);
+    ok = ok && make_map_mn_weights(&k.tmSV, sv, 1, q.K, q.N);
+  }
+  const int ld = sw ? 2 * ((q.N + BK - 1) / BK * BK) : q.N;   // da | db, db at column Fp
+  ok = ok && make_map_out(&k.tmD, q.out, q.rows_max, ld);
+  if (!ok) return cudaErrorInvalidValue;
+  k.b_packed = q.b_packed;
+  k.off = q.off;
+  k.status = q.status;
+  k.mode = DHZ;
+  k.E = q.E;
+  k.n_shared = q.n_shared;
+  k.act = q.act;
+  k.rows_max = q.rows_max;
+  k.K = q.K;
+  k.N = q.N;
+  k.as_sep = q.a_shared != nullptr;
+  k.dz_ld = ld;
   return launch(k, (q.rows_max / BM) * ((q.N + n_step - 1) / n_step), stream);
 }
 

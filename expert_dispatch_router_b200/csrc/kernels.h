@@ -202,11 +202,16 @@ struct BwdGemm {
   DevStatus* status;
   int64_t T, rows_max;
   int K, K0, N, M, E, n_shared, act, k_switch, m_split, m_valid;
-  int b_packed;             // dgrad / dact: weights in the packed block layout
+  int b_packed;             // dgrad / dact / dhz: weights in the packed block layout
+  const void* a2;           // dhz: dyrow (A of the dh pass)
+  const void* v;            // dhz: W2 [E, K, N] (B of the dh pass, read along N)
+  const void* sv;           // dhz: the shared expert's W2, or null
 };
 cudaError_t launch_bwd_dgrad(const BwdGemm& q, cudaStream_t stream);
 cudaError_t launch_bwd_dact(const BwdGemm& q, cudaStream_t stream);
 cudaError_t launch_bwd_wgrad(const BwdGemm& q, cudaStream_t stream);
+// dz = bf16(dyrow W2) * act'(x_rows W1^T) in one kernel (dh is not stored)
+cudaError_t launch_bwd_dhz(const BwdGemm& q, cudaStream_t stream);
 
 // Packed weight layout for the grouped GEMM: w [G, N, K] bf16 (K contiguous) ->
 // [G][ceil(N/128)][ceil(K/64)][128][64], zero-padded, so every TMA box of 128

@@ -609,17 +609,37 @@ int moe_layer_bwd(const moe_cfg* cfg, const void* x, const float* wg, const moe_
   q.n_shared = cfg->n_shared;
   q.act = cfg->act;
   const int packed = (cfg->flags & MOE_FLAG_PACKED_WEIGHTS) ? 1 : 0;
-  // 2. dh = dyrow W2 (W2 read along F)
+  // 2. dh = dyrow W2 (W2 read along F); fused (the default): dz = bf16(dh) *
+  //    act'(z) straight away, with z recomputed from the dispatched rows, and
+  //    dh never stored
+  const bool fused = !(cfg->flags & MOE_FLAG_UNFUSED);
   BwdGemm g = q;
-  g.a = bf(L.dyrow);
-  g.b0 = w->w2;
-  g.sb0 = sh ? w->sw2 : nullptr;
-  g.out = bf(L.dh);
-  g.K = H;
-  g.K0 = H;
-  g.N = F;
-  g.b_packed = packed;
-  if (launch_bwd_dgrad(g, s) != cudaSuccess) return MOE_ECUDA;
+  if (fused) {
+    g.a = bf(L.xbuf);
+    g.a_shared = sh ? x : nullptr;
+    g.b0 = w->w1;
+    g.b1 = sw ? w->w3 : nullptr;
+    g.sb0 = sh ? w->sw1 : nullptr;
+    g.sb1 = sh && sw ? w->sw3 : nullptr;
+    g.a2 = bf(L.dyrow);
+    g.v = w->w2;
+    g.sv = sh ? w->sw2 : nullptr;
+    g.out = bf(L.dz);
+    g.K = H;
+    g.N = F;
+    g.b_packed = packed;
+    if (launch_bwd_dhz(g, s) != cudaSuccess) return MOE_ECUDA;
+  } else {
+    g.a = bf(L.dyrow);
+    g.b0 = w->w2;
+    g.sb0 = sh ? w->sw2 : nullptr;
+    g.out = bf(L.dh);
+    g.K = H;
+    g.K0 = H;
+    g.N = F;
+    g.b_packed = packed;
+    if (launch_bwd_dgrad(g, s) != cudaSuccess) return MOE_ECUDA;
+  }
   if ((st = record(stage_events, 2, s)) != MOE_OK) return st;
   // 3. dW2 = dyrow^T h per expert
   g = q;
@@ -646,7 +666,7 @@ int moe_layer_bwd(const moe_cfg* cfg, const void* x, const float* wg, const moe_
   g.K = H;
   g.N = F;
   g.b_packed = packed;
-  if (launch_bwd_dact(g, s) != cudaSuccess) return MOE_ECUDA;
+  if (!fused && launch_bwd_dact(g, s) != cudaSuccess) return MOE_ECUDA;
   if ((st = record(stage_events, 4, s)) != MOE_OK) return st;
   // 5. dW1 (and dW3) = dz^T x_rows per expert; the shared block's rows are x
   g = q;

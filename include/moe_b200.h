@@ -105,6 +105,8 @@ enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
  *   and, for k == 1 without a shared expert, the second contraction writes
  *   gate * row to y[token] and zeroes the rows of fully dropped tokens (ybuf's
  *   routed rows are not written).  Larger layers run the separate kernels.
+ *   moe_layer_bwd with UNFUSED computes and stores dh, then dz, in two kernels
+ *   (default: one kernel, dh kept on chip); results are bitwise the same.
  * RANDOM_SECOND: GShard top-2 ([EP] router section: the second expert receives
  *   the token at random, according to its weight).  For k >= 2 the rank-1
  *   choice of token t is dispatched iff uniform[t] < 2 * gate[t,1], with
@@ -177,7 +179,7 @@ typedef struct moe_ws_views {
   float* dgate;            /* [T,k] gradient of each gate (0 for choices that add nothing to y) */
   float* dlogits;          /* [T,E] gradient of the router logits */
   void* dyrow;             /* [rows_max, H] gate-weighted output gradient of every row (bf16) */
-  void* dh;                /* [rows_max, F] gradient of the activations */
+  void* dh;                /* [rows_max, F] gradient of the activations (written with MOE_FLAG_UNFUSED only) */
   void* dz;                /* [rows_max, F] gradient of the pre-activations ([rows_max, 2*round_up(F,64)] for SwiGLU) */
   void* dxrow;             /* [rows_max, H] input gradient of every row */
 } moe_ws_views;
@@ -358,10 +360,14 @@ typedef struct moe_weight_grads {
  * recomputed with the activation's derivative applied (no pre-activations are
  * stored), its data and weight gradients, the router backward, the dispatch
  * backward (tokens sum their rows, plus dlogits Wg), and dWg = dlogits^T x.
+ * By default dh and dz come from one kernel (dz = bf16(dh) * act'(z), dh not
+ * stored: ws views' dh is left unwritten); with MOE_FLAG_UNFUSED two kernels
+ * compute and store dh, then dz.  Results are bitwise the same.
  * `stage_events`, if non-NULL, is an array of MOE_N_BWD_STAGE_EVENTS events
  * recorded on `stream` before the first kernel and after each of: combine
- * backward (with the zeroing of padding rows), dh, dW2, dz, dW1/dW3, router
- * backward, the rows' input gradients, dispatch backward, dWg.
+ * backward (with the zeroing of padding rows), dh (fused: dh and dz), dW2, dz
+ * (fused: an empty interval), dW1/dW3, router backward, the rows' input
+ * gradients, dispatch backward, dWg.
  * With MOE_FLAG_PACKED_WEIGHTS the data-gradient contractions read the packed
  * blocks (the weight gradients are always written in the linear-layer layout);
  * results are bitwise the same.

@@ -57,8 +57,9 @@ def _lib():
     B.load()
 
 
-def run_fwd_bwd(shape, inp, dy, d_aux, d_z, packed=False):
-    cfg = B.make_cfg(shape, flags=B.MOE_FLAG_TRAINING | (B.MOE_FLAG_PACKED_WEIGHTS if packed else 0))
+def run_fwd_bwd(shape, inp, dy, d_aux, d_z, packed=False, unfused=False):
+    cfg = B.make_cfg(shape, flags=B.MOE_FLAG_TRAINING | (B.MOE_FLAG_PACKED_WEIGHTS if packed else 0)
+                     | (B.MOE_FLAG_UNFUSED if unfused else 0))
     ws = B.alloc_workspace(cfg)
     T, H, F, E = shape.T, shape.H, shape.F, shape.E
     dev = "cuda"
@@ -251,6 +252,27 @@ def test_backward_packed_matches_unpacked(name):
     a = run_fwd_bwd(shape, inp, dy, 1.0, 1.0)
     b = run_fwd_bwd(shape, inp, dy, 1.0, 1.0, packed=True)
     for n in ("y", "dx", "dwg", "dgate", "dlogits"):
+        assert torch.equal(a[n].view(torch.uint8), b[n].view(torch.uint8)), n
+    for n, v in a["grads"].items():
+        if v is not None:
+            assert torch.equal(v.view(torch.uint8), b["grads"][n].view(torch.uint8)), n
+
+
+@pytest.mark.parametrize("name", list(BWD_SHAPES))
+def test_backward_fused_matches_unfused(name):
+    """dz from the fused dh/dz kernel (dh rounded to bf16 in registers) is
+    bitwise the unfused pair's (dh stored in bf16, then read); so is every
+    gradient downstream.  Packed weights on the fused side."""
+    shape = BWD_SHAPES[name]
+    inp = synth.make_inputs(shape, seed=9, device="cuda", scale="unit")
+    condition_uniform(shape, inp)
+    dy = torch.randn((shape.T, shape.H), device="cuda").to(torch.bfloat16)
+    a = run_fwd_bwd(shape, inp, dy, 1.0, 1.0, unfused=True)
+    a = {k: (v.clone() if torch.is_tensor(v) else v) for k, v in a.items()}
+    b = run_fwd_bwd(shape, inp, dy, 1.0, 1.0, packed=True)
+    R = int(a["expert_offset"][-1].item())
+    assert torch.equal(a["dz"][:R].view(torch.uint8), b["dz"][:R].view(torch.uint8)), "dz"
+    for n in ("dx", "dwg", "dgate", "dlogits"):
         assert torch.equal(a[n].view(torch.uint8), b[n].view(torch.uint8)), n
     for n, v in a["grads"].items():
         if v is not None:
