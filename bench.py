@@ -332,14 +332,15 @@ def roofline(stage: str, work: dict, ms: float, peaks: dict, workload: str, bf16
 def train_launches_per_step(shape) -> int:
     """Kernels of one training step: the forward with MOE_FLAG_TRAINING (always
     unfused, plus the zeroing of xbuf's padding rows), then moe_layer_bwd:
-    combine backward and the zeroing of dyrow's padding rows, four expert
-    contractions (dh and dz, with the first one recomputed, in one), the router
+    combine backward and the zeroing of dyrow's padding rows, five expert
+    contractions (four when T*k <= 256*E: dh and dz in one), the router
     backward (the aux coefficients, then dlogits), the dispatch backward and
     dWg (partial sums, then their reduction)."""
     router = 3 if shape.dtype == 1 else 1
     slots = 4 + (1 if shape.drop_policy == 1 and shape.cap_mode == 0 else 0)
     fwd = router + slots + 1 + 1 + 2 + 1
-    bwd = 2 + 4 + 2 + 1 + 2            # dh and dz in one kernel
+    fused = shape.T * shape.k <= 256 * shape.E    # dh and dz in one kernel
+    bwd = 2 + (4 if fused else 5) + 2 + 1 + 2
     return fwd + bwd
 
 
@@ -789,10 +790,13 @@ def run_train(args, world, rank, local):
     fwd_ms = sum(e[0].elapsed_time(e[-1]) for e in fevs) / n_stage_steps
     stage_ms = {name: sum(e[j].elapsed_time(e[j + 1]) for e in bevs) / n_stage_steps
                 for j, name in enumerate(B.BWD_STAGES)}
-    # dh and dz come from one kernel: its interval is the dh one, dz's is empty
-    stage_ms["dh_dz"] = stage_ms.pop("dgrad_dh") + stage_ms.pop("dact_dz")
-    bwd_names = ["combine_bwd", "dh_dz", "wgrad_w2", "wgrad_w1", "router_bwd", "dgrad_dx", "dispatch_bwd",
-                 "router_wgrad"]
+    # T*k <= 256*E: dh and dz come from one kernel, in the dh interval (dz's is empty)
+    bwd_fused = T * shape.k <= 256 * E
+    if bwd_fused:
+        stage_ms["dh_dz"] = stage_ms.pop("dgrad_dh") + stage_ms.pop("dact_dz")
+    dh_names = ["dh_dz"] if bwd_fused else ["dgrad_dh", "dact_dz"]
+    bwd_names = ["combine_bwd"] + dh_names + ["wgrad_w2", "wgrad_w1", "router_bwd", "dgrad_dx", "dispatch_bwd",
+                                              "router_wgrad"]
     bwd_ms = sum(e[0].elapsed_time(e[-1]) for e in bevs) / n_stage_steps
     work = bwd_stage_work(shape, kept, experts_used)
     long_step = ms_local > 5.0
@@ -860,6 +864,7 @@ def run_train(args, world, rank, local):
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "weights": "packed once before timing (moe_pack_weight)" if packed else "linear-layer layout"},
             "forward_ms": fwd_ms, "backward_ms": bwd_ms, "backward_stages_ms": stage_ms,
+            "backward_dh_dz_fused": bwd_fused,
             "stages_note": f"second timed pass of {n_stage_steps} steps with per-stage events",
             "roofline": {k_: roof[k_] for k_ in ("bound", "achieved", "peak", "unit", "frac", "traffic", "peak_source")},
             "roofline_detail": {s_: {k_: v[k_] for k_ in ("bound", "achieved", "unit", "frac", "ms_per_launch")}
