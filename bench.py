@@ -333,13 +333,13 @@ def train_launches_per_step(shape) -> int:
     """Kernels of one training step: the forward with MOE_FLAG_TRAINING (always
     unfused, plus the zeroing of xbuf's padding rows), then moe_layer_bwd:
     combine backward and the zeroing of dyrow's padding rows, five expert
-    contractions (four when T*k <= 256*E: dh and dz in one), the router
+    contractions (four when T*k <= 256*E or H <= 512: dh and dz in one), the router
     backward (the aux coefficients, then dlogits), the dispatch backward and
     dWg (partial sums, then their reduction)."""
     router = 3 if shape.dtype == 1 else 1
     slots = 4 + (1 if shape.drop_policy == 1 and shape.cap_mode == 0 else 0)
     fwd = router + slots + 1 + 1 + 2 + 1
-    fused = shape.T * shape.k <= 256 * shape.E    # dh and dz in one kernel
+    fused = shape.T * shape.k <= 256 * shape.E or shape.H <= 512    # dh and dz in one kernel
     bwd = 2 + (4 if fused else 5) + 2 + 1 + 2
     return fwd + bwd
 
@@ -790,8 +790,8 @@ def run_train(args, world, rank, local):
     fwd_ms = sum(e[0].elapsed_time(e[-1]) for e in fevs) / n_stage_steps
     stage_ms = {name: sum(e[j].elapsed_time(e[j + 1]) for e in bevs) / n_stage_steps
                 for j, name in enumerate(B.BWD_STAGES)}
-    # T*k <= 256*E: dh and dz come from one kernel, in the dh interval (dz's is empty)
-    bwd_fused = T * shape.k <= 256 * E
+    # T*k <= 256*E or H <= 512: dh and dz come from one kernel, in the dh interval (dz's is empty)
+    bwd_fused = T * shape.k <= 256 * E or H <= 512
     if bwd_fused:
         stage_ms["dh_dz"] = stage_ms.pop("dgrad_dh") + stage_ms.pop("dact_dz")
     dh_names = ["dh_dz"] if bwd_fused else ["dgrad_dh", "dact_dz"]

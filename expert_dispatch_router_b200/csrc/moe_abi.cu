@@ -612,10 +612,13 @@ int moe_layer_bwd(const moe_cfg* cfg, const void* x, const float* wg, const moe_
   // 2. dh = dyrow W2 (W2 read along F); fused: dz = bf16(dh) * act'(z) straight
   //    away, with z recomputed from the dispatched rows, and dh never stored.
   //    The fused kernel's tiles are narrower (128 or 64 output columns), so it
-  //    pays only where the contractions stream their weights from HBM: the
-  //    forward's rule, T*k <= 256*E (at most two 128-row blocks per expert on
-  //    average).  Larger layers run the two N = 256 kernels.
-  const bool fused = !(cfg->flags & MOE_FLAG_UNFUSED) && cfg->T * cfg->k <= 2 * kRowPad * (int64_t)E;
+  //    pays where the contractions stream their weights from HBM (the
+  //    forward's rule, T*k <= 256*E: at most two 128-row blocks per expert on
+  //    average) or where the contraction over H is short (H <= 512), which
+  //    leaves the unfused dz kernel bound by its epilogue.  Otherwise the two
+  //    N = 256 kernels run.
+  const bool fused = !(cfg->flags & MOE_FLAG_UNFUSED) &&
+                     (cfg->T * cfg->k <= 2 * kRowPad * (int64_t)E || H <= 512);
   BwdGemm g = q;
   if (fused) {
     g.a = bf(L.xbuf);

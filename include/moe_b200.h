@@ -106,7 +106,7 @@ enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
  *   gate * row to y[token] and zeroes the rows of fully dropped tokens (ybuf's
  *   routed rows are not written).  Larger layers run the separate kernels.
  *   moe_layer_bwd with UNFUSED computes and stores dh, then dz, in two kernels
- *   (default for T*k <= 256*E: one kernel, dh kept on chip); results are
+ *   (default for T*k <= 256*E or H <= 512: one kernel, dh kept on chip); results are
  *   bitwise the same.
  * RANDOM_SECOND: GShard top-2 ([EP] router section: the second expert receives
  *   the token at random, according to its weight).  For k >= 2 the rank-1
@@ -362,7 +362,7 @@ typedef struct moe_weight_grads {
  * stored), its data and weight gradients, the router backward, the dispatch
  * backward (tokens sum their rows, plus dlogits Wg), and dWg = dlogits^T x.
  * When T*k <= 256*E (the weight-streaming regime, as for the forward's fusion)
- * dh and dz come from one kernel (dz = bf16(dh) * act'(z), dh not stored: ws
+ * or H <= 512, dh and dz come from one kernel (dz = bf16(dh) * act'(z), dh not stored: ws
  * views' dh is left unwritten); otherwise, or with MOE_FLAG_UNFUSED, two
  * kernels compute and store dh, then dz.  Results are bitwise the same.
  * `stage_events`, if non-NULL, is an array of MOE_N_BWD_STAGE_EVENTS events

@@ -258,13 +258,12 @@ def test_backward_packed_matches_unpacked(name):
             assert torch.equal(v.view(torch.uint8), b["grads"][n].view(torch.uint8)), n
 
 
-@pytest.mark.parametrize("name", [n for n in BWD_SHAPES if n != "ds_k4"])
+@pytest.mark.parametrize("name", list(BWD_SHAPES))
 def test_backward_fused_matches_unfused(name):
     """dz from the fused dh/dz kernel (dh rounded to bf16 in registers) is
     bitwise the unfused pair's (dh stored in bf16, then read); so is every
     gradient downstream.  Packed weights on the fused side.  Every shape here
-    has T*k <= 256*E, where the library fuses; ds_k4 (T*k = 6000 > 3072) runs
-    the two kernels in both calls and is left out."""
+    has H <= 512, where the library fuses by default."""
     shape = BWD_SHAPES[name]
     inp = synth.make_inputs(shape, seed=9, device="cuda", scale="unit")
     condition_uniform(shape, inp)
