@@ -152,3 +152,61 @@ def test_packed_weight_sizes(lib):
     # packed weights are a bf16 feature
     with pytest.raises(B.MoeError):
         B.moe_workspace_size(B.make_cfg(synth.SWITCH_TINY_F32, flags=B.MOE_FLAG_PACKED_WEIGHTS))
+
+
+def test_backward_validation(lib):
+    """moe_layer_bwd rejects bad calls on the host, before any CUDA call (dummy
+    device pointers are never touched)."""
+    d = ctypes.c_void_p(256)
+    P = ctypes.c_void_p
+
+    def call(shape, flags, grads=None, ws_bytes=None):
+        cfg = B.make_cfg(shape, flags=flags)
+        w = B.moe_weights(*([256] * 6))
+        g = grads if grads is not None else B.moe_weight_grads(*([256] * 6))
+        nbytes = ws_bytes if ws_bytes is not None else B.moe_workspace_size(cfg)
+        return lib.moe_layer_bwd(ctypes.byref(cfg), d, d, ctypes.byref(w), d, ctypes.c_float(1.0),
+                                 ctypes.c_float(1.0), d, d, ctypes.byref(g), d, ctypes.c_size_t(nbytes), None, None)
+
+    small = synth.SWITCH_TOP1.replace(T=300, H=64, F=128, E=8)
+    # the backward runs on bf16 layers only
+    assert call(synth.SWITCH_TINY_F32, B.MOE_FLAG_TRAINING) == B.MOE_EUNSUPPORTED
+    # it needs the workspace of a forward with MOE_FLAG_TRAINING
+    assert call(small, 0) == B.MOE_EINVAL
+    # every weight gradient the layer has must be given
+    assert call(small, B.MOE_FLAG_TRAINING, grads=B.moe_weight_grads(0, 0, 256, 0, 0, 0)) == B.MOE_EINVAL
+    sw = small.replace(act=synth.ACT_SWIGLU)
+    assert call(sw, B.MOE_FLAG_TRAINING, grads=B.moe_weight_grads(256, 0, 256, 0, 0, 0)) == B.MOE_EINVAL
+    shared = small.replace(n_shared=1)
+    assert call(shared, B.MOE_FLAG_TRAINING, grads=B.moe_weight_grads(256, 0, 256, 0, 0, 0)) == B.MOE_EINVAL
+    # a workspace sized without the backward's buffers is too small
+    assert call(small, B.MOE_FLAG_TRAINING, ws_bytes=B.moe_workspace_size(B.make_cfg(small))) == B.MOE_EWORKSPACE
+
+
+@pytest.mark.parametrize("shape", [s for s in synth.WORKLOADS.values() if s.dtype == synth.DTYPE_BF16],
+                         ids=[n for n, s in synth.WORKLOADS.items() if s.dtype == synth.DTYPE_BF16])
+def test_training_workspace(lib, shape):
+    """MOE_FLAG_TRAINING adds the backward's buffers to the workspace (dgate,
+    dlogits, dyrow, dh, dz, dxrow), each at its documented size, and exposes
+    them in the views; without the flag the views are NULL."""
+    import torch
+    plain = B.make_cfg(shape)
+    tr = B.make_cfg(shape, flags=B.MOE_FLAG_TRAINING)
+    rows = B.moe_rows_max(tr)
+    T, H, F, E, k = shape.T, shape.H, shape.F, shape.E, shape.k
+    dzw = 2 * ((F + 63) // 64 * 64) if shape.act == synth.ACT_SWIGLU else F
+    need = T * k * 4 + T * E * 4 + rows * (2 * H + F + dzw) * 2
+    extra = B.moe_workspace_size(tr) - B.moe_workspace_size(plain)
+    assert extra >= need
+    fake = torch.empty(16, dtype=torch.uint8)         # views are host arithmetic on the base address only
+    v0 = B.moe_workspace_views(plain, fake)
+    assert not (v0.dgate or v0.dlogits or v0.dyrow or v0.dh or v0.dz or v0.dxrow)
+    v = B.moe_workspace_views(tr, fake)
+    base = fake.data_ptr()
+    size = B.moe_workspace_size(tr)
+    spans = sorted([(v.dgate, T * k * 4), (v.dlogits, T * E * 4), (v.dyrow, rows * H * 2), (v.dh, rows * F * 2),
+                    (v.dz, rows * dzw * 2), (v.dxrow, rows * H * 2)])
+    for (a, n), (b, _) in zip(spans, spans[1:]):
+        assert a + n <= b, "training buffers overlap"
+    assert all(base <= a and a + n <= base + size for a, n in spans)
+    assert all(a % 256 == base % 256 for a, _ in spans)
