@@ -74,6 +74,7 @@ struct BParams {
   int m_split;                    // WGRAD: output rows >= m_split go to tmW2 / tmWs2 (a multiple of 64)
   int m_valid;                    // WGRAD: rows of each output part (rows beyond are padding, not stored)
   int b_packed;                   // DGRAD / DACT / DHZ: weight maps are 5-D over packed 128 x 64 blocks
+  int wg_deep;                    // WGRAD: the deep variant (maps' box 16 x 32 x 1, 64-byte swizzle)
   CUtensorMap tmA2;               // DHZ: dyrow rows (K-major A of the dh pass)
   CUtensorMap tmV, tmSV;          // DHZ: W2 (routed, shared) read along F (MN-major B of the dh pass)
 };
@@ -96,15 +97,20 @@ __device__ __forceinline__ float gelu_grad(float z) {
   return 0.5f * (1.0f + erf_as7126(z * 0.70710678118654752f)) + z * phi;
 }
 
-// MODE and SWI (SwiGLU, DACT only) are template parameters so that each
-// variant's epilogue gets its own register allocation.
-template <int MODE, bool SWI>
+// MODE and V are template parameters so that each variant's epilogue gets its
+// own register allocation.  V: SwiGLU for DACT and DHZ; for WGRAD the deep
+// variant (the four-stage ring of the other modes, fp32 stored through one
+// 2 KB buffer per warp as 32 x 16 blocks), for layers whose experts have
+// many rows, where the k loop is long and the output a small part of the work.
+template <int MODE, bool V>
 __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __grid_constant__ BParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr bool wgrad = MODE == WGRAD;
+  constexpr bool wdeep = wgrad && V;
+  constexpr bool wshallow = wgrad && !V;
   uint8_t* stage_base = smem;
-  uint8_t* staging = smem + (wgrad ? WG_RING_BYTES : RING_BYTES);
+  uint8_t* staging = smem + (wshallow ? WG_RING_BYTES : RING_BYTES);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + RING_BYTES + STAGING_BYTES);
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + MAX_STAGES);
   const uint32_t tfull0 = smem_u32(bars + 2 * MAX_STAGES), tempty0 = smem_u32(bars + 2 * MAX_STAGES + 2);
@@ -114,7 +120,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr bool dhz = MODE == DHZ;
-  constexpr bool swiglu = (MODE == DACT || dhz) && SWI;
+  constexpr bool swiglu = (MODE == DACT || dhz) && V;
   constexpr int a_mn = wgrad ? 1 : 0, b_mn = MODE == DACT ? 0 : 1;
   const int ngroups = p.E + (p.n_shared ? 1 : 0);
 
@@ -172,7 +178,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
   };
   const int b_bytes = dhz ? 128 * BK * 2 : bn * BK * 2;    // 16 KB (DHZ) or 32 KB
   const int stage_bytes = A_BYTES + b_bytes;
-  const int n_stages = min(MAX_STAGES, (wgrad ? WG_RING_BYTES : RING_BYTES) / stage_bytes);
+  const int n_stages = min(MAX_STAGES, (wshallow ? WG_RING_BYTES : RING_BYTES) / stage_bytes);
 
   if (warp == 0) {
     // ---------------- TMA producer
@@ -336,7 +342,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
     const int sub = warp & 3;
     const int quarter = ew >> 2;
     const int row_in_tile = sub * 32 + lane;
-    const uint32_t stage_out = smem_u32(staging + ew * (wgrad ? 2 * WG_OUT_BYTES : STAGE_OUT_BYTES));
+    const uint32_t stage_out = smem_u32(staging + ew * (wshallow ? 2 * WG_OUT_BYTES : STAGE_OUT_BYTES));
     int wbuf = 0;                                    // WGRAD: staging buffer of the next store
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -400,6 +406,29 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
           const int m0 = (int)d.row0 + sub * 32;
           if (m0 >= p.M) continue;
           const bool hi = m0 >= p.m_split;
+          const bool sh = d.g == p.E;
+          const CUtensorMap* mw = sh ? (hi ? &p.tmWs2 : &p.tmWs) : (hi ? &p.tmW2 : &p.tmW);
+          if constexpr (wdeep) {
+            // two 32 x 16 fp32 blocks (64-byte rows, 64-byte swizzle) through the
+            // warp's one 2 KB buffer
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              if (lane == 0) bulk_wait_read0();
+              __syncwarp();
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                st_shared_v4(stage_out + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4),
+                             __float_as_uint(v[16 * h + 4 * q]), __float_as_uint(v[16 * h + 4 * q + 1]),
+                             __float_as_uint(v[16 * h + 4 * q + 2]), __float_as_uint(v[16 * h + 4 * q + 3]));
+              fence_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_3d(mw, stage_out, col + 16 * h, hi ? m0 - p.m_split : m0, sh ? 0 : d.g);
+                bulk_commit();
+              }
+            }
+            continue;
+          }
           const uint32_t buf = stage_out + wbuf * WG_OUT_BYTES;
           if (lane == 0) bulk_wait_read1();          // the store that last read `buf` is done with it
           __syncwarp();
@@ -410,8 +439,6 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
           fence_async_smem();
           __syncwarp();
           if (lane == 0) {
-            const bool sh = d.g == p.E;
-            const CUtensorMap* mw = sh ? (hi ? &p.tmWs2 : &p.tmWs) : (hi ? &p.tmW2 : &p.tmW);
             tma_store_3d(mw, buf, col, hi ? m0 - p.m_split : m0, sh ? 0 : d.g);
             bulk_commit();
           }
@@ -578,20 +605,21 @@ static bool make_map_k_weights(CUtensorMap* m, const void* base, int G, int N, i
   key.box[2] = 1;
   return encode_cached(m, key);
 }
-// fp32 weight gradients [G, rows, W], box 32 x 32 x 1, 128-byte swizzle (TMA store)
-static bool make_map_wout(CUtensorMap* m, const float* base, int G, int rows, int W) {
+// fp32 weight gradients [G, rows, W], box 32 x 32 x 1 with 128-byte swizzle, or
+// (deep) 16 x 32 x 1 with 64-byte swizzle (TMA store)
+static bool make_map_wout(CUtensorMap* m, const float* base, int G, int rows, int W, bool deep) {
   MapKey key;
   memset(&key, 0, sizeof(key));
   key.base = base;
   key.rank = 3;
   key.f32 = 1;
-  key.swizzle = CU_TENSOR_MAP_SWIZZLE_128B;
+  key.swizzle = deep ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   key.dims[0] = (cuuint64_t)W;
   key.dims[1] = (cuuint64_t)rows;
   key.dims[2] = (cuuint64_t)G;
   key.strides[0] = (cuuint64_t)W * 4;
   key.strides[1] = (cuuint64_t)rows * W * 4;
-  key.box[0] = 32;
+  key.box[0] = deep ? 16 : 32;
   key.box[1] = 32;
   key.box[2] = 1;
   return encode_cached(m, key);
@@ -623,7 +651,8 @@ static cudaError_t launch(BParams& k, int64_t max_tiles, cudaStream_t stream) {
   const int sms = sm_count();
   const int grid = (int)(max_tiles < sms ? (max_tiles > 0 ? max_tiles : 1) : sms);
   if (k.mode == DGRAD) return launch_variant<DGRAD, false>(k, grid, stream);
-  if (k.mode == WGRAD) return launch_variant<WGRAD, false>(k, grid, stream);
+  if (k.mode == WGRAD)
+    return k.wg_deep ? launch_variant<WGRAD, true>(k, grid, stream) : launch_variant<WGRAD, false>(k, grid, stream);
   if (k.mode == DHZ)
     return k.act == MOE_ACT_SWIGLU ? launch_variant<DHZ, true>(k, grid, stream)
                                    : launch_variant<DHZ, false>(k, grid, stream);
@@ -790,10 +819,12 @@ cudaError_t launch_bwd_wgrad(const BwdGemm& q, cudaStream_t stream) {
   k.m_split = q.m_split > 0 ? q.m_split : q.M;
   k.m_valid = q.m_valid > 0 ? q.m_valid : q.M;
   if (k.m_split < q.M && k.m_split % 64 != 0) return cudaErrorInvalidValue;
-  ok = make_map_wout(&k.tmW, q.w_out, q.E, k.m_valid, q.N);
-  ok = ok && make_map_wout(&k.tmW2, q.w_out2 ? q.w_out2 : q.w_out, q.E, k.m_valid, q.N);
-  ok = ok && make_map_wout(&k.tmWs, q.w_sh ? q.w_sh : q.w_out, 1, k.m_valid, q.N);
-  ok = ok && make_map_wout(&k.tmWs2, q.w_sh2 ? q.w_sh2 : (q.w_sh ? q.w_sh : q.w_out), 1, k.m_valid, q.N);
+  const bool deep = q.wg_deep != 0;
+  ok = make_map_wout(&k.tmW, q.w_out, q.E, k.m_valid, q.N, deep);
+  ok = ok && make_map_wout(&k.tmW2, q.w_out2 ? q.w_out2 : q.w_out, q.E, k.m_valid, q.N, deep);
+  ok = ok && make_map_wout(&k.tmWs, q.w_sh ? q.w_sh : q.w_out, 1, k.m_valid, q.N, deep);
+  ok = ok && make_map_wout(&k.tmWs2, q.w_sh2 ? q.w_sh2 : (q.w_sh ? q.w_sh : q.w_out), 1, k.m_valid, q.N, deep);
+  k.wg_deep = deep ? 1 : 0;
   if (!ok) return cudaErrorInvalidValue;
   const int64_t tiles = (int64_t)(q.E + (q.n_shared ? 1 : 0)) * ((q.M + BM - 1) / BM) * ((q.N + BNMAX - 1) / BNMAX);
   return launch(k, tiles, stream);

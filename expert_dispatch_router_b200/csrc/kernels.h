@@ -206,6 +206,7 @@ struct BwdGemm {
   const void* a2;           // dhz: dyrow (A of the dh pass)
   const void* v;            // dhz: W2 [E, K, N] (B of the dh pass, read along N)
   const void* sv;           // dhz: the shared expert's W2, or null
+  int wg_deep;              // wgrad: four-stage ring, fp32 stored as 32 x 16 blocks (experts with many rows)
 };
 cudaError_t launch_bwd_dgrad(const BwdGemm& q, cudaStream_t stream);
 cudaError_t launch_bwd_dact(const BwdGemm& q, cudaStream_t stream);

@@ -647,8 +647,13 @@ int moe_layer_bwd(const moe_cfg* cfg, const void* x, const float* wg, const moe_
     if (launch_bwd_dgrad(g, s) != cudaSuccess) return MOE_ECUDA;
   }
   if ((st = record(stage_events, 2, s)) != MOE_OK) return st;
-  // 3. dW2 = dyrow^T h per expert
+  // 3. dW2 = dyrow^T h per expert.  With at least 192 rows per expert on
+  //    average the k loops are long and the fp32 output a small part of the
+  //    work: the deep variant (four-stage ring) runs.  With fewer, the output
+  //    dominates and the two-stage ring with double-buffered stores runs.
+  const int wg_deep = cfg->T * cfg->k >= 192 * (int64_t)E ? 1 : 0;
   g = q;
+  g.wg_deep = wg_deep;
   g.a = bf(L.dyrow);
   g.b0 = bf(L.hbuf);
   g.M = H;
@@ -676,6 +681,7 @@ int moe_layer_bwd(const moe_cfg* cfg, const void* x, const float* wg, const moe_
   if ((st = record(stage_events, 4, s)) != MOE_OK) return st;
   // 5. dW1 (and dW3) = dz^T x_rows per expert; the shared block's rows are x
   g = q;
+  g.wg_deep = wg_deep;
   g.a = bf(L.dz);
   g.b0 = bf(L.xbuf);
   g.b_shared = sh ? x : nullptr;

@@ -212,6 +212,8 @@ BWD_SHAPES = {
     "sigmoid_zloss_random": synth.GSHARD_TOP2.replace(name="gshard_sigmoid", T=640, H=128, F=192, E=8,
                                                       score=synth.SCORE_SIGMOID_TOPK, renorm=1, z_coef=1e-2,
                                                       random_second=1),
+    # T*k/E = 200: the weight gradients take the deep variant (four-stage ring)
+    "swiglu_shared_deep": synth.WIDEEP_DROPLESS.replace(name="swiglu_shared_deep", T=800, H=128, F=136, E=8, k=2),
     "swiglu_softmax_renorm": synth.WIDEEP_DROPLESS.replace(name="swiglu_renorm", T=400, H=128, F=128, E=8, k=2,
                                                            score=synth.SCORE_SOFTMAX_TOPK, renorm=1, n_shared=0,
                                                            cap_mode=synth.CAP_CAPACITY, cf_num=1, cf_den=1,
