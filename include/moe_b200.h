@@ -362,9 +362,10 @@ typedef struct moe_weight_grads {
  * stored), its data and weight gradients, the router backward, the dispatch
  * backward (tokens sum their rows, plus dlogits Wg), and dWg = dlogits^T x.
  * When T*k <= 256*E (the weight-streaming regime, as for the forward's fusion)
- * or H <= 512, dh and dz come from one kernel (dz = bf16(dh) * act'(z), dh not stored: ws
- * views' dh is left unwritten); otherwise, or with MOE_FLAG_UNFUSED, two
- * kernels compute and store dh, then dz.  Results are bitwise the same.
+ * or H <= 512, dh and dz come from one kernel (dz = bf16(dh) * act'(z), dh
+ * not stored: ws views' dh is left unwritten); otherwise, or with
+ * MOE_FLAG_UNFUSED, two kernels compute and store dh, then dz.  Results are
+ * bitwise the same.
  * `stage_events`, if non-NULL, is an array of MOE_N_BWD_STAGE_EVENTS events
  * recorded on `stream` before the first kernel and after each of: combine
  * backward (with the zeroing of padding rows), dh (fused: dh and dz), dW2, dz
@@ -373,7 +374,15 @@ typedef struct moe_weight_grads {
  * With MOE_FLAG_PACKED_WEIGHTS the data-gradient contractions read the packed
  * blocks (the weight gradients are always written in the linear-layer layout);
  * results are bitwise the same.
- * Errors: MOE_EUNSUPPORTED for fp32 layers. */
+ * Ownership: every buffer is the caller's; nothing is allocated.  Gradients are
+ * written, not accumulated (add them into a master copy to accumulate).
+ * Asynchronous on `stream`; deterministic (fixed reduction orders).
+ * Errors: MOE_EUNSUPPORTED for fp32 layers; MOE_EINVAL for a bad cfg, a cfg
+ * without MOE_FLAG_TRAINING, a NULL input/output or a missing weight gradient
+ * (dw3 for SwiGLU, the shared ones with n_shared); MOE_EWORKSPACE when ws_bytes
+ * is below moe_workspace_size of the training cfg; MOE_ECUDA for a launch
+ * failure.  Bounded in-kernel waits that run out report MOE_ETIMEOUT through
+ * moe_sync_status. */
 enum { MOE_N_BWD_STAGE_EVENTS = 10 };
 MOE_API int moe_layer_bwd(const moe_cfg* cfg, const void* x, const float* wg, const moe_weights* w, const void* dy,
                           float d_aux, float d_z, void* dx, float* dwg, const moe_weight_grads* dw, void* ws,
