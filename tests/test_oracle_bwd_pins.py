@@ -202,3 +202,80 @@ def test_router_gradient_closed_forms():
     wrong = p * (wrong - (wrong * p).sum(1, keepdims=True))
     right = OB.router_backward(layer, lv, s2, dg, d_aux=0.0)
     assert np.abs(wrong - right).max() > 1e-3
+
+
+# ---------------------------------------------------------------- planted mistakes
+# Each plants one plausible slip in the backward oracle (on the CPU, by
+# replacing one of its functions for the duration of the test) and checks that
+# the autograd pin above catches it.
+_orig_router = OB.router_backward
+_orig_expert = OB.expert_backward
+_orig_act = OB.act_backward
+
+
+def _gelu_grad_without_z_phi(z):
+    from scipy.special import erf
+    return 0.5 * (1.0 + erf(np.asarray(z, dtype=np.float64) / np.sqrt(2.0)))
+
+
+def _swiglu_db_without_sigmoid(act, a, b, dh):
+    da, db = _orig_act(act, a, b, dh)
+    return (da, dh * a) if act == O.ACT_SWIGLU else (da, db)
+
+
+def _router_without_aux(layer, logits, selected, dgate, d_aux=1.0, d_z=1.0):
+    return _orig_router(layer, logits, selected, dgate, 0.0, d_z)
+
+
+def _router_zloss_halved(layer, logits, selected, dgate, d_aux=1.0, d_z=1.0):
+    return _orig_router(layer, logits, selected, dgate, d_aux, 0.5 * d_z)
+
+
+def _router_ignores_renorm(layer, logits, selected, dgate, d_aux=1.0, d_z=1.0):
+    import dataclasses
+    return _orig_router(dataclasses.replace(layer, renorm=0), logits, selected, dgate, d_aux, d_z)
+
+
+def _expert_dw2_sign(*a, **kw):
+    yrow, dX, d1, d2, d3 = _orig_expert(*a, **kw)
+    return yrow, dX, d1, -d2, d3
+
+
+def _expert_dx_without_up(*a, **kw):
+    yrow, dX, d1, d2, d3 = _orig_expert(*a, **kw)
+    if d3 is None:
+        return yrow, dX, d1, d2, d3
+    X, w1, w2, act, w3, dyrow = a[:6]
+    inter = {}
+    _orig_expert(X, w1, w2, act, w3, dyrow, inter)
+    return yrow, dX - inter["db"] @ np.asarray(w3, dtype=np.float64), d1, d2, d3
+
+
+PLANTED = {
+    "gelu_grad_without_z_phi": ("gelu_grad", _gelu_grad_without_z_phi, 1),
+    "swiglu_db_without_sigmoid": ("act_backward", _swiglu_db_without_sigmoid, 3),
+    "router_without_aux": ("router_backward", _router_without_aux, 0),
+    "router_zloss_halved": ("router_backward", _router_zloss_halved, 1),
+    "router_ignores_renorm": ("router_backward", _router_ignores_renorm, 1),
+    "expert_dw2_sign": ("expert_backward", _expert_dw2_sign, 0),
+    "expert_dx_without_up": ("expert_backward", _expert_dx_without_up, 3),
+}
+
+
+@pytest.mark.parametrize("name", list(PLANTED))
+def test_planted_mistake_is_caught(name, monkeypatch):
+    attr, fake, ci = PLANTED[name]
+    act, score, renorm, k, n_shared, cf, rnd, zc = CASES[ci]
+    T, H, F, E = 40, 6, 10, 5
+    x, wg, w1, w2, w3, sh, dy, u = _inputs(T, H, F, E, act, n_shared, seed=hash(CASES[ci]) % 1000, bias=0.8)
+    layer = O.OracleLayer(T=T, H=H, F=F, E=E, k=k, act=act, score=score, renorm=renorm,
+                          cap_mode=O.CAP_DROPLESS if cf is None else O.CAP_CAPACITY,
+                          cf_num=1 if cf is None else cf[0], cf_den=1 if cf is None else cf[1],
+                          n_shared=n_shared, random_second=rnd, z_coef=zc, aux_alpha=0.05)
+    monkeypatch.setattr(OB, attr, fake)
+    got = OB.layer_backward(layer, x, wg, w1, w2, w3, *sh, dy=dy, uniform=u, d_aux=1.7, d_z=0.9)
+    monkeypatch.undo()
+    want = _torch_grads(layer, x, wg, w1, w2, w3, sh, dy, got["fwd"], 1.7, 0.9)
+    caught = [n for n in ("dx", "dwg", "dw1", "dw2", "dw3", "dsw1", "dsw2", "dsw3")
+              if want[n] is not None and not np.allclose(got[n], want[n], rtol=1e-9, atol=1e-11)]
+    assert caught, f"planted mistake {name} not caught by the autograd pin"
