@@ -1,9 +1,11 @@
 #!/usr/bin/env python
 """Benchmark of the single-GPU MoE FFN forward pass (router -> slots -> dispatch
--> grouped expert FFN -> combine -> aux loss) through the C ABI.
+-> grouped expert FFN -> combine -> aux loss) through the C ABI, and with
+--pass train of one training step (the forward with MOE_FLAG_TRAINING, then
+moe_layer_bwd).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
-                  [--set FIELD=VALUE ...]
+                  [--set FIELD=VALUE ...] [--pass forward|train] [--unpacked] [--no-cpu-baseline]
 
 --set overrides one routing option of the workload (score, renorm, z_coef,
 random_second, drop_policy, cf_num, cf_den); the workload name then carries the
@@ -19,7 +21,8 @@ max-over-ranks timing reduction are plumbing.
 
 Prints one JSON line (rank 0).  `value` = tokens/s over all ranks, device-timed
 with CUDA events; `e2e` = the same metric with the step's inputs copied from
-pinned host memory and the result read back inside the timed region.
+pinned host memory and the result read back inside the timed region (the
+training step: x and dy in, the loss terms out).
 """
 from __future__ import annotations
 
