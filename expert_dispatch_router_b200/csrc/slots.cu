@@ -8,8 +8,8 @@
 // The assignment sequence is a = r*T + t (every first choice in token order,
 // then every second choice, ...).  slot(a) = number of earlier assignments of
 // the same expert.  Four small kernels, all deterministic:
-//   1. count   : CTA c counts its 2048-assignment chunk per expert (shared-memory
-//                histogram) -> chunk_cnt[e][c].
+//   1. count   : CTA c counts its 256-assignment chunk (kSlotChunk) per expert
+//                (shared-memory histogram) -> chunk_cnt[e][c].
 //   2. scan    : CTA e scans chunk_cnt[e][*] -> chunk base offsets, the expert's
 //                pre-drop count and kept count.
 //   3. offsets : one CTA: exclusive scan of the 128-padded kept counts -> the
@@ -32,7 +32,7 @@ namespace moe {
 
 constexpr int kSlotThreads = 256;
 constexpr int kSlotWarps = kSlotThreads / 32;
-constexpr int kStepsPerWarp = kSlotChunk / (kSlotWarps * 32);   // 8
+constexpr int kStepsPerWarp = kSlotChunk / (kSlotWarps * 32);   // 32-assignment steps per warp
 
 __device__ __forceinline__ int load_assignment(const SlotParams& p, int64_t a, int64_t A) {
   if (a >= A) return -1;

@@ -11,6 +11,8 @@
 // The array is loaded with the library, so every GPU that loads the library
 // holds it until the process exits.  The kernels are the same ones
 // moe_assign_slots launches.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -27,24 +29,58 @@ constexpr int64_t kStaticChunkInts = (int64_t)((kStaticScratchBytes - kStatusByt
 // Shared by every call on a device; holds the last call's contents.
 static __device__ __align__(256) unsigned char g_slot_scratch[kStaticScratchBytes];
 
-// Device address of g_slot_scratch, looked up once per device with that device
-// current.  (In host code the array's name is only a host-side stand-in.)
+// Unique id of the calling thread's current CUDA context (0 if unknown).  A
+// context re-created after cudaDeviceReset gets a new id, and the module (with
+// g_slot_scratch) is loaded again at a possibly different address.
+unsigned long long current_context_id() {
+  typedef CUresult (*GetCurrentFn)(CUcontext*);
+  typedef CUresult (*GetIdFn)(CUcontext, unsigned long long*);
+  static GetCurrentFn get_current = nullptr;
+  static GetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of g_slot_scratch, looked up with the device current the first
+// time a device (and each later context of it) calls.  (In host code the array's
+// name is only a host-side stand-in.)
 void* scratch_address(int& err) {
   static void* addr[64] = {nullptr};
+  static unsigned long long ctx_of[64] = {0};
   static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
     err = MOE_ECUDA;
     return nullptr;
   }
+  // 0 while no context is current on this thread: then look the address up (the
+  // lookup makes the device's primary context current) and note the context
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
+  if (addr[dev] == nullptr || ctx == 0 || ctx != ctx_of[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_slot_scratch) != cudaSuccess || p == nullptr) {
       err = MOE_ECUDA;
       return nullptr;
     }
     addr[dev] = p;
+    ctx_of[dev] = current_context_id();
   }
   err = MOE_OK;
   return addr[dev];
