@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(PKG, "libmoe_b200.so")
 MOE_OK, MOE_EINVAL, MOE_EUNSUPPORTED, MOE_ECUDA, MOE_ETIMEOUT, MOE_EDEVICE, MOE_EWORKSPACE = range(7)
 MOE_FLAG_KEEP_LOGITS, MOE_FLAG_RANDOM_SECOND, MOE_FLAG_UNFUSED, MOE_FLAG_PACKED_WEIGHTS, MOE_FLAG_TRAINING = \
     1, 2, 4, 8, 16
+MOE_FLAG_PACKED_ROUTER = 32
 MOE_N_STAGE_EVENTS = 8
 STAGES = ("router", "slots", "dispatch", "ffn_gemm1", "ffn_gemm2", "combine", "aux")
 MOE_N_BWD_STAGE_EVENTS = 10
@@ -85,6 +86,9 @@ _SIGS = {
     "moe_packed_weight_bytes": [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, SZP],
     "moe_pack_weight": [P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, P, P],
     "moe_clear_status": [P, P],
+    "moe_selftest_bounded_wait": [ctypes.c_int64, ctypes.c_int64, P, P, P],
+    "moe_router_planes_bytes": [ctypes.c_int32, ctypes.c_int32, SZP],
+    "moe_pack_router_weight": [P, ctypes.c_int32, ctypes.c_int32, P, P],
 }
 
 
@@ -276,6 +280,32 @@ def pack_weights(inp: dict, stream=None) -> dict:
         moe_pack_weight(w, buf, stream)
         out[n] = buf
     return out
+
+
+def moe_router_planes_bytes(E: int, H: int) -> int:
+    v = ctypes.c_size_t()
+    _check(load().moe_router_planes_bytes(E, H, ctypes.byref(v)), "moe_router_planes_bytes")
+    return v.value
+
+
+def moe_pack_router_weight(wg, planes, stream=None):
+    E, H = wg.shape
+    _check(load().moe_pack_router_weight(_ptr(wg), E, H, _ptr(planes), _stream(stream)), "moe_pack_router_weight")
+
+
+def pack_router(wg, stream=None):
+    """The three bf16 planes of the fp32 router weight (moe_pack_router_weight),
+    to pass as wg with MOE_FLAG_PACKED_ROUTER."""
+    E, H = wg.shape
+    buf = torch.empty(moe_router_planes_bytes(E, H) // 2, dtype=torch.bfloat16, device=wg.device)
+    moe_pack_router_weight(wg, buf, stream)
+    return buf
+
+
+def moe_selftest_bounded_wait(limit_cycles, abort_after_cycles, waited, ws, stream=None):
+    """One kernel whose bounded mbarrier wait nothing satisfies (see the header)."""
+    _check(load().moe_selftest_bounded_wait(int(limit_cycles), int(abort_after_cycles), _ptr(waited), _ptr(ws),
+                                            _stream(stream)), "moe_selftest_bounded_wait")
 
 
 def moe_sync_status(ws, stream=None) -> int:

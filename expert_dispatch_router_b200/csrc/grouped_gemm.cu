@@ -42,6 +42,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "route_common.cuh"
 #include "tc_common.cuh"
 
 namespace moe {
@@ -92,12 +93,109 @@ struct KParams {
   const float* sgate;
   const int32_t* sslot;
   int64_t sT;
+  // router: planes_per_stage 3 = a stage holds the A chunk and the matching
+  // chunk of all three planes; 1 = one plane per stage (the k loop visits
+  // (k block, plane) in the same order), for wide N where three planes would
+  // leave too few stages.
+  int planes_per_stage;
+  // router with routing fused (ROUTE_EJ > 0): after a tile's logits are stored,
+  // the epilogue warps route its 128 tokens (route_common.cuh) and store the
+  // tile's partial sums in row 4 * m-block of the 32-token partial arrays (the
+  // other three rows of the tile are zero).
+  RouterParams rp;
+  int64_t nblk;          // rows of the partial arrays (32 tokens each)
 };
+
+__device__ __forceinline__ void epilogue_bar() {
+  asm volatile("bar.sync 1, %0;" :: "r"(EPI_WARPS * 32) : "memory");
+}
+// True iff `v` holds in every epilogue thread (a barrier: every epilogue warp
+// takes the same branch after it, so none is left waiting at a later barrier).
+__device__ __forceinline__ bool epilogue_all(bool v) {
+  uint32_t r;
+  asm volatile("{\n\t.reg .pred pi, po;\n\t"
+               "setp.ne.u32 pi, %1, 0;\n\t"
+               "bar.red.and.pred po, 1, %2, pi;\n\t"
+               "selp.u32 %0, 1, 0, po;\n\t}"
+               : "=r"(r) : "r"((uint32_t)v), "r"(EPI_WARPS * 32) : "memory");
+  return r != 0;
+}
+
+// Routing of one router tile's 128 tokens by the 16 epilogue warps, once the
+// tile's fp32 logits are in memory (plain stores of this CTA: visible to its
+// threads after the barrier).  Warp w routes tokens w, w + 16, ...; the warps'
+// per-expert sums are then added in warp order through the staging buffer
+// (deterministic) into row 4 * mt of the 32-token partial arrays, and rows
+// 4 mt + 1 .. 4 mt + 3 are zeroed, so the reductions over all rows see the same
+// totals as with one row per 32 tokens.
+template <int EJ>
+__device__ __forceinline__ void route_tile(const KParams& p, int64_t mt, int ew, int lane, uint8_t* staging,
+                                           float* route_z) {
+  constexpr int EP = 32 * EJ;
+  static_assert(2 * EPI_WARPS * EP * 4 <= STAGING_BYTES, "router partials exceed the staging buffer");
+  const RouterParams& rp = p.rp;
+  const int E = rp.E;
+  const float* logits = static_cast<const float*>(p.d);
+  epilogue_bar();                                        // every warp's logits stores are done
+  float psum[EJ], zacc = 0.0f;
+  int cnt[EJ];
+#pragma unroll
+  for (int j = 0; j < EJ; ++j) { psum[j] = 0.0f; cnt[j] = 0; }
+  const int64_t t0 = mt * BM;
+  for (int i = ew; i < BM; i += EPI_WARPS) {
+    const int64_t t = t0 + i;
+    if (t >= rp.T) break;
+    float val[EJ];
+#pragma unroll
+    for (int j = 0; j < EJ; ++j) {
+      const int e = lane_expert<EJ>(lane, j);
+      val[j] = e < E ? logits[t * E + e] : 0.0f;
+    }
+    route_token<EJ>(rp, t, lane, val, psum, cnt, zacc);
+  }
+  float* sp = reinterpret_cast<float*>(staging);                       // [EPI_WARPS][EP]
+  int* sc = reinterpret_cast<int*>(staging) + EPI_WARPS * EP;           // [EPI_WARPS][EP]
+#pragma unroll
+  for (int j = 0; j < EJ; ++j) {
+    const int e = lane_expert<EJ>(lane, j);
+    sp[ew * EP + e] = psum[j];
+    sc[ew * EP + e] = cnt[j];
+  }
+  if (lane == 0) route_z[ew] = zacc;
+  epilogue_bar();
+  const int tid = ew * 32 + lane;
+  const int64_t row0 = 4 * mt;
+  for (int idx = tid; idx < 4 * E; idx += EPI_WARPS * 32) {
+    const int q = idx / E, e = idx - q * E;
+    const int64_t row = row0 + q;
+    if (row >= p.nblk) continue;
+    float ps = 0.0f;
+    int cs = 0;
+    if (q == 0) {
+#pragma unroll
+      for (int w = 0; w < EPI_WARPS; ++w) { ps += sp[w * EP + e]; cs += sc[w * EP + e]; }
+    }
+    rp.psum_part[row * E + e] = ps;
+    rp.cnt_part[row * E + e] = cs;
+  }
+  if (tid == 0) {
+    if (rp.zsum_part != nullptr) {
+      float z = 0.0f;
+#pragma unroll
+      for (int w = 0; w < EPI_WARPS; ++w) z += route_z[w];
+      for (int q = 0; q < 4; ++q)
+        if (row0 + q < p.nblk) rp.zsum_part[row0 + q] = q == 0 ? z : 0.0f;
+    }
+    if (mt == 0 && rp.aux_counter != nullptr) *rp.aux_counter = 0u;   // re-armed for moe_aux_loss
+  }
+  epilogue_bar();                                        // the staging buffer is free again
+}
 
 // GATHER: routed A rows are gathered from p.gsrc by warps 18-19 (fused
 // dispatch).  SCATTER: routed output rows go to p.sdst[token] * gate (fused
-// top-1 combine).  Both false: every operand moves by TMA.
-template <bool GATHER, bool SCATTER>
+// top-1 combine).  Both false: every operand moves by TMA.  ROUTE_EJ > 0:
+// router logits with routing fused into the epilogue (E <= 32 * ROUTE_EJ).
+template <bool GATHER, bool SCATTER, int ROUTE_EJ = 0>
 __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ KParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -111,6 +209,7 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
   const uint32_t drain = smem_u32(bars + 2 * MAX_STAGES + 4);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * MAX_STAGES + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* route_z = reinterpret_cast<float*>(tmem_slot + 2);     // [EPI_WARPS] z-loss sums (router)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool swiglu = p.epi == MOE_ACT_SWIGLU;
@@ -164,7 +263,9 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
   const int box_bytes = p.bbox * BK * 2;
   const int n_boxes = swiglu ? 2 : bn / p.bbox;
   const int plane_bytes = n_boxes * box_bytes;          // one plane's B chunk
-  const int stage_bytes = A_BYTES + p.b_planes * plane_bytes;
+  const int pps = p.b_planes == 1 ? 1 : p.planes_per_stage;   // planes per stage
+  const int pass = p.b_planes / pps;                    // stages per k block
+  const int stage_bytes = A_BYTES + pps * plane_bytes;
   const int n_stages = min(MAX_STAGES, RING_BYTES / stage_bytes);
 
   if (warp == 0) {
@@ -198,7 +299,8 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
         const int arow = (int)(sep ? row0 - p.off[p.E] : row0);
         const int z = sh ? 0 : g;
         const int n0 = nt * n_step;
-        for (int kb = kb0; kb < kb1; ++kb) {
+        for (int ks = kb0 * pass; ks < kb1 * pass; ++ks) {
+          const int kb = ks / pass, j1 = ks - kb * pass;   // k block; its plane when pps == 1
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag)) { ok = false; break; }
           const uint32_t sa = smem_u32(stage_base + stage * stage_bytes);
           const uint32_t sb = sa + A_BYTES;
@@ -218,9 +320,10 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
             tma_load_3d(sb, mb0, kbb, n0, z, fb);                 // gate rows
             tma_load_3d(sb + box_bytes, mb1, kbb, n0, z, fb);     // up rows
           } else {
-            for (int j = 0; j < p.b_planes; ++j)
+            for (int j = 0; j < pps; ++j)
               for (int b = 0; b < n_boxes; ++b)
-                tma_load_3d(sb + j * plane_bytes + b * box_bytes, mb0, j * p.plane_k + kbb, n0 + b * p.bbox, z, fb);
+                tma_load_3d(sb + j * plane_bytes + b * box_bytes, mb0, (j + j1) * p.plane_k + kbb,
+                            n0 + b * p.bbox, z, fb);
           }
           fills[stage]++;
           if (++stage == n_stages) { stage = 0; phase ^= 1u; }
@@ -303,19 +406,19 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
         if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-        for (int kb = kb0; kb < kb1; ++kb) {
+        for (int ks = kb0 * pass; ks < kb1 * pass; ++ks) {
           if (!mbar_wait(full0 + 8 * stage, phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
           if (GATHER) fence_async_smem();       // cp.async data (generic proxy) -> tensor-core reads
           const uint32_t sa = smem_u32(stage_base + stage * stage_bytes);
           const uint32_t sb = sa + A_BYTES;
           const uint64_t ad = sw128_desc(sa);
-          for (int j = 0; j < p.b_planes; ++j) {
+          for (int j = 0; j < pps; ++j) {
             const uint64_t bd = sw128_desc(sb + j * plane_bytes);
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk)   // advance 16 elements = 32 bytes along K
               umma(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc,
-                   ((kb - kb0) | kk | j) != 0 ? 1u : 0u);
+                   ((ks - kb0 * pass) | kk | j) != 0 ? 1u : 0u);
           }
           umma_commit(empty0 + 8 * stage);      // stage free once these MMAs finish
           if (++stage == n_stages) { stage = 0; phase ^= 1u; }
@@ -344,7 +447,9 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-      if (!mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag)) {
+      bool got = mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag);
+      if constexpr (ROUTE_EJ > 0) got = epilogue_all(got);   // the routing below has barriers
+      if (!got) {
         *abort_flag = 1;
         set_status(p.status, MOE_ETIMEOUT, 12);
         break;
@@ -448,6 +553,7 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
       tc_fence_before();
       mbar_arrive(tempty0 + 8 * acc);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      if constexpr (ROUTE_EJ > 0) route_tile<ROUTE_EJ>(p, mt, ew, lane, staging, route_z);
     }
     if (lane == 0) bulk_wait0();                 // this warp's output stores are complete
     __syncwarp();
@@ -536,19 +642,23 @@ static bool make_map_d(CUtensorMap* m, const void* base, int64_t rows, int N) {
   return encode_cached(m, key);
 }
 
-template <bool GATHER, bool SCATTER>
+template <bool GATHER, bool SCATTER, int ROUTE_EJ = 0>
 static cudaError_t launch_variant(KParams& k, int grid, cudaStream_t stream) {
-  auto kern = grouped_gemm_kernel<GATHER, SCATTER>;
+  auto kern = grouped_gemm_kernel<GATHER, SCATTER, ROUTE_EJ>;
   cudaError_t e = ensure_smem(kern, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   launch_pdl(kern, grid, GATHER ? THREADS_GATHER : THREADS, SMEM_BYTES, stream, k);
   return cudaGetLastError();
 }
 
-static cudaError_t launch_kernel(KParams& k, int64_t max_tiles, cudaStream_t stream) {
+static cudaError_t launch_kernel(KParams& k, int64_t max_tiles, cudaStream_t stream, int route_ej = 0) {
   const int sms = sm_count();
   // grid: one CTA per SM, never more than the largest possible tile count
   const int grid = (int)(max_tiles < sms ? (max_tiles > 0 ? max_tiles : 1) : sms);
+  if (route_ej == 1) return launch_variant<false, false, 1>(k, grid, stream);
+  if (route_ej == 2) return launch_variant<false, false, 2>(k, grid, stream);
+  if (route_ej == 4) return launch_variant<false, false, 4>(k, grid, stream);
+  if (route_ej == 8) return launch_variant<false, false, 8>(k, grid, stream);
   const bool gather = k.gsrc != nullptr, scatter = k.sdst != nullptr;
   if (gather) return scatter ? launch_variant<true, true>(k, grid, stream) : launch_variant<true, false>(k, grid, stream);
   return scatter ? launch_variant<false, true>(k, grid, stream) : launch_variant<false, false>(k, grid, stream);
@@ -559,6 +669,7 @@ static cudaError_t launch_kernel(KParams& k, int64_t max_tiles, cudaStream_t str
 cudaError_t launch_grouped_gemm(const GemmParams& p, cudaStream_t stream) {
   using namespace gg;
   if (p.rows_max == 0) return cudaSuccess;
+  if (p.two_sm && grouped_gemm_2sm_supported(p)) return launch_grouped_gemm_2sm(p, stream);
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
   const int box_n = 128;
   KParams k{};
@@ -597,6 +708,7 @@ cudaError_t launch_grouped_gemm(const GemmParams& p, cudaStream_t stream) {
   k.k_split = 1;
   k.out_f32 = 0;
   k.b_packed = p.b_packed;
+  k.planes_per_stage = 1;
   k.gsrc = static_cast<const __nv_bfloat16*>(p.gather_src);
   k.gidx = p.gather_idx;
   k.sdst = static_cast<__nv_bfloat16*>(p.scatter_dst);
@@ -633,21 +745,33 @@ __global__ void split_router_weight_kernel(const float* wg, __nv_bfloat16* plane
 
 int router_plane_width(int H) { return (H + gg::BK - 1) / gg::BK * gg::BK; }
 
-cudaError_t launch_router_gemm(const void* x, const float* wg, void* planes, float* logits, int64_t T, int H, int E,
-                               DevStatus* status, int* parts, cudaStream_t stream) {
+cudaError_t launch_split_router_weight(const float* wg, void* planes, int E, int H, cudaStream_t stream) {
+  const int Hp = router_plane_width(H);
+  const int64_t n = (int64_t)E * Hp;
+  const int64_t blocks = (n + 255) / 256;
+  launch_pdl(split_router_weight_kernel, (unsigned)(blocks < 2048 ? blocks : 2048), 256, 0, stream, wg,
+             static_cast<__nv_bfloat16*>(planes), E, H, Hp);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_router_gemm(const void* x, const float* wg, void* planes, bool planes_ready, float* logits,
+                               int64_t T, int H, int E, DevStatus* status, const RouterParams* route, int64_t nblk,
+                               int* parts, bool* routed, cudaStream_t stream) {
   using namespace gg;
+  *routed = false;
   if (T == 0) return cudaSuccess;
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
   const int Hp = router_plane_width(H);
-  {
-    const int64_t n = (int64_t)E * Hp;
-    const int64_t blocks = (n + 255) / 256;
-    launch_pdl(split_router_weight_kernel, (unsigned)(blocks < 2048 ? blocks : 2048), 256, 0, stream, 
-        wg, static_cast<__nv_bfloat16*>(planes), E, H, Hp);
+  if (!planes_ready) {
+    cudaError_t e = launch_split_router_weight(wg, planes, E, H, stream);
+    if (e != cudaSuccess) return e;
   }
-  // one stage = an A chunk plus the matching 64-k chunk of all three planes, so
-  // the N tile stays <= 128 columns to keep at least three stages in the ring
-  const int bn = E >= 128 ? 128 : (E + 15) / 16 * 16;
+  // Routing fused into the epilogue needs a token's E logits in one tile
+  // (N <= 256).  A stage holds the A chunk and the matching chunk of all three
+  // planes while that leaves three stages (N <= 128); wider tiles take one
+  // plane per stage.
+  const bool fuse = route != nullptr && E <= 256;
+  const int bn = fuse ? (E + 15) / 16 * 16 : (E >= 128 ? 128 : (E + 15) / 16 * 16);
   const int bbox = bn;
   KParams k{};
   bool ok = make_map_a(&k.tmA, x, T, H);
@@ -673,16 +797,24 @@ cudaError_t launch_router_gemm(const void* x, const float* wg, void* planes, flo
   k.bbox = bbox;
   k.b_planes = 3;
   k.plane_k = Hp;
+  k.planes_per_stage = 3 * (A_BYTES + 3 * bn * BK * 2) <= RING_BYTES ? 3 : 1;
   k.out_f32 = 1;
   // One tile per (m-block, n-tile); each k step multiplies the A chunk by the
-  // hi, mid and lo planes in that order, into one fp32 accumulator.  When the
-  // tiles cannot fill half the SMs, each tile's k blocks are split in two and
-  // the partial logits are added by the routing kernel.
+  // hi, mid and lo planes in that order, into one fp32 accumulator.  Unfused,
+  // when the tiles cannot fill half the SMs, each tile's k blocks are split in
+  // two and the partial logits are added by the routing kernel.
   const int64_t tiles = ((T + BM - 1) / BM) * ((E + bn - 1) / bn);
   const int nk = Hp / BK;
-  k.k_split = (tiles * 2 <= sm_count() && nk >= 4) ? 2 : 1;
+  k.k_split = (!fuse && tiles * 2 <= sm_count() && nk >= 4) ? 2 : 1;
   *parts = k.k_split;
-  return launch_kernel(k, tiles * k.k_split, stream);
+  int ej = 0;
+  if (fuse) {
+    k.rp = *route;
+    k.nblk = nblk;
+    ej = E <= 32 ? 1 : E <= 64 ? 2 : E <= 128 ? 4 : 8;
+    *routed = true;
+  }
+  return launch_kernel(k, tiles * k.k_split, stream, ej);
 }
 
 }  // namespace moe

@@ -25,13 +25,18 @@ struct RouterParams {
   int H, E, k, score, renorm;
 };
 int router_tile_tokens(int E);
-// bf16 x: fp32 router logits [T,E] on the tensor cores (Wg split into three bf16
-// planes in `planes`, E * 3 * router_plane_width(H) bf16 of scratch).
+// bf16 x: fp32 router logits [T,E] on the tensor cores from three bf16 planes
+// of Wg (hi + mid + lo = Wg exactly), laid out [E][3][router_plane_width(H)].
 int router_plane_width(int H);
-// `logits` holds 3*T*E floats; *parts (1 or 3) is how many fp32 partial [T,E]
-// arrays were written (their sum, in order, is the logits).
-cudaError_t launch_router_gemm(const void* x, const float* wg, void* planes, float* logits, int64_t T, int H, int E,
-                               DevStatus* status, int* parts, cudaStream_t stream);
+cudaError_t launch_split_router_weight(const float* wg, void* planes, int E, int H, cudaStream_t stream);
+// `planes` holds the planes already (planes_ready) or receives them from wg.
+// `logits` holds 3*T*E floats; *parts (1 or 2) is how many fp32 partial [T,E]
+// arrays were written (their sum, in order, is the logits).  With `route`
+// (E <= 256) the same launch also routes every token (ids, gates, partial sums
+// in rows of 32 tokens, nblk rows) and *routed is set: no launch_router needed.
+cudaError_t launch_router_gemm(const void* x, const float* wg, void* planes, bool planes_ready, float* logits,
+                               int64_t T, int H, int E, DevStatus* status, const RouterParams* route, int64_t nblk,
+                               int* parts, bool* routed, cudaStream_t stream);
 cudaError_t launch_router(const RouterParams& p, bool bf16, cudaStream_t stream);
 // term: E doubles of scratch followed by one unsigned ticket counter.
 // zsum_part (or null): per-CTA sums of lse^2; aux[1] = z_coef * their mean.
@@ -176,8 +181,18 @@ struct GemmParams {
   const float* scatter_gate;
   const int32_t* scatter_slot;
   int b_packed;             // 1: b0/b1/sb0/sb1 are packed (launch_pack_weight)
+  // Pairs of SMs (tcgen05 cta_group::2, 256 x 256 tiles) instead of one SM per
+  // 128 x 256 tile: for compute-bound layers, without gather or scatter.
+  // pair_prefix: ngroups + 1 ints of scratch for the groups' pair-tile prefix,
+  // computed by this launch unless pair_prefix_ready (same expert_offset as the
+  // launch that computed it).
+  int two_sm;
+  int32_t* pair_prefix;
+  int pair_prefix_ready;
 };
 cudaError_t launch_grouped_gemm(const GemmParams& p, cudaStream_t stream);
+bool grouped_gemm_2sm_supported(const GemmParams& p);
+cudaError_t launch_grouped_gemm_2sm(const GemmParams& p, cudaStream_t stream);
 
 // Grouped GEMMs of the backward pass (grouped_gemm_bwd.cu).
 //   dgrad: out[rows, N] = a[rows, K] * B, B the weights [G, K0, N] read along N

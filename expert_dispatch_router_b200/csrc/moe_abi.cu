@@ -15,7 +15,8 @@ namespace {
 constexpr int64_t kMaxCf = int64_t(1) << 20;
 
 struct Layout {
-  size_t status, psum, cnt, zsum, term, chunk, cum, lkey, lidx, ids, gates, slot, ecount, kept, off, rowtok, logits, lparts, planes, xbuf,
+  size_t status, psum, cnt, zsum, term, chunk, cum, lkey, lidx, ids, gates, slot, ecount, kept, off, pairs, rowtok, logits, lparts,
+      planes, xbuf,
       hbuf, ybuf, dyrow, dh, dz, dxrow, dgate, dlog, fcoef, dwgp;
   size_t total;
   int nblk_router, nchunk;
@@ -36,9 +37,9 @@ bool valid_cfg(const moe_cfg* c) {
   if (c->min_capacity < 0) return false;
   if (!(c->z_coef >= 0.0f) || isinf(c->z_coef)) return false;
   if (c->flags & ~(MOE_FLAG_KEEP_LOGITS | MOE_FLAG_RANDOM_SECOND | MOE_FLAG_UNFUSED | MOE_FLAG_PACKED_WEIGHTS |
-                   MOE_FLAG_TRAINING))
+                   MOE_FLAG_TRAINING | MOE_FLAG_PACKED_ROUTER))
     return false;
-  if ((c->flags & MOE_FLAG_PACKED_WEIGHTS) && c->dtype != MOE_DTYPE_BF16) return false;
+  if ((c->flags & (MOE_FLAG_PACKED_WEIGHTS | MOE_FLAG_PACKED_ROUTER)) && c->dtype != MOE_DTYPE_BF16) return false;
   if (c->drop_policy != MOE_DROP_POSITION && c->drop_policy != MOE_DROP_PROBS) return false;
   return true;
 }
@@ -111,6 +112,7 @@ Layout layout_of(const moe_cfg* c) {
   L.ecount = take(sizeof(int32_t) * E);
   L.kept = take(sizeof(int32_t) * E);
   L.off = take(sizeof(int32_t) * (E + 2));
+  L.pairs = take(sizeof(int32_t) * (E + 2));
   L.rowtok = take(sizeof(int32_t) * (size_t)L.rows_max);
   const bool tc_router = c->dtype == MOE_DTYPE_BF16;   // bf16 x: router logits on the tensor cores
   L.logits = take(((c->flags & (MOE_FLAG_KEEP_LOGITS | MOE_FLAG_TRAINING)) || tc_router) ? sizeof(float) * T * E : 0);
@@ -164,23 +166,29 @@ int run_route(const moe_cfg* c, const Layout& L, const void* x, const float* wg,
   RouterParams p = router_params(c, L, ws);
   p.uniform = random_second(c) ? uniform : nullptr;
   p.logits_parts = 1;
-  if (logits_in == nullptr && c->dtype == MOE_DTYPE_BF16 && c->T > 0) {
-    // logits on the tensor cores, then the softmax / top-k / gate kernel on them
-    float* buf = at<float>(ws, L.lparts);
-    int parts = 1;
-    if (launch_router_gemm(x, wg, at<void>(ws, L.planes), buf, c->T, c->H, c->E, at<DevStatus>(ws, L.status), &parts,
-                           s) != cudaSuccess)
-      return MOE_ECUDA;
-    logits_in = buf;
-    p.logits_parts = parts;
-  }
   p.x = x;
   p.wg = wg;
   p.logit_add = logit_add;
-  p.logits_in = logits_in;
   p.ids = ids;
   p.gates = gates;
   p.logits_out = logits_out;
+  if (logits_in == nullptr && c->dtype == MOE_DTYPE_BF16 && c->T > 0) {
+    // logits on the tensor cores; for E <= 256 the same launch routes the
+    // tokens, otherwise the softmax / top-k / gate kernel runs on the logits.
+    // With MOE_FLAG_PACKED_ROUTER, wg already holds the three bf16 planes.
+    float* buf = at<float>(ws, L.lparts);
+    int parts = 1;
+    bool routed = false;
+    const bool ready = (c->flags & MOE_FLAG_PACKED_ROUTER) != 0;
+    void* planes = ready ? const_cast<float*>(wg) : at<void>(ws, L.planes);
+    if (launch_router_gemm(x, wg, planes, ready, buf, c->T, c->H, c->E, at<DevStatus>(ws, L.status), &p,
+                           L.nblk_router, &parts, &routed, s) != cudaSuccess)
+      return MOE_ECUDA;
+    if (routed) return MOE_OK;
+    logits_in = buf;
+    p.logits_parts = parts;
+  }
+  p.logits_in = logits_in;
   return cuda_status(launch_router(p, c->dtype == MOE_DTYPE_BF16, s));
 }
 
@@ -239,6 +247,13 @@ int record(const moe_event_t* ev, int i, cudaStream_t s) {
   return cuda_status(cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev[i]), s));
 }
 
+// Compute-bound expert contractions (more than two 128-row blocks per expert
+// on average) run on pairs of SMs; the others stream their weights and run one
+// SM per tile (where dispatch and the top-1 combine can be fused in).
+bool two_sm_ffn(const moe_cfg* c) {
+  return c->dtype == MOE_DTYPE_BF16 && c->T * c->k > 2 * kRowPad * (int64_t)c->E;
+}
+
 // Both contractions of the expert FFN; `ev_mid`, if non-NULL, is recorded between them.
 // bf16 only: with `rowtok`, GEMM1 gathers its routed A rows from x (fused
 // dispatch; xbuf unused); with `y_top1` as well, GEMM2 writes gate * row to
@@ -268,6 +283,9 @@ int run_ffn(const moe_cfg* c, const Layout& L, const void* xbuf, const void* x, 
     g1.epi = c->act;
     g1.status = at<DevStatus>(ws, L.status);
     g1.b_packed = (c->flags & MOE_FLAG_PACKED_WEIGHTS) ? 1 : 0;
+    g1.two_sm = two_sm_ffn(c) ? 1 : 0;
+    g1.pair_prefix = at<int32_t>(ws, L.pairs);
+    g1.pair_prefix_ready = 0;
     if (rowtok != nullptr) {
       g1.a_routed = nullptr;
       g1.gather_src = x;
@@ -289,6 +307,7 @@ int run_ffn(const moe_cfg* c, const Layout& L, const void* xbuf, const void* x, 
     g2.epi = -1;
     g2.gather_src = nullptr;
     g2.gather_idx = nullptr;
+    g2.pair_prefix_ready = 1;                   // same offsets as GEMM1
     if (y_top1 != nullptr) {
       g2.gather_idx = rowtok;
       g2.scatter_dst = y_top1;
@@ -799,6 +818,22 @@ int moe_pack_weight(const void* w, int32_t G, int32_t N, int32_t K, void* packed
   return cuda_status(launch_pack_weight(w, G, N, K, packed, S(stream)));
 }
 
-const char* moe_version(void) { return "moe_b200 0.1 sm_100a"; }
+int moe_router_planes_bytes(int32_t E, int32_t H, size_t* bytes) {
+  if (bytes == nullptr || E < 1 || H < 1) return MOE_EINVAL;
+  if (E > kMaxE || H % 8 != 0) return MOE_EUNSUPPORTED;
+  *bytes = sizeof(uint16_t) * (size_t)E * 3 * (size_t)router_plane_width(H);
+  return MOE_OK;
+}
+
+int moe_pack_router_weight(const float* wg, int32_t E, int32_t H, void* planes, moe_stream_t stream) {
+  size_t bytes = 0;
+  const int st = moe_router_planes_bytes(E, H, &bytes);
+  if (st != MOE_OK) return st;
+  if (wg == nullptr || planes == nullptr) return MOE_EINVAL;
+  if (reinterpret_cast<uintptr_t>(planes) & 15) return MOE_EINVAL;
+  return cuda_status(launch_split_router_weight(wg, planes, E, H, S(stream)));
+}
+
+const char* moe_version(void) { return "moe_b200 0.2 sm_100a"; }
 
 }  // extern "C"

@@ -91,8 +91,13 @@ WIDEEP_DROPLESS = LayerShape("wideep_dropless_T16384_H7168_E256_k8", T=16384, H=
                              E=256, k=8, act=ACT_SWIGLU, score=SCORE_TOPK_SOFTMAX,
                              cap_mode=CAP_DROPLESS, n_shared=1, zipf_skew=1.1)
 
+# Profiling slice of the WideEP layer: the same H, F, SwiGLU, shared expert and
+# top-8 skewed routing, with 16 experts and T chosen so that an expert gets the
+# same ~512 rows on average (T*k/E = 512), in ~1.5 GB of weights.
+WIDEEP_SLICE = WIDEEP_DROPLESS.replace(name="wideep_slice_T1024_H7168_E16_k8", T=1024, E=16)
+
 WORKLOADS = {s.name: s for s in (SWITCH_TINY_F32, SWITCH_TOP1, GSHARD_TOP2, DS_HIGHK,
-                                  WIDEEP_DROPLESS)}
+                                  WIDEEP_DROPLESS, WIDEEP_SLICE)}
 
 
 def _normal(gen, shape, std, device):

@@ -96,7 +96,12 @@ enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
  *   padding rows, activations, un-gated expert rows; it runs unfused), and
  *   moe_workspace_size includes the backward pass's buffers.
  * PACKED_WEIGHTS (bf16 only): every pointer of moe_weights is a packed buffer
- *   written by moe_pack_weight (see there); results are bitwise the same. 
+ *   written by moe_pack_weight (see there); results are bitwise the same.
+ * PACKED_ROUTER (bf16 only): the `wg` argument of moe_route and moe_layer_fwd
+ *   points to the router planes written by moe_pack_router_weight instead of
+ *   the fp32 [E,H] weight (which those calls otherwise split into the same
+ *   planes on every call); results are bitwise the same.  moe_layer_bwd still
+ *   takes the fp32 weight.
  * UNFUSED: moe_layer_fwd runs dispatch and combine as separate kernels (the
  *   pages' literal sequence, filling xbuf and ybuf).  Without it, a bf16 layer
  *   with T*k <= 256*E (at most two 128-row blocks per expert on average, where
@@ -119,7 +124,8 @@ enum {
   MOE_FLAG_RANDOM_SECOND = 2,
   MOE_FLAG_UNFUSED = 4,
   MOE_FLAG_PACKED_WEIGHTS = 8,
-  MOE_FLAG_TRAINING = 16
+  MOE_FLAG_TRAINING = 16,
+  MOE_FLAG_PACKED_ROUTER = 32
 };
 
 /* Layer configuration.  Limits of this build: 1 <= E <= 1024, 1 <= k <= min(E,16),
@@ -217,7 +223,11 @@ MOE_API int moe_workspace_views(const moe_cfg* cfg, void* ws, moe_ws_views* view
  * Writes ids [T,k] int32 (-1: a second choice not dispatched), gates [T,k]
  * fp32, logits_out [T,E] fp32 if non-NULL, and per-block sums of p, selection
  * counts and, when cfg->z_coef != 0, squared log-sum-exps into `ws` for
- * moe_aux_loss. */
+ * moe_aux_loss.
+ * bf16 x: the logits come from the tensor cores, with wg split into three bf16
+ * planes whose sum is wg exactly (so every product is exact and the sum is
+ * accumulated in fp32); for E <= 256 the same launch also routes the tokens.
+ * With MOE_FLAG_PACKED_ROUTER, wg points to planes from moe_pack_router_weight. */
 MOE_API int moe_route(const moe_cfg* cfg, const void* x, const float* wg, const float* logit_add,
                       const float* uniform, int32_t* ids, float* gates, float* logits_out, void* ws,
                       moe_stream_t stream);
@@ -260,7 +270,9 @@ MOE_API int moe_assign_slots(const moe_cfg* cfg, const int32_t* ids, const float
  * the call clears the part that must start at zero.  Calls whose work
  * overlaps on the GPU (concurrent streams) race on the array: order them.
  * The first call on each device looks up the array's device address (with that
- * device current); make that first call before any stream capture.  An expert
+ * device current), and so does the first call in each later context of the
+ * device (after cudaDeviceReset the module, and the array, are loaded again);
+ * make that first call before any stream capture.  An expert
  * id outside [0,E) gives slot -1 for that assignment; this variant has no
  * status word for the caller to read. */
 MOE_API int moe_assign_slots_static(const moe_cfg* cfg, const int32_t* ids, int32_t* slot, int32_t* expert_count,
@@ -336,6 +348,17 @@ MOE_API int moe_activation_eval(int act, const float* z, const float* u, float* 
 MOE_API int moe_packed_weight_bytes(int32_t G, int32_t N, int32_t K, size_t* bytes);
 MOE_API int moe_pack_weight(const void* w, int32_t G, int32_t N, int32_t K, void* packed, moe_stream_t stream);
 
+/* One-time split of the fp32 router weight for the tensor-core router ([SWITCH]
+ * 2.2: the router computes in fp32).  Each element w of wg [E,H] (device, fp32)
+ * becomes three bf16 values hi = bf16(w), mid = bf16(w - hi), lo = bf16(w - hi -
+ * mid) with hi + mid + lo = w exactly, stored in `planes` (device, 16-byte
+ * aligned, moe_router_planes_bytes bytes) as [E][3][Hp], Hp = H rounded up to
+ * 64, zero-padded.  Pass `planes` as wg with MOE_FLAG_PACKED_ROUTER.
+ * Asynchronous on `stream`.  Errors: MOE_EINVAL (NULL, misaligned, E or H < 1),
+ * MOE_EUNSUPPORTED (E > 1024 or H % 8 != 0), MOE_ECUDA. */
+MOE_API int moe_router_planes_bytes(int32_t E, int32_t H, size_t* bytes);
+MOE_API int moe_pack_router_weight(const float* wg, int32_t E, int32_t H, void* planes, moe_stream_t stream);
+
 /* Gradients of the expert weights (device pointers, fp32, the shapes of
  * moe_weights: dw1/dw3 [E,F,H], dw2 [E,H,F], shared [1,...]; NULL where absent). */
 typedef struct moe_weight_grads {
@@ -396,6 +419,22 @@ MOE_API int moe_sync_status(void* ws, moe_stream_t stream);
 
 /* Clears the device status word of `ws` (asynchronously on `stream`). */
 MOE_API int moe_clear_status(void* ws, moe_stream_t stream);
+
+/* Self-check of the device-side failure detection (no page counterpart: it
+ * exercises this library's bounded waits).  Launches one tiny kernel on
+ * `stream` whose warp waits on an mbarrier that nothing arrives at, with the
+ * same bounded-wait routine every tensor-core kernel here uses, limited to
+ * `limit_cycles` SM clock cycles (0 .. about 1 s worth, the kernels' own limit).
+ * With abort_after_cycles >= 0 a second warp raises the CTA's abort flag after
+ * that many cycles and the wait must end through the flag instead.  Either way
+ * the kernel records MOE_ETIMEOUT in the status word at the start of `ws` (any
+ * workspace of at least 256 bytes) and returns: read it with moe_sync_status.
+ * *waited_cycles (DEVICE pointer to one int64) receives the cycles the wait
+ * lasted.  No copy or MMA is in flight when the wait gives up, so the context
+ * stays usable.  Errors: MOE_EINVAL for NULL pointers or limits above the
+ * kernels' own; MOE_ECUDA for a launch failure. */
+MOE_API int moe_selftest_bounded_wait(int64_t limit_cycles, int64_t abort_after_cycles, int64_t* waited_cycles,
+                                      void* ws, moe_stream_t stream);
 
 /* Static description of a status code. */
 MOE_API const char* moe_strerror(int status);

@@ -114,16 +114,23 @@ def condition_uniform(shape: synth.LayerShape, inp: dict, margin: float = 1e-4) 
     inp["uniform"].copy_(torch.from_numpy(np.clip(u, 0.0, np.nextafter(1.0, 0.0)).astype(np.float32)))
 
 
-def run_layer(shape: synth.LayerShape, inp: dict, keep_logits=True, ws=None, unfused=False, packed=False):
+def run_layer(shape: synth.LayerShape, inp: dict, keep_logits=True, ws=None, unfused=False, packed=False,
+              packed_router=False):
     """One moe_layer_fwd call.  By default dispatch (and, for top-1 without a
     shared expert, the combine) run fused into the expert contractions;
     unfused=True runs them as separate kernels and fills xbuf / ybuf.
-    packed=True packs the expert weights first (moe_pack_weight)."""
+    packed=True packs the expert weights first (moe_pack_weight);
+    packed_router=True splits the router weight into its planes first
+    (moe_pack_router_weight)."""
     flags = (B.MOE_FLAG_KEEP_LOGITS if keep_logits else 0) | (B.MOE_FLAG_UNFUSED if unfused else 0)
     wsrc = inp
     if packed:
         flags |= B.MOE_FLAG_PACKED_WEIGHTS
         wsrc = B.pack_weights(inp)
+    wg = inp["wg"]
+    if packed_router:
+        flags |= B.MOE_FLAG_PACKED_ROUTER
+        wg = B.pack_router(inp["wg"])
     cfg = B.make_cfg(shape, flags=flags)
     if ws is None:
         ws = B.alloc_workspace(cfg)
@@ -131,8 +138,7 @@ def run_layer(shape: synth.LayerShape, inp: dict, keep_logits=True, ws=None, unf
     y = torch.full((T, H), float("nan"), dtype=inp["x"].dtype, device="cuda")
     aux = torch.full((2,), float("nan"), dtype=torch.float32, device="cuda")
     ecount = torch.full((shape.E,), -7, dtype=torch.int32, device="cuda")
-    B.moe_layer_fwd(cfg, inp["x"], inp["wg"], inp["logit_add"], inp.get("uniform"), B.make_weights(wsrc), y, aux, ecount,
-                    ws)
+    B.moe_layer_fwd(cfg, inp["x"], wg, inp["logit_add"], inp.get("uniform"), B.make_weights(wsrc), y, aux, ecount, ws)
     st = B.moe_sync_status(ws)
     assert st == B.MOE_OK, f"device status {st}: {B.strerror(st)}"
     out = B.workspace_tensors(cfg, ws)

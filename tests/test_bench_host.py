@@ -11,22 +11,24 @@ def test_forward_launch_counts():
     # Switch top-1 (profiles/launches_switch_top1_T8192_H768_E64.md): split, router GEMM,
     # route_logits, 4 slot kernels, GEMM1 with the dispatch, GEMM2 with the combine
     assert bench.launches_per_step(synth.SWITCH_TOP1) == 9
-    # unfused bf16 layers add the dispatch and combine kernels
-    assert bench.launches_per_step(synth.GSHARD_TOP2) == 11
+    # unfused bf16 layers add the dispatch and combine kernels, and (T*k > 256*E) the
+    # pair-tile prefix of the SM-pair contractions
+    assert bench.launches_per_step(synth.GSHARD_TOP2) == 12
     # fp32 router in one launch; the fp32 layer is never fused
     assert bench.launches_per_step(synth.SWITCH_TINY_F32) == 1 + 4 + 1 + 2 + 1
     # the "probs" drop policy adds the per-expert select
-    assert bench.launches_per_step(synth.DS_HIGHK.replace(drop_policy=1)) == 12
+    assert bench.launches_per_step(synth.DS_HIGHK.replace(drop_policy=1)) == 13
 
 
 def test_training_launch_counts():
     # Switch top-1 (profiles/launches_train_switch_top1_T8192_H768_E64.md): 12 forward
     # launches with MOE_FLAG_TRAINING, 11 backward (dh and dz fused)
     assert bench.train_launches_per_step(synth.SWITCH_TOP1) == 23
-    # GShard top-2: T*k > 256*E and H > 512, so dh and dz are two kernels
-    assert bench.train_launches_per_step(synth.GSHARD_TOP2) == 24
+    # GShard top-2: T*k > 256*E (SM-pair forward, + the pair prefix) and H > 512, so
+    # dh and dz are two kernels
+    assert bench.train_launches_per_step(synth.GSHARD_TOP2) == 25
     # DeepSpeed k=4: H <= 512 fuses them again
-    assert bench.train_launches_per_step(synth.DS_HIGHK) == 23
+    assert bench.train_launches_per_step(synth.DS_HIGHK) == 24
 
 
 def test_workload_overrides():
@@ -57,3 +59,17 @@ def test_roofline_bound_selection():
     r1 = bench.roofline("ffn_gemm1", wg, 0.3, peaks, g.name)
     r2 = bench.roofline("ffn_gemm1", wg, 0.3, peaks, g.name, sustained=True)
     assert r1["bound"] == "tensor" and r2["peak"] == peaks["bf16_tflops_sustained"] < r1["peak"]
+
+
+def test_oracle_sample_choice_and_extrapolation():
+    import torch
+    # the WideEP layer's experts would take ~90 GB in float64: it is timed by sample
+    assert bench.oracle_weights_fp64_bytes(synth.WIDEEP_DROPLESS) > bench.ORACLE_FULL_LAYER_BYTES
+    assert bench.oracle_weights_fp64_bytes(synth.SWITCH_TOP1) < bench.ORACLE_FULL_LAYER_BYTES
+    shape = synth.WIDEEP_DROPLESS.replace(name="tiny", T=96, H=32, F=24, E=8, k=2)
+    inp = synth.make_inputs(shape, seed=0)
+    host = bench.host_inputs(inp)
+    sec, what = bench.oracle_extrapolated_time(shape, host, kept_rows=shape.T * shape.k, n_route=48, n_experts=2,
+                                               n_shared_tok=16)
+    assert sec > 0 and "extrapolated" in what and "48 of 96" in what
+    assert torch.is_tensor(inp["x"])

@@ -38,6 +38,12 @@ SMALL = {
                                                              bias_row0=0.0),
     "tiny_f32_swiglu_shared": synth.SWITCH_TINY_F32.replace(name="tiny_f32_swiglu", act=synth.ACT_SWIGLU, k=2,
                                                             n_shared=1, score=synth.SCORE_TOPK_SOFTMAX),
+    # more than two 128-row blocks per expert on average: the contractions run on
+    # pairs of SMs (256-row tiles; odd block counts leave half a pair tile idle)
+    "wideep_2sm": synth.WIDEEP_DROPLESS.replace(name="wideep_2sm", T=600, H=200, F=200, E=4, k=2),
+    "gshard_2sm": synth.GSHARD_TOP2.replace(name="gshard_2sm", T=1200, H=136, F=520, E=4),
+    "relu_2sm_shared": synth.SWITCH_TOP1.replace(name="relu_2sm_shared", T=900, H=96, F=264, E=3, k=2,
+                                                 cap_mode=synth.CAP_DROPLESS, n_shared=1, bias_row0=0.0),
 }
 
 
@@ -74,7 +80,7 @@ def test_fused_matches_unfused(name):
         assert torch.equal(snap["y"], b["y"])
 
 
-@pytest.mark.parametrize("name", ["switch_top1", "gshard_top2", "wideep", "ds_k4_cf05"])
+@pytest.mark.parametrize("name", ["switch_top1", "gshard_top2", "wideep", "ds_k4_cf05", "wideep_2sm", "gshard_2sm"])
 def test_layer_small_unit_scale(name):
     shape = SMALL[name]
     inp = synth.make_inputs(shape, seed=3, device="cuda", scale="unit")
@@ -311,7 +317,8 @@ def test_pack_weight_layout(G, N, K):
     assert torch.equal(got.view(torch.int16), want.view(torch.int16))
 
 
-@pytest.mark.parametrize("name", ["switch_top1", "gshard_top2", "wideep", "ds_k4_cf05", "switch_relu_dropless_shared"])
+@pytest.mark.parametrize("name", ["switch_top1", "gshard_top2", "wideep", "ds_k4_cf05", "switch_relu_dropless_shared",
+                                  "wideep_2sm", "gshard_2sm", "relu_2sm_shared"])
 def test_packed_weights_bitwise(name):
     """Packed weights change only where the contractions read B from."""
     shape = SMALL[name]
@@ -326,3 +333,24 @@ def test_packed_weights_bitwise(name):
     if not a["fused_combine"]:
         assert torch.equal(snap["ybuf"][:used][live], b["ybuf"][:used][live])
     check_layer(shape, inp, b)
+
+
+@pytest.mark.slow
+def test_wideep_full_size_repeat_bitwise():
+    """Three calls of the full WideEP layer (its contractions run on SM pairs
+    over many tiles per pair) give bitwise the same rows and output, packed
+    weights or not: nothing in the pipeline depends on timing."""
+    shape = synth.WIDEEP_DROPLESS
+    inp = synth.make_inputs(shape, seed=0, device="cuda")
+    first = None
+    for i in range(3):
+        out = run_layer(shape, inp, keep_logits=False, packed=i == 1)
+        used = int(out["expert_offset"][-1])
+        live = out["row_token"][:used] >= 0
+        cur = (out["hbuf"][:used][live].clone(), out["ybuf"][:used][live].clone(), out["y"].clone())
+        if first is None:
+            first = cur
+        else:
+            for a, b, n in zip(first, cur, ("h", "ybuf", "y")):
+                assert torch.equal(a.view(torch.int16), b.view(torch.int16)), (i, n)
+        del out
