@@ -48,20 +48,28 @@ SETTABLE = {"score": int, "renorm": int, "z_coef": float, "random_second": int, 
             "cf_num": int, "cf_den": int}
 
 
-def launches_per_step(shape) -> int:
-    """Kernels one moe_layer_fwd call launches: router 3 for bf16 x (weight split,
-    logits GEMM, softmax/top-k) or 1 for fp32 x; slots 4 (aux loss folded in),
-    plus the per-expert select of the "probs" policy; dispatch 1 (0 when fused
-    into the first expert contraction: bf16 with T*k <= 256*E); expert FFN 2,
-    plus the pair-tile prefix when the contractions run on SM pairs (bf16 with
-    T*k > 256*E); combine 1 (0 when fused into the second: the fused case with
-    top-1 and no shared expert)."""
-    router = 3 if shape.dtype == 1 else 1
-    slots = 4 + (1 if shape.drop_policy == 1 and shape.cap_mode == 0 else 0)
-    fused = shape.dtype == 1 and shape.T * shape.k <= 256 * shape.E
+def router_launches(shape, packed_router: bool) -> int:
+    """bf16 x: the weight split (none with pre-split planes), the tensor-core
+    logits kernel (which also routes for E <= 256), and for wider E the routing
+    kernel; fp32 x: one FFMA router kernel."""
+    if shape.dtype != 1:
+        return 1
+    return (0 if packed_router else 1) + 1 + (0 if shape.E <= 256 else 1)
+
+
+def launches_per_step(shape, packed_router: bool = True) -> int:
+    """Kernels one moe_layer_fwd call launches: the router (router_launches);
+    slots 3 (count; scan, with the offsets and aux loss in its last CTA; rank),
+    plus the per-expert select of the "probs" policy; dispatch 1 (0 when fused into the first expert contraction: bf16
+    with T*k <= 256*E); expert FFN 2, plus the pair-tile prefix when the
+    contractions run on SM pairs (bf16 with T*k > 256*E); combine 1 (0 when
+    fused into the second: top-1 without a shared expert on the gather path)."""
+    router = router_launches(shape, packed_router)
+    slots = 3 + (1 if shape.drop_policy == 1 and shape.cap_mode == 0 else 0)
+    fused, fused_combine = fused_stages(shape)
     dispatch = 0 if fused else 1
     ffn = 2 + (1 if shape.dtype == 1 and not fused else 0)
-    combine = 0 if fused and shape.k == 1 and shape.n_shared == 0 else 1
+    combine = 0 if fused_combine else 1
     return router + slots + dispatch + ffn + combine
 
 
@@ -289,7 +297,9 @@ SIMT_STAGES = ("dispatch_bwd", "router_wgrad")
 # ------------------------------------------------------------------ algorithmic work
 def stage_work(shape, kept: int, experts_used: int):
     """Algorithmic bytes and flops of one launch of each kernel (padding rows and
-    unused capacity count as waste, not work)."""
+    unused capacity count as waste, not work).  Where the top-1 combine runs
+    inside the second contraction, that launch writes y (zero rows for dropped
+    tokens) instead of the routed rows."""
     b = 2 if shape.dtype == 1 else 4
     T, H, F, E, k = shape.T, shape.H, shape.F, shape.E, shape.k
     sh = shape.n_shared
@@ -297,12 +307,14 @@ def stage_work(shape, kept: int, experts_used: int):
     nm1 = 2 if shape.act == 2 else 1
     wexp = experts_used + sh
     add = T * E * 4 if shape.zipf_skew else 0
+    _, fused_combine = fused_stages(shape)
+    g2_out = T * H * b + T * k * 8 if fused_combine else rows * H * b
     return {
         "router": {"flops": 2.0 * T * H * E, "bytes": T * H * b + E * H * 4 + T * k * 8 + add},
         "dispatch": {"flops": 0.0, "bytes": T * H * b + kept * H * b + T * k * 8},
         "ffn_gemm1": {"flops": 2.0 * rows * H * F * nm1,
                       "bytes": wexp * nm1 * F * H * b + rows * H * b + rows * F * b},
-        "ffn_gemm2": {"flops": 2.0 * rows * F * H, "bytes": wexp * H * F * b + rows * F * b + rows * H * b},
+        "ffn_gemm2": {"flops": 2.0 * rows * F * H, "bytes": wexp * H * F * b + rows * F * b + g2_out},
         "combine": {"flops": 0.0, "bytes": kept * H * b + sh * T * H * b + T * H * b + T * k * 12},
     }
 
@@ -338,15 +350,16 @@ def roofline(stage: str, work: dict, ms: float, peaks: dict, workload: str, bf16
 
 def train_launches_per_step(shape) -> int:
     """Kernels of one training step: the forward with MOE_FLAG_TRAINING (always
-    unfused, plus the zeroing of xbuf's padding rows), then moe_layer_bwd:
+    unfused, plus the zeroing of xbuf's padding rows; the router weight is
+    split on each call, since the backward takes it in fp32), then moe_layer_bwd:
     combine backward and the zeroing of dyrow's padding rows, five expert
     contractions (four when T*k <= 256*E or H <= 512: dh and dz in one; with
     T*k > 256*E the forward contractions run on SM pairs after a pair-tile
     prefix kernel), the router
     backward (the aux coefficients, then dlogits), the dispatch backward and
     dWg (partial sums, then their reduction)."""
-    router = 3 if shape.dtype == 1 else 1
-    slots = 4 + (1 if shape.drop_policy == 1 and shape.cap_mode == 0 else 0)
+    router = router_launches(shape, packed_router=False)
+    slots = 3 + (1 if shape.drop_policy == 1 and shape.cap_mode == 0 else 0)
     pairs = 1 if shape.T * shape.k > 256 * shape.E else 0        # pair-tile prefix of the SM-pair GEMMs
     fwd = router + slots + 1 + 1 + 2 + pairs + 1
     fused = shape.T * shape.k <= 256 * shape.E or shape.H <= 512    # dh and dz in one kernel
@@ -592,7 +605,9 @@ class LayerRun:
         self.B, self.shape, self.stream = B, shape, stream
         self.inp = synth.make_inputs(shape, seed=seed, device="cuda")
         self.packed = packed and shape.dtype == 1
-        self.cfg = B.make_cfg(shape, flags=B.MOE_FLAG_PACKED_WEIGHTS if self.packed else 0)
+        # expert weights and the router weight's bf16 planes prepared once
+        self.cfg = B.make_cfg(shape, flags=(B.MOE_FLAG_PACKED_WEIGHTS | B.MOE_FLAG_PACKED_ROUTER) if self.packed
+                              else 0)
         self.ws = B.alloc_workspace(self.cfg)
         self.edt = self.inp["x"].dtype
         self.y = torch.empty((shape.T, shape.H), dtype=self.edt, device=dev)
@@ -600,6 +615,7 @@ class LayerRun:
         # expert weights packed once into 16 KB TMA blocks (weight preprocessing,
         # outside every timed region), as a serving engine stores them
         wsrc = B.pack_weights(self.inp) if self.packed else self.inp
+        self.wg = B.pack_router(self.inp["wg"]) if self.packed else self.inp["wg"]
         torch.cuda.synchronize()
         self.wts = B.make_weights(wsrc)
         self._wsrc = wsrc
@@ -617,7 +633,7 @@ class LayerRun:
 
     def call(self, events=None):
         i = self.inp
-        self.B.moe_layer_fwd(self.cfg, i["x"], i["wg"], i["logit_add"], i["uniform"], self.wts, self.y, self.aux,
+        self.B.moe_layer_fwd(self.cfg, i["x"], self.wg, i["logit_add"], i["uniform"], self.wts, self.y, self.aux,
                              None, self.ws, stage_events=events, stream=self.stream)
 
     def check_status(self, when):
@@ -665,7 +681,10 @@ class LayerRun:
 
 
 def fused_stages(shape):
-    """(dispatch fused into GEMM1, combine fused into GEMM2) for this layer."""
+    """(dispatch fused into GEMM1, combine fused into GEMM2) for this layer: bf16
+    layers with T*k <= 256*E gather x inside GEMM1 and, top-1 without a shared
+    expert, scatter gate * row inside GEMM2; larger bf16 layers run their
+    contractions on SM pairs between the dispatch and combine kernels."""
     fused = shape.dtype == 1 and shape.T * shape.k <= 256 * shape.E
     return fused, fused and shape.k == 1 and shape.n_shared == 0
 
@@ -824,7 +843,7 @@ def run_ours(args, world, rank, local):
         b["loaded"].record(s_in)
         stream.wait_event(b["loaded"])
         stream.wait_event(b["drained"])     # this y buffer has been read back
-        B.moe_layer_fwd(cfg, b["x"], inp["wg"], b["add"], b["uni"], wts, b["y"], b["aux"], None, ws, stream=stream)
+        B.moe_layer_fwd(cfg, b["x"], run.wg, b["add"], b["uni"], wts, b["y"], b["aux"], None, ws, stream=stream)
         b["computed"].record(stream)
         s_out.wait_event(b["computed"])
         with torch.cuda.stream(s_out):
@@ -868,7 +887,8 @@ def run_ours(args, world, rank, local):
                        "capacity": C, "kept_assignments": kept, "rows_used": rows_used,
                        "l2": "flushed before every step (320 MiB write + 320 MiB read, outside the timed events)",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "weights": "packed once before timing (moe_pack_weight)" if packed else "linear-layer layout"},
+                       "weights": "packed once before timing (moe_pack_weight, moe_pack_router_weight)" if packed
+                       else "linear-layer layout, router weight split on every call"},
             "stages_ms": stage_ms,
             "stages_note": f"second timed pass of {n_stage_steps} steps with per-stage events "
                            f"({stage_sum_ms:.4f} ms per step including the events' own cost)",
@@ -883,7 +903,7 @@ def run_ours(args, world, rank, local):
             "dominant_kernel": dom,
             "e2e": {"value": job_tokens_per_s(T, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "pipelining": "2 buffer sets; copy-in, layer, copy-out streams"},
-            "gpu_launches": launches_per_step(shape) * args.steps,
+            "gpu_launches": launches_per_step(shape, packed) * args.steps,
             "clocks": clocks,
             "cpu_baseline": cpu,
             "other_workloads": others,

@@ -669,7 +669,8 @@ static cudaError_t launch_kernel(KParams& k, int64_t max_tiles, cudaStream_t str
 cudaError_t launch_grouped_gemm(const GemmParams& p, cudaStream_t stream) {
   using namespace gg;
   if (p.rows_max == 0) return cudaSuccess;
-  if (p.two_sm && grouped_gemm_2sm_supported(p)) return launch_grouped_gemm_2sm(p, stream);
+  if (p.two_sm && p.gather_src == nullptr && p.scatter_dst == nullptr && p.pair_prefix != nullptr)
+    return launch_grouped_gemm_tn(p, stream);
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
   const int box_n = 128;
   KParams k{};

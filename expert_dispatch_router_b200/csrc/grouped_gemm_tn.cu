@@ -1,0 +1,530 @@
+// Grouped GEMM with the tokens on the MMA's N side, on pairs of SMs
+// (tcgen05.mma.cta_group::2), for the expert contractions of compute-bound
+// layers.
+//
+// Method: the per-expert FFN of an MoE layer ("Expert-parallel MoE training"
+// explainer: experts as grouped MLPs, SwiGLU experts with gate / up / down
+// matrices in worked example 2; MegaBlocks' dropless layout with every expert
+// batch padded to a multiple of 128 rows).  For every group g and its rows,
+//     D[rows, features] = epi( X_g[rows, :] * W_g[features, :]^T ),
+// bf16 operands, fp32 accumulation in tensor memory, bf16 output.
+//
+// Why tokens on N: with the rows of a group on the MMA's M side, every group
+// is computed in whole 128-row blocks (256 on a pair of SMs), and a group's
+// padding rows cost as much as its tokens: 23% extra work on the WideEP layer
+// (skewed loads over 256 experts).  Here the MMA computes D^T = W_g * X_g^T:
+// M = 256 output features (128 per SM of the pair), N = the group's next
+// tokens, at most 256 and rounded up to 16, so a group costs its token count
+// rounded up to 16.  The buffers keep the 128-row-padded layout; only the
+// computation skips the padding.
+//
+// Per pair tile (group g, token tile j, feature tile f):
+//   tokens r0 = off[g] + 256 j .. r0 + N, N = round_up(min(256, valid_g - 256 j), 16);
+//   the even CTA computes features 256 f .. +128, the odd CTA the next 128.
+// Each CTA loads its 128 weight rows (A, 16 KB per 64-k step) and half of the
+// token rows (B: rows r0 + rank * N/2, a 128-row box of which the MMA reads
+// N/2); one MMA instruction issued by the even CTA reads both CTAs' shared
+// memory.  SwiGLU: two MMAs per k step, gate and up rows of the same features
+// (A 32 KB per step), into two accumulators, so a thread holds gate and up of
+// its feature; plain: double-buffered accumulators.
+//
+// Roles per CTA (576 threads): warp 0 issues the TMA loads (both CTAs; each
+// copy completes on the even CTA's full barrier, armed by the even CTA with
+// both CTAs' bytes); warp 1 of the even CTA issues the MMAs and commits with a
+// multicast to both CTAs' barriers; warps 2-17 read the accumulator (lane =
+// feature, columns = tokens), apply the activation, transpose 32 x 32 tiles
+// through shared memory and store them by TMA.
+//
+// No load in this file uses cluster multicast.  Every wait is bounded: on
+// expiry the CTA records MOE_ETIMEOUT, raises both CTAs' abort flags, and the
+// pair drains what it issued and frees TMEM.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "pair_common.cuh"
+#include "tc_common.cuh"
+
+namespace moe {
+namespace gtn {
+
+using namespace tcx;
+using namespace pairx;
+
+constexpr int BK = 64;
+constexpr int FT = 256;                         // output features per pair tile
+constexpr int TT = 256;                         // tokens per pair tile at most
+constexpr int HALF = 128;                       // rows of one CTA's A (and of its B box)
+constexpr int A_BYTES = HALF * BK * 2;          // 16 KB
+constexpr int B_BYTES = HALF * BK * 2;          // 16 KB
+constexpr int RING_BYTES = 192 * 1024;
+constexpr int MAX_STAGES = 6;
+constexpr int EPI_WARPS = 16;
+constexpr int THREADS = 64 + EPI_WARPS * 32;
+constexpr int TMEM_COLS = 512;
+constexpr int STAGE_OUT_BYTES = 32 * 32 * 2;
+constexpr int STAGING_BYTES = EPI_WARPS * STAGE_OUT_BYTES;
+constexpr int SMEM_BYTES = RING_BYTES + STAGING_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+
+struct KParams {
+  CUtensorMap tmA, tmA1, tmSA, tmSA1;   // weights [G, N_out, K] (SwiGLU: gate, up); the shared expert's
+  CUtensorMap tmB, tmBs;                // token rows [rows_max, K]; the shared block's rows from x [T, K]
+  CUtensorMap tmD;                      // bf16 output [rows_max, N_out], box 32 x 32, 64-byte swizzle
+  const int32_t* off;                   // [ngroups + 1] row offsets (multiples of 128)
+  const int32_t* tp;                    // [ngroups + 1] exclusive prefix of the groups' token tiles
+  const int32_t* valid;                 // [E] rows of each routed group (kept counts), or null: whole blocks
+  DevStatus* status;
+  int64_t rows_max, T;
+  int K, N_out, E, n_shared, epi;
+  int as_sep;                           // 1: the shared block's token rows come from tmBs (row - off[E])
+  int b_packed;                         // 1: weight maps are 5-D over packed blocks
+};
+
+// Rows of group g that carry tokens: the routed groups' kept counts, the
+// shared block's T, clipped to the group's rows (<= rows_max).
+__device__ __forceinline__ int64_t group_rows(const int32_t* off, const int32_t* valid, int g, int E, int64_t T,
+                                              int64_t rows_max) {
+  const int64_t b = min((int64_t)off[g], rows_max), e = min((int64_t)off[g + 1], rows_max);
+  const int64_t pad = e > b ? e - b : 0;
+  const int64_t v = g == E ? T : (valid != nullptr ? (int64_t)valid[g] : pad);
+  return v < pad ? (v > 0 ? v : 0) : pad;
+}
+
+struct Tile {
+  int g;           // group
+  int ft;          // feature tile
+  int n;           // MMA N: tokens of the tile rounded up to 16
+  int64_t r0;      // first row of the tile
+};
+__device__ __forceinline__ Tile decode(const KParams& p, int ngroups, int nf, int64_t tile) {
+  Tile t;
+  const int64_t tt = tile / nf;
+  t.ft = (int)(tile - tt * nf);
+  int lo = 0, hi = ngroups - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(p.tp + mid) <= tt) lo = mid; else hi = mid - 1;
+  }
+  t.g = lo;
+  const int64_t j = tt - __ldg(p.tp + lo);
+  t.r0 = min((int64_t)__ldg(p.off + lo), p.rows_max) + j * TT;
+  const int64_t v = group_rows(p.off, p.valid, lo, p.E, p.T, p.rows_max) - j * TT;
+  const int64_t nv = v < TT ? v : TT;
+  t.n = (int)((nv + 15) / 16 * 16);
+  return t;
+}
+
+__global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tn_kernel(const __grid_constant__ KParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stage_base = smem;
+  uint8_t* staging = smem + RING_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + RING_BYTES + STAGING_BYTES);
+  // bars: full[MAX_STAGES], empty[MAX_STAGES], tfull[2], tempty[2], drain
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + MAX_STAGES);
+  const uint32_t tfull0 = smem_u32(bars + 2 * MAX_STAGES), tempty0 = smem_u32(bars + 2 * MAX_STAGES + 2);
+  const uint32_t drain = smem_u32(bars + 2 * MAX_STAGES + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * MAX_STAGES + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const bool swiglu = p.epi == MOE_ACT_SWIGLU;
+  const int ngroups = p.E + (p.n_shared ? 1 : 0);
+  const int stage_bytes = (swiglu ? 2 : 1) * A_BYTES + B_BYTES;
+  const int n_stages = min(MAX_STAGES, RING_BYTES / stage_bytes);
+  const int n_acc = swiglu ? 1 : 2;              // SwiGLU: gate | up fill all 512 columns
+  auto abort_pair = [&](int info) {
+    *abort_flag = 1;
+    st_cluster_u32(map_to(smem_u32((const void*)abort_flag), rank ^ 1u), 1u);
+    set_status(p.status, MOE_ETIMEOUT, info);
+  };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < MAX_STAGES; ++s) { mbar_init(full0 + 8 * s, 1); mbar_init(empty0 + 8 * s, 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(tfull0 + 8 * b, 1); mbar_init(tempty0 + 8 * b, 2 * EPI_WARPS); }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    prefetch_map(&p.tmA); prefetch_map(&p.tmB); prefetch_map(&p.tmD);
+    if (swiglu) prefetch_map(&p.tmA1);
+    if (p.n_shared) { prefetch_map(&p.tmSA); prefetch_map(&p.tmBs); if (swiglu) prefetch_map(&p.tmSA1); }
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(smem_u32(tmem_slot)), "r"(TMEM_COLS) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  // the pair's MMA writes both CTAs' accumulators at the even CTA's columns
+  const bool tmem_same = ld_cluster_u32(map_to(smem_u32(tmem_slot), rank ^ 1u)) == tmem_base;
+  pdl_wait();
+  if (!tmem_same && threadIdx.x == 0) set_status(p.status, MOE_EDEVICE, 31);
+
+  const int nf = (p.N_out + FT - 1) / FT;                      // feature tiles
+  const int64_t n_tok_tiles = tmem_same ? __ldg(p.tp + ngroups) : 0;
+  const int64_t n_tiles = n_tok_tiles * nf;
+  const int nk = (p.K + BK - 1) / BK;
+  const int64_t cid = cluster_id(), ncl = cluster_count();
+
+  if (warp == 0) {
+    // ---------------- TMA producer (both CTAs)
+    if (lane == 0) {
+      const uint32_t full_leader0 = map_to(full0, 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t fills[MAX_STAGES] = {0, 0, 0, 0, 0, 0};
+      bool ok = true;
+      const uint32_t tx = 2u * (uint32_t)stage_bytes;          // both CTAs load whole boxes
+      for (int64_t tile = cid; tile < n_tiles && ok; tile += ncl) {
+        const Tile t = decode(p, ngroups, nf, tile);
+        const bool sh = t.g == p.E;
+        const bool sep = sh && p.as_sep;
+        const CUtensorMap* ma = sh ? &p.tmSA : &p.tmA;
+        const CUtensorMap* ma1 = sh ? &p.tmSA1 : &p.tmA1;
+        const CUtensorMap* mb = sep ? &p.tmBs : &p.tmB;
+        const int z = sh ? 0 : t.g;
+        const int wrow = t.ft * FT + (int)rank * HALF;          // this CTA's weight rows
+        const int64_t brow64 = (sep ? t.r0 - __ldg(p.off + p.E) : t.r0) + (int64_t)rank * (t.n / 2);
+        const int brow = (int)brow64;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait_cl(empty0 + 8 * stage, phase ^ 1u, abort_flag)) { ok = false; break; }
+          const uint32_t sa = smem_u32(stage_base + stage * stage_bytes);
+          const uint32_t sb = sa + (swiglu ? 2 : 1) * A_BYTES;
+          const uint32_t fb = full_leader0 + 8 * stage;
+          if (leader) mbar_expect_tx(full0 + 8 * stage, tx);
+          if (p.b_packed) {
+            tma2_load_5d(sa, ma, kb, wrow / 128, z, fb);
+            if (swiglu) tma2_load_5d(sa + A_BYTES, ma1, kb, wrow / 128, z, fb);
+          } else {
+            tma2_load_3d(sa, ma, kb * BK, wrow, z, fb);
+            if (swiglu) tma2_load_3d(sa + A_BYTES, ma1, kb * BK, wrow, z, fb);
+          }
+          tma2_load_2d(sb, mb, kb * BK, brow, fb);
+          fills[stage]++;
+          if (++stage == n_stages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) abort_pair(40);
+      for (int s = 0; s < n_stages; ++s)
+        if (fills[s]) {
+          if (leader) mbar_drain_cl(full0 + 8 * s, (fills[s] - 1) & 1u);
+          else mbar_drain_cl(empty0 + 8 * s, (fills[s] - 1) & 1u);
+        }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (even CTA)
+    if (leader && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int64_t tile = cid; tile < n_tiles && ok; tile += ncl) {
+        const Tile t = decode(p, ngroups, nf, tile);
+        const uint32_t idesc = make_idesc(t.n, 2 * HALF);
+        if (!mbar_wait_cl(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + (uint32_t)(acc * 256);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait_cl(full0 + 8 * stage, phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(stage_base + stage * stage_bytes);
+          const uint64_t bd = sw128_desc(sa + (swiglu ? 2 : 1) * A_BYTES);
+          const uint64_t ad = sw128_desc(sa);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)               // 16 elements = 32 bytes along K
+            umma2(d0, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
+          if (swiglu) {
+            const uint64_t ud = sw128_desc(sa + A_BYTES);
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+              umma2(d0 + 256, ud + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          umma2_commit_both(empty0 + 8 * stage);
+          if (++stage == n_stages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma2_commit_both(tfull0 + 8 * acc);
+        if (++acc == n_acc) { acc = 0; acc_phase ^= 1u; }
+      }
+      if (!ok) abort_pair(41);
+      umma2_commit_both(drain);
+    }
+    if (lane == 0) mbar_drain_cl(drain, 0);
+  } else {
+    // ---------------- epilogue (both CTAs)
+    const int ew = warp - 2;
+    const int sub = warp & 3;                   // TMEM sub-partition: features 32 sub .. +32 of this CTA
+    const int quarter = ew >> 2;                // token columns quarter * 32, + 128
+    const uint32_t stage_out = smem_u32(staging + ew * STAGE_OUT_BYTES);
+    const uint32_t tempty_leader0 = map_to(tempty0, 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int64_t tile = cid; tile < n_tiles; tile += ncl) {
+      // lane = feature f0 + lane, columns = the tile's tokens
+      const Tile t = decode(p, ngroups, nf, tile);           // before the wait: off its critical path
+      if (!mbar_wait_cl(tfull0 + 8 * acc, acc_phase, abort_flag)) {
+        if (lane == 0) abort_pair(42);
+        break;
+      }
+      tc_fence_after();
+      const int f0 = t.ft * FT + (int)rank * HALF + sub * 32;
+      const uint32_t tbase = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * 256);
+      if (f0 < p.N_out) {
+        for (int c = quarter * 32; c < t.n; c += 4 * 32) {
+          __syncwarp();
+          float v[32];
+          tmem_ld(tbase + (uint32_t)c, v, 32);
+          if (swiglu) {
+            float u[32];
+            tmem_ld(tbase + 256u + (uint32_t)c, u, 32);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = act_silu(v[i]) * u[i];
+          } else {
+            tmem_wait_ld();
+            if (p.epi == MOE_ACT_RELU) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[i] = act_relu(v[i]);
+            } else if (p.epi == MOE_ACT_GELU) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[i] = act_gelu(v[i]);
+            }
+          }
+          // transpose through the staging buffer: token j's 32 features form a
+          // 64-byte row (16-byte chunk q of row j at q ^ ((j >> 1) & 3): the TMA
+          // 64-byte swizzle); this lane writes its feature's element of every row
+          if (lane == 0) bulk_wait_read0();
+          __syncwarp();
+          const uint32_t col_b = (uint32_t)((lane & 7) * 2);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const __nv_bfloat16 h = __float2bfloat16_rn(v[j]);
+            const uint32_t addr = stage_out + (uint32_t)(j * 64) + ((((uint32_t)lane >> 3) ^ (((uint32_t)j >> 1) & 3u)) << 4) + col_b;
+            asm volatile("st.shared.b16 [%0], %1;" :: "r"(addr), "h"(*reinterpret_cast<const uint16_t*>(&h)) : "memory");
+          }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            // rows past the tile's tokens lie in the group's padding: harmless
+            tma_store_2d(&p.tmD, stage_out, f0, (int)(t.r0 + c));
+            bulk_commit();
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8 * acc);
+      if (++acc == n_acc) { acc = 0; acc_phase ^= 1u; }
+    }
+    if (lane == 0) bulk_wait0();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  tc_fence_after();
+  pdl_trigger();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" :: "r"(tmem_base), "r"(TMEM_COLS) : "memory");
+  }
+}
+
+// One warp: tp[g] = sum over g' < g of ceil(rows(g') / 256) token tiles, rows
+// as in group_rows; tp[ngroups] = the total.
+__global__ void token_tile_prefix_kernel(const int32_t* off, const int32_t* valid, int ngroups, int E, int64_t T,
+                                         int64_t rows_max, int32_t* tp) {
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x;
+  const int seg = (ngroups + 31) / 32;
+  const int g0 = min(ngroups, lane * seg), g1 = min(ngroups, g0 + seg);
+  auto tiles = [&](int g) { return (int)((group_rows(off, valid, g, E, T, rows_max) + TT - 1) / TT); };
+  int s = 0;
+  for (int g = g0; g < g1; ++g) s += tiles(g);
+  int incl = s;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  int run = incl - s;
+  for (int g = g0; g < g1; ++g) {
+    tp[g] = run;
+    run += tiles(g);
+  }
+  if (lane == 31) tp[ngroups] = incl;
+}
+
+// 2-D map over a row-major bf16 matrix [rows, K], box 64 x 128.
+static bool map_rows(CUtensorMap* m, const void* base, int64_t rows, int K) {
+  MapKey key;
+  memset(&key, 0, sizeof(key));
+  key.base = base;
+  key.rank = 2;
+  key.swizzle = CU_TENSOR_MAP_SWIZZLE_128B;
+  key.dims[0] = (cuuint64_t)K;
+  key.dims[1] = (cuuint64_t)rows;
+  key.strides[0] = (cuuint64_t)K * 2;
+  key.box[0] = BK;
+  key.box[1] = HALF;
+  return encode_cached(m, key);
+}
+
+// 3-D map over stacked weights [G, N, K], box 64 x 128 x 1 (rows past N read as zero).
+static bool map_weights(CUtensorMap* m, const void* base, int G, int N, int K) {
+  MapKey key;
+  memset(&key, 0, sizeof(key));
+  key.base = base;
+  key.rank = 3;
+  key.swizzle = CU_TENSOR_MAP_SWIZZLE_128B;
+  key.dims[0] = (cuuint64_t)K;
+  key.dims[1] = (cuuint64_t)N;
+  key.dims[2] = (cuuint64_t)G;
+  key.strides[0] = (cuuint64_t)K * 2;
+  key.strides[1] = (cuuint64_t)N * K * 2;
+  key.box[0] = BK;
+  key.box[1] = HALF;
+  key.box[2] = 1;
+  return encode_cached(m, key);
+}
+
+// 5-D map over packed weights [G][N/128][K/64][128][64]: one box = one 16 KB block.
+static bool map_packed(CUtensorMap* m, const void* base, int G, int N, int K) {
+  const cuuint64_t kb = (cuuint64_t)((K + BK - 1) / BK), nb = (cuuint64_t)((N + 127) / 128);
+  MapKey key;
+  memset(&key, 0, sizeof(key));
+  key.base = base;
+  key.rank = 5;
+  key.swizzle = CU_TENSOR_MAP_SWIZZLE_128B;
+  key.dims[0] = BK;
+  key.dims[1] = 128;
+  key.dims[2] = kb;
+  key.dims[3] = nb;
+  key.dims[4] = (cuuint64_t)G;
+  key.strides[0] = BK * 2;
+  key.strides[1] = (cuuint64_t)BK * 128 * 2;
+  key.strides[2] = key.strides[1] * kb;
+  key.strides[3] = key.strides[2] * nb;
+  key.box[0] = BK;
+  key.box[1] = 128;
+  key.box[2] = key.box[3] = key.box[4] = 1;
+  return encode_cached(m, key);
+}
+
+// 2-D map over a bf16 output [rows, N], box 32 x 32, 64-byte swizzle (TMA store).
+static bool map_out(CUtensorMap* m, const void* base, int64_t rows, int N) {
+  MapKey key;
+  memset(&key, 0, sizeof(key));
+  key.base = base;
+  key.rank = 2;
+  key.swizzle = CU_TENSOR_MAP_SWIZZLE_64B;
+  key.dims[0] = (cuuint64_t)N;
+  key.dims[1] = (cuuint64_t)rows;
+  key.strides[0] = (cuuint64_t)N * 2;
+  key.box[0] = 32;
+  key.box[1] = 32;
+  return encode_cached(m, key);
+}
+
+static int resident_pairs() {
+  static int cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int& c = cache[dev & 63];
+  if (c == 0) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(2 * sm_count());
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_tn_kernel, &cfg) != cudaSuccess || n < 1) {
+      cudaGetLastError();
+      n = sm_count() / 2;
+    }
+    c = n;
+  }
+  return c;
+}
+
+}  // namespace gtn
+
+cudaError_t launch_grouped_gemm_tn(const GemmParams& p, cudaStream_t stream) {
+  using namespace gtn;
+  if (p.rows_max == 0) return cudaSuccess;
+  if (encode_fn() == nullptr) return cudaErrorNotSupported;
+  KParams k{};
+  const void* b1 = p.b1 ? p.b1 : p.b0;
+  const void* s0 = p.sb0 ? p.sb0 : p.b0;
+  const void* s1 = p.sb1 ? p.sb1 : s0;
+  bool ok = true;
+  if (p.b_packed) {
+    ok = ok && map_packed(&k.tmA, p.b0, p.E, p.Nw, p.K);
+    ok = ok && map_packed(&k.tmA1, b1, p.E, p.Nw, p.K);
+    ok = ok && map_packed(&k.tmSA, s0, 1, p.Nw, p.K);
+    ok = ok && map_packed(&k.tmSA1, s1, 1, p.Nw, p.K);
+  } else {
+    ok = ok && map_weights(&k.tmA, p.b0, p.E, p.Nw, p.K);
+    ok = ok && map_weights(&k.tmA1, b1, p.E, p.Nw, p.K);
+    ok = ok && map_weights(&k.tmSA, s0, 1, p.Nw, p.K);
+    ok = ok && map_weights(&k.tmSA1, s1, 1, p.Nw, p.K);
+  }
+  ok = ok && map_rows(&k.tmB, p.a_routed, p.rows_max, p.K);
+  ok = ok && map_rows(&k.tmBs, p.a_shared ? p.a_shared : p.a_routed, p.a_shared ? p.T : p.rows_max, p.K);
+  ok = ok && map_out(&k.tmD, p.d, p.rows_max, p.Nw);
+  if (!ok) return cudaErrorInvalidValue;
+  const int ngroups = p.E + (p.n_shared ? 1 : 0);
+  if (p.pair_prefix_ready == 0)
+    launch_pdl(token_tile_prefix_kernel, 1, 32, 0, stream, p.expert_offset, p.valid_rows, ngroups, p.E, p.T,
+               p.rows_max, p.pair_prefix);
+  k.off = p.expert_offset;
+  k.tp = p.pair_prefix;
+  k.valid = p.valid_rows;
+  k.status = p.status;
+  k.rows_max = p.rows_max;
+  k.T = p.T;
+  k.K = p.K;
+  k.N_out = p.Nw;
+  k.E = p.E;
+  k.n_shared = p.n_shared;
+  k.epi = p.epi;
+  k.as_sep = p.a_shared != nullptr;
+  k.b_packed = p.b_packed;
+  cudaError_t e = ensure_smem(grouped_gemm_tn_kernel, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(2 * resident_pairs());
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  e = cudaLaunchKernelEx(&cfg, grouped_gemm_tn_kernel, k);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -124,6 +124,7 @@ struct SlotParams {
   int32_t* cum;             // [E] exclusive prefix of expert_count
   uint32_t* list_key;       // [T*k] order-preserving gate keys
   uint32_t* list_idx;       // [T*k] the assignment's flat index t*k + r
+  unsigned* ticket;         // zero between calls: counts the count kernel's finished CTAs
 };
 constexpr int kSlotChunk = 256;    // assignments per CTA of the slot kernels (one per thread)
 cudaError_t launch_slots(const SlotParams& p, cudaStream_t stream);
@@ -181,18 +182,20 @@ struct GemmParams {
   const float* scatter_gate;
   const int32_t* scatter_slot;
   int b_packed;             // 1: b0/b1/sb0/sb1 are packed (launch_pack_weight)
-  // Pairs of SMs (tcgen05 cta_group::2, 256 x 256 tiles) instead of one SM per
-  // 128 x 256 tile: for compute-bound layers, without gather or scatter.
-  // pair_prefix: ngroups + 1 ints of scratch for the groups' pair-tile prefix,
-  // computed by this launch unless pair_prefix_ready (same expert_offset as the
-  // launch that computed it).
+  // Pairs of SMs (tcgen05 cta_group::2, 256 output features x up to 256
+  // tokens, tokens on the MMA's N) instead of one SM per 128 x 256 tile: for
+  // compute-bound layers, without gather or scatter.  pair_prefix: ngroups + 1
+  // ints of scratch for the groups' token-tile prefix, computed by this launch
+  // unless pair_prefix_ready (same offsets and valid_rows as the launch that
+  // computed it).  valid_rows: rows of each routed group that carry tokens
+  // (kept counts, [E]), or null: whole 128-row blocks; the shared block has T.
   int two_sm;
   int32_t* pair_prefix;
   int pair_prefix_ready;
+  const int32_t* valid_rows;
 };
 cudaError_t launch_grouped_gemm(const GemmParams& p, cudaStream_t stream);
-bool grouped_gemm_2sm_supported(const GemmParams& p);
-cudaError_t launch_grouped_gemm_2sm(const GemmParams& p, cudaStream_t stream);
+cudaError_t launch_grouped_gemm_tn(const GemmParams& p, cudaStream_t stream);
 
 // Grouped GEMMs of the backward pass (grouped_gemm_bwd.cu).
 //   dgrad: out[rows, N] = a[rows, K] * B, B the weights [G, K0, N] read along N

@@ -15,8 +15,8 @@ namespace {
 constexpr int64_t kMaxCf = int64_t(1) << 20;
 
 struct Layout {
-  size_t status, psum, cnt, zsum, term, chunk, cum, lkey, lidx, ids, gates, slot, ecount, kept, off, pairs, rowtok, logits, lparts,
-      planes, xbuf,
+  size_t status, psum, cnt, zsum, term, chunk, cum, lkey, lidx, ids, gates, slot, ecount, kept, off, pairs, rowtok,
+      logits, lparts, planes, xbuf,
       hbuf, ybuf, dyrow, dh, dz, dxrow, dgate, dlog, fcoef, dwgp;
   size_t total;
   int nblk_router, nchunk;
@@ -100,7 +100,7 @@ Layout layout_of(const moe_cfg* c) {
   L.psum = take(sizeof(float) * L.nblk_router * E);
   L.cnt = take(sizeof(int32_t) * L.nblk_router * E);
   L.zsum = take(sizeof(float) * L.nblk_router);
-  L.term = take(sizeof(double) * (E + 1));      // E terms + the aux ticket counter
+  L.term = take(sizeof(double) * (E + 2));      // E terms, the aux ticket counter, the slot ticket
   L.chunk = take(sizeof(int32_t) * E * (size_t)L.nchunk);
   const bool probs = drop_probs(c);
   L.cum = take(probs ? sizeof(int32_t) * E : 0);
@@ -210,6 +210,7 @@ int run_slots(const moe_cfg* c, const Layout& L, const int32_t* ids, const float
   p.expert_offset = off;
   p.row_token = rowtok;
   p.chunk_cnt = at<int32_t>(ws, L.chunk);
+  p.ticket = reinterpret_cast<unsigned*>(at<double>(ws, L.term) + c->E + 1);
   p.T = c->T;
   p.E = c->E;
   p.k = c->k;
@@ -257,11 +258,13 @@ bool two_sm_ffn(const moe_cfg* c) {
 // Both contractions of the expert FFN; `ev_mid`, if non-NULL, is recorded between them.
 // bf16 only: with `rowtok`, GEMM1 gathers its routed A rows from x (fused
 // dispatch; xbuf unused); with `y_top1` as well, GEMM2 writes gate * row to
-// y[token] (fused top-1 combine; ybuf's routed rows are not written).
+// y[token] (fused top-1 combine; ybuf's routed rows are not written).  `kept`
+// (optional): the routed groups' kept counts, so the SM-pair contractions skip
+// the padding rows.
 int run_ffn(const moe_cfg* c, const Layout& L, const void* xbuf, const void* x, const int32_t* off,
             const moe_weights* w, void* ybuf, void* ws, cudaStream_t s, const moe_event_t* ev_mid = nullptr,
             const int32_t* rowtok = nullptr, void* y_top1 = nullptr, const float* gates_top1 = nullptr,
-            const int32_t* slot_top1 = nullptr) {
+            const int32_t* slot_top1 = nullptr, const int32_t* kept = nullptr) {
   void* hbuf = at<void>(ws, L.hbuf);
   const bool sh = c->n_shared != 0;
   if (c->dtype == MOE_DTYPE_BF16) {
@@ -286,6 +289,7 @@ int run_ffn(const moe_cfg* c, const Layout& L, const void* xbuf, const void* x, 
     g1.two_sm = two_sm_ffn(c) ? 1 : 0;
     g1.pair_prefix = at<int32_t>(ws, L.pairs);
     g1.pair_prefix_ready = 0;
+    g1.valid_rows = kept;
     if (rowtok != nullptr) {
       g1.a_routed = nullptr;
       g1.gather_src = x;
@@ -554,7 +558,7 @@ int moe_layer_fwd(const moe_cfg* cfg, const void* x, const float* wg, const floa
   if ((st = record(stage_events, 3, s)) != MOE_OK) return st;
   if ((st = run_ffn(cfg, L, xbuf, x, off, w, ybuf, ws, s, stage_events ? stage_events + 4 : nullptr,
                     fuse ? rowtok : nullptr, fuse_combine ? y : nullptr, fuse_combine ? gates : nullptr,
-                    fuse_combine ? slot : nullptr)) != MOE_OK)
+                    fuse_combine ? slot : nullptr, at<int32_t>(ws, L.kept))) != MOE_OK)
     return st;
   if ((st = record(stage_events, 5, s)) != MOE_OK) return st;
   pp.src = ybuf;

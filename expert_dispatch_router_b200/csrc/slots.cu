@@ -7,14 +7,16 @@
 //
 // The assignment sequence is a = r*T + t (every first choice in token order,
 // then every second choice, ...).  slot(a) = number of earlier assignments of
-// the same expert.  Four small kernels, all deterministic:
+// the same expert.  Three small kernels, all deterministic:
 //   1. count   : CTA c counts its 256-assignment chunk (kSlotChunk) per expert
 //                (shared-memory histogram) -> chunk_cnt[e][c].
 //   2. scan    : CTA e scans chunk_cnt[e][*] -> chunk base offsets, the expert's
-//                pre-drop count and kept count.
-//   3. offsets : one CTA: exclusive scan of the 128-padded kept counts -> the
-//                per-expert row blocks, then the padding / shared rows of row_token.
-//   4. rank    : CTA c re-reads its chunk; warps rank equal experts inside each
+//                pre-drop count and kept count, and its aux-loss term.  The CTA
+//                that finishes last (an atomic ticket; no CTA waits for another)
+//                scans the 128-padded kept counts into the per-expert row
+//                blocks, sums the aux loss (and z-loss) and writes row_token's
+//                padding and shared rows, then resets the ticket.
+//   3. rank    : CTA c re-reads its chunk; warps rank equal experts inside each
 //                32-assignment step with match_any, carry per-warp running counts,
 //                prefix them over the warps in order, and add the chunk base.
 // Total metadata traffic is O(T*k + E*chunks); nothing scales with C.
@@ -90,6 +92,93 @@ __device__ __forceinline__ int block_scan_excl(int v, int* sh, int& total) {
   return excl;
 }
 
+// Row blocks (exclusive scan of the 128-padded kept counts; the shared block
+// last), the "probs" lists' starts, the aux-loss and z-loss totals, and
+// row_token's padding and shared rows.  Run by one CTA of kSlotThreads threads.
+__device__ __forceinline__ void slot_offsets(const SlotParams& p) {
+  __shared__ int sh[kSlotWarps];
+  __shared__ int sh_off[kMaxE + 2];
+  __shared__ int sh_kept[kMaxE];
+  __shared__ double red[kSlotThreads];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int kPer = (kMaxE + kSlotThreads - 1) / kSlotThreads;   // experts per thread, contiguous
+  const int e0 = tid * kPer;
+  int loc = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i)
+    if (e0 + i < p.E) {
+      const int kept = __ldcg(p.kept_count + e0 + i);
+      sh_kept[e0 + i] = kept;
+      loc += (int)round_up(kept, kRowPad);
+    }
+  int routed;
+  int run = block_scan_excl<kSlotWarps>(loc, sh, routed);
+#pragma unroll
+  for (int i = 0; i < kPer; ++i)
+    if (e0 + i < p.E) {
+      sh_off[e0 + i] = run;
+      run += (int)round_up(sh_kept[e0 + i], kRowPad);
+    }
+  if (p.gates != nullptr) {
+    // "probs" policy: where each expert's arrival-ordered list starts
+    int loc_c = 0;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i)
+      if (e0 + i < p.E) loc_c += __ldcg(p.expert_count + e0 + i);
+    int total;
+    int c = block_scan_excl<kSlotWarps>(loc_c, sh, total);
+#pragma unroll
+    for (int i = 0; i < kPer; ++i)
+      if (e0 + i < p.E) {
+        p.cum[e0 + i] = c;
+        c += __ldcg(p.expert_count + e0 + i);
+      }
+  }
+  if (tid == 0) {
+    sh_off[p.E] = routed;
+    const int64_t end = routed + (p.n_shared ? round_up(p.T, kRowPad) : 0);
+    sh_off[p.E + 1] = (int)end;
+    if (end > p.rows_max) set_status(p.status, MOE_EDEVICE, 2);
+  }
+  __syncthreads();
+  for (int i = tid; i < p.E + 2; i += kSlotThreads) p.expert_offset[i] = sh_off[i];
+  if (p.aux != nullptr) {
+    // aux loss = alpha * E * sum_e term[e]: per-thread sums in expert order, then a fixed tree
+    double t = 0.0;
+    for (int e = tid; e < p.E; e += kSlotThreads) t += p.T > 0 ? __ldcg(p.aux_term + e) : 0.0;
+    red[tid] = t;
+    __syncthreads();
+    for (int s = kSlotThreads / 2; s > 0; s >>= 1) {
+      if (tid < s) red[tid] += red[tid + s];
+      __syncthreads();
+    }
+    if (tid == 0) *p.aux = (float)((double)p.aux_alpha * (double)p.E * red[0]);
+    __syncthreads();
+    if (p.zsum_part != nullptr) {
+      // z-loss = coef * mean_t lse_t^2 from the router's per-block sums, fixed order
+      double z = 0.0;
+      for (int b = tid; b < p.nblk_router; b += kSlotThreads) z += (double)p.zsum_part[b];
+      red[tid] = z;
+      __syncthreads();
+      for (int s = kSlotThreads / 2; s > 0; s >>= 1) {
+        if (tid < s) red[tid] += red[tid + s];
+        __syncthreads();
+      }
+      if (tid == 0) p.aux[1] = p.T > 0 ? (float)((double)p.z_coef * red[0] / (double)p.T) : 0.0f;
+    }
+  }
+  // padding rows of each routed block -> -1; the shared block's rows -> their tokens
+  for (int e = warp; e < p.E; e += kSlotWarps) {
+    const int start = sh_off[e] + sh_kept[e], stop = sh_off[e + 1];
+    for (int r = start + lane; r < stop; r += 32) p.row_token[r] = -1;
+  }
+  if (p.n_shared) {
+    const int64_t s0 = sh_off[p.E], n = round_up(p.T, kRowPad);
+    for (int64_t i = tid; i < n; i += kSlotThreads)
+      if (s0 + i < p.rows_max) p.row_token[s0 + i] = i < p.T ? (int)i : -1;
+  }
+}
+
 __global__ void __launch_bounds__(kSlotThreads) slot_scan_kernel(SlotParams p, int nchunk) {
   pdl_wait();
   pdl_trigger();
@@ -137,65 +226,17 @@ __global__ void __launch_bounds__(kSlotThreads) slot_scan_kernel(SlotParams p, i
       p.aux_term[e] = f * (red[0] / (double)p.T);
     }
   }
-}
-
-__global__ void __launch_bounds__(1024) slot_offsets_kernel(SlotParams p) {
-  pdl_wait();
-  pdl_trigger();
-  __shared__ int sh[32];
-  __shared__ int sh_off[kMaxE + 2];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int kept = tid < p.E ? p.kept_count[tid] : 0;
-  int routed;
-  const int excl = block_scan_excl<32>((int)round_up(kept, kRowPad), sh, routed);
-  if (tid < p.E) sh_off[tid] = excl;
-  if (p.gates != nullptr) {
-    // "probs" policy: where each expert's arrival-ordered list starts
-    int total;
-    const int c = block_scan_excl<32>(tid < p.E ? p.expert_count[tid] : 0, sh, total);
-    if (tid < p.E) p.cum[tid] = c;
-  }
-  if (tid == 0) {
-    sh_off[p.E] = routed;
-    const int64_t end = routed + (p.n_shared ? round_up(p.T, kRowPad) : 0);
-    sh_off[p.E + 1] = (int)end;
-    if (end > p.rows_max) set_status(p.status, MOE_EDEVICE, 2);
-  }
+  // The last expert CTA to finish (fence + ticket; no CTA waits for another)
+  // lays out the row blocks from every expert's kept count.
+  __shared__ int s_last;
+  __threadfence();
   __syncthreads();
-  for (int i = tid; i < p.E + 2; i += 1024) p.expert_offset[i] = sh_off[i];
-  if (p.aux != nullptr) {
-    // aux loss = alpha * E * sum_e term[e], summed by a fixed tree
-    __shared__ double red[1024];
-    red[tid] = (p.T > 0 && tid < p.E) ? p.aux_term[tid] : 0.0;
-    __syncthreads();
-    for (int s = 512; s > 0; s >>= 1) {
-      if (tid < s) red[tid] += red[tid + s];
-      __syncthreads();
-    }
-    if (tid == 0) *p.aux = (float)((double)p.aux_alpha * (double)p.E * red[0]);
-    if (p.zsum_part != nullptr) {
-      // z-loss = coef * mean_t lse_t^2 from the router's per-CTA sums, fixed tree
-      __syncthreads();
-      double z = 0.0;
-      for (int b = tid; b < p.nblk_router; b += 1024) z += (double)p.zsum_part[b];
-      red[tid] = z;
-      __syncthreads();
-      for (int s = 512; s > 0; s >>= 1) {
-        if (tid < s) red[tid] += red[tid + s];
-        __syncthreads();
-      }
-      if (tid == 0) p.aux[1] = p.T > 0 ? (float)((double)p.z_coef * red[0] / (double)p.T) : 0.0f;
-    }
-  }
-  // padding rows of each routed block -> -1
-  for (int e = warp; e < p.E; e += 32) {
-    const int start = sh_off[e] + p.kept_count[e], stop = sh_off[e + 1];
-    for (int r = start + lane; r < stop; r += 32) p.row_token[r] = -1;
-  }
-  if (p.n_shared) {
-    const int64_t s0 = sh_off[p.E], n = round_up(p.T, kRowPad);
-    for (int64_t i = tid; i < n; i += 1024) p.row_token[s0 + i] = i < p.T ? (int)i : -1;
-  }
+  if (threadIdx.x == 0) s_last = atomicAdd(p.ticket, 1u) == (unsigned)(p.E - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  slot_offsets(p);
+  if (threadIdx.x == 0) *p.ticket = 0u;       // ready for the next call
 }
 
 __global__ void __launch_bounds__(kSlotThreads) slot_rank_kernel(SlotParams p, int nchunk) {
@@ -379,14 +420,9 @@ __global__ void __launch_bounds__(kSelThreads) slot_select_kernel(SlotParams p) 
 cudaError_t launch_slots(const SlotParams& p, cudaStream_t stream) {
   const int64_t A = p.T * p.k;
   const int nchunk = (int)((A + kSlotChunk - 1) / kSlotChunk);
-  if (A > 0) {
-    launch_pdl(slot_count_kernel, nchunk, kSlotThreads, p.E * sizeof(int), stream, p, nchunk);
-    launch_pdl(slot_scan_kernel, p.E, kSlotThreads, 0, stream, p, nchunk);
-  } else {
-    cudaMemsetAsync(p.expert_count, 0, p.E * sizeof(int32_t), stream);
-    cudaMemsetAsync(p.kept_count, 0, p.E * sizeof(int32_t), stream);
-  }
-  launch_pdl(slot_offsets_kernel, 1, 1024, 0, stream, p);
+  if (A > 0) launch_pdl(slot_count_kernel, nchunk, kSlotThreads, p.E * sizeof(int), stream, p, nchunk);
+  // one CTA per expert; the last one to finish lays out the row blocks
+  launch_pdl(slot_scan_kernel, p.E, kSlotThreads, 0, stream, p, nchunk);
   if (A > 0) {
     const size_t sm = (size_t)kSlotWarps * p.E * sizeof(int);
     cudaError_t e = ensure_smem(slot_rank_kernel, sm);

@@ -23,7 +23,8 @@ using namespace moe;
 namespace {
 
 constexpr size_t kStaticScratchBytes = size_t(1) << 20;          // 1 MiB
-constexpr size_t kStatusBytes = 256;                             // DevStatus, padded
+constexpr size_t kStatusBytes = 256;                             // DevStatus and the ticket, padded
+constexpr size_t kTicketOffset = 128;
 constexpr int64_t kStaticChunkInts = (int64_t)((kStaticScratchBytes - kStatusBytes) / sizeof(int32_t));
 
 // Shared by every call on a device; holds the last call's contents.
@@ -105,8 +106,9 @@ extern "C" int moe_assign_slots_static(const moe_cfg* cfg, const int32_t* ids, i
   unsigned char* base = static_cast<unsigned char*>(scratch_address(err));
   if (base == nullptr) return err;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // the status word must start at zero; the chunk counts are fully rewritten
-  if (cudaMemsetAsync(base, 0, sizeof(DevStatus), s) != cudaSuccess) return MOE_ECUDA;
+  // the status word and the ticket must start at zero; the chunk counts are
+  // fully rewritten
+  if (cudaMemsetAsync(base, 0, kStatusBytes, s) != cudaSuccess) return MOE_ECUDA;
   SlotParams p{};
   p.ids = ids;
   p.slot = slot;
@@ -116,6 +118,7 @@ extern "C" int moe_assign_slots_static(const moe_cfg* cfg, const int32_t* ids, i
   p.row_token = row_token;
   p.chunk_cnt = reinterpret_cast<int32_t*>(base + kStatusBytes);
   p.status = reinterpret_cast<DevStatus*>(base);
+  p.ticket = reinterpret_cast<unsigned*>(base + kTicketOffset);
   p.T = cfg->T;
   p.E = cfg->E;
   p.k = cfg->k;

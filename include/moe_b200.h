@@ -25,7 +25,9 @@
  *   - Pointers named x, wg, ids, ... are DEVICE pointers owned by the caller;
  *     `cfg` and `w` point to HOST structs read during the call only.
  *   - The library never allocates device memory.  Scratch lives in a caller
- *     workspace of moe_workspace_size() bytes, 256-byte aligned.
+ *     workspace of moe_workspace_size() bytes, 256-byte aligned, zero-filled
+ *     before its first use (the calls leave the parts that must start at zero,
+ *     the status word and the kernels' tickets, at zero).
  *   - Every compute call is asynchronous on `stream` and never synchronises.
  *     The return value reports host-side validation and launch errors only;
  *     errors found on the device (a bad expert id, an exhausted wait) are

@@ -8,27 +8,33 @@ from expert_dispatch_router_b200 import synth
 
 
 def test_forward_launch_counts():
-    # Switch top-1 (profiles/launches_switch_top1_T8192_H768_E64.md): split, router GEMM,
-    # route_logits, 4 slot kernels, GEMM1 with the dispatch, GEMM2 with the combine
-    assert bench.launches_per_step(synth.SWITCH_TOP1) == 9
-    # unfused bf16 layers add the dispatch and combine kernels, and (T*k > 256*E) the
-    # pair-tile prefix of the SM-pair contractions
-    assert bench.launches_per_step(synth.GSHARD_TOP2) == 12
+    # Switch top-1: router (pre-split planes; the logits kernel routes too), 3 slot
+    # kernels, GEMM1 with the dispatch, GEMM2 with the combine
+    assert bench.launches_per_step(synth.SWITCH_TOP1) == 6
+    # the router weight split on every call adds one launch
+    assert bench.launches_per_step(synth.SWITCH_TOP1, packed_router=False) == 7
+    # T*k > 256*E: dispatch kernel, token-tile prefix, two SM-pair contractions,
+    # combine kernel
+    assert bench.launches_per_step(synth.GSHARD_TOP2) == 1 + 3 + 1 + 1 + 2 + 1
     # fp32 router in one launch; the fp32 layer is never fused
-    assert bench.launches_per_step(synth.SWITCH_TINY_F32) == 1 + 4 + 1 + 2 + 1
+    assert bench.launches_per_step(synth.SWITCH_TINY_F32) == 1 + 3 + 1 + 2 + 1
     # the "probs" drop policy adds the per-expert select
-    assert bench.launches_per_step(synth.DS_HIGHK.replace(drop_policy=1)) == 13
+    assert bench.launches_per_step(synth.DS_HIGHK.replace(drop_policy=1)) == 1 + 4 + 1 + 1 + 2 + 1
+    # wider than 256 experts: a separate routing kernel after the logits (top-2 on the
+    # gather path: the combine runs as its own kernel)
+    assert bench.launches_per_step(synth.GSHARD_TOP2.replace(E=300, T=100)) == 2 + 3 + 2 + 1
 
 
 def test_training_launch_counts():
-    # Switch top-1 (profiles/launches_train_switch_top1_T8192_H768_E64.md): 12 forward
-    # launches with MOE_FLAG_TRAINING, 11 backward (dh and dz fused)
-    assert bench.train_launches_per_step(synth.SWITCH_TOP1) == 23
+    # Switch top-1 (the forward with MOE_FLAG_TRAINING: router split + logits/routing,
+    # 3 slot kernels, dispatch, zeroing of padding rows, 2 GEMMs, combine; then 11
+    # backward launches with dh and dz fused)
+    assert bench.train_launches_per_step(synth.SWITCH_TOP1) == 10 + 11
     # GShard top-2: T*k > 256*E (SM-pair forward, + the pair prefix) and H > 512, so
     # dh and dz are two kernels
-    assert bench.train_launches_per_step(synth.GSHARD_TOP2) == 25
+    assert bench.train_launches_per_step(synth.GSHARD_TOP2) == 11 + 12
     # DeepSpeed k=4: H <= 512 fuses them again
-    assert bench.train_launches_per_step(synth.DS_HIGHK) == 24
+    assert bench.train_launches_per_step(synth.DS_HIGHK) == 11 + 11
 
 
 def test_workload_overrides():

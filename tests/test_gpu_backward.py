@@ -4,9 +4,12 @@ The oracle runs the forward on the library's own float32 logits, so both sides
 take the same discrete decisions, then differentiates it in float64.
 
 Tolerances, derived from the arithmetic:
-  * dx sums a token's rows (bf16, fp32 accumulation): |gpu - ref| <= 3e-2 |ref|
-    + 3e-2 rms_row(ref).  Each bf16 rounding contributes a relative error of at
-    most 2^-8; a wrong term is of the order of the values themselves.
+  * dx sums a token's rows dxrow = da W1 (+ db W3) (bf16, fp32 accumulation)
+    and adds dlogits Wg.  Each row carries the rounded dz's noise carried
+    through the contraction over F (sigma^2 = sum_f sigma_dz^2 W1_fh^2, with
+    sigma_dz as for the weight gradients below) and its own bf16 rounding
+    (relative sigma s_u); the token's rows add in quadrature, and dx's final
+    rounding adds at most 2^-8 |dx|: 7 sigma of the rows' noise + 2^-8 |ref|.
   * weight gradients are sums over rows of products of bf16 operands.  One
     rounding to bf16 has relative sigma s_u = 2^-8 / sqrt 3 (8 significant
     bits).  dW2 = dyrow^T h carries two roundings per product.  dW1 (dW3)
@@ -31,9 +34,10 @@ Tolerances, derived from the arithmetic:
     is sum_r |J_rj| 6 sigma_g(r) + 1e-3 |ref| + 1e-7.  When two gates of one token
     have nearly equal dgate, dlogits is their small difference and this bound is
     what keeps the comparison honest.
-  * dx and dWg add that propagated router error (through |Wg| and |x|; summed
-    over tokens in quadrature for dWg, the tokens' errors being independent) to
-    the bf16 rule above.
+  * dx adds that propagated router error through |Wg|.  dWg = dlogits^T x sums
+    independent per-token errors, each bounded by the dlogits bound (a 6 sigma
+    figure): 7/6 of their root-sum-square against x, plus the fp32 accumulation
+    bound over T terms, gamma_T sum_t |dlogits x|.
 """
 import numpy as np
 import pytest
@@ -142,6 +146,7 @@ def check_backward(shape, inp, out, dy, d_aux, d_z):
     # accumulation error of zero is ambiguous: such (row, f) pairs may take
     # either value, so their whole contribution joins the tolerance.
     flip_dx = np.zeros((T, H))
+    var_dx = np.zeros((T, H))          # noise variance of the sum of a token's dxrow rows
     tol_w = {}
     for e, it in ref["experts"].items():
         ts = it["ts"]
@@ -170,9 +175,17 @@ def check_backward(shape, inp, out, dy, d_aux, d_z):
         t2 = K_SIG * np.sqrt(2.0) * S_U * np.sqrt((it["dyrow"] ** 2).T @ (it["h"] ** 2))
         t1 = K_SIG * np.sqrt((s_da ** 2).T @ (Xr ** 2)) + flip.T @ np.abs(Xr)
         t3 = None
+        # dxrow = da W1 (+ db W3): the rounded dz's noise propagated through the
+        # contraction over F, and the row's own bf16 rounding
+        var_row = (s_da ** 2) @ (W1 ** 2)
+        dxr = it["da"] @ W1
         if it["db"] is not None:
             s_db = np.abs(O.silu(a_)) * n_dh + S_U * np.abs(it["db"])
             t3 = K_SIG * np.sqrt((s_db ** 2).T @ (Xr ** 2))
+            W3 = sw[2][0] if e == E else w3[e]
+            var_row = var_row + (s_db ** 2) @ (W3 ** 2)
+            dxr = dxr + it["db"] @ W3
+        np.add.at(var_dx, ts, var_row + (S_U * dxr) ** 2)
         tol_w[e] = (t1, t2, t3)
     gx = out["grads"]
     for n, idx in (("dw1", 0), ("dw2", 1), ("dw3", 2), ("dsw1", 0), ("dsw2", 1), ("dsw3", 2)):
@@ -188,17 +201,25 @@ def check_backward(shape, inp, out, dy, d_aux, d_z):
         bad = np.abs(gw - rw) > tol
         assert np.isfinite(gw).all() and not bad.any(), \
             f"{n}: {int(bad.sum())} of {bad.size} outside the derived bound; {_worst(gw, rw, tol)}"
+    # dx = the token's dxrow rows summed in fp32 + dlogits Wg, rounded once to bf16:
+    # K_SIG sigma of the rows' noise, the final rounding (at most 2^-8 |dx|), the
+    # dlogits bound carried through |Wg|, and the ambiguous ReLU terms
     gdx = out["dx"].double().cpu().numpy()
-    rms = np.sqrt(np.mean(ref["dx"] ** 2, axis=-1, keepdims=True))
-    tol_dx = 3e-2 * np.abs(ref["dx"]) + 3e-2 * rms + tol_dl @ np.abs(wg64) + flip_dx
+    tol_dx = K_SIG * np.sqrt(var_dx) + 2.0 ** -8 * np.abs(ref["dx"]) + tol_dl @ np.abs(wg64) + flip_dx + 1e-9
     bad = np.abs(gdx - ref["dx"]) > tol_dx
     assert np.isfinite(gdx).all() and not bad.any(), \
-        f"dx: {int(bad.sum())} of {bad.size} outside tolerance in {int(bad.any(axis=1).sum())} rows"
+        f"dx: {int(bad.sum())} of {bad.size} outside tolerance in {int(bad.any(axis=1).sum())} rows; " \
+        f"{_worst(gdx, ref['dx'], tol_dx)}"
+    # dWg = dlogits^T x in fp32: each dlogits error is bounded by tol_dl (a 6 sigma
+    # bound), so the weighted sum over tokens has K_SIG sigma <= K_SIG/6 of the
+    # root-sum-square of the bounds; plus fp32 accumulation over T terms
     gwg = out["dwg"].double().cpu().numpy()
-    tol_wg = 3e-2 * np.abs(ref["dwg"]) + 3e-2 * np.sqrt(np.mean(ref["dwg"] ** 2)) \
-        + 3 * np.sqrt((tol_dl ** 2).T @ (x64 ** 2))
+    gam_t = T * 2.0 ** -24 / (1.0 - T * 2.0 ** -24)
+    tol_wg = (K_SIG / 6.0) * np.sqrt((tol_dl ** 2).T @ (x64 ** 2)) \
+        + gam_t * (np.abs(ref["dlogits"]).T @ np.abs(x64)) + 1e-12
     bad = np.abs(gwg - ref["dwg"]) > tol_wg
-    assert np.isfinite(gwg).all() and not bad.any(), f"dWg: {int(bad.sum())} of {bad.size} outside tolerance"
+    assert np.isfinite(gwg).all() and not bad.any(), \
+        f"dWg: {int(bad.sum())} of {bad.size} outside tolerance; {_worst(gwg, ref['dwg'], tol_wg)}"
     return ref
 
 

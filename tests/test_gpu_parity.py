@@ -44,6 +44,9 @@ SMALL = {
     "gshard_2sm": synth.GSHARD_TOP2.replace(name="gshard_2sm", T=1200, H=136, F=520, E=4),
     "relu_2sm_shared": synth.SWITCH_TOP1.replace(name="relu_2sm_shared", T=900, H=96, F=264, E=3, k=2,
                                                  cap_mode=synth.CAP_DROPLESS, n_shared=1, bias_row0=0.0),
+    # skewed loads over 8 experts: groups from a handful of tokens (16-token MMA
+    # tiles) to several 256-token tiles, T not a multiple of 16
+    "skewed_2sm": synth.WIDEEP_DROPLESS.replace(name="skewed_2sm", T=701, H=136, F=72, E=8, k=3, zipf_skew=2.5),
 }
 
 
@@ -57,11 +60,14 @@ def test_layer_small(name, seed, mode):
     check_layer(shape, inp, out)
 
 
-@pytest.mark.parametrize("name", ["switch_top1", "gshard_top2", "wideep", "ds_k4_cf05"])
+@pytest.mark.parametrize("name", ["switch_top1", "gshard_top2", "wideep", "ds_k4_cf05", "wideep_2sm", "gshard_2sm",
+                                  "relu_2sm_shared", "skewed_2sm"])
 def test_fused_matches_unfused(name):
     """Fusing dispatch into the first contraction changes nothing but where A
     comes from: routing, slots, h and the expert outputs are bitwise equal.  The
-    fused top-1 combine rounds gate * accumulator once instead of twice."""
+    fused top-1 combine rounds gate * accumulator once instead of twice.  Layers
+    whose contractions run on SM pairs never fuse: every output is bitwise
+    equal."""
     shape = SMALL[name]
     inp = synth.make_inputs(shape, seed=9, device="cuda")
     a = run_layer(shape, inp)
@@ -72,8 +78,8 @@ def test_fused_matches_unfused(name):
     for n in ("ids", "slot", "expert_offset"):
         assert torch.equal(snap[n], b[n]), n
     assert torch.equal(snap["hbuf"][:used][live], b["hbuf"][:used][live])
+    ya, yb = snap["y"].float(), b["y"].float()
     if a["fused_combine"]:
-        ya, yb = snap["y"].float(), b["y"].float()
         assert ((ya - yb).abs() <= 2.0 ** -7 * yb.abs()).all()   # one bf16 rounding apart
     else:
         assert torch.equal(snap["ybuf"][:used][live], b["ybuf"][:used][live])
@@ -111,18 +117,52 @@ def test_layer_full_size_sampled(shape):
     check_layer(shape, inp, out, tokens=tokens, logit_rows=tokens)
 
 
+def _layer_ms(shape, inp, reps=7):
+    """Median device time of one moe_layer_fwd call (CUDA events)."""
+    cfg = B.make_cfg(shape)
+    ws = B.alloc_workspace(cfg)
+    y = torch.empty((shape.T, shape.H), dtype=torch.bfloat16, device="cuda")
+    aux = torch.empty(2, device="cuda")
+    w = B.make_weights(inp)
+    call = lambda: B.moe_layer_fwd(cfg, inp["x"], inp["wg"], inp["logit_add"], None, w, y, aux, None, ws)
+    for _ in range(3):
+        call()
+    times = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        call()
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    assert B.moe_sync_status(ws) == 0
+    return float(np.median(times))
+
+
 def test_ds_k4_cost_follows_kept_rows():
-    """cf sweep: rows used follow kept assignments, not E*C."""
-    used = {}
-    for den in (1, 2, 4):
-        shape = synth.DS_HIGHK.replace(cf_den=den)
+    """The DeepSpeed k=4 capacity sweep ([DS7508] follow-ups: with a fixed
+    capacity buffer the step time grows with cf).  Here rows used follow the
+    kept assignments, not E*C: at cf = 2.0, E*C is twice the assignments, yet
+    the rows (and the time) stay those of cf = 1.0, and halving cf below 1
+    shrinks both."""
+    used, kept, ms = {}, {}, {}
+    for num, den in ((2, 1), (1, 1), (1, 2), (1, 4)):
+        shape = synth.DS_HIGHK.replace(cf_num=num, cf_den=den)
         inp = synth.make_inputs(shape, seed=0, device="cuda", experts=shape.E)
         out = run_layer(shape, inp, keep_logits=False)
-        kept = int(out["kept_count"].sum())
+        cf = num / den
+        kept[cf] = int(out["kept_count"].sum())
         rows = int(out["expert_offset"][-1])
-        assert rows - kept < 128 * shape.E
-        used[den] = rows
-    assert used[1] > used[2] > used[4]
+        assert rows - kept[cf] < 128 * shape.E
+        used[cf] = rows
+        ms[cf] = _layer_ms(shape, inp)
+    E, A = synth.DS_HIGHK.E, synth.DS_HIGHK.T * synth.DS_HIGHK.k
+    C2 = O.capacity(synth.DS_HIGHK.T, E, synth.DS_HIGHK.k, 2, 1)
+    assert kept[2.0] == A and E * C2 >= 2 * A                  # nothing dropped, capacity far above the load
+    assert used[2.0] < 0.6 * E * C2                            # rows follow kept, not E*C
+    assert used[2.0] >= used[1.0] > used[0.5] > used[0.25]
+    assert ms[2.0] < 1.25 * ms[1.0]                            # doubling C costs ~nothing
+    assert ms[0.25] < ms[1.0]
 
 
 def test_route_from_logits_bitexact_with_ties():
