@@ -27,7 +27,6 @@ library's kernels through the C ABI; the collectives are torch.distributed's.
 """
 from __future__ import annotations
 
-import math
 from typing import Optional
 
 import torch
@@ -84,9 +83,9 @@ class LocalOps:
         raise NotImplementedError
 
 
-def _all_to_all_rows(out: torch.Tensor, inp: torch.Tensor, out_splits, in_splits, group):
+def _all_to_all_rows(out: torch.Tensor, inp: torch.Tensor, out_splits, in_splits, group, world: int):
     """all_to_all of row blocks (variable row counts per peer)."""
-    if dist.get_world_size(group) == 1:
+    if world == 1:
         out.copy_(inp)
         return
     dist.all_to_all_single(out, inp, output_split_sizes=list(out_splits), input_split_sizes=list(in_splits),
@@ -115,7 +114,7 @@ def ep_layer_forward(x: torch.Tensor, wg: torch.Tensor, logit_add: Optional[torc
     # 2. dispatch all-to-all: rows of rank d's experts go to rank d
     send = r["xbuf"][: off[E]]
     recv = torch.empty((sum(recv_rows), H), dtype=x.dtype, device=x.device)
-    _all_to_all_rows(recv, send, recv_rows, send_rows, group)
+    _all_to_all_rows(recv, send, recv_rows, send_rows, group, world)
     # 3. this rank's experts over every source's block
     out = torch.empty_like(recv)
     base = 0
@@ -126,7 +125,7 @@ def ep_layer_forward(x: torch.Tensor, wg: torch.Tensor, logit_add: Optional[torc
         base += n
     # 4. combine all-to-all: the rows return to their source, in their layout
     back = torch.empty((off[E], H), dtype=x.dtype, device=x.device)
-    _all_to_all_rows(back, out, send_rows, recv_rows, group)
+    _all_to_all_rows(back, out, send_rows, recv_rows, group, world)
     y = ops.combine(back, ops.shared_ffn(x), r)
     return y, r["aux"]
 
