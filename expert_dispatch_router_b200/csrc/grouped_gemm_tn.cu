@@ -80,6 +80,7 @@ struct KParams {
   int K, N_out, E, n_shared, epi;
   int as_sep;                           // 1: the shared block's token rows come from tmBs (row - off[E])
   int b_packed;                         // 1: weight maps are 5-D over packed blocks
+  int wide;                             // 1 (no SwiGLU): 512 features per pair tile, two MMAs share each B tile
 };
 
 // Rows of group g that carry tokens: the routed groups' kept counts, the
@@ -133,10 +134,14 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tn_kernel(const __gri
   const uint32_t rank = cluster_rank();
   const bool leader = rank == 0;
   const bool swiglu = p.epi == MOE_ACT_SWIGLU;
+  // two accumulators per tile, fed by one B tile: gate | up (SwiGLU), or two
+  // 256-feature halves of a 512-feature tile (wide); they fill all 512 columns
+  const bool two = swiglu || p.wide;
+  const int span = p.wide ? 2 * FT : FT;        // output features per pair tile
   const int ngroups = p.E + (p.n_shared ? 1 : 0);
-  const int stage_bytes = (swiglu ? 2 : 1) * A_BYTES + B_BYTES;
+  const int stage_bytes = (two ? 2 : 1) * A_BYTES + B_BYTES;
   const int n_stages = min(MAX_STAGES, RING_BYTES / stage_bytes);
-  const int n_acc = swiglu ? 1 : 2;              // SwiGLU: gate | up fill all 512 columns
+  const int n_acc = two ? 1 : 2;
   auto abort_pair = [&](int info) {
     *abort_flag = 1;
     st_cluster_u32(map_to(smem_u32((const void*)abort_flag), rank ^ 1u), 1u);
@@ -168,7 +173,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tn_kernel(const __gri
   pdl_wait();
   if (!tmem_same && threadIdx.x == 0) set_status(p.status, MOE_EDEVICE, 31);
 
-  const int nf = (p.N_out + FT - 1) / FT;                      // feature tiles
+  const int nf = (p.N_out + span - 1) / span;                  // feature tiles
   const int64_t n_tok_tiles = tmem_same ? __ldg(p.tp + ngroups) : 0;
   const int64_t n_tiles = n_tok_tiles * nf;
   const int nk = (p.K + BK - 1) / BK;
@@ -191,21 +196,23 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tn_kernel(const __gri
         const CUtensorMap* ma1 = sh ? &p.tmSA1 : &p.tmA1;
         const CUtensorMap* mb = sep ? &p.tmBs : &p.tmB;
         const int z = sh ? 0 : t.g;
-        const int wrow = t.ft * FT + (int)rank * HALF;          // this CTA's weight rows
+        const int wrow = t.ft * span + (int)rank * HALF;        // this CTA's weight rows
+        const CUtensorMap* ma2 = swiglu ? ma1 : ma;             // the second accumulator's rows
+        const int wrow2 = swiglu ? wrow : wrow + FT;
         const int64_t brow64 = (sep ? t.r0 - __ldg(p.off + p.E) : t.r0) + (int64_t)rank * (t.n / 2);
         const int brow = (int)brow64;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait_cl(empty0 + 8 * stage, phase ^ 1u, abort_flag)) { ok = false; break; }
           const uint32_t sa = smem_u32(stage_base + stage * stage_bytes);
-          const uint32_t sb = sa + (swiglu ? 2 : 1) * A_BYTES;
+          const uint32_t sb = sa + (two ? 2 : 1) * A_BYTES;
           const uint32_t fb = full_leader0 + 8 * stage;
           if (leader) mbar_expect_tx(full0 + 8 * stage, tx);
           if (p.b_packed) {
             tma2_load_5d(sa, ma, kb, wrow / 128, z, fb);
-            if (swiglu) tma2_load_5d(sa + A_BYTES, ma1, kb, wrow / 128, z, fb);
+            if (two) tma2_load_5d(sa + A_BYTES, ma2, kb, wrow2 / 128, z, fb);
           } else {
             tma2_load_3d(sa, ma, kb * BK, wrow, z, fb);
-            if (swiglu) tma2_load_3d(sa + A_BYTES, ma1, kb * BK, wrow, z, fb);
+            if (two) tma2_load_3d(sa + A_BYTES, ma2, kb * BK, wrow2, z, fb);
           }
           tma2_load_2d(sb, mb, kb * BK, brow, fb);
           fills[stage]++;
@@ -227,7 +234,67 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tn_kernel(const __gri
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int64_t tile = cid; tile < n_tiles && ok; tile += ncl) {
+      for (int64_t tile = cid; tile < n_tiles && ok && p.wide; tile += ncl) {
+        // wide: the epilogue frees accumulator 0 (columns 0-255) before
+        // accumulator 1, so this tile's MMAs into accumulator 0 start as soon
+        // as it is free; a stage whose accumulator-1 MMAs cannot go yet is held
+        // (at most n_stages - 1 of them) until accumulator 1 is free too
+        const Tile t = decode(p, ngroups, nf, tile);
+        const uint32_t idesc = make_idesc(t.n, 2 * HALF);
+        if (!mbar_wait_cl(tempty0, acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        bool have1 = false;
+        int held = 0, held_stage = 0;
+        // k step nk only flushes what is still held (K shorter than the ring)
+        for (int kb = 0; kb <= nk; ++kb) {
+          const bool past = kb == nk;
+          const uint32_t sa = smem_u32(stage_base + stage * stage_bytes);
+          const uint64_t bd = sw128_desc(sa + 2 * A_BYTES);
+          if (!past) {
+            if (!mbar_wait_cl(full0 + 8 * stage, phase, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint64_t ad = sw128_desc(sa);
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+              umma2(tmem_base, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          if (!have1) {
+            if (!past && held + 1 < n_stages && !mbar_test_cl(tempty0 + 8, acc_phase ^ 1u)) {
+              if (held++ == 0) held_stage = stage;
+              if (++stage == n_stages) { stage = 0; phase ^= 1u; }
+              continue;
+            }
+            // accumulator 1 is free: the held stages' accumulator-1 MMAs, in
+            // k order (the last held stage is k step kb - 1), then their release
+            if (!mbar_wait_cl(tempty0 + 8, acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            have1 = true;
+            for (int h = 0, hs = held_stage; h < held; ++h) {
+              const uint32_t ha = smem_u32(stage_base + hs * stage_bytes);
+              const uint64_t hb = sw128_desc(ha + 2 * A_BYTES), hu = sw128_desc(ha + A_BYTES);
+              const int hk = kb - held + h;
+#pragma unroll
+              for (int kk = 0; kk < BK / 16; ++kk)
+                umma2(tmem_base + 256, hu + (uint64_t)(kk * 2), hb + (uint64_t)(kk * 2), idesc,
+                      (hk | kk) != 0 ? 1u : 0u);
+              umma2_commit_both(empty0 + 8 * hs);
+              if (++hs == n_stages) hs = 0;
+            }
+            held = 0;
+          }
+          if (past) break;
+          const uint64_t ud = sw128_desc(sa + A_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma2(tmem_base + 256, ud + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
+          umma2_commit_both(empty0 + 8 * stage);
+          if (++stage == n_stages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma2_commit_both(tfull0);
+        acc_phase ^= 1u;
+      }
+      for (int64_t tile = cid; tile < n_tiles && ok && !p.wide; tile += ncl) {
         const Tile t = decode(p, ngroups, nf, tile);
         const uint32_t idesc = make_idesc(t.n, 2 * HALF);
         if (!mbar_wait_cl(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag)) { ok = false; break; }
@@ -237,12 +304,12 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tn_kernel(const __gri
           if (!mbar_wait_cl(full0 + 8 * stage, phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(stage_base + stage * stage_bytes);
-          const uint64_t bd = sw128_desc(sa + (swiglu ? 2 : 1) * A_BYTES);
+          const uint64_t bd = sw128_desc(sa + (two ? 2 : 1) * A_BYTES);
           const uint64_t ad = sw128_desc(sa);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)               // 16 elements = 32 bytes along K
             umma2(d0, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
-          if (swiglu) {
+          if (two) {
             const uint64_t ud = sw128_desc(sa + A_BYTES);
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk)
@@ -276,13 +343,15 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tn_kernel(const __gri
         break;
       }
       tc_fence_after();
-      const int f0 = t.ft * FT + (int)rank * HALF + sub * 32;
       const uint32_t tbase = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * 256);
-      if (f0 < p.N_out) {
-        for (int c = quarter * 32; c < t.n; c += 4 * 32) {
+      // wide: accumulator a (columns 256 a ..) holds features 256 a .. of the tile
+      for (int a = 0; a < (p.wide ? 2 : 1); ++a) {
+        const int f0 = t.ft * span + a * FT + (int)rank * HALF + sub * 32;
+        const uint32_t tb = tbase + (uint32_t)(a * 256);
+        for (int c = quarter * 32; c < t.n && f0 < p.N_out; c += 4 * 32) {
           __syncwarp();
           float v[32];
-          tmem_ld(tbase + (uint32_t)c, v, 32);
+          tmem_ld(tb + (uint32_t)c, v, 32);
           if (swiglu) {
             float u[32];
             tmem_ld(tbase + 256u + (uint32_t)c, u, 32);
@@ -319,10 +388,18 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tn_kernel(const __gri
             bulk_commit();
           }
         }
+        if (p.wide) {
+          // accumulator a is read: the next tile's MMAs may write it
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8 * a);
+        }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8 * acc);
+      if (!p.wide) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8 * acc);
+      }
       if (++acc == n_acc) { acc = 0; acc_phase ^= 1u; }
     }
     if (lane == 0) bulk_wait0();
@@ -506,6 +583,12 @@ cudaError_t launch_grouped_gemm_tn(const GemmParams& p, cudaStream_t stream) {
   k.epi = p.epi;
   k.as_sep = p.a_shared != nullptr;
   k.b_packed = p.b_packed;
+  // 512-feature tiles where the epilogue is cheap (no activation, or ReLU): two
+  // accumulators share every B tile, so a pair moves 48 KB per 64-k step for
+  // twice the MMA work of a 32 KB step.  They are single-buffered, so an
+  // expensive epilogue (GELU) would stall the MMAs: those keep 256-feature,
+  // double-buffered tiles.
+  k.wide = ((p.epi < 0 || p.epi == MOE_ACT_RELU) && p.Nw >= 2 * FT) ? 1 : 0;
   cudaError_t e = ensure_smem(grouped_gemm_tn_kernel, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg{};

@@ -68,6 +68,15 @@ __device__ __forceinline__ bool mbar_wait_cl(uint32_t bar, uint32_t parity, vola
     if (clock64() - t0 > kWaitCycles) return false;
   }
 }
+// Non-blocking test of the same phase.
+__device__ __forceinline__ bool mbar_test_cl(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile("{\n\t.reg .pred p;\n\t"
+               "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+               "selp.u32 %0, 1, 0, p;\n\t}"
+               : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0;
+}
 // Drain wait (no abort check): bounded by kWaitCycles.
 __device__ __forceinline__ void mbar_drain_cl(uint32_t bar, uint32_t parity) {
   const long long t0 = clock64();

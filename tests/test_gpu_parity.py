@@ -47,6 +47,11 @@ SMALL = {
     # skewed loads over 8 experts: groups from a handful of tokens (16-token MMA
     # tiles) to several 256-token tiles, T not a multiple of 16
     "skewed_2sm": synth.WIDEEP_DROPLESS.replace(name="skewed_2sm", T=701, H=136, F=72, E=8, k=3, zipf_skew=2.5),
+    # plain (ReLU) contractions of 512 output features per pair tile (two
+    # accumulators share each token tile) in both GEMMs: H = 2 * 512 + 8 and
+    # F = 512 + 72 leave a ragged last tile, with a shared expert
+    "wide_2sm_shared": synth.SWITCH_TOP1.replace(name="wide_2sm_shared", T=1100, H=1032, F=584, E=4, k=2,
+                                                 cap_mode=synth.CAP_DROPLESS, n_shared=1, bias_row0=0.0),
 }
 
 
@@ -61,7 +66,7 @@ def test_layer_small(name, seed, mode):
 
 
 @pytest.mark.parametrize("name", ["switch_top1", "gshard_top2", "wideep", "ds_k4_cf05", "wideep_2sm", "gshard_2sm",
-                                  "relu_2sm_shared", "skewed_2sm"])
+                                  "relu_2sm_shared", "skewed_2sm", "wide_2sm_shared"])
 def test_fused_matches_unfused(name):
     """Fusing dispatch into the first contraction changes nothing but where A
     comes from: routing, slots, h and the expert outputs are bitwise equal.  The
@@ -358,7 +363,7 @@ def test_pack_weight_layout(G, N, K):
 
 
 @pytest.mark.parametrize("name", ["switch_top1", "gshard_top2", "wideep", "ds_k4_cf05", "switch_relu_dropless_shared",
-                                  "wideep_2sm", "gshard_2sm", "relu_2sm_shared"])
+                                  "wideep_2sm", "gshard_2sm", "relu_2sm_shared", "wide_2sm_shared"])
 def test_packed_weights_bitwise(name):
     """Packed weights change only where the contractions read B from."""
     shape = SMALL[name]
