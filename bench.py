@@ -269,7 +269,7 @@ def traffic_from_profiles(workload: str, kernel: str):
     p = os.path.join(ROOT, "profiles", "traffic.md")
     if not os.path.exists(p):
         return None
-    src = os.path.join(ROOT, "expert_dispatch_router_b200", "csrc", kernel_source(kernel))
+    src = os.path.join(ROOT, "expert_dispatch_router_b200", "csrc", kernel_source(kernel, workload))
     sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:12]
     for line in open(p):
         cells = [c.strip() for c in line.strip().strip("|").split("|")]
@@ -281,7 +281,17 @@ def traffic_from_profiles(workload: str, kernel: str):
     return None
 
 
-def kernel_source(stage: str) -> str:
+def kernel_source(stage: str, workload: str = None) -> str:
+    """The source file of the kernel a stage runs: the expert contractions of
+    bf16 layers with T*k > 256*E run on SM pairs (grouped_gemm_tn.cu); the bf16
+    router's logits GEMM (with the routing in its epilogue) is in grouped_gemm.cu."""
+    from expert_dispatch_router_b200 import synth
+    shape = synth.WORKLOADS.get(workload) if workload else None
+    bf16 = shape is not None and shape.dtype == 1
+    if stage in ("ffn_gemm1", "ffn_gemm2") and bf16 and shape.T * shape.k > 256 * shape.E:
+        return "grouped_gemm_tn.cu"
+    if stage == "router" and bf16:
+        return "grouped_gemm.cu"
     return {"router": "router.cu", "dispatch": "permute.cu", "combine": "permute.cu",
             "ffn_gemm1": "grouped_gemm.cu", "ffn_gemm2": "grouped_gemm.cu",
             "combine_bwd": "backward.cu", "dispatch_bwd": "backward.cu", "router_wgrad": "backward.cu",
