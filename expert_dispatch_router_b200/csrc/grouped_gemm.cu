@@ -42,7 +42,6 @@
 
 #include "common.cuh"
 #include "kernels.h"
-#include "route_common.cuh"
 #include "tc_common.cuh"
 
 namespace moe {
@@ -98,10 +97,10 @@ struct KParams {
   // (k block, plane) in the same order), for wide N where three planes would
   // leave too few stages.
   int planes_per_stage;
-  // router with routing fused (ROUTE_EJ > 0): after a tile's logits are stored,
-  // the epilogue warps route its 128 tokens (route_common.cuh) and store the
-  // tile's partial sums in row 4 * m-block of the 32-token partial arrays (the
-  // other three rows of the tile are zero).
+  // router with routing fused (ROUTE_KM > 0): the epilogue routes the tile's
+  // 128 tokens from the accumulator (route_tile_tmem) and stores the tile's
+  // partial sums in row 4 * m-block of the 32-token partial arrays (the other
+  // three rows of the tile are zero).
   RouterParams rp;
   int64_t nblk;          // rows of the partial arrays (32 tokens each)
 };
@@ -121,49 +120,207 @@ __device__ __forceinline__ bool epilogue_all(bool v) {
   return r != 0;
 }
 
-// Routing of one router tile's 128 tokens by the 16 epilogue warps, once the
-// tile's fp32 logits are in memory (plain stores of this CTA: visible to its
-// threads after the barrier).  Warp w routes tokens w, w + 16, ...; the warps'
-// per-expert sums are then added in warp order through the staging buffer
-// (deterministic) into row 4 * mt of the 32-token partial arrays, and rows
-// 4 mt + 1 .. 4 mt + 3 are zeroed, so the reductions over all rows see the same
-// totals as with one row per 32 tokens.
-template <int EJ>
-__device__ __forceinline__ void route_tile(const KParams& p, int64_t mt, int ew, int lane, uint8_t* staging,
-                                           float* route_z) {
-  constexpr int EP = 32 * EJ;
-  static_assert(2 * EPI_WARPS * EP * 4 <= STAGING_BYTES, "router partials exceed the staging buffer");
+// Routing of one router tile's 128 tokens straight from its accumulator
+// (lane = token, columns = experts), a token per thread.  The four warps of a
+// TMEM sub-partition (the same 32 tokens) take four ranges of W columns each
+// and meet at their own named barrier (2 + sub) to combine, in a fixed order:
+// the maximum, the sums of exp(l - m) (and of the sigmoids), and the top-k,
+// chosen one rank at a time from the four ranges' sorted lists (keys: larger
+// logit first, equal logits -> smaller expert; the order the oracle uses).
+// Selection counts add up in shared memory (integers: any order gives the same
+// total); each expert's probability sum over the tile's tokens is a fixed
+// butterfly over the lanes, then the four sub-partitions in order.  The tile's
+// sums go to row 4 * mt of the 32-token partial arrays and rows 4 mt + 1 ..
+// 4 mt + 3 are zeroed.  The logit offset, where there is one, is added once
+// and the sums written back to TMEM for the later passes.
+__device__ __forceinline__ void sub_bar(int sub) {
+  asm volatile("bar.sync %0, 128;" :: "r"(2 + sub) : "memory");
+}
+__device__ __forceinline__ unsigned long long route_key(float l, int e) {
+  return ((unsigned long long)to_ordered(l) << 32) | (unsigned long long)(0xffffffffu - (uint32_t)e);
+}
+template <int KM>
+__device__ __forceinline__ void route_tile_tmem(const KParams& p, int64_t mt, int sub, int quarter, int lane,
+                                                uint8_t* staging, uint32_t tacc, int ncols) {
   const RouterParams& rp = p.rp;
-  const int E = rp.E;
-  const float* logits = static_cast<const float*>(p.d);
-  epilogue_bar();                                        // every warp's logits stores are done
-  float psum[EJ], zacc = 0.0f;
-  int cnt[EJ];
+  const int E = rp.E, k = rp.k;
+  const int tid = (sub * 4 + quarter) * 32 + lane;                 // 0 .. 511, unique per thread
+  const int64_t t = mt * BM + sub * 32 + lane;
+  const bool tv = t < rp.T;
+  // columns per quarter: 8, 16, 32 or 64 (a multiple of the columns of one
+  // TMEM access, so that no access reaches into the next quarter's range);
+  // columns at or past E are masked
+  const int q4 = (ncols + 3) / 4;
+  const int W = q4 <= 8 ? 8 : q4 <= 16 ? 16 : q4 <= 32 ? 32 : 64;
+  const int c0 = quarter * W;
+  const int ch = W >= 32 ? 32 : W;                                 // columns per TMEM access
+  const bool sigmoid = rp.score == MOE_SCORE_SIGMOID_TOPK;
+  float* xmax = reinterpret_cast<float*>(staging);                 // [4 sub][4 quarter][32]
+  float* xsum = xmax + 512;
+  float* xss = xsum + 512;
+  unsigned long long* xhead = reinterpret_cast<unsigned long long*>(xss + 512);   // [2][4][4][32]
+  float* xps = reinterpret_cast<float*>(xhead + 1024);            // [4 sub][256]
+  int* xcnt = reinterpret_cast<int*>(xps + 1024);                 // [256]
+  float* xz = reinterpret_cast<float*>(xcnt + 256);               // [4]
+  static_assert(512 * 4 * 3 + 1024 * 8 + 1024 * 4 + 256 * 4 + 16 <= STAGING_BYTES, "routing exchange area");
+  if (tid < 256) xcnt[tid] = 0;
+  epilogue_bar();                                                  // the staging area is free; counts zeroed
+
+  // 1. logits (+ offset) -> this range's maximum and sorted top-k keys
+  unsigned long long key[KM];
 #pragma unroll
-  for (int j = 0; j < EJ; ++j) { psum[j] = 0.0f; cnt[j] = 0; }
-  const int64_t t0 = mt * BM;
-  for (int i = ew; i < BM; i += EPI_WARPS) {
-    const int64_t t = t0 + i;
-    if (t >= rp.T) break;
-    float val[EJ];
+  for (int i = 0; i < KM; ++i) key[i] = 0ull;
+  float m = -INFINITY;
+  for (int cc = 0; cc < W; cc += ch) {
+    float v[32];
+    tmem_ld(tacc + (uint32_t)(c0 + cc), v, ch);
+    tmem_wait_ld();
 #pragma unroll
-    for (int j = 0; j < EJ; ++j) {
-      const int e = lane_expert<EJ>(lane, j);
-      val[j] = e < E ? logits[t * E + e] : 0.0f;
+    for (int j = 0; j < 32; ++j) {
+      const int e = c0 + cc + j;
+      if (j >= ch) break;
+      if (tv && e < E) {
+        if (rp.logit_add != nullptr) v[j] += rp.logit_add[t * E + e];
+        if (rp.logits_out != nullptr) rp.logits_out[t * E + e] = v[j];
+        m = fmaxf(m, v[j]);
+        unsigned long long x = route_key(v[j], e);
+#pragma unroll
+        for (int i = 0; i < KM; ++i)
+          if (i < k) {
+            const unsigned long long hi = key[i] > x ? key[i] : x;
+            x = key[i] > x ? x : key[i];
+            key[i] = hi;
+          }
+      }
     }
-    route_token<EJ>(rp, t, lane, val, psum, cnt, zacc);
+    if (rp.logit_add != nullptr) tmem_st(tacc + (uint32_t)(c0 + cc), v, ch);
   }
-  float* sp = reinterpret_cast<float*>(staging);                       // [EPI_WARPS][EP]
-  int* sc = reinterpret_cast<int*>(staging) + EPI_WARPS * EP;           // [EPI_WARPS][EP]
+  if (rp.logit_add != nullptr) tmem_wait_st();
+  xmax[tid] = m;
+  sub_bar(sub);
+  {
+    const float* q = xmax + sub * 128 + lane;
+    m = fmaxf(fmaxf(q[0], q[32]), fmaxf(q[64], q[96]));
+  }
+
+  // 2. sums of exp(l - m) (and of sigmoid(l)) over the whole token
+  float s = 0.0f, ss = 0.0f;
+  for (int cc = 0; cc < W; cc += ch) {
+    float v[32];
+    tmem_ld(tacc + (uint32_t)(c0 + cc), v, ch);
+    tmem_wait_ld();
 #pragma unroll
-  for (int j = 0; j < EJ; ++j) {
-    const int e = lane_expert<EJ>(lane, j);
-    sp[ew * EP + e] = psum[j];
-    sc[ew * EP + e] = cnt[j];
+    for (int j = 0; j < 32; ++j) {
+      if (j >= ch) break;
+      if (tv && c0 + cc + j < E) {
+        s += expf(v[j] - m);
+        if (sigmoid) ss += 1.0f / (1.0f + expf(-v[j]));
+      }
+    }
   }
-  if (lane == 0) route_z[ew] = zacc;
+  xsum[tid] = s;
+  xss[tid] = ss;
+  sub_bar(sub);
+  {
+    const float* q = xsum + sub * 128 + lane;
+    s = ((q[0] + q[32]) + q[64]) + q[96];
+    const float* r = xss + sub * 128 + lane;
+    ss = ((r[0] + r[32]) + r[64]) + r[96];
+  }
+
+  // 3. the top-k, one rank at a time: the best of the four ranges' heads
+  unsigned long long sel[KM];
+  int pos = 0;
+#pragma unroll
+  for (int r = 0; r < KM; ++r) {
+    sel[r] = 0ull;
+    if (r < k) {
+      unsigned long long h = 0ull;
+#pragma unroll
+      for (int i = 0; i < KM; ++i)
+        if (i == pos) h = key[i];
+      unsigned long long* buf = xhead + (r & 1) * 512 + sub * 128 + lane;
+      buf[quarter * 32] = h;
+      sub_bar(sub);
+      unsigned long long w = 0ull;
+      int wq = 0;
+#pragma unroll
+      for (int q2 = 0; q2 < 4; ++q2) {
+        const unsigned long long hq = buf[q2 * 32];
+        if (hq > w) { w = hq; wq = q2; }
+      }
+      sel[r] = w;
+      if (wq == quarter && w != 0ull) {
+        ++pos;
+        if (tv) atomicAdd(xcnt + (int)(0xffffffffu - (uint32_t)(w & 0xffffffffull)), 1);
+      }
+    }
+  }
+
+  // 4. gates and ids (the first quarter's warp writes its tokens' rows)
+  if (quarter == 0 && tv) {
+    float g[KM];
+    float gs = 0.0f;
+#pragma unroll
+    for (int r = 0; r < KM; ++r) {
+      g[r] = 0.0f;
+      if (r < k) {
+        const float l = from_ordered((uint32_t)(sel[r] >> 32));
+        g[r] = sigmoid ? 1.0f / (1.0f + expf(-l)) : expf(l - m);
+        gs += g[r];
+      }
+    }
+    const bool renorm = rp.score == MOE_SCORE_TOPK_SOFTMAX || rp.renorm;
+#pragma unroll
+    for (int r = 0; r < KM; ++r) {
+      if (r >= k) break;
+      if (renorm) g[r] = g[r] / gs;
+      else if (rp.score == MOE_SCORE_SOFTMAX_TOPK) g[r] = g[r] / s;
+    }
+#pragma unroll
+    for (int r = 0; r < KM; ++r) {
+      if (r >= k) break;
+      int e = sel[r] != 0ull ? (int)(0xffffffffu - (uint32_t)(sel[r] & 0xffffffffull)) : -1;
+      float gr = g[r];
+      // GShard top-2: the second choice is dispatched iff u_t < 2 g_t1
+      if (r == 1 && rp.uniform != nullptr && !(rp.uniform[t] < 2.0f * gr)) { e = -1; gr = 0.0f; }
+      rp.ids[t * k + r] = e;
+      rp.gates[t * k + r] = gr;
+    }
+  }
+
+  // 5. z-loss: lse^2 summed over the tile's tokens
+  if (rp.zsum_part != nullptr && quarter == 0) {
+    float z = 0.0f;
+    if (tv) {
+      const float lse = m + logf(s);
+      z = lse * lse;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    if (lane == 0) xz[sub] = z;
+  }
+
+  // 6. each expert's probability sum over the tile's tokens
+  if (rp.psum_part != nullptr) {
+    const float inv = 1.0f / (sigmoid ? ss : s);
+    for (int cc = 0; cc < W; cc += ch) {
+      float v[32];
+      tmem_ld(tacc + (uint32_t)(c0 + cc), v, ch);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (j >= ch) break;
+        const int e = c0 + cc + j;
+        float pe = 0.0f;
+        if (tv && e < E) pe = (sigmoid ? 1.0f / (1.0f + expf(-v[j])) : expf(v[j] - m)) * inv;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) pe += __shfl_xor_sync(0xffffffffu, pe, o);
+        if (lane == 0 && e < E) xps[sub * 256 + e] = pe;
+      }
+    }
+  }
   epilogue_bar();
-  const int tid = ew * 32 + lane;
   const int64_t row0 = 4 * mt;
   for (int idx = tid; idx < 4 * E; idx += EPI_WARPS * 32) {
     const int q = idx / E, e = idx - q * E;
@@ -172,30 +329,28 @@ __device__ __forceinline__ void route_tile(const KParams& p, int64_t mt, int ew,
     float ps = 0.0f;
     int cs = 0;
     if (q == 0) {
-#pragma unroll
-      for (int w = 0; w < EPI_WARPS; ++w) { ps += sp[w * EP + e]; cs += sc[w * EP + e]; }
+      ps = ((xps[e] + xps[256 + e]) + xps[512 + e]) + xps[768 + e];
+      cs = xcnt[e];
     }
-    rp.psum_part[row * E + e] = ps;
-    rp.cnt_part[row * E + e] = cs;
+    if (rp.psum_part != nullptr) rp.psum_part[row * E + e] = ps;
+    if (rp.cnt_part != nullptr) rp.cnt_part[row * E + e] = cs;
   }
   if (tid == 0) {
     if (rp.zsum_part != nullptr) {
-      float z = 0.0f;
-#pragma unroll
-      for (int w = 0; w < EPI_WARPS; ++w) z += route_z[w];
+      const float z = ((xz[0] + xz[1]) + xz[2]) + xz[3];
       for (int q = 0; q < 4; ++q)
         if (row0 + q < p.nblk) rp.zsum_part[row0 + q] = q == 0 ? z : 0.0f;
     }
     if (mt == 0 && rp.aux_counter != nullptr) *rp.aux_counter = 0u;   // re-armed for moe_aux_loss
   }
-  epilogue_bar();                                        // the staging buffer is free again
+  epilogue_bar();                                                  // the staging area is free again
 }
 
 // GATHER: routed A rows are gathered from p.gsrc by warps 18-19 (fused
 // dispatch).  SCATTER: routed output rows go to p.sdst[token] * gate (fused
-// top-1 combine).  Both false: every operand moves by TMA.  ROUTE_EJ > 0:
-// router logits with routing fused into the epilogue (E <= 32 * ROUTE_EJ).
-template <bool GATHER, bool SCATTER, int ROUTE_EJ = 0>
+// top-1 combine).  Both false: every operand moves by TMA.  ROUTE_KM > 0:
+// router logits with routing fused into the epilogue (E <= 256, k <= ROUTE_KM).
+template <bool GATHER, bool SCATTER, int ROUTE_KM = 0>
 __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ KParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -209,7 +364,6 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
   const uint32_t drain = smem_u32(bars + 2 * MAX_STAGES + 4);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * MAX_STAGES + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* route_z = reinterpret_cast<float*>(tmem_slot + 2);     // [EPI_WARPS] z-loss sums (router)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool swiglu = p.epi == MOE_ACT_SWIGLU;
@@ -448,7 +602,7 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
     uint32_t acc_phase = 0;
     for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
       bool got = mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag);
-      if constexpr (ROUTE_EJ > 0) got = epilogue_all(got);   // the routing below has barriers
+      if constexpr (ROUTE_KM > 0) got = epilogue_all(got);   // the routing below has barriers
       if (!got) {
         *abort_flag = 1;
         set_status(p.status, MOE_ETIMEOUT, 12);
@@ -469,91 +623,95 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
       }
       const int ncol0 = nt * n_step;                           // first output column of the tile
       const uint32_t tbase = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * BN);
-      for (int c = quarter * chunk; c < n_step; c += 4 * chunk) {
-        __syncwarp();                                // converged for the warp-wide tcgen05.ld
-        float v[32];
-        const int acol = c;                                     // accumulator column
-        tmem_ld(tbase + (uint32_t)acol, v, chunk);
-        if (swiglu) {
-          float u[32];
-          tmem_ld(tbase + (uint32_t)(BN / 2 + acol), u, chunk);
-          tmem_wait_ld();
+      if constexpr (ROUTE_KM > 0) {
+        // the router: route the tile's tokens from the accumulator itself
+        route_tile_tmem<ROUTE_KM>(p, mt, sub, quarter, lane, staging, tbase, bn);
+      } else {
+        for (int c = quarter * chunk; c < n_step; c += 4 * chunk) {
+          __syncwarp();                                // converged for the warp-wide tcgen05.ld
+          float v[32];
+          const int acol = c;                                     // accumulator column
+          tmem_ld(tbase + (uint32_t)acol, v, chunk);
+          if (swiglu) {
+            float u[32];
+            tmem_ld(tbase + (uint32_t)(BN / 2 + acol), u, chunk);
+            tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = act_silu(v[i]) * u[i];
-        } else {
-          tmem_wait_ld();
-          if (p.epi == MOE_ACT_RELU) {
+            for (int i = 0; i < 32; ++i) v[i] = act_silu(v[i]) * u[i];
+          } else {
+            tmem_wait_ld();
+            if (p.epi == MOE_ACT_RELU) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = act_relu(v[i]);
-          } else if (p.epi == MOE_ACT_GELU) {
+              for (int i = 0; i < 32; ++i) v[i] = act_relu(v[i]);
+            } else if (p.epi == MOE_ACT_GELU) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = act_gelu(v[i]);
-          }
-        }
-        const int col = ncol0 + c;
-        if (p.out_f32) {
-          if (!row_ok) continue;
-          float* drow = static_cast<float*>(p.d) + (int64_t)part * p.rows_store * p.ld_d + grow * p.ld_d;
-          const bool vec = (p.ld_d & 3) == 0;
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            if (4 * q >= chunk) continue;
-            const int cc = col + 4 * q;
-            if (vec && cc + 4 <= p.N_out) {
-              *reinterpret_cast<float4*>(drow + cc) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-            } else {
-#pragma unroll
-              for (int i = 0; i < 4; ++i)
-                if (cc + i < p.N_out) drow[cc + i] = v[4 * q + i];
+              for (int i = 0; i < 32; ++i) v[i] = act_gelu(v[i]);
             }
           }
-        } else if (SCATTER) {
-          // the warp's 32 rows x 32 columns go through its staging buffer (same
-          // swizzle as below), then out row by row: lanes 4j..4j+3 write the 64
-          // bytes of one row, eight rows per store instruction
-          __syncwarp();                              // the previous chunk's reads are done
+          const int col = ncol0 + c;
+          if (p.out_f32) {
+            if (!row_ok) continue;
+            float* drow = static_cast<float*>(p.d) + (int64_t)part * p.rows_store * p.ld_d + grow * p.ld_d;
+            const bool vec = (p.ld_d & 3) == 0;
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            st_shared_v4(stage_out + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4),
-                         pack_bf16(sg * v[8 * q + 0], sg * v[8 * q + 1]), pack_bf16(sg * v[8 * q + 2], sg * v[8 * q + 3]),
-                         pack_bf16(sg * v[8 * q + 4], sg * v[8 * q + 5]), pack_bf16(sg * v[8 * q + 6], sg * v[8 * q + 7]));
-          __syncwarp();
-          const int j = lane & 3;
+            for (int q = 0; q < 8; ++q) {
+              if (4 * q >= chunk) continue;
+              const int cc = col + 4 * q;
+              if (vec && cc + 4 <= p.N_out) {
+                *reinterpret_cast<float4*>(drow + cc) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+              } else {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int r = 8 * q + (lane >> 2);
-            const int tr = __shfl_sync(0xffffffffu, st, r);
-            if (tr >= 0 && 8 * j < chunk && col + 8 * j < p.N_out) {
-              int4 val;
-              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                           : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
-                           : "r"(stage_out + r * 64 + ((j ^ ((r >> 1) & 3)) << 4)));
-              st_v4(p.sdst + (int64_t)tr * p.N_out + col + 8 * j, val);
+                for (int i = 0; i < 4; ++i)
+                  if (cc + i < p.N_out) drow[cc + i] = v[4 * q + i];
+              }
             }
-          }
-        } else {
-          // bf16: this warp's 32 rows x 32 columns go through its staging buffer
-          // (16-byte chunk j of row r at chunk j ^ ((r >> 1) & 3): the TMA 64-byte
-          // swizzle, bank-conflict free) and out with one TMA store of full lines.
-          if (lane == 0) bulk_wait_read0();          // the previous store has read the buffer
-          __syncwarp();
+          } else if (SCATTER) {
+            // the warp's 32 rows x 32 columns go through its staging buffer (same
+            // swizzle as below), then out row by row: lanes 4j..4j+3 write the 64
+            // bytes of one row, eight rows per store instruction
+            __syncwarp();                              // the previous chunk's reads are done
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            st_shared_v4(stage_out + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4),
-                         pack_bf16(v[8 * q + 0], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
-                         pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7]));
-          fence_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&p.tmD, stage_out, col, (int)(mt * BM + sub * 32));
-            bulk_commit();
+            for (int q = 0; q < 4; ++q)
+              st_shared_v4(stage_out + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4),
+                           pack_bf16(sg * v[8 * q + 0], sg * v[8 * q + 1]), pack_bf16(sg * v[8 * q + 2], sg * v[8 * q + 3]),
+                           pack_bf16(sg * v[8 * q + 4], sg * v[8 * q + 5]), pack_bf16(sg * v[8 * q + 6], sg * v[8 * q + 7]));
+            __syncwarp();
+            const int j = lane & 3;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int r = 8 * q + (lane >> 2);
+              const int tr = __shfl_sync(0xffffffffu, st, r);
+              if (tr >= 0 && 8 * j < chunk && col + 8 * j < p.N_out) {
+                int4 val;
+                asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
+                             : "r"(stage_out + r * 64 + ((j ^ ((r >> 1) & 3)) << 4)));
+                st_v4(p.sdst + (int64_t)tr * p.N_out + col + 8 * j, val);
+              }
+            }
+          } else {
+            // bf16: this warp's 32 rows x 32 columns go through its staging buffer
+            // (16-byte chunk j of row r at chunk j ^ ((r >> 1) & 3): the TMA 64-byte
+            // swizzle, bank-conflict free) and out with one TMA store of full lines.
+            if (lane == 0) bulk_wait_read0();          // the previous store has read the buffer
+            __syncwarp();
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              st_shared_v4(stage_out + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4),
+                           pack_bf16(v[8 * q + 0], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
+                           pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7]));
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&p.tmD, stage_out, col, (int)(mt * BM + sub * 32));
+              bulk_commit();
+            }
           }
         }
       }
       tc_fence_before();
       mbar_arrive(tempty0 + 8 * acc);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
-      if constexpr (ROUTE_EJ > 0) route_tile<ROUTE_EJ>(p, mt, ew, lane, staging, route_z);
     }
     if (lane == 0) bulk_wait0();                 // this warp's output stores are complete
     __syncwarp();
@@ -642,23 +800,21 @@ static bool make_map_d(CUtensorMap* m, const void* base, int64_t rows, int N) {
   return encode_cached(m, key);
 }
 
-template <bool GATHER, bool SCATTER, int ROUTE_EJ = 0>
+template <bool GATHER, bool SCATTER, int ROUTE_KM = 0>
 static cudaError_t launch_variant(KParams& k, int grid, cudaStream_t stream) {
-  auto kern = grouped_gemm_kernel<GATHER, SCATTER, ROUTE_EJ>;
+  auto kern = grouped_gemm_kernel<GATHER, SCATTER, ROUTE_KM>;
   cudaError_t e = ensure_smem(kern, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   launch_pdl(kern, grid, GATHER ? THREADS_GATHER : THREADS, SMEM_BYTES, stream, k);
   return cudaGetLastError();
 }
 
-static cudaError_t launch_kernel(KParams& k, int64_t max_tiles, cudaStream_t stream, int route_ej = 0) {
+static cudaError_t launch_kernel(KParams& k, int64_t max_tiles, cudaStream_t stream, int route_km = 0) {
   const int sms = sm_count();
   // grid: one CTA per SM, never more than the largest possible tile count
   const int grid = (int)(max_tiles < sms ? (max_tiles > 0 ? max_tiles : 1) : sms);
-  if (route_ej == 1) return launch_variant<false, false, 1>(k, grid, stream);
-  if (route_ej == 2) return launch_variant<false, false, 2>(k, grid, stream);
-  if (route_ej == 4) return launch_variant<false, false, 4>(k, grid, stream);
-  if (route_ej == 8) return launch_variant<false, false, 8>(k, grid, stream);
+  if (route_km == 8) return launch_variant<false, false, 8>(k, grid, stream);
+  if (route_km == 16) return launch_variant<false, false, 16>(k, grid, stream);
   const bool gather = k.gsrc != nullptr, scatter = k.sdst != nullptr;
   if (gather) return scatter ? launch_variant<true, true>(k, grid, stream) : launch_variant<true, false>(k, grid, stream);
   return scatter ? launch_variant<false, true>(k, grid, stream) : launch_variant<false, false>(k, grid, stream);
@@ -808,14 +964,14 @@ cudaError_t launch_router_gemm(const void* x, const float* wg, void* planes, boo
   const int nk = Hp / BK;
   k.k_split = (!fuse && tiles * 2 <= sm_count() && nk >= 4) ? 2 : 1;
   *parts = k.k_split;
-  int ej = 0;
+  int km = 0;
   if (fuse) {
     k.rp = *route;
     k.nblk = nblk;
-    ej = E <= 32 ? 1 : E <= 64 ? 2 : E <= 128 ? 4 : 8;
+    km = route->k <= 8 ? 8 : 16;
     *routed = true;
   }
-  return launch_kernel(k, tiles * k.k_split, stream, ej);
+  return launch_kernel(k, tiles * k.k_split, stream, km);
 }
 
 }  // namespace moe

@@ -78,3 +78,25 @@ def test_packed_router_rejects_fp32_layers_and_bad_args():
     with pytest.raises(B.MoeError) as ei:
         B.pack_router(wg)                                  # H % 8 != 0
     assert ei.value.code == B.MOE_EUNSUPPORTED
+
+
+@pytest.mark.parametrize("shape", [
+    synth.GSHARD_TOP2.replace(name="ties_k2", T=300, H=72, F=72, E=32, k=2),
+    synth.GSHARD_TOP2.replace(name="ties_k12_renorm", T=300, H=72, F=72, E=64, k=12),
+    synth.GSHARD_TOP2.replace(name="ties_k3_softmax", T=257, H=136, F=72, E=200, k=3, renorm=0),
+], ids=lambda s: s.name)
+def test_fused_router_exact_ties_and_wide_k(shape):
+    """The fused router ranks each token's experts by (larger logit, then smaller
+    index), the oracle's order: every third token has x = 0, so all its logits
+    are exactly 0 and it must take experts 0 .. k-1 with equal gates.  k = 12
+    runs the 16-wide selection; E = 200 leaves ragged column ranges."""
+    inp = synth.make_inputs(shape, seed=4, device="cuda")
+    inp["x"][::3] = 0
+    out = run_layer(shape, inp)
+    check_layer(shape, inp, out)
+    k = shape.k
+    ids = out["ids"][::3].cpu()
+    assert (ids == torch.arange(k, dtype=ids.dtype)).all()
+    gates = out["gates"][::3].cpu()
+    want = 1.0 / k if shape.renorm else 1.0 / shape.E
+    assert torch.allclose(gates, torch.full_like(gates, want), rtol=1e-6, atol=0)
