@@ -38,6 +38,11 @@ cudaError_t launch_router_gemm(const void* x, const float* wg, void* planes, boo
                                int64_t T, int H, int E, DevStatus* status, const RouterParams* route, int64_t nblk,
                                int* parts, bool* routed, cudaStream_t stream);
 cudaError_t launch_router(const RouterParams& p, bool bf16, cudaStream_t stream);
+// Routers with a long GEMM (E <= 256, T >= 256, H >= 2048): logits and routing
+// on pairs of SMs from precomputed planes (router_pair.cu).
+bool router_pair_fits(int64_t T, int H, int E);
+cudaError_t launch_router_pair(const void* x, const void* planes, int64_t T, int H, int E, DevStatus* status,
+                               const RouterParams& route, int64_t nblk, cudaStream_t stream);
 // term: E doubles of scratch followed by one unsigned ticket counter.
 // zsum_part (or null): per-CTA sums of lse^2; aux[1] = z_coef * their mean.
 cudaError_t launch_aux(const float* psum_part, const int32_t* cnt_part, const float* zsum_part, int nblk, int E,

@@ -48,6 +48,14 @@ CASES = {
     "wide_e300": synth.GSHARD_TOP2.replace(name="wide_e300", T=400, H=72, F=136, E=300, k=2),
     "sigmoid_zloss": synth.SWITCH_TOP1.replace(name="sigmoid_zloss", T=517, H=96, F=136, E=32, k=2,
                                                score=synth.SCORE_SIGMOID_TOPK, z_coef=1e-3, bias_row0=0.0),
+    # H >= 2048: the router runs on pairs of SMs (256 tokens per pair tile; T
+    # not a multiple of 256 leaves the last pair's odd CTA without tokens)
+    "pair_e256_k8_skew": synth.WIDEEP_DROPLESS.replace(name="pair_e256_k8_skew", T=777, H=2048, F=72, E=256, k=8,
+                                                       n_shared=0),
+    "pair_e200_sigmoid_zloss": synth.SWITCH_TOP1.replace(name="pair_e200_sigmoid_zloss", T=300, H=2112, F=72,
+                                                         E=200, k=2, score=synth.SCORE_SIGMOID_TOPK, z_coef=1e-3,
+                                                         bias_row0=0.0),
+    "pair_e16_k12": synth.GSHARD_TOP2.replace(name="pair_e16_k12", T=513, H=2048, F=72, E=16, k=12),
 }
 
 
