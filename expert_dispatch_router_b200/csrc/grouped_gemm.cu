@@ -588,6 +588,9 @@ static cudaError_t launch_kernel(KParams& k, int64_t max_tiles, cudaStream_t str
   const int sms = sm_count();
   // grid: one CTA per SM, never more than the largest possible tile count
   const int grid = (int)(max_tiles < sms ? (max_tiles > 0 ? max_tiles : 1) : sms);
+  if (route_km == 1) return launch_variant<false, false, 1>(k, grid, stream);
+  if (route_km == 2) return launch_variant<false, false, 2>(k, grid, stream);
+  if (route_km == 4) return launch_variant<false, false, 4>(k, grid, stream);
   if (route_km == 8) return launch_variant<false, false, 8>(k, grid, stream);
   if (route_km == 16) return launch_variant<false, false, 16>(k, grid, stream);
   const bool gather = k.gsrc != nullptr, scatter = k.sdst != nullptr;
@@ -748,7 +751,7 @@ cudaError_t launch_router_gemm(const void* x, const float* wg, void* planes, boo
   if (fuse) {
     k.rp = *route;
     k.nblk = nblk;
-    km = route->k <= 8 ? 8 : 16;
+    km = route_km_of(route->k);
     *routed = true;
   }
   return launch_kernel(k, tiles * k.k_split, stream, km);

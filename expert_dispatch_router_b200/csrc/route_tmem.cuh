@@ -21,6 +21,29 @@ constexpr int kRouteTokens = 128;               // tokens of one router tile (TM
 constexpr int kRouteThreads = 512;              // the 16 epilogue warps
 constexpr int kRouteStagingBytes = 512 * 4 * 3 + 1024 * 8 + 1024 * 4 + 256 * 4 + 16;
 
+// 8 columns of this warp's 32 lanes from / to tensor memory (one load shape:
+// the routing's code runs once per tile and is fetched cold).
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&v)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+               :: "r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+                  "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+                  "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7]))
+               : "memory");
+}
+
+// The routing's top-k bound for k choices: one instantiation each for k = 1,
+// 2, <= 4, <= 8 and <= 16 (the sorted key lists live in registers).
+inline int route_km_of(int k) { return k <= 1 ? 1 : k <= 2 ? 2 : k <= 4 ? 4 : k <= 8 ? 8 : 16; }
+
 __device__ __forceinline__ void route_bar() {
   asm volatile("bar.sync 1, %0;" :: "r"(kRouteThreads) : "memory");
 }
@@ -58,7 +81,6 @@ __device__ __forceinline__ void route_tile_tmem(const RouterParams& rp, int64_t 
   const int q4 = (ncols + 3) / 4;
   const int W = q4 <= 8 ? 8 : q4 <= 16 ? 16 : q4 <= 32 ? 32 : 64;
   const int c0 = quarter * W;
-  const int ch = W >= 32 ? 32 : W;                                 // columns per TMEM access
   const bool sigmoid = rp.score == MOE_SCORE_SIGMOID_TOPK;
   float* xmax = reinterpret_cast<float*>(staging);                 // [4 sub][4 quarter][32]
   float* xsum = xmax + 512;
@@ -76,14 +98,13 @@ __device__ __forceinline__ void route_tile_tmem(const RouterParams& rp, int64_t 
 #pragma unroll
   for (int i = 0; i < KM; ++i) key[i] = 0ull;
   float m = -INFINITY;
-  for (int cc = 0; cc < W; cc += ch) {
-    float v[32];
-    tmem_ld(tacc + (uint32_t)(c0 + cc), v, ch);
-    tmem_wait_ld();
+#pragma unroll 1
+  for (int cc = 0; cc < W; cc += 8) {
+    float v[8];
+    tmem_ld8(tacc + (uint32_t)(c0 + cc), v);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
+    for (int j = 0; j < 8; ++j) {
       const int e = c0 + cc + j;
-      if (j >= ch) break;
       if (tv && e < E) {
         if (rp.logit_add != nullptr) v[j] += rp.logit_add[t * E + e];
         if (rp.logits_out != nullptr) rp.logits_out[t * E + e] = v[j];
@@ -98,7 +119,7 @@ __device__ __forceinline__ void route_tile_tmem(const RouterParams& rp, int64_t 
           }
       }
     }
-    if (rp.logit_add != nullptr) tmem_st(tacc + (uint32_t)(c0 + cc), v, ch);
+    if (rp.logit_add != nullptr) tmem_st8(tacc + (uint32_t)(c0 + cc), v);
   }
   if (rp.logit_add != nullptr) tmem_wait_st();
   xmax[tid] = m;
@@ -110,13 +131,12 @@ __device__ __forceinline__ void route_tile_tmem(const RouterParams& rp, int64_t 
 
   // 2. sums of exp(l - m) (and of sigmoid(l)) over the whole token
   float s = 0.0f, ss = 0.0f;
-  for (int cc = 0; cc < W; cc += ch) {
-    float v[32];
-    tmem_ld(tacc + (uint32_t)(c0 + cc), v, ch);
-    tmem_wait_ld();
+#pragma unroll 1
+  for (int cc = 0; cc < W; cc += 8) {
+    float v[8];
+    tmem_ld8(tacc + (uint32_t)(c0 + cc), v);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      if (j >= ch) break;
+    for (int j = 0; j < 8; ++j) {
       if (tv && c0 + cc + j < E) {
         s += expf(v[j] - m);
         if (sigmoid) ss += 1.0f / (1.0f + expf(-v[j]));
@@ -209,13 +229,12 @@ __device__ __forceinline__ void route_tile_tmem(const RouterParams& rp, int64_t 
   // 6. each expert's probability sum over the tile's tokens
   if (rp.psum_part != nullptr) {
     const float inv = 1.0f / (sigmoid ? ss : s);
-    for (int cc = 0; cc < W; cc += ch) {
-      float v[32];
-      tmem_ld(tacc + (uint32_t)(c0 + cc), v, ch);
-      tmem_wait_ld();
+#pragma unroll 1
+    for (int cc = 0; cc < W; cc += 8) {
+      float v[8];
+      tmem_ld8(tacc + (uint32_t)(c0 + cc), v);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        if (j >= ch) break;
+      for (int j = 0; j < 8; ++j) {
         const int e = c0 + cc + j;
         float pe = 0.0f;
         if (tv && e < E) pe = (sigmoid ? 1.0f / (1.0f + expf(-v[j])) : expf(v[j] - m)) * inv;

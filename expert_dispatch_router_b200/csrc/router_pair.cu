@@ -345,7 +345,13 @@ cudaError_t launch_router_pair(const void* x, const void* planes, int64_t T, int
   k.T = T;
   k.Hp = Hp;
   const int64_t n_tiles = (T + 2 * HALF - 1) / (2 * HALF);
-  return route.k <= 8 ? launch_km<8>(k, n_tiles, stream) : launch_km<16>(k, n_tiles, stream);
+  switch (route_km_of(route.k)) {
+    case 1: return launch_km<1>(k, n_tiles, stream);
+    case 2: return launch_km<2>(k, n_tiles, stream);
+    case 4: return launch_km<4>(k, n_tiles, stream);
+    case 8: return launch_km<8>(k, n_tiles, stream);
+    default: return launch_km<16>(k, n_tiles, stream);
+  }
 }
 
 }  // namespace moe
