@@ -117,6 +117,7 @@ struct SlotParams {
   const float* psum_part;   // [nblk_router, E] or null
   const int32_t* cnt_part;  // [nblk_router, E] selection counts, or null: count the dispatched ids
   int nblk_router;
+  int part_stride;          // only every part_stride-th partial row is non-zero (0 or 1: all)
   double* aux_term;         // [E]
   float* aux;               // [1], or [2] with the z-loss in aux[1]
   float aux_alpha;

@@ -221,6 +221,10 @@ int run_slots(const moe_cfg* c, const Layout& L, const int32_t* ids, const float
   if (aux != nullptr) {            // fuse the aux loss into the slot kernels
     p.psum_part = at<float>(ws, L.psum);
     p.nblk_router = L.nblk_router;
+    // bf16 layers with E <= 256 are routed from the router GEMM's accumulator,
+    // 128 tokens a tile: one partial row in every 128 / router_tile_tokens
+    // holds the tile's sums and the rows between hold zeros
+    p.part_stride = (c->dtype == MOE_DTYPE_BF16 && c->E <= 256) ? 128 / router_tile_tokens(c->E) : 1;
     p.aux_term = at<double>(ws, L.term);
     p.aux = aux;
     p.aux_alpha = c->aux_alpha;

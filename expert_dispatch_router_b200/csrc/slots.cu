@@ -20,6 +20,9 @@
 //                32-assignment step with match_any, carry per-warp running counts,
 //                prefix them over the warps in order, and add the chunk base.
 // Total metadata traffic is O(T*k + E*chunks); nothing scales with C.
+// Layers whose assignments fit one resident CTA per SM (1024 assignments each)
+// and that use the "position" policy or none run the same steps in one launch
+// with two grid barriers (slot_fused_kernel below).
 //
 // "probs" policy (same section: drop the lowest-probability assignments): the
 // rank kernel lists every assignment of an over-full expert, in arrival order,
@@ -417,8 +420,272 @@ __global__ void __launch_bounds__(kSelThreads) slot_select_kernel(SlotParams p) 
   }
 }
 
+// ---------------------------------------------------------------- one launch
+// The same assignment in one launch, for the "position" policy and dropless
+// layers whose assignments fit one resident CTA per SM at kFuseSpan each.
+//   phase 1: CTA c ranks its span warp by warp (match_any, as the rank kernel
+//            does) and publishes its per-expert totals at chunk_cnt[e][c]; its
+//            warps also sum the router's partials of the experts it owns
+//            (e = c, c + G, ...: a warp each);
+//   grid barrier;
+//   phase 2: the owner warp of expert e scans chunk_cnt[e][*] in place into the
+//            spans' bases and writes the expert's count, kept count and aux term;
+//   grid barrier;
+//   phase 3: every CTA reads its base and the kept count of every expert, lays
+//            out the 128-padded row blocks (the same scan in every CTA) and
+//            writes its slots and row_token entries; the owner CTAs write the
+//            padding rows, every CTA a share of the shared block, and CTA 0 the
+//            offsets and the aux loss.
+// The grid barriers are one counter with bounded waits.  Every CTA is resident
+// at once: the grid is at most one CTA per SM and no CTA waits on a later
+// kernel.  Slots, counts, offsets and row_token equal the three-kernel path's
+// bit for bit (integers); the aux loss is summed in this path's own fixed order.
+constexpr int kFuseSteps = 4;                                  // 32-assignment steps per warp
+constexpr int kFuseSpan = kSlotWarps * 32 * kFuseSteps;        // assignments per CTA
+constexpr int kFuseMaxPer = 5;                                 // chunk counts per lane in the scan (G <= 160)
+
+// Thread 0 of each CTA: arrive at grid barrier number `n` (1, 2, ...) and wait
+// until all G CTAs have arrived (bounded; false and MOE_ETIMEOUT in the status
+// word if the wait runs out).
+__device__ __forceinline__ bool slot_grid_barrier(unsigned* ctr, unsigned G, unsigned n, DevStatus* st) {
+  __threadfence();
+  atomicAdd(ctr, 1u);
+  const long long t0 = clock64();
+  unsigned v = 0;
+  while (true) {
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    if (v >= n * G) return true;
+    if (clock64() - t0 > kWaitCycles) {
+      set_status(st, MOE_ETIMEOUT, 3);
+      return false;
+    }
+    __nanosleep(64);
+  }
+}
+
+__global__ void __launch_bounds__(kSlotThreads) slot_fused_kernel(SlotParams p, int G) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ int fsm[];
+  const int E = p.E;
+  int* wcnt = fsm;                          // [warps][E]: counts, then exclusive prefixes over the warps
+  int* s_base = wcnt + kSlotWarps * E;      // [E] this span's base per expert
+  int* s_kept = s_base + E;                 // [E]
+  int* s_off = s_kept + E;                  // [E + 2]
+  __shared__ int sh[kSlotWarps];
+  __shared__ double red[kSlotWarps];
+  __shared__ int s_ok;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, c = blockIdx.x;
+  const int64_t A = p.T * p.k;
+  const bool aux = p.aux != nullptr;
+  for (int i = tid; i < kSlotWarps * E; i += kSlotThreads) wcnt[i] = 0;
+  __syncthreads();
+
+  // phase 1: ranks inside each warp's 128 assignments (in sequence order)
+  const int64_t a_warp = (int64_t)c * kFuseSpan + (int64_t)warp * (kFuseSteps * 32);
+  const unsigned lt_mask = (1u << lane) - 1u;
+  int local[kFuseSteps], expert[kFuseSteps];
+#pragma unroll
+  for (int s = 0; s < kFuseSteps; ++s) {
+    const int64_t a = a_warp + s * 32 + lane;
+    int e = load_assignment(p, a, A);          // -1 past the end
+    if (a < A && (e < 0 || e >= E)) {
+      if (e != -1) set_status(p.status, MOE_EDEVICE, 1);   // -1: a choice that is not dispatched
+      e = -2;
+    }
+    expert[s] = e;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    int prior = 0;
+    if (e >= 0) prior = wcnt[warp * E + e];
+    local[s] = prior + __popc(peers & lt_mask);
+    __syncwarp();
+    if (e >= 0 && lane == __ffs(peers) - 1) wcnt[warp * E + e] = prior + __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += kSlotThreads) {
+    int run = 0;
+#pragma unroll
+    for (int w = 0; w < kSlotWarps; ++w) {
+      const int v = wcnt[w * E + e];
+      wcnt[w * E + e] = run;
+      run += v;
+    }
+    __stcg(p.chunk_cnt + (int64_t)e * G + c, run);
+  }
+  if (aux) {
+    // P_e / T of the experts this CTA owns (and, with selection counts, the
+    // whole term f_e * P_e): lanes stride the router's partial rows in fp64
+    // (rows between the strided ones hold zeros), then a fixed butterfly
+    const int rs = p.part_stride > 1 ? p.part_stride : 1;
+    for (int e = c + G * warp; e < E; e += G * kSlotWarps) {
+      double ps = 0.0;
+      long long cs = 0;
+#pragma unroll 4
+      for (int b = lane * rs; b < p.nblk_router; b += 32 * rs) {
+        ps += (double)__ldcg(p.psum_part + (int64_t)b * E + e);
+        if (p.cnt_part != nullptr) cs += __ldcg(p.cnt_part + (int64_t)b * E + e);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        ps += __shfl_xor_sync(0xffffffffu, ps, o);
+        cs += __shfl_xor_sync(0xffffffffu, cs, o);
+      }
+      const double pt = ps / (double)p.T;
+      if (lane == 0) __stcg(p.aux_term + e, p.cnt_part != nullptr ? ((double)cs / ((double)p.T * p.k)) * pt : pt);
+    }
+    if (c == 0 && warp == kSlotWarps - 1 && p.zsum_part != nullptr) {
+      // z-loss = coef * mean_t lse_t^2 from the router's per-block sums
+      double z = 0.0;
+      for (int b = lane * rs; b < p.nblk_router; b += 32 * rs) z += (double)__ldcg(p.zsum_part + b);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+      if (lane == 0) p.aux[1] = (float)((double)p.z_coef * z / (double)p.T);
+    }
+  }
+  __syncthreads();
+  if (tid == 0) s_ok = slot_grid_barrier(p.ticket, (unsigned)G, 1u, p.status) ? 1 : 0;
+  __syncthreads();
+  if (!s_ok) return;
+
+  // phase 2: the owner warp scans expert e's span totals into bases, in place;
+  // lane l holds the contiguous entries [l * per, (l + 1) * per)
+  {
+    const int per = (G + 31) / 32;
+    for (int e = c + G * warp; e < E; e += G * kSlotWarps) {
+      int* row = p.chunk_cnt + (int64_t)e * G;
+      int v[kFuseMaxPer];
+      int mine = 0;
+#pragma unroll
+      for (int i = 0; i < kFuseMaxPer; ++i) {
+        const int j = lane * per + i;
+        v[i] = (i < per && j < G) ? __ldcg(row + j) : 0;
+        mine += v[i];
+      }
+      int incl = mine;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int run = incl - mine;
+#pragma unroll
+      for (int i = 0; i < kFuseMaxPer; ++i) {
+        const int j = lane * per + i;
+        if (i < per && j < G) __stcg(row + j, run);
+        run += v[i];
+      }
+      const int tot = __shfl_sync(0xffffffffu, incl, 31);
+      if (lane == 0) {
+        const int kept = p.capacity < 0 ? tot : (int)min((int64_t)tot, p.capacity);
+        p.expert_count[e] = tot;
+        __stcg(p.kept_count + e, kept);
+        if (aux && p.T > 0 && p.cnt_part == nullptr)
+          __stcg(p.aux_term + e, ((double)tot / ((double)p.T * p.k)) * __ldcg(p.aux_term + e));
+      }
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    s_ok = slot_grid_barrier(p.ticket, (unsigned)G, 2u, p.status) ? 1 : 0;
+    // the last CTA to leave re-arms the counter for the next call
+    if (s_ok && atomicAdd(p.ticket, 1u) == 3u * G - 1u) atomicExch(p.ticket, 0u);
+  }
+  __syncthreads();
+  if (!s_ok) return;
+
+  // phase 3: this span's bases, every expert's kept count, the row blocks
+  for (int e = tid; e < E; e += kSlotThreads) {
+    s_base[e] = __ldcg(p.chunk_cnt + (int64_t)e * G + c);
+    s_kept[e] = __ldcg(p.kept_count + e);
+  }
+  __syncthreads();
+  {
+    constexpr int kPer = (kMaxE + kSlotThreads - 1) / kSlotThreads;   // experts per thread, contiguous
+    const int e0 = tid * kPer;
+    int loc = 0;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i)
+      if (e0 + i < E) loc += (int)round_up(s_kept[e0 + i], kRowPad);
+    int routed;
+    int run = block_scan_excl<kSlotWarps>(loc, sh, routed);
+#pragma unroll
+    for (int i = 0; i < kPer; ++i)
+      if (e0 + i < E) {
+        s_off[e0 + i] = run;
+        run += (int)round_up(s_kept[e0 + i], kRowPad);
+      }
+    if (tid == 0) {
+      s_off[E] = routed;
+      const int64_t end = routed + (p.n_shared ? round_up(p.T, kRowPad) : 0);
+      s_off[E + 1] = (int)end;
+      if (c == 0 && end > p.rows_max) set_status(p.status, MOE_EDEVICE, 2);
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int s = 0; s < kFuseSteps; ++s) {
+    const int e = expert[s];
+    if (e == -1) continue;
+    const int64_t a = a_warp + s * 32 + lane;
+    const int64_t r = a / p.T, t = a - r * p.T;
+    if (e < 0) { p.slot[t * p.k + r] = -1; continue; }
+    const int pos = s_base[e] + wcnt[warp * E + e] + local[s];
+    const bool kept = p.capacity < 0 || pos < p.capacity;
+    p.slot[t * p.k + r] = kept ? pos : -1;
+    const int64_t row = (int64_t)s_off[e] + pos;
+    if (kept && row < p.rows_max) p.row_token[row] = (int)t;
+  }
+  // padding rows of the experts this CTA owns -> -1; a share of the shared block
+  for (int e = c + G * warp; e < E; e += G * kSlotWarps) {
+    const int start = s_off[e] + s_kept[e], stop = s_off[e + 1];
+    for (int r = start + lane; r < stop; r += 32) p.row_token[r] = -1;
+  }
+  if (p.n_shared) {
+    const int64_t s0 = s_off[E], n = round_up(p.T, kRowPad);
+    for (int64_t i = (int64_t)c * kSlotThreads + tid; i < n; i += (int64_t)G * kSlotThreads)
+      if (s0 + i < p.rows_max) p.row_token[s0 + i] = i < p.T ? (int)i : -1;
+  }
+  if (c != 0) return;
+  for (int i = tid; i < E + 2; i += kSlotThreads) p.expert_offset[i] = s_off[i];
+  if (aux) {
+    // aux loss = alpha * E * sum_e f_e * P_e: thread-strided sums in expert
+    // order, a fixed butterfly per warp, then the warps in order
+    double v = 0.0;
+    if (p.T > 0)
+      for (int e = tid; e < E; e += kSlotThreads) v += __ldcg(p.aux_term + e);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    if (tid == 0) {
+      double s = 0.0;
+#pragma unroll
+      for (int w = 0; w < kSlotWarps; ++w) s += red[w];
+      p.aux[0] = (float)((double)p.aux_alpha * (double)E * s);
+    }
+  }
+}
+
+// The one-launch path applies when every CTA can be resident at once (one per
+// SM at most) and no "probs" lists are needed.
+static int fused_slot_grid(const SlotParams& p) {
+  const int64_t A = p.T * p.k;
+  if (A <= 0 || p.gates != nullptr) return 0;
+  const int64_t G = (A + kFuseSpan - 1) / kFuseSpan;
+  if (G > sm_count() || G > 32 * kFuseMaxPer) return 0;
+  return (int)G;
+}
+
 cudaError_t launch_slots(const SlotParams& p, cudaStream_t stream) {
   const int64_t A = p.T * p.k;
+  if (const int G = fused_slot_grid(p)) {
+    const size_t sm = ((size_t)(kSlotWarps + 3) * p.E + 2) * sizeof(int);   // wcnt, base, kept, off
+    cudaError_t e = ensure_smem(slot_fused_kernel, sm);
+    if (e != cudaSuccess) return e;
+    launch_pdl(slot_fused_kernel, G, kSlotThreads, sm, stream, p, G);
+    return cudaGetLastError();
+  }
   const int nchunk = (int)((A + kSlotChunk - 1) / kSlotChunk);
   if (A > 0) launch_pdl(slot_count_kernel, nchunk, kSlotThreads, p.E * sizeof(int), stream, p, nchunk);
   // one CTA per expert; the last one to finish lays out the row blocks

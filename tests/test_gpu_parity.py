@@ -229,7 +229,10 @@ def test_slots_every_pattern_tiny():
 
 
 @pytest.mark.parametrize("E,k,T,mode", [(64, 1, 5000, 0), (12, 4, 32768, 0), (256, 8, 16384, 1), (1024, 3, 7001, 1),
-                                         (7, 7, 2049, 0), (1, 1, 3000, 0)])
+                                         (7, 7, 2049, 0), (1, 1, 3000, 0),
+                                         # beyond the one-launch path: more than 148 CTAs of 1024
+                                         # assignments, and E * CTAs above its limit of 32768
+                                         (64, 2, 80000, 0), (1024, 2, 20000, 1)])
 def test_slots_random_large(E, k, T, mode):
     rng = np.random.default_rng(E * 7 + k)
     w = rng.dirichlet(np.ones(E) * 0.5)
