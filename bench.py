@@ -284,15 +284,15 @@ def traffic_from_profiles(workload: str, kernel: str):
 def kernel_source(stage: str, workload: str = None) -> str:
     """The source file of the kernel a stage runs: the expert contractions of
     bf16 layers with T*k > 256*E run on SM pairs (grouped_gemm_tn.cu); the bf16
-    router's logits GEMM (with the routing in its epilogue) is in grouped_gemm.cu,
-    or on SM pairs in router_pair.cu for H >= 2048."""
+    router's logits GEMM (with the routing in its epilogue) runs on SM pairs in
+    router_pair.cu for E <= 256 and T >= 256, else in grouped_gemm.cu."""
     from expert_dispatch_router_b200 import synth
     shape = synth.WORKLOADS.get(workload) if workload else None
     bf16 = shape is not None and shape.dtype == 1
     if stage in ("ffn_gemm1", "ffn_gemm2") and bf16 and shape.T * shape.k > 256 * shape.E:
         return "grouped_gemm_tn.cu"
     if stage == "router" and bf16:
-        pair = shape.E <= 256 and shape.T >= 256 and -(-shape.H // 64) >= 32
+        pair = shape.E <= 256 and shape.T >= 256
         return "router_pair.cu" if pair else "grouped_gemm.cu"
     return {"router": "router.cu", "dispatch": "permute.cu", "combine": "permute.cu",
             "ffn_gemm1": "grouped_gemm.cu", "ffn_gemm2": "grouped_gemm.cu",

@@ -38,8 +38,8 @@ cudaError_t launch_router_gemm(const void* x, const float* wg, void* planes, boo
                                int64_t T, int H, int E, DevStatus* status, const RouterParams* route, int64_t nblk,
                                int* parts, bool* routed, cudaStream_t stream);
 cudaError_t launch_router(const RouterParams& p, bool bf16, cudaStream_t stream);
-// Routers with a long GEMM (E <= 256, T >= 256, H >= 2048): logits and routing
-// on pairs of SMs from precomputed planes (router_pair.cu).
+// Routers with E <= 256 and T >= 256: logits and routing on pairs of SMs from
+// precomputed planes (router_pair.cu).
 bool router_pair_fits(int64_t T, int H, int E);
 cudaError_t launch_router_pair(const void* x, const void* planes, int64_t T, int H, int E, DevStatus* status,
                                const RouterParams& route, int64_t nblk, cudaStream_t stream);

@@ -1,6 +1,6 @@
 // Router logits and routing on pairs of SMs (tcgen05.mma.cta_group::2), for
-// routers whose GEMM is long (H >= 2048): 256 tokens per pair tile, each CTA
-// holding 128 tokens (A) and half of the experts of every weight plane (B).
+// every router with E <= 256 and at least 256 tokens: 256 tokens per pair tile,
+// each CTA holding 128 tokens (A) and half of the experts of every weight plane (B).
 //
 // Method: the router of an MoE layer ("Expert-parallel MoE training"
 // explainer, router section: a linear gate with E outputs in fp32; "Switch
@@ -11,14 +11,16 @@
 // step, the A chunk by the hi, mid and lo planes in that order: the order of
 // the one-SM router (grouped_gemm.cu), so the logits are bitwise the same.
 //
-// Why a pair: on one SM a 128-token tile loads its A chunk and all E rows of
-// every plane per k step (16 + 3 * 32 KB at E = 256) for 3 * 2*128*256*64
-// flops, about twice what the L2 feeds per clock.  A pair shares the plane
-// rows: each CTA loads its own 128 tokens and E/2 rows of each plane (16 +
-// 3 * 16 KB), and one MMA instruction from the even CTA writes every CTA's 128
-// rows x E columns into that CTA's tensor memory, so each CTA still holds its
-// tokens' complete logits and routes them as the one-SM router does
-// (route_tmem.cuh).
+// Why a pair: an SM takes in its operands at a fixed rate (about 45 GB/s on
+// a B200 SM, from L2 or HBM alike), so the router's k loop costs what its CTA
+// loads.  On one SM a 128-token tile loads its A chunk and all E rows of every
+// plane per k step (16 + 3 * 32 KB at E = 256; 16 + 3 * 8 KB at E = 64).  A
+// pair shares the plane rows: each CTA loads its own 128 tokens and E/2 rows
+// of each plane, and one MMA instruction from the even CTA writes every CTA's
+// 128 rows x E columns into that CTA's tensor memory, so each CTA still holds
+// its tokens' complete logits and routes them as the one-SM router does
+// (route_tmem.cuh).  The CTA count is the one-SM router's (two CTAs per
+// 256 tokens), each loading less.
 //
 // Roles per CTA (576 threads): warp 0 issues the TMA loads (both CTAs; every
 // copy completes on the even CTA's full barrier, armed with both CTAs'
@@ -325,7 +327,7 @@ static cudaError_t launch_km(const RParams& k, int64_t n_tiles, cudaStream_t str
 }  // namespace rpair
 
 bool router_pair_fits(int64_t T, int H, int E) {
-  return E <= 256 && T >= 256 && router_plane_width(H) >= 32 * rpair::BK;
+  return E <= 256 && T >= 256 && router_plane_width(H) >= rpair::BK;
 }
 
 cudaError_t launch_router_pair(const void* x, const void* planes, int64_t T, int H, int E, DevStatus* status,

@@ -56,6 +56,11 @@ CASES = {
                                                          E=200, k=2, score=synth.SCORE_SIGMOID_TOPK, z_coef=1e-3,
                                                          bias_row0=0.0),
     "pair_e16_k12": synth.GSHARD_TOP2.replace(name="pair_e16_k12", T=513, H=2048, F=72, E=16, k=12),
+    # fewer than 256 tokens: the one-SM router (128-token tiles, routing from TMEM)
+    "onesm_e64_k2": synth.GSHARD_TOP2.replace(name="onesm_e64_k2", T=200, H=200, F=72, E=64, k=2),
+    "onesm_e256_k8_skew": synth.WIDEEP_DROPLESS.replace(name="onesm_e256_k8_skew", T=255, H=136, F=72, E=256,
+                                                        k=8, n_shared=0),
+    "onesm_e12_k4_zloss": synth.DS_HIGHK.replace(name="onesm_e12_k4_zloss", T=129, H=64, F=72, z_coef=1e-3),
 }
 
 
@@ -92,6 +97,7 @@ def test_packed_router_rejects_fp32_layers_and_bad_args():
     synth.GSHARD_TOP2.replace(name="ties_k2", T=300, H=72, F=72, E=32, k=2),
     synth.GSHARD_TOP2.replace(name="ties_k12_renorm", T=300, H=72, F=72, E=64, k=12),
     synth.GSHARD_TOP2.replace(name="ties_k3_softmax", T=257, H=136, F=72, E=200, k=3, renorm=0),
+    synth.GSHARD_TOP2.replace(name="ties_onesm_k4", T=250, H=72, F=72, E=48, k=4),
 ], ids=lambda s: s.name)
 def test_fused_router_exact_ties_and_wide_k(shape):
     """The fused router ranks each token's experts by (larger logit, then smaller
