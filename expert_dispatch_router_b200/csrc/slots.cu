@@ -431,6 +431,9 @@ __global__ void __launch_bounds__(kSelThreads) slot_select_kernel(SlotParams p) 
 //   phase 2: the owner warp of expert e scans chunk_cnt[e][*] in place into the
 //            spans' bases and writes the expert's count, kept count and aux term;
 //   grid barrier;
+//   (with E * G <= kFuseSmallTotals every CTA instead reads all span totals
+//   after the first barrier and adds up those before its span and all of
+//   them, and the second barrier goes);
 //   phase 3: every CTA reads its base and the kept count of every expert, lays
 //            out the 128-padded row blocks (the same scan in every CTA) and
 //            writes its slots and row_token entries; the owner CTAs write the
@@ -443,6 +446,7 @@ __global__ void __launch_bounds__(kSelThreads) slot_select_kernel(SlotParams p) 
 constexpr int kFuseSteps = 4;                                  // 32-assignment steps per warp
 constexpr int kFuseSpan = kSlotWarps * 32 * kFuseSteps;        // assignments per CTA
 constexpr int kFuseMaxPer = 5;                                 // chunk counts per lane in the scan (G <= 160)
+constexpr int kFuseSmallTotals = 4096;                         // E * G read by every CTA on the one-barrier path
 
 // Thread 0 of each CTA: arrive at grid barrier number `n` (1, 2, ...) and wait
 // until all G CTAs have arrived (bounded; false and MOE_ETIMEOUT in the status
@@ -471,7 +475,8 @@ __global__ void __launch_bounds__(kSlotThreads) slot_fused_kernel(SlotParams p, 
   int* wcnt = fsm;                          // [warps][E]: counts, then exclusive prefixes over the warps
   int* s_base = wcnt + kSlotWarps * E;      // [E] this span's base per expert
   int* s_kept = s_base + E;                 // [E]
-  int* s_off = s_kept + E;                  // [E + 2]
+  int* s_tot = s_kept + E;                  // [E] (one-barrier path)
+  int* s_off = s_tot + E;                   // [E + 2]
   __shared__ int sh[kSlotWarps];
   __shared__ double red[kSlotWarps];
   __shared__ int s_ok;
@@ -479,6 +484,10 @@ __global__ void __launch_bounds__(kSlotThreads) slot_fused_kernel(SlotParams p, 
   const int64_t A = p.T * p.k;
   const bool aux = p.aux != nullptr;
   for (int i = tid; i < kSlotWarps * E; i += kSlotThreads) wcnt[i] = 0;
+  for (int i = tid; i < E; i += kSlotThreads) {
+    s_base[i] = 0;
+    s_tot[i] = 0;
+  }
   __syncthreads();
 
   // phase 1: ranks inside each warp's 128 assignments (in sequence order)
@@ -543,11 +552,50 @@ __global__ void __launch_bounds__(kSlotThreads) slot_fused_kernel(SlotParams p, 
       if (lane == 0) p.aux[1] = (float)((double)p.z_coef * z / (double)p.T);
     }
   }
+  // with few span totals (E * G <= kFuseSmallTotals) every CTA reads them all
+  // after the first barrier, and the second barrier is not needed
+  const bool one = (int64_t)E * G <= kFuseSmallTotals;
   __syncthreads();
-  if (tid == 0) s_ok = slot_grid_barrier(p.ticket, (unsigned)G, 1u, p.status) ? 1 : 0;
+  if (tid == 0) {
+    s_ok = slot_grid_barrier(p.ticket, (unsigned)G, 1u, p.status) ? 1 : 0;
+    // the last CTA to leave re-arms the counter for the next call
+    if (one && s_ok && atomicAdd(p.ticket, 1u) == 2u * G - 1u) atomicExch(p.ticket, 0u);
+  }
   __syncthreads();
   if (!s_ok) return;
 
+  if (one) {
+    // all E * G span totals at once (coalesced, one round trip), added into this
+    // span's bases (spans before it) and the experts' totals with integer
+    // shared-memory atomics (zeroed in phase 1; any order gives the same sums)
+    constexpr int kPerThread = kFuseSmallTotals / kSlotThreads;
+    const int n = E * G;
+    int v[kPerThread];
+#pragma unroll
+    for (int m = 0; m < kPerThread; ++m) {
+      const int idx = m * kSlotThreads + tid;
+      v[m] = idx < n ? __ldcg(p.chunk_cnt + idx) : 0;
+    }
+#pragma unroll
+    for (int m = 0; m < kPerThread; ++m) {
+      const int idx = m * kSlotThreads + tid;
+      if (idx < n && v[m] != 0) {
+        const int e = idx / G, j = idx - e * G;
+        atomicAdd(s_tot + e, v[m]);
+        if (j < c) atomicAdd(s_base + e, v[m]);
+      }
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += kSlotThreads) {
+      const int all = s_tot[e];
+      const int kept = p.capacity < 0 ? all : (int)min((int64_t)all, p.capacity);
+      s_kept[e] = kept;
+      if (c == 0) {
+        p.expert_count[e] = all;
+        p.kept_count[e] = kept;
+      }
+    }
+  } else {
   // phase 2: the owner warp scans expert e's span totals into bases, in place;
   // lane l holds the contiguous entries [l * per, (l + 1) * per)
   {
@@ -598,6 +646,7 @@ __global__ void __launch_bounds__(kSlotThreads) slot_fused_kernel(SlotParams p, 
   for (int e = tid; e < E; e += kSlotThreads) {
     s_base[e] = __ldcg(p.chunk_cnt + (int64_t)e * G + c);
     s_kept[e] = __ldcg(p.kept_count + e);
+  }
   }
   __syncthreads();
   {
@@ -653,7 +702,11 @@ __global__ void __launch_bounds__(kSlotThreads) slot_fused_kernel(SlotParams p, 
     // order, a fixed butterfly per warp, then the warps in order
     double v = 0.0;
     if (p.T > 0)
-      for (int e = tid; e < E; e += kSlotThreads) v += __ldcg(p.aux_term + e);
+      for (int e = tid; e < E; e += kSlotThreads) {
+        // the whole term, or P_e / T still to be scaled by f_e (one-barrier path)
+        const double pt = __ldcg(p.aux_term + e);
+        v += (one && p.cnt_part == nullptr) ? ((double)s_tot[e] / ((double)p.T * p.k)) * pt : pt;
+      }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     if (lane == 0) red[warp] = v;
@@ -680,7 +733,7 @@ static int fused_slot_grid(const SlotParams& p) {
 cudaError_t launch_slots(const SlotParams& p, cudaStream_t stream) {
   const int64_t A = p.T * p.k;
   if (const int G = fused_slot_grid(p)) {
-    const size_t sm = ((size_t)(kSlotWarps + 3) * p.E + 2) * sizeof(int);   // wcnt, base, kept, off
+    const size_t sm = ((size_t)(kSlotWarps + 4) * p.E + 2) * sizeof(int);   // wcnt, base, kept, tot, off
     cudaError_t e = ensure_smem(slot_fused_kernel, sm);
     if (e != cudaSuccess) return e;
     launch_pdl(slot_fused_kernel, G, kSlotThreads, sm, stream, p, G);
