@@ -81,15 +81,7 @@ struct BParams {
 
 // MN-major operand descriptor (128-byte swizzle): 64-feature chunks `lbo`
 // bytes apart, 8-row k groups 1 KB apart.
-__device__ __forceinline__ uint64_t mn_desc(uint32_t saddr, uint32_t lbo) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-  d |= (uint64_t)(1024u >> 4) << 32;
-  d |= (uint64_t)1u << 46;
-  d |= (uint64_t)2u << 61;
-  return d;
-}
+__device__ __forceinline__ uint64_t mn_desc(uint32_t saddr, uint32_t lbo) { return sw128_mn_desc(saddr, lbo); }
 
 __device__ __forceinline__ float gelu_grad(float z) {
   // d/dz [z Phi(z)] = Phi(z) + z phi(z); Phi from erf (Abramowitz & Stegun 7.1.26)

@@ -81,6 +81,12 @@ struct KParams {
   int as_sep;                           // 1: the shared block's token rows come from tmBs (row - off[E])
   int b_packed;                         // 1: weight maps are 5-D over packed blocks
   int wide;                             // 1 (no SwiGLU): 512 features per pair tile, two MMAs share each B tile
+  // 1: the weights are read along their columns (MN-major A; the backward's
+  // dh = dY W2 and dX = dz [W1; W3]): stored [G, K, N_out], so this CTA's 128
+  // output features are two 64-column boxes of 64 k rows; k blocks >= k_switch
+  // (when > 0) come from tmA1 / tmSA1 at k - 64 k_switch
+  int a_mn;
+  int k_switch;
 };
 
 // Rows of group g that carry tokens: the routed groups' kept counts, the
@@ -207,7 +213,23 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tn_kernel(const __gri
           const uint32_t sb = sa + (two ? 2 : 1) * A_BYTES;
           const uint32_t fb = full_leader0 + 8 * stage;
           if (leader) mbar_expect_tx(full0 + 8 * stage, tx);
-          if (p.b_packed) {
+          if (p.a_mn) {
+            const bool up = p.k_switch > 0 && kb >= p.k_switch;
+            const CUtensorMap* mk = up ? ma1 : ma;
+            const int kr = (up ? kb - p.k_switch : kb) * BK;    // k row of the stored weights
+#pragma unroll
+            for (int acc2 = 0; acc2 < 2; ++acc2) {
+              if (acc2 == 1 && !two) break;
+              const int col0 = acc2 == 0 ? wrow : wrow2;
+              const uint32_t dst = sa + (uint32_t)(acc2 * A_BYTES);
+#pragma unroll
+              for (int j = 0; j < 2; ++j) {                     // 64-feature chunks, 8 KB apart
+                const int col = col0 + 64 * j;
+                if (p.b_packed) tma2_load_5d_half(dst + (uint32_t)(j * 8192), mk, kr % 128, col / 64, kr / 128, z, fb);
+                else tma2_load_3d(dst + (uint32_t)(j * 8192), mk, col, kr, z, fb);
+              }
+            }
+          } else if (p.b_packed) {
             tma2_load_5d(sa, ma, kb, wrow / 128, z, fb);
             if (two) tma2_load_5d(sa + A_BYTES, ma2, kb, wrow2 / 128, z, fb);
           } else {
@@ -234,13 +256,17 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tn_kernel(const __gri
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
+      // A descriptors: K-major, or MN-major (64-feature chunks 8 KB apart); a
+      // 16-k step moves 32 bytes (K-major) or 2 KB (MN-major), in 16-byte units
+      auto a_desc = [&](uint32_t a) { return p.a_mn ? sw128_mn_desc(a, 8192) : sw128_desc(a); };
+      const uint64_t astep = p.a_mn ? 128 : 2;
       for (int64_t tile = cid; tile < n_tiles && ok && p.wide; tile += ncl) {
         // wide: the epilogue frees accumulator 0 (columns 0-255) before
         // accumulator 1, so this tile's MMAs into accumulator 0 start as soon
         // as it is free; a stage whose accumulator-1 MMAs cannot go yet is held
         // (at most n_stages - 1 of them) until accumulator 1 is free too
         const Tile t = decode(p, ngroups, nf, tile);
-        const uint32_t idesc = make_idesc(t.n, 2 * HALF);
+        const uint32_t idesc = make_idesc(t.n, 2 * HALF, p.a_mn);
         if (!mbar_wait_cl(tempty0, acc_phase ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         bool have1 = false;
@@ -253,10 +279,10 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tn_kernel(const __gri
           if (!past) {
             if (!mbar_wait_cl(full0 + 8 * stage, phase, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            const uint64_t ad = sw128_desc(sa);
+            const uint64_t ad = a_desc(sa);
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk)
-              umma2(tmem_base, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
+              umma2(tmem_base, ad + astep * kk, bd + (uint64_t)(kk * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           if (!have1) {
             if (!past && held + 1 < n_stages && !mbar_test_cl(tempty0 + 8, acc_phase ^ 1u)) {
@@ -271,11 +297,11 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tn_kernel(const __gri
             have1 = true;
             for (int h = 0, hs = held_stage; h < held; ++h) {
               const uint32_t ha = smem_u32(stage_base + hs * stage_bytes);
-              const uint64_t hb = sw128_desc(ha + 2 * A_BYTES), hu = sw128_desc(ha + A_BYTES);
+              const uint64_t hb = sw128_desc(ha + 2 * A_BYTES), hu = a_desc(ha + A_BYTES);
               const int hk = kb - held + h;
 #pragma unroll
               for (int kk = 0; kk < BK / 16; ++kk)
-                umma2(tmem_base + 256, hu + (uint64_t)(kk * 2), hb + (uint64_t)(kk * 2), idesc,
+                umma2(tmem_base + 256, hu + astep * kk, hb + (uint64_t)(kk * 2), idesc,
                       (hk | kk) != 0 ? 1u : 0u);
               umma2_commit_both(empty0 + 8 * hs);
               if (++hs == n_stages) hs = 0;
@@ -283,10 +309,10 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tn_kernel(const __gri
             held = 0;
           }
           if (past) break;
-          const uint64_t ud = sw128_desc(sa + A_BYTES);
+          const uint64_t ud = a_desc(sa + A_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            umma2(tmem_base + 256, ud + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
+            umma2(tmem_base + 256, ud + astep * kk, bd + (uint64_t)(kk * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
           umma2_commit_both(empty0 + 8 * stage);
           if (++stage == n_stages) { stage = 0; phase ^= 1u; }
         }
@@ -296,7 +322,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tn_kernel(const __gri
       }
       for (int64_t tile = cid; tile < n_tiles && ok && !p.wide; tile += ncl) {
         const Tile t = decode(p, ngroups, nf, tile);
-        const uint32_t idesc = make_idesc(t.n, 2 * HALF);
+        const uint32_t idesc = make_idesc(t.n, 2 * HALF, p.a_mn);
         if (!mbar_wait_cl(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d0 = tmem_base + (uint32_t)(acc * 256);
@@ -305,15 +331,15 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tn_kernel(const __gri
           tc_fence_after();
           const uint32_t sa = smem_u32(stage_base + stage * stage_bytes);
           const uint64_t bd = sw128_desc(sa + (two ? 2 : 1) * A_BYTES);
-          const uint64_t ad = sw128_desc(sa);
+          const uint64_t ad = a_desc(sa);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)               // 16 elements = 32 bytes along K
-            umma2(d0, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < BK / 16; ++kk)               // 16 elements along K
+            umma2(d0, ad + astep * kk, bd + (uint64_t)(kk * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
           if (two) {
-            const uint64_t ud = sw128_desc(sa + A_BYTES);
+            const uint64_t ud = a_desc(sa + A_BYTES);
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk)
-              umma2(d0 + 256, ud + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
+              umma2(d0 + 256, ud + astep * kk, bd + (uint64_t)(kk * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           umma2_commit_both(empty0 + 8 * stage);
           if (++stage == n_stages) { stage = 0; phase ^= 1u; }
@@ -498,6 +524,48 @@ static bool map_packed(CUtensorMap* m, const void* base, int G, int N, int K) {
   return encode_cached(m, key);
 }
 
+// 5-D map over packed weights [G][N/128][K/64][128][64] (a stored [G, N, K]
+// matrix) read along K, the columns: box 64 x 64, half a block.
+static bool map_packed_half(CUtensorMap* m, const void* base, int G, int N, int K) {
+  const cuuint64_t kb = (cuuint64_t)((K + BK - 1) / BK), nb = (cuuint64_t)((N + 127) / 128);
+  MapKey key;
+  memset(&key, 0, sizeof(key));
+  key.base = base;
+  key.rank = 5;
+  key.swizzle = CU_TENSOR_MAP_SWIZZLE_128B;
+  key.dims[0] = BK;
+  key.dims[1] = 128;
+  key.dims[2] = kb;
+  key.dims[3] = nb;
+  key.dims[4] = (cuuint64_t)G;
+  key.strides[0] = BK * 2;
+  key.strides[1] = (cuuint64_t)BK * 128 * 2;
+  key.strides[2] = key.strides[1] * kb;
+  key.strides[3] = key.strides[2] * nb;
+  key.box[0] = BK;
+  key.box[1] = 64;
+  key.box[2] = key.box[3] = key.box[4] = 1;
+  return encode_cached(m, key);
+}
+
+// 3-D map over stacked weights [G, N, K] read along K: box 64 x 64 x 1.
+static bool map_weights_half(CUtensorMap* m, const void* base, int G, int N, int K) {
+  MapKey key;
+  memset(&key, 0, sizeof(key));
+  key.base = base;
+  key.rank = 3;
+  key.swizzle = CU_TENSOR_MAP_SWIZZLE_128B;
+  key.dims[0] = (cuuint64_t)K;
+  key.dims[1] = (cuuint64_t)N;
+  key.dims[2] = (cuuint64_t)G;
+  key.strides[0] = (cuuint64_t)K * 2;
+  key.strides[1] = (cuuint64_t)N * K * 2;
+  key.box[0] = BK;
+  key.box[1] = 64;
+  key.box[2] = 1;
+  return encode_cached(m, key);
+}
+
 // 2-D map over a bf16 output [rows, N], box 32 x 32, 64-byte swizzle (TMA store).
 static bool map_out(CUtensorMap* m, const void* base, int64_t rows, int N) {
   MapKey key;
@@ -539,6 +607,8 @@ static int resident_pairs() {
   }
   return c;
 }
+
+static cudaError_t launch_pairs(const KParams& k, cudaStream_t stream);
 
 }  // namespace gtn
 
@@ -589,6 +659,61 @@ cudaError_t launch_grouped_gemm_tn(const GemmParams& p, cudaStream_t stream) {
   // expensive epilogue (GELU) would stall the MMAs: those keep 256-feature,
   // double-buffered tiles.
   k.wide = ((p.epi < 0 || p.epi == MOE_ACT_RELU) && p.Nw >= 2 * FT) ? 1 : 0;
+  return launch_pairs(k, stream);
+}
+
+// The backward's weight-side contractions on pairs of SMs (see KParams::a_mn):
+// out[rows, N] = a[rows, K] * W, W stored [G, K0, N] and read along N, k blocks
+// >= k_switch from b1; the same token tiles as the forward (kept rows rounded up
+// to 16 per group, the shared block's T rows in place).
+cudaError_t launch_bwd_dgrad_pair(const BwdGemm& q, int32_t* pair_prefix, const int32_t* valid,
+                                  cudaStream_t stream) {
+  using namespace gtn;
+  if (q.rows_max == 0) return cudaSuccess;
+  if (encode_fn() == nullptr) return cudaErrorNotSupported;
+  KParams k{};
+  const void* b1 = q.b1 ? q.b1 : q.b0;
+  const void* s0 = q.sb0 ? q.sb0 : q.b0;
+  const void* s1 = q.sb1 ? q.sb1 : s0;
+  bool ok = true;
+  if (q.b_packed) {
+    ok = ok && map_packed_half(&k.tmA, q.b0, q.E, q.K0, q.N);
+    ok = ok && map_packed_half(&k.tmA1, b1, q.E, q.K0, q.N);
+    ok = ok && map_packed_half(&k.tmSA, s0, 1, q.K0, q.N);
+    ok = ok && map_packed_half(&k.tmSA1, s1, 1, q.K0, q.N);
+  } else {
+    ok = ok && map_weights_half(&k.tmA, q.b0, q.E, q.K0, q.N);
+    ok = ok && map_weights_half(&k.tmA1, b1, q.E, q.K0, q.N);
+    ok = ok && map_weights_half(&k.tmSA, s0, 1, q.K0, q.N);
+    ok = ok && map_weights_half(&k.tmSA1, s1, 1, q.K0, q.N);
+  }
+  ok = ok && map_rows(&k.tmB, q.a, q.rows_max, q.K);
+  ok = ok && map_rows(&k.tmBs, q.a, q.rows_max, q.K);
+  ok = ok && map_out(&k.tmD, q.out, q.rows_max, q.N);
+  if (!ok) return cudaErrorInvalidValue;
+  const int ngroups = q.E + (q.n_shared ? 1 : 0);
+  launch_pdl(token_tile_prefix_kernel, 1, 32, 0, stream, q.off, valid, ngroups, q.E, q.T, q.rows_max, pair_prefix);
+  k.off = q.off;
+  k.tp = pair_prefix;
+  k.valid = valid;
+  k.status = q.status;
+  k.rows_max = q.rows_max;
+  k.T = q.T;
+  k.K = q.K;
+  k.N_out = q.N;
+  k.E = q.E;
+  k.n_shared = q.n_shared;
+  k.epi = -1;
+  k.as_sep = 0;
+  k.b_packed = q.b_packed;
+  k.wide = q.N >= 2 * FT ? 1 : 0;
+  k.a_mn = 1;
+  k.k_switch = q.k_switch;
+  return launch_pairs(k, stream);
+}
+
+namespace gtn {
+static cudaError_t launch_pairs(const KParams& k, cudaStream_t stream) {
   cudaError_t e = ensure_smem(grouped_gemm_tn_kernel, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg{};
@@ -609,5 +734,6 @@ cudaError_t launch_grouped_gemm_tn(const GemmParams& p, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
+}  // namespace gtn
 
 }  // namespace moe

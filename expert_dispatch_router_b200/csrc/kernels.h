@@ -237,6 +237,13 @@ cudaError_t launch_bwd_dact(const BwdGemm& q, cudaStream_t stream);
 cudaError_t launch_bwd_wgrad(const BwdGemm& q, cudaStream_t stream);
 // dz = bf16(dyrow W2) * act'(x_rows W1^T) in one kernel (dh is not stored)
 cudaError_t launch_bwd_dhz(const BwdGemm& q, cudaStream_t stream);
+// dgrad on pairs of SMs (grouped_gemm_tn.cu), for layers with T*k > 256*E:
+// the same product as launch_bwd_dgrad, computed for each group's kept rows
+// rounded up to 16 (valid: the routed groups' kept counts; pair_prefix:
+// ngroups + 1 ints of scratch).  Rows past them in each 128-row block are not
+// written.
+cudaError_t launch_bwd_dgrad_pair(const BwdGemm& q, int32_t* pair_prefix, const int32_t* valid,
+                                  cudaStream_t stream);
 
 // Packed weight layout for the grouped GEMM: w [G, N, K] bf16 (K contiguous) ->
 // [G][ceil(N/128)][ceil(K/64)][128][64], zero-padded, so every TMA box of 128

@@ -671,7 +671,10 @@ int moe_layer_bwd(const moe_cfg* cfg, const void* x, const float* wg, const moe_
     g.K0 = H;
     g.N = F;
     g.b_packed = packed;
-    if (launch_bwd_dgrad(g, s) != cudaSuccess) return MOE_ECUDA;
+    // compute-bound layers (the forward's rule): pairs of SMs, W2 read along F
+    const cudaError_t e = two_sm_ffn(cfg) ? launch_bwd_dgrad_pair(g, at<int32_t>(ws, L.pairs), at<int32_t>(ws, L.kept), s)
+                                          : launch_bwd_dgrad(g, s);
+    if (e != cudaSuccess) return MOE_ECUDA;
   }
   if ((st = record(stage_events, 2, s)) != MOE_OK) return st;
   // 3. dW2 = dyrow^T h per expert.  With at least 192 rows per expert on
@@ -751,7 +754,12 @@ int moe_layer_bwd(const moe_cfg* cfg, const void* x, const float* wg, const moe_
   g.k_switch = sw ? Fp / 64 : 0;
   g.N = H;
   g.b_packed = packed;
-  if (launch_bwd_dgrad(g, s) != cudaSuccess) return MOE_ECUDA;
+  {
+    const cudaError_t e = two_sm_ffn(cfg)
+                              ? launch_bwd_dgrad_pair(g, at<int32_t>(ws, L.pairs), at<int32_t>(ws, L.kept), s)
+                              : launch_bwd_dgrad(g, s);
+    if (e != cudaSuccess) return MOE_ECUDA;
+  }
   if ((st = record(stage_events, 7, s)) != MOE_OK) return st;
   // 8. dx: tokens sum their rows' gradients, plus the router's dlogits Wg
   DispatchBwdParams db{};

@@ -95,6 +95,16 @@ __device__ __forceinline__ void tma2_load_3d(uint32_t dst, const CUtensorMap* ma
                " [%0], [%1, {%2, %3, %4}], [%5];"
                :: "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar) : "memory");
 }
+// Packed weights, half a block (64 of its 128 rows: an MN-major box):
+// coordinates (0, row in block, column block, row block, group).
+__device__ __forceinline__ void tma2_load_5d_half(uint32_t dst, const CUtensorMap* map, int c1, int c2, int c3,
+                                                  int c4, uint32_t bar) {
+  asm volatile("cp.async.bulk.tensor.5d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+               " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];"
+               :: "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(c1), "r"(c2), "r"(c3), "r"(c4),
+                  "r"(bar)
+               : "memory");
+}
 // Packed weights: coordinates (0, 0, k block, n block, group).
 __device__ __forceinline__ void tma2_load_5d(uint32_t dst, const CUtensorMap* map, int c2, int c3, int c4,
                                              uint32_t bar) {

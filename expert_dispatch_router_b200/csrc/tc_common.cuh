@@ -117,6 +117,18 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
   d |= (uint64_t)2u << 61;                          // layout: 128-byte swizzle
   return d;
 }
+// Shared-memory matrix descriptor: MN-major operand, 128-byte swizzle: rows of
+// 64 M (or N) elements per k, 64-element chunks `lbo` bytes apart, 8-row k
+// groups 1024 bytes apart.  A 16-k step advances the start by 2 KB.
+__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr, uint32_t lbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;
+  return d;
+}
 // Instruction descriptor: bf16 x bf16 -> fp32, M = m, N = n; each operand
 // K-major (0) or MN-major (1, bits 15 and 16).
 __device__ __forceinline__ uint32_t make_idesc(int n, int m = 128, int a_mn = 0, int b_mn = 0) {

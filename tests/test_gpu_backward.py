@@ -242,6 +242,48 @@ BWD_SHAPES = {
 }
 
 
+# T*k > 256*E with H > 512: dh and dxrow run on pairs of SMs with the weights
+# read along their columns.  SwiGLU + shared expert: 512-feature tiles in both
+# (F = 584, H = 1032: ragged last tiles and a ragged last k block), the W1 -> W3
+# switch at Fp = 640; GELU + capacity: 256-feature dh tiles (F = 392).
+BWD_PAIR_SHAPES = {
+    "swiglu_shared_pairs": synth.WIDEEP_DROPLESS.replace(name="swiglu_shared_pairs", T=1200, H=1032, F=584, E=4,
+                                                         k=2),
+    "gelu_capacity_pairs": synth.GSHARD_TOP2.replace(name="gelu_capacity_pairs", T=1500, H=520, F=392, E=4),
+}
+
+
+@pytest.mark.parametrize("name", list(BWD_PAIR_SHAPES))
+def test_backward_pairs(name):
+    shape = BWD_PAIR_SHAPES[name]
+    inp = synth.make_inputs(shape, seed=5, device="cuda", scale="unit")
+    condition_uniform(shape, inp)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(19)
+    dy = torch.randn((shape.T, shape.H), generator=gen, device="cuda").to(torch.bfloat16)
+    out = run_fwd_bwd(shape, inp, dy, 1.1, 0.9)
+    check_backward(shape, inp, out, dy, 1.1, 0.9)
+
+
+@pytest.mark.parametrize("name", list(BWD_PAIR_SHAPES))
+def test_backward_pairs_packed_matches_unpacked(name):
+    """The pair kernels read packed weights as half blocks and plain ones as
+    64 x 64 boxes: the same bytes reach shared memory, so every output is
+    bitwise the same."""
+    shape = BWD_PAIR_SHAPES[name]
+    inp = synth.make_inputs(shape, seed=8, device="cuda", scale="unit")
+    condition_uniform(shape, inp)
+    dy = torch.randn((shape.T, shape.H), device="cuda").to(torch.bfloat16)
+    a = run_fwd_bwd(shape, inp, dy, 1.0, 1.0)
+    a = {k: (v.clone() if torch.is_tensor(v) else v) for k, v in a.items()}
+    b = run_fwd_bwd(shape, inp, dy, 1.0, 1.0, packed=True)
+    for n in ("y", "dx", "dwg", "dgate", "dlogits"):
+        assert torch.equal(a[n].view(torch.uint8), b[n].view(torch.uint8)), n
+    for n, v in a["grads"].items():
+        if v is not None:
+            assert torch.equal(v.view(torch.uint8), b["grads"][n].view(torch.uint8)), n
+
+
 @pytest.mark.parametrize("name", list(BWD_SHAPES))
 def test_backward_small(name):
     shape = BWD_SHAPES[name]
