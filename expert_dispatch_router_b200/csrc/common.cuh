@@ -108,6 +108,11 @@ __device__ __forceinline__ float act_gelu(float z) {
   const float h = z * (q * t) * e;                                          // 0.5 z erfc(|z| / sqrt 2)
   return z >= 0.0f ? z - h : h;
 }
+// GELU'(z) = d/dz [z Phi(z)] = Phi(z) + z phi(z); Phi from erf (Abramowitz & Stegun 7.1.26).
+__device__ __forceinline__ float gelu_grad(float z) {
+  const float phi = 0.3989422804014327f * __expf(-0.5f * z * z);
+  return 0.5f * (1.0f + erf_as7126(z * 0.70710678118654752f)) + z * phi;
+}
 // SiLU: z * sigmoid(z) = z / (1 + exp(-z)).
 __device__ __forceinline__ float act_silu(float z) { return z * rcp_approx(1.0f + __expf(-z)); }
 

@@ -83,11 +83,6 @@ struct BParams {
 // bytes apart, 8-row k groups 1 KB apart.
 __device__ __forceinline__ uint64_t mn_desc(uint32_t saddr, uint32_t lbo) { return sw128_mn_desc(saddr, lbo); }
 
-__device__ __forceinline__ float gelu_grad(float z) {
-  // d/dz [z Phi(z)] = Phi(z) + z phi(z); Phi from erf (Abramowitz & Stegun 7.1.26)
-  const float phi = 0.3989422804014327f * __expf(-0.5f * z * z);
-  return 0.5f * (1.0f + erf_as7126(z * 0.70710678118654752f)) + z * phi;
-}
 
 // MODE and V are template parameters so that each variant's epilogue gets its
 // own register allocation.  V: SwiGLU for DACT and DHZ; for WGRAD the deep

@@ -87,6 +87,12 @@ struct KParams {
   // (when > 0) come from tmA1 / tmSA1 at k - 64 k_switch
   int a_mn;
   int k_switch;
+  // 1: the backward's dz = dh * act'(z) from the recomputed z (the epilogue
+  // reads dh [rows_max, N_out]; SwiGLU writes da at column f and db at
+  // dz_half + f of the output)
+  int dact;
+  int dz_half;
+  const __nv_bfloat16* dh;
 };
 
 // Rows of group g that carry tokens: the routed groups' kept counts, the
@@ -123,6 +129,9 @@ __device__ __forceinline__ Tile decode(const KParams& p, int ngroups, int nf, in
   return t;
 }
 
+// DACT: the backward's dz epilogue (KParams::dact), a separate instance so
+// that the forward's epilogue keeps its own register allocation.
+template <bool DACT>
 __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tn_kernel(const __grid_constant__ KParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -376,6 +385,63 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tn_kernel(const __gri
         const uint32_t tb = tbase + (uint32_t)(a * 256);
         for (int c = quarter * 32; c < t.n && f0 < p.N_out; c += 4 * 32) {
           __syncwarp();
+          if constexpr (DACT) {
+            // dz = dh * act'(z): the chunk's 32 x 32 dh block comes in by
+            // 16-byte loads into the staging buffer (its layout below), then
+            // each lane takes its feature's column (features past N_out read
+            // as zero); da (or dz) and SwiGLU's db go out as two stores
+            float v[32], u[32];
+            tmem_ld(tb + (uint32_t)c, v, 32);
+            if (swiglu) tmem_ld(tbase + 256u + (uint32_t)c, u, 32);
+            tmem_wait_ld();
+            const uint32_t col_b = (uint32_t)((lane & 7) * 2);
+            if (lane == 0) bulk_wait_read0();
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int q = lane + 32 * i, j = q >> 2, ch = q & 3;
+              const int64_t row = t.r0 + c + j;
+              const int fc = f0 + 8 * ch;
+              int4 w = make_int4(0, 0, 0, 0);
+              if (fc < p.N_out && row < p.rows_max) w = ld_nc_v4(p.dh + row * p.N_out + fc);
+              const uint32_t addr = stage_out + (uint32_t)(j * 64) + (((uint32_t)ch ^ (((uint32_t)j >> 1) & 3u)) << 4);
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                           :: "r"(addr), "r"(w.x), "r"(w.y), "r"(w.z), "r"(w.w) : "memory");
+            }
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const uint32_t addr = stage_out + (uint32_t)(j * 64) + ((((uint32_t)lane >> 3) ^ (((uint32_t)j >> 1) & 3u)) << 4) + col_b;
+              uint16_t hb;
+              asm volatile("ld.shared.b16 %0, [%1];" : "=h"(hb) : "r"(addr) : "memory");
+              const float gi = __bfloat162float(__ushort_as_bfloat16(hb));
+              const float z = v[j];
+              if (swiglu) {
+                const float sg = 1.0f / (1.0f + __expf(-z));
+                v[j] = gi * u[j] * sg * (1.0f + z * (1.0f - sg));   // da
+                u[j] = gi * z * sg;                                 // db = dh * silu(a)
+              } else {
+                v[j] = p.epi == MOE_ACT_RELU ? (z > 0.0f ? gi : 0.0f) : gi * gelu_grad(z);
+              }
+            }
+            for (int o = 0; o < (swiglu ? 2 : 1); ++o) {
+              if (lane == 0) bulk_wait_read0();
+              __syncwarp();
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const __nv_bfloat16 h = __float2bfloat16_rn(o == 0 ? v[j] : u[j]);
+                const uint32_t addr = stage_out + (uint32_t)(j * 64) + ((((uint32_t)lane >> 3) ^ (((uint32_t)j >> 1) & 3u)) << 4) + col_b;
+                asm volatile("st.shared.b16 [%0], %1;" :: "r"(addr), "h"(*reinterpret_cast<const uint16_t*>(&h)) : "memory");
+              }
+              fence_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&p.tmD, stage_out, (o == 0 ? 0 : p.dz_half) + f0, (int)(t.r0 + c));
+                bulk_commit();
+              }
+            }
+            continue;
+          }
           float v[32];
           tmem_ld(tb + (uint32_t)c, v, 32);
           if (swiglu) {
@@ -599,7 +665,7 @@ static int resident_pairs() {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_tn_kernel, &cfg) != cudaSuccess || n < 1) {
+    if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_tn_kernel<false>, &cfg) != cudaSuccess || n < 1) {
       cudaGetLastError();
       n = sm_count() / 2;
     }
@@ -712,9 +778,62 @@ cudaError_t launch_bwd_dgrad_pair(const BwdGemm& q, int32_t* pair_prefix, const 
   return launch_pairs(k, stream);
 }
 
+// The backward's dz = dh * act'(z) on pairs of SMs: z (and SwiGLU's up
+// projection) recomputed from the dispatched rows as the forward's first
+// contraction does, dh read in the epilogue, dz [rows_max, dz_ld] written with
+// SwiGLU's db at column dz_ld / 2.
+cudaError_t launch_bwd_dact_pair(const BwdGemm& q, int dz_ld, int32_t* pair_prefix, const int32_t* valid,
+                                 cudaStream_t stream) {
+  using namespace gtn;
+  if (q.rows_max == 0) return cudaSuccess;
+  if (encode_fn() == nullptr) return cudaErrorNotSupported;
+  KParams k{};
+  const bool swiglu = q.act == MOE_ACT_SWIGLU;
+  const void* b1 = q.b1 ? q.b1 : q.b0;
+  const void* s0 = q.sb0 ? q.sb0 : q.b0;
+  const void* s1 = q.sb1 ? q.sb1 : s0;
+  bool ok = true;
+  if (q.b_packed) {
+    ok = ok && map_packed(&k.tmA, q.b0, q.E, q.N, q.K);
+    ok = ok && map_packed(&k.tmA1, b1, q.E, q.N, q.K);
+    ok = ok && map_packed(&k.tmSA, s0, 1, q.N, q.K);
+    ok = ok && map_packed(&k.tmSA1, s1, 1, q.N, q.K);
+  } else {
+    ok = ok && map_weights(&k.tmA, q.b0, q.E, q.N, q.K);
+    ok = ok && map_weights(&k.tmA1, b1, q.E, q.N, q.K);
+    ok = ok && map_weights(&k.tmSA, s0, 1, q.N, q.K);
+    ok = ok && map_weights(&k.tmSA1, s1, 1, q.N, q.K);
+  }
+  ok = ok && map_rows(&k.tmB, q.a, q.rows_max, q.K);
+  ok = ok && map_rows(&k.tmBs, q.a_shared ? q.a_shared : q.a, q.a_shared ? q.T : q.rows_max, q.K);
+  ok = ok && map_out(&k.tmD, q.out, q.rows_max, dz_ld);
+  if (!ok) return cudaErrorInvalidValue;
+  const int ngroups = q.E + (q.n_shared ? 1 : 0);
+  launch_pdl(token_tile_prefix_kernel, 1, 32, 0, stream, q.off, valid, ngroups, q.E, q.T, q.rows_max, pair_prefix);
+  k.off = q.off;
+  k.tp = pair_prefix;
+  k.valid = valid;
+  k.status = q.status;
+  k.rows_max = q.rows_max;
+  k.T = q.T;
+  k.K = q.K;
+  k.N_out = q.N;
+  k.E = q.E;
+  k.n_shared = q.n_shared;
+  k.epi = q.act;
+  k.as_sep = q.a_shared != nullptr;
+  k.b_packed = q.b_packed;
+  k.wide = (q.act == MOE_ACT_RELU && q.N >= 2 * FT) ? 1 : 0;
+  k.dact = 1;
+  k.dz_half = swiglu ? dz_ld / 2 : 0;
+  k.dh = static_cast<const __nv_bfloat16*>(q.dh);
+  return launch_pairs(k, stream);
+}
+
 namespace gtn {
 static cudaError_t launch_pairs(const KParams& k, cudaStream_t stream) {
-  cudaError_t e = ensure_smem(grouped_gemm_tn_kernel, SMEM_BYTES);
+  auto kern = k.dact ? grouped_gemm_tn_kernel<true> : grouped_gemm_tn_kernel<false>;
+  cudaError_t e = ensure_smem(kern, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(2 * resident_pairs());
@@ -730,7 +849,7 @@ static cudaError_t launch_pairs(const KParams& k, cudaStream_t stream) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  e = cudaLaunchKernelEx(&cfg, grouped_gemm_tn_kernel, k);
+  e = cudaLaunchKernelEx(&cfg, kern, k);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

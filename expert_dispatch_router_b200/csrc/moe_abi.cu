@@ -707,7 +707,13 @@ int moe_layer_bwd(const moe_cfg* cfg, const void* x, const float* wg, const moe_
   g.K = H;
   g.N = F;
   g.b_packed = packed;
-  if (!fused && launch_bwd_dact(g, s) != cudaSuccess) return MOE_ECUDA;
+  if (!fused) {
+    // compute-bound layers: pairs of SMs, as the forward's first contraction
+    const cudaError_t e = two_sm_ffn(cfg)
+                              ? launch_bwd_dact_pair(g, dzw, at<int32_t>(ws, L.pairs), at<int32_t>(ws, L.kept), s)
+                              : launch_bwd_dact(g, s);
+    if (e != cudaSuccess) return MOE_ECUDA;
+  }
   if ((st = record(stage_events, 4, s)) != MOE_OK) return st;
   // 5. dW1 (and dW3) = dz^T x_rows per expert; the shared block's rows are x
   g = q;
