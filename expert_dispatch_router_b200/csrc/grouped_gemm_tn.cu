@@ -93,6 +93,14 @@ struct KParams {
   int dact;
   int dz_half;
   const __nv_bfloat16* dh;
+  // weight gradients (the WGRAD instance): per expert g, out[g] = A_g^T B_g
+  // (fp32 [m_valid, N_out]) with A rows [rows_max, M_out] (tmA) and B rows
+  // [rows_max, N_out] (tmB; the shared block's from tmBs at row - off[E] when
+  // b_sep), both read along their columns; output rows >= m_split go to
+  // w_out2 / w_sh2 at m - m_split
+  int M_out, m_split, m_valid, b_sep;
+  float *w_out, *w_out2, *w_sh, *w_sh2;
+  CUtensorMap tmW, tmW2, tmWs, tmWs2;   // those outputs [G, m_valid, N_out] fp32, box 16 x 32 x 1, 64-byte swizzle
 };
 
 // Rows of group g that carry tokens: the routed groups' kept counts, the
@@ -129,10 +137,12 @@ __device__ __forceinline__ Tile decode(const KParams& p, int ngroups, int nf, in
   return t;
 }
 
-// DACT: the backward's dz epilogue (KParams::dact), a separate instance so
-// that the forward's epilogue keeps its own register allocation.
-template <bool DACT>
+// MODE 0: the forward's contractions and the backward's dh / dX (a_mn);
+// MODE 1: the backward's dz epilogue (KParams::dact); MODE 2: the weight
+// gradients.  Separate instances keep the forward's register allocation.
+template <int MODE>
 __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tn_kernel(const __grid_constant__ KParams p) {
+  constexpr bool DACT = MODE == 1, WG = MODE == 2;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
@@ -189,12 +199,170 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tn_kernel(const __gri
   if (!tmem_same && threadIdx.x == 0) set_status(p.status, MOE_EDEVICE, 31);
 
   const int nf = (p.N_out + span - 1) / span;                  // feature tiles
-  const int64_t n_tok_tiles = tmem_same ? __ldg(p.tp + ngroups) : 0;
-  const int64_t n_tiles = n_tok_tiles * nf;
+  // WG: tiles (group, 256 output rows, 256 output columns), columns fastest
+  const int wg_nm = WG ? (p.M_out + 2 * HALF - 1) / (2 * HALF) : 0, wg_nn = WG ? (p.N_out + 2 * HALF - 1) / (2 * HALF) : 0;
+  const int64_t n_tok_tiles = tmem_same && !WG ? __ldg(p.tp + ngroups) : 0;
+  const int64_t n_tiles = WG ? (tmem_same ? (int64_t)ngroups * wg_nm * wg_nn : 0) : n_tok_tiles * nf;
+  // WG: a tile's group, output row and column blocks, and 64-row k blocks
+  auto wg_tile = [&](int64_t tile, int& g, int& mt, int& nt, int& nkb, int64_t& r0) {
+    const int64_t per = (int64_t)wg_nm * wg_nn;
+    g = (int)(tile / per);
+    const int rest = (int)(tile - (int64_t)g * per);
+    mt = rest / wg_nn;
+    nt = rest - mt * wg_nn;
+    r0 = min((int64_t)__ldg(p.off + g), p.rows_max);
+    nkb = (int)((group_rows(p.off, p.valid, g, p.E, p.T, p.rows_max) + BK - 1) / BK);
+  };
   const int nk = (p.K + BK - 1) / BK;
   const int64_t cid = cluster_id(), ncl = cluster_count();
 
-  if (warp == 0) {
+  if (WG && warp == 0) {
+    // ---------------- TMA producer, weight gradients (both CTAs): per 64-row
+    // k block, this CTA's 128 A columns and 128 B columns as 64 x 64 boxes
+    if (lane == 0) {
+      const uint32_t full_leader0 = map_to(full0, 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t fills[MAX_STAGES] = {0, 0, 0, 0, 0, 0};
+      bool ok = true;
+      const uint32_t tx = 2u * (uint32_t)stage_bytes;
+      for (int64_t tile = cid; tile < n_tiles && ok; tile += ncl) {
+        int g, mt, nt, nkb;
+        int64_t r0;
+        wg_tile(tile, g, mt, nt, nkb, r0);
+        const bool bsep = g == p.E && p.b_sep;
+        const CUtensorMap* mb = bsep ? &p.tmBs : &p.tmB;
+        const int64_t rb0 = bsep ? r0 - __ldg(p.off + p.E) : r0;
+        const int m0 = mt * 2 * HALF + (int)rank * HALF, n0 = nt * 2 * HALF + (int)rank * HALF;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_cl(empty0 + 8 * stage, phase ^ 1u, abort_flag)) { ok = false; break; }
+          const uint32_t sa = smem_u32(stage_base + stage * stage_bytes);
+          const uint32_t sb = sa + A_BYTES;
+          const uint32_t fb = full_leader0 + 8 * stage;
+          if (leader) mbar_expect_tx(full0 + 8 * stage, tx);
+          const int ra = (int)(r0 + kb * BK), rb = (int)(rb0 + kb * BK);
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            tma2_load_2d(sa + (uint32_t)(j * 8192), &p.tmA, m0 + 64 * j, ra, fb);
+            tma2_load_2d(sb + (uint32_t)(j * 8192), mb, n0 + 64 * j, rb, fb);
+          }
+          fills[stage]++;
+          if (++stage == n_stages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) abort_pair(43);
+      for (int s = 0; s < n_stages; ++s)
+        if (fills[s]) {
+          if (leader) mbar_drain_cl(full0 + 8 * s, (fills[s] - 1) & 1u);
+          else mbar_drain_cl(empty0 + 8 * s, (fills[s] - 1) & 1u);
+        }
+    }
+  } else if (WG && warp == 1) {
+    // ---------------- MMA issuer, weight gradients (even CTA): both operands
+    // MN-major; a group with no rows commits an untouched accumulator, which
+    // the epilogue replaces by zeros
+    if (leader && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      const uint32_t idesc = make_idesc(2 * HALF, 2 * HALF, 1, 1);
+      for (int64_t tile = cid; tile < n_tiles && ok; tile += ncl) {
+        int g, mt, nt, nkb;
+        int64_t r0;
+        wg_tile(tile, g, mt, nt, nkb, r0);
+        if (!mbar_wait_cl(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + (uint32_t)(acc * 256);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_cl(full0 + 8 * stage, phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(stage_base + stage * stage_bytes);
+          const uint64_t ad = sw128_mn_desc(sa, 8192), bd = sw128_mn_desc(sa + A_BYTES, 8192);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)                // 16 rows = 2 KB in both operands
+            umma2(d0, ad + (uint64_t)(128 * kk), bd + (uint64_t)(128 * kk), idesc, (kb | kk) != 0 ? 1u : 0u);
+          umma2_commit_both(empty0 + 8 * stage);
+          if (++stage == n_stages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma2_commit_both(tfull0 + 8 * acc);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      if (!ok) abort_pair(44);
+      umma2_commit_both(drain);
+    }
+    if (lane == 0) mbar_drain_cl(drain, 0);
+  } else if (WG) {
+    // ---------------- epilogue, weight gradients (both CTAs): lane = output
+    // row m; each 32-column TMEM load leaves as two 32-row x 16-column fp32
+    // blocks through this warp's staging buffer (rows of 64 bytes, 16-byte
+    // chunk q of row j at q ^ ((j >> 1) & 3): the TMA 64-byte swizzle)
+    const int ew = warp - 2;
+    const int sub = warp & 3;
+    const int quarter = ew >> 2;
+    const uint32_t stage_out = smem_u32(staging + ew * STAGE_OUT_BYTES);
+    const uint32_t tempty_leader0 = map_to(tempty0, 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int64_t tile = cid; tile < n_tiles; tile += ncl) {
+      int g, mt, nt, nkb;
+      int64_t r0;
+      wg_tile(tile, g, mt, nt, nkb, r0);
+      if (!mbar_wait_cl(tfull0 + 8 * acc, acc_phase, abort_flag)) {
+        if (lane == 0) abort_pair(45);
+        break;
+      }
+      tc_fence_after();
+      const bool sh = g == p.E;
+      // this warp's 32 rows: m0w .. m0w + 31, all in one output part (m_split
+      // is a multiple of 64)
+      const int m0w = mt * 2 * HALF + (int)rank * HALF + sub * 32;
+      const bool second = m0w >= p.m_split;
+      const int mr0 = second ? m0w - p.m_split : m0w;
+      const CUtensorMap* mw = second ? (sh ? &p.tmWs2 : &p.tmW2) : (sh ? &p.tmWs : &p.tmW);
+      const bool part_ok = (second ? (sh ? p.w_sh2 : p.w_out2) : (sh ? p.w_sh : p.w_out)) != nullptr &&
+                           mr0 < p.m_valid && (second || m0w < p.m_split);
+      const uint32_t tbase = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * 256);
+      for (int c = quarter * 32; c < 2 * HALF; c += 4 * 32) {
+        const int n = nt * 2 * HALF + c;
+        if (n >= p.N_out) break;                                 // warp-uniform
+        __syncwarp();
+        float v[32];
+        tmem_ld(tbase + (uint32_t)c, v, 32);
+        tmem_wait_ld();
+        if (!part_ok) continue;                                  // warp-uniform
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (n + 16 * h >= p.N_out) break;
+          if (lane == 0) bulk_wait_read0();
+          __syncwarp();
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t addr = stage_out + (uint32_t)(lane * 64) + (((uint32_t)q ^ (((uint32_t)lane >> 1) & 3u)) << 4);
+            const float* x4 = v + 16 * h + 4 * q;
+            const uint32_t z = nkb > 0 ? 0xffffffffu : 0u;       // a group with no rows stores zeros
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                         :: "r"(addr), "r"(__float_as_uint(x4[0]) & z), "r"(__float_as_uint(x4[1]) & z),
+                            "r"(__float_as_uint(x4[2]) & z), "r"(__float_as_uint(x4[3]) & z) : "memory");
+          }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(mw, stage_out, n + 16 * h, mr0, sh ? 0 : g);
+            bulk_commit();
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8 * acc);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+    if (lane == 0) bulk_wait0();
+    __syncwarp();
+  } else if (warp == 0) {
     // ---------------- TMA producer (both CTAs)
     if (lane == 0) {
       const uint32_t full_leader0 = map_to(full0, 0);
@@ -632,6 +800,40 @@ static bool map_weights_half(CUtensorMap* m, const void* base, int G, int N, int
   return encode_cached(m, key);
 }
 
+// 2-D map over a row-major bf16 matrix [rows, W] read along W: box 64 x 64.
+static bool map_rows_half(CUtensorMap* m, const void* base, int64_t rows, int W) {
+  MapKey key;
+  memset(&key, 0, sizeof(key));
+  key.base = base;
+  key.rank = 2;
+  key.swizzle = CU_TENSOR_MAP_SWIZZLE_128B;
+  key.dims[0] = (cuuint64_t)W;
+  key.dims[1] = (cuuint64_t)rows;
+  key.strides[0] = (cuuint64_t)W * 2;
+  key.box[0] = BK;
+  key.box[1] = 64;
+  return encode_cached(m, key);
+}
+
+// 3-D map over an fp32 output [G, rows, N], box 16 x 32 x 1, 64-byte swizzle (TMA store).
+static bool map_out_f32(CUtensorMap* m, const void* base, int G, int rows, int N) {
+  MapKey key;
+  memset(&key, 0, sizeof(key));
+  key.base = base;
+  key.rank = 3;
+  key.f32 = 1;
+  key.swizzle = CU_TENSOR_MAP_SWIZZLE_64B;
+  key.dims[0] = (cuuint64_t)N;
+  key.dims[1] = (cuuint64_t)rows;
+  key.dims[2] = (cuuint64_t)G;
+  key.strides[0] = (cuuint64_t)N * 4;
+  key.strides[1] = (cuuint64_t)rows * N * 4;
+  key.box[0] = 16;
+  key.box[1] = 32;
+  key.box[2] = 1;
+  return encode_cached(m, key);
+}
+
 // 2-D map over a bf16 output [rows, N], box 32 x 32, 64-byte swizzle (TMA store).
 static bool map_out(CUtensorMap* m, const void* base, int64_t rows, int N) {
   MapKey key;
@@ -665,7 +867,7 @@ static int resident_pairs() {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_tn_kernel<false>, &cfg) != cudaSuccess || n < 1) {
+    if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_tn_kernel<0>, &cfg) != cudaSuccess || n < 1) {
       cudaGetLastError();
       n = sm_count() / 2;
     }
@@ -830,9 +1032,50 @@ cudaError_t launch_bwd_dact_pair(const BwdGemm& q, int dz_ld, int32_t* pair_pref
   return launch_pairs(k, stream);
 }
 
+// The weight gradients on pairs of SMs: per expert g, w_out[g] = a_g^T b_g in
+// fp32, over the group's kept rows in 64-row blocks (the padding rows past them
+// in a block are zero in b for dW1 and in a for dW2); tiles of 256 output rows
+// x 256 columns; output rows >= m_split go to w_out2 (m_valid rows each); the
+// shared expert's to w_sh / w_sh2, its b rows from b_shared (row - off[E]).
+cudaError_t launch_bwd_wgrad_pair(const BwdGemm& q, const int32_t* valid, cudaStream_t stream) {
+  using namespace gtn;
+  if (q.rows_max == 0 && q.E == 0) return cudaSuccess;
+  if (encode_fn() == nullptr) return cudaErrorNotSupported;
+  KParams k{};
+  bool ok = true;
+  const int64_t rows = q.rows_max > 0 ? q.rows_max : 1;
+  ok = ok && map_rows_half(&k.tmA, q.a, rows, q.M);
+  ok = ok && map_rows_half(&k.tmB, q.b0, rows, q.N);
+  ok = ok && map_rows_half(&k.tmBs, q.b_shared ? q.b_shared : q.b0, q.b_shared ? (q.T > 0 ? q.T : 1) : rows, q.N);
+  // absent outputs map the first one: the kernel never stores through them
+  ok = ok && map_out_f32(&k.tmW, q.w_out, q.E > 0 ? q.E : 1, q.m_valid, q.N);
+  ok = ok && map_out_f32(&k.tmW2, q.w_out2 ? q.w_out2 : q.w_out, q.E > 0 ? q.E : 1, q.m_valid, q.N);
+  ok = ok && map_out_f32(&k.tmWs, q.w_sh ? q.w_sh : q.w_out, 1, q.m_valid, q.N);
+  ok = ok && map_out_f32(&k.tmWs2, q.w_sh2 ? q.w_sh2 : (q.w_sh ? q.w_sh : q.w_out), 1, q.m_valid, q.N);
+  if (!ok) return cudaErrorInvalidValue;
+  k.off = q.off;
+  k.valid = valid;
+  k.status = q.status;
+  k.rows_max = q.rows_max;
+  k.T = q.T;
+  k.N_out = q.N;
+  k.M_out = q.M;
+  k.E = q.E;
+  k.n_shared = q.n_shared;
+  k.epi = -1;
+  k.m_split = q.m_split;
+  k.m_valid = q.m_valid;
+  k.b_sep = q.b_shared != nullptr;
+  k.w_out = q.w_out;
+  k.w_out2 = q.w_out2;
+  k.w_sh = q.w_sh;
+  k.w_sh2 = q.w_sh2;
+  return launch_pairs(k, stream);
+}
+
 namespace gtn {
 static cudaError_t launch_pairs(const KParams& k, cudaStream_t stream) {
-  auto kern = k.dact ? grouped_gemm_tn_kernel<true> : grouped_gemm_tn_kernel<false>;
+  auto kern = k.M_out > 0 ? grouped_gemm_tn_kernel<2> : k.dact ? grouped_gemm_tn_kernel<1> : grouped_gemm_tn_kernel<0>;
   cudaError_t e = ensure_smem(kern, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg{};

@@ -248,6 +248,9 @@ cudaError_t launch_bwd_dgrad_pair(const BwdGemm& q, int32_t* pair_prefix, const 
 // dz [rows_max, dz_ld], SwiGLU's db at column dz_ld / 2.
 cudaError_t launch_bwd_dact_pair(const BwdGemm& q, int dz_ld, int32_t* pair_prefix, const int32_t* valid,
                                  cudaStream_t stream);
+// wgrad on pairs of SMs (grouped_gemm_tn.cu): the same outputs as
+// launch_bwd_wgrad, over each group's kept rows (valid) in 64-row blocks.
+cudaError_t launch_bwd_wgrad_pair(const BwdGemm& q, const int32_t* valid, cudaStream_t stream);
 
 // Packed weight layout for the grouped GEMM: w [G, N, K] bf16 (K contiguous) ->
 // [G][ceil(N/128)][ceil(K/64)][128][64], zero-padded, so every TMA box of 128

@@ -692,7 +692,10 @@ int moe_layer_bwd(const moe_cfg* cfg, const void* x, const float* wg, const moe_
   g.m_valid = H;
   g.w_out = dw->dw2;
   g.w_sh = sh ? dw->dsw2 : nullptr;
-  if (launch_bwd_wgrad(g, s) != cudaSuccess) return MOE_ECUDA;
+  // compute-bound layers: pairs of SMs
+  if ((two_sm_ffn(cfg) ? launch_bwd_wgrad_pair(g, at<int32_t>(ws, L.kept), s) : launch_bwd_wgrad(g, s)) !=
+      cudaSuccess)
+    return MOE_ECUDA;
   if ((st = record(stage_events, 3, s)) != MOE_OK) return st;
   // 4. dz = dh * act'(z), z recomputed from the dispatched rows
   g = q;
@@ -729,7 +732,9 @@ int moe_layer_bwd(const moe_cfg* cfg, const void* x, const float* wg, const moe_
   g.w_out2 = sw ? dw->dw3 : nullptr;
   g.w_sh = sh ? dw->dsw1 : nullptr;
   g.w_sh2 = sh && sw ? dw->dsw3 : nullptr;
-  if (launch_bwd_wgrad(g, s) != cudaSuccess) return MOE_ECUDA;
+  if ((two_sm_ffn(cfg) ? launch_bwd_wgrad_pair(g, at<int32_t>(ws, L.kept), s) : launch_bwd_wgrad(g, s)) !=
+      cudaSuccess)
+    return MOE_ECUDA;
   if ((st = record(stage_events, 5, s)) != MOE_OK) return st;
   // 6. router backward
   RouterBwdParams rb{};
