@@ -711,8 +711,10 @@ int moe_layer_bwd(const moe_cfg* cfg, const void* x, const float* wg, const moe_
   g.N = F;
   g.b_packed = packed;
   if (!fused) {
-    // compute-bound layers: pairs of SMs, as the forward's first contraction
-    const cudaError_t e = two_sm_ffn(cfg)
+    // compute-bound SwiGLU layers: pairs of SMs, as the forward's first
+    // contraction (GShard's GELU layer measured 0.67 ms there against 0.42 ms on
+    // one SM per tile: the epilogue's GELU' outweighs the feed)
+    const cudaError_t e = two_sm_ffn(cfg) && sw
                               ? launch_bwd_dact_pair(g, dzw, at<int32_t>(ws, L.pairs), at<int32_t>(ws, L.kept), s)
                               : launch_bwd_dact(g, s);
     if (e != cudaSuccess) return MOE_ECUDA;
