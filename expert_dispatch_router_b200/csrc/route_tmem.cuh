@@ -57,7 +57,7 @@ __device__ __forceinline__ void route_bar() {
 // logit first, equal logits -> smaller expert; the order the oracle uses).
 // Selection counts add up in shared memory (integers: any order gives the same
 // total); each expert's probability sum over the tile's tokens is a fixed
-// butterfly over the lanes, then the four sub-partitions in order.  The tile's
+// reduce-scatter butterfly over the lanes, then the four sub-partitions in order.  The tile's
 // sums go to row 4 * mt of the 32-token partial arrays and rows 4 mt + 1 ..
 // 4 mt + 3 are zeroed.  The logit offset, where there is one, is added once
 // and the sums written back to TMEM for the later passes.
@@ -226,9 +226,13 @@ __device__ __forceinline__ void route_tile_tmem(const RouterParams& rp, int64_t 
     if (lane == 0) xz[sub] = z;
   }
 
-  // 6. each expert's probability sum over the tile's tokens
+  // 6. each expert's probability sum over the tile's tokens: per 8 columns a
+  // reduce-scatter butterfly over the lanes (lane bits 4, 3, 2 halve the
+  // columns each lane carries; bits 1, 0 finish the sum), after which lanes
+  // 4c .. 4c + 3 hold column c's sum
   if (rp.psum_part != nullptr) {
     const float inv = 1.0f / (sigmoid ? ss : s);
+    const bool b16 = (lane & 16) != 0, b8 = (lane & 8) != 0, b4 = (lane & 4) != 0;
 #pragma unroll 1
     for (int cc = 0; cc < W; cc += 8) {
       float v[8];
@@ -236,12 +240,20 @@ __device__ __forceinline__ void route_tile_tmem(const RouterParams& rp, int64_t 
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const int e = c0 + cc + j;
-        float pe = 0.0f;
-        if (tv && e < E) pe = (sigmoid ? 1.0f / (1.0f + expf(-v[j])) : expf(v[j] - m)) * inv;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) pe += __shfl_xor_sync(0xffffffffu, pe, o);
-        if (lane == 0 && e < E) xps[sub * 256 + e] = pe;
+        v[j] = (tv && e < E) ? (sigmoid ? 1.0f / (1.0f + expf(-v[j])) : expf(v[j] - m)) * inv : 0.0f;
       }
+      float q4[4], q2[2];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)      // bit 4 clear keeps columns 0-3, set keeps 4-7
+        q4[i] = (b16 ? v[i + 4] : v[i]) + __shfl_xor_sync(0xffffffffu, b16 ? v[i] : v[i + 4], 16);
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+        q2[i] = (b8 ? q4[i + 2] : q4[i]) + __shfl_xor_sync(0xffffffffu, b8 ? q4[i] : q4[i + 2], 8);
+      float q1 = (b4 ? q2[1] : q2[0]) + __shfl_xor_sync(0xffffffffu, b4 ? q2[0] : q2[1], 4);
+      q1 += __shfl_xor_sync(0xffffffffu, q1, 2);
+      q1 += __shfl_xor_sync(0xffffffffu, q1, 1);
+      const int e = c0 + cc + ((lane >> 2) & 7);
+      if ((lane & 3) == 0 && e < E) xps[sub * 256 + e] = q1;
     }
   }
   route_bar();
