@@ -65,6 +65,7 @@ constexpr int SMEM_BYTES = RING_BYTES + STAGING_BYTES + 1024 /*align*/ + 256 /*b
 
 struct KParams {
   CUtensorMap tmA, tmAs, tmB0, tmB1, tmSB0, tmSB1;
+  CUtensorMap tmB0h, tmSB0h;   // 192-column tiles: the same weights in 64-row boxes (half a packed block)
   CUtensorMap tmD;       // bf16 output [rows, N_out], box 32 x 32, 64-byte swizzle (TMA store)
   void* d;
   const int32_t* off;
@@ -74,7 +75,8 @@ struct KParams {
   int64_t rows_store;    // rows >= rows_store are not stored
   int K, N_out, E, n_shared, epi;
   int as_sep;            // 1: the shared block's A rows come from tmAs (row - off[E]); 0: from tmA in place
-  int bn_fixed;          // 0: N tile chosen on the device (256 or 128); else this MMA N (multiple of 16)
+  int bn_fixed;          // 0: N tile chosen on the device (256, 192 or 128); else this MMA N (multiple of 16)
+  int allow192;          // 1: 192-column tiles may be chosen (tmB0h / tmSB0h are set)
   int bbox;              // rows of one B TMA box (128, or bn_fixed when smaller)
   int b_planes;          // router: 3 weight planes laid side by side along B's K; one stage holds the A
                          // chunk and the matching chunk of every plane, multiplied into one accumulator
@@ -172,16 +174,22 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
   const int64_t rows_used = grouped ? min((int64_t)p.off[ngroups], p.rows_max) : p.rows_static;
   const int64_t n_mtiles = (rows_used + BM - 1) / BM;
   const int nk = (p.K + BK - 1) / BK;
-  // Tile width: SwiGLU tiles hold 128 gate + 128 up columns (128 outputs).
-  // Otherwise 256 columns, or 128 when the wider tile leaves the last wave of
-  // CTAs mostly idle (a narrow tile costs ~0.55 of a wide one), or a fixed N.
-  bool narrow = false;
+  // Tile width: SwiGLU tiles hold 128 gate + 128 up columns (128 outputs),
+  // the router a fixed N.  Otherwise 256, 192 or 128 columns, whichever keeps
+  // the busiest SM's operand bytes lowest: a tile loads BM + bn rows of K per
+  // k step through an SM whose intake rate is fixed, and the SM with the most
+  // tiles (ceil(tiles / grid)) finishes last.  Ties go to the wider tile.
+  int bn_auto = 256;
   if (!swiglu && p.bn_fixed == 0) {
-    const int64_t t256 = n_mtiles * ((p.N_out + 255) / 256), t128 = n_mtiles * ((p.N_out + 127) / 128);
-    const int64_t w256 = (t256 + gridDim.x - 1) / gridDim.x, w128 = (t128 + gridDim.x - 1) / gridDim.x;
-    narrow = 0.55 * (double)w128 < (double)w256;
+    auto cost = [&](int b) {
+      const int64_t t = n_mtiles * ((p.N_out + b - 1) / b);
+      return ((t + gridDim.x - 1) / gridDim.x) * (int64_t)(BM + b);
+    };
+    int64_t best = cost(256);
+    if (p.allow192 && cost(192) < best) { best = cost(192); bn_auto = 192; }
+    if (cost(128) < best) bn_auto = 128;
   }
-  const int bn = p.bn_fixed ? p.bn_fixed : (narrow ? 128 : 256);   // MMA N
+  const int bn = p.bn_fixed ? p.bn_fixed : bn_auto;                 // MMA N
   const int n_step = swiglu ? BN / 2 : bn;                          // output columns per tile
   const int n_tiles_n = (p.N_out + n_step - 1) / n_step;
   // tile = (m-block, n-tile, k part), k part fastest; part q owns k blocks
@@ -190,8 +198,8 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
   const int nk_part = (nk + n_parts - 1) / n_parts;
   const int64_t n_tiles = n_mtiles * n_tiles_n * n_parts;
   const int box_bytes = p.bbox * BK * 2;
-  const int n_boxes = swiglu ? 2 : bn / p.bbox;
-  const int plane_bytes = n_boxes * box_bytes;          // one plane's B chunk
+  const int n_boxes = swiglu ? 2 : bn / p.bbox;         // (192: a 128-row and a 64-row box)
+  const int plane_bytes = swiglu ? 2 * box_bytes : bn * BK * 2;   // one plane's B chunk
   const int pps = p.b_planes == 1 ? 1 : p.planes_per_stage;   // planes per stage
   const int pass = p.b_planes / pps;                    // stages per k block
   const int stage_bytes = A_BYTES + pps * plane_bytes;
@@ -237,7 +245,26 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
           const int ka = kb * BK, kbb = kb * BK;
           mbar_expect_tx(fb, gat ? stage_bytes - A_BYTES : stage_bytes);
           if (!gat) tma_load_2d(sa, ma, ka, arow, fb);
-          if (p.b_packed) {
+          if (bn == 192) {
+            // a 128-row box and a 64-row half box in row order (n0 is a multiple of 64)
+            const CUtensorMap* mh = sh ? &p.tmSB0h : &p.tmB0h;
+            const bool lead_half = (n0 & 127) != 0;
+            if (p.b_packed) {
+              if (lead_half) {
+                tma_load_5d_at(sb, mh, 64, kbb / BK, n0 / 128, z, fb);
+                tma_load_5d(sb + 8192, mb0, kbb / BK, n0 / 128 + 1, z, fb);
+              } else {
+                tma_load_5d(sb, mb0, kbb / BK, n0 / 128, z, fb);
+                tma_load_5d_at(sb + 16384, mh, 0, kbb / BK, n0 / 128 + 1, z, fb);
+              }
+            } else if (lead_half) {
+              tma_load_3d(sb, mh, kbb, n0, z, fb);
+              tma_load_3d(sb + 8192, mb0, kbb, n0 + 64, z, fb);
+            } else {
+              tma_load_3d(sb, mb0, kbb, n0, z, fb);
+              tma_load_3d(sb + 16384, mh, kbb, n0 + 128, z, fb);
+            }
+          } else if (p.b_packed) {
             // packed weights: every box is one contiguous 16 KB block
             if (swiglu) {
               tma_load_5d(sb, mb0, kbb / BK, n0 / 128, z, fb);
@@ -538,7 +565,7 @@ static bool make_map_b(CUtensorMap* m, const void* base, int G, int N, int K, in
 
 // 5-D map over packed weights [G][N/128][K/64][128][64] (see launch_pack_weight):
 // dims (64, 128, K/64, N/128, G), box 64 x 128 x 1 x 1 x 1 = one 16 KB block.
-static bool make_map_b_packed(CUtensorMap* m, const void* base, int G, int N, int K) {
+static bool make_map_b_packed(CUtensorMap* m, const void* base, int G, int N, int K, int box_rows = 128) {
   const cuuint64_t kb = (cuuint64_t)((K + BK - 1) / BK), nb = (cuuint64_t)((N + 127) / 128);
   MapKey key;
   memset(&key, 0, sizeof(key));
@@ -555,7 +582,7 @@ static bool make_map_b_packed(CUtensorMap* m, const void* base, int G, int N, in
   key.strides[2] = key.strides[1] * kb;
   key.strides[3] = key.strides[2] * nb;
   key.box[0] = BK;
-  key.box[1] = 128;
+  key.box[1] = (cuuint32_t)box_rows;
   key.box[2] = key.box[3] = key.box[4] = 1;
   return encode_cached(m, key);
 }
@@ -621,8 +648,20 @@ cudaError_t launch_grouped_gemm(const GemmParams& p, cudaStream_t stream) {
     ok = ok && make_map_b(&k.tmSB0, p.sb0 ? p.sb0 : p.b0, 1, p.Nw, p.K, box_n);
     ok = ok && make_map_b(&k.tmSB1, p.sb1 ? p.sb1 : (p.sb0 ? p.sb0 : p.b0), 1, p.Nw, p.K, box_n);
   }
+  // 192-column tiles (no SwiGLU): the same weights in 64-row boxes
+  const bool allow192 = p.epi != MOE_ACT_SWIGLU && p.Nw > 128;
+  if (allow192) {
+    if (p.b_packed) {
+      ok = ok && make_map_b_packed(&k.tmB0h, p.b0, p.E, p.Nw, p.K, 64);
+      ok = ok && make_map_b_packed(&k.tmSB0h, p.sb0 ? p.sb0 : p.b0, 1, p.Nw, p.K, 64);
+    } else {
+      ok = ok && make_map_b(&k.tmB0h, p.b0, p.E, p.Nw, p.K, 64);
+      ok = ok && make_map_b(&k.tmSB0h, p.sb0 ? p.sb0 : p.b0, 1, p.Nw, p.K, 64);
+    }
+  }
   ok = ok && make_map_d(&k.tmD, p.d, p.rows_max, p.Nw);
   if (!ok) return cudaErrorInvalidValue;
+  k.allow192 = allow192 ? 1 : 0;
   k.d = p.d;
   k.off = p.expert_offset;
   k.status = p.status;

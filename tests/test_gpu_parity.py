@@ -52,6 +52,13 @@ SMALL = {
     # F = 512 + 72 leave a ragged last tile, with a shared expert
     "wide_2sm_shared": synth.SWITCH_TOP1.replace(name="wide_2sm_shared", T=1100, H=1032, F=584, E=4, k=2,
                                                  cap_mode=synth.CAP_DROPLESS, n_shared=1, bias_row0=0.0),
+    # one SM per tile with 192-column tiles (about 40 row blocks: 3 x 192 columns
+    # fit one wave where 128-column tiles need two); H = 568 and F = 392 leave
+    # ragged last tiles.  Top-1 with the fused gather and scatter; then k = 2
+    # with a shared expert (its weights in half-block boxes too)
+    "tiles192_top1": synth.SWITCH_TOP1.replace(name="tiles192_top1", T=4000, H=568, F=392, E=40),
+    "tiles192_shared": synth.SWITCH_TOP1.replace(name="tiles192_shared", T=1200, H=568, F=392, E=24, k=2,
+                                                 cap_mode=synth.CAP_DROPLESS, n_shared=1, bias_row0=0.0),
 }
 
 
@@ -365,7 +372,8 @@ def test_pack_weight_layout(G, N, K):
     assert torch.equal(got.view(torch.int16), want.view(torch.int16))
 
 
-@pytest.mark.parametrize("name", ["switch_top1", "gshard_top2", "wideep", "ds_k4_cf05", "switch_relu_dropless_shared",
+@pytest.mark.parametrize("name", ["switch_top1", "gshard_top2", "wideep", "ds_k4_cf05", "tiles192_top1", "tiles192_shared",
+                                  "switch_relu_dropless_shared",
                                   "wideep_2sm", "gshard_2sm", "relu_2sm_shared", "wide_2sm_shared"])
 def test_packed_weights_bitwise(name):
     """Packed weights change only where the contractions read B from."""
