@@ -136,10 +136,15 @@ static void launch_dispatch_km(const PermuteParams& p, unsigned grid, cudaStream
   launch_pdl(dispatch_kernel<KM, U>, grid, kPermWarps * 32, 0, s, p);
 }
 
+// U: vector positions per lane in flight, at most what one row needs (a
+// lane's U * KM loads are held in registers, which bound the warps per SM).
 template <typename ET, int KM>
 static void launch_combine_km(const PermuteParams& p, unsigned grid, cudaStream_t s) {
-  constexpr int U = KM >= 16 ? 1 : KM >= 8 ? 2 : 4;
-  launch_pdl(combine_kernel<ET, KM, U>, grid, kPermWarps * 32, 0, s, p);
+  constexpr int UMAX = KM >= 16 ? 1 : KM >= 8 ? 2 : 4;
+  const int64_t nvec = (int64_t)p.H * (int64_t)sizeof(ET) / 16;
+  if (UMAX >= 2 && nvec <= 32) launch_pdl(combine_kernel<ET, KM, 1>, grid, kPermWarps * 32, 0, s, p);
+  else if (UMAX >= 4 && nvec <= 64) launch_pdl(combine_kernel<ET, KM, 2>, grid, kPermWarps * 32, 0, s, p);
+  else launch_pdl(combine_kernel<ET, KM, UMAX>, grid, kPermWarps * 32, 0, s, p);
 }
 
 cudaError_t launch_dispatch(const PermuteParams& p, cudaStream_t stream) {
