@@ -179,7 +179,12 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
   // the busiest SM's operand bytes lowest: a tile loads BM + bn rows of K per
   // k step through an SM whose intake rate is fixed, and the SM with the most
   // tiles (ceil(tiles / grid)) finishes last.  Ties go to the wider tile.
+  // A 384-column tile (two 192-column accumulators, both TMEM buffers, sharing
+  // each A stage: the A rows load half as often) when such tiles fit one wave,
+  // so that no tile waits for the previous one's epilogue (not with the fused
+  // gather, whose instance keeps its registers for the gather warps).
   int bn_auto = 256;
+  bool wide = false;
   if (!swiglu && p.bn_fixed == 0) {
     auto cost = [&](int b) {
       const int64_t t = n_mtiles * ((p.N_out + b - 1) / b);
@@ -187,10 +192,15 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
     };
     int64_t best = cost(256);
     if (p.allow192 && cost(192) < best) { best = cost(192); bn_auto = 192; }
-    if (cost(128) < best) bn_auto = 128;
+    if (cost(128) < best) { best = cost(128); bn_auto = 128; }
+    if (!GATHER && p.allow192 && n_mtiles * ((p.N_out + 383) / 384) <= (int64_t)gridDim.x &&
+        (int64_t)(BM + 384) < best) {
+      wide = true;
+      bn_auto = 192;
+    }
   }
   const int bn = p.bn_fixed ? p.bn_fixed : bn_auto;                 // MMA N
-  const int n_step = swiglu ? BN / 2 : bn;                          // output columns per tile
+  const int n_step = swiglu ? BN / 2 : (wide ? 2 * bn : bn);        // output columns per tile
   const int n_tiles_n = (p.N_out + n_step - 1) / n_step;
   // tile = (m-block, n-tile, k part), k part fastest; part q owns k blocks
   // [q * nk_part, min(nk, (q + 1) * nk_part))
@@ -198,8 +208,9 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
   const int nk_part = (nk + n_parts - 1) / n_parts;
   const int64_t n_tiles = n_mtiles * n_tiles_n * n_parts;
   const int box_bytes = p.bbox * BK * 2;
-  const int n_boxes = swiglu ? 2 : bn / p.bbox;         // (192: a 128-row and a 64-row box)
-  const int plane_bytes = swiglu ? 2 * box_bytes : bn * BK * 2;   // one plane's B chunk
+  const int brows = wide ? 2 * bn : bn;                 // B rows of a tile
+  const int n_boxes = swiglu ? 2 : brows / p.bbox;      // (192: a 128-row and a 64-row box)
+  const int plane_bytes = swiglu ? 2 * box_bytes : brows * BK * 2;   // one plane's B chunk
   const int pps = p.b_planes == 1 ? 1 : p.planes_per_stage;   // planes per stage
   const int pass = p.b_planes / pps;                    // stages per k block
   const int stage_bytes = A_BYTES + pps * plane_bytes;
@@ -245,7 +256,7 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
           const int ka = kb * BK, kbb = kb * BK;
           mbar_expect_tx(fb, gat ? stage_bytes - A_BYTES : stage_bytes);
           if (!gat) tma_load_2d(sa, ma, ka, arow, fb);
-          if (bn == 192) {
+          if (bn == 192 && !wide) {
             // a 128-row box and a 64-row half box in row order (n0 is a multiple of 64)
             const CUtensorMap* mh = sh ? &p.tmSB0h : &p.tmB0h;
             const bool lead_half = (n0 & 127) != 0;
@@ -357,7 +368,36 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       const uint32_t idesc = make_idesc(bn);
-      for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+      // wide: both accumulator buffers per tile, one 192-column MMA into each per
+      // 16-k step, the B rows of the second starting 192 rows into the stage
+      for (int64_t tile = blockIdx.x; tile < n_tiles && ok && wide; tile += gridDim.x) {
+        const int kb0 = (int)(tile % n_parts) * nk_part, kb1 = min(nk, kb0 + nk_part);
+        if (!mbar_wait(tempty0, acc_phase ^ 1u, abort_flag) || !mbar_wait(tempty0 + 8, acc_phase ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int ks = kb0; ks < kb1; ++ks) {
+          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          if (GATHER) fence_async_smem();
+          const uint32_t sa = smem_u32(stage_base + stage * stage_bytes);
+          const uint32_t sb = sa + A_BYTES;
+          const uint64_t ad = sw128_desc(sa), bd0 = sw128_desc(sb), bd1 = sw128_desc(sb + (uint32_t)(bn * 128));
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint32_t acc_in = ((ks - kb0) | kk) != 0 ? 1u : 0u;
+            umma(tmem_base, ad + (uint64_t)(kk * 2), bd0 + (uint64_t)(kk * 2), idesc, acc_in);
+            umma(tmem_base + (uint32_t)BN, ad + (uint64_t)(kk * 2), bd1 + (uint64_t)(kk * 2), idesc, acc_in);
+          }
+          umma_commit(empty0 + 8 * stage);
+          if (++stage == n_stages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(tfull0);
+        acc_phase ^= 1u;
+      }
+      for (int64_t tile = blockIdx.x; tile < n_tiles && ok && !wide; tile += gridDim.x) {
         const int kb0 = (int)(tile % n_parts) * nk_part, kb1 = min(nk, kb0 + nk_part);
         if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
@@ -432,7 +472,7 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
         for (int c = quarter * chunk; c < n_step; c += 4 * chunk) {
           __syncwarp();                                // converged for the warp-wide tcgen05.ld
           float v[32];
-          const int acol = c;                                     // accumulator column
+          const int acol = (wide && c >= bn) ? BN + (c - bn) : c;   // accumulator column (wide: second buffer)
           tmem_ld(tbase + (uint32_t)acol, v, chunk);
           if (swiglu) {
             float u[32];
@@ -512,8 +552,14 @@ __global__ void __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(tempty0 + 8 * acc);
-      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      if (wide) {
+        mbar_arrive(tempty0);
+        mbar_arrive(tempty0 + 8);
+        acc_phase ^= 1u;
+      } else {
+        mbar_arrive(tempty0 + 8 * acc);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
     }
     if (lane == 0) bulk_wait0();                 // this warp's output stores are complete
     __syncwarp();

@@ -59,6 +59,12 @@ SMALL = {
     "tiles192_top1": synth.SWITCH_TOP1.replace(name="tiles192_top1", T=4000, H=568, F=392, E=40),
     "tiles192_shared": synth.SWITCH_TOP1.replace(name="tiles192_shared", T=1200, H=568, F=392, E=24, k=2,
                                                  cap_mode=synth.CAP_DROPLESS, n_shared=1, bias_row0=0.0),
+    # 384-column tiles (two 192-column accumulators sharing each A stage) in the
+    # second contraction: about 40-50 row blocks, so those tiles fit one wave
+    # where 192-column ones need two; H = 760 leaves a ragged second tile
+    "wide384_top1": synth.SWITCH_TOP1.replace(name="wide384_top1", T=4000, H=760, F=392, E=40),
+    "wide384_shared": synth.SWITCH_TOP1.replace(name="wide384_shared", T=1800, H=760, F=392, E=36, k=2,
+                                                cap_mode=synth.CAP_DROPLESS, n_shared=1, bias_row0=0.0),
 }
 
 
@@ -373,7 +379,7 @@ def test_pack_weight_layout(G, N, K):
 
 
 @pytest.mark.parametrize("name", ["switch_top1", "gshard_top2", "wideep", "ds_k4_cf05", "tiles192_top1", "tiles192_shared",
-                                  "switch_relu_dropless_shared",
+                                  "wide384_top1", "wide384_shared", "switch_relu_dropless_shared",
                                   "wideep_2sm", "gshard_2sm", "relu_2sm_shared", "wide_2sm_shared"])
 def test_packed_weights_bitwise(name):
     """Packed weights change only where the contractions read B from."""
