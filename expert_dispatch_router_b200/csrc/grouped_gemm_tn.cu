@@ -558,11 +558,13 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tn_kernel(const __gri
             // 16-byte loads into the staging buffer (its layout below), then
             // each lane takes its feature's column (features past N_out read
             // as zero); da (or dz) and SwiGLU's db go out as two stores
-            float v[32], u[32];
-            tmem_ld(tb + (uint32_t)c, v, 32);
-            if (swiglu) tmem_ld(tbase + 256u + (uint32_t)c, u, 32);
-            tmem_wait_ld();
-            const uint32_t col_b = (uint32_t)((lane & 7) * 2);
+            // the chunk in the forward's 16-lane fragment layout (below): the dh
+            // block comes in by 16-byte loads into the staging buffer (features
+            // past N_out read as zero) and back by transposing matrix loads, so
+            // gk[4 tg + fg] holds dh of features 8 fg + lane / 4 at tokens
+            // 8 tg + 2 (lane % 4) and + 1, the elements v[4 tg + 2 h + e] of load
+            // L = fg / 2, h = fg % 2 multiply; da (or dz) and SwiGLU's db go out as
+            // two stores
             if (lane == 0) bulk_wait_read0();
             __syncwarp();
 #pragma unroll
@@ -577,29 +579,60 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tn_kernel(const __gri
                            :: "r"(addr), "r"(w.x), "r"(w.y), "r"(w.z), "r"(w.w) : "memory");
             }
             __syncwarp();
+            uint32_t gk[16];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const uint32_t addr = stage_out + (uint32_t)(j * 64) + ((((uint32_t)lane >> 3) ^ (((uint32_t)j >> 1) & 3u)) << 4) + col_b;
-              uint16_t hb;
-              asm volatile("ld.shared.b16 %0, [%1];" : "=h"(hb) : "r"(addr) : "memory");
-              const float gi = __bfloat162float(__ushort_as_bfloat16(hb));
-              const float z = v[j];
-              if (swiglu) {
-                const float sg = 1.0f / (1.0f + __expf(-z));
-                v[j] = gi * u[j] * sg * (1.0f + z * (1.0f - sg));   // da
-                u[j] = gi * z * sg;                                 // db = dh * silu(a)
-              } else {
-                v[j] = p.epi == MOE_ACT_RELU ? (z > 0.0f ? gi : 0.0f) : gi * gelu_grad(z);
-              }
+            for (int tg = 0; tg < 4; ++tg) {
+              const uint32_t jr = (uint32_t)(8 * tg + (lane & 7));
+              const uint32_t addr = stage_out + jr * 64u + ((((uint32_t)lane >> 3) ^ ((jr >> 1) & 3u)) << 4);
+              asm volatile("ldmatrix.sync.aligned.x4.trans.m8n8.shared.b16 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(gk[4 * tg]), "=r"(gk[4 * tg + 1]), "=r"(gk[4 * tg + 2]), "=r"(gk[4 * tg + 3])
+                           : "r"(addr) : "memory");
+            }
+            uint32_t pa[16], pb[16];
+#pragma unroll
+            for (int L = 0; L < 2; ++L) {
+              const uint32_t lo = ((uint32_t)(16 * L) << 16) + (uint32_t)c;
+              float z[16], u[16];
+              tmem_ld_16x256b(tb + lo, z);
+              if (swiglu) tmem_ld_16x256b(tbase + 256u + lo, u);
+              tmem_wait_ld();
+#pragma unroll
+              for (int tg = 0; tg < 4; ++tg)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                  const int k = 4 * tg + 2 * L + h;
+                  const __nv_bfloat162 g2 = *reinterpret_cast<const __nv_bfloat162*>(&gk[k]);
+                  float da[2], db[2];
+#pragma unroll
+                  for (int e = 0; e < 2; ++e) {
+                    const float gi = __bfloat162float(e == 0 ? g2.x : g2.y);
+                    const float zz = z[4 * tg + 2 * h + e];
+                    if (swiglu) {
+                      const float sg = 1.0f / (1.0f + __expf(-zz));
+                      da[e] = gi * u[4 * tg + 2 * h + e] * sg * (1.0f + zz * (1.0f - sg));
+                      db[e] = gi * zz * sg;                         // dh * silu(a)
+                    } else {
+                      da[e] = p.epi == MOE_ACT_RELU ? (zz > 0.0f ? gi : 0.0f) : gi * gelu_grad(zz);
+                      db[e] = 0.0f;
+                    }
+                  }
+                  const __nv_bfloat162 a2 = __floats2bfloat162_rn(da[0], da[1]);
+                  const __nv_bfloat162 b2 = __floats2bfloat162_rn(db[0], db[1]);
+                  pa[k] = *reinterpret_cast<const uint32_t*>(&a2);
+                  pb[k] = *reinterpret_cast<const uint32_t*>(&b2);
+                }
             }
             for (int o = 0; o < (swiglu ? 2 : 1); ++o) {
               if (lane == 0) bulk_wait_read0();
               __syncwarp();
 #pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const __nv_bfloat16 h = __float2bfloat16_rn(o == 0 ? v[j] : u[j]);
-                const uint32_t addr = stage_out + (uint32_t)(j * 64) + ((((uint32_t)lane >> 3) ^ (((uint32_t)j >> 1) & 3u)) << 4) + col_b;
-                asm volatile("st.shared.b16 [%0], %1;" :: "r"(addr), "h"(*reinterpret_cast<const uint16_t*>(&h)) : "memory");
+              for (int tg = 0; tg < 4; ++tg) {
+                const uint32_t jr = (uint32_t)(8 * tg + (lane & 7));
+                const uint32_t addr = stage_out + jr * 64u + ((((uint32_t)lane >> 3) ^ ((jr >> 1) & 3u)) << 4);
+                const uint32_t* pk = o == 0 ? pa : pb;
+                asm volatile("stmatrix.sync.aligned.x4.trans.m8n8.shared.b16 [%0], {%1, %2, %3, %4};"
+                             :: "r"(addr), "r"(pk[4 * tg]), "r"(pk[4 * tg + 1]), "r"(pk[4 * tg + 2]),
+                                "r"(pk[4 * tg + 3]) : "memory");
               }
               fence_async_smem();
               __syncwarp();
@@ -610,35 +643,54 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tn_kernel(const __gri
             }
             continue;
           }
-          float v[32];
-          tmem_ld(tb + (uint32_t)c, v, 32);
-          if (swiglu) {
-            float u[32];
-            tmem_ld(tbase + 256u + (uint32_t)c, u, 32);
-            tmem_wait_ld();
+          // the chunk in the 16-lane shape: load L holds features 16 L + lane / 4
+          // (v[4 i], v[4 i + 1]) and 16 L + 8 + lane / 4 (v[4 i + 2], v[4 i + 3])
+          // at tokens 8 i + 2 (lane % 4) and + 1, the fragment layout of an 8 x 8
+          // matrix; pk[4 tg + fg] is the bf16 fragment of features 8 fg .. + 8 by
+          // tokens 8 tg .. + 8
+          uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = act_silu(v[i]) * u[i];
-          } else {
-            tmem_wait_ld();
-            if (p.epi == MOE_ACT_RELU) {
+          for (int L = 0; L < 2; ++L) {
+            const uint32_t ta = tb + ((uint32_t)(16 * L) << 16) + (uint32_t)c;
+            float v[16];
+            tmem_ld_16x256b(ta, v);
+            if (swiglu) {
+              float u[16];
+              tmem_ld_16x256b(ta + 256u, u);
+              tmem_wait_ld();
 #pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = act_relu(v[i]);
-            } else if (p.epi == MOE_ACT_GELU) {
+              for (int i = 0; i < 16; ++i) v[i] = act_silu(v[i]) * u[i];
+            } else {
+              tmem_wait_ld();
+              if (p.epi == MOE_ACT_RELU) {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = act_gelu(v[i]);
+                for (int i = 0; i < 16; ++i) v[i] = act_relu(v[i]);
+              } else if (p.epi == MOE_ACT_GELU) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] = act_gelu(v[i]);
+              }
             }
+#pragma unroll
+            for (int tg = 0; tg < 4; ++tg)
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[4 * tg + 2 * h], v[4 * tg + 2 * h + 1]);
+                pk[4 * tg + 2 * L + h] = *reinterpret_cast<const uint32_t*>(&b2);
+              }
           }
-          // transpose through the staging buffer: token j's 32 features form a
+          // transpose into the staging buffer: token j's 32 features form a
           // 64-byte row (16-byte chunk q of row j at q ^ ((j >> 1) & 3): the TMA
-          // 64-byte swizzle); this lane writes its feature's element of every row
+          // 64-byte swizzle); one transposing matrix store per token group, this
+          // lane giving the address of token 8 tg + lane % 8 in feature group lane / 8
           if (lane == 0) bulk_wait_read0();
           __syncwarp();
-          const uint32_t col_b = (uint32_t)((lane & 7) * 2);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const __nv_bfloat16 h = __float2bfloat16_rn(v[j]);
-            const uint32_t addr = stage_out + (uint32_t)(j * 64) + ((((uint32_t)lane >> 3) ^ (((uint32_t)j >> 1) & 3u)) << 4) + col_b;
-            asm volatile("st.shared.b16 [%0], %1;" :: "r"(addr), "h"(*reinterpret_cast<const uint16_t*>(&h)) : "memory");
+          for (int tg = 0; tg < 4; ++tg) {
+            const uint32_t jr = (uint32_t)(8 * tg + (lane & 7));
+            const uint32_t addr = stage_out + jr * 64u + ((((uint32_t)lane >> 3) ^ ((jr >> 1) & 3u)) << 4);
+            asm volatile("stmatrix.sync.aligned.x4.trans.m8n8.shared.b16 [%0], {%1, %2, %3, %4};"
+                         :: "r"(addr), "r"(pk[4 * tg]), "r"(pk[4 * tg + 1]), "r"(pk[4 * tg + 2]), "r"(pk[4 * tg + 3])
+                         : "memory");
           }
           fence_async_smem();
           __syncwarp();

@@ -180,6 +180,20 @@ __device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[32], int n) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
+// tcgen05.ld in the 16-lane x 256-bit shape, four repeats (32 columns) from
+// lane (taddr >> 16) .. + 16: v[4 i .. 4 i + 1] = lane + lane_id / 4, columns
+// 8 i + 2 (lane_id % 4) + 0, 1; v[4 i + 2 .. 4 i + 3] the same columns of lane + 8
+__device__ __forceinline__ void tmem_ld_16x256b(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile("tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+               "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                 "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+                 "=r"(r[15])
+               : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 // Store v[0 .. n) (n = 32, 16 or 8 columns) to this warp's lanes at taddr.
 __device__ __forceinline__ void tmem_st(uint32_t taddr, const float (&v)[32], int n) {
