@@ -108,6 +108,58 @@ __device__ __forceinline__ float act_gelu(float z) {
   const float h = z * (q * t) * e;                                          // 0.5 z erfc(|z| / sqrt 2)
   return z >= 0.0f ? z - h : h;
 }
+// Two fp32 values in one 64-bit register for the packed fp32 pipes of sm_100
+// (add / sub / mul / fma .f32x2: each half the same IEEE operation as the
+// scalar instruction, two values per issue).
+__device__ __forceinline__ unsigned long long f32x2_pack(float lo, float hi) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f32x2_unpack(unsigned long long r, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+__device__ __forceinline__ unsigned long long f32x2_fma(unsigned long long a, unsigned long long b,
+                                                        unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ unsigned long long f32x2_mul(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long f32x2_sub(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// act_gelu of two values: the same steps and constants, the FMA-pipe work on
+// packed pairs, the reciprocal and the exponential per value.
+__device__ __forceinline__ void act_gelu_x2(float& z0, float& z1) {
+  const unsigned long long z = f32x2_pack(z0, z1);
+  const unsigned long long a =
+      f32x2_fma(f32x2_pack(0.23164189f, 0.23164189f), f32x2_pack(fabsf(z0), fabsf(z1)), f32x2_pack(1.0f, 1.0f));
+  float a0, a1;
+  f32x2_unpack(a, a0, a1);
+  const unsigned long long t = f32x2_pack(rcp_approx(a0), rcp_approx(a1));
+  unsigned long long q = f32x2_fma(f32x2_pack(0.5307027145f, 0.5307027145f), t, f32x2_pack(-0.7265760135f, -0.7265760135f));
+  q = f32x2_fma(q, t, f32x2_pack(0.7107068705f, 0.7107068705f));
+  q = f32x2_fma(q, t, f32x2_pack(-0.142248368f, -0.142248368f));
+  q = f32x2_fma(q, t, f32x2_pack(0.127414796f, 0.127414796f));
+  const unsigned long long sq = f32x2_mul(f32x2_mul(z, z), f32x2_pack(-0.72134752044448170f, -0.72134752044448170f));
+  float s0, s1;
+  f32x2_unpack(sq, s0, s1);
+  const unsigned long long e = f32x2_pack(exp2f_approx(s0), exp2f_approx(s1));
+  const unsigned long long h = f32x2_mul(f32x2_mul(z, f32x2_mul(q, t)), e);   // 0.5 z erfc(|z| / sqrt 2)
+  const unsigned long long r = f32x2_sub(z, h);
+  float h0, h1, r0, r1;
+  f32x2_unpack(h, h0, h1);
+  f32x2_unpack(r, r0, r1);
+  z0 = z0 >= 0.0f ? r0 : h0;
+  z1 = z1 >= 0.0f ? r1 : h1;
+}
 // GELU'(z) = d/dz [z Phi(z)] = Phi(z) + z phi(z); Phi from erf (Abramowitz & Stegun 7.1.26).
 __device__ __forceinline__ float gelu_grad(float z) {
   const float phi = 0.3989422804014327f * __expf(-0.5f * z * z);

@@ -667,7 +667,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tn_kernel(const __gri
                 for (int i = 0; i < 16; ++i) v[i] = act_relu(v[i]);
               } else if (p.epi == MOE_ACT_GELU) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) v[i] = act_gelu(v[i]);
+                for (int i = 0; i < 16; i += 2) act_gelu_x2(v[i], v[i + 1]);
               }
             }
 #pragma unroll
