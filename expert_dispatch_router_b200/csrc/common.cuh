@@ -165,6 +165,41 @@ __device__ __forceinline__ float gelu_grad(float z) {
   const float phi = 0.3989422804014327f * __expf(-0.5f * z * z);
   return 0.5f * (1.0f + erf_as7126(z * 0.70710678118654752f)) + z * phi;
 }
+// gelu_grad of two values: Phi(z) = 0.5 (1 + erf(z / sqrt 2)) from the same
+// erf formula (Abramowitz & Stegun 7.1.26) and phi(z) = exp(-z^2 / 2) / sqrt(2 pi),
+// the FMA-pipe work on packed pairs, exp(a) as 2^(a log2 e) and the reciprocal
+// per value.
+__device__ __forceinline__ void gelu_grad_x2(float& z0, float& z1) {
+  const unsigned long long z = f32x2_pack(z0, z1);
+  const unsigned long long a = f32x2_mul(f32x2_mul(z, z), f32x2_pack(-0.72134752044448170f, -0.72134752044448170f));
+  float a0, a1;
+  f32x2_unpack(a, a0, a1);
+  const unsigned long long phi =
+      f32x2_mul(f32x2_pack(0.3989422804014327f, 0.3989422804014327f), f32x2_pack(exp2f_approx(a0), exp2f_approx(a1)));
+  const unsigned long long x = f32x2_mul(z, f32x2_pack(0.70710678118654752f, 0.70710678118654752f));
+  float x0, x1;
+  f32x2_unpack(x, x0, x1);
+  const unsigned long long ax = f32x2_pack(fabsf(x0), fabsf(x1));
+  const unsigned long long d = f32x2_fma(f32x2_pack(0.3275911f, 0.3275911f), ax, f32x2_pack(1.0f, 1.0f));
+  float d0, d1;
+  f32x2_unpack(d, d0, d1);
+  const unsigned long long t = f32x2_pack(rcp_approx(d0), rcp_approx(d1));
+  unsigned long long poly = f32x2_fma(f32x2_pack(1.061405429f, 1.061405429f), t, f32x2_pack(-1.453152027f, -1.453152027f));
+  poly = f32x2_fma(poly, t, f32x2_pack(1.421413741f, 1.421413741f));
+  poly = f32x2_fma(poly, t, f32x2_pack(-0.284496736f, -0.284496736f));
+  poly = f32x2_fma(poly, t, f32x2_pack(0.254829592f, 0.254829592f));
+  poly = f32x2_mul(poly, t);
+  const unsigned long long b = f32x2_mul(f32x2_mul(ax, ax), f32x2_pack(-1.4426950408889634f, -1.4426950408889634f));
+  float b0, b1;
+  f32x2_unpack(b, b0, b1);
+  const unsigned long long r =
+      f32x2_sub(f32x2_pack(1.0f, 1.0f), f32x2_mul(poly, f32x2_pack(exp2f_approx(b0), exp2f_approx(b1))));
+  float r0, r1;
+  f32x2_unpack(r, r0, r1);
+  const unsigned long long erf = f32x2_pack(copysignf(r0, x0), copysignf(r1, x1));
+  const unsigned long long g = f32x2_fma(z, phi, f32x2_fma(f32x2_pack(0.5f, 0.5f), erf, f32x2_pack(0.5f, 0.5f)));
+  f32x2_unpack(g, z0, z1);
+}
 // SiLU: z * sigmoid(z) = z / (1 + exp(-z)).
 __device__ __forceinline__ float act_silu(float z) { return z * rcp_approx(1.0f + __expf(-z)); }
 

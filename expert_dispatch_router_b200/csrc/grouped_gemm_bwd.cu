@@ -446,6 +446,19 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
           float u[32];
           if constexpr (swiglu) tmem_ld(tbase + (uint32_t)(2 * n_step + c), u, 32);
           tmem_wait_ld();
+          if constexpr (!swiglu) {
+            if (p.act == MOE_ACT_GELU) {                        // GELU' two values at a time
+#pragma unroll
+              for (int i = 0; i < 32; i += 2) {
+                float g0 = zv[i], g1 = zv[i + 1];
+                gelu_grad_x2(g0, g1);
+                v[i] = __bfloat162float(__float2bfloat16_rn(v[i])) * g0;
+                v[i + 1] = __bfloat162float(__float2bfloat16_rn(v[i + 1])) * g1;
+              }
+              store_bf16(v, col, row_base);
+              continue;
+            }
+          }
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const float gi = __bfloat162float(__float2bfloat16_rn(v[i]));
@@ -467,6 +480,24 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
         if constexpr (swiglu) tmem_ld(tbase + (uint32_t)(BNMAX / 2 + c), u, 32);
         tmem_wait_ld();
         const int ci = c >= 128 ? 1 : 0;
+        if constexpr (!swiglu) {
+          if (p.act == MOE_ACT_GELU) {                          // GELU' two values at a time
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int4 w = ci ? dhv[1][q] : dhv[0][q];
+              const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&w);
+#pragma unroll
+              for (int i = 0; i < 8; i += 2) {
+                float g0 = v[8 * q + i], g1 = v[8 * q + i + 1];
+                gelu_grad_x2(g0, g1);
+                v[8 * q + i] = __bfloat162float(e[i]) * g0;
+                v[8 * q + i + 1] = __bfloat162float(e[i + 1]) * g1;
+              }
+            }
+            store_bf16(v, col, row_base);
+            continue;
+          }
+        }
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int4 w = ci ? dhv[1][q] : dhv[0][q];
