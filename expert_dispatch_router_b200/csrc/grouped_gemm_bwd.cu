@@ -464,7 +464,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
             const float gi = __bfloat162float(__float2bfloat16_rn(v[i]));
             const float z = zv[i];
             if constexpr (swiglu) {
-              const float s = 1.0f / (1.0f + __expf(-z));
+              const float s = rcp_approx(1.0f + __expf(-z));
               v[i] = gi * u[i] * s * (1.0f + z * (1.0f - s));    // da
               zv[i] = gi * z * s;                                 // db = dh * silu(a)
             } else {
@@ -507,7 +507,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_bwd_kernel(const __gr
             const float gi = __bfloat162float(e[i]);
             const float z = v[8 * q + i];
             if constexpr (swiglu) {
-              const float s = 1.0f / (1.0f + __expf(-z));
+              const float s = rcp_approx(1.0f + __expf(-z));
               v[8 * q + i] = gi * u[8 * q + i] * s * (1.0f + z * (1.0f - s));   // da
               u[8 * q + i] = gi * z * s;                                        // db = dh * silu(a)
             } else {

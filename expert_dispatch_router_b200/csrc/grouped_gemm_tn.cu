@@ -608,7 +608,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tn_kernel(const __gri
                     const float gi = __bfloat162float(e == 0 ? g2.x : g2.y);
                     const float zz = z[4 * tg + 2 * h + e];
                     if (swiglu) {
-                      const float sg = 1.0f / (1.0f + __expf(-zz));
+                      const float sg = rcp_approx(1.0f + __expf(-zz));
                       da[e] = gi * u[4 * tg + 2 * h + e] * sg * (1.0f + zz * (1.0f - sg));
                       db[e] = gi * zz * sg;                         // dh * silu(a)
                     } else {
